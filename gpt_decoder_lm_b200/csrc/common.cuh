@@ -1,0 +1,92 @@
+// Shared device/host helpers of the sm_100a GPT-2 training-step library.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#define GPT_HD __host__ __device__ __forceinline__
+
+namespace gpt {
+
+typedef __nv_bfloat16 bf16;
+
+// ----------------------------------------------------------------------------
+// SplitMix64 (Steele, Lea & Flood 2014) used as a counter-based hash: the
+// output of a generator whose state is x before its golden-gamma increment.
+// ----------------------------------------------------------------------------
+GPT_HD uint64_t splitmix64(uint64_t x) {
+  uint64_t z = x + 0x9E3779B97F4A7C15ull;
+  z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+  z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+  return z ^ (z >> 31);
+}
+
+// Dropout sites (GPT-2 placement): 0 embedding output (layer = n_layer),
+// 1 attention probabilities, 2 attention projection output, 3 MLP output.
+struct DropKey {
+  uint64_t key;      // splitmix64(seed ^ splitmix64(counter<<32 ^ layer<<8 ^ site))
+  uint32_t thresh;   // floor(p * 2^32); keep iff hash >> 32 >= thresh
+  float scale;       // 1 / (1 - p)
+  int active;
+};
+
+GPT_HD DropKey make_drop_key(uint64_t seed, uint64_t counter, int layer, int site, float p) {
+  DropKey k;
+  uint64_t tag = (counter << 32) ^ ((uint64_t)layer << 8) ^ (uint64_t)site;
+  k.key = splitmix64(seed ^ splitmix64(tag));
+  double t = (double)p * 4294967296.0;
+  k.thresh = (uint32_t)(t >= 4294967295.0 ? 4294967295.0 : t);
+  k.scale = p > 0.f ? 1.0f / (1.0f - p) : 1.0f;
+  k.active = p > 0.f;
+  return k;
+}
+
+GPT_HD bool drop_keep(const DropKey& k, uint64_t elem) {
+  return (uint32_t)(splitmix64(k.key ^ elem) >> 32) >= k.thresh;
+}
+
+// multiplier applied to an element: 0 or 1/(1-p); 1 when dropout is off
+GPT_HD float drop_mul(const DropKey& k, uint64_t elem) {
+  if (!k.active) return 1.0f;
+  return drop_keep(k, elem) ? k.scale : 0.0f;
+}
+
+// ----------------------------------------------------------------------------
+// type helpers
+// ----------------------------------------------------------------------------
+template <typename T> GPT_HD float to_f(T v);
+template <> GPT_HD float to_f<float>(float v) { return v; }
+template <> GPT_HD float to_f<bf16>(bf16 v) { return __bfloat162float(v); }
+template <typename T> GPT_HD T from_f(float v);
+template <> GPT_HD float from_f<float>(float v) { return v; }
+template <> GPT_HD bf16 from_f<bf16>(float v) { return __float2bfloat16_rn(v); }
+
+// flags (device word in the workspace)
+enum : uint32_t { FLAG_TOKEN = 1u, FLAG_LOSS = 2u, FLAG_NORM = 4u, FLAG_TIMEOUT = 8u };
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+__device__ __forceinline__ double warp_sum_d(double v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// GELU, exact erf form x * Phi(x), and its derivative Phi(x) + x phi(x).
+__device__ __forceinline__ float gelu_f(float x) { return 0.5f * x * (1.0f + erff(x * 0.70710678118654752f)); }
+__device__ __forceinline__ float gelu_grad_f(float x) {
+  float cdf = 0.5f * (1.0f + erff(x * 0.70710678118654752f));
+  float pdf = 0.3989422804014327f * expf(-0.5f * x * x);
+  return cdf + x * pdf;
+}
+
+}  // namespace gpt

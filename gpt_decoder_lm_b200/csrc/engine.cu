@@ -1,0 +1,1098 @@
+// Step engine behind the C ABI of include/gpt.h: validates the config, lays
+// out every device buffer inside the caller's workspace, initialises the
+// weights from the seed, and enqueues the kernels of one training step on the
+// model's stream.  No device allocation happens here.
+#include <math.h>
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <algorithm>
+#include <map>
+#include <string>
+#include <thread>
+#include <vector>
+
+#include "../../include/gpt.h"
+#include "kernels.cuh"
+
+using namespace gpt;
+
+// ============================================================================
+// timing by kernel name (CUDA events on the model's stream)
+// ============================================================================
+namespace gpt {
+struct Timing {
+  struct Rec {
+    std::vector<cudaEvent_t> ev;  // begin/end pairs
+    int launches = 0;
+  };
+  std::map<std::string, Rec> recs;
+  std::vector<cudaEvent_t> pool;
+  size_t used = 0;
+  cudaEvent_t get() {
+    if (used == pool.size()) {
+      cudaEvent_t e;
+      cudaEventCreate(&e);
+      pool.push_back(e);
+    }
+    return pool[used++];
+  }
+  void reset() {
+    recs.clear();
+    used = 0;
+  }
+  ~Timing() {
+    for (auto e : pool) cudaEventDestroy(e);
+  }
+};
+void timing_begin(Ctx& c, const char* name) {
+  auto& r = c.timing->recs[name];
+  cudaEvent_t e = c.timing->get();
+  cudaEventRecord(e, c.stream);
+  r.ev.push_back(e);
+  r.launches++;
+}
+void timing_end(Ctx& c, const char* name) {
+  auto& r = c.timing->recs[name];
+  cudaEvent_t e = c.timing->get();
+  cudaEventRecord(e, c.stream);
+  r.ev.push_back(e);
+}
+}  // namespace gpt
+
+// ============================================================================
+// model
+// ============================================================================
+namespace {
+
+struct TensorRec {
+  std::string name;
+  int64_t rows, cols;   // logical shape (cols = 1 for vectors)
+  int64_t alloc_rows;   // rows in the arena (wte / lm_head: padded vocab)
+  int64_t off;          // element offset in the arenas
+  int init;             // 0 normal, 1 ones, 2 zeros
+  bool decay;
+};
+
+struct LayerP {  // element offsets of one block's tensors (-1 when absent)
+  int64_t ln1_w = -1, ln1_b = -1, qkv_w, qkv_b = -1, ap_w, ap_b = -1, ln2_w = -1, ln2_b = -1, fc_w, fc_b = -1, pr_w,
+          pr_b = -1;
+};
+
+struct Layout {
+  size_t off = 0;
+  size_t take(size_t bytes) {
+    size_t o = off;
+    off += (bytes + 255) & ~size_t(255);
+    return o;
+  }
+};
+
+int choose_splits(long M, long N, long K) {
+  // dW GEMMs: 128x128 tiles; split K until there are ~2 tiles per SM (148 SMs)
+  long tiles = ((M + 127) / 128) * ((N + 127) / 128);
+  long nkb = (K + 63) / 64;
+  if (tiles >= 148) return 1;
+  long s = (2 * 148 + tiles - 1) / tiles;
+  if (s > 16) s = 16;
+  if (s > nkb / 4) s = std::max(1L, nkb / 4);
+  return (int)s;
+}
+
+}  // namespace
+
+struct gpt_model {
+  gpt_config cfg;
+  int V, Vp, L, H, d, T, B, ga, hd;
+  long M;
+  bool bf16m, micro;
+  size_t asz;  // bytes per activation element (2 bf16 / 4 fp32)
+  std::vector<TensorRec> tensors;
+  std::vector<LayerP> layers;
+  int64_t wte, wpe, lnf_w = -1, lnf_b = -1, head;  // offsets
+  int64_t n_total = 0, n_decay = 0;
+
+  uint8_t* ws = nullptr;
+  size_t ws_bytes = 0;
+  // arenas
+  float *w = nullptr, *g = nullptr, *am = nullptr, *av = nullptr;
+  bf16* wb = nullptr;
+  // activations
+  float* res;  // [(2L+1), M, d]
+  uint8_t *ln1, *qkv, *atto, *ln2, *fch, *fcg, *lnf, *logits;
+  float *ln1_mean, *ln1_rstd, *ln2_mean, *ln2_rstd, *lnf_mean, *lnf_rstd, *lse;
+  float *row_loss, *row_lse;
+  int32_t *idx, *tgt, *stage_idx, *stage_tgt;
+  // backward scratch
+  float *dres, *dln, *dsum, *part, *colsum_scr, *splitk;
+  uint8_t *dyb, *dqkv, *datt, *dh;
+  int32_t *stok, *spos, *nuniq;
+  double* norm_part;
+  float* scal;  // [0] micro loss, [1] step loss, [2] grad norm, [3] flags (uint32)
+  int32_t* argmax_out;
+  size_t splitk_floats = 0;
+  int part_blocks = 0;
+
+  Ctx ctx;
+  Timing* timing = nullptr;
+  bool have_forward = false;
+  bool ce_grad_done = false;
+  int64_t drop_counter = 0;
+  uint32_t reported = 0;
+  std::string err;
+
+  float* P(int64_t off) const { return w + off; }
+  float* G(int64_t off) const { return g + off; }
+  const void* Wop(int64_t off) const {  // GEMM operand copy of a weight
+    return bf16m ? (const void*)(wb + off) : (const void*)(w + off);
+  }
+};
+
+namespace {
+
+gpt_status fail(gpt_model* m, gpt_status s, const char* fmt, ...) {
+  if (m) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    m->err = buf;
+  }
+  return s;
+}
+
+gpt_status check_cuda(gpt_model* m, const char* where) {
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(m, GPT_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
+  return GPT_OK;
+}
+
+// Validation of a config; fills derived fields when m != nullptr.
+gpt_status validate(const gpt_config* c, std::string* why) {
+  auto bad = [&](const char* s) {
+    if (why) *why = s;
+    return GPT_ERR_CONFIG;
+  };
+  if (!c) {
+    if (why) *why = "null config";
+    return GPT_ERR_INVALID_ARG;
+  }
+  if (c->abi_version != GPT_ABI_VERSION) return bad("abi_version mismatch");
+  if (c->vocab_size < 2 || c->vocab_size > 65535) return bad("vocab_size must be in [2, 65535]");
+  int Vp = c->padded_vocab ? c->padded_vocab : ((c->vocab_size + 63) / 64) * 64;
+  if (Vp < c->vocab_size || Vp % 64) return bad("padded_vocab must be >= vocab_size and a multiple of 64");
+  if (c->n_layer < 1 || c->n_head < 1 || c->n_embd < 8) return bad("n_layer, n_head >= 1 and n_embd >= 8 required");
+  if (c->n_embd % c->n_head) return bad("n_embd must be divisible by n_head");
+  int hd = c->n_embd / c->n_head;
+  if (hd != 4 && hd != 8 && hd != 16 && hd != 32 && hd != 64 && hd != 128) return bad("head_dim must be 4..128, power of 2");
+  if (c->n_embd % 8) return bad("n_embd must be a multiple of 8");
+  if (c->n_embd > 2048) return bad("n_embd must be <= 2048");
+  if (c->block_size < 1 || c->batch_size < 1 || c->grad_accum < 1) return bad("block_size, batch_size, grad_accum >= 1");
+  long M = (long)c->block_size * c->batch_size;
+  if (M > 32768) return bad("batch_size * block_size must be <= 32768");
+  if (c->precision != GPT_PREC_FP32 && c->precision != GPT_PREC_BF16) return bad("precision");
+  if (c->variant != GPT_VARIANT_GPT2 && c->variant != GPT_VARIANT_MICRO) return bad("variant");
+  if (c->token_dtype != GPT_TOK_I32 && c->token_dtype != GPT_TOK_U16) return bad("token_dtype");
+  if (!(c->dropout >= 0.f && c->dropout < 1.f)) return bad("dropout must be in [0, 1)");
+  if (!(c->beta1 >= 0.f && c->beta1 < 1.f && c->beta2 >= 0.f && c->beta2 < 1.f)) return bad("betas in [0, 1)");
+  if (!(c->eps > 0.f) || !(c->init_std >= 0.f)) return bad("eps > 0 and init_std >= 0 required");
+  return GPT_OK;
+}
+
+// tensor table in canonical order; returns arena sizes
+void build_tensors(gpt_model& m) {
+  int V = m.V, Vp = m.Vp, d = m.d, T = m.T, L = m.L;
+  bool gpt2 = !m.micro;
+  std::vector<TensorRec> t;
+  auto add = [&](const std::string& n, int64_t r, int64_t c, int64_t ar, int init) {
+    TensorRec x;
+    x.name = n;
+    x.rows = r;
+    x.cols = c;
+    x.alloc_rows = ar;
+    x.off = -1;
+    x.init = init;
+    x.decay = (c > 1) || m.cfg.decay_1d;
+    t.push_back(x);
+  };
+  add("wte", V, d, Vp, 0);
+  add("wpe", T, d, T, 0);
+  for (int l = 0; l < L; l++) {
+    std::string p = "h." + std::to_string(l) + ".";
+    if (gpt2) {
+      add(p + "ln_1.weight", d, 1, d, 1);
+      add(p + "ln_1.bias", d, 1, d, 2);
+    }
+    add(p + "attn.c_attn.weight", 3 * d, d, 3 * d, 0);
+    if (gpt2) add(p + "attn.c_attn.bias", 3 * d, 1, 3 * d, 2);
+    add(p + "attn.c_proj.weight", d, d, d, 0);
+    if (gpt2) {
+      add(p + "attn.c_proj.bias", d, 1, d, 2);
+      add(p + "ln_2.weight", d, 1, d, 1);
+      add(p + "ln_2.bias", d, 1, d, 2);
+    }
+    add(p + "mlp.c_fc.weight", 4 * d, d, 4 * d, 0);
+    if (gpt2) add(p + "mlp.c_fc.bias", 4 * d, 1, 4 * d, 2);
+    add(p + "mlp.c_proj.weight", d, 4 * d, d, 0);
+    if (gpt2) add(p + "mlp.c_proj.bias", d, 1, d, 2);
+  }
+  if (gpt2) {
+    add("ln_f.weight", d, 1, d, 1);
+    add("ln_f.bias", d, 1, d, 2);
+  } else {
+    add("lm_head.weight", V, d, Vp, 0);
+  }
+  // arena: decayed tensors first, each aligned to 64 elements
+  int64_t off = 0;
+  for (int pass = 0; pass < 2; pass++) {
+    for (auto& x : t) {
+      if (x.decay != (pass == 0)) continue;
+      x.off = off;
+      off += ((x.alloc_rows * x.cols + 63) / 64) * 64;
+    }
+    if (pass == 0) m.n_decay = off;
+  }
+  m.n_total = off;
+  m.tensors = t;
+  // named offsets
+  auto find = [&](const std::string& n) -> int64_t {
+    for (auto& x : m.tensors)
+      if (x.name == n) return x.off;
+    return -1;
+  };
+  m.wte = find("wte");
+  m.wpe = find("wpe");
+  m.layers.assign(L, LayerP());
+  for (int l = 0; l < L; l++) {
+    std::string p = "h." + std::to_string(l) + ".";
+    LayerP& y = m.layers[l];
+    y.ln1_w = find(p + "ln_1.weight");
+    y.ln1_b = find(p + "ln_1.bias");
+    y.qkv_w = find(p + "attn.c_attn.weight");
+    y.qkv_b = find(p + "attn.c_attn.bias");
+    y.ap_w = find(p + "attn.c_proj.weight");
+    y.ap_b = find(p + "attn.c_proj.bias");
+    y.ln2_w = find(p + "ln_2.weight");
+    y.ln2_b = find(p + "ln_2.bias");
+    y.fc_w = find(p + "mlp.c_fc.weight");
+    y.fc_b = find(p + "mlp.c_fc.bias");
+    y.pr_w = find(p + "mlp.c_proj.weight");
+    y.pr_b = find(p + "mlp.c_proj.bias");
+  }
+  m.lnf_w = find("ln_f.weight");
+  m.lnf_b = find("ln_f.bias");
+  m.head = gpt2 ? m.wte : find("lm_head.weight");
+}
+
+void derive(gpt_model& m, const gpt_config* c) {
+  m.cfg = *c;
+  m.V = c->vocab_size;
+  m.Vp = c->padded_vocab ? c->padded_vocab : ((c->vocab_size + 63) / 64) * 64;
+  m.L = c->n_layer;
+  m.H = c->n_head;
+  m.d = c->n_embd;
+  m.T = c->block_size;
+  m.B = c->batch_size;
+  m.ga = c->grad_accum;
+  m.hd = m.d / m.H;
+  m.M = (long)m.B * m.T;
+  m.bf16m = c->precision == GPT_PREC_BF16;
+  m.micro = c->variant == GPT_VARIANT_MICRO;
+  m.asz = m.bf16m ? 2 : 4;
+  build_tensors(m);
+}
+
+// Carves the workspace (base may be null to size it).  Returns total bytes.
+size_t carve(gpt_model& m, uint8_t* base) {
+  Layout lay;
+  auto F = [&](size_t n) { return (float*)(base + lay.take(n * 4)); };
+  auto Bt = [&](size_t n) { return base + lay.take(n * m.asz); };
+  auto I = [&](size_t n) { return (int32_t*)(base + lay.take(n * 4)); };
+  long M = m.M;
+  int d = m.d, L = m.L;
+  size_t P = (size_t)m.n_total;
+  m.scal = F(64);
+  m.w = F(P);
+  m.g = F(P);
+  m.am = F(P);
+  m.av = F(P);
+  m.wb = m.bf16m ? (bf16*)(base + lay.take(P * 2)) : nullptr;
+  m.res = F((size_t)(2 * L + 1) * M * d);
+  m.ln1 = Bt((size_t)L * M * d);
+  m.ln1_mean = F((size_t)L * M);
+  m.ln1_rstd = F((size_t)L * M);
+  m.qkv = Bt((size_t)L * M * 3 * d);
+  m.atto = Bt((size_t)L * M * d);
+  m.lse = F((size_t)L * M * m.H);
+  m.ln2 = Bt((size_t)L * M * d);
+  m.ln2_mean = F((size_t)L * M);
+  m.ln2_rstd = F((size_t)L * M);
+  m.fch = Bt((size_t)L * M * 4 * d);
+  m.fcg = Bt((size_t)L * M * 4 * d);
+  m.lnf = Bt((size_t)M * d);
+  m.lnf_mean = F(M);
+  m.lnf_rstd = F(M);
+  m.logits = Bt((size_t)M * m.Vp);
+  m.row_loss = F(M);
+  m.row_lse = F(M);
+  m.idx = I(M);
+  m.tgt = I(M);
+  m.stage_idx = I((size_t)m.ga * M);
+  m.stage_tgt = I((size_t)m.ga * M);
+  m.dres = F((size_t)M * d);
+  m.dln = F((size_t)M * d);
+  m.dsum = F((size_t)M * m.H);
+  m.part_blocks = (int)std::min<long>(M, 148 * 4);
+  m.part = F((size_t)m.part_blocks * 3 * d);
+  m.colsum_scr = F((size_t)64 * 4 * d);
+  // split-K scratch: the largest dW partial set
+  size_t sk = 0;
+  long shapes[4][2] = {{3L * d, d}, {d, d}, {4L * d, d}, {d, 4L * d}};
+  for (auto& s : shapes) {
+    int sp = choose_splits(s[0], s[1], M);
+    if (sp > 1) sk = std::max(sk, (size_t)sp * s[0] * s[1]);
+  }
+  {
+    int sp = choose_splits(m.Vp, d, M);
+    if (sp > 1) sk = std::max(sk, (size_t)sp * m.Vp * d);
+  }
+  m.splitk_floats = sk;
+  m.splitk = F(std::max<size_t>(sk, 64));
+  m.dyb = Bt((size_t)M * d);
+  m.dqkv = Bt((size_t)M * 3 * d);
+  m.datt = Bt((size_t)M * d);
+  m.dh = Bt((size_t)M * 4 * d);
+  m.stok = I(M);
+  m.spos = I(M);
+  m.nuniq = I(64);
+  m.norm_part = (double*)(base + lay.take(148 * 4 * 8 + 64));
+  m.argmax_out = I(M + 64);
+  return lay.off + 1024;
+}
+
+// ---------------------------------------------------------------- host init
+uint64_t sm64(uint64_t x) { return splitmix64(x); }
+
+void init_tensor_host(const TensorRec& t, float std_, uint64_t seed, int index, float* out /* rows*cols */) {
+  int64_t n = t.rows * t.cols;
+  if (t.init == 1) {
+    std::fill(out, out + n, 1.0f);
+    return;
+  }
+  if (t.init == 2) {
+    std::fill(out, out + n, 0.0f);
+    return;
+  }
+  uint64_t k = sm64(seed ^ sm64((uint64_t)index));
+  unsigned nt = std::max(1u, std::min(64u, std::thread::hardware_concurrency()));
+  if (n < (1 << 16)) nt = 1;
+  std::vector<std::thread> th;
+  for (unsigned w = 0; w < nt; w++) {
+    th.emplace_back([=] {
+      int64_t a = n * w / nt, b = n * (w + 1) / nt;
+      for (int64_t e = a; e < b; e++) {
+        uint64_t b1 = sm64(k ^ (uint64_t)(2 * e));
+        uint64_t b2 = sm64(k ^ (uint64_t)(2 * e + 1));
+        double u1 = ((double)(b1 >> 11) + 1.0) * (1.0 / 9007199254740992.0);
+        double u2 = (double)(b2 >> 11) * (1.0 / 9007199254740992.0);
+        double z = sqrt(-2.0 * log(u1)) * cos(2.0 * 3.14159265358979323846 * u2);
+        out[e] = (float)((double)std_ * z);
+      }
+    });
+  }
+  for (auto& x : th) x.join();
+}
+
+gpt_status sync_and_flags(gpt_model* m, const char* where, float* h_scal /* 4 floats or null */) {
+  float tmp[4];
+  cudaMemcpyAsync(tmp, m->scal, 16, cudaMemcpyDeviceToHost, m->ctx.stream);
+  cudaError_t e = cudaStreamSynchronize(m->ctx.stream);
+  if (e != cudaSuccess) return fail(m, GPT_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
+  if (h_scal) memcpy(h_scal, tmp, 16);
+  uint32_t fl;
+  memcpy(&fl, &tmp[3], 4);
+  uint32_t fresh = fl & ~m->reported;
+  m->reported |= fl;
+  if (fresh & FLAG_TIMEOUT) return fail(m, GPT_ERR_TIMEOUT, "%s: a bounded device wait ran out", where);
+  if (fresh & FLAG_TOKEN) return fail(m, GPT_ERR_TOKEN_RANGE, "%s: token id outside [0, vocab_size)", where);
+  if (fresh & (FLAG_LOSS | FLAG_NORM)) return fail(m, GPT_ERR_NONFINITE, "%s: non-finite loss or gradient norm", where);
+  return GPT_OK;
+}
+
+// ---------------------------------------------------------------- step pieces
+bool gemm(gpt_model* m, GemmDesc& g) {
+  if (!m->bf16m) {
+    gemm_simt_f32(m->ctx, g);
+    return true;
+  }
+  if (gemm_tc_supported(g)) return gemm_tc_bf16(m->ctx, g);
+  gemm_simt_bf16(m->ctx, g);
+  return true;
+}
+
+GemmDesc gd(int M, int N, int K, const void* A, long lda, bool ak, const void* B, long ldb, bool bk) {
+  GemmDesc g;
+  g.M = M;
+  g.N = N;
+  g.K = K;
+  g.A = A;
+  g.lda = lda;
+  g.a_kmajor = ak;
+  g.B = B;
+  g.ldb = ldb;
+  g.b_kmajor = bk;
+  return g;
+}
+
+DropKey dkey(gpt_model* m, int layer, int site) {
+  return make_drop_key(m->cfg.dropout_seed, (uint64_t)m->drop_counter, layer, site, m->cfg.dropout);
+}
+
+template <typename T> T* at(uint8_t* base, size_t elems) { return reinterpret_cast<T*>(base) + elems; }
+
+template <typename T>
+gpt_status forward_t(gpt_model* m, bool fuse_ce_grad, float* loss_acc, float loss_scale, int accumulate) {
+  Ctx& c = m->ctx;
+  long M = m->M;
+  int d = m->d, L = m->L;
+  bool rms = m->micro;
+  float eps = 1e-5f;
+  int act = m->micro ? ACT_RELU : ACT_GELU;
+  size_t Md = (size_t)M * d;
+  embed_fwd<T>(c, m->idx, m->P(m->wte), m->P(m->wpe), m->res, m->B, m->T, d, dkey(m, L, 0));
+  for (int l = 0; l < L; l++) {
+    const LayerP& y = m->layers[l];
+    float* x = m->res + (size_t)(2 * l) * Md;
+    float* xm = m->res + (size_t)(2 * l + 1) * Md;
+    float* xo = m->res + (size_t)(2 * l + 2) * Md;
+    T* a1 = at<T>(m->ln1, l * Md);
+    T* qkv = at<T>(m->qkv, l * 3 * Md);
+    T* o = at<T>(m->atto, l * Md);
+    T* a2 = at<T>(m->ln2, l * Md);
+    T* h = at<T>(m->fch, l * 4 * Md);
+    T* gg = at<T>(m->fcg, l * 4 * Md);
+    norm_fwd<T>(c, x, rms ? nullptr : m->P(y.ln1_w), rms ? nullptr : m->P(y.ln1_b), a1, m->ln1_mean + l * M,
+                m->ln1_rstd + l * M, M, d, rms, eps);
+    GemmDesc g = gd((int)M, 3 * d, d, a1, d, true, m->Wop(y.qkv_w), d, true);
+    g.epi.kind = EPI_BIAS;
+    g.epi.bias = y.qkv_b >= 0 ? m->P(y.qkv_b) : nullptr;
+    g.epi.out = qkv;
+    g.epi.ldo = 3 * d;
+    if (!gemm(m, g)) return fail(m, GPT_ERR_CUDA, "qkv gemm: tensor map encode failed");
+    AttnDesc ad{m->B, m->T, m->H, m->hd, qkv, o, m->lse + (size_t)l * M * m->H, nullptr, nullptr, nullptr,
+                dkey(m, l, 1)};
+    if (sizeof(T) == 2 && attn_tc_supported(ad)) attn_fwd_tc(c, ad);
+    else attn_fwd_simt<T>(c, ad);
+    g = gd((int)M, d, d, o, d, true, m->Wop(y.ap_w), d, true);
+    g.epi.kind = EPI_RESADD;
+    g.epi.bias = y.ap_b >= 0 ? m->P(y.ap_b) : nullptr;
+    g.epi.res_in = x;
+    g.epi.res_out = xm;
+    g.epi.ld_res = d;
+    g.epi.ldo = d;
+    g.epi.drop = dkey(m, l, 2);
+    if (!gemm(m, g)) return fail(m, GPT_ERR_CUDA, "attn proj gemm failed");
+    norm_fwd<T>(c, xm, rms ? nullptr : m->P(y.ln2_w), rms ? nullptr : m->P(y.ln2_b), a2, m->ln2_mean + l * M,
+                m->ln2_rstd + l * M, M, d, rms, eps);
+    g = gd((int)M, 4 * d, d, a2, d, true, m->Wop(y.fc_w), d, true);
+    g.epi.kind = EPI_BIAS_ACT;
+    g.epi.act = act;
+    g.epi.bias = y.fc_b >= 0 ? m->P(y.fc_b) : nullptr;
+    g.epi.out = h;
+    g.epi.out2 = gg;
+    g.epi.ldo = 4 * d;
+    if (!gemm(m, g)) return fail(m, GPT_ERR_CUDA, "fc gemm failed");
+    g = gd((int)M, d, 4 * d, gg, 4 * d, true, m->Wop(y.pr_w), 4 * d, true);
+    g.epi.kind = EPI_RESADD;
+    g.epi.bias = y.pr_b >= 0 ? m->P(y.pr_b) : nullptr;
+    g.epi.res_in = xm;
+    g.epi.res_out = xo;
+    g.epi.ld_res = d;
+    g.epi.ldo = d;
+    g.epi.drop = dkey(m, l, 3);
+    if (!gemm(m, g)) return fail(m, GPT_ERR_CUDA, "mlp proj gemm failed");
+  }
+  T* xf = reinterpret_cast<T*>(m->lnf);
+  norm_fwd<T>(c, m->res + (size_t)(2 * L) * Md, rms ? nullptr : m->P(m->lnf_w), rms ? nullptr : m->P(m->lnf_b), xf,
+              m->lnf_mean, m->lnf_rstd, M, d, rms, eps);
+  GemmDesc g = gd((int)M, m->Vp, d, xf, d, true, m->Wop(m->head), d, true);
+  g.epi.kind = EPI_STORE;
+  g.epi.out = m->logits;
+  g.epi.ldo = m->Vp;
+  if (!gemm(m, g)) return fail(m, GPT_ERR_CUDA, "lm_head gemm failed");
+  ce_fwd_bwd<T>(c, reinterpret_cast<T*>(m->logits), m->tgt, M, m->V, m->Vp, m->row_lse, m->row_loss, fuse_ce_grad,
+                1.0f / (float)(M * m->ga));
+  loss_reduce(c, m->row_loss, M, loss_scale, loss_acc, accumulate);
+  m->have_forward = true;
+  m->ce_grad_done = fuse_ce_grad;
+  return check_cuda(m, "forward");
+}
+
+void add_bias_grads_from_norm(gpt_model* m, int64_t gain, int64_t beta, int64_t next_bias) {
+  Ctx& c = m->ctx;
+  if (gain >= 0) partial_reduce(c, m->part, m->part_blocks, 3, 0, m->d, m->G(gain));
+  if (beta >= 0) partial_reduce(c, m->part, m->part_blocks, 3, 1, m->d, m->G(beta));
+  if (next_bias >= 0) partial_reduce(c, m->part, m->part_blocks, 3, 2, m->d, m->G(next_bias));
+}
+
+template <typename T>
+gpt_status backward_t(gpt_model* m) {
+  Ctx& c = m->ctx;
+  long M = m->M;
+  int d = m->d, L = m->L, Vp = m->Vp;
+  bool rms = m->micro;
+  int act = m->micro ? ACT_RELU : ACT_GELU;
+  size_t Md = (size_t)M * d;
+  T* dl = reinterpret_cast<T*>(m->logits);
+  if (!m->ce_grad_done)
+    ce_fwd_bwd<T>(c, dl, m->tgt, M, m->V, Vp, m->row_lse, m->row_loss, true, 1.0f / (float)(M * m->ga));
+  m->ce_grad_done = true;
+  T* dyb = reinterpret_cast<T*>(m->dyb);
+  T* dh = reinterpret_cast<T*>(m->dh);
+  T* dqkv = reinterpret_cast<T*>(m->dqkv);
+  T* datt = reinterpret_cast<T*>(m->datt);
+  auto dW = [&](int Mo, int No, const void* A, const void* Bm, float* out) -> bool {
+    // out[Mo, No] += A^T B with A [M, Mo], B [M, No] (tokens outermost)
+    GemmDesc g = gd(Mo, No, (int)M, A, Mo, false, Bm, No, false);
+    g.epi.kind = EPI_ACC_F32;
+    g.epi.out = out;
+    g.epi.ldo = No;
+    if (m->bf16m) {
+      g.split_k = choose_splits(Mo, No, M);
+      g.partial = m->splitk;
+    }
+    return gemm(m, g);
+  };
+  // lm_head: dx_f = dlogits W_head; dW_head += dlogits^T x_f
+  GemmDesc g = gd((int)M, d, Vp, dl, Vp, true, m->Wop(m->head), d, false);
+  g.epi.kind = EPI_STORE_F32;
+  g.epi.out = m->dln;
+  g.epi.ldo = d;
+  if (!gemm(m, g)) return fail(m, GPT_ERR_CUDA, "lm_head dX gemm failed");
+  if (!dW(Vp, d, dl, m->lnf, m->G(m->head))) return fail(m, GPT_ERR_CUDA, "lm_head dW gemm failed");
+  // final norm
+  NormBwd nb;
+  nb.dy = m->dln;
+  nb.x = m->res + (size_t)(2 * L) * Md;
+  nb.mean = m->lnf_mean;
+  nb.rstd = m->lnf_rstd;
+  nb.w = rms ? nullptr : m->P(m->lnf_w);
+  nb.dres = m->dres;
+  nb.accumulate = false;
+  nb.dyb = dyb;
+  nb.drop = dkey(m, L - 1, 3);
+  nb.want_dyb = true;
+  nb.part = m->part;
+  nb.blocks = m->part_blocks;
+  nb.rows = M;
+  nb.d = d;
+  nb.rms = rms;
+  norm_bwd<T>(c, nb);
+  add_bias_grads_from_norm(m, m->lnf_w, m->lnf_b, m->layers[L - 1].pr_b);
+  for (int l = L - 1; l >= 0; l--) {
+    const LayerP& y = m->layers[l];
+    T* a1 = at<T>(m->ln1, l * Md);
+    T* qkv = at<T>(m->qkv, l * 3 * Md);
+    T* o = at<T>(m->atto, l * Md);
+    T* a2 = at<T>(m->ln2, l * Md);
+    T* h = at<T>(m->fch, l * 4 * Md);
+    T* gg = at<T>(m->fcg, l * 4 * Md);
+    // MLP projection
+    if (!dW(d, 4 * d, dyb, gg, m->G(y.pr_w))) return fail(m, GPT_ERR_CUDA, "proj dW failed");
+    g = gd((int)M, 4 * d, d, dyb, d, true, m->Wop(y.pr_w), 4 * d, false);
+    g.epi.kind = EPI_ACT_BWD;
+    g.epi.act = act;
+    g.epi.aux = h;
+    g.epi.out = dh;
+    g.epi.ldo = 4 * d;
+    if (!gemm(m, g)) return fail(m, GPT_ERR_CUDA, "proj dX failed");
+    if (y.fc_b >= 0) colsum_acc<T>(c, dh, M, 4 * d, m->colsum_scr, m->G(y.fc_b));
+    if (!dW(4 * d, d, dh, a2, m->G(y.fc_w))) return fail(m, GPT_ERR_CUDA, "fc dW failed");
+    g = gd((int)M, d, 4 * d, dh, 4 * d, true, m->Wop(y.fc_w), d, false);
+    g.epi.kind = EPI_STORE_F32;
+    g.epi.out = m->dln;
+    g.epi.ldo = d;
+    if (!gemm(m, g)) return fail(m, GPT_ERR_CUDA, "fc dX failed");
+    nb.dy = m->dln;
+    nb.x = m->res + (size_t)(2 * l + 1) * Md;
+    nb.mean = m->ln2_mean + l * M;
+    nb.rstd = m->ln2_rstd + l * M;
+    nb.w = rms ? nullptr : m->P(y.ln2_w);
+    nb.accumulate = true;
+    nb.drop = dkey(m, l, 2);
+    nb.want_dyb = true;
+    norm_bwd<T>(c, nb);
+    add_bias_grads_from_norm(m, y.ln2_w, y.ln2_b, y.ap_b);
+    // attention projection
+    if (!dW(d, d, dyb, o, m->G(y.ap_w))) return fail(m, GPT_ERR_CUDA, "attn proj dW failed");
+    g = gd((int)M, d, d, dyb, d, true, m->Wop(y.ap_w), d, false);
+    g.epi.kind = EPI_STORE;
+    g.epi.out = datt;
+    g.epi.ldo = d;
+    if (!gemm(m, g)) return fail(m, GPT_ERR_CUDA, "attn proj dX failed");
+    AttnDesc ad{m->B, m->T, m->H, m->hd, qkv, o, m->lse + (size_t)l * M * m->H, datt, dqkv, m->dsum, dkey(m, l, 1)};
+    if (sizeof(T) == 2 && attn_tc_supported(ad)) attn_bwd_tc(c, ad);
+    else attn_bwd_simt<T>(c, ad);
+    if (y.qkv_b >= 0) colsum_acc<T>(c, dqkv, M, 3 * d, m->colsum_scr, m->G(y.qkv_b));
+    if (!dW(3 * d, d, dqkv, a1, m->G(y.qkv_w))) return fail(m, GPT_ERR_CUDA, "qkv dW failed");
+    g = gd((int)M, d, 3 * d, dqkv, 3 * d, true, m->Wop(y.qkv_w), d, false);
+    g.epi.kind = EPI_STORE_F32;
+    g.epi.out = m->dln;
+    g.epi.ldo = d;
+    if (!gemm(m, g)) return fail(m, GPT_ERR_CUDA, "qkv dX failed");
+    nb.dy = m->dln;
+    nb.x = m->res + (size_t)(2 * l) * Md;
+    nb.mean = m->ln1_mean + l * M;
+    nb.rstd = m->ln1_rstd + l * M;
+    nb.w = rms ? nullptr : m->P(y.ln1_w);
+    nb.accumulate = true;
+    nb.drop = l > 0 ? dkey(m, l - 1, 3) : DropKey{};
+    nb.want_dyb = l > 0;
+    norm_bwd<T>(c, nb);
+    add_bias_grads_from_norm(m, y.ln1_w, y.ln1_b, l > 0 ? m->layers[l - 1].pr_b : -1);
+  }
+  embed_sort(c, m->idx, M, m->stok, m->spos, m->nuniq);
+  embed_bwd(c, m->dres, m->stok, m->spos, M, m->T, m->B, d, dkey(m, L, 0), m->G(m->wte), m->G(m->wpe));
+  return check_cuda(m, "backward");
+}
+
+gpt_status forward_any(gpt_model* m, bool fuse, float* acc, float scale, int accumulate) {
+  return m->bf16m ? forward_t<bf16>(m, fuse, acc, scale, accumulate)
+                  : forward_t<float>(m, fuse, acc, scale, accumulate);
+}
+gpt_status backward_any(gpt_model* m) { return m->bf16m ? backward_t<bf16>(m) : backward_t<float>(m); }
+
+gpt_status adamw_step(gpt_model* m, float lr, int step) {
+  Ctx& c = m->ctx;
+  int blocks = sumsq_blocks(c);
+  sumsq_partials(c, m->g, m->n_total, m->norm_part, blocks);
+  AdamArgs a;
+  a.w = m->w;
+  a.g = m->g;
+  a.m = m->am;
+  a.v = m->av;
+  a.wb = m->wb;
+  a.n = m->n_total;
+  a.n_decay = m->n_decay;
+  a.norm_partials = m->norm_part;
+  a.norm_blocks = blocks;
+  a.norm_out = m->scal + 2;
+  a.lr = lr;
+  a.beta1 = m->cfg.beta1;
+  a.beta2 = m->cfg.beta2;
+  a.eps = m->cfg.eps;
+  a.wd = m->cfg.weight_decay;
+  a.clip = m->cfg.grad_clip;
+  a.bc1 = (float)(1.0 - pow((double)m->cfg.beta1, (double)step));
+  a.bc2 = (float)(1.0 - pow((double)m->cfg.beta2, (double)step));
+  adamw(c, a);
+  return check_cuda(m, "adamw");
+}
+
+}  // namespace
+
+// ============================================================================
+// C ABI
+// ============================================================================
+extern "C" {
+
+const char* gpt_status_string(gpt_status s) {
+  switch (s) {
+    case GPT_OK: return "ok";
+    case GPT_ERR_INVALID_ARG: return "invalid argument";
+    case GPT_ERR_CONFIG: return "invalid config";
+    case GPT_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
+    case GPT_ERR_CUDA: return "CUDA error";
+    case GPT_ERR_TOKEN_RANGE: return "token id out of range";
+    case GPT_ERR_NONFINITE: return "non-finite value";
+    case GPT_ERR_STATE: return "call out of sequence";
+    case GPT_ERR_UNSUPPORTED: return "unsupported";
+    case GPT_ERR_TIMEOUT: return "device wait timed out";
+  }
+  return "unknown status";
+}
+
+const char* gpt_last_error(const gpt_model* m) { return m ? m->err.c_str() : "null model"; }
+
+size_t gpt_param_count(const gpt_config* c) {
+  if (validate(c, nullptr) != GPT_OK) return 0;
+  size_t V = c->vocab_size, d = c->n_embd, T = c->block_size, L = c->n_layer;
+  if (c->variant == GPT_VARIANT_GPT2) return V * d + T * d + L * (12 * d * d + 13 * d) + 2 * d;
+  return 2 * V * d + T * d + 12 * L * d * d;
+}
+
+gpt_status gpt_workspace_bytes(const gpt_config* c, size_t* out) {
+  if (!out) return GPT_ERR_INVALID_ARG;
+  gpt_status s = validate(c, nullptr);
+  if (s != GPT_OK) return s;
+  gpt_model m;
+  derive(m, c);
+  *out = carve(m, nullptr);
+  return GPT_OK;
+}
+
+float gpt_lr_cosine(float lr, int32_t it, int32_t warmup, int32_t max_iters) {
+  if (it < warmup) return (float)((double)lr * it / warmup);
+  double r = (double)(it - warmup) / (double)(max_iters - warmup);
+  return (float)((double)lr * 0.5 * (1.0 + cos(3.14159265358979323846 * r)));
+}
+
+float gpt_lr_linear(float lr, int32_t it, int32_t max_iters) {
+  return (float)((double)lr * (1.0 - (double)it / (double)max_iters));
+}
+
+gpt_status gpt_create(const gpt_config* cfg, uint64_t seed, void* d_workspace, size_t bytes, void* cuda_stream,
+                      gpt_model** out) {
+  if (!out || !d_workspace) return GPT_ERR_INVALID_ARG;
+  *out = nullptr;
+  std::string why;
+  gpt_status s = validate(cfg, &why);
+  if (s != GPT_OK) return s;
+  gpt_model* m = new gpt_model();
+  derive(*m, cfg);
+  size_t need = carve(*m, nullptr);
+  if (bytes < need) {
+    delete m;
+    return GPT_ERR_WORKSPACE_TOO_SMALL;
+  }
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(d_workspace) + 1023) & ~uintptr_t(1023));
+  carve(*m, base);
+  m->ws = (uint8_t*)d_workspace;
+  m->ws_bytes = bytes;
+  m->ctx.stream = (cudaStream_t)cuda_stream;
+  m->ctx.flags = reinterpret_cast<uint32_t*>(m->scal + 3);
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess) m->ctx.num_sms = sms;
+  cudaStream_t st = m->ctx.stream;
+  // zero the arenas (weights, grads, moments) and the scalars
+  cudaMemsetAsync(m->scal, 0, 64 * 4, st);
+  cudaMemsetAsync(m->w, 0, (size_t)m->n_total * 4, st);
+  cudaMemsetAsync(m->g, 0, (size_t)m->n_total * 4, st);
+  cudaMemsetAsync(m->am, 0, (size_t)m->n_total * 4, st);
+  cudaMemsetAsync(m->av, 0, (size_t)m->n_total * 4, st);
+  // weights from the seed, uploaded one tensor at a time
+  std::vector<float> host;
+  for (size_t i = 0; i < m->tensors.size(); i++) {
+    const TensorRec& t = m->tensors[i];
+    host.resize((size_t)t.rows * t.cols);
+    init_tensor_host(t, cfg->init_std, seed, (int)i, host.data());
+    cudaMemcpyAsync(m->w + t.off, host.data(), host.size() * 4, cudaMemcpyHostToDevice, st);
+    cudaStreamSynchronize(st);
+  }
+  if (m->bf16m) to_bf16(m->ctx, m->w, m->wb, m->n_total);
+  cudaError_t e = cudaStreamSynchronize(st);
+  if (e == cudaSuccess) e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    delete m;
+    return GPT_ERR_CUDA;
+  }
+  *out = m;
+  return GPT_OK;
+}
+
+void gpt_destroy(gpt_model* m) {
+  if (!m) return;
+  delete m->timing;
+  delete m;
+}
+
+gpt_status gpt_set_stream(gpt_model* m, void* st) {
+  if (!m) return GPT_ERR_INVALID_ARG;
+  m->ctx.stream = (cudaStream_t)st;
+  return GPT_OK;
+}
+
+gpt_status gpt_set_dropout_cursor(gpt_model* m, int32_t step, int32_t micro) {
+  if (!m || step < 0 || micro < 0) return GPT_ERR_INVALID_ARG;
+  m->drop_counter = (int64_t)step * m->ga + micro;
+  return GPT_OK;
+}
+
+gpt_status gpt_forward_loss(gpt_model* m, const int32_t* d_idx, const int32_t* d_tgt, float* h_loss) {
+  if (!m || !d_idx || !d_tgt) return fail(m, GPT_ERR_INVALID_ARG, "forward_loss: null argument");
+  check_tokens(m->ctx, d_idx, d_tgt, m->M, m->V, m->idx, m->tgt);
+  gpt_status s = forward_any(m, false, m->scal + 0, 1.0f / (float)m->M, 0);
+  if (s != GPT_OK) return s;
+  if (h_loss) {
+    float sc[4];
+    s = sync_and_flags(m, "forward_loss", sc);
+    *h_loss = sc[0];
+  }
+  return s;
+}
+
+gpt_status gpt_backward(gpt_model* m) {
+  if (!m) return GPT_ERR_INVALID_ARG;
+  if (!m->have_forward) return fail(m, GPT_ERR_STATE, "backward called without a preceding forward_loss");
+  gpt_status s = backward_any(m);
+  m->have_forward = false;
+  return s;
+}
+
+gpt_status gpt_clip_adamw_step(gpt_model* m, float lr, int32_t step, float* h_grad_norm) {
+  if (!m) return GPT_ERR_INVALID_ARG;
+  if (step < 1) return fail(m, GPT_ERR_INVALID_ARG, "step must be >= 1");
+  gpt_status s = adamw_step(m, lr, step);
+  if (s != GPT_OK) return s;
+  if (h_grad_norm) {
+    float sc[4];
+    s = sync_and_flags(m, "clip_adamw_step", sc);
+    *h_grad_norm = sc[2];
+  }
+  return s;
+}
+
+static gpt_status train_common(gpt_model* m, const void* d_stream, uint64_t len, uint64_t seed, const int32_t* h_idx,
+                               const int32_t* h_tgt, float lr, int32_t step, float* h_loss, float* h_norm) {
+  if (step < 1) return fail(m, GPT_ERR_INVALID_ARG, "step must be >= 1");
+  Ctx& c = m->ctx;
+  for (int mu = 0; mu < m->ga; mu++) {
+    m->drop_counter = (int64_t)step * m->ga + mu;
+    if (d_stream) {
+      gather_batch(c, d_stream, m->cfg.token_dtype == GPT_TOK_U16, len, seed, step, mu, m->B, m->T, m->V, m->idx,
+                   m->tgt);
+    } else {
+      int32_t* si = m->stage_idx + (size_t)mu * m->M;
+      int32_t* stg = m->stage_tgt + (size_t)mu * m->M;
+      check_tokens(c, si, stg, m->M, m->V, m->idx, m->tgt);
+    }
+    gpt_status s = forward_any(m, true, m->scal + 1, 1.0f / (float)(m->M * m->ga), mu > 0);
+    if (s != GPT_OK) return s;
+    s = backward_any(m);
+    if (s != GPT_OK) return s;
+  }
+  m->have_forward = false;
+  gpt_status s = adamw_step(m, lr, step);
+  if (s != GPT_OK) return s;
+  if (h_loss || h_norm) {
+    float sc[4];
+    s = sync_and_flags(m, "train_step", sc);
+    if (h_loss) *h_loss = sc[1];
+    if (h_norm) *h_norm = sc[2];
+  }
+  return s;
+}
+
+gpt_status gpt_train_step(gpt_model* m, const void* d_stream, uint64_t stream_len, uint64_t data_seed, float lr,
+                          int32_t step, float* h_loss, float* h_grad_norm) {
+  if (!m || !d_stream) return fail(m, GPT_ERR_INVALID_ARG, "train_step: null argument");
+  if (stream_len <= (uint64_t)m->T) return fail(m, GPT_ERR_INVALID_ARG, "stream shorter than block_size + 1");
+  return train_common(m, d_stream, stream_len, data_seed, nullptr, nullptr, lr, step, h_loss, h_grad_norm);
+}
+
+gpt_status gpt_train_step_host(gpt_model* m, const int32_t* h_idx, const int32_t* h_tgt, float lr, int32_t step,
+                               float* h_loss, float* h_grad_norm) {
+  if (!m || !h_idx || !h_tgt) return fail(m, GPT_ERR_INVALID_ARG, "train_step_host: null argument");
+  size_t bytes = (size_t)m->ga * m->M * 4;
+  cudaMemcpyAsync(m->stage_idx, h_idx, bytes, cudaMemcpyHostToDevice, m->ctx.stream);
+  cudaMemcpyAsync(m->stage_tgt, h_tgt, bytes, cudaMemcpyHostToDevice, m->ctx.stream);
+  return train_common(m, nullptr, 0, 0, h_idx, h_tgt, lr, step, h_loss, h_grad_norm);
+}
+
+gpt_status gpt_gather_batch(gpt_model* m, const void* d_stream, uint64_t stream_len, uint64_t data_seed, int32_t step,
+                            int32_t micro, int32_t* d_idx, int32_t* d_tgt) {
+  if (!m || !d_stream || !d_idx || !d_tgt) return fail(m, GPT_ERR_INVALID_ARG, "gather_batch: null argument");
+  if (stream_len <= (uint64_t)m->T) return fail(m, GPT_ERR_INVALID_ARG, "stream shorter than block_size + 1");
+  gather_batch(m->ctx, d_stream, m->cfg.token_dtype == GPT_TOK_U16, stream_len, data_seed, step, micro, m->B, m->T,
+               m->V, d_idx, d_tgt);
+  return check_cuda(m, "gather_batch");
+}
+
+gpt_status gpt_num_tensors(gpt_model* m, int32_t* n) {
+  if (!m || !n) return GPT_ERR_INVALID_ARG;
+  *n = (int32_t)m->tensors.size();
+  return GPT_OK;
+}
+
+gpt_status gpt_tensor_info(gpt_model* m, int32_t i, const char** name, int64_t shape[2]) {
+  if (!m || i < 0 || i >= (int32_t)m->tensors.size()) return GPT_ERR_INVALID_ARG;
+  if (name) *name = m->tensors[i].name.c_str();
+  if (shape) {
+    shape[0] = m->tensors[i].rows;
+    shape[1] = m->tensors[i].cols;
+  }
+  return GPT_OK;
+}
+
+static float* kind_arena(gpt_model* m, int kind) {
+  switch (kind) {
+    case GPT_PARAM: return m->w;
+    case GPT_GRAD: return m->g;
+    case GPT_ADAM_M: return m->am;
+    case GPT_ADAM_V: return m->av;
+  }
+  return nullptr;
+}
+
+gpt_status gpt_get_tensor(gpt_model* m, int32_t i, int32_t kind, float* h_out) {
+  if (!m || !h_out || i < 0 || i >= (int32_t)m->tensors.size()) return GPT_ERR_INVALID_ARG;
+  float* a = kind_arena(m, kind);
+  if (!a) return GPT_ERR_INVALID_ARG;
+  const TensorRec& t = m->tensors[i];
+  cudaMemcpyAsync(h_out, a + t.off, (size_t)t.rows * t.cols * 4, cudaMemcpyDeviceToHost, m->ctx.stream);
+  return sync_and_flags(m, "get_tensor", nullptr);
+}
+
+gpt_status gpt_set_tensor(gpt_model* m, int32_t i, int32_t kind, const float* h_in) {
+  if (!m || !h_in || i < 0 || i >= (int32_t)m->tensors.size()) return GPT_ERR_INVALID_ARG;
+  float* a = kind_arena(m, kind);
+  if (!a) return GPT_ERR_INVALID_ARG;
+  const TensorRec& t = m->tensors[i];
+  size_t n = (size_t)t.rows * t.cols;
+  cudaMemcpyAsync(a + t.off, h_in, n * 4, cudaMemcpyHostToDevice, m->ctx.stream);
+  if (kind == GPT_PARAM && m->bf16m) to_bf16(m->ctx, m->w + t.off, m->wb + t.off, (long)n);
+  return sync_and_flags(m, "set_tensor", nullptr);
+}
+
+gpt_status gpt_get_logits(gpt_model* m, float* h_out) {
+  if (!m || !h_out) return GPT_ERR_INVALID_ARG;
+  gpt_status s = sync_and_flags(m, "get_logits", nullptr);
+  if (s != GPT_OK) return s;
+  size_t rows = m->M;
+  if (m->bf16m) {
+    std::vector<uint16_t> tmp((size_t)rows * m->Vp);
+    cudaMemcpy(tmp.data(), m->logits, tmp.size() * 2, cudaMemcpyDeviceToHost);
+    for (size_t r = 0; r < rows; r++)
+      for (int j = 0; j < m->V; j++) {
+        uint32_t u = (uint32_t)tmp[r * m->Vp + j] << 16;
+        memcpy(&h_out[r * m->V + j], &u, 4);
+      }
+  } else {
+    cudaMemcpy2D(h_out, (size_t)m->V * 4, m->logits, (size_t)m->Vp * 4, (size_t)m->V * 4, rows,
+                 cudaMemcpyDeviceToHost);
+  }
+  return check_cuda(m, "get_logits");
+}
+
+gpt_status gpt_get_argmax(gpt_model* m, int32_t* h_out) {
+  if (!m || !h_out) return GPT_ERR_INVALID_ARG;
+  argmax_rows(m->ctx, m->logits, m->bf16m ? 1 : 0, m->M, m->V, m->Vp, m->argmax_out);
+  cudaMemcpyAsync(h_out, m->argmax_out, (size_t)m->M * 4, cudaMemcpyDeviceToHost, m->ctx.stream);
+  return sync_and_flags(m, "get_argmax", nullptr);
+}
+
+gpt_status gpt_argmax_rows(gpt_model* m, const float* d_rows, int32_t rows, int32_t cols, int32_t* h_out) {
+  if (!m || !d_rows || !h_out || rows <= 0 || cols <= 0 || rows > m->M + 64) return GPT_ERR_INVALID_ARG;
+  argmax_rows(m->ctx, d_rows, 0, rows, cols, cols, m->argmax_out);
+  cudaMemcpyAsync(h_out, m->argmax_out, (size_t)rows * 4, cudaMemcpyDeviceToHost, m->ctx.stream);
+  return sync_and_flags(m, "argmax_rows", nullptr);
+}
+
+gpt_status gpt_get_lse(gpt_model* m, float* h_out) {
+  if (!m || !h_out) return GPT_ERR_INVALID_ARG;
+  cudaMemcpyAsync(h_out, m->row_lse, (size_t)m->M * 4, cudaMemcpyDeviceToHost, m->ctx.stream);
+  return sync_and_flags(m, "get_lse", nullptr);
+}
+
+gpt_status gpt_get_embed_routing(gpt_model* m, int32_t* h_n_unique, int32_t* h_sorted_tok, int32_t* h_sorted_pos) {
+  if (!m || !h_n_unique || !h_sorted_tok || !h_sorted_pos) return GPT_ERR_INVALID_ARG;
+  cudaMemcpyAsync(h_n_unique, m->nuniq, 4, cudaMemcpyDeviceToHost, m->ctx.stream);
+  cudaMemcpyAsync(h_sorted_tok, m->stok, (size_t)m->M * 4, cudaMemcpyDeviceToHost, m->ctx.stream);
+  cudaMemcpyAsync(h_sorted_pos, m->spos, (size_t)m->M * 4, cudaMemcpyDeviceToHost, m->ctx.stream);
+  return sync_and_flags(m, "get_embed_routing", nullptr);
+}
+
+gpt_status gpt_dropout_mask(gpt_model* m, int64_t counter, int32_t layer, int32_t site, int64_t n, uint8_t* h_out) {
+  if (!m || !h_out || n <= 0 || counter < 0) return GPT_ERR_INVALID_ARG;
+  size_t cap = (size_t)m->M * 4 * m->d * m->asz;  // the MLP-gradient buffer serves as scratch
+  if ((size_t)n > cap) return fail(m, GPT_ERR_INVALID_ARG, "dropout_mask: n larger than the scratch buffer");
+  DropKey k = make_drop_key(m->cfg.dropout_seed, (uint64_t)counter, layer, site, m->cfg.dropout);
+  dropout_mask(m->ctx, k, n, m->dh);
+  cudaMemcpyAsync(h_out, m->dh, (size_t)n, cudaMemcpyDeviceToHost, m->ctx.stream);
+  return sync_and_flags(m, "dropout_mask", nullptr);
+}
+
+size_t gpt_state_floats(gpt_model* m) {
+  if (!m) return 0;
+  size_t n = 0;
+  for (auto& t : m->tensors) n += (size_t)t.rows * t.cols;
+  return n;
+}
+
+gpt_status gpt_get_state(gpt_model* m, float* hp, float* hm, float* hv) {
+  if (!m || !hp || !hm || !hv) return GPT_ERR_INVALID_ARG;
+  size_t o = 0;
+  for (auto& t : m->tensors) {
+    size_t n = (size_t)t.rows * t.cols;
+    cudaMemcpyAsync(hp + o, m->w + t.off, n * 4, cudaMemcpyDeviceToHost, m->ctx.stream);
+    cudaMemcpyAsync(hm + o, m->am + t.off, n * 4, cudaMemcpyDeviceToHost, m->ctx.stream);
+    cudaMemcpyAsync(hv + o, m->av + t.off, n * 4, cudaMemcpyDeviceToHost, m->ctx.stream);
+    o += n;
+  }
+  return sync_and_flags(m, "get_state", nullptr);
+}
+
+gpt_status gpt_set_state(gpt_model* m, const float* hp, const float* hm, const float* hv) {
+  if (!m || !hp || !hm || !hv) return GPT_ERR_INVALID_ARG;
+  size_t o = 0;
+  for (auto& t : m->tensors) {
+    size_t n = (size_t)t.rows * t.cols;
+    cudaMemcpyAsync(m->w + t.off, hp + o, n * 4, cudaMemcpyHostToDevice, m->ctx.stream);
+    cudaMemcpyAsync(m->am + t.off, hm + o, n * 4, cudaMemcpyHostToDevice, m->ctx.stream);
+    cudaMemcpyAsync(m->av + t.off, hv + o, n * 4, cudaMemcpyHostToDevice, m->ctx.stream);
+    o += n;
+  }
+  if (m->bf16m) to_bf16(m->ctx, m->w, m->wb, m->n_total);
+  return sync_and_flags(m, "set_state", nullptr);
+}
+
+gpt_status gpt_read_flags(gpt_model* m, uint32_t* h_flags) {
+  if (!m || !h_flags) return GPT_ERR_INVALID_ARG;
+  float sc[4];
+  cudaMemcpyAsync(sc, m->scal, 16, cudaMemcpyDeviceToHost, m->ctx.stream);
+  if (cudaStreamSynchronize(m->ctx.stream) != cudaSuccess) return check_cuda(m, "read_flags");
+  memcpy(h_flags, &sc[3], 4);
+  return GPT_OK;
+}
+
+gpt_status gpt_clear_flags(gpt_model* m) {
+  if (!m) return GPT_ERR_INVALID_ARG;
+  cudaMemsetAsync(m->scal + 3, 0, 4, m->ctx.stream);
+  m->reported = 0;
+  return check_cuda(m, "clear_flags");
+}
+
+gpt_status gpt_enable_timing(gpt_model* m, int32_t on) {
+  if (!m) return GPT_ERR_INVALID_ARG;
+  if (on) {
+    if (!m->timing) m->timing = new Timing();
+    m->timing->reset();
+    m->ctx.timing = m->timing;
+  } else {
+    m->ctx.timing = nullptr;
+  }
+  return GPT_OK;
+}
+
+gpt_status gpt_kernel_times(gpt_model* m, int32_t cap, const char** names, float* total_ms, int32_t* launches,
+                            int32_t* n_out) {
+  if (!m || !n_out) return GPT_ERR_INVALID_ARG;
+  if (!m->timing) {
+    *n_out = 0;
+    return GPT_OK;
+  }
+  cudaStreamSynchronize(m->ctx.stream);
+  int k = 0;
+  for (auto& kv : m->timing->recs) {
+    if (k >= cap) break;
+    float tot = 0.f;
+    for (size_t j = 0; j + 1 < kv.second.ev.size(); j += 2) {
+      float ms = 0.f;
+      cudaEventElapsedTime(&ms, kv.second.ev[j], kv.second.ev[j + 1]);
+      tot += ms;
+    }
+    if (names) names[k] = kv.first.c_str();
+    if (total_ms) total_ms[k] = tot;
+    if (launches) launches[k] = kv.second.launches;
+    k++;
+  }
+  *n_out = k;
+  return check_cuda(m, "kernel_times");
+}
+
+uint64_t gpt_launch_count(gpt_model* m) { return m ? m->ctx.launches : 0; }
+
+}  // extern "C"

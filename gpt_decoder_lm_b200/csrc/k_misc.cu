@@ -1,0 +1,691 @@
+// Memory-bound kernels of the training step: batch gather, embedding,
+// LayerNorm/RMSNorm, cross-entropy, column sums, embedding backward,
+// gradient norm and the fused clip + AdamW update.
+#include "kernels.cuh"
+
+#include <math.h>
+
+namespace gpt {
+
+// ============================================================================
+// get_batch: random windows of the token stream (run log section 1.3; the
+// target is the window shifted by one).  One thread per (b, t).
+// ============================================================================
+__global__ void k_gather(const void* __restrict__ stream, int tok_u16, uint64_t len, uint64_t seed, int step,
+                         int micro, int B, int T, int V, int32_t* __restrict__ idx, int32_t* __restrict__ tgt,
+                         uint32_t* flags) {
+  long i = (long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= (long)B * T) return;
+  int b = (int)(i / T), t = (int)(i % T);
+  uint64_t key = ((uint64_t)(uint32_t)step << 40) ^ ((uint64_t)(uint32_t)micro << 20) ^ (uint64_t)b;
+  uint64_t ix = splitmix64(seed ^ splitmix64(key)) % (len - (uint64_t)T);
+  int x, y;
+  if (tok_u16) {
+    const uint16_t* s = (const uint16_t*)stream;
+    x = s[ix + t];
+    y = s[ix + t + 1];
+  } else {
+    const int32_t* s = (const int32_t*)stream;
+    x = s[ix + t];
+    y = s[ix + t + 1];
+  }
+  if (x < 0 || x >= V || y < 0 || y >= V) {
+    atomicOr(flags, FLAG_TOKEN);
+    x = (x < 0 || x >= V) ? 0 : x;
+    y = (y < 0 || y >= V) ? 0 : y;
+  }
+  idx[i] = x;
+  tgt[i] = y;
+}
+
+void gather_batch(Ctx& c, const void* stream, int tok_u16, uint64_t len, uint64_t seed, int step, int micro, int B,
+                  int T, int V, int32_t* idx, int32_t* tgt) {
+  long n = (long)B * T;
+  LaunchScope s(c, "gather_batch");
+  k_gather<<<(unsigned)((n + 255) / 256), 256, 0, c.stream>>>(stream, tok_u16, len, seed, step, micro, B, T, V, idx,
+                                                              tgt, c.flags);
+}
+
+__global__ void k_check_tokens(const int32_t* __restrict__ idx, const int32_t* __restrict__ tgt, long n, int V,
+                               int32_t* __restrict__ io, int32_t* __restrict__ to, uint32_t* flags) {
+  long i = (long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n) return;
+  int x = idx[i], y = tgt[i];
+  if (x < 0 || x >= V || y < 0 || y >= V) {
+    atomicOr(flags, FLAG_TOKEN);
+    x = (x < 0 || x >= V) ? 0 : x;
+    y = (y < 0 || y >= V) ? 0 : y;
+  }
+  io[i] = x;
+  to[i] = y;
+}
+
+void check_tokens(Ctx& c, const int32_t* idx, const int32_t* tgt, long n, int V, int32_t* io, int32_t* to) {
+  LaunchScope s(c, "check_tokens");
+  k_check_tokens<<<(unsigned)((n + 255) / 256), 256, 0, c.stream>>>(idx, tgt, n, V, io, to, c.flags);
+}
+
+// ============================================================================
+// embedding: res = drop0(wte[idx] + wpe[t]) in fp32 (microGPT "模型核心":
+// token embedding plus learned position embedding).
+// ============================================================================
+__global__ void k_embed_fwd(const int32_t* __restrict__ idx, const float* __restrict__ wte,
+                            const float* __restrict__ wpe, float* __restrict__ res, int T, int d, long n4,
+                            DropKey drop) {
+  long i = (long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n4) return;
+  int d4 = d >> 2;
+  long m = i / d4;
+  int c4 = (int)(i % d4);
+  int t = (int)(m % T);
+  int tok = idx[m];
+  float4 a = reinterpret_cast<const float4*>(wte + (long)tok * d)[c4];
+  float4 p = reinterpret_cast<const float4*>(wpe + (long)t * d)[c4];
+  float4 r = make_float4(a.x + p.x, a.y + p.y, a.z + p.z, a.w + p.w);
+  if (drop.active) {
+    uint64_t e = (uint64_t)m * d + c4 * 4;
+    r.x *= drop_mul(drop, e);
+    r.y *= drop_mul(drop, e + 1);
+    r.z *= drop_mul(drop, e + 2);
+    r.w *= drop_mul(drop, e + 3);
+  }
+  reinterpret_cast<float4*>(res)[i] = r;
+}
+
+template <typename T>
+void embed_fwd(Ctx& c, const int32_t* idx, const float* wte, const float* wpe, float* res, int B, int Tn, int d,
+               DropKey drop) {
+  long n4 = (long)B * Tn * d / 4;
+  LaunchScope s(c, "embed_fwd");
+  k_embed_fwd<<<(unsigned)((n4 + 255) / 256), 256, 0, c.stream>>>(idx, wte, wpe, res, Tn, d, n4, drop);
+}
+template void embed_fwd<float>(Ctx&, const int32_t*, const float*, const float*, float*, int, int, int, DropKey);
+template void embed_fwd<bf16>(Ctx&, const int32_t*, const float*, const float*, float*, int, int, int, DropKey);
+
+// ============================================================================
+// norm forward: one warp per row, the row held in registers (VPL float4 per
+// lane).  LayerNorm: biased variance, y = (x - mean) * rstd * w + b.
+// RMSNorm (micro variant): y = x * rstd with rstd = 1/sqrt(mean(x^2) + eps).
+// ============================================================================
+template <typename T> __device__ __forceinline__ void store4(T* p, float4 v);
+template <> __device__ __forceinline__ void store4<float>(float* p, float4 v) { *reinterpret_cast<float4*>(p) = v; }
+template <> __device__ __forceinline__ void store4<bf16>(bf16* p, float4 v) {
+  __nv_bfloat162 a = __floats2bfloat162_rn(v.x, v.y);
+  __nv_bfloat162 b = __floats2bfloat162_rn(v.z, v.w);
+  uint2 u;
+  u.x = *reinterpret_cast<uint32_t*>(&a);
+  u.y = *reinterpret_cast<uint32_t*>(&b);
+  *reinterpret_cast<uint2*>(p) = u;
+}
+
+template <typename T, int VPL>
+__global__ void k_norm_fwd(const float* __restrict__ x, const float* __restrict__ w, const float* __restrict__ b,
+                           T* __restrict__ y, float* __restrict__ mean_out, float* __restrict__ rstd_out, long rows,
+                           int d, int rms, float eps) {
+  long row = (long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  int lane = threadIdx.x & 31;
+  if (row >= rows) return;
+  int d4 = d >> 2;
+  const float4* xr = reinterpret_cast<const float4*>(x + row * d);
+  float4 v[VPL];
+  float s = 0.f;
+#pragma unroll
+  for (int k = 0; k < VPL; k++) {
+    int c = lane + 32 * k;
+    v[k] = c < d4 ? xr[c] : make_float4(0.f, 0.f, 0.f, 0.f);
+    s += rms ? (v[k].x * v[k].x + v[k].y * v[k].y + v[k].z * v[k].z + v[k].w * v[k].w)
+             : (v[k].x + v[k].y + v[k].z + v[k].w);
+  }
+  s = warp_sum(s);
+  float mean = 0.f, rstd;
+  if (rms) {
+    rstd = 1.0f / sqrtf(s / d + eps);
+  } else {
+    mean = s / d;
+    float q = 0.f;
+#pragma unroll
+    for (int k = 0; k < VPL; k++) {
+      int c = lane + 32 * k;
+      if (c < d4) {
+        float a = v[k].x - mean, bb = v[k].y - mean, cc = v[k].z - mean, dd = v[k].w - mean;
+        q += a * a + bb * bb + cc * cc + dd * dd;
+      }
+    }
+    q = warp_sum(q);
+    rstd = 1.0f / sqrtf(q / d + eps);
+  }
+  T* yr = y + row * d;
+#pragma unroll
+  for (int k = 0; k < VPL; k++) {
+    int c = lane + 32 * k;
+    if (c < d4) {
+      float4 o;
+      o.x = (v[k].x - mean) * rstd;
+      o.y = (v[k].y - mean) * rstd;
+      o.z = (v[k].z - mean) * rstd;
+      o.w = (v[k].w - mean) * rstd;
+      if (!rms) {
+        float4 ww = reinterpret_cast<const float4*>(w)[c];
+        float4 bb = reinterpret_cast<const float4*>(b)[c];
+        o.x = o.x * ww.x + bb.x;
+        o.y = o.y * ww.y + bb.y;
+        o.z = o.z * ww.z + bb.z;
+        o.w = o.w * ww.w + bb.w;
+      }
+      store4<T>(yr + 4 * c, o);
+    }
+  }
+  if (lane == 0) {
+    mean_out[row] = mean;
+    rstd_out[row] = rstd;
+  }
+}
+
+template <typename T>
+void norm_fwd(Ctx& c, const float* x, const float* w, const float* b, T* y, float* mean, float* rstd, long rows,
+              int d, bool rms, float eps) {
+  int d4 = d / 4;
+  int vpl = (d4 + 31) / 32;
+  unsigned grid = (unsigned)((rows + 7) / 8);
+  LaunchScope s(c, "norm_fwd");
+#define NF(V) k_norm_fwd<T, V><<<grid, 256, 0, c.stream>>>(x, w, b, y, mean, rstd, rows, d, rms, eps)
+  if (vpl <= 1) NF(1);
+  else if (vpl <= 2) NF(2);
+  else if (vpl <= 4) NF(4);
+  else if (vpl <= 8) NF(8);
+  else NF(16);
+#undef NF
+}
+template void norm_fwd<float>(Ctx&, const float*, const float*, const float*, float*, float*, float*, long, int,
+                              bool, float);
+template void norm_fwd<bf16>(Ctx&, const float*, const float*, const float*, bf16*, float*, float*, long, int, bool,
+                             float);
+
+// ============================================================================
+// norm backward.  A block of ceil(d/4) threads (rounded to warps) walks a
+// contiguous range of rows; thread j owns columns 4j..4j+3, so the column
+// partial sums stay in registers and the result is deterministic.
+//   LayerNorm: g = dy * w; dx = rstd * (g - mean(g) - xhat * mean(g * xhat))
+//   RMSNorm:   g = dy;     dx = rstd * (g - xhat * mean(g * xhat))
+// ============================================================================
+template <typename T>
+__global__ void k_norm_bwd(NormBwd p) {
+  extern __shared__ float red[];  // [2 buffers][warps][2]
+  int tid = threadIdx.x;
+  int d4 = p.d >> 2;
+  int nw = blockDim.x >> 5;
+  bool own = tid < d4;
+  long per = (p.rows + gridDim.x - 1) / gridDim.x;
+  long r0 = blockIdx.x * per, r1 = min(p.rows, r0 + per);
+  float4 gw = make_float4(1.f, 1.f, 1.f, 1.f);
+  if (own && !p.rms) gw = reinterpret_cast<const float4*>(p.w)[tid];
+  float pg[4] = {0, 0, 0, 0}, pb[4] = {0, 0, 0, 0}, pn[4] = {0, 0, 0, 0};
+  int buf = 0;
+  for (long r = r0; r < r1; r++) {
+    float4 dy = make_float4(0, 0, 0, 0), xv = make_float4(0, 0, 0, 0);
+    float mean = p.rms ? 0.f : p.mean[r];
+    float rstd = p.rstd[r];
+    if (own) {
+      dy = reinterpret_cast<const float4*>(p.dy + r * p.d)[tid];
+      xv = reinterpret_cast<const float4*>(p.x + r * p.d)[tid];
+    }
+    float xh[4] = {(xv.x - mean) * rstd, (xv.y - mean) * rstd, (xv.z - mean) * rstd, (xv.w - mean) * rstd};
+    float dyv[4] = {dy.x, dy.y, dy.z, dy.w};
+    float wv[4] = {gw.x, gw.y, gw.z, gw.w};
+    float g[4], s1 = 0.f, s2 = 0.f;
+#pragma unroll
+    for (int k = 0; k < 4; k++) {
+      g[k] = dyv[k] * wv[k];
+      s1 += g[k];
+      s2 += g[k] * xh[k];
+    }
+    s1 = warp_sum(s1);
+    s2 = warp_sum(s2);
+    if ((tid & 31) == 0) {
+      red[(buf * nw + (tid >> 5)) * 2 + 0] = s1;
+      red[(buf * nw + (tid >> 5)) * 2 + 1] = s2;
+    }
+    __syncthreads();
+    float t1 = 0.f, t2 = 0.f;
+    for (int w = 0; w < nw; w++) {
+      t1 += red[(buf * nw + w) * 2 + 0];
+      t2 += red[(buf * nw + w) * 2 + 1];
+    }
+    buf ^= 1;
+    float mg = p.rms ? 0.f : t1 / p.d;
+    float mgx = t2 / p.d;
+    if (own) {
+      float4* dr = reinterpret_cast<float4*>(p.dres + r * p.d) + tid;
+      float4 old = p.accumulate ? *dr : make_float4(0, 0, 0, 0);
+      float ov[4] = {old.x, old.y, old.z, old.w};
+      float nv[4];
+#pragma unroll
+      for (int k = 0; k < 4; k++) {
+        nv[k] = ov[k] + rstd * (g[k] - mg - xh[k] * mgx);
+        pg[k] += dyv[k] * xh[k];
+        pb[k] += dyv[k];
+      }
+      *dr = make_float4(nv[0], nv[1], nv[2], nv[3]);
+      if (p.want_dyb) {
+        float q[4];
+#pragma unroll
+        for (int k = 0; k < 4; k++) {
+          q[k] = nv[k] * drop_mul(p.drop, (uint64_t)r * p.d + 4 * tid + k);
+          pn[k] += q[k];
+        }
+        store4<T>(reinterpret_cast<T*>(p.dyb) + r * p.d + 4 * tid, make_float4(q[0], q[1], q[2], q[3]));
+      }
+    }
+  }
+  if (own) {
+    float* out = p.part + (long)blockIdx.x * 3 * p.d;
+    reinterpret_cast<float4*>(out)[tid] = make_float4(pg[0], pg[1], pg[2], pg[3]);
+    reinterpret_cast<float4*>(out + p.d)[tid] = make_float4(pb[0], pb[1], pb[2], pb[3]);
+    reinterpret_cast<float4*>(out + 2 * p.d)[tid] = make_float4(pn[0], pn[1], pn[2], pn[3]);
+  }
+}
+
+int norm_bwd_blocks(Ctx& c, long rows) {
+  long b = (long)c.num_sms * 4;
+  return (int)(rows < b ? rows : b);
+}
+
+template <typename T>
+void norm_bwd(Ctx& c, const NormBwd& p) {
+  int d4 = p.d / 4;
+  int threads = ((d4 + 31) / 32) * 32;
+  int nw = threads / 32;
+  LaunchScope s(c, "norm_bwd");
+  k_norm_bwd<T><<<p.blocks, threads, 2 * nw * 2 * sizeof(float), c.stream>>>(p);
+}
+template void norm_bwd<float>(Ctx&, const NormBwd&);
+template void norm_bwd<bf16>(Ctx&, const NormBwd&);
+
+__global__ void k_partial_reduce(const float* __restrict__ part, int blocks, int slots, int slot, int d,
+                                 float* __restrict__ grad) {
+  int j = blockIdx.x * blockDim.x + threadIdx.x;
+  if (j >= d) return;
+  float s = 0.f;
+  for (int b = 0; b < blocks; b++) s += part[((long)b * slots + slot) * d + j];
+  grad[j] += s;
+}
+
+void partial_reduce(Ctx& c, const float* part, int blocks, int slots, int slot, int d, float* grad) {
+  LaunchScope s(c, "partial_reduce");
+  k_partial_reduce<<<(d + 127) / 128, 128, 0, c.stream>>>(part, blocks, slots, slot, d, grad);
+}
+
+// ============================================================================
+// column sums (bias gradients): chunk partials then a fixed-order reduce
+// ============================================================================
+template <typename T>
+__global__ void k_colsum(const T* __restrict__ x, long rows, int N, int chunks, float* __restrict__ part) {
+  int j = blockIdx.x * blockDim.x + threadIdx.x;
+  if (j >= N) return;
+  long per = (rows + chunks - 1) / chunks;
+  long r0 = blockIdx.y * per, r1 = min(rows, r0 + per);
+  float s = 0.f;
+  for (long r = r0; r < r1; r++) s += to_f<T>(x[r * N + j]);
+  part[(long)blockIdx.y * N + j] = s;
+}
+
+template <typename T>
+void colsum_acc(Ctx& c, const T* x, long rows, int N, float* scratch, float* grad) {
+  int chunks = (int)min(64L, rows);
+  {
+    LaunchScope s(c, "colsum");
+    dim3 grid((N + 127) / 128, chunks);
+    k_colsum<T><<<grid, 128, 0, c.stream>>>(x, rows, N, chunks, scratch);
+  }
+  partial_reduce(c, scratch, chunks, 1, 0, N, grad);
+}
+template void colsum_acc<float>(Ctx&, const float*, long, int, float*, float*);
+template void colsum_acc<bf16>(Ctx&, const bf16*, long, int, float*, float*);
+
+// ============================================================================
+// cross-entropy (microGPT "核心训练循环": loss = -log softmax(z)[target],
+// mean over positions).  One block per row: pass 1 keeps an online
+// (max, sum exp) per thread and merges them; pass 2 writes
+// (softmax - onehot) * scale over the logits in place (pad columns 0).
+// ============================================================================
+template <typename T>
+__global__ void k_ce(T* __restrict__ logits, const int32_t* __restrict__ tgt, int V, int Vp,
+                     float* __restrict__ lse_out, float* __restrict__ row_loss, int want_grad, float scale) {
+  __shared__ float sm[32], ss[32];
+  long row = blockIdx.x;
+  T* z = logits + row * Vp;
+  float m = -INFINITY, s = 0.f;
+  for (int j = threadIdx.x; j < V; j += blockDim.x) {
+    float v = to_f<T>(z[j]);
+    if (v > m) {
+      s = s * expf(m - v) + 1.f;
+      m = v;
+    } else {
+      s += expf(v - m);
+    }
+  }
+  // merge (m, s) pairs: warp then block
+  for (int o = 16; o > 0; o >>= 1) {
+    float m2 = __shfl_xor_sync(0xffffffffu, m, o);
+    float s2 = __shfl_xor_sync(0xffffffffu, s, o);
+    float mm = fmaxf(m, m2);
+    s = (m == -INFINITY ? 0.f : s * expf(m - mm)) + (m2 == -INFINITY ? 0.f : s2 * expf(m2 - mm));
+    m = mm;
+  }
+  int w = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  if ((threadIdx.x & 31) == 0) {
+    sm[w] = m;
+    ss[w] = s;
+  }
+  __syncthreads();
+  float M = -INFINITY;
+  for (int k = 0; k < nw; k++) M = fmaxf(M, sm[k]);
+  float S = 0.f;
+  for (int k = 0; k < nw; k++) S += (sm[k] == -INFINITY ? 0.f : ss[k] * expf(sm[k] - M));
+  float lse = M + logf(S);
+  int t = tgt[row];
+  if (threadIdx.x == 0) {
+    lse_out[row] = lse;
+    row_loss[row] = lse - to_f<T>(z[t]);
+  }
+  __syncthreads();  // the target logit is read before pass 2 overwrites it
+  if (!want_grad) return;
+  for (int j = threadIdx.x; j < Vp; j += blockDim.x) {
+    float g = 0.f;
+    if (j < V) g = (expf(to_f<T>(z[j]) - lse) - (j == t ? 1.f : 0.f)) * scale;
+    z[j] = from_f<T>(g);
+  }
+}
+
+template <typename T>
+void ce_fwd_bwd(Ctx& c, T* logits, const int32_t* tgt, long M, int V, int Vp, float* lse, float* row_loss,
+                bool want_grad, float scale) {
+  LaunchScope s(c, want_grad ? "ce_fwd_bwd" : "ce_fwd");
+  k_ce<T><<<(unsigned)M, 512, 0, c.stream>>>(logits, tgt, V, Vp, lse, row_loss, want_grad ? 1 : 0, scale);
+}
+template void ce_fwd_bwd<float>(Ctx&, float*, const int32_t*, long, int, int, float*, float*, bool, float);
+template void ce_fwd_bwd<bf16>(Ctx&, bf16*, const int32_t*, long, int, int, float*, float*, bool, float);
+
+// loss_acc[0] (+)= scale * sum(row_loss); fixed-order double reduction.
+__global__ void k_loss_reduce(const float* __restrict__ rl, long M, float scale, float* acc, int accumulate,
+                              uint32_t* flags) {
+  __shared__ double sh[32];
+  double s = 0.0;
+  for (long i = threadIdx.x; i < M; i += blockDim.x) s += (double)rl[i];
+  s = warp_sum_d(s);
+  if ((threadIdx.x & 31) == 0) sh[threadIdx.x >> 5] = s;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double t = 0.0;
+    for (int k = 0; k < (int)(blockDim.x >> 5); k++) t += sh[k];
+    float v = (float)(t * (double)scale);
+    if (!isfinite(v)) atomicOr(flags, FLAG_LOSS);
+    acc[0] = accumulate ? acc[0] + v : v;
+  }
+}
+
+void loss_reduce(Ctx& c, const float* row_loss, long M, float scale, float* loss_acc, int accumulate) {
+  LaunchScope s(c, "loss_reduce");
+  k_loss_reduce<<<1, 1024, 0, c.stream>>>(row_loss, M, scale, loss_acc, accumulate, c.flags);
+}
+
+// ============================================================================
+// embedding backward.  Routing: key = token << 16 | position is unique, so a
+// plain bitonic sort of the keys equals a stable sort of positions by token.
+// ============================================================================
+__global__ void k_embed_sort(const int32_t* __restrict__ idx, int M, int P2, int32_t* __restrict__ stok,
+                             int32_t* __restrict__ spos, int32_t* __restrict__ n_unique) {
+  extern __shared__ uint32_t key[];
+  __shared__ int cnt[32];
+  for (int i = threadIdx.x; i < P2; i += blockDim.x)
+    key[i] = i < M ? (((uint32_t)idx[i] << 16) | (uint32_t)i) : 0xFFFFFFFFu;
+  __syncthreads();
+  for (int k = 2; k <= P2; k <<= 1) {
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      for (int i = threadIdx.x; i < P2; i += blockDim.x) {
+        int l = i ^ j;
+        if (l > i) {
+          uint32_t a = key[i], b = key[l];
+          bool up = (i & k) == 0;
+          if ((a > b) == up) {
+            key[i] = b;
+            key[l] = a;
+          }
+        }
+      }
+      __syncthreads();
+    }
+  }
+  int u = 0;
+  for (int i = threadIdx.x; i < M; i += blockDim.x) {
+    uint32_t kk = key[i];
+    stok[i] = (int32_t)(kk >> 16);
+    spos[i] = (int32_t)(kk & 0xFFFFu);
+    if (i == 0 || (key[i - 1] >> 16) != (kk >> 16)) u++;
+  }
+  for (int o = 16; o > 0; o >>= 1) u += __shfl_xor_sync(0xffffffffu, u, o);
+  if ((threadIdx.x & 31) == 0) cnt[threadIdx.x >> 5] = u;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int t = 0;
+    for (int k = 0; k < (int)(blockDim.x >> 5); k++) t += cnt[k];
+    *n_unique = t;
+  }
+}
+
+void embed_sort(Ctx& c, const int32_t* idx, long M, int32_t* sorted_tok, int32_t* sorted_pos, int32_t* n_unique) {
+  int P2 = 1;
+  while (P2 < M) P2 <<= 1;
+  size_t smem = (size_t)P2 * 4;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaFuncSetAttribute(k_embed_sort, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+    attr_set = true;
+  }
+  LaunchScope s(c, "embed_sort");
+  k_embed_sort<<<1, 1024, smem, c.stream>>>(idx, (int)M, P2, sorted_tok, sorted_pos, n_unique);
+}
+
+// dwte[v] += sum over the sorted positions of token v (in position order) of
+// drop0(dres[pos]); one block per sorted slot, active only at segment starts.
+__global__ void k_embed_bwd_wte(const float* __restrict__ dres, const int32_t* __restrict__ stok,
+                                const int32_t* __restrict__ spos, int M, int d, DropKey drop,
+                                float* __restrict__ dwte) {
+  int i = blockIdx.x;
+  int tok = stok[i];
+  if (i > 0 && stok[i - 1] == tok) return;
+  for (int c = threadIdx.x; c < d; c += blockDim.x) {
+    float acc = 0.f;
+    for (int j = i; j < M && stok[j] == tok; j++) {
+      long p = spos[j];
+      acc += dres[p * d + c] * drop_mul(drop, (uint64_t)p * d + c);
+    }
+    dwte[(long)tok * d + c] += acc;
+  }
+}
+
+// dwpe[t] += sum_b drop0(dres[b, t]) (b ascending)
+__global__ void k_embed_bwd_wpe(const float* __restrict__ dres, int Bn, int Tn, int d, DropKey drop,
+                                float* __restrict__ dwpe) {
+  long i = (long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= (long)Tn * d) return;
+  int t = (int)(i / d), c = (int)(i % d);
+  float acc = 0.f;
+  for (int b = 0; b < Bn; b++) {
+    long m = (long)b * Tn + t;
+    acc += dres[m * d + c] * drop_mul(drop, (uint64_t)m * d + c);
+  }
+  dwpe[i] += acc;
+}
+
+void embed_bwd(Ctx& c, const float* dres, const int32_t* sorted_tok, const int32_t* sorted_pos, long M, int Tn,
+               int Bn, int d, DropKey drop, float* dwte, float* dwpe) {
+  {
+    LaunchScope s(c, "embed_bwd_wte");
+    int th = d >= 256 ? 256 : ((d + 31) / 32) * 32;
+    k_embed_bwd_wte<<<(unsigned)M, th, 0, c.stream>>>(dres, sorted_tok, sorted_pos, (int)M, d, drop, dwte);
+  }
+  {
+    LaunchScope s(c, "embed_bwd_wpe");
+    long n = (long)Tn * d;
+    k_embed_bwd_wpe<<<(unsigned)((n + 255) / 256), 256, 0, c.stream>>>(dres, Bn, Tn, d, drop, dwpe);
+  }
+}
+
+// ============================================================================
+// global gradient norm: per-block partial sums of squares (double)
+// ============================================================================
+int sumsq_blocks(Ctx& c) { return c.num_sms * 4 < 592 ? c.num_sms * 4 : 592; }  // partial buffer holds 592
+
+__global__ void k_sumsq(const float* __restrict__ g, long n4, double* __restrict__ part) {
+  __shared__ double sh[32];
+  double s = 0.0;
+  for (long i = (long)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += (long)gridDim.x * blockDim.x) {
+    float4 v = reinterpret_cast<const float4*>(g)[i];
+    s += (double)(v.x * v.x + v.y * v.y) + (double)(v.z * v.z + v.w * v.w);
+  }
+  s = warp_sum_d(s);
+  if ((threadIdx.x & 31) == 0) sh[threadIdx.x >> 5] = s;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double t = 0.0;
+    for (int k = 0; k < (int)(blockDim.x >> 5); k++) t += sh[k];
+    part[blockIdx.x] = t;
+  }
+}
+
+void sumsq_partials(Ctx& c, const float* g, long n, double* partials, int blocks) {
+  LaunchScope s(c, "grad_norm");
+  k_sumsq<<<blocks, 512, 0, c.stream>>>(g, n / 4, partials);
+}
+
+// ============================================================================
+// clip + AdamW (one pass over the fp32 arenas; decayed tensors first).
+//   c = min(1, clip / (norm + 1e-6)); g <- c g
+//   w <- w (1 - lr wd)                      (decayed tensors only)
+//   m <- b1 m + (1 - b1) g;  v <- b2 v + (1 - b2) g^2
+//   w <- w - lr (m / bc1) / (sqrt(v / bc2) + eps);  wb <- bf16(w);  g <- 0
+// A non-finite norm skips the update (gradients are still zeroed).
+// ============================================================================
+__global__ void k_adamw(AdamArgs a, uint32_t* flags) {
+  __shared__ float s_coef;
+  __shared__ int s_ok;
+  if (threadIdx.x < 32) {
+    double t = 0.0;
+    for (int k = threadIdx.x; k < a.norm_blocks; k += 32) t += a.norm_partials[k];
+    t = warp_sum_d(t);
+    if (threadIdx.x == 0) {
+      double norm = sqrt(t);
+      int ok = isfinite(norm) ? 1 : 0;
+      float coef = 1.f;
+      if (a.clip > 0.f && ok) coef = (float)fmin(1.0, (double)a.clip / (norm + 1e-6));
+      s_coef = coef;
+      s_ok = ok;
+      if (blockIdx.x == 0) {
+        a.norm_out[0] = (float)norm;
+        if (!ok) atomicOr(flags, FLAG_NORM);
+      }
+    }
+  }
+  __syncthreads();
+  float coef = s_coef;
+  int ok = s_ok;
+  float om1 = 1.f - a.beta1, om2 = 1.f - a.beta2;
+  float decay = 1.f - a.lr * a.wd;
+  long n4 = a.n / 4;
+  for (long i = (long)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += (long)gridDim.x * blockDim.x) {
+    float4 g4 = reinterpret_cast<float4*>(a.g)[i];
+    reinterpret_cast<float4*>(a.g)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (!ok) continue;
+    float4 w4 = reinterpret_cast<float4*>(a.w)[i];
+    float4 m4 = reinterpret_cast<float4*>(a.m)[i];
+    float4 v4 = reinterpret_cast<float4*>(a.v)[i];
+    float* w = &w4.x;
+    float* m = &m4.x;
+    float* v = &v4.x;
+    const float* g = &g4.x;
+    bool dec = (i * 4) < a.n_decay;
+#pragma unroll
+    for (int k = 0; k < 4; k++) {
+      float gg = g[k] * coef;
+      float ww = dec ? w[k] * decay : w[k];
+      m[k] = a.beta1 * m[k] + om1 * gg;
+      v[k] = a.beta2 * v[k] + om2 * gg * gg;
+      ww -= a.lr * (m[k] / a.bc1) / (sqrtf(v[k] / a.bc2) + a.eps);
+      w[k] = ww;
+    }
+    reinterpret_cast<float4*>(a.w)[i] = w4;
+    reinterpret_cast<float4*>(a.m)[i] = m4;
+    reinterpret_cast<float4*>(a.v)[i] = v4;
+    if (a.wb) store4<bf16>(a.wb + 4 * i, w4);
+  }
+}
+
+void adamw(Ctx& c, const AdamArgs& a) {
+  LaunchScope s(c, "adamw");
+  k_adamw<<<c.num_sms * 8, 256, 0, c.stream>>>(a, c.flags);
+}
+
+__global__ void k_to_bf16(const float* __restrict__ s, bf16* __restrict__ d, long n) {
+  long i = (long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) d[i] = __float2bfloat16_rn(s[i]);
+}
+
+void to_bf16(Ctx& c, const float* src, bf16* dst, long n) {
+  LaunchScope s(c, "to_bf16");
+  k_to_bf16<<<(unsigned)((n + 255) / 256), 256, 0, c.stream>>>(src, dst, n);
+}
+
+// row argmax, ties to the lowest index
+__global__ void k_argmax(const void* __restrict__ x, int is_bf16, int cols, int ld, int32_t* __restrict__ out) {
+  __shared__ float bv[32];
+  __shared__ int bi[32];
+  long row = blockIdx.x;
+  float best = -INFINITY;
+  int bidx = 0x7fffffff;
+  for (int j = threadIdx.x; j < cols; j += blockDim.x) {
+    float v = is_bf16 ? __bfloat162float(((const bf16*)x)[row * ld + j]) : ((const float*)x)[row * ld + j];
+    if (v > best || (v == best && j < bidx)) {
+      best = v;
+      bidx = j;
+    }
+  }
+  for (int o = 16; o > 0; o >>= 1) {
+    float v2 = __shfl_xor_sync(0xffffffffu, best, o);
+    int i2 = __shfl_xor_sync(0xffffffffu, bidx, o);
+    if (v2 > best || (v2 == best && i2 < bidx)) {
+      best = v2;
+      bidx = i2;
+    }
+  }
+  if ((threadIdx.x & 31) == 0) {
+    bv[threadIdx.x >> 5] = best;
+    bi[threadIdx.x >> 5] = bidx;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    for (int k = 1; k < (int)(blockDim.x >> 5); k++)
+      if (bv[k] > best || (bv[k] == best && bi[k] < bidx)) {
+        best = bv[k];
+        bidx = bi[k];
+      }
+    out[row] = bidx == 0x7fffffff ? 0 : bidx;
+  }
+}
+
+void argmax_rows(Ctx& c, const void* x, int is_bf16, long rows, int cols, int ld, int32_t* out) {
+  LaunchScope s(c, "argmax");
+  k_argmax<<<(unsigned)rows, 256, 0, c.stream>>>(x, is_bf16, cols, ld, out);
+}
+
+__global__ void k_dropmask(DropKey k, long n, uint8_t* out) {
+  long i = (long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) out[i] = drop_keep(k, (uint64_t)i) ? 1 : 0;
+}
+
+void dropout_mask(Ctx& c, DropKey k, long n, uint8_t* out) {
+  LaunchScope s(c, "dropout_mask");
+  k_dropmask<<<(unsigned)((n + 255) / 256), 256, 0, c.stream>>>(k, n, out);
+}
+
+}  // namespace gpt

@@ -1,0 +1,163 @@
+// Internal launch interface between the step engine and the kernels.
+#pragma once
+
+#include "common.cuh"
+
+namespace gpt {
+
+// Per-launch bookkeeping: launch counter and optional CUDA-event timing by
+// kernel name (used by the bench's per-kernel roofline report).
+struct Timing;
+struct Ctx {
+  cudaStream_t stream = nullptr;
+  uint32_t* flags = nullptr;  // device flag word
+  int num_sms = 148;
+  uint64_t launches = 0;
+  Timing* timing = nullptr;   // null when timing is off
+};
+
+void timing_begin(Ctx& c, const char* name);
+void timing_end(Ctx& c, const char* name);
+
+struct LaunchScope {
+  Ctx& c;
+  const char* name;
+  LaunchScope(Ctx& c_, const char* n) : c(c_), name(n) {
+    c.launches++;
+    if (c.timing) timing_begin(c, name);
+  }
+  ~LaunchScope() {
+    if (c.timing) timing_end(c, name);
+  }
+};
+
+// ---------------------------------------------------------------- GEMM
+// D[m, n] = sum_k A[m, k] * B[n, k], fp32 accumulation, then an epilogue.
+enum EpiKind {
+  EPI_STORE = 0,      // out = acc                                   (operand type)
+  EPI_BIAS = 1,       // out = acc + bias                            (operand type)
+  EPI_BIAS_ACT = 2,   // out = acc + bias (pre-activation), out2 = act(out)
+  EPI_RESADD = 3,     // res_out = res_in + drop(acc + bias)         (fp32)
+  EPI_ACT_BWD = 4,    // out = acc * act'(aux)                       (operand type)
+  EPI_ACC_F32 = 5,    // outf += acc                                 (fp32, grad accumulation)
+  EPI_STORE_F32 = 6   // outf = acc                                  (fp32)
+};
+enum ActKind { ACT_GELU = 0, ACT_RELU = 1 };
+
+struct GemmEpi {
+  int kind = EPI_STORE;
+  int act = ACT_GELU;
+  void* out = nullptr;        // operand-typed output (kinds 0,1,2,4) or fp32 (5,6)
+  void* out2 = nullptr;       // activation output of EPI_BIAS_ACT (same ld as out)
+  int ldo = 0;
+  const void* aux = nullptr;  // pre-activation h of EPI_ACT_BWD (operand type, ld = ldo)
+  const float* bias = nullptr;
+  const float* res_in = nullptr;
+  float* res_out = nullptr;
+  int ld_res = 0;
+  DropKey drop{};             // EPI_RESADD; element index = m * N + n
+};
+
+struct GemmDesc {
+  int M = 0, N = 0, K = 0;
+  const void* A = nullptr;
+  long lda = 0;
+  bool a_kmajor = true;       // true: A[m,k] at A[m*lda + k]; false: at A[k*lda + m]
+  const void* B = nullptr;
+  long ldb = 0;
+  bool b_kmajor = true;       // true: B[n,k] at B[n*ldb + k]; false: at B[k*ldb + n]
+  GemmEpi epi;
+  int split_k = 1;            // > 1 only with EPI_ACC_F32: partials in `partial`
+  float* partial = nullptr;   // [split_k, M, N] fp32 scratch
+};
+
+// fp32 operands on CUDA cores (fp32 mode); bf16 operands on CUDA cores
+// (reference path used by tests); bf16 operands on tcgen05 tensor cores.
+void gemm_simt_f32(Ctx& c, const GemmDesc& g);
+void gemm_simt_bf16(Ctx& c, const GemmDesc& g);
+bool gemm_tc_supported(const GemmDesc& g);
+bool gemm_tc_bf16(Ctx& c, const GemmDesc& g);  // false: tensor-map encode failed
+// split-K reduction: out[m,n] += sum_s partial[s,m,n] (fixed order)
+void splitk_reduce(Ctx& c, const float* partial, int splits, long MN, float* out);
+
+// ---------------------------------------------------------------- attention
+// qkv: [B, T, 3, H, hd] (row m = b*T + t holds q | k | v, heads contiguous)
+// o: [B, T, H, hd]; lse: [B, H, T] natural-log log-sum-exp of the scaled scores.
+struct AttnDesc {
+  int B, T, H, hd;
+  const void* qkv;
+  void* o;
+  float* lse;
+  const void* dout;   // bwd: dO [B, T, H, hd]
+  void* dqkv;         // bwd: [B, T, 3, H, hd]
+  float* dsum;        // bwd scratch: rowsum(dO * O) [B, H, T]
+  DropKey drop;       // site 1; elem = ((b*H + h)*T + i)*T + j
+};
+template <typename T> void attn_fwd_simt(Ctx& c, const AttnDesc& a);
+template <typename T> void attn_bwd_simt(Ctx& c, const AttnDesc& a);
+bool attn_tc_supported(const AttnDesc& a);
+void attn_fwd_tc(Ctx& c, const AttnDesc& a);
+void attn_bwd_tc(Ctx& c, const AttnDesc& a);
+
+// ---------------------------------------------------------------- memory-bound kernels
+void gather_batch(Ctx& c, const void* stream, int tok_u16, uint64_t len, uint64_t seed, int step, int micro,
+                  int B, int T, int V, int32_t* idx, int32_t* tgt);
+void check_tokens(Ctx& c, const int32_t* idx, const int32_t* tgt, long n, int V, int32_t* idx_out,
+                  int32_t* tgt_out);
+
+template <typename T>
+void embed_fwd(Ctx& c, const int32_t* idx, const float* wte, const float* wpe, float* res, int B, int Tn, int d,
+               DropKey drop);
+
+// LayerNorm / RMSNorm forward: y (T), mean, rstd fp32 [rows]
+template <typename T>
+void norm_fwd(Ctx& c, const float* x, const float* w, const float* b, T* y, float* mean, float* rstd, long rows,
+              int d, bool rms, float eps);
+
+// Norm backward.  dx = norm'(dy) is added to dres (or stored when !accumulate);
+// then dyb = drop(dres) is written (operand type) and its column sums, together
+// with dgain = sum dy*xhat and dbias = sum dy, go to per-block partials
+// part[blocks, 3, d] (order: dgain, dbeta, dbias_next).
+struct NormBwd {
+  const float* dy; const float* x; const float* mean; const float* rstd; const float* w;
+  float* dres; bool accumulate;
+  void* dyb; DropKey drop; bool want_dyb;
+  float* part; int blocks;
+  long rows; int d; bool rms;
+};
+template <typename T> void norm_bwd(Ctx& c, const NormBwd& p);
+int norm_bwd_blocks(Ctx& c, long rows);
+// grad[j] += sum_b part[b, slot, j] for the given slot
+void partial_reduce(Ctx& c, const float* part, int blocks, int slots, int slot, int d, float* grad);
+
+// column sums of an operand-typed [rows, N] matrix into grad (+=), deterministic
+template <typename T> void colsum_acc(Ctx& c, const T* x, long rows, int N, float* scratch, float* grad);
+
+// Cross-entropy over [M, Vp] logits (operand type).  Writes per-row lse and
+// loss terms; with want_grad, overwrites logits with (softmax - onehot)*scale
+// (pad columns 0).
+template <typename T>
+void ce_fwd_bwd(Ctx& c, T* logits, const int32_t* tgt, long M, int V, int Vp, float* lse, float* row_loss,
+                bool want_grad, float scale);
+void loss_reduce(Ctx& c, const float* row_loss, long M, float scale, float* loss_acc, int accumulate);
+
+// embedding backward: routing (stable sort of positions by token) + sums
+void embed_sort(Ctx& c, const int32_t* idx, long M, int32_t* sorted_tok, int32_t* sorted_pos, int32_t* n_unique);
+void embed_bwd(Ctx& c, const float* dres, const int32_t* sorted_tok, const int32_t* sorted_pos, long M, int Tn,
+               int Bn, int d, DropKey drop, float* dwte, float* dwpe);
+
+// grad norm partials, clip + AdamW
+void sumsq_partials(Ctx& c, const float* g, long n, double* partials, int blocks);
+int sumsq_blocks(Ctx& c);
+struct AdamArgs {
+  float* w; float* g; float* m; float* v; bf16* wb;  // wb may be null (fp32 mode)
+  long n; long n_decay;
+  const double* norm_partials; int norm_blocks; float* norm_out;
+  float lr, beta1, beta2, eps, wd, clip, bc1, bc2;
+};
+void adamw(Ctx& c, const AdamArgs& a);
+void to_bf16(Ctx& c, const float* src, bf16* dst, long n);
+void argmax_rows(Ctx& c, const void* x, int is_bf16, long rows, int cols, int ld, int32_t* out);
+void dropout_mask(Ctx& c, DropKey k, long n, uint8_t* out);
+
+}  // namespace gpt

@@ -1,0 +1,82 @@
+// Kernel-level entry points for the parity tests (include/gpt_testing.h).
+#include "../../include/gpt_testing.h"
+#include "kernels.cuh"
+
+using namespace gpt;
+
+extern "C" gpt_status gpt_test_gemm(int32_t backend, int32_t M, int32_t N, int32_t K, const void* A, int64_t lda,
+                                    int32_t a_kmajor, const void* B, int64_t ldb, int32_t b_kmajor, int32_t epi_kind,
+                                    int32_t act, void* out, void* out2, int32_t ldo, const void* aux,
+                                    const float* bias, const float* res_in, float* res_out, int32_t split_k,
+                                    float* partial, void* stream, uint32_t* d_flags) {
+  if (M <= 0 || N <= 0 || K <= 0 || !A || !B || epi_kind < 0 || epi_kind > 6) return GPT_ERR_INVALID_ARG;
+  Ctx c;
+  c.stream = (cudaStream_t)stream;
+  c.flags = d_flags;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess) c.num_sms = sms;
+  GemmDesc g;
+  g.M = M;
+  g.N = N;
+  g.K = K;
+  g.A = A;
+  g.lda = lda;
+  g.a_kmajor = a_kmajor != 0;
+  g.B = B;
+  g.ldb = ldb;
+  g.b_kmajor = b_kmajor != 0;
+  g.epi.kind = epi_kind;
+  g.epi.act = act;
+  g.epi.out = out;
+  g.epi.out2 = out2;
+  g.epi.ldo = ldo;
+  g.epi.aux = aux;
+  g.epi.bias = bias;
+  g.epi.res_in = res_in;
+  g.epi.res_out = res_out;
+  g.epi.ld_res = ldo;
+  g.split_k = split_k;
+  g.partial = partial;
+  switch (backend) {
+    case GPT_GEMM_SIMT_F32: gemm_simt_f32(c, g); break;
+    case GPT_GEMM_SIMT_BF16: gemm_simt_bf16(c, g); break;
+    case GPT_GEMM_TC_BF16:
+      if (!gemm_tc_supported(g)) return GPT_ERR_UNSUPPORTED;
+      if (!gemm_tc_bf16(c, g)) return GPT_ERR_CUDA;
+      break;
+    default: return GPT_ERR_INVALID_ARG;
+  }
+  if (cudaStreamSynchronize(c.stream) != cudaSuccess || cudaGetLastError() != cudaSuccess) return GPT_ERR_CUDA;
+  return GPT_OK;
+}
+
+extern "C" gpt_status gpt_test_attention(int32_t backend, int32_t backward, int32_t dtype, int32_t B, int32_t T,
+                                         int32_t H, int32_t hd, const void* qkv, void* o, float* lse,
+                                         const void* dout, void* dqkv, float* dsum, float p, uint64_t seed,
+                                         uint64_t counter, int32_t layer, void* stream, uint32_t* d_flags) {
+  if (B <= 0 || T <= 0 || H <= 0 || !qkv || !o || !lse) return GPT_ERR_INVALID_ARG;
+  if (backward && (!dout || !dqkv || !dsum)) return GPT_ERR_INVALID_ARG;
+  Ctx c;
+  c.stream = (cudaStream_t)stream;
+  c.flags = d_flags;
+  AttnDesc a{B, T, H, hd, qkv, o, lse, dout, dqkv, dsum, make_drop_key(seed, counter, layer, 1, p)};
+  if (backend == 1) {
+    if (dtype != 1 || !attn_tc_supported(a)) return GPT_ERR_UNSUPPORTED;
+    if (backward) attn_bwd_tc(c, a);
+    else attn_fwd_tc(c, a);
+  } else if (backend == 0) {
+    if (hd != 4 && hd != 8 && hd != 16 && hd != 32 && hd != 64 && hd != 128) return GPT_ERR_UNSUPPORTED;
+    if (dtype == 1) {
+      if (backward) attn_bwd_simt<bf16>(c, a);
+      else attn_fwd_simt<bf16>(c, a);
+    } else {
+      if (backward) attn_bwd_simt<float>(c, a);
+      else attn_fwd_simt<float>(c, a);
+    }
+  } else {
+    return GPT_ERR_INVALID_ARG;
+  }
+  if (cudaStreamSynchronize(c.stream) != cudaSuccess || cudaGetLastError() != cudaSuccess) return GPT_ERR_CUDA;
+  return GPT_OK;
+}

@@ -1,0 +1,250 @@
+/*
+ * gpt.h -- C ABI of the B200 (sm_100a) GPT-2 causal-LM training step.
+ *
+ * The library implements one training step of a nanoGPT-style GPT-2:
+ * token + learned position embedding, n_layer pre-norm blocks (norm, fused
+ * QKV projection, causal scaled-dot-product attention, output projection,
+ * residual; norm, 4x MLP, residual), a final norm, an lm_head tied to the
+ * token embedding, mean cross-entropy, the full backward pass, global-norm
+ * gradient clipping and AdamW.
+ *
+ * Sources (web pages; section names are the pages' own):
+ *   - "nanoGPT README" (translated): model.py / train.py, GPT-2 124M
+ *     reproduction ("复现 GPT-2"), benchmarking ("效率说明").
+ *   - "从零实现GPT训练与推理：基于nanoGPT的实战指南": section 3 (config
+ *     n_layer/n_head/n_embd), section 6 ("性能优化技巧": get_lr warmup +
+ *     cosine, bf16, gradient accumulation).
+ *   - nanoGPT run log (wmrh.cn): section 1.3 (train.bin token stream,
+ *     block_size windows), 2.1 (config table), 2.2 (head_dim), 2.3
+ *     (parameter count), 3.1 (gradient accumulation), 4.5 (fixed seeds).
+ *   - "微型 GPT 从零构建：核心训练循环、分词与单 GPU 高效推理": sections
+ *     "模型核心" (microGPT architecture: RMSNorm, ReLU, 4192 params) and
+ *     "核心训练循环" (forward, -log p loss, backward, Adam, clip 1.0).
+ *
+ * Conventions for every entry point:
+ *   - Device pointers are plain CUDA device addresses on the device that
+ *     was current when the model was created; host pointers are ordinary
+ *     (preferably pinned) host memory.
+ *   - All device work is enqueued on the model's stream (gpt_create /
+ *     gpt_set_stream).  A call that takes a host output pointer (h_loss,
+ *     h_grad_norm, h_out ...) synchronises that stream before it returns;
+ *     passing NULL keeps the call asynchronous.
+ *   - The caller owns the device workspace (see gpt_workspace_bytes); the
+ *     library carves every device buffer it uses out of it and performs no
+ *     device allocation.  The workspace must outlive the model.
+ *   - Errors are returned as gpt_status; nothing aborts the process or
+ *     traps the GPU.  Argument and sequencing errors are detected on the
+ *     host before any launch.  Conditions only the device can see (a token
+ *     id >= vocab_size, a non-finite loss or gradient norm, a bounded wait
+ *     in a kernel that ran out) set bits in a device flag word that the
+ *     next synchronising call reports (and gpt_read_flags returns).
+ *   - gpt_last_error() gives a human-readable message for the last failing
+ *     call on a model.
+ */
+#ifndef GPT_B200_H
+#define GPT_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define GPT_ABI_VERSION 1u
+
+typedef enum {
+  GPT_OK = 0,
+  GPT_ERR_INVALID_ARG = 1,       /* NULL pointer, bad size, bad enum value            */
+  GPT_ERR_CONFIG = 2,            /* inconsistent config (n_embd % n_head != 0 ...)    */
+  GPT_ERR_WORKSPACE_TOO_SMALL = 3,
+  GPT_ERR_CUDA = 4,              /* a CUDA runtime/driver call failed                 */
+  GPT_ERR_TOKEN_RANGE = 5,       /* a token id was outside [0, vocab_size)            */
+  GPT_ERR_NONFINITE = 6,         /* loss or gradient norm was NaN/Inf                 */
+  GPT_ERR_STATE = 7,             /* call out of sequence (backward before forward)    */
+  GPT_ERR_UNSUPPORTED = 8,       /* valid request this build does not implement       */
+  GPT_ERR_TIMEOUT = 9            /* a bounded device-side wait ran out                */
+} gpt_status;
+
+enum { GPT_PREC_FP32 = 0, GPT_PREC_BF16 = 1 };
+/* GPT2: LayerNorm with gain/bias, biases on every linear layer, GELU (erf
+ * form), lm_head tied to wte.  MICRO (microGPT page, "模型核心"):
+ * parameter-free RMSNorm, no biases, ReLU, untied lm_head. */
+enum { GPT_VARIANT_GPT2 = 0, GPT_VARIANT_MICRO = 1 };
+enum { GPT_TOK_I32 = 0, GPT_TOK_U16 = 1 };
+/* kinds of per-parameter arrays for gpt_get_tensor / gpt_set_tensor */
+enum { GPT_PARAM = 0, GPT_GRAD = 1, GPT_ADAM_M = 2, GPT_ADAM_V = 3 };
+/* device flag bits (gpt_read_flags) */
+enum {
+  GPT_FLAG_TOKEN_RANGE = 1u << 0,
+  GPT_FLAG_NONFINITE_LOSS = 1u << 1,
+  GPT_FLAG_NONFINITE_NORM = 1u << 2,
+  GPT_FLAG_TIMEOUT = 1u << 3
+};
+
+/* Plain-old-data model + optimiser configuration.  Field names follow the
+ * nanoGPT config files (practical guide section 3; run log section 2.1). */
+typedef struct gpt_config {
+  uint32_t abi_version;   /* must be GPT_ABI_VERSION                                 */
+  int32_t vocab_size;     /* V: token ids are in [0, V)                              */
+  int32_t padded_vocab;   /* Vp >= V, multiple of 64; 0 = round V up to 64.  Rows
+                             V..Vp-1 of wte are layout padding: zero, never updated,
+                             excluded from the loss (their logits are masked).       */
+  int32_t n_layer;        /* L >= 1                                                  */
+  int32_t n_head;         /* H; head_dim = n_embd / n_head (run log section 2.2)     */
+  int32_t n_embd;         /* d, multiple of 8 (multiple of 64 in bf16 mode)          */
+  int32_t block_size;     /* T: sequence length of every window                      */
+  int32_t batch_size;     /* B: windows per micro-batch                              */
+  int32_t grad_accum;     /* micro-batches per optimiser step (>= 1)                 */
+  int32_t precision;      /* GPT_PREC_FP32 (all fp32, SIMT) or GPT_PREC_BF16         */
+  int32_t variant;        /* GPT_VARIANT_GPT2 or GPT_VARIANT_MICRO                   */
+  int32_t token_dtype;    /* element type of the token stream in gpt_train_step      */
+  float init_std;         /* std of the Gaussian init of matrices and embeddings     */
+  float dropout;          /* p in [0, 1); 0 disables every dropout site              */
+  float beta1, beta2, eps;
+  float weight_decay;     /* decoupled (AdamW); applied to 2-D tensors only unless
+                             decay_1d != 0                                           */
+  float grad_clip;        /* global-norm clip threshold; <= 0 disables clipping      */
+  int32_t decay_1d;
+  int32_t reserved0;
+  uint64_t dropout_seed;  /* key of the dropout counter hash                         */
+} gpt_config;
+
+typedef struct gpt_model gpt_model;
+
+/* ---------------------------------------------------------------- pure host */
+
+/* Number of trainable parameters (padding excluded): for GPT2
+ * V*d + T*d + L*(12 d^2 + 13 d) + 2 d (run log section 2.3 breakdown);
+ * for MICRO 2*V*d + T*d + 12*L*d^2 (4192 at the microGPT size).
+ * Returns 0 for an invalid config. */
+size_t gpt_param_count(const gpt_config* cfg);
+
+/* Bytes of device workspace a model with this config needs (out). */
+gpt_status gpt_workspace_bytes(const gpt_config* cfg, size_t* out);
+
+/* get_lr of the practical guide, section 6: lr*it/warmup while it < warmup,
+ * then lr*0.5*(1+cos(pi*(it-warmup)/(max_iters-warmup))).  Pure function. */
+float gpt_lr_cosine(float lr, int32_t it, int32_t warmup, int32_t max_iters);
+/* microGPT "核心训练循环": lr*(1 - it/max_iters).  Pure function. */
+float gpt_lr_linear(float lr, int32_t it, int32_t max_iters);
+
+/* ---------------------------------------------------------------- lifetime */
+
+/* Creates a model in a caller-owned device workspace of `bytes` bytes
+ * (>= gpt_workspace_bytes) and initialises its weights from `seed`
+ * (matrices/embeddings ~ N(0, init_std^2) from a SplitMix64 counter hash
+ * with Box-Muller, biases 0, norm gains 1; AdamW moments 0).  `cuda_stream`
+ * is a cudaStream_t (NULL = legacy default stream).  Synchronises. */
+gpt_status gpt_create(const gpt_config* cfg, uint64_t seed, void* d_workspace, size_t bytes,
+                      void* cuda_stream, gpt_model** out);
+void gpt_destroy(gpt_model* m);
+gpt_status gpt_set_stream(gpt_model* m, void* cuda_stream);
+
+/* ---------------------------------------------------------------- the step */
+
+/* Forward pass and mean cross-entropy of one micro-batch.
+ * d_idx, d_tgt: device int32 [batch_size, block_size] token ids and next-token
+ * targets (owned by the caller, read during the call's device work).
+ * h_loss (nullable): receives the loss (synchronises).
+ * The dropout masks use the cursor set by gpt_set_dropout_cursor. */
+gpt_status gpt_forward_loss(gpt_model* m, const int32_t* d_idx, const int32_t* d_tgt, float* h_loss);
+
+/* Backward pass of the last gpt_forward_loss; gradients of loss/grad_accum
+ * are ADDED into the fp32 gradient arena.  GPT_ERR_STATE without a
+ * preceding forward. */
+gpt_status gpt_backward(gpt_model* m);
+
+/* Global-norm clip + one AdamW update of every parameter with learning rate
+ * `lr` and bias-correction index `step` (>= 1); zeroes the gradients and
+ * refreshes the bf16 weight copy.  h_grad_norm (nullable) receives the
+ * pre-clip norm.  A non-finite norm skips the update on the device (weights
+ * and moments unchanged, gradients still zeroed) and, when h_grad_norm is
+ * given, returns GPT_ERR_NONFINITE. */
+gpt_status gpt_clip_adamw_step(gpt_model* m, float lr, int32_t step, float* h_grad_norm);
+
+/* One full optimiser step: for micro = 0..grad_accum-1, gather a batch of
+ * random windows from the device-resident token stream (d_stream,
+ * stream_len tokens of cfg.token_dtype), forward, backward; then clip +
+ * AdamW with (lr, step).  Window starts: SplitMix64 hash of
+ * (data_seed, step, micro, b) mod (stream_len - block_size).
+ * Dropout counter = step*grad_accum + micro.  h_loss (mean over the
+ * micro-batches) and h_grad_norm are nullable. */
+gpt_status gpt_train_step(gpt_model* m, const void* d_stream, uint64_t stream_len, uint64_t data_seed,
+                          float lr, int32_t step, float* h_loss, float* h_grad_norm);
+
+/* Same step with the micro-batches supplied from HOST memory: h_idx and
+ * h_tgt are int32 [grad_accum, batch_size, block_size] (pinned memory keeps
+ * the copies asynchronous).  The host->device copies are part of the call. */
+gpt_status gpt_train_step_host(gpt_model* m, const int32_t* h_idx, const int32_t* h_tgt, float lr,
+                               int32_t step, float* h_loss, float* h_grad_norm);
+
+/* The batch gather of gpt_train_step on its own: writes int32
+ * [batch_size, block_size] ids and targets to d_idx / d_tgt. */
+gpt_status gpt_gather_batch(gpt_model* m, const void* d_stream, uint64_t stream_len, uint64_t data_seed,
+                            int32_t step, int32_t micro, int32_t* d_idx, int32_t* d_tgt);
+
+/* Dropout cursor used by gpt_forward_loss / gpt_backward: counter =
+ * step*grad_accum + micro. */
+gpt_status gpt_set_dropout_cursor(gpt_model* m, int32_t step, int32_t micro);
+
+/* ---------------------------------------------------------------- introspection (tests, resume) */
+
+gpt_status gpt_num_tensors(gpt_model* m, int32_t* n);
+/* Name (static storage) and logical shape of tensor i in the canonical
+ * order: wte, wpe, per layer ln_1.{weight,bias}, attn.c_attn.{weight,bias},
+ * attn.c_proj.{weight,bias}, ln_2.{weight,bias}, mlp.c_fc.{weight,bias},
+ * mlp.c_proj.{weight,bias} (MICRO: weights only), then ln_f.{weight,bias}
+ * (GPT2) or lm_head.weight (MICRO).  shape[1] = 1 for vectors.  The logical
+ * shape of wte / lm_head is [vocab_size, n_embd] (padding rows hidden). */
+gpt_status gpt_tensor_info(gpt_model* m, int32_t i, const char** name, int64_t shape[2]);
+/* Copies tensor i of the given kind (GPT_PARAM .. GPT_ADAM_V) as fp32
+ * to / from host memory (shape as gpt_tensor_info).  Setting GPT_PARAM also
+ * refreshes the bf16 copy.  Synchronising. */
+gpt_status gpt_get_tensor(gpt_model* m, int32_t i, int32_t kind, float* h_out);
+gpt_status gpt_set_tensor(gpt_model* m, int32_t i, int32_t kind, const float* h_in);
+/* Logits of the last forward as fp32 [B*T, vocab_size] (pad columns
+ * dropped), and their row argmax (ties -> lowest index) as int32 [B*T]. */
+gpt_status gpt_get_logits(gpt_model* m, float* h_out);
+gpt_status gpt_get_argmax(gpt_model* m, int32_t* h_out);
+/* Argmax of caller-supplied fp32 rows [rows, cols] held in device memory
+ * (same kernel as gpt_get_argmax); h_out int32 [rows]. */
+gpt_status gpt_argmax_rows(gpt_model* m, const float* d_rows, int32_t rows, int32_t cols, int32_t* h_out);
+/* Per-row log-sum-exp of the last forward's logits, fp32 [B*T]. */
+gpt_status gpt_get_lse(gpt_model* m, float* h_out);
+/* The embedding-gradient routing of the last backward: number of distinct
+ * token ids touched (h_n_unique), the sorted token of each position
+ * (h_sorted_tok int32 [B*T]) and the position each sorted slot came from
+ * (h_sorted_pos int32 [B*T]); positions of one token are ascending. */
+gpt_status gpt_get_embed_routing(gpt_model* m, int32_t* h_n_unique, int32_t* h_sorted_tok, int32_t* h_sorted_pos);
+/* Dropout keep mask of one site as uint8 [n] for elements [0, n) of
+ * (counter, layer, site) -- the same device function the kernels use. */
+gpt_status gpt_dropout_mask(gpt_model* m, int64_t counter, int32_t layer, int32_t site, int64_t n, uint8_t* h_out);
+
+/* Optimiser state for checkpoint / resume: fp32 master weights, AdamW m and
+ * v (each gpt_param_count()-sized in canonical tensor order) and the step
+ * counter.  Buffers are host memory of state_floats() floats each. */
+size_t gpt_state_floats(gpt_model* m);
+gpt_status gpt_get_state(gpt_model* m, float* h_param, float* h_m, float* h_v);
+gpt_status gpt_set_state(gpt_model* m, const float* h_param, const float* h_m, const float* h_v);
+
+/* Device flag word (GPT_FLAG_*) since the last gpt_clear_flags; synchronising. */
+gpt_status gpt_read_flags(gpt_model* m, uint32_t* h_flags);
+gpt_status gpt_clear_flags(gpt_model* m);
+
+/* Per-kernel timing of the last step (CUDA events on the model's stream):
+ * enable with on != 0; gpt_kernel_times copies up to `cap` (name, total ms,
+ * launches) records.  Used by the bench's roofline report. */
+gpt_status gpt_enable_timing(gpt_model* m, int32_t on);
+gpt_status gpt_kernel_times(gpt_model* m, int32_t cap, const char** names, float* total_ms, int32_t* launches,
+                            int32_t* n_out);
+/* Number of kernel launches the library made since the model was created. */
+uint64_t gpt_launch_count(gpt_model* m);
+
+const char* gpt_last_error(const gpt_model* m);
+const char* gpt_status_string(gpt_status s);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* GPT_B200_H */

@@ -1,0 +1,55 @@
+/*
+ * gpt_testing.h -- kernel-level entry points of libgpt.so used by the parity
+ * tests to check one kernel at a time (the GEMM with its epilogues, the
+ * attention forward/backward) against the CPU oracle.  Not part of the
+ * training step's hot path.  All pointers are device pointers on the current
+ * device; work is enqueued on `stream` (a cudaStream_t) and the call
+ * synchronises it before returning.  `d_flags` is a device uint32 that
+ * receives the GPT_FLAG_* bits the kernels raise.
+ */
+#ifndef GPT_B200_TESTING_H
+#define GPT_B200_TESTING_H
+
+#include <stdint.h>
+
+#include "gpt.h"
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Backends of gpt_test_gemm. */
+enum { GPT_GEMM_SIMT_F32 = 0, GPT_GEMM_SIMT_BF16 = 1, GPT_GEMM_TC_BF16 = 2 };
+
+/* D[m, n] = sum_k A[m, k] * B[n, k] followed by epilogue `epi_kind`:
+ *   0 out = D; 1 out = D + bias; 2 out = D + bias, out2 = act(out);
+ *   3 res_out = res_in + D + bias; 4 out = D * act'(aux);
+ *   5 out += D (fp32); 6 out = D (fp32).
+ * A is [M, K] row-major with pitch lda when a_kmajor, else [K, M] (pitch lda);
+ * B is [N, K] when b_kmajor, else [K, N].  Operands are fp32 for
+ * GPT_GEMM_SIMT_F32 and bf16 otherwise; outputs of kinds 0-2 and 4 have the
+ * operand type, kinds 3, 5 and 6 are fp32.  act: 0 GELU (erf), 1 ReLU.
+ * split_k > 1 (kind 5 only, tensor-core backend) needs `partial`
+ * [split_k, M, N] fp32 scratch.  GPT_ERR_UNSUPPORTED when the tensor-core
+ * backend cannot take the shape. */
+gpt_status gpt_test_gemm(int32_t backend, int32_t M, int32_t N, int32_t K, const void* A, int64_t lda,
+                         int32_t a_kmajor, const void* B, int64_t ldb, int32_t b_kmajor, int32_t epi_kind,
+                         int32_t act, void* out, void* out2, int32_t ldo, const void* aux, const float* bias,
+                         const float* res_in, float* res_out, int32_t split_k, float* partial, void* stream,
+                         uint32_t* d_flags);
+
+/* Causal attention of one layer.  qkv [B, T, 3, H, hd], o [B, T, H, hd],
+ * lse fp32 [B, H, T]; backward also takes dout [B, T, H, hd] and writes
+ * dqkv [B, T, 3, H, hd] using dsum fp32 [B, H, T] as scratch.  dtype: 0 fp32,
+ * 1 bf16.  backend: 0 CUDA cores, 1 tensor cores (GPT_ERR_UNSUPPORTED when
+ * the shape is not supported).  Dropout on the probabilities with
+ * (p, seed, counter, layer) as in the model (site 1); p = 0 disables it. */
+gpt_status gpt_test_attention(int32_t backend, int32_t backward, int32_t dtype, int32_t B, int32_t T, int32_t H,
+                              int32_t hd, const void* qkv, void* o, float* lse, const void* dout, void* dqkv,
+                              float* dsum, float p, uint64_t seed, uint64_t counter, int32_t layer, void* stream,
+                              uint32_t* d_flags);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* GPT_B200_TESTING_H */

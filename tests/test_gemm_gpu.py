@@ -1,0 +1,140 @@
+"""Tensor-core (tcgen05) GEMM and its epilogues against the fp64 definition.
+
+Inputs are bf16-rounded on the host; the reference is the float64 matrix
+product of those rounded values (the oracle's contraction primitive), then
+the epilogue written out element-wise.
+"""
+
+import math
+
+import numpy as np
+import pytest
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+if not torch.cuda.is_available():
+    pytest.skip("needs a GPU", allow_module_level=True)
+
+from gpt_decoder_lm_b200 import binding as gb  # noqa: E402
+from scipy.special import erf  # noqa: E402
+
+TC, SIMT_BF16, SIMT_F32 = 2, 1, 0
+
+
+def bf16_round(x: np.ndarray) -> np.ndarray:
+    return torch.from_numpy(np.asarray(x, np.float32)).bfloat16().float().numpy().astype(np.float64)
+
+
+def dev_bf16(x):
+    return torch.from_numpy(np.ascontiguousarray(x, np.float32)).cuda().bfloat16()
+
+
+def dev_f32(x):
+    return torch.from_numpy(np.ascontiguousarray(x, np.float32)).cuda()
+
+
+def gelu(x):
+    return x * 0.5 * (1 + erf(x / math.sqrt(2)))
+
+
+def gelu_grad(x):
+    return 0.5 * (1 + erf(x / math.sqrt(2))) + x * np.exp(-0.5 * x * x) / math.sqrt(2 * math.pi)
+
+
+def operands(M, N, K, ak, bk, seed):
+    rng = np.random.default_rng(seed)
+    A = bf16_round(rng.standard_normal((M, K)))
+    B = bf16_round(rng.standard_normal((N, K)))
+    Ad = dev_bf16(A if ak else A.T)
+    Bd = dev_bf16(B if bk else B.T)
+    lda = K if ak else M
+    ldb = K if bk else N
+    return A, B, Ad, Bd, lda, ldb
+
+
+def run(backend, M, N, K, Ad, lda, ak, Bd, ldb, bk, kind, **kw):
+    flags = torch.zeros(1, dtype=torch.int32, device="cuda")
+    st = gb.test_gemm(backend, M, N, K, Ad, lda, ak, Bd, ldb, bk, kind,
+                      stream=torch.cuda.current_stream().cuda_stream, flags=flags, **kw)
+    assert gb.STATUS[st] == "GPT_OK", gb.STATUS[st]
+    assert int(flags.item()) == 0
+
+
+LAYOUTS = [(1, 1), (1, 0), (0, 0)]   # forward (TN), dX (B MN-major), dW (both MN-major)
+SHAPES = [(128, 128, 64), (256, 384, 192), (200, 328, 136), (1024, 2304, 256), (4096, 1024, 128), (64, 96, 520)]
+
+
+@pytest.mark.parametrize("ak,bk", LAYOUTS, ids=["tn", "b_mn", "ab_mn"])
+@pytest.mark.parametrize("M,N,K", SHAPES, ids=[f"{m}x{n}x{k}" for m, n, k in SHAPES])
+def test_tc_gemm_store_f32(M, N, K, ak, bk):
+    A, B, Ad, Bd, lda, ldb = operands(M, N, K, ak, bk, M + N + K)
+    out = torch.full((M, N), float("nan"), device="cuda")
+    run(TC, M, N, K, Ad, lda, ak, Bd, ldb, bk, 6, out=out, ldo=N)
+    ref = A @ B.T
+    got = out.double().cpu().numpy()
+    err = np.abs(got - ref).max() / np.abs(ref).max()
+    assert err < 2e-6, err
+
+
+@pytest.mark.parametrize("backend", [TC, SIMT_BF16], ids=["tc", "simt"])
+def test_epilogues(backend):
+    M, N, K = 384, 512, 256
+    rng = np.random.default_rng(7)
+    A, B, Ad, Bd, lda, ldb = operands(M, N, K, 1, 1, 3)
+    D = A @ B.T
+    bias = rng.standard_normal(N).astype(np.float32)
+    bias_d = dev_f32(bias)
+    # 1: bias
+    out = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    run(backend, M, N, K, Ad, lda, 1, Bd, ldb, 1, 1, out=out, ldo=N, bias=bias_d)
+    np.testing.assert_allclose(out.double().cpu().numpy(), D + bias, rtol=1e-2, atol=0.06)
+    # 2: bias + GELU (pre-activation and activation)
+    out2 = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    run(backend, M, N, K, Ad, lda, 1, Bd, ldb, 1, 2, act=0, out=out, out2=out2, ldo=N, bias=bias_d)
+    h = D + bias
+    np.testing.assert_allclose(out.double().cpu().numpy(), h, rtol=1e-2, atol=0.06)
+    np.testing.assert_allclose(out2.double().cpu().numpy(), gelu(h), rtol=1e-2, atol=0.06)
+    run(backend, M, N, K, Ad, lda, 1, Bd, ldb, 1, 2, act=1, out=out, out2=out2, ldo=N, bias=bias_d)
+    np.testing.assert_allclose(out2.double().cpu().numpy(), np.maximum(h, 0), rtol=1e-2, atol=0.06)
+    # 3: residual add (fp32)
+    res = rng.standard_normal((M, N)).astype(np.float32)
+    res_in = dev_f32(res)
+    res_out = torch.empty_like(res_in)
+    run(backend, M, N, K, Ad, lda, 1, Bd, ldb, 1, 3, ldo=N, bias=bias_d, res_in=res_in, res_out=res_out)
+    np.testing.assert_allclose(res_out.double().cpu().numpy(), res + D + bias, rtol=1e-5, atol=1e-4)
+    # 4: activation backward
+    hh = bf16_round(rng.standard_normal((M, N)))
+    aux = dev_bf16(hh)
+    run(backend, M, N, K, Ad, lda, 1, Bd, ldb, 1, 4, act=0, out=out, ldo=N, aux=aux)
+    np.testing.assert_allclose(out.double().cpu().numpy(), D * gelu_grad(hh), rtol=1e-2, atol=0.06)
+    # 5: fp32 accumulate
+    acc0 = rng.standard_normal((M, N)).astype(np.float32)
+    acc = dev_f32(acc0)
+    run(backend, M, N, K, Ad, lda, 1, Bd, ldb, 1, 5, out=acc, ldo=N)
+    np.testing.assert_allclose(acc.double().cpu().numpy(), acc0 + D, rtol=1e-5, atol=1e-4)
+
+
+@pytest.mark.parametrize("splits", [2, 5])
+def test_tc_split_k_accumulate(splits):
+    M, N, K = 256, 384, 4096      # dW-like: both operands MN-major, long contraction
+    A, B, Ad, Bd, lda, ldb = operands(M, N, K, 0, 0, 11)
+    acc0 = np.random.default_rng(2).standard_normal((M, N)).astype(np.float32)
+    acc = dev_f32(acc0)
+    partial = torch.empty((splits, M, N), device="cuda")
+    run(TC, M, N, K, Ad, lda, 0, Bd, ldb, 0, 5, out=acc, ldo=N, split_k=splits, partial=partial)
+    ref = acc0 + A @ B.T
+    err = np.abs(acc.double().cpu().numpy() - ref).max() / np.abs(ref).max()
+    assert err < 2e-6, err
+
+
+def test_tc_matches_simt_bitwise_close():
+    M, N, K = 512, 768, 768
+    A, B, Ad, Bd, lda, ldb = operands(M, N, K, 1, 0, 5)
+    o1 = torch.empty((M, N), device="cuda")
+    o2 = torch.empty((M, N), device="cuda")
+    run(TC, M, N, K, Ad, lda, 1, Bd, ldb, 0, 6, out=o1, ldo=N)
+    run(SIMT_BF16, M, N, K, Ad, lda, 1, Bd, ldb, 0, 6, out=o2, ldo=N)
+    ref = A @ B.T
+    for o in (o1, o2):
+        assert np.abs(o.double().cpu().numpy() - ref).max() / np.abs(ref).max() < 2e-6
