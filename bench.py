@@ -1,0 +1,348 @@
+"""Training-step benchmark: tokens/s and MFU of the GPT-2 training step.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+A step is one full optimiser step of the GPT-2 124M workload (vocab 50257,
+12 layers, 12 heads, d 768, block 1024, micro-batch 12, grad-accum 5 ->
+61,440 tokens): batch gather from a device-resident synthetic token stream,
+forward, cross-entropy, backward, clip and AdamW, all in libgpt.so.  For
+N > 1 (torchrun) every rank trains its own replica on its own data: the
+step does not shard, so there is no collective on the data path; the
+barrier and the max-over-ranks timing use torch.distributed.
+
+`--impl reference` times the CPU oracle (float64 numpy) on a bounded sample
+of the same workload on the host cores (rank 0 only).
+
+Prints one JSON line.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from gpt_decoder_lm_b200 import workloads as W  # noqa: E402
+
+METRIC = "train tokens/sec (GPT-2 124M bf16, T=1024, 1 B200 per replica)"
+UNIT = "tokens/s"
+NOMINAL_BF16_TFLOPS = 2250.0
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16": d["bf16_tflops"], "bf16_sustained": d["bf16_tflops_sustained"],
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16": 1590.0, "bf16_sustained": 1400.0, "source": "fallback"}
+
+
+def flops_per_token(w) -> float:
+    """6 N + 12 L d T with N = parameters excluding wpe (PaLM appendix convention)."""
+    d, L, T, V = w.n_embd, w.n_layer, w.block_size, w.vocab_size
+    n = V * d + L * (12 * d * d + 13 * d) + 2 * d
+    return 6.0 * n + 12.0 * L * d * T
+
+
+def gemm_flops_per_step(w) -> float:
+    """Algorithmic dense-contraction FLOPs of one step (forward x3 for dX and dW)."""
+    d, L, V = w.n_embd, w.n_layer, w.vocab_size
+    M = w.batch_size * w.block_size
+    fwd = 2.0 * M * (L * (3 * d * d + d * d + 4 * d * d + 4 * d * d) + V * d)
+    return 3.0 * fwd * w.grad_accum
+
+
+def attn_flops_per_step(w) -> float:
+    """Causal attention FLOPs (S = QK^T and PV, lower triangle): fwd 2 matmuls, bwd 5 (+1 recompute)."""
+    T, d, L = w.block_size, w.n_embd, w.n_layer
+    per_layer_fwd = 2 * 2.0 * w.batch_size * d * T * (T + 1) / 2
+    return L * w.grad_accum * per_layer_fwd * (1 + 2.5)
+
+
+class Clocks:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        try:
+            self.p = subprocess.Popen(["nvidia-smi", f"--id={gpu_index}", f"--query-gpu={self.FIELDS}",
+                                       "--format=csv,noheader,nounits", "-lms", "100"], stdout=self.f,
+                                      stderr=subprocess.DEVNULL)
+        except Exception:
+            self.p = None
+
+    def stop(self):
+        if self.p is None:
+            return None
+        self.p.terminate()
+        try:
+            self.p.wait(5)
+        except Exception:
+            self.p.kill()
+        self.f.flush()
+        rows = [l.split(",") for l in open(self.f.name).read().splitlines() if l.strip()]
+        os.unlink(self.f.name)
+        sm = []
+        smax = None
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            try:
+                sm.append(float(r[1]))
+                smax = float(r[2])
+                for n, v in zip(names, r[5:9]):
+                    if v.strip() == "Active":
+                        reasons.add(n)
+            except Exception:
+                continue
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": smax, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def reduce_max(value: float, device) -> float:
+    """Max of a per-rank float over the process group (identity without one)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def oracle_sample_step(w, T_sample: int, state=None):
+    """One oracle training step (fwd + bwd + clip + AdamW) on a B=1 window of T_sample tokens
+    at the workload's model dims.  Returns (seconds, tokens, state)."""
+    import oracle
+    cfg = oracle.Config(vocab_size=w.vocab_size, n_layer=w.n_layer, n_head=w.n_head, n_embd=w.n_embd,
+                        block_size=T_sample, batch_size=1, grad_accum=1, variant=w.variant,
+                        init_std=w.init_std, beta1=w.beta1, beta2=w.beta2, eps=w.eps,
+                        weight_decay=w.weight_decay, grad_clip=w.grad_clip)
+    if state is None:
+        P = oracle.init_params(cfg, w.weight_seed)
+        state = (cfg, P, oracle.AdamState(), W.token_stream(w, n=1 << 16), 0)
+    cfg, P, S, stream, it = state
+    it += 1
+    t0 = time.perf_counter()
+    oracle.train_step(cfg, P, S, stream.astype(np.int64), w.data_seed, w.lr, it)
+    dt = time.perf_counter() - t0
+    return dt, T_sample, (cfg, P, S, stream, it)
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return int(max(n)) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def run_reference(args, w, rank):
+    if rank != 0:
+        return
+    T_sample = 256
+    state = None
+    for _ in range(args.warmup):
+        _, _, state = oracle_sample_step(w, T_sample, state)
+    tot, toks = 0.0, 0
+    for _ in range(args.steps):
+        dt, n, state = oracle_sample_step(w, T_sample, state)
+        tot += dt
+        toks += n
+    value = toks / tot
+    cores = blas_threads()
+    sample = (f"1 window x {T_sample} tokens per step at the full model dims (fp64 numpy oracle, "
+              f"fwd+bwd+clip+AdamW over all 124M parameters)")
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": 1000 * tot / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "impl": "reference",
+        "config": {"workload": w.name, "sample": sample},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args, w, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    from gpt_decoder_lm_b200 import binding as gb
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    gb.lib()
+    cfg = gb.make_config(w)
+    model = gb.Model(cfg, seed=w.weight_seed, device=dev)
+    stream_host = W.token_stream(w)
+    d_stream = torch.from_numpy(stream_host.view(np.int16)).to(dev)
+    data_seed = w.data_seed + 1000003 * rank
+    tok_step = w.tokens_per_step
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    st = 0
+
+    def lr_at(i):
+        return gb.lr_cosine(w.lr, i, 100, 5000)
+
+    # warm-up (untimed)
+    for _ in range(args.warmup):
+        st += 1
+        model.train_step(d_stream, data_seed, lr_at(st), st, sync=False)
+    torch.cuda.synchronize()
+    clocks = Clocks(local_rank) if rank == 0 else None
+    time.sleep(0.3)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    l0 = model.launch_count()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record()
+    for _ in range(args.steps):
+        st += 1
+        model.train_step(d_stream, data_seed, lr_at(st), st, sync=False)
+        flush.zero_()          # L2 flush between steps (256 MiB > 126 MB L2)
+    ev1.record()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    launches = model.launch_count() - l0
+    ms = ev0.elapsed_time(ev1)
+    ms_max = reduce_max(ms, dev)
+    clk = clocks.stop() if clocks else None
+    loss, norm = model.train_step(d_stream, data_seed, lr_at(st + 1), st + 1)
+    st += 1
+    value = world * args.steps * tok_step / (ms_max / 1000.0)
+
+    # per-kernel durations: instrumented pass of the same steps (events around every launch)
+    model.enable_timing(True)
+    for _ in range(args.steps):
+        st += 1
+        model.train_step(d_stream, data_seed, lr_at(st), st, sync=False)
+        flush.zero_()
+    torch.cuda.synchronize()
+    kt = model.kernel_times()
+    model.enable_timing(False)
+
+    # end to end through the host-buffer entry point (H2D of the batch + D2H of loss/norm each step)
+    B, T, ga = w.batch_size, w.block_size, w.grad_accum
+    rng = np.random.default_rng(7 + rank)
+    hb = []
+    for k in range(args.steps):
+        starts = rng.integers(0, len(stream_host) - T - 1, size=(ga, B))
+        rows = starts[..., None] + np.arange(T)
+        xi = torch.from_numpy(stream_host[rows].astype(np.int32)).pin_memory()
+        yi = torch.from_numpy(stream_host[rows + 1].astype(np.int32)).pin_memory()
+        hb.append((xi, yi))
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for xi, yi in hb:
+        st += 1
+        model.train_step_host(xi, yi, lr_at(st), st)
+    e1.record()
+    torch.cuda.synchronize()
+    e2e_ms = reduce_max(e0.elapsed_time(e1), dev)
+    e2e_value = world * args.steps * tok_step / (e2e_ms / 1000.0)
+
+    pk = peaks()
+    gemm_names = [k for k in kt if k.startswith("gemm")]
+    gemm_ms = sum(kt[k][0] for k in gemm_names)
+    gemm_n = sum(kt[k][1] for k in gemm_names)
+    top = max(kt.items(), key=lambda kv: kv[1][0]) if kt else ("", (0.0, 0))
+    gemm_flops = gemm_flops_per_step(w) * args.steps
+    achieved = gemm_flops / (gemm_ms / 1000.0) / 1e12 if gemm_ms > 0 else 0.0
+    roofline = {"bound": "tensor", "kernel": "gemm_tc (all dense contractions)", "achieved": achieved,
+                "peak": pk["bf16_sustained"], "unit": "TFLOP/s", "frac": achieved / pk["bf16_sustained"],
+                "traffic": None, "peak_source": pk["source"] + " sustained bf16",
+                "launches": gemm_n, "avg_launch_ms": gemm_ms / max(gemm_n, 1)}
+    step_ms = ms_max / args.steps
+    kern = {k: {"ms_per_step": v[0] / args.steps, "launches_per_step": v[1] / args.steps,
+                "share": v[0] / max(sum(x[0] for x in kt.values()), 1e-9)} for k, v in kt.items()}
+    fpt = flops_per_token(w)
+    mfu_nom = (value / world) * fpt / (NOMINAL_BF16_TFLOPS * 1e12)
+    mfu_meas = (value / world) * fpt / (pk["bf16"] * 1e12)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        dt, n, _ = oracle_sample_step(w, 1024)
+        cpu = {"value": n / dt, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+               "sample": "1 window x 1024 tokens (B=1) at the full GPT-2 124M dims, one oracle step "
+                         "(fp64 numpy fwd+bwd+clip+AdamW)"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": w.name, "vocab": w.vocab_size, "n_layer": w.n_layer, "n_head": w.n_head,
+                       "n_embd": w.n_embd, "seq_len": w.block_size, "micro_batch": w.batch_size,
+                       "grad_accum": w.grad_accum, "tokens_per_step_per_gpu": tok_step,
+                       "global_batch_tokens": tok_step * world, "parallelism": f"replicas x{world}",
+                       "l2": "256 MiB buffer zeroed between timed steps; step working set ~8 GB"},
+            "mfu": {"nominal_2250": mfu_nom, "measured_peak": mfu_meas, "flops_per_token": fpt},
+            "roofline": roofline,
+            "cpu_baseline": cpu,
+            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": 2 * ga * B * T * 4,
+                    "d2h_bytes_per_step": 16},
+            "gpu_launches": int(launches),
+            "clocks": clk,
+            "final_loss": loss, "final_grad_norm": norm,
+            "kernels": kern,
+        }
+        print(json.dumps(line), flush=True)
+    model.close()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default=W.GPT2_124M.name, choices=list(W.ALL))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    w = W.ALL[args.workload]
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    local_rank = int(os.environ.get("LOCAL_RANK", 0))
+    if args.impl == "reference":
+        run_reference(args, w, rank)
+        return
+    import torch
+    import torch.distributed as dist
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        run_ours(args, w, rank, world, local_rank)
+    finally:
+        if world > 1 and dist.is_initialized():
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

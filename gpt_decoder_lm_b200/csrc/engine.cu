@@ -197,7 +197,7 @@ gpt_status validate(const gpt_config* c, std::string* why) {
   if (c->token_dtype != GPT_TOK_I32 && c->token_dtype != GPT_TOK_U16) return bad("token_dtype");
   if (!(c->dropout >= 0.f && c->dropout < 1.f)) return bad("dropout must be in [0, 1)");
   if (!(c->beta1 >= 0.f && c->beta1 < 1.f && c->beta2 >= 0.f && c->beta2 < 1.f)) return bad("betas in [0, 1)");
-  if (!(c->eps > 0.f) || !(c->init_std >= 0.f)) return bad("eps > 0 and init_std >= 0 required");
+  if (!(c->eps > 0.f) || !(c->init_std >= 0.0)) return bad("eps > 0 and init_std >= 0 required");
   return GPT_OK;
 }
 
@@ -375,7 +375,7 @@ size_t carve(gpt_model& m, uint8_t* base) {
 // ---------------------------------------------------------------- host init
 uint64_t sm64(uint64_t x) { return splitmix64(x); }
 
-void init_tensor_host(const TensorRec& t, float std_, uint64_t seed, int index, float* out /* rows*cols */) {
+void init_tensor_host(const TensorRec& t, double std_, uint64_t seed, int index, float* out /* rows*cols */) {
   int64_t n = t.rows * t.cols;
   if (t.init == 1) {
     std::fill(out, out + n, 1.0f);
@@ -398,7 +398,7 @@ void init_tensor_host(const TensorRec& t, float std_, uint64_t seed, int index, 
         double u1 = ((double)(b1 >> 11) + 1.0) * (1.0 / 9007199254740992.0);
         double u2 = (double)(b2 >> 11) * (1.0 / 9007199254740992.0);
         double z = sqrt(-2.0 * log(u1)) * cos(2.0 * 3.14159265358979323846 * u2);
-        out[e] = (float)((double)std_ * z);
+        out[e] = (float)(std_ * z);
       }
     });
   }

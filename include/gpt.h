@@ -99,7 +99,6 @@ typedef struct gpt_config {
   int32_t precision;      /* GPT_PREC_FP32 (all fp32, SIMT) or GPT_PREC_BF16         */
   int32_t variant;        /* GPT_VARIANT_GPT2 or GPT_VARIANT_MICRO                   */
   int32_t token_dtype;    /* element type of the token stream in gpt_train_step      */
-  float init_std;         /* std of the Gaussian init of matrices and embeddings     */
   float dropout;          /* p in [0, 1); 0 disables every dropout site              */
   float beta1, beta2, eps;
   float weight_decay;     /* decoupled (AdamW); applied to 2-D tensors only unless
@@ -108,6 +107,9 @@ typedef struct gpt_config {
   int32_t decay_1d;
   int32_t reserved0;
   uint64_t dropout_seed;  /* key of the dropout counter hash                         */
+  double init_std;        /* std of the Gaussian init of matrices and embeddings
+                             (double: the init is computed in double precision and
+                             rounded to fp32 once)                                   */
 } gpt_config;
 
 typedef struct gpt_model gpt_model;
@@ -204,7 +206,9 @@ gpt_status gpt_tensor_info(gpt_model* m, int32_t i, const char** name, int64_t s
 gpt_status gpt_get_tensor(gpt_model* m, int32_t i, int32_t kind, float* h_out);
 gpt_status gpt_set_tensor(gpt_model* m, int32_t i, int32_t kind, const float* h_in);
 /* Logits of the last forward as fp32 [B*T, vocab_size] (pad columns
- * dropped), and their row argmax (ties -> lowest index) as int32 [B*T]. */
+ * dropped), and their row argmax (ties -> lowest index) as int32 [B*T].
+ * Valid between gpt_forward_loss and the next gpt_backward, which reuses the
+ * logits buffer for the logits' gradient. */
 gpt_status gpt_get_logits(gpt_model* m, float* h_out);
 gpt_status gpt_get_argmax(gpt_model* m, int32_t* h_out);
 /* Argmax of caller-supplied fp32 rows [rows, cols] held in device memory

@@ -125,7 +125,8 @@ def test_tc_split_k_accumulate(splits):
     run(TC, M, N, K, Ad, lda, 0, Bd, ldb, 0, 5, out=acc, ldo=N, split_k=splits, partial=partial)
     ref = acc0 + A @ B.T
     err = np.abs(acc.double().cpu().numpy() - ref).max() / np.abs(ref).max()
-    assert err < 2e-6, err
+    # fp32 accumulation over K = 4096 products: rounding grows like sqrt(K) * 2^-24
+    assert err < 1e-5, err
 
 
 def test_tc_matches_simt_bitwise_close():
