@@ -59,7 +59,7 @@ except Exception:  # pragma: no cover - scipy is in the image
 __all__ = [
     "Config", "TensorSpec", "tensor_specs", "param_count", "param_count_closed_form",
     "sm64", "init_tensor", "init_params", "batch_offsets", "gather_batch",
-    "dropout_keep", "forward", "backward", "loss_and_grads", "global_grad_norm",
+    "dropout_keep", "attention_fwd", "attention_bwd", "forward", "backward", "loss_and_grads", "global_grad_norm",
     "clip_adamw", "AdamState", "train_step", "lr_cosine", "lr_linear", "argmax_rows",
 ]
 
@@ -339,6 +339,42 @@ class DropCtx:
     counter: int
 
 
+def attention_fwd(q: np.ndarray, k: np.ndarray, v: np.ndarray, keep: Optional[np.ndarray] = None,
+                  p_drop: float = 0.0):
+    """Causal scaled dot-product attention of [B, H, T, hd] inputs (README /
+    microGPT "模型核心": scores q k^T / sqrt(head_dim), future keys masked,
+    softmax, weighted sum of V).  Dropout (``keep`` mask, [B, H, T, T]) acts
+    on the probabilities.  Returns (o, p, lse) with lse the natural-log
+    log-sum-exp of each row of scaled scores."""
+    T, hd = q.shape[-2], q.shape[-1]
+    s = (q @ k.transpose(0, 1, 3, 2)) / math.sqrt(hd)
+    causal = np.tril(np.ones((T, T), dtype=bool))
+    s = np.where(causal, s, -np.inf)
+    mx = s.max(axis=-1, keepdims=True)
+    e = np.exp(s - mx)
+    z = e.sum(axis=-1, keepdims=True)
+    pr = e / z
+    lse = (mx + np.log(z))[..., 0]
+    pd = pr * keep / (1.0 - p_drop) if keep is not None else pr
+    return pd @ v, pr, lse
+
+
+def attention_bwd(q, k, v, pr, do, keep: Optional[np.ndarray] = None, p_drop: float = 0.0):
+    """Gradients (dq, dk, dv) of attention_fwd: dV = P~^T dO, dP = dO V^T
+    (times the dropout mask), dS = P * (dP - rowsum(dP * P)),
+    dQ = dS K / sqrt(hd), dK = dS^T Q / sqrt(hd)."""
+    hd = q.shape[-1]
+    inv_keep = 1.0 / (1.0 - p_drop) if keep is not None else 1.0
+    pd = pr * keep * inv_keep if keep is not None else pr
+    dv = pd.transpose(0, 1, 3, 2) @ do
+    dpd = do @ v.transpose(0, 1, 3, 2)
+    dp = dpd * keep * inv_keep if keep is not None else dpd
+    ds = pr * (dp - (dp * pr).sum(axis=-1, keepdims=True))
+    dq = (ds @ k) / math.sqrt(hd)
+    dk = (ds.transpose(0, 1, 3, 2) @ q) / math.sqrt(hd)
+    return dq, dk, dv
+
+
 def forward(cfg: Config, P: Dict[str, np.ndarray], idx: np.ndarray, tgt: Optional[np.ndarray],
             drop: Optional[DropCtx] = None, keep_cache: bool = True):
     """Loss of one micro-batch (mean over its B*T positions) and the cache.
@@ -381,14 +417,9 @@ def forward(cfg: Config, P: Dict[str, np.ndarray], idx: np.ndarray, tgt: Optiona
         q = q.reshape(B, T, H, hd).transpose(0, 2, 1, 3)
         k = k.reshape(B, T, H, hd).transpose(0, 2, 1, 3)
         v = v.reshape(B, T, H, hd).transpose(0, 2, 1, 3)
-        s = (q @ k.transpose(0, 1, 3, 2)) / math.sqrt(hd)
-        causal = np.tril(np.ones((T, T), dtype=bool))
-        s = np.where(causal, s, -np.inf)
-        pr = np.exp(s - s.max(axis=-1, keepdims=True))
-        pr = pr / pr.sum(axis=-1, keepdims=True)
-        m1 = _mask(l, 1, pr.shape)
-        pd = pr * m1 * inv_keep if m1 is not None else pr
-        o = (pd @ v).transpose(0, 2, 1, 3).reshape(B, T, d)
+        m1 = _mask(l, 1, (B, H, T, T))
+        o, pr, _ = attention_fwd(q, k, v, m1, p_drop)
+        o = o.transpose(0, 2, 1, 3).reshape(B, T, d)
         y = o @ P[pre + "attn.c_proj.weight"].T
         if gpt2:
             y = y + P[pre + "attn.c_proj.bias"]
@@ -491,13 +522,7 @@ def backward(cfg: Config, P: Dict[str, np.ndarray], cache, loss_scale: float = 1
         G[pre + "attn.c_proj.weight"] += dy.reshape(M, d).T @ lc["o"].reshape(M, d)
         do = (dy @ P[pre + "attn.c_proj.weight"]).reshape(B, T, H, hd).transpose(0, 2, 1, 3)
         q, k, v, pr, m1 = lc["q"], lc["k"], lc["v"], lc["p"], lc["m1"]
-        pd = pr * m1 * inv_keep if m1 is not None else pr
-        dv = pd.transpose(0, 1, 3, 2) @ do
-        dpd = do @ v.transpose(0, 1, 3, 2)
-        dp = dpd * m1 * inv_keep if m1 is not None else dpd
-        ds = pr * (dp - (dp * pr).sum(axis=-1, keepdims=True))
-        dq = (ds @ k) / math.sqrt(hd)
-        dk = (ds.transpose(0, 1, 3, 2) @ q) / math.sqrt(hd)
+        dq, dk, dv = attention_bwd(q, k, v, pr, do, m1, p_drop)
         dqkv = np.concatenate([t.transpose(0, 2, 1, 3).reshape(B, T, d) for t in (dq, dk, dv)], axis=-1)
         if gpt2:
             G[pre + "attn.c_attn.bias"] += dqkv.reshape(M, 3 * d).sum(axis=0)

@@ -368,3 +368,35 @@ def test_resume_equals_uninterrupted():
 def test_argmax_ties_lowest_index():
     z = np.array([[1.0, 3.0, 3.0, 0.0], [5.0, 5.0, 5.0, 5.0]])
     assert list(oracle.argmax_rows(z)) == [1, 0]
+
+
+def test_attention_uniform_scores_is_causal_mean():
+    # q = 0 makes every allowed score equal: output i is the mean of v_0..v_i
+    rng = np.random.default_rng(3)
+    v = rng.standard_normal((2, 3, 7, 4))
+    k = rng.standard_normal((2, 3, 7, 4))
+    q = np.zeros_like(k)
+    o, p, lse = oracle.attention_fwd(q, k, v)
+    want = np.cumsum(v, axis=2) / np.arange(1, 8)[None, None, :, None]
+    np.testing.assert_allclose(o, want, atol=1e-14)
+    np.testing.assert_allclose(lse, np.log(np.arange(1, 8))[None, None, :].repeat(2, 0).repeat(3, 1), atol=1e-14)
+
+
+def test_attention_backward_finite_differences():
+    rng = np.random.default_rng(4)
+    q, k, v, w = (rng.standard_normal((1, 2, 5, 4)) for _ in range(4))
+    keep = rng.random((1, 2, 5, 5)) > 0.3
+    o, p, _ = oracle.attention_fwd(q, k, v, keep, 0.3)
+    dq, dk, dv = oracle.attention_bwd(q, k, v, p, w, keep, 0.3)
+    h = 1e-6
+    for x, g in ((q, dq), (k, dk), (v, dv)):
+        fd = np.zeros_like(x)
+        for i in np.ndindex(x.shape):
+            old = x[i]
+            x[i] = old + h
+            lp = (oracle.attention_fwd(q, k, v, keep, 0.3)[0] * w).sum()
+            x[i] = old - h
+            lm = (oracle.attention_fwd(q, k, v, keep, 0.3)[0] * w).sum()
+            x[i] = old
+            fd[i] = (lp - lm) / (2 * h)
+        assert rel_l2(g, fd) < 1e-7
