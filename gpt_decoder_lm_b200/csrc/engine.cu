@@ -344,7 +344,7 @@ size_t carve(gpt_model& m, uint8_t* base) {
   m.dres = F((size_t)M * d);
   m.dln = F((size_t)M * d);
   m.dsum = F((size_t)M * m.H);
-  m.part_blocks = (int)std::min<long>(M, 148 * 4);
+  m.part_blocks = (int)std::min<long>(M, 148 * 2);
   m.part = F((size_t)m.part_blocks * 3 * d);
   m.colsum_scr = F((size_t)64 * 4 * d);
   // split-K scratch: the largest dW partial set
@@ -531,10 +531,8 @@ gpt_status forward_t(gpt_model* m, bool fuse_ce_grad, float* loss_acc, float los
 }
 
 void add_bias_grads_from_norm(gpt_model* m, int64_t gain, int64_t beta, int64_t next_bias) {
-  Ctx& c = m->ctx;
-  if (gain >= 0) partial_reduce(c, m->part, m->part_blocks, 3, 0, m->d, m->G(gain));
-  if (beta >= 0) partial_reduce(c, m->part, m->part_blocks, 3, 1, m->d, m->G(beta));
-  if (next_bias >= 0) partial_reduce(c, m->part, m->part_blocks, 3, 2, m->d, m->G(next_bias));
+  partial_reduce3(m->ctx, m->part, m->part_blocks, m->d, gain >= 0 ? m->G(gain) : nullptr,
+                  beta >= 0 ? m->G(beta) : nullptr, next_bias >= 0 ? m->G(next_bias) : nullptr);
 }
 
 template <typename T>

@@ -315,6 +315,36 @@ void partial_reduce(Ctx& c, const float* part, int blocks, int slots, int slot, 
   k_partial_reduce<<<(d + 127) / 128, 128, 0, c.stream>>>(part, blocks, slots, slot, d, grad);
 }
 
+// grad_s[j] += sum_b part[b, s, j] for the three slots of the norm-backward
+// partials at once.  Block (32 columns x 8 row groups): row group y sums
+// blocks y, y+8, ...; the 8 group sums are then added in a fixed order.
+__global__ void k_partial_reduce3(const float* __restrict__ part, int blocks, int d, float* g0, float* g1, float* g2) {
+  __shared__ float sh[8][33];
+  int x = threadIdx.x, y = threadIdx.y;
+  int j = blockIdx.x * 32 + x;
+  int slot = blockIdx.y;
+  float* dst = slot == 0 ? g0 : (slot == 1 ? g1 : g2);
+  if (!dst) return;  // uniform per block
+  float s = 0.f;
+  if (j < d)
+    for (int b = y; b < blocks; b += 8) s += part[((long)b * 3 + slot) * d + j];
+  sh[y][x] = s;
+  __syncthreads();
+  if (y == 0 && j < d) {
+    float t = 0.f;
+#pragma unroll
+    for (int k = 0; k < 8; k++) t += sh[k][x];
+    dst[j] += t;
+  }
+}
+
+void partial_reduce3(Ctx& c, const float* part, int blocks, int d, float* g0, float* g1, float* g2) {
+  if (!g0 && !g1 && !g2) return;
+  LaunchScope s(c, "partial_reduce");
+  dim3 grid((d + 31) / 32, 3);
+  k_partial_reduce3<<<grid, dim3(32, 8), 0, c.stream>>>(part, blocks, d, g0, g1, g2);
+}
+
 // ============================================================================
 // column sums (bias gradients): chunk partials then a fixed-order reduce
 // ============================================================================
@@ -397,11 +427,94 @@ __global__ void k_ce(T* __restrict__ logits, const int32_t* __restrict__ tgt, in
   }
 }
 
+// Register-resident variant: the row is read from HBM once with 16-byte
+// loads (EPV elements per vector, up to 16 vectors per thread), max and
+// sum-exp come from registers, and the gradient is written once.
+template <typename T>
+__global__ void __launch_bounds__(512) k_ce_vec(T* __restrict__ logits, const int32_t* __restrict__ tgt, int V,
+                                                int Vp, float* __restrict__ lse_out, float* __restrict__ row_loss,
+                                                int want_grad, float scale) {
+  constexpr int EPV = 16 / sizeof(T);
+  constexpr int NV = 16;
+  __shared__ float red[16];
+  __shared__ float s_zt;
+  const long row = blockIdx.x;
+  T* z = logits + row * Vp;
+  const int nvec = Vp / EPV;
+  const int t = tgt[row];
+  if (threadIdx.x == 0) s_zt = to_f<T>(z[t]);
+  uint4 buf[NV];
+#pragma unroll
+  for (int k = 0; k < NV; k++) {
+    int vi = threadIdx.x + k * 512;
+    buf[k] = vi < nvec ? reinterpret_cast<const uint4*>(z)[vi] : make_uint4(0, 0, 0, 0);
+  }
+  auto elem = [&](const uint4& u, int e) -> float {
+    const T* p = reinterpret_cast<const T*>(&u);
+    return to_f<T>(p[e]);
+  };
+  float mx = -INFINITY;
+#pragma unroll
+  for (int k = 0; k < NV; k++) {
+    int vi = threadIdx.x + k * 512;
+#pragma unroll
+    for (int e = 0; e < EPV; e++)
+      if (vi < nvec && vi * EPV + e < V) mx = fmaxf(mx, elem(buf[k], e));
+  }
+  mx = warp_max(mx);
+  const int w = threadIdx.x >> 5;
+  if ((threadIdx.x & 31) == 0) red[w] = mx;
+  __syncthreads();
+  float M = red[0];
+#pragma unroll
+  for (int k = 1; k < 16; k++) M = fmaxf(M, red[k]);
+  __syncthreads();
+  float sum = 0.f;
+#pragma unroll
+  for (int k = 0; k < NV; k++) {
+    int vi = threadIdx.x + k * 512;
+#pragma unroll
+    for (int e = 0; e < EPV; e++)
+      if (vi < nvec && vi * EPV + e < V) sum += expf(elem(buf[k], e) - M);
+  }
+  sum = warp_sum(sum);
+  if ((threadIdx.x & 31) == 0) red[w] = sum;
+  __syncthreads();
+  float S = 0.f;
+#pragma unroll
+  for (int k = 0; k < 16; k++) S += red[k];
+  const float lse = M + logf(S);
+  if (threadIdx.x == 0) {
+    lse_out[row] = lse;
+    row_loss[row] = lse - s_zt;
+  }
+  if (!want_grad) return;
+#pragma unroll
+  for (int k = 0; k < NV; k++) {
+    int vi = threadIdx.x + k * 512;
+    if (vi >= nvec) continue;
+    uint4 outv;
+    T* o = reinterpret_cast<T*>(&outv);
+#pragma unroll
+    for (int e = 0; e < EPV; e++) {
+      int j = vi * EPV + e;
+      float g = 0.f;
+      if (j < V) g = (expf(elem(buf[k], e) - lse) - (j == t ? 1.f : 0.f)) * scale;
+      o[e] = from_f<T>(g);
+    }
+    reinterpret_cast<uint4*>(z)[vi] = outv;
+  }
+}
+
 template <typename T>
 void ce_fwd_bwd(Ctx& c, T* logits, const int32_t* tgt, long M, int V, int Vp, float* lse, float* row_loss,
                 bool want_grad, float scale) {
   LaunchScope s(c, want_grad ? "ce_fwd_bwd" : "ce_fwd");
-  k_ce<T><<<(unsigned)M, 512, 0, c.stream>>>(logits, tgt, V, Vp, lse, row_loss, want_grad ? 1 : 0, scale);
+  constexpr int EPV = 16 / sizeof(T);
+  if (Vp % EPV == 0 && Vp / EPV <= 16 * 512)
+    k_ce_vec<T><<<(unsigned)M, 512, 0, c.stream>>>(logits, tgt, V, Vp, lse, row_loss, want_grad ? 1 : 0, scale);
+  else
+    k_ce<T><<<(unsigned)M, 512, 0, c.stream>>>(logits, tgt, V, Vp, lse, row_loss, want_grad ? 1 : 0, scale);
 }
 template void ce_fwd_bwd<float>(Ctx&, float*, const int32_t*, long, int, int, float*, float*, bool, float);
 template void ce_fwd_bwd<bf16>(Ctx&, bf16*, const int32_t*, long, int, int, float*, float*, bool, float);
@@ -488,19 +601,45 @@ void embed_sort(Ctx& c, const int32_t* idx, long M, int32_t* sorted_tok, int32_t
 
 // dwte[v] += sum over the sorted positions of token v (in position order) of
 // drop0(dres[pos]); one block per sorted slot, active only at segment starts.
-__global__ void k_embed_bwd_wte(const float* __restrict__ dres, const int32_t* __restrict__ stok,
-                                const int32_t* __restrict__ spos, int M, int d, DropKey drop,
-                                float* __restrict__ dwte) {
-  int i = blockIdx.x;
-  int tok = stok[i];
-  if (i > 0 && stok[i - 1] == tok) return;
-  for (int c = threadIdx.x; c < d; c += blockDim.x) {
-    float acc = 0.f;
-    for (int j = i; j < M && stok[j] == tok; j++) {
+// Warp w of the 8 sums the segment's rows w, w+8, ... (float4 columns per
+// lane); the 8 warp sums are added in warp order through shared memory.
+__global__ void __launch_bounds__(256) k_embed_bwd_wte(const float* __restrict__ dres,
+                                                       const int32_t* __restrict__ stok,
+                                                       const int32_t* __restrict__ spos, int M, int d, DropKey drop,
+                                                       float* __restrict__ dwte) {
+  extern __shared__ float wsum[];  // [8][d]
+  const int i = blockIdx.x;
+  const int tok = stok[i];
+  if (i > 0 && stok[i - 1] == tok) return;  // uniform per block
+  int end = i + 1;
+  while (end < M && stok[end] == tok) end++;
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int d4 = d >> 2;
+  for (int c4 = lane; c4 < d4; c4 += 32) {
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int j = i + w; j < end; j += 8) {
       long p = spos[j];
-      acc += dres[p * d + c] * drop_mul(drop, (uint64_t)p * d + c);
+      float4 v = reinterpret_cast<const float4*>(dres + p * d)[c4];
+      if (drop.active) {
+        uint64_t e = (uint64_t)p * d + 4 * c4;
+        v.x *= drop_mul(drop, e);
+        v.y *= drop_mul(drop, e + 1);
+        v.z *= drop_mul(drop, e + 2);
+        v.w *= drop_mul(drop, e + 3);
+      }
+      acc.x += v.x;
+      acc.y += v.y;
+      acc.z += v.z;
+      acc.w += v.w;
     }
-    dwte[(long)tok * d + c] += acc;
+    reinterpret_cast<float4*>(wsum + w * d)[c4] = acc;
+  }
+  __syncthreads();
+  for (int c = threadIdx.x; c < d; c += blockDim.x) {
+    float s = 0.f;
+#pragma unroll
+    for (int k = 0; k < 8; k++) s += wsum[k * d + c];
+    dwte[(long)tok * d + c] += s;
   }
 }
 
@@ -522,8 +661,13 @@ void embed_bwd(Ctx& c, const float* dres, const int32_t* sorted_tok, const int32
                int Bn, int d, DropKey drop, float* dwte, float* dwpe) {
   {
     LaunchScope s(c, "embed_bwd_wte");
-    int th = d >= 256 ? 256 : ((d + 31) / 32) * 32;
-    k_embed_bwd_wte<<<(unsigned)M, th, 0, c.stream>>>(dres, sorted_tok, sorted_pos, (int)M, d, drop, dwte);
+    size_t smem = (size_t)8 * d * sizeof(float);
+    static bool attr = false;
+    if (!attr) {
+      cudaFuncSetAttribute(k_embed_bwd_wte, cudaFuncAttributeMaxDynamicSharedMemorySize, 8 * 2048 * 4);
+      attr = true;
+    }
+    k_embed_bwd_wte<<<(unsigned)M, 256, smem, c.stream>>>(dres, sorted_tok, sorted_pos, (int)M, d, drop, dwte);
   }
   {
     LaunchScope s(c, "embed_bwd_wpe");
@@ -588,36 +732,57 @@ __global__ void k_adamw(AdamArgs a, uint32_t* flags) {
     }
   }
   __syncthreads();
-  float coef = s_coef;
-  int ok = s_ok;
-  float om1 = 1.f - a.beta1, om2 = 1.f - a.beta2;
-  float decay = 1.f - a.lr * a.wd;
-  long n4 = a.n / 4;
-  for (long i = (long)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += (long)gridDim.x * blockDim.x) {
-    float4 g4 = reinterpret_cast<float4*>(a.g)[i];
-    reinterpret_cast<float4*>(a.g)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (!ok) continue;
-    float4 w4 = reinterpret_cast<float4*>(a.w)[i];
-    float4 m4 = reinterpret_cast<float4*>(a.m)[i];
-    float4 v4 = reinterpret_cast<float4*>(a.v)[i];
-    float* w = &w4.x;
-    float* m = &m4.x;
-    float* v = &v4.x;
-    const float* g = &g4.x;
-    bool dec = (i * 4) < a.n_decay;
+  const float coef = s_coef;
+  const int ok = s_ok;
+  const float om1 = 1.f - a.beta1, om2 = 1.f - a.beta2;
+  const float decay = 1.f - a.lr * a.wd;
+  const long n4 = a.n / 4;
+  float4* __restrict__ W4 = reinterpret_cast<float4*>(a.w);
+  float4* __restrict__ G4 = reinterpret_cast<float4*>(a.g);
+  float4* __restrict__ M4 = reinterpret_cast<float4*>(a.m);
+  float4* __restrict__ V4 = reinterpret_cast<float4*>(a.v);
+  bf16* __restrict__ WB = a.wb;
+  const long stride = (long)gridDim.x * blockDim.x;
+  for (long i0 = (long)blockIdx.x * blockDim.x + threadIdx.x; i0 < n4; i0 += 2 * stride) {
+    // two independent float4 per iteration: more loads in flight
+    float4 g4[2], w4[2], m4[2], v4[2];
+    bool in[2] = {true, i0 + stride < n4};
 #pragma unroll
-    for (int k = 0; k < 4; k++) {
-      float gg = g[k] * coef;
-      float ww = dec ? w[k] * decay : w[k];
-      m[k] = a.beta1 * m[k] + om1 * gg;
-      v[k] = a.beta2 * v[k] + om2 * gg * gg;
-      ww -= a.lr * (m[k] / a.bc1) / (sqrtf(v[k] / a.bc2) + a.eps);
-      w[k] = ww;
+    for (int u = 0; u < 2; u++) {
+      long i = i0 + u * stride;
+      if (!in[u]) continue;
+      g4[u] = G4[i];
+      if (ok) {
+        w4[u] = W4[i];
+        m4[u] = M4[i];
+        v4[u] = V4[i];
+      }
     }
-    reinterpret_cast<float4*>(a.w)[i] = w4;
-    reinterpret_cast<float4*>(a.m)[i] = m4;
-    reinterpret_cast<float4*>(a.v)[i] = v4;
-    if (a.wb) store4<bf16>(a.wb + 4 * i, w4);
+#pragma unroll
+    for (int u = 0; u < 2; u++) {
+      long i = i0 + u * stride;
+      if (!in[u]) continue;
+      G4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (!ok) continue;
+      float* w = &w4[u].x;
+      float* m = &m4[u].x;
+      float* v = &v4[u].x;
+      const float* g = &g4[u].x;
+      const bool dec = (i * 4) < a.n_decay;
+#pragma unroll
+      for (int k = 0; k < 4; k++) {
+        float gg = g[k] * coef;
+        float ww = dec ? w[k] * decay : w[k];
+        m[k] = a.beta1 * m[k] + om1 * gg;
+        v[k] = a.beta2 * v[k] + om2 * gg * gg;
+        ww -= a.lr * (m[k] / a.bc1) / (sqrtf(v[k] / a.bc2) + a.eps);
+        w[k] = ww;
+      }
+      W4[i] = w4[u];
+      M4[i] = m4[u];
+      V4[i] = v4[u];
+      if (WB) store4<bf16>(WB + 4 * i, w4[u]);
+    }
   }
 }
 

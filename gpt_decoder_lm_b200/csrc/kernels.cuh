@@ -129,6 +129,8 @@ template <typename T> void norm_bwd(Ctx& c, const NormBwd& p);
 int norm_bwd_blocks(Ctx& c, long rows);
 // grad[j] += sum_b part[b, slot, j] for the given slot
 void partial_reduce(Ctx& c, const float* part, int blocks, int slots, int slot, int d, float* grad);
+// the three slots of part[blocks, 3, d] into g0, g1, g2 (each nullable), one launch
+void partial_reduce3(Ctx& c, const float* part, int blocks, int d, float* g0, float* g1, float* g2);
 
 // column sums of an operand-typed [rows, N] matrix into grad (+=), deterministic
 template <typename T> void colsum_acc(Ctx& c, const T* x, long rows, int N, float* scratch, float* grad);
