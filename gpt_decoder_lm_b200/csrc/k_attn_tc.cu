@@ -9,11 +9,13 @@
 // dK/dV and dQ come from two kernels (each output tile owned by one CTA, no
 // atomics), so the result is deterministic.
 //
-// Every kernel: warp 0 issues TMA loads of 128-row bf16 tiles (128-byte
-// swizzle) from the [B*T, 3, H, 64] qkv activations, warp 1 owns TMEM and
-// issues tcgen05.mma, warps 2..5 (one TMEM lane / tile row per thread) do the
-// softmax arithmetic, write bf16 probability tiles to shared memory as the
-// A operand of the next MMA, and run the epilogue.
+// Every kernel: warp 0 issues TMA loads of bf16 tiles (128-byte swizzle) from
+// the [B*T, 3, H, 64] qkv activations, warp 1 owns TMEM and issues
+// tcgen05.mma, warps 2..5 (one TMEM lane / tile row per thread) do the softmax
+// arithmetic, write bf16 probability tiles to shared memory as the A operand
+// of the next MMA, and run the epilogue.  Each kernel keeps its TMEM at 256
+// columns and its shared memory under 113 KB so that two CTAs share an SM:
+// one CTA's softmax overlaps the other's MMAs.
 #include <cudaTypedefs.h>
 
 #include <mutex>
@@ -26,13 +28,13 @@ namespace {
 
 using namespace sm100;
 
-constexpr int TILE = 16384;                 // 128 rows x 64 bf16, 128-byte swizzle
+constexpr int TILE = 16384;  // 128 rows x 64 bf16 (128 bytes), 128-byte swizzle
+constexpr int HTILE = 8192;  // 64 rows x 64 bf16
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr float LN2 = 0.6931471805599453f;
 
 struct AttnTcArgs {
   int B, T, H;
-  const bf16* o;      // fwd output / bwd input O
   bf16* o_out;
   float* lse;         // [B, H, T] natural log
   const float* dsum;  // [B, H, T]
@@ -47,11 +49,17 @@ __device__ __forceinline__ uint32_t pack2(float a, float b) {
   __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
   return *reinterpret_cast<uint32_t*>(&v);
 }
+// 2^x with the SFU instruction (relative error ~2^-22; 2^-inf = 0)
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
 
-// Row r, 32-column chunk c (0..3) of a 128 x 128 K-major bf16 operand tile
-// stored as two 64-wide K-blocks of 128 rows x 128 bytes (128-byte swizzle).
-__device__ __forceinline__ void store_chunk32(uint32_t tile, int r, int c, const uint32_t (&pk)[16]) {
-  uint32_t rowbase = tile + (c >> 1) * TILE + r * 128;
+// Row r, 32-column chunk c of a K-major bf16 operand tile whose K extent is
+// split in 64-wide K-blocks of kb_bytes each (128 rows x 128 bytes, or 64).
+__device__ __forceinline__ void store_chunk32(uint32_t tile, int kb_bytes, int r, int c, const uint32_t (&pk)[16]) {
+  uint32_t rowbase = tile + (c >> 1) * kb_bytes + r * 128;
 #pragma unroll
   for (int q = 0; q < 4; q++) {
     int chunk = (c & 1) * 4 + q;
@@ -59,17 +67,21 @@ __device__ __forceinline__ void store_chunk32(uint32_t tile, int r, int c, const
   }
 }
 
-// A operand descriptor of K-step kk (16 elements) of such a 128-wide tile
-__device__ __forceinline__ uint64_t desc_k128(uint32_t tile, int kk) {
-  return desc_sw128(tile + (kk >> 2) * TILE + (kk & 3) * 32, 16, 1024);
+// K-major operand: K-step kk (16 elements) of a tile with 64-wide K-blocks
+__device__ __forceinline__ uint64_t desc_k(uint32_t tile, int kb_bytes, int kk) {
+  return desc_sw128(tile + (kk >> 2) * kb_bytes + (kk & 3) * 32, 16, 1024);
 }
-// K-major 64-wide tile (Q, K, V, dO as [rows, hd]), K-step kk (0..3)
-__device__ __forceinline__ uint64_t desc_k64(uint32_t tile, int kk) { return desc_sw128(tile + kk * 32, 16, 1024); }
-// the same [rows, 64] tile read MN-major (N = the 64 columns, K = rows), K-step kk (0..7)
+// a [rows, 64] tile read MN-major (N = the 64 columns, K = rows), K-step kk
 __device__ __forceinline__ uint64_t desc_mn64(uint32_t tile, int kk) { return desc_sw128(tile + kk * 2048, TILE, 1024); }
 
+__device__ __forceinline__ void ld64(uint32_t taddr, uint32_t (&a)[32], uint32_t (&b)[32]) {
+  tmem_ld_32x32b_x32(taddr, a);
+  tmem_ld_32x32b_x32(taddr + 32, b);
+  tmem_ld_wait();
+}
+
 // ============================================================================
-// forward
+// forward: one CTA per (128-query block, b, h), 128-key blocks
 // smem: Q | K[2] | V[2] | P (2 K-blocks) | barriers   (112 KB + 128 B)
 // TMEM: S cols [0,128), PV cols [128,192)  (256 allocated)
 // ============================================================================
@@ -103,7 +115,7 @@ __global__ void __launch_bounds__(192, 2) k_attn_fwd_tc(const __grid_constant__ 
     mbar_init(kv_empty0, 1);
     mbar_init(kv_empty0 + 8, 1);
     mbar_init(s_full, 1);
-    mbar_init(p_full, 128);
+    mbar_init(p_full, 4);
     mbar_init(pv_full, 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -141,13 +153,13 @@ __global__ void __launch_bounds__(192, 2) k_attn_fwd_tc(const __grid_constant__ 
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 4; kk++)
-          mma_bf16_ss(tmem, desc_k64(sb + F_Q, kk), desc_k64(sb + F_K + s * TILE, kk), id_s, kk > 0);
+          mma_bf16_ss(tmem, desc_k(sb + F_Q, TILE, kk), desc_k(sb + F_K + s * TILE, TILE, kk), id_s, kk > 0);
         mma_commit(s_full);
         if (!(ok = mbar_wait(p_full, j & 1, abort_flag, a.flags))) break;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 8; kk++)
-          mma_bf16_ss(tmem + 128, desc_k128(sb + F_P, kk), desc_mn64(sb + F_V + s * TILE, kk), id_pv, kk > 0);
+          mma_bf16_ss(tmem + 128, desc_k(sb + F_P, TILE, kk), desc_mn64(sb + F_V + s * TILE, kk), id_pv, kk > 0);
         mma_commit(pv_full);
         mma_commit(kv_empty0 + 8 * s);
       }
@@ -157,6 +169,7 @@ __global__ void __launch_bounds__(192, 2) k_attn_fwd_tc(const __grid_constant__ 
     const int r = quad * 32 + lane;
     const int qi = qb * 128 + r;
     const uint32_t trow = tmem + ((uint32_t)(quad * 32) << 16);
+    const float sl2 = a.scale_log2;
     float m = -INFINITY, l = 0.f;
     float o[64];
 #pragma unroll
@@ -167,55 +180,81 @@ __global__ void __launch_bounds__(192, 2) k_attn_fwd_tc(const __grid_constant__ 
       if (!(ok = mbar_wait(s_full, j & 1, abort_flag, a.flags))) break;
       tc_fence_after();
       const bool diag = (j == qb);
-      float mx = -INFINITY;
+      const int key0 = j * 128;
+      // pass 1: row maximum of the raw scores (scale > 0 commutes with max)
+      float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
+#pragma unroll 1
+      for (int c = 0; c < 4; c += 2) {
+        uint32_t v0[32], v1[32];
+        ld64(trow + c * 32, v0, v1);
+        if (!diag) {
 #pragma unroll
-      for (int c = 0; c < 4; c++) {
-        uint32_t v[32];
-        tmem_ld_32x32b_x32(trow + c * 32, v);
-        tmem_ld_wait();
+          for (int i = 0; i < 32; i += 2) {
+            mx0 = fmaxf(mx0, __uint_as_float(v0[i]));
+            mx1 = fmaxf(mx1, __uint_as_float(v0[i + 1]));
+            mx2 = fmaxf(mx2, __uint_as_float(v1[i]));
+            mx3 = fmaxf(mx3, __uint_as_float(v1[i + 1]));
+          }
+        } else {
 #pragma unroll
-        for (int i = 0; i < 32; i++) {
-          int key = j * 128 + c * 32 + i;
-          float s = __uint_as_float(v[i]) * a.scale_log2;
-          if (!(diag && key > qi)) mx = fmaxf(mx, s);
+          for (int i = 0; i < 32; i++) {
+            if (key0 + c * 32 + i <= qi) mx0 = fmaxf(mx0, __uint_as_float(v0[i]));
+            if (key0 + c * 32 + 32 + i <= qi) mx1 = fmaxf(mx1, __uint_as_float(v1[i]));
+          }
         }
       }
-      const float mn = fmaxf(m, mx);
-      const float alpha = exp2f(m - mn);
-      float ls = 0.f;
-#pragma unroll
-      for (int c = 0; c < 4; c++) {
-        uint32_t v[32];
-        tmem_ld_32x32b_x32(trow + c * 32, v);
-        tmem_ld_wait();
-        uint32_t pk[16];
+      const float mn = fmaxf(m, fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2);
+      const float alpha = ex2(m - mn);
+      float ls0 = 0.f, ls1 = 0.f;
+      // pass 2: probabilities -> bf16 A operand of P V
+#pragma unroll 1
+      for (int c = 0; c < 4; c += 2) {
+        uint32_t v0[32], v1[32];
+        ld64(trow + c * 32, v0, v1);
+        uint32_t pk0[16], pk1[16];
 #pragma unroll
         for (int i = 0; i < 32; i += 2) {
-          int key = j * 128 + c * 32 + i;
-          float p0 = (diag && key > qi) ? 0.f : exp2f(__uint_as_float(v[i]) * a.scale_log2 - mn);
-          float p1 = (diag && key + 1 > qi) ? 0.f : exp2f(__uint_as_float(v[i + 1]) * a.scale_log2 - mn);
-          ls += p0 + p1;
-          if (a.drop.active) {
-            p0 *= drop_mul(a.drop, ebase + key);
-            p1 *= drop_mul(a.drop, ebase + key + 1);
+          float p0 = ex2(fmaf(__uint_as_float(v0[i]), sl2, -mn));
+          float p1 = ex2(fmaf(__uint_as_float(v0[i + 1]), sl2, -mn));
+          float p2 = ex2(fmaf(__uint_as_float(v1[i]), sl2, -mn));
+          float p3 = ex2(fmaf(__uint_as_float(v1[i + 1]), sl2, -mn));
+          if (diag) {
+            int k = key0 + c * 32 + i;
+            if (k > qi) p0 = 0.f;
+            if (k + 1 > qi) p1 = 0.f;
+            if (k + 32 > qi) p2 = 0.f;
+            if (k + 33 > qi) p3 = 0.f;
           }
-          pk[i >> 1] = pack2(p0, p1);
+          ls0 += p0 + p1;
+          ls1 += p2 + p3;
+          if (a.drop.active) {
+            uint64_t e = ebase + key0 + c * 32 + i;
+            p0 *= drop_mul(a.drop, e);
+            p1 *= drop_mul(a.drop, e + 1);
+            p2 *= drop_mul(a.drop, e + 32);
+            p3 *= drop_mul(a.drop, e + 33);
+          }
+          pk0[i >> 1] = pack2(p0, p1);
+          pk1[i >> 1] = pack2(p2, p3);
         }
-        store_chunk32(sb + F_P, r, c, pk);
+        store_chunk32(sb + F_P, TILE, r, c, pk0);
+        store_chunk32(sb + F_P, TILE, r, c + 1, pk1);
       }
-      l = l * alpha + ls;
+      l = l * alpha + (ls0 + ls1);
       fence_proxy_async_smem();
       tc_fence_before();
-      mbar_arrive(p_full);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(p_full);  // one arrival per math warp
       if (!(ok = mbar_wait(pv_full, j & 1, abort_flag, a.flags))) break;
       tc_fence_after();
+      {
+        uint32_t v0[32], v1[32];
+        ld64(trow + 128, v0, v1);
 #pragma unroll
-      for (int c = 0; c < 2; c++) {
-        uint32_t v[32];
-        tmem_ld_32x32b_x32(trow + 128 + c * 32, v);
-        tmem_ld_wait();
-#pragma unroll
-        for (int i = 0; i < 32; i++) o[c * 32 + i] = o[c * 32 + i] * alpha + __uint_as_float(v[i]);
+        for (int i = 0; i < 32; i++) {
+          o[i] = fmaf(o[i], alpha, __uint_as_float(v0[i]));
+          o[32 + i] = fmaf(o[32 + i], alpha, __uint_as_float(v1[i]));
+        }
       }
       m = mn;
     }
@@ -236,19 +275,20 @@ __global__ void __launch_bounds__(192, 2) k_attn_fwd_tc(const __grid_constant__ 
 }
 
 // ============================================================================
-// backward, dK and dV: one CTA per (128-key block, b, h), walking the query
-// blocks i >= key block.  Keys are the MMA rows:
-//   S^T = K Q^T, dP^T = V dO^T  ->  P^T, dS^T (bf16, smem)
+// backward, dK and dV: one CTA per (128-key block, b, h), walking 64-query
+// blocks from the key block on.  Keys are the MMA rows:
+//   S^T = K Q^T, dP^T = V dO^T  ->  P~^T, dS^T (bf16, smem)
 //   dV += P~^T dO,  dK += dS^T Q
-// smem: K | V | Q[2] | dO[2] | P^T (2 blk) | dS^T (2 blk) | lse,D [2][128] | barriers
-// TMEM: S^T [0,128), dP^T [128,256), dV [256,320), dK [320,384)  (512 allocated)
+// smem: K | V | (Q, dO)[2 stages] | P^T | dS^T | (lse, D)[2] | barriers (~97 KB)
+// TMEM: S^T [0,64), dP^T [64,128), dV [128,192), dK [192,256)
 // ============================================================================
-constexpr int K_K = 0, K_V = TILE, K_Q = 2 * TILE, K_DO = 4 * TILE, K_P = 6 * TILE, K_DS = 8 * TILE,
-              K_LD = 10 * TILE, K_BAR = K_LD + 2 * 2 * 128 * 4;
+constexpr int K_K = 0, K_V = TILE, K_ST = 2 * TILE, K_P = 4 * TILE, K_DS = 5 * TILE, K_LD = 6 * TILE,
+              K_BAR = K_LD + 1024;
 constexpr int K_SMEM = K_BAR + 128;
 
-__global__ void __launch_bounds__(192, 1) k_attn_bwd_kv_tc(const __grid_constant__ CUtensorMap tq,
-                                                           const __grid_constant__ CUtensorMap tdo, AttnTcArgs a) {
+__global__ void __launch_bounds__(192, 2) k_attn_bwd_kv_tc(const __grid_constant__ CUtensorMap tkv,
+                                                           const __grid_constant__ CUtensorMap tq64,
+                                                           const __grid_constant__ CUtensorMap tdo64, AttnTcArgs a) {
   extern __shared__ __align__(1024) uint8_t smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (smem_u32(smem) & 1023) {
@@ -260,14 +300,15 @@ __global__ void __launch_bounds__(192, 1) k_attn_bwd_kv_tc(const __grid_constant
   uint32_t sdp_full = smem_u32(bars + 5), pds_full = smem_u32(bars + 6), acc_full = smem_u32(bars + 7);
   uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tslot + 1);
-  float* sld = reinterpret_cast<float*>(smem + K_LD);  // [2][lse2 128 | D 128]
+  const float* sld = reinterpret_cast<const float*>(smem + K_LD);  // [2][lse 64 | D 64]
   const uint32_t sb = smem_u32(smem);
 
-  const int nqb = a.T / 128;
+  const int nq64 = a.T / 64;
   const int kb = (int)blockIdx.x;  // key block 0 has the most query blocks: first
   const int bh = blockIdx.y, b = bh / a.H, h = bh % a.H;
   const int row0 = b * a.T;
-  const int nit = nqb - kb;
+  const int i0 = 2 * kb;
+  const int nit = nq64 - i0;
 
   if (threadIdx.x == 0) {
     mbar_init(kv_full, 1);
@@ -276,15 +317,16 @@ __global__ void __launch_bounds__(192, 1) k_attn_bwd_kv_tc(const __grid_constant
     mbar_init(st_empty0, 1);
     mbar_init(st_empty0 + 8, 1);
     mbar_init(sdp_full, 1);
-    mbar_init(pds_full, 128);
+    mbar_init(pds_full, 4);
     mbar_init(acc_full, 1);
     *abort_flag = 0;
     fence_barrier_init();
-    prefetch_tmap(&tq);
-    prefetch_tmap(&tdo);
+    prefetch_tmap(&tkv);
+    prefetch_tmap(&tq64);
+    prefetch_tmap(&tdo64);
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(tslot), 512);
+    tmem_alloc(smem_u32(tslot), 256);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -295,42 +337,44 @@ __global__ void __launch_bounds__(192, 1) k_attn_bwd_kv_tc(const __grid_constant
   if (warp == 0) {
     if (lane == 0) {
       mbar_expect_tx(kv_full, 2 * TILE);
-      tma_load_3d(sb + K_K, &tq, kv_full, 0, a.H + h, row0 + kb * 128);
-      tma_load_3d(sb + K_V, &tq, kv_full, 0, 2 * a.H + h, row0 + kb * 128);
+      tma_load_3d(sb + K_K, &tkv, kv_full, 0, a.H + h, row0 + kb * 128);
+      tma_load_3d(sb + K_V, &tkv, kv_full, 0, 2 * a.H + h, row0 + kb * 128);
       for (int it = 0; it < nit; it++) {
-        int i = kb + it, s = it & 1;
+        int i = i0 + it, s = it & 1;
+        uint32_t fb = st_full0 + 8 * s;
         if (!mbar_wait(st_empty0 + 8 * s, ((it >> 1) & 1) ^ 1, abort_flag, a.flags)) break;
-        mbar_expect_tx(st_full0 + 8 * s, 2 * TILE + 1024);
-        tma_load_3d(sb + K_Q + s * TILE, &tq, st_full0 + 8 * s, 0, h, row0 + i * 128);
-        tma_load_3d(sb + K_DO + s * TILE, &tdo, st_full0 + 8 * s, 0, h, row0 + i * 128);
-        bulk_load(sb + K_LD + s * 1024, a.lse + (size_t)bh * a.T + i * 128, 512, st_full0 + 8 * s);
-        bulk_load(sb + K_LD + s * 1024 + 512, a.dsum + (size_t)bh * a.T + i * 128, 512, st_full0 + 8 * s);
+        mbar_expect_tx(fb, 2 * HTILE + 512);
+        tma_load_3d(sb + K_ST + s * TILE, &tq64, fb, 0, h, row0 + i * 64);
+        tma_load_3d(sb + K_ST + s * TILE + HTILE, &tdo64, fb, 0, h, row0 + i * 64);
+        bulk_load(sb + K_LD + s * 512, a.lse + (size_t)bh * a.T + i * 64, 256, fb);
+        bulk_load(sb + K_LD + s * 512 + 256, a.dsum + (size_t)bh * a.T + i * 64, 256, fb);
       }
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      constexpr uint32_t id_s = idesc_bf16_f32(128, 128, false, false);
+      constexpr uint32_t id_s = idesc_bf16_f32(128, 64, false, false);
       constexpr uint32_t id_acc = idesc_bf16_f32(128, 64, false, true);
       bool ok = mbar_wait(kv_full, 0, abort_flag, a.flags);
       for (int it = 0; it < nit && ok; it++) {
         int s = it & 1;
         if (!(ok = mbar_wait(st_full0 + 8 * s, (it >> 1) & 1, abort_flag, a.flags))) break;
         tc_fence_after();
-        uint32_t q = sb + K_Q + s * TILE, dO = sb + K_DO + s * TILE;
-#pragma unroll
-        for (int kk = 0; kk < 4; kk++) mma_bf16_ss(tmem, desc_k64(sb + K_K, kk), desc_k64(q, kk), id_s, kk > 0);
+        uint32_t q = sb + K_ST + s * TILE, dO = q + HTILE;
 #pragma unroll
         for (int kk = 0; kk < 4; kk++)
-          mma_bf16_ss(tmem + 128, desc_k64(sb + K_V, kk), desc_k64(dO, kk), id_s, kk > 0);
+          mma_bf16_ss(tmem, desc_k(sb + K_K, TILE, kk), desc_k(q, HTILE, kk), id_s, kk > 0);
+#pragma unroll
+        for (int kk = 0; kk < 4; kk++)
+          mma_bf16_ss(tmem + 64, desc_k(sb + K_V, TILE, kk), desc_k(dO, HTILE, kk), id_s, kk > 0);
         mma_commit(sdp_full);
         if (!(ok = mbar_wait(pds_full, it & 1, abort_flag, a.flags))) break;
         tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < 8; kk++)
-          mma_bf16_ss(tmem + 256, desc_k128(sb + K_P, kk), desc_mn64(dO, kk), id_acc, (it > 0 || kk > 0));
+        for (int kk = 0; kk < 4; kk++)
+          mma_bf16_ss(tmem + 128, desc_k(sb + K_P, TILE, kk), desc_mn64(dO, kk), id_acc, (it > 0 || kk > 0));
 #pragma unroll
-        for (int kk = 0; kk < 8; kk++)
-          mma_bf16_ss(tmem + 320, desc_k128(sb + K_DS, kk), desc_mn64(q, kk), id_acc, (it > 0 || kk > 0));
+        for (int kk = 0; kk < 4; kk++)
+          mma_bf16_ss(tmem + 192, desc_k(sb + K_DS, TILE, kk), desc_mn64(q, kk), id_acc, (it > 0 || kk > 0));
         mma_commit(st_empty0 + 8 * s);
       }
       mma_commit(acc_full);
@@ -340,42 +384,56 @@ __global__ void __launch_bounds__(192, 1) k_attn_bwd_kv_tc(const __grid_constant
     const int r = quad * 32 + lane;
     const int kj = kb * 128 + r;
     const uint32_t trow = tmem + ((uint32_t)(quad * 32) << 16);
+    const float sl2 = a.scale_log2;
     bool ok = true;
     for (int it = 0; it < nit; it++) {
-      const int i = kb + it;
-      const float* ld = sld + (it & 1) * 256;  // [lse 128 | D 128] of query block i (bulk-copied)
+      const int i = i0 + it;
+      const int q0 = i * 64;
+      const float* ld = sld + (it & 1) * 128;  // lse[64] | D[64] of this query block
       if (!(ok = mbar_wait(st_full0 + 8 * (it & 1), (it >> 1) & 1, abort_flag, a.flags))) break;
       if (!(ok = mbar_wait(sdp_full, it & 1, abort_flag, a.flags))) break;
       tc_fence_after();
-      const bool diag = (it == 0);
+      const bool diag = q0 < kb * 128 + 128;  // the block straddles this CTA's keys
+      uint32_t s0[32], s1[32], d0[32], d1[32];
+      tmem_ld_32x32b_x32(trow, s0);
+      tmem_ld_32x32b_x32(trow + 32, s1);
+      tmem_ld_32x32b_x32(trow + 64, d0);
+      tmem_ld_32x32b_x32(trow + 96, d1);
+      tmem_ld_wait();
+      uint32_t pp0[16], pp1[16], pd0[16], pd1[16];
 #pragma unroll
-      for (int c = 0; c < 4; c++) {
-        uint32_t sv[32], dv[32];
-        tmem_ld_32x32b_x32(trow + c * 32, sv);
-        tmem_ld_32x32b_x32(trow + 128 + c * 32, dv);
-        tmem_ld_wait();
-        uint32_t pp[16], pd[16];
+      for (int e = 0; e < 32; e += 2) {
+        float pv[4], dsv[4];
 #pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          float pv[2], dsv[2];
-#pragma unroll
-          for (int u = 0; u < 2; u++) {
-            int col = c * 32 + e + u;
-            int qi = i * 128 + col;
-            float p = (diag && kj > qi) ? 0.f : exp2f(__uint_as_float(sv[e + u]) * a.scale_log2 - ld[col] * LOG2E);
-            float mk = drop_mul(a.drop, ((uint64_t)bh * a.T + qi) * a.T + kj);
+        for (int u = 0; u < 4; u++) {
+          const int col = (u >> 1) * 32 + e + (u & 1);
+          const uint32_t sraw = (u >> 1) ? s1[e + (u & 1)] : s0[e + (u & 1)];
+          const uint32_t draw = (u >> 1) ? d1[e + (u & 1)] : d0[e + (u & 1)];
+          float p = ex2(fmaf(__uint_as_float(sraw), sl2, -ld[col] * LOG2E));
+          if (diag && kj > q0 + col) p = 0.f;
+          float dp = __uint_as_float(draw);
+          if (a.drop.active) {
+            float mk = drop_mul(a.drop, ((uint64_t)bh * a.T + q0 + col) * a.T + kj);
             pv[u] = p * mk;
-            dsv[u] = p * (__uint_as_float(dv[e + u]) * mk - ld[128 + col]);
+            dp *= mk;
+          } else {
+            pv[u] = p;
           }
-          pp[e >> 1] = pack2(pv[0], pv[1]);
-          pd[e >> 1] = pack2(dsv[0], dsv[1]);
+          dsv[u] = p * (dp - ld[64 + col]);
         }
-        store_chunk32(sb + K_P, r, c, pp);
-        store_chunk32(sb + K_DS, r, c, pd);
+        pp0[e >> 1] = pack2(pv[0], pv[1]);
+        pp1[e >> 1] = pack2(pv[2], pv[3]);
+        pd0[e >> 1] = pack2(dsv[0], dsv[1]);
+        pd1[e >> 1] = pack2(dsv[2], dsv[3]);
       }
+      store_chunk32(sb + K_P, TILE, r, 0, pp0);
+      store_chunk32(sb + K_P, TILE, r, 1, pp1);
+      store_chunk32(sb + K_DS, TILE, r, 0, pd0);
+      store_chunk32(sb + K_DS, TILE, r, 1, pd1);
       fence_proxy_async_smem();
       tc_fence_before();
-      mbar_arrive(pds_full);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(pds_full);
     }
     if (ok && mbar_wait(acc_full, 0, abort_flag, a.flags)) {
       tc_fence_after();
@@ -385,17 +443,16 @@ __global__ void __launch_bounds__(192, 1) k_attn_bwd_kv_tc(const __grid_constant
       for (int w2 = 0; w2 < 2; w2++) {
         const float f = w2 == 0 ? 1.0f : a.scale;
         uint4* dst = reinterpret_cast<uint4*>(rowp + (size_t)((w2 == 0 ? 2 : 1) * a.H + h) * 64);
+        uint32_t v0[32], v1[32];
+        ld64(trow + 128 + w2 * 64, v0, v1);
 #pragma unroll
-        for (int c = 0; c < 2; c++) {
-          uint32_t v[32];
-          tmem_ld_32x32b_x32(trow + 256 + w2 * 64 + c * 32, v);
-          tmem_ld_wait();
-#pragma unroll
-          for (int q = 0; q < 4; q++) {
-            const float* x = reinterpret_cast<const float*>(v) + 8 * q;
-            dst[c * 4 + q] = make_uint4(pack2(x[0] * f, x[1] * f), pack2(x[2] * f, x[3] * f),
-                                        pack2(x[4] * f, x[5] * f), pack2(x[6] * f, x[7] * f));
-          }
+        for (int q = 0; q < 4; q++) {
+          const float* x = reinterpret_cast<const float*>(v0) + 8 * q;
+          const float* y = reinterpret_cast<const float*>(v1) + 8 * q;
+          dst[q] = make_uint4(pack2(x[0] * f, x[1] * f), pack2(x[2] * f, x[3] * f), pack2(x[4] * f, x[5] * f),
+                              pack2(x[6] * f, x[7] * f));
+          dst[4 + q] = make_uint4(pack2(y[0] * f, y[1] * f), pack2(y[2] * f, y[3] * f), pack2(y[4] * f, y[5] * f),
+                                  pack2(y[6] * f, y[7] * f));
         }
       }
     }
@@ -403,20 +460,21 @@ __global__ void __launch_bounds__(192, 1) k_attn_bwd_kv_tc(const __grid_constant
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 1) tmem_dealloc(tmem, 512);
+  if (warp == 1) tmem_dealloc(tmem, 256);
 }
 
 // ============================================================================
-// backward, dQ: one CTA per (128-query block, b, h), walking key blocks <= it.
-//   S = Q K^T, dP = dO V^T  ->  dS (bf16, smem);  dQ += dS K
-// smem: Q | dO | K[2] | V[2] | dS (2 blk) | barriers
-// TMEM: S [0,128), dP [128,256), dQ [256,320)  (512 allocated)
+// backward, dQ: one CTA per (128-query block, b, h), walking 64-key blocks
+// up to the diagonal.  S = Q K^T, dP = dO V^T -> dS (bf16, smem); dQ += dS K
+// smem: Q | dO | (K, V)[2 stages] | dS | barriers   (~80 KB)
+// TMEM: S [0,64), dP [64,128), dQ [128,192)  (256 allocated)
 // ============================================================================
-constexpr int Q_Q = 0, Q_DO = TILE, Q_K = 2 * TILE, Q_V = 4 * TILE, Q_DS = 6 * TILE, Q_BAR = 8 * TILE;
+constexpr int Q_Q = 0, Q_DO = TILE, Q_ST = 2 * TILE, Q_DS = 4 * TILE, Q_BAR = 5 * TILE;
 constexpr int Q_SMEM = Q_BAR + 128;
 
-__global__ void __launch_bounds__(192, 1) k_attn_bwd_q_tc(const __grid_constant__ CUtensorMap tq,
-                                                          const __grid_constant__ CUtensorMap tdo, AttnTcArgs a) {
+__global__ void __launch_bounds__(192, 2) k_attn_bwd_q_tc(const __grid_constant__ CUtensorMap tq,
+                                                          const __grid_constant__ CUtensorMap tdo,
+                                                          const __grid_constant__ CUtensorMap tkv64, AttnTcArgs a) {
   extern __shared__ __align__(1024) uint8_t smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (smem_u32(smem) & 1023) {
@@ -434,7 +492,7 @@ __global__ void __launch_bounds__(192, 1) k_attn_bwd_q_tc(const __grid_constant_
   const int qb = nqb - 1 - (int)blockIdx.x;
   const int bh = blockIdx.y, b = bh / a.H, h = bh % a.H;
   const int row0 = b * a.T;
-  const int nkb = qb + 1;
+  const int nkb = 2 * (qb + 1);  // 64-key blocks up to and including the diagonal
 
   if (threadIdx.x == 0) {
     mbar_init(qd_full, 1);
@@ -443,15 +501,16 @@ __global__ void __launch_bounds__(192, 1) k_attn_bwd_q_tc(const __grid_constant_
     mbar_init(kv_empty0, 1);
     mbar_init(kv_empty0 + 8, 1);
     mbar_init(sdp_full, 1);
-    mbar_init(ds_full, 128);
+    mbar_init(ds_full, 4);
     mbar_init(acc_full, 1);
     *abort_flag = 0;
     fence_barrier_init();
     prefetch_tmap(&tq);
     prefetch_tmap(&tdo);
+    prefetch_tmap(&tkv64);
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(tslot), 512);
+    tmem_alloc(smem_u32(tslot), 256);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -466,33 +525,34 @@ __global__ void __launch_bounds__(192, 1) k_attn_bwd_q_tc(const __grid_constant_
       tma_load_3d(sb + Q_DO, &tdo, qd_full, 0, h, row0 + qb * 128);
       for (int j = 0; j < nkb; j++) {
         int s = j & 1;
+        uint32_t fb = kv_full0 + 8 * s;
         if (!mbar_wait(kv_empty0 + 8 * s, ((j >> 1) & 1) ^ 1, abort_flag, a.flags)) break;
-        mbar_expect_tx(kv_full0 + 8 * s, 2 * TILE);
-        tma_load_3d(sb + Q_K + s * TILE, &tq, kv_full0 + 8 * s, 0, a.H + h, row0 + j * 128);
-        tma_load_3d(sb + Q_V + s * TILE, &tq, kv_full0 + 8 * s, 0, 2 * a.H + h, row0 + j * 128);
+        mbar_expect_tx(fb, 2 * HTILE);
+        tma_load_3d(sb + Q_ST + s * TILE, &tkv64, fb, 0, a.H + h, row0 + j * 64);
+        tma_load_3d(sb + Q_ST + s * TILE + HTILE, &tkv64, fb, 0, 2 * a.H + h, row0 + j * 64);
       }
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      constexpr uint32_t id_s = idesc_bf16_f32(128, 128, false, false);
+      constexpr uint32_t id_s = idesc_bf16_f32(128, 64, false, false);
       constexpr uint32_t id_acc = idesc_bf16_f32(128, 64, false, true);
       bool ok = mbar_wait(qd_full, 0, abort_flag, a.flags);
       for (int j = 0; j < nkb && ok; j++) {
         int s = j & 1;
         if (!(ok = mbar_wait(kv_full0 + 8 * s, (j >> 1) & 1, abort_flag, a.flags))) break;
         tc_fence_after();
-        uint32_t k = sb + Q_K + s * TILE, v = sb + Q_V + s * TILE;
+        uint32_t k = sb + Q_ST + s * TILE, v = k + HTILE;
 #pragma unroll
-        for (int kk = 0; kk < 4; kk++) mma_bf16_ss(tmem, desc_k64(sb + Q_Q, kk), desc_k64(k, kk), id_s, kk > 0);
+        for (int kk = 0; kk < 4; kk++) mma_bf16_ss(tmem, desc_k(sb + Q_Q, TILE, kk), desc_k(k, HTILE, kk), id_s, kk > 0);
 #pragma unroll
         for (int kk = 0; kk < 4; kk++)
-          mma_bf16_ss(tmem + 128, desc_k64(sb + Q_DO, kk), desc_k64(v, kk), id_s, kk > 0);
+          mma_bf16_ss(tmem + 64, desc_k(sb + Q_DO, TILE, kk), desc_k(v, HTILE, kk), id_s, kk > 0);
         mma_commit(sdp_full);
         if (!(ok = mbar_wait(ds_full, j & 1, abort_flag, a.flags))) break;
         tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < 8; kk++)
-          mma_bf16_ss(tmem + 256, desc_k128(sb + Q_DS, kk), desc_mn64(k, kk), id_acc, (j > 0 || kk > 0));
+        for (int kk = 0; kk < 4; kk++)
+          mma_bf16_ss(tmem + 128, desc_k(sb + Q_DS, TILE, kk), desc_mn64(k, kk), id_acc, (j > 0 || kk > 0));
         mma_commit(kv_empty0 + 8 * s);
       }
       mma_commit(acc_full);
@@ -502,6 +562,7 @@ __global__ void __launch_bounds__(192, 1) k_attn_bwd_q_tc(const __grid_constant_
     const int r = quad * 32 + lane;
     const int qi = qb * 128 + r;
     const uint32_t trow = tmem + ((uint32_t)(quad * 32) << 16);
+    const float sl2 = a.scale_log2;
     const float lse2 = a.lse[(size_t)bh * a.T + qi] * LOG2E;
     const float Di = a.dsum[(size_t)bh * a.T + qi];
     const uint64_t ebase = ((uint64_t)bh * a.T + qi) * a.T;
@@ -509,54 +570,60 @@ __global__ void __launch_bounds__(192, 1) k_attn_bwd_q_tc(const __grid_constant_
     for (int j = 0; j < nkb; j++) {
       if (!(ok = mbar_wait(sdp_full, j & 1, abort_flag, a.flags))) break;
       tc_fence_after();
-      const bool diag = (j == qb);
+      const int key0 = j * 64;
+      const bool diag = key0 + 64 > qb * 128;
+      uint32_t s0[32], s1[32], d0[32], d1[32];
+      tmem_ld_32x32b_x32(trow, s0);
+      tmem_ld_32x32b_x32(trow + 32, s1);
+      tmem_ld_32x32b_x32(trow + 64, d0);
+      tmem_ld_32x32b_x32(trow + 96, d1);
+      tmem_ld_wait();
+      uint32_t pd0[16], pd1[16];
 #pragma unroll
-      for (int c = 0; c < 4; c++) {
-        uint32_t sv[32], dv[32];
-        tmem_ld_32x32b_x32(trow + c * 32, sv);
-        tmem_ld_32x32b_x32(trow + 128 + c * 32, dv);
-        tmem_ld_wait();
-        uint32_t pd[16];
+      for (int e = 0; e < 32; e += 2) {
+        float dsv[4];
 #pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          float dsv[2];
-#pragma unroll
-          for (int u = 0; u < 2; u++) {
-            int key = j * 128 + c * 32 + e + u;
-            float p = (diag && key > qi) ? 0.f : exp2f(__uint_as_float(sv[e + u]) * a.scale_log2 - lse2);
-            float mk = drop_mul(a.drop, ebase + key);
-            dsv[u] = p * (__uint_as_float(dv[e + u]) * mk - Di);
-          }
-          pd[e >> 1] = pack2(dsv[0], dsv[1]);
+        for (int u = 0; u < 4; u++) {
+          const int col = (u >> 1) * 32 + e + (u & 1);
+          const uint32_t sraw = (u >> 1) ? s1[e + (u & 1)] : s0[e + (u & 1)];
+          const uint32_t draw = (u >> 1) ? d1[e + (u & 1)] : d0[e + (u & 1)];
+          float p = ex2(fmaf(__uint_as_float(sraw), sl2, -lse2));
+          if (diag && key0 + col > qi) p = 0.f;
+          float dp = __uint_as_float(draw);
+          if (a.drop.active) dp *= drop_mul(a.drop, ebase + key0 + col);
+          dsv[u] = p * (dp - Di);
         }
-        store_chunk32(sb + Q_DS, r, c, pd);
+        pd0[e >> 1] = pack2(dsv[0], dsv[1]);
+        pd1[e >> 1] = pack2(dsv[2], dsv[3]);
       }
+      store_chunk32(sb + Q_DS, TILE, r, 0, pd0);
+      store_chunk32(sb + Q_DS, TILE, r, 1, pd1);
       fence_proxy_async_smem();
       tc_fence_before();
-      mbar_arrive(ds_full);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(ds_full);
     }
     if (ok && mbar_wait(acc_full, 0, abort_flag, a.flags)) {
       tc_fence_after();
       uint4* dst = reinterpret_cast<uint4*>(a.dqkv + (size_t)(row0 + qi) * (3 * a.H * 64) + (size_t)h * 64);
+      uint32_t v0[32], v1[32];
+      ld64(trow + 128, v0, v1);
+      const float f = a.scale;
 #pragma unroll
-      for (int c = 0; c < 2; c++) {
-        uint32_t v[32];
-        tmem_ld_32x32b_x32(trow + 256 + c * 32, v);
-        tmem_ld_wait();
-#pragma unroll
-        for (int q = 0; q < 4; q++) {
-          const float* x = reinterpret_cast<const float*>(v) + 8 * q;
-          const float f = a.scale;
-          dst[c * 4 + q] = make_uint4(pack2(x[0] * f, x[1] * f), pack2(x[2] * f, x[3] * f),
-                                      pack2(x[4] * f, x[5] * f), pack2(x[6] * f, x[7] * f));
-        }
+      for (int q = 0; q < 4; q++) {
+        const float* x = reinterpret_cast<const float*>(v0) + 8 * q;
+        const float* y = reinterpret_cast<const float*>(v1) + 8 * q;
+        dst[q] = make_uint4(pack2(x[0] * f, x[1] * f), pack2(x[2] * f, x[3] * f), pack2(x[4] * f, x[5] * f),
+                            pack2(x[6] * f, x[7] * f));
+        dst[4 + q] = make_uint4(pack2(y[0] * f, y[1] * f), pack2(y[2] * f, y[3] * f), pack2(y[4] * f, y[5] * f),
+                                pack2(y[6] * f, y[7] * f));
       }
     }
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 1) tmem_dealloc(tmem, 512);
+  if (warp == 1) tmem_dealloc(tmem, 256);
 }
 
 // D[b,h,i] = sum_d dO[b,i,h,d] * O[b,i,h,d]: one warp per (row, head), 2 elements per lane
@@ -592,13 +659,13 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// [rows, slots, 64] bf16 viewed as 3-D {64, slots, rows}; box = one slot x 128 rows
-bool map_rows(CUtensorMap* m, const void* base, int slots, long rows) {
+// [rows, slots, 64] bf16 viewed as 3-D {64, slots, rows}; box = one slot x box_rows rows
+bool map_rows(CUtensorMap* m, const void* base, int slots, long rows, int box_rows) {
   auto enc = encode_fn();
   if (!enc) return false;
   cuuint64_t dims[3] = {64, (cuuint64_t)slots, (cuuint64_t)rows};
   cuuint64_t strides[2] = {128, (cuuint64_t)slots * 128};
-  cuuint32_t box[3] = {64, 1, 128};
+  cuuint32_t box[3] = {64, 1, (cuuint32_t)box_rows};
   cuuint32_t estr[3] = {1, 1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -610,7 +677,6 @@ AttnTcArgs make_args(const AttnDesc& d, uint32_t* flags) {
   a.B = d.B;
   a.T = d.T;
   a.H = d.H;
-  a.o = reinterpret_cast<const bf16*>(d.o);
   a.o_out = reinterpret_cast<bf16*>(d.o);
   a.lse = d.lse;
   a.dsum = d.dsum;
@@ -628,12 +694,14 @@ bool attn_tc_supported(const AttnDesc& a) {
   if (a.hd != 64 || a.T % 128 != 0 || a.T <= 0 || !encode_fn()) return false;
   if ((reinterpret_cast<uintptr_t>(a.qkv) & 15) || (reinterpret_cast<uintptr_t>(a.o) & 15)) return false;
   if (a.dout && (reinterpret_cast<uintptr_t>(a.dout) & 15)) return false;
+  if (a.lse && (reinterpret_cast<uintptr_t>(a.lse) & 15)) return false;
+  if (a.dsum && (reinterpret_cast<uintptr_t>(a.dsum) & 15)) return false;
   return true;
 }
 
 void attn_fwd_tc(Ctx& c, const AttnDesc& d) {
   CUtensorMap tm;
-  if (!map_rows(&tm, d.qkv, 3 * d.H, (long)d.B * d.T)) {
+  if (!map_rows(&tm, d.qkv, 3 * d.H, (long)d.B * d.T, 128)) {
     attn_fwd_simt<bf16>(c, d);
     return;
   }
@@ -648,11 +716,14 @@ void attn_fwd_tc(Ctx& c, const AttnDesc& d) {
 }
 
 void attn_bwd_tc(Ctx& c, const AttnDesc& d) {
-  CUtensorMap tq, tdo;
-  if (!map_rows(&tq, d.qkv, 3 * d.H, (long)d.B * d.T) || !map_rows(&tdo, d.dout, d.H, (long)d.B * d.T)) {
+  CUtensorMap tkv, tkv64, tq64, tdo, tdo64;
+  long rows = (long)d.B * d.T;
+  if (!map_rows(&tkv, d.qkv, 3 * d.H, rows, 128) || !map_rows(&tkv64, d.qkv, 3 * d.H, rows, 64) ||
+      !map_rows(&tdo, d.dout, d.H, rows, 128) || !map_rows(&tdo64, d.dout, d.H, rows, 64)) {
     attn_bwd_simt<bf16>(c, d);
     return;
   }
+  tq64 = tkv64;
   {
     long warps = (long)d.B * d.T * d.H;
     LaunchScope s(c, "attn_bwd_dsum");
@@ -669,11 +740,11 @@ void attn_bwd_tc(Ctx& c, const AttnDesc& d) {
   dim3 grid(d.T / 128, d.B * d.H);
   {
     LaunchScope s(c, "attn_bwd_kv_tc");
-    k_attn_bwd_kv_tc<<<grid, 192, K_SMEM, c.stream>>>(tq, tdo, a);
+    k_attn_bwd_kv_tc<<<grid, 192, K_SMEM, c.stream>>>(tkv, tq64, tdo64, a);
   }
   {
     LaunchScope s(c, "attn_bwd_q_tc");
-    k_attn_bwd_q_tc<<<grid, 192, Q_SMEM, c.stream>>>(tq, tdo, a);
+    k_attn_bwd_q_tc<<<grid, 192, Q_SMEM, c.stream>>>(tkv, tdo, tkv64, a);
   }
 }
 

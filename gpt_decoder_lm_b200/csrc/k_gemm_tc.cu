@@ -8,8 +8,8 @@
 //               (128-byte swizzle; K-major or MN-major operands, so dX and dW
 //               need no transposed copies)
 //   warp 1      TMEM allocator + MMA issuer (tcgen05.mma, M=128, N=BN, K=16)
-//   warps 2..5  epilogue: tcgen05.ld of the 128 x BN fp32 tile, one row per
-//               thread, fused element-wise work, vector stores
+//   warps 2..9  epilogue: tcgen05.ld of the 128 x BN fp32 tile, one row and
+//               half of the columns per thread, fused element-wise work
 // TMEM holds two BN-column accumulators so the epilogue of tile i overlaps
 // the MMAs of tile i+1.  Every mbarrier wait is bounded.
 #include <cudaTypedefs.h>
@@ -25,7 +25,7 @@ namespace {
 using namespace sm100;
 
 constexpr int BM = 128, BK = 64;
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;   // producer, MMA, 8 epilogue warps (2 per TMEM lane quadrant)
 
 struct TcArgs {
   int M, N, K;
@@ -68,12 +68,18 @@ __device__ __forceinline__ void epi_chunk(const TcArgs& p, long row, int col0, i
 #pragma unroll
       for (int i = 0; i < 8; i++) reinterpret_cast<float4*>(dst)[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
     } else {
-      for (int i = 0; i < p.N - col0; i++) dst[i] = v[i];
+      const int n = p.N - col0;
+#pragma unroll
+      for (int i = 0; i < 32; i++)  // static indices keep v[] in registers
+        if (i < n) dst[i] = v[i];
     }
     return;
   }
   if (col0 + 32 > p.N) {  // ragged right edge: scalar path
-    for (int i = 0; i < p.N - col0; i++) epi_apply<bf16>(e, p.N, row, col0 + i, v[i]);
+    const int n = p.N - col0;
+#pragma unroll
+    for (int i = 0; i < 32; i++)
+      if (i < n) epi_apply<bf16>(e, p.N, row, col0 + i, v[i]);
     return;
   }
   switch (e.kind) {
@@ -188,7 +194,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int b = 0; b < 2; b++) {
       mbar_init(smem_u32(&tfull[b]), 1);
-      mbar_init(smem_u32(&tempty[b]), 128);
+      mbar_init(smem_u32(&tempty[b]), 8);  // one arrival per epilogue warp
     }
     *abort_flag = 0;
     fence_barrier_init();
@@ -298,7 +304,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    const int quad = warp & 3;  // TMEM lanes quad*32 .. quad*32+31
+    const int quad = warp & 3;         // TMEM lanes quad*32 .. quad*32+31
+    const int half = (warp - 2) >> 2;  // which half of the BN columns
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int t = blockIdx.x; t < tiles; t += gridDim.x) {
@@ -310,14 +317,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       long row = (long)mb * BM + quad * 32 + lane;
       uint32_t tbase = tmem_base + ((uint32_t)(quad * 32) << 16) + acc * BN;
 #pragma unroll 1
-      for (int c = 0; c < BN / 32; c++) {
+      for (int c = half * (BN / 64); c < (half + 1) * (BN / 64); c++) {
         uint32_t v[32];
         tmem_ld_32x32b_x32(tbase + c * 32, v);
         tmem_ld_wait();
         epi_chunk(p, row, nb * BN + c * 32, split, v);
       }
       tc_fence_before();
-      mbar_arrive(smem_u32(&tempty[acc]));
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&tempty[acc]));
       if (++acc == 2) {
         acc = 0;
         acc_phase ^= 1;
