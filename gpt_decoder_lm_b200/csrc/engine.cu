@@ -89,16 +89,9 @@ struct Layout {
   }
 };
 
-int choose_splits(long M, long N, long K) {
-  // dW GEMMs: 128x128 tiles; split K until there are ~2 tiles per SM (148 SMs)
-  long tiles = ((M + 127) / 128) * ((N + 127) / 128);
-  long nkb = (K + 63) / 64;
-  if (tiles >= 148) return 1;
-  long s = (2 * 148 + tiles - 1) / tiles;
-  if (s > 16) s = 16;
-  if (s > nkb / 4) s = std::max(1L, nkb / 4);
-  return (int)s;
-}
+// split-K count of a weight-gradient GEMM (sizes the partial-sum scratch; the
+// plan of a 148-SM B200)
+int choose_splits(long M, long N, long K) { return gemm_tc_plan(M, N, K, true, 148).splits; }
 
 }  // namespace
 
@@ -344,7 +337,7 @@ size_t carve(gpt_model& m, uint8_t* base) {
   m.dres = F((size_t)M * d);
   m.dln = F((size_t)M * d);
   m.dsum = F((size_t)M * m.H);
-  m.part_blocks = (int)std::min<long>(M, 148 * 2);
+  m.part_blocks = (int)std::min<long>(M, 148 * 8);
   m.part = F((size_t)m.part_blocks * 3 * d);
   m.colsum_scr = F((size_t)64 * 4 * d);
   // split-K scratch: the largest dW partial set
@@ -477,6 +470,7 @@ gpt_status forward_t(gpt_model* m, bool fuse_ce_grad, float* loss_acc, float los
                 m->ln1_rstd + l * M, M, d, rms, eps);
     GemmDesc g = gd((int)M, 3 * d, d, a1, d, true, m->Wop(y.qkv_w), d, true);
     g.epi.kind = EPI_BIAS;
+    g.name = "gemm_qkv_fwd";
     g.epi.bias = y.qkv_b >= 0 ? m->P(y.qkv_b) : nullptr;
     g.epi.out = qkv;
     g.epi.ldo = 3 * d;
@@ -487,6 +481,7 @@ gpt_status forward_t(gpt_model* m, bool fuse_ce_grad, float* loss_acc, float los
     else attn_fwd_simt<T>(c, ad);
     g = gd((int)M, d, d, o, d, true, m->Wop(y.ap_w), d, true);
     g.epi.kind = EPI_RESADD;
+    g.name = "gemm_attnproj_fwd";
     g.epi.bias = y.ap_b >= 0 ? m->P(y.ap_b) : nullptr;
     g.epi.res_in = x;
     g.epi.res_out = xm;
@@ -498,6 +493,7 @@ gpt_status forward_t(gpt_model* m, bool fuse_ce_grad, float* loss_acc, float los
                 m->ln2_rstd + l * M, M, d, rms, eps);
     g = gd((int)M, 4 * d, d, a2, d, true, m->Wop(y.fc_w), d, true);
     g.epi.kind = EPI_BIAS_ACT;
+    g.name = "gemm_fc_fwd";
     g.epi.act = act;
     g.epi.bias = y.fc_b >= 0 ? m->P(y.fc_b) : nullptr;
     g.epi.out = h;
@@ -506,6 +502,7 @@ gpt_status forward_t(gpt_model* m, bool fuse_ce_grad, float* loss_acc, float los
     if (!gemm(m, g)) return fail(m, GPT_ERR_CUDA, "fc gemm failed");
     g = gd((int)M, d, 4 * d, gg, 4 * d, true, m->Wop(y.pr_w), 4 * d, true);
     g.epi.kind = EPI_RESADD;
+    g.name = "gemm_mlpproj_fwd";
     g.epi.bias = y.pr_b >= 0 ? m->P(y.pr_b) : nullptr;
     g.epi.res_in = xm;
     g.epi.res_out = xo;
@@ -519,6 +516,7 @@ gpt_status forward_t(gpt_model* m, bool fuse_ce_grad, float* loss_acc, float los
               m->lnf_mean, m->lnf_rstd, M, d, rms, eps);
   GemmDesc g = gd((int)M, m->Vp, d, xf, d, true, m->Wop(m->head), d, true);
   g.epi.kind = EPI_STORE;
+  g.name = "gemm_lmhead_fwd";
   g.epi.out = m->logits;
   g.epi.ldo = m->Vp;
   if (!gemm(m, g)) return fail(m, GPT_ERR_CUDA, "lm_head gemm failed");
@@ -551,10 +549,11 @@ gpt_status backward_t(gpt_model* m) {
   T* dh = reinterpret_cast<T*>(m->dh);
   T* dqkv = reinterpret_cast<T*>(m->dqkv);
   T* datt = reinterpret_cast<T*>(m->datt);
-  auto dW = [&](int Mo, int No, const void* A, const void* Bm, float* out) -> bool {
+  auto dW = [&](int Mo, int No, const void* A, const void* Bm, float* out, const char* name) -> bool {
     // out[Mo, No] += A^T B with A [M, Mo], B [M, No] (tokens outermost)
     GemmDesc g = gd(Mo, No, (int)M, A, Mo, false, Bm, No, false);
     g.epi.kind = EPI_ACC_F32;
+    g.name = name;
     g.epi.out = out;
     g.epi.ldo = No;
     if (m->bf16m) {
@@ -566,10 +565,11 @@ gpt_status backward_t(gpt_model* m) {
   // lm_head: dx_f = dlogits W_head; dW_head += dlogits^T x_f
   GemmDesc g = gd((int)M, d, Vp, dl, Vp, true, m->Wop(m->head), d, false);
   g.epi.kind = EPI_STORE_F32;
+  g.name = "gemm_lmhead_dx";
   g.epi.out = m->dln;
   g.epi.ldo = d;
   if (!gemm(m, g)) return fail(m, GPT_ERR_CUDA, "lm_head dX gemm failed");
-  if (!dW(Vp, d, dl, m->lnf, m->G(m->head))) return fail(m, GPT_ERR_CUDA, "lm_head dW gemm failed");
+  if (!dW(Vp, d, dl, m->lnf, m->G(m->head), "gemm_lmhead_dw")) return fail(m, GPT_ERR_CUDA, "lm_head dW gemm failed");
   // final norm
   NormBwd nb;
   nb.dy = m->dln;
@@ -598,18 +598,20 @@ gpt_status backward_t(gpt_model* m) {
     T* h = at<T>(m->fch, l * 4 * Md);
     T* gg = at<T>(m->fcg, l * 4 * Md);
     // MLP projection
-    if (!dW(d, 4 * d, dyb, gg, m->G(y.pr_w))) return fail(m, GPT_ERR_CUDA, "proj dW failed");
+    if (!dW(d, 4 * d, dyb, gg, m->G(y.pr_w), "gemm_mlpproj_dw")) return fail(m, GPT_ERR_CUDA, "proj dW failed");
     g = gd((int)M, 4 * d, d, dyb, d, true, m->Wop(y.pr_w), 4 * d, false);
     g.epi.kind = EPI_ACT_BWD;
+    g.name = "gemm_mlpproj_dx";
     g.epi.act = act;
     g.epi.aux = h;
     g.epi.out = dh;
     g.epi.ldo = 4 * d;
     if (!gemm(m, g)) return fail(m, GPT_ERR_CUDA, "proj dX failed");
     if (y.fc_b >= 0) colsum_acc<T>(c, dh, M, 4 * d, m->colsum_scr, m->G(y.fc_b));
-    if (!dW(4 * d, d, dh, a2, m->G(y.fc_w))) return fail(m, GPT_ERR_CUDA, "fc dW failed");
+    if (!dW(4 * d, d, dh, a2, m->G(y.fc_w), "gemm_fc_dw")) return fail(m, GPT_ERR_CUDA, "fc dW failed");
     g = gd((int)M, d, 4 * d, dh, 4 * d, true, m->Wop(y.fc_w), d, false);
     g.epi.kind = EPI_STORE_F32;
+    g.name = "gemm_fc_dx";
     g.epi.out = m->dln;
     g.epi.ldo = d;
     if (!gemm(m, g)) return fail(m, GPT_ERR_CUDA, "fc dX failed");
@@ -624,9 +626,10 @@ gpt_status backward_t(gpt_model* m) {
     norm_bwd<T>(c, nb);
     add_bias_grads_from_norm(m, y.ln2_w, y.ln2_b, y.ap_b);
     // attention projection
-    if (!dW(d, d, dyb, o, m->G(y.ap_w))) return fail(m, GPT_ERR_CUDA, "attn proj dW failed");
+    if (!dW(d, d, dyb, o, m->G(y.ap_w), "gemm_attnproj_dw")) return fail(m, GPT_ERR_CUDA, "attn proj dW failed");
     g = gd((int)M, d, d, dyb, d, true, m->Wop(y.ap_w), d, false);
     g.epi.kind = EPI_STORE;
+    g.name = "gemm_attnproj_dx";
     g.epi.out = datt;
     g.epi.ldo = d;
     if (!gemm(m, g)) return fail(m, GPT_ERR_CUDA, "attn proj dX failed");
@@ -634,9 +637,10 @@ gpt_status backward_t(gpt_model* m) {
     if (sizeof(T) == 2 && attn_tc_supported(ad)) attn_bwd_tc(c, ad);
     else attn_bwd_simt<T>(c, ad);
     if (y.qkv_b >= 0) colsum_acc<T>(c, dqkv, M, 3 * d, m->colsum_scr, m->G(y.qkv_b));
-    if (!dW(3 * d, d, dqkv, a1, m->G(y.qkv_w))) return fail(m, GPT_ERR_CUDA, "qkv dW failed");
+    if (!dW(3 * d, d, dqkv, a1, m->G(y.qkv_w), "gemm_qkv_dw")) return fail(m, GPT_ERR_CUDA, "qkv dW failed");
     g = gd((int)M, d, 3 * d, dqkv, 3 * d, true, m->Wop(y.qkv_w), d, false);
     g.epi.kind = EPI_STORE_F32;
+    g.name = "gemm_qkv_dx";
     g.epi.out = m->dln;
     g.epi.ldo = d;
     if (!gemm(m, g)) return fail(m, GPT_ERR_CUDA, "qkv dX failed");

@@ -8,8 +8,14 @@
 //               (128-byte swizzle; K-major or MN-major operands, so dX and dW
 //               need no transposed copies)
 //   warp 1      TMEM allocator + MMA issuer (tcgen05.mma, M=128, N=BN, K=16)
-//   warps 2..9  epilogue: tcgen05.ld of the 128 x BN fp32 tile, one row and
-//               half of the columns per thread, fused element-wise work
+//   warps 2..9  epilogue: two warps per TMEM lane quadrant, each taking half
+//               of the BN columns in 32x32 chunks: tcgen05.ld -> fused
+//               element-wise work -> swizzled shared-memory staging tile ->
+//               TMA tensor store (or TMA reduce-add for gradient
+//               accumulation).  Inputs the epilogue needs (the residual
+//               stream, the saved pre-activation) arrive by TMA into the same
+//               staging tiles, so every global access of the epilogue is a
+//               coalesced bulk transfer.
 // TMEM holds two BN-column accumulators so the epilogue of tile i overlaps
 // the MMAs of tile i+1.  Every mbarrier wait is bounded.
 #include <cudaTypedefs.h>
@@ -25,13 +31,16 @@ namespace {
 using namespace sm100;
 
 constexpr int BM = 128, BK = 64;
-constexpr int kThreads = 320;   // producer, MMA, 8 epilogue warps (2 per TMEM lane quadrant)
+constexpr int kThreads = 320;    // producer, MMA, 8 epilogue warps
+constexpr int EPI_WARPS = 8;
+constexpr int EPI_BUF = 4096;    // one 32x32 fp32 (or bf16) staging tile
 
 struct TcArgs {
   int M, N, K;
   int num_m, num_n, splits, kb_per_split, nkb;
-  GemmEpi epi;
-  float* partial;
+  int kind, act;
+  const float* bias;
+  DropKey drop;
   uint32_t* flags;
 };
 
@@ -40,10 +49,11 @@ struct TcCfg {
   static constexpr int A_BYTES = BM * BK * 2;
   static constexpr int B_BYTES = BN * BK * 2;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-  static constexpr int STAGES = BN == 256 ? 4 : 6;
+  static constexpr int STAGES = BN == 256 ? 3 : 5;
   static constexpr int TMEM_COLS = 2 * BN;
-  static constexpr int BAR_OFF = STAGES * STAGE_BYTES;
-  static constexpr int SMEM_BYTES = BAR_OFF + 256 + 1024;  // + barriers + alignment slack
+  static constexpr int EPI_OFF = STAGES * STAGE_BYTES;
+  static constexpr int BAR_OFF = EPI_OFF + EPI_WARPS * 2 * EPI_BUF;
+  static constexpr int SMEM_BYTES = BAR_OFF + 512 + 1024;  // + barriers + alignment slack
 };
 
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
@@ -55,124 +65,71 @@ __device__ __forceinline__ float2 unpack_bf16(uint32_t u) {
   return __bfloat1622float2(v);
 }
 
-// Epilogue of one 32-column chunk of one row.
-__device__ __forceinline__ void epi_chunk(const TcArgs& p, long row, int col0, int split, const uint32_t (&r)[32]) {
-  if (row >= p.M || col0 >= p.N) return;
-  const GemmEpi& e = p.epi;
-  float v[32];
+// Staging tiles hold 32 rows x 32 columns; row r belongs to lane r.
+// fp32 rows are 128 bytes (TMA 128-byte swizzle: 16-byte chunk q of row r at
+// q ^ (r & 7)); bf16 rows are 64 bytes (64-byte swizzle: chunk q at
+// q ^ ((r >> 1) & 3)).  Both keep a warp's 16-byte accesses conflict-free.
+__device__ __forceinline__ void stage_f32(uint32_t buf, int r, const float (&x)[32]) {
 #pragma unroll
-  for (int i = 0; i < 32; i++) v[i] = __uint_as_float(r[i]);
-  if (p.splits > 1) {  // split-K partial of an fp32 accumulation
-    float* dst = p.partial + ((long)split * p.M + row) * p.N + col0;
-    if (col0 + 32 <= p.N) {
+  for (int q = 0; q < 8; q++)
+    st_shared_v4(buf + r * 128 + ((q ^ (r & 7)) << 4), __float_as_uint(x[4 * q]), __float_as_uint(x[4 * q + 1]),
+                 __float_as_uint(x[4 * q + 2]), __float_as_uint(x[4 * q + 3]));
+}
+__device__ __forceinline__ void unstage_f32(uint32_t buf, int r, float (&x)[32]) {
 #pragma unroll
-      for (int i = 0; i < 8; i++) reinterpret_cast<float4*>(dst)[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
-    } else {
-      const int n = p.N - col0;
-#pragma unroll
-      for (int i = 0; i < 32; i++)  // static indices keep v[] in registers
-        if (i < n) dst[i] = v[i];
-    }
-    return;
+  for (int q = 0; q < 8; q++) {
+    uint4 u = ld_shared_v4(buf + r * 128 + ((q ^ (r & 7)) << 4));
+    x[4 * q] = __uint_as_float(u.x);
+    x[4 * q + 1] = __uint_as_float(u.y);
+    x[4 * q + 2] = __uint_as_float(u.z);
+    x[4 * q + 3] = __uint_as_float(u.w);
   }
-  if (col0 + 32 > p.N) {  // ragged right edge: scalar path
-    const int n = p.N - col0;
+}
+__device__ __forceinline__ void stage_bf16(uint32_t buf, int r, const float (&x)[32]) {
+#pragma unroll
+  for (int q = 0; q < 4; q++)
+    st_shared_v4(buf + r * 64 + ((q ^ ((r >> 1) & 3)) << 4), pack_bf16(x[8 * q], x[8 * q + 1]),
+                 pack_bf16(x[8 * q + 2], x[8 * q + 3]), pack_bf16(x[8 * q + 4], x[8 * q + 5]),
+                 pack_bf16(x[8 * q + 6], x[8 * q + 7]));
+}
+__device__ __forceinline__ void unstage_bf16(uint32_t buf, int r, float (&x)[32]) {
+#pragma unroll
+  for (int q = 0; q < 4; q++) {
+    uint4 u = ld_shared_v4(buf + r * 64 + ((q ^ ((r >> 1) & 3)) << 4));
+    uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int k = 0; k < 4; k++) {
+      float2 f = unpack_bf16(w[k]);
+      x[8 * q + 2 * k] = f.x;
+      x[8 * q + 2 * k + 1] = f.y;
+    }
+  }
+}
+
+__device__ __forceinline__ void add_bias(const TcArgs& p, int col0, float (&v)[32]) {
+  if (!p.bias) return;
+  if (col0 + 32 <= p.N) {
+    const float4* b4 = reinterpret_cast<const float4*>(p.bias + col0);
+#pragma unroll
+    for (int i = 0; i < 8; i++) {
+      float4 b = b4[i];
+      v[4 * i] += b.x;
+      v[4 * i + 1] += b.y;
+      v[4 * i + 2] += b.z;
+      v[4 * i + 3] += b.w;
+    }
+  } else {
 #pragma unroll
     for (int i = 0; i < 32; i++)
-      if (i < n) epi_apply<bf16>(e, p.N, row, col0 + i, v[i]);
-    return;
-  }
-  switch (e.kind) {
-    case EPI_STORE:
-    case EPI_BIAS:
-    case EPI_BIAS_ACT: {
-      if (e.bias) {
-        const float4* b4 = reinterpret_cast<const float4*>(e.bias + col0);
-#pragma unroll
-        for (int i = 0; i < 8; i++) {
-          float4 b = b4[i];
-          v[4 * i] += b.x;
-          v[4 * i + 1] += b.y;
-          v[4 * i + 2] += b.z;
-          v[4 * i + 3] += b.w;
-        }
-      }
-      uint4* o = reinterpret_cast<uint4*>(reinterpret_cast<bf16*>(e.out) + row * e.ldo + col0);
-#pragma unroll
-      for (int i = 0; i < 4; i++)
-        o[i] = make_uint4(pack_bf16(v[8 * i], v[8 * i + 1]), pack_bf16(v[8 * i + 2], v[8 * i + 3]),
-                          pack_bf16(v[8 * i + 4], v[8 * i + 5]), pack_bf16(v[8 * i + 6], v[8 * i + 7]));
-      if (e.kind == EPI_BIAS_ACT) {
-#pragma unroll
-        for (int i = 0; i < 32; i++) v[i] = act_fwd(e.act, v[i]);
-        uint4* o2 = reinterpret_cast<uint4*>(reinterpret_cast<bf16*>(e.out2) + row * e.ldo + col0);
-#pragma unroll
-        for (int i = 0; i < 4; i++)
-          o2[i] = make_uint4(pack_bf16(v[8 * i], v[8 * i + 1]), pack_bf16(v[8 * i + 2], v[8 * i + 3]),
-                             pack_bf16(v[8 * i + 4], v[8 * i + 5]), pack_bf16(v[8 * i + 6], v[8 * i + 7]));
-      }
-      break;
-    }
-    case EPI_RESADD: {
-      const float4* ri = reinterpret_cast<const float4*>(e.res_in + row * e.ld_res + col0);
-      float4* ro = reinterpret_cast<float4*>(e.res_out + row * e.ld_res + col0);
-      const float4* b4 = e.bias ? reinterpret_cast<const float4*>(e.bias + col0) : nullptr;
-#pragma unroll
-      for (int i = 0; i < 8; i++) {
-        float4 x = ri[i];
-        float4 b = b4 ? b4[i] : make_float4(0.f, 0.f, 0.f, 0.f);
-        float y0 = v[4 * i] + b.x, y1 = v[4 * i + 1] + b.y, y2 = v[4 * i + 2] + b.z, y3 = v[4 * i + 3] + b.w;
-        if (e.drop.active) {
-          uint64_t el = (uint64_t)row * p.N + col0 + 4 * i;
-          y0 *= drop_mul(e.drop, el);
-          y1 *= drop_mul(e.drop, el + 1);
-          y2 *= drop_mul(e.drop, el + 2);
-          y3 *= drop_mul(e.drop, el + 3);
-        }
-        ro[i] = make_float4(x.x + y0, x.y + y1, x.z + y2, x.w + y3);
-      }
-      break;
-    }
-    case EPI_ACT_BWD: {
-      const uint4* h4 = reinterpret_cast<const uint4*>(reinterpret_cast<const bf16*>(e.aux) + row * e.ldo + col0);
-      uint4* o = reinterpret_cast<uint4*>(reinterpret_cast<bf16*>(e.out) + row * e.ldo + col0);
-#pragma unroll
-      for (int i = 0; i < 4; i++) {
-        uint4 hv = h4[i];
-        uint32_t hw[4] = {hv.x, hv.y, hv.z, hv.w};
-        uint32_t ow[4];
-#pragma unroll
-        for (int q = 0; q < 4; q++) {
-          float2 h = unpack_bf16(hw[q]);
-          ow[q] = pack_bf16(v[8 * i + 2 * q] * act_grad(e.act, h.x), v[8 * i + 2 * q + 1] * act_grad(e.act, h.y));
-        }
-        o[i] = make_uint4(ow[0], ow[1], ow[2], ow[3]);
-      }
-      break;
-    }
-    case EPI_ACC_F32:
-    case EPI_STORE_F32: {
-      float4* o = reinterpret_cast<float4*>(reinterpret_cast<float*>(e.out) + row * e.ldo + col0);
-#pragma unroll
-      for (int i = 0; i < 8; i++) {
-        float4 a = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
-        if (e.kind == EPI_ACC_F32) {
-          float4 old = o[i];
-          a.x += old.x;
-          a.y += old.y;
-          a.z += old.z;
-          a.w += old.w;
-        }
-        o[i] = a;
-      }
-      break;
-    }
+      if (col0 + i < p.N) v[i] += p.bias[col0 + i];
   }
 }
 
 template <int BN, bool A_MN, bool B_MN>
 __global__ void __launch_bounds__(kThreads, 1)
-    k_gemm_tc(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUtensorMap tma_b, TcArgs p) {
+    k_gemm_tc(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUtensorMap tma_b,
+              const __grid_constant__ CUtensorMap tm_out, const __grid_constant__ CUtensorMap tm_out2,
+              const __grid_constant__ CUtensorMap tm_in, TcArgs p) {
   using C = TcCfg<BN>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -181,7 +138,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* empty = bars + C::STAGES;
   uint64_t* tfull = bars + 2 * C::STAGES;
   uint64_t* tempty = tfull + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
+  uint64_t* ebar = tempty + 2;  // [EPI_WARPS] staging-tile loads
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ebar + EPI_WARPS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -194,8 +152,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int b = 0; b < 2; b++) {
       mbar_init(smem_u32(&tfull[b]), 1);
-      mbar_init(smem_u32(&tempty[b]), 8);  // one arrival per epilogue warp
+      mbar_init(smem_u32(&tempty[b]), EPI_WARPS);  // one arrival per epilogue warp
     }
+    for (int w = 0; w < EPI_WARPS; w++) mbar_init(smem_u32(&ebar[w]), 1);
     *abort_flag = 0;
     fence_barrier_init();
     prefetch_tmap(&tma_a);
@@ -304,24 +263,106 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    const int quad = warp & 3;         // TMEM lanes quad*32 .. quad*32+31
-    const int half = (warp - 2) >> 2;  // which half of the BN columns
+    const int ew = warp - 2;          // 0..7
+    const int quad = warp & 3;        // TMEM lanes quad*32 .. quad*32+31
+    const int half = ew >> 2;         // which half of the BN columns
+    // two 4 KB staging sets per warp, used by alternate chunks: a set holds one
+    // fp32 tile, or two bf16 tiles (A at +0, B at +2 KB)
+    const uint32_t stg = smem_u32(smem + C::EPI_OFF + ew * 2 * EPI_BUF);
+    int set = 0;
+    const uint32_t lbar = smem_u32(&ebar[ew]);
+    uint32_t lphase = 0;
+    const int kind = p.kind;
+    const bool f32_in = kind == EPI_RESADD, bf16_in = kind == EPI_ACT_BWD;
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int t = blockIdx.x; t < tiles; t += gridDim.x) {
+    bool ok = true;
+    for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
       int split = t / (p.num_m * p.num_n);
       int r = t % (p.num_m * p.num_n);
       int mb = r % p.num_m, nb = r / p.num_m;
-      if (!mbar_wait(smem_u32(&tfull[acc]), acc_phase, abort_flag, p.flags)) break;
+      if (!(ok = mbar_wait(smem_u32(&tfull[acc]), acc_phase, abort_flag, p.flags))) break;
       tc_fence_after();
-      long row = (long)mb * BM + quad * 32 + lane;
-      uint32_t tbase = tmem_base + ((uint32_t)(quad * 32) << 16) + acc * BN;
+      const int row0 = mb * BM + quad * 32;
+      const long row = row0 + lane;
+      const uint32_t tbase = tmem_base + ((uint32_t)(quad * 32) << 16) + acc * BN;
 #pragma unroll 1
       for (int c = half * (BN / 64); c < (half + 1) * (BN / 64); c++) {
-        uint32_t v[32];
-        tmem_ld_32x32b_x32(tbase + c * 32, v);
+        const int col0 = nb * BN + c * 32;
+        uint32_t raw[32];
+        tmem_ld_32x32b_x32(tbase + c * 32, raw);
+        const uint32_t bufA = stg + set * EPI_BUF, bufB = bufA + 2048;
+        set ^= 1;
+        if (lane == 0) bulk_wait_read1();  // the set used two chunks ago is free again
+        __syncwarp();
+        if (f32_in || bf16_in) {
+          if (lane == 0) {
+            mbar_expect_tx(lbar, f32_in ? 4096 : 2048);
+            tma_load_2d(f32_in ? bufA : bufB, &tm_in, lbar, col0, row0);
+          }
+          if (!mbar_wait(lbar, lphase, abort_flag, p.flags)) {
+            tmem_ld_wait();  // no TMEM load left in flight
+            ok = false;
+            break;
+          }
+          lphase ^= 1;
+        }
         tmem_ld_wait();
-        epi_chunk(p, row, nb * BN + c * 32, split, v);
+        float v[32];
+#pragma unroll
+        for (int i = 0; i < 32; i++) v[i] = __uint_as_float(raw[i]);
+        if (p.splits > 1) {
+          stage_f32(bufA, lane, v);
+        } else {
+          switch (kind) {
+            case EPI_STORE:
+            case EPI_BIAS:
+              add_bias(p, col0, v);
+              stage_bf16(bufA, lane, v);
+              break;
+            case EPI_BIAS_ACT:
+              add_bias(p, col0, v);
+              stage_bf16(bufA, lane, v);
+#pragma unroll
+              for (int i = 0; i < 32; i++) v[i] = act_fwd(p.act, v[i]);
+              stage_bf16(bufB, lane, v);
+              break;
+            case EPI_ACT_BWD: {
+              float hv[32];
+              unstage_bf16(bufB, lane, hv);
+#pragma unroll
+              for (int i = 0; i < 32; i++) v[i] *= act_grad(p.act, hv[i]);
+              stage_bf16(bufA, lane, v);
+              break;
+            }
+            case EPI_RESADD: {
+              float x[32];
+              unstage_f32(bufA, lane, x);
+              add_bias(p, col0, v);
+              if (p.drop.active) {
+                const uint64_t el = (uint64_t)row * p.N + col0;
+#pragma unroll
+                for (int i = 0; i < 32; i++) v[i] *= drop_mul(p.drop, el + i);
+              }
+#pragma unroll
+              for (int i = 0; i < 32; i++) v[i] += x[i];
+              stage_f32(bufA, lane, v);
+              break;
+            }
+            default:  // EPI_ACC_F32, EPI_STORE_F32
+              stage_f32(bufA, lane, v);
+              break;
+          }
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          if (p.splits > 1) tma_store_3d(&tm_out, bufA, col0, row0, split);
+          else if (kind == EPI_ACC_F32) tma_reduce_add_2d(&tm_out, bufA, col0, row0);
+          else tma_store_2d(&tm_out, bufA, col0, row0);
+          if (kind == EPI_BIAS_ACT && p.splits == 1) tma_store_2d(&tm_out2, bufB, col0, row0);
+          bulk_commit();
+        }
       }
       tc_fence_before();
       __syncwarp();
@@ -331,6 +372,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         acc_phase ^= 1;
       }
     }
+    if (lane == 0) bulk_wait0();  // every store of this warp has landed
   }
   tc_fence_before();
   __syncthreads();
@@ -352,31 +394,77 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
   return fn;
 }
 
-// 2-D bf16 tensor map: `inner` contiguous elements per row, `outer` rows,
-// row pitch `ld` elements; box = box_inner x box_outer, 128-byte swizzle.
-bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint64_t ld, uint32_t box_inner,
-              uint32_t box_outer) {
+// 2-D tensor map: `inner` contiguous elements per row, `outer` rows, row
+// pitch `ld` elements; box = box_inner x box_outer.
+bool make_map(CUtensorMap* m, CUtensorMapDataType dt, int esize, const void* base, uint64_t inner, uint64_t outer,
+              uint64_t ld, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle sw) {
   auto enc = get_encode();
   if (!enc) return false;
   cuuint64_t dims[2] = {inner, outer};
-  cuuint64_t strides[1] = {ld * 2};
+  cuuint64_t strides[1] = {ld * esize};
   cuuint32_t box[2] = {box_inner, box_outer};
   cuuint32_t estr[2] = {1, 1};
-  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
-                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
+  return enc(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool make_out_map(CUtensorMap* m, bool f32, const void* base, int M, int N, long ld) {
+  return f32 ? make_map(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, base, N, M, ld, 32, 32, CU_TENSOR_MAP_SWIZZLE_128B)
+             : make_map(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, N, M, ld, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B);
+}
+
+// split-K partials [splits, M, N] fp32 as a 3-D map so boxes clip per split
+bool make_partial_map(CUtensorMap* m, const void* base, int M, int N, int splits) {
+  auto enc = get_encode();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)N, (cuuint64_t)M, (cuuint64_t)splits};
+  cuuint64_t strides[2] = {(cuuint64_t)N * 4, (cuuint64_t)M * N * 4};
+  cuuint32_t box[3] = {32, 32, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 template <int BN, bool A_MN, bool B_MN>
 bool launch(Ctx& c, const GemmDesc& g, int splits) {
   using Cf = TcCfg<BN>;
-  CUtensorMap ma, mb;
+  const GemmEpi& e = g.epi;
+  CUtensorMap ma, mb, mo, mo2, mi;
   bool ok = true;
-  if (!A_MN) ok &= make_map(&ma, g.A, g.K, g.M, g.lda, BK, BM);
-  else ok &= make_map(&ma, g.A, g.M, g.K, g.lda, 64, BK);
-  if (!B_MN) ok &= make_map(&mb, g.B, g.K, g.N, g.ldb, BK, BN);
-  else ok &= make_map(&mb, g.B, g.N, g.K, g.ldb, 64, BK);
+  constexpr auto BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  constexpr auto SW = CU_TENSOR_MAP_SWIZZLE_128B;
+  if (!A_MN) ok &= make_map(&ma, BF, 2, g.A, g.K, g.M, g.lda, BK, BM, SW);
+  else ok &= make_map(&ma, BF, 2, g.A, g.M, g.K, g.lda, 64, BK, SW);
+  if (!B_MN) ok &= make_map(&mb, BF, 2, g.B, g.K, g.N, g.ldb, BK, BN, SW);
+  else ok &= make_map(&mb, BF, 2, g.B, g.N, g.K, g.ldb, 64, BK, SW);
+  mo2 = mb;  // unused unless EPI_BIAS_ACT
+  mi = mb;   // unused unless the epilogue reads an input tile
+  if (splits > 1) {
+    ok &= make_partial_map(&mo, g.partial, g.M, g.N, splits);
+  } else {
+    switch (e.kind) {
+      case EPI_STORE:
+      case EPI_BIAS:
+        ok &= make_out_map(&mo, false, e.out, g.M, g.N, e.ldo);
+        break;
+      case EPI_BIAS_ACT:
+        ok &= make_out_map(&mo, false, e.out, g.M, g.N, e.ldo);
+        ok &= make_out_map(&mo2, false, e.out2, g.M, g.N, e.ldo);
+        break;
+      case EPI_ACT_BWD:
+        ok &= make_out_map(&mo, false, e.out, g.M, g.N, e.ldo);
+        ok &= make_out_map(&mi, false, e.aux, g.M, g.N, e.ldo);
+        break;
+      case EPI_RESADD:
+        ok &= make_out_map(&mo, true, e.res_out, g.M, g.N, e.ld_res);
+        ok &= make_out_map(&mi, true, e.res_in, g.M, g.N, e.ld_res);
+        break;
+      default:
+        ok &= make_out_map(&mo, true, e.out, g.M, g.N, e.ldo);
+        break;
+    }
+  }
   if (!ok) return false;
   TcArgs a;
   a.M = g.M;
@@ -387,8 +475,10 @@ bool launch(Ctx& c, const GemmDesc& g, int splits) {
   a.nkb = (g.K + BK - 1) / BK;
   a.splits = splits;
   a.kb_per_split = (a.nkb + splits - 1) / splits;
-  a.epi = g.epi;
-  a.partial = g.partial;
+  a.kind = e.kind;
+  a.act = e.act;
+  a.bias = e.bias;
+  a.drop = e.drop;
   a.flags = c.flags;
   int tiles = a.num_m * a.num_n * splits;
   int grid = tiles < c.num_sms ? tiles : c.num_sms;
@@ -397,12 +487,39 @@ bool launch(Ctx& c, const GemmDesc& g, int splits) {
     cudaFuncSetAttribute(k_gemm_tc<BN, A_MN, B_MN>, cudaFuncAttributeMaxDynamicSharedMemorySize, Cf::SMEM_BYTES);
     attr = true;
   }
-  LaunchScope s(c, "gemm_tc");
-  k_gemm_tc<BN, A_MN, B_MN><<<grid, kThreads, Cf::SMEM_BYTES, c.stream>>>(ma, mb, a);
+  LaunchScope s(c, g.name ? g.name : "gemm_tc");
+  k_gemm_tc<BN, A_MN, B_MN><<<grid, kThreads, Cf::SMEM_BYTES, c.stream>>>(ma, mb, mo, mo2, mi, a);
   return true;
 }
 
 }  // namespace
+
+// Tile width and split-K count from a simple cost model: MMA cycles per work
+// unit (k-blocks x cycles per k-block, 128-wide tiles paying for their lower
+// operand reuse), whole waves over the SMs, and the traffic of split-K
+// partials (written and read back once).
+TcPlan gemm_tc_plan(long M, long N, long K, bool split_ok, int num_sms) {
+  TcPlan best{256, 1};
+  double best_t = 1e30;
+  long nkb = (K + BK - 1) / BK;
+  for (int bn : {256, 128}) {
+    if (bn == 256 && N <= 128) continue;
+    long tiles = ((M + BM - 1) / BM) * ((N + bn - 1) / bn);
+    for (int s = 1; s <= 16; s++) {
+      if (s > 1 && (!split_ok || s > nkb / 8)) break;
+      long units = tiles * s;
+      long waves = (units + num_sms - 1) / num_sms;
+      double per_unit = (double)((nkb + s - 1) / s) * (bn == 256 ? 512.0 : 330.0) + bn * 12.0;
+      double t = waves * per_unit;
+      if (s > 1) t += 2.0 * s * M * N * 4 / (num_sms * 48.0);
+      if (t < best_t * 0.98) {
+        best_t = t;
+        best = TcPlan{bn, s};
+      }
+    }
+  }
+  return best;
+}
 
 bool gemm_tc_supported(const GemmDesc& g) {
   if (!get_encode()) return false;
@@ -413,28 +530,34 @@ bool gemm_tc_supported(const GemmDesc& g) {
   if (!g.b_kmajor && (g.N % 8)) return false;
   if (g.a_kmajor && (g.K % 8)) return false;
   if (g.b_kmajor && (g.K % 8)) return false;
-  // vector epilogue alignment
-  if (g.epi.ldo % 8 || (g.epi.kind == EPI_RESADD && g.epi.ld_res % 4)) return false;
+  if (g.N % 4) return false;  // fp32 output rows: 16-byte multiple
+  const GemmEpi& e = g.epi;
+  if (e.kind == EPI_RESADD) {
+    if (e.ld_res % 4 || (reinterpret_cast<uintptr_t>(e.res_in) & 15) || (reinterpret_cast<uintptr_t>(e.res_out) & 15))
+      return false;
+  } else {
+    if (e.ldo % 8 || (reinterpret_cast<uintptr_t>(e.out) & 15)) return false;
+  }
+  if (e.kind == EPI_BIAS_ACT && (reinterpret_cast<uintptr_t>(e.out2) & 15)) return false;
+  if (e.kind == EPI_ACT_BWD && (reinterpret_cast<uintptr_t>(e.aux) & 15)) return false;
+  if (e.bias && (reinterpret_cast<uintptr_t>(e.bias) & 15)) return false;
   if (!(g.a_kmajor && g.b_kmajor) && !(g.a_kmajor && !g.b_kmajor) && !(!g.a_kmajor && !g.b_kmajor)) return false;
   return true;
 }
 
 bool gemm_tc_bf16(Ctx& c, const GemmDesc& g) {
-  int num_m = (g.M + BM - 1) / BM;
-  int nkb = (g.K + BK - 1) / BK;
-  bool wide = (long)num_m * ((g.N + 255) / 256) >= c.num_sms && g.N >= 256;
-  int BNsel = wide ? 256 : 128;
-  int splits = 1;
-  if (g.epi.kind == EPI_ACC_F32 && g.partial && g.split_k > 1) {
-    splits = g.split_k;
-    if (splits > nkb) splits = nkb;
-    // keep every split non-empty
+  bool split_ok = g.epi.kind == EPI_ACC_F32 && g.partial && g.split_k > 1;
+  TcPlan plan = gemm_tc_plan(g.M, g.N, g.K, split_ok, c.num_sms);
+  int splits = plan.splits;
+  if (splits > g.split_k) splits = g.split_k < 1 ? 1 : g.split_k;  // never beyond the caller's scratch
+  if (splits > 1) {  // keep every split non-empty
+    int nkb = (g.K + BK - 1) / BK;
     int kbps = (nkb + splits - 1) / splits;
     splits = (nkb + kbps - 1) / kbps;
   }
   bool amn = !g.a_kmajor, bmn = !g.b_kmajor;
   bool ok;
-  if (BNsel == 256) {
+  if (plan.bn == 256) {
     if (!amn && !bmn) ok = launch<256, false, false>(c, g, splits);
     else if (!amn && bmn) ok = launch<256, false, true>(c, g, splits);
     else ok = launch<256, true, true>(c, g, splits);

@@ -506,13 +506,100 @@ __global__ void __launch_bounds__(512) k_ce_vec(T* __restrict__ logits, const in
   }
 }
 
+__device__ __forceinline__ float sfu_ex2(float x) {  // 2^x on the SFU (rel. error ~2^-22)
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ void lse_merge(float& m, float& s, float m2, float s2) {
+  float M = fmaxf(m, m2);
+  if (M == -INFINITY) return;
+  s = (m == -INFINITY ? 0.f : s * sfu_ex2(m - M)) + (m2 == -INFINITY ? 0.f : s2 * sfu_ex2(m2 - M));
+  m = M;
+}
+
+// Streaming variant, 256 threads per row and several rows per SM.  Pass 1
+// keeps an online (max, sum) of 2^(z log2 e) per thread over 16-byte vectors
+// (one rescale per vector); the block merges them into the row's
+// log-sum-exp.  Pass 2 re-reads the row (it is still in L2) and writes
+// (softmax - onehot) * scale.
+template <typename T>
+__global__ void __launch_bounds__(256, 4) k_ce_stream(T* __restrict__ logits, const int32_t* __restrict__ tgt, int V,
+                                                      int Vp, float* __restrict__ lse_out,
+                                                      float* __restrict__ row_loss, int want_grad, float scale) {
+  constexpr int EPV = 16 / sizeof(T);
+  constexpr float LOG2E = 1.4426950408889634f;
+  __shared__ float sm[8], ss[8];
+  const long row = blockIdx.x;
+  T* z = logits + row * Vp;
+  const int nvec = Vp / EPV;
+  const int t = tgt[row];
+  float zt = 0.f;
+  if (threadIdx.x == 0) zt = to_f<T>(z[t]);
+  float m = -INFINITY, s = 0.f;
+  for (int vi = threadIdx.x; vi < nvec; vi += 256) {
+    uint4 u = reinterpret_cast<const uint4*>(z)[vi];
+    const T* e = reinterpret_cast<const T*>(&u);
+    float x[EPV];
+    float mv = -INFINITY;
+#pragma unroll
+    for (int k = 0; k < EPV; k++) {
+      x[k] = (vi * EPV + k < V) ? to_f<T>(e[k]) * LOG2E : -INFINITY;
+      mv = fmaxf(mv, x[k]);
+    }
+    if (mv > m) {
+      s = (m == -INFINITY) ? 0.f : s * sfu_ex2(m - mv);
+      m = mv;
+    }
+#pragma unroll
+    for (int k = 0; k < EPV; k++) s += sfu_ex2(x[k] - m);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    float m2 = __shfl_xor_sync(0xffffffffu, m, o);
+    float s2 = __shfl_xor_sync(0xffffffffu, s, o);
+    lse_merge(m, s, m2, s2);
+  }
+  const int w = threadIdx.x >> 5;
+  if ((threadIdx.x & 31) == 0) {
+    sm[w] = m;
+    ss[w] = s;
+  }
+  __syncthreads();
+  float M = sm[0], S = ss[0];
+#pragma unroll
+  for (int k = 1; k < 8; k++) lse_merge(M, S, sm[k], ss[k]);
+  const float lse2 = M + log2f(S);  // log2-domain log-sum-exp
+  const float lse = lse2 * 0.6931471805599453f;
+  if (threadIdx.x == 0) {
+    lse_out[row] = lse;
+    row_loss[row] = lse - zt;
+  }
+  if (!want_grad) return;
+  __syncthreads();  // the target logit is read before any gradient is written
+  for (int vi = threadIdx.x; vi < nvec; vi += 256) {
+    uint4 u = reinterpret_cast<const uint4*>(z)[vi];
+    const T* e = reinterpret_cast<const T*>(&u);
+    uint4 outv;
+    T* o = reinterpret_cast<T*>(&outv);
+#pragma unroll
+    for (int k = 0; k < EPV; k++) {
+      const int j = vi * EPV + k;
+      float g = 0.f;
+      if (j < V) g = (sfu_ex2(fmaf(to_f<T>(e[k]), LOG2E, -lse2)) - (j == t ? 1.f : 0.f)) * scale;
+      o[k] = from_f<T>(g);
+    }
+    reinterpret_cast<uint4*>(z)[vi] = outv;
+  }
+}
+
 template <typename T>
 void ce_fwd_bwd(Ctx& c, T* logits, const int32_t* tgt, long M, int V, int Vp, float* lse, float* row_loss,
                 bool want_grad, float scale) {
   LaunchScope s(c, want_grad ? "ce_fwd_bwd" : "ce_fwd");
   constexpr int EPV = 16 / sizeof(T);
-  if (Vp % EPV == 0 && Vp / EPV <= 16 * 512)
-    k_ce_vec<T><<<(unsigned)M, 512, 0, c.stream>>>(logits, tgt, V, Vp, lse, row_loss, want_grad ? 1 : 0, scale);
+  if (Vp % EPV == 0)
+    k_ce_stream<T><<<(unsigned)M, 256, 0, c.stream>>>(logits, tgt, V, Vp, lse, row_loss, want_grad ? 1 : 0, scale);
   else
     k_ce<T><<<(unsigned)M, 512, 0, c.stream>>>(logits, tgt, V, Vp, lse, row_loss, want_grad ? 1 : 0, scale);
 }

@@ -67,9 +67,18 @@ struct GemmDesc {
   long ldb = 0;
   bool b_kmajor = true;       // true: B[n,k] at B[n*ldb + k]; false: at B[k*ldb + n]
   GemmEpi epi;
-  int split_k = 1;            // > 1 only with EPI_ACC_F32: partials in `partial`
+  int split_k = 1;            // > 1 only with EPI_ACC_F32: most splits `partial` holds
   float* partial = nullptr;   // [split_k, M, N] fp32 scratch
+  const char* name = nullptr; // timing label
 };
+
+// Tile width (256 or 128 columns) and split-K count the tensor-core GEMM uses
+// for an M x N x K problem on `num_sms` SMs (split_ok: fp32-accumulating dW).
+struct TcPlan {
+  int bn;
+  int splits;
+};
+TcPlan gemm_tc_plan(long M, long N, long K, bool split_ok, int num_sms);
 
 // fp32 operands on CUDA cores (fp32 mode); bf16 operands on CUDA cores
 // (reference path used by tests); bf16 operands on tcgen05 tensor cores.
