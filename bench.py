@@ -315,6 +315,45 @@ def run_ours(args, w, rank, world, local_rank):
     model.close()
 
 
+def run_kernels(w):
+    """One launch of each hot kernel at the workload's micro-batch shapes through
+    the kernel-level test entry points (the small case for ncu captures)."""
+    import torch
+
+    from gpt_decoder_lm_b200 import binding as gb
+    st = torch.cuda.current_stream().cuda_stream
+    flags = torch.zeros(1, dtype=torch.int32, device="cuda")
+    M, d, Vp = w.batch_size * w.block_size, w.n_embd, ((w.vocab_size + 63) // 64) * 64
+
+    def bf(*s):
+        return torch.randn(*s, device="cuda").bfloat16()
+
+    x, wqkv, wfc = bf(M, d), bf(3 * d, d), bf(4 * d, d)
+    qkv_out = torch.empty(M, 3 * d, dtype=torch.bfloat16, device="cuda")
+    h, g = (torch.empty(M, 4 * d, dtype=torch.bfloat16, device="cuda") for _ in range(2))
+    assert gb.test_gemm(2, M, 3 * d, d, x, d, 1, wqkv, d, 1, 1, 0, qkv_out, None, 3 * d, None, None, None, None,
+                        1, None, st, flags) == 0
+    assert gb.test_gemm(2, M, 4 * d, d, x, d, 1, wfc, d, 1, 2, 0, h, g, 4 * d, None, torch.zeros(4 * d, device="cuda"),
+                        None, None, 1, None, st, flags) == 0
+    wte = bf(Vp, d)
+    logits = torch.empty(M, Vp, dtype=torch.bfloat16, device="cuda")
+    assert gb.test_gemm(2, M, Vp, d, x, d, 1, wte, d, 1, 0, 0, logits, None, Vp, None, None, None, None, 1, None, st,
+                        flags) == 0
+    dwte = torch.zeros(Vp, d, device="cuda")
+    assert gb.test_gemm(2, Vp, d, M, logits, Vp, 0, x, d, 0, 5, 0, dwte, None, d, None, None, None, None, 1, None, st,
+                        flags) == 0
+    B, T, H = w.batch_size, w.block_size, w.n_head
+    q = bf(B, T, 3, H, 64)
+    o = torch.empty(B, T, H, 64, dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty(B, H, T, device="cuda")
+    do, dq, ds = bf(B, T, H, 64), torch.empty_like(q), torch.empty_like(lse)
+    assert gb.test_attention(1, 0, 1, B, T, H, 64, q, o, lse, stream=st, flags=flags) == 0
+    assert gb.test_attention(1, 1, 1, B, T, H, 64, q, o, lse, do, dq, ds, stream=st, flags=flags) == 0
+    torch.cuda.synchronize()
+    assert int(flags.item()) == 0
+    print(json.dumps({"kernels": "ok", "workload": w.name}))
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -323,8 +362,13 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default=W.GPT2_124M.name, choices=list(W.ALL))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--kernels", action="store_true",
+                    help="one launch of each hot kernel at the workload's shapes (for ncu), then exit")
     args = ap.parse_args()
     w = W.ALL[args.workload]
+    if args.kernels:
+        run_kernels(w)
+        return
     rank = int(os.environ.get("RANK", 0))
     world = int(os.environ.get("WORLD_SIZE", 1))
     local_rank = int(os.environ.get("LOCAL_RANK", 0))
