@@ -81,12 +81,27 @@ __device__ __forceinline__ double warp_sum_d(double v) {
   return v;
 }
 
-// GELU, exact erf form x * Phi(x), and its derivative Phi(x) + x phi(x).
-__device__ __forceinline__ float gelu_f(float x) { return 0.5f * x * (1.0f + erff(x * 0.70710678118654752f)); }
+// erf by Abramowitz & Stegun (1964), formula 7.1.26, |error| <= 1.5e-7:
+// for z >= 0, erf(z) = 1 - t (a1 + t (a2 + t (a3 + t (a4 + t a5)))) e^{-z^2},
+// t = 1 / (1 + p z); odd extension for z < 0.  Also returns e^{-z^2}.
+__device__ __forceinline__ float erf_as(float z, float& e) {
+  const float az = fabsf(z);
+  const float t = __fdividef(1.0f, fmaf(0.3275911f, az, 1.0f));
+  const float poly =
+      t * fmaf(t, fmaf(t, fmaf(t, fmaf(t, 1.061405429f, -1.453152027f), 1.421413741f), -0.284496736f), 0.254829592f);
+  e = __expf(-az * az);
+  return copysignf(fmaf(-poly, e, 1.0f), z);
+}
+// GELU, exact erf form x * Phi(x) with Phi(x) = (1 + erf(x / sqrt 2)) / 2, and
+// its derivative Phi(x) + x phi(x), phi(x) = e^{-x^2/2} / sqrt(2 pi).
+__device__ __forceinline__ float gelu_f(float x) {
+  float e;
+  return 0.5f * x * (1.0f + erf_as(x * 0.70710678118654752f, e));
+}
 __device__ __forceinline__ float gelu_grad_f(float x) {
-  float cdf = 0.5f * (1.0f + erff(x * 0.70710678118654752f));
-  float pdf = 0.3989422804014327f * expf(-0.5f * x * x);
-  return cdf + x * pdf;
+  float e;  // e^{-(x / sqrt 2)^2} = e^{-x^2 / 2}
+  const float cdf = 0.5f * (1.0f + erf_as(x * 0.70710678118654752f, e));
+  return fmaf(x * 0.3989422804014327f, e, cdf);
 }
 
 }  // namespace gpt

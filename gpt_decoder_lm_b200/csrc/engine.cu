@@ -118,7 +118,7 @@ struct gpt_model {
   float *row_loss, *row_lse;
   int32_t *idx, *tgt, *stage_idx, *stage_tgt;
   // backward scratch
-  float *dres, *dln, *dsum, *part, *colsum_scr, *splitk;
+  float *dres, *dln, *dsum, *part, *colsum_scr, *splitk, *seg;
   uint8_t *dyb, *dqkv, *datt, *dh;
   int32_t *stok, *spos, *nuniq;
   double* norm_part;
@@ -357,6 +357,7 @@ size_t carve(gpt_model& m, uint8_t* base) {
   m.dqkv = Bt((size_t)M * 3 * d);
   m.datt = Bt((size_t)M * d);
   m.dh = Bt((size_t)M * 4 * d);
+  m.seg = F((size_t)2 * ((M + 31) / 32) * d);
   m.stok = I(M);
   m.spos = I(M);
   m.nuniq = I(64);
@@ -656,7 +657,7 @@ gpt_status backward_t(gpt_model* m) {
     add_bias_grads_from_norm(m, y.ln1_w, y.ln1_b, l > 0 ? m->layers[l - 1].pr_b : -1);
   }
   embed_sort(c, m->idx, M, m->stok, m->spos, m->nuniq);
-  embed_bwd(c, m->dres, m->stok, m->spos, M, m->T, m->B, d, dkey(m, L, 0), m->G(m->wte), m->G(m->wpe));
+  embed_bwd(c, m->dres, m->stok, m->spos, M, m->T, m->B, d, dkey(m, L, 0), m->G(m->wte), m->G(m->wpe), m->seg);
   return check_cuda(m, "backward");
 }
 

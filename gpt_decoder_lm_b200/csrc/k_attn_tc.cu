@@ -275,6 +275,218 @@ __global__ void __launch_bounds__(192, 2) k_attn_fwd_tc(const __grid_constant__ 
 }
 
 // ============================================================================
+// forward, pipelined: one CTA per (128-query block, b, h), 64-key blocks.
+// S and P V are double-buffered in TMEM, so the MMA warp computes S of block
+// j+1 while the softmax warps work on block j, and the softmax warps fold the
+// P V product of block j-1 into O after handing over P of block j (deferred
+// rescaling: O <- O * alpha_{j-1} + PV_{j-1}).
+// smem: Q | (K, V)[3 stages] | P[2] | barriers   (96 KB + 256 B)
+// TMEM: S[2] cols [0,64), [64,128); PV[2] cols [128,192), [192,256)
+// ============================================================================
+constexpr int D_Q = 0, D_KV = TILE, D_P = 4 * TILE, D_BAR = 6 * TILE;
+constexpr int D_SMEM = D_BAR + 256;
+constexpr int D_STAGES = 3;
+
+__global__ void __launch_bounds__(192, 2) k_attn_fwd_db(const __grid_constant__ CUtensorMap tq,
+                                                        const __grid_constant__ CUtensorMap tkv64, AttnTcArgs a) {
+  extern __shared__ __align__(1024) uint8_t smem[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (smem_u32(smem) & 1023) {  // swizzled tiles need 1024-byte alignment
+    if (threadIdx.x == 0) atomicOr(a.flags, FLAG_TIMEOUT);
+    return;
+  }
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + D_BAR);
+  const uint32_t q_full = smem_u32(bars + 0);
+  const uint32_t kv_full0 = smem_u32(bars + 1), kv_empty0 = smem_u32(bars + 1 + D_STAGES);
+  const uint32_t s_full0 = smem_u32(bars + 1 + 2 * D_STAGES), p_full0 = s_full0 + 16, pv_full0 = s_full0 + 32;
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + 7 + 2 * D_STAGES);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tslot + 1);
+  const uint32_t sb = smem_u32(smem);
+
+  const int nqb = a.T / 128;
+  const int qb = nqb - 1 - (int)blockIdx.x;  // longest rows first
+  const int bh = blockIdx.y, b = bh / a.H, h = bh % a.H;
+  const int nkb = 2 * (qb + 1);  // 64-key blocks up to and including the diagonal
+  const int row0 = b * a.T;
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int s = 0; s < D_STAGES; s++) {
+      mbar_init(kv_full0 + 8 * s, 1);
+      mbar_init(kv_empty0 + 8 * s, 1);
+    }
+    for (int u = 0; u < 2; u++) {
+      mbar_init(s_full0 + 8 * u, 1);
+      mbar_init(p_full0 + 8 * u, 4);
+      mbar_init(pv_full0 + 8 * u, 1);
+    }
+    *abort_flag = 0;
+    fence_barrier_init();
+    prefetch_tmap(&tq);
+    prefetch_tmap(&tkv64);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tslot), 256);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tslot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      mbar_expect_tx(q_full, TILE);
+      tma_load_3d(sb + D_Q, &tq, q_full, 0, h, row0 + qb * 128);
+      for (int j = 0; j < nkb; j++) {
+        const int s = j % D_STAGES;
+        const uint32_t fb = kv_full0 + 8 * s;
+        if (!mbar_wait(kv_empty0 + 8 * s, ((j / D_STAGES) & 1) ^ 1, abort_flag, a.flags)) break;
+        mbar_expect_tx(fb, 2 * HTILE);
+        tma_load_3d(sb + D_KV + s * TILE, &tkv64, fb, 0, a.H + h, row0 + j * 64);
+        tma_load_3d(sb + D_KV + s * TILE + HTILE, &tkv64, fb, 0, 2 * a.H + h, row0 + j * 64);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t id_n64 = idesc_bf16_f32(128, 64, false, false);
+      constexpr uint32_t id_pv = idesc_bf16_f32(128, 64, false, true);
+      bool ok = mbar_wait(q_full, 0, abort_flag, a.flags);
+      // PV of block i: P[i&1] (K = 64 keys) times V of block i (MN-major, N = 64)
+      auto issue_pv = [&](int i) -> bool {
+        const int u = i & 1;
+        if (!mbar_wait(p_full0 + 8 * u, (i >> 1) & 1, abort_flag, a.flags)) return false;
+        tc_fence_after();
+        const uint32_t v = sb + D_KV + (i % D_STAGES) * TILE + HTILE;
+#pragma unroll
+        for (int kk = 0; kk < 4; kk++)
+          mma_bf16_ss(tmem + 128 + 64 * u, desc_k(sb + D_P + u * TILE, TILE, kk), desc_mn64(v, kk), id_pv, kk > 0);
+        mma_commit(pv_full0 + 8 * u);
+        mma_commit(kv_empty0 + 8 * (i % D_STAGES));
+        return true;
+      };
+      for (int j = 0; j < nkb && ok; j++) {
+        const int s = j % D_STAGES;
+        if (!(ok = mbar_wait(kv_full0 + 8 * s, (j / D_STAGES) & 1, abort_flag, a.flags))) break;
+        tc_fence_after();
+        // S[j&1] is free: its previous block's P (j-2) was waited for below
+#pragma unroll
+        for (int kk = 0; kk < 4; kk++)
+          mma_bf16_ss(tmem + 64 * (j & 1), desc_k(sb + D_Q, TILE, kk), desc_k(sb + D_KV + s * TILE, HTILE, kk), id_n64,
+                      kk > 0);
+        mma_commit(s_full0 + 8 * (j & 1));
+        if (j >= 1 && !(ok = issue_pv(j - 1))) break;
+      }
+      if (ok) issue_pv(nkb - 1);
+    }
+  } else {
+    const int quad = warp & 3;
+    const int r = quad * 32 + lane;
+    const int qi = qb * 128 + r;
+    const uint32_t trow = tmem + ((uint32_t)(quad * 32) << 16);
+    const float sl2 = a.scale_log2;
+    float m = -INFINITY, l = 0.f, alpha_prev = 0.f;
+    float o[64];
+#pragma unroll
+    for (int i = 0; i < 64; i++) o[i] = 0.f;
+    const uint64_t ebase = ((uint64_t)bh * a.T + qi) * a.T;
+    bool ok = true;
+    // O <- O * alpha + PV of block i
+    auto fold_pv = [&](int i, float alpha) -> bool {
+      const int u = i & 1;
+      if (!mbar_wait(pv_full0 + 8 * u, (i >> 1) & 1, abort_flag, a.flags)) return false;
+      tc_fence_after();
+      uint32_t v0[32], v1[32];
+      ld64(trow + 128 + 64 * u, v0, v1);
+#pragma unroll
+      for (int i2 = 0; i2 < 32; i2++) {
+        o[i2] = fmaf(o[i2], alpha, __uint_as_float(v0[i2]));
+        o[32 + i2] = fmaf(o[32 + i2], alpha, __uint_as_float(v1[i2]));
+      }
+      return true;
+    };
+    for (int j = 0; j < nkb; j++) {
+      const int u = j & 1;
+      if (!(ok = mbar_wait(s_full0 + 8 * u, (j >> 1) & 1, abort_flag, a.flags))) break;
+      tc_fence_after();
+      uint32_t v0[32], v1[32];
+      ld64(trow + 64 * u, v0, v1);
+      const int key0 = j * 64;
+      const bool diag = key0 + 63 > qb * 128;
+      float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
+      if (!diag) {
+#pragma unroll
+        for (int i = 0; i < 32; i += 2) {
+          mx0 = fmaxf(mx0, __uint_as_float(v0[i]));
+          mx1 = fmaxf(mx1, __uint_as_float(v0[i + 1]));
+          mx2 = fmaxf(mx2, __uint_as_float(v1[i]));
+          mx3 = fmaxf(mx3, __uint_as_float(v1[i + 1]));
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; i++) {
+          if (key0 + i <= qi) mx0 = fmaxf(mx0, __uint_as_float(v0[i]));
+          if (key0 + 32 + i <= qi) mx1 = fmaxf(mx1, __uint_as_float(v1[i]));
+        }
+      }
+      const float mn = fmaxf(m, fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2);
+      const float alpha = ex2(m - mn);  // 0 for the first block, 1 while the row is still empty
+      float ls0 = 0.f, ls1 = 0.f;
+      uint32_t pk0[16], pk1[16];
+#pragma unroll
+      for (int i = 0; i < 32; i += 2) {
+        float p0 = ex2(fmaf(__uint_as_float(v0[i]), sl2, -mn));
+        float p1 = ex2(fmaf(__uint_as_float(v0[i + 1]), sl2, -mn));
+        float p2 = ex2(fmaf(__uint_as_float(v1[i]), sl2, -mn));
+        float p3 = ex2(fmaf(__uint_as_float(v1[i + 1]), sl2, -mn));
+        if (diag) {
+          const int k = key0 + i;
+          if (k > qi) p0 = 0.f;
+          if (k + 1 > qi) p1 = 0.f;
+          if (k + 32 > qi) p2 = 0.f;
+          if (k + 33 > qi) p3 = 0.f;
+        }
+        ls0 += p0 + p1;
+        ls1 += p2 + p3;
+        if (a.drop.active) {
+          const uint64_t e = ebase + key0 + i;
+          p0 *= drop_mul(a.drop, e);
+          p1 *= drop_mul(a.drop, e + 1);
+          p2 *= drop_mul(a.drop, e + 32);
+          p3 *= drop_mul(a.drop, e + 33);
+        }
+        pk0[i >> 1] = pack2(p0, p1);
+        pk1[i >> 1] = pack2(p2, p3);
+      }
+      store_chunk32(sb + D_P + u * TILE, TILE, r, 0, pk0);
+      store_chunk32(sb + D_P + u * TILE, TILE, r, 1, pk1);
+      l = l * alpha + (ls0 + ls1);
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(p_full0 + 8 * u);  // one arrival per math warp
+      if (j >= 1 && !(ok = fold_pv(j - 1, alpha_prev))) break;
+      alpha_prev = alpha;
+      m = mn;
+    }
+    if (ok) ok = fold_pv(nkb - 1, alpha_prev);
+    if (ok) {
+      const float inv = 1.0f / l;
+      uint4* dst = reinterpret_cast<uint4*>(a.o_out + ((size_t)(row0 + qi) * a.H + h) * 64);
+#pragma unroll
+      for (int q = 0; q < 8; q++)
+        dst[q] = make_uint4(pack2(o[8 * q] * inv, o[8 * q + 1] * inv), pack2(o[8 * q + 2] * inv, o[8 * q + 3] * inv),
+                            pack2(o[8 * q + 4] * inv, o[8 * q + 5] * inv), pack2(o[8 * q + 6] * inv, o[8 * q + 7] * inv));
+      a.lse[(size_t)bh * a.T + qi] = (m + log2f(l)) * LN2;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, 256);
+}
+
+// ============================================================================
 // backward, dK and dV: one CTA per (128-key block, b, h), walking 64-query
 // blocks from the key block on.  Keys are the MMA rows:
 //   S^T = K Q^T, dP^T = V dO^T  ->  P~^T, dS^T (bf16, smem)
@@ -700,19 +912,20 @@ bool attn_tc_supported(const AttnDesc& a) {
 }
 
 void attn_fwd_tc(Ctx& c, const AttnDesc& d) {
-  CUtensorMap tm;
-  if (!map_rows(&tm, d.qkv, 3 * d.H, (long)d.B * d.T, 128)) {
+  CUtensorMap tq, tkv64;
+  long rows = (long)d.B * d.T;
+  if (!map_rows(&tq, d.qkv, 3 * d.H, rows, 128) || !map_rows(&tkv64, d.qkv, 3 * d.H, rows, 64)) {
     attn_fwd_simt<bf16>(c, d);
     return;
   }
   static bool attr = false;
   if (!attr) {
-    cudaFuncSetAttribute(k_attn_fwd_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, F_SMEM);
+    cudaFuncSetAttribute(k_attn_fwd_db, cudaFuncAttributeMaxDynamicSharedMemorySize, D_SMEM);
     attr = true;
   }
   dim3 grid(d.T / 128, d.B * d.H);
   LaunchScope s(c, "attn_fwd_tc");
-  k_attn_fwd_tc<<<grid, 192, F_SMEM, c.stream>>>(tm, make_args(d, c.flags));
+  k_attn_fwd_db<<<grid, 192, D_SMEM, c.stream>>>(tq, tkv64, make_args(d, c.flags));
 }
 
 void attn_bwd_tc(Ctx& c, const AttnDesc& d) {

@@ -38,6 +38,7 @@ constexpr int EPI_BUF = 4096;    // one 32x32 fp32 (or bf16) staging tile
 struct TcArgs {
   int M, N, K;
   int num_m, num_n, splits, kb_per_split, nkb;
+  int n_fast;  // tile order: 1 = N-fastest (concurrent CTAs share A tiles in L2), 0 = M-fastest
   int kind, act;
   const float* bias;
   DropKey drop;
@@ -178,7 +179,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
         int split = t / (p.num_m * p.num_n);
         int r = t % (p.num_m * p.num_n);
-        int mb = r % p.num_m, nb = r / p.num_m;
+        int mb = p.n_fast ? r / p.num_n : r % p.num_m, nb = p.n_fast ? r % p.num_n : r / p.num_m;
         int kb0 = split * p.kb_per_split, kb1 = min(p.nkb, kb0 + p.kb_per_split);
         for (int kb = kb0; kb < kb1; kb++) {
           if (!mbar_wait(smem_u32(&empty[stage]), phase ^ 1, abort_flag, p.flags)) {
@@ -280,7 +281,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
       int split = t / (p.num_m * p.num_n);
       int r = t % (p.num_m * p.num_n);
-      int mb = r % p.num_m, nb = r / p.num_m;
+      int mb = p.n_fast ? r / p.num_n : r % p.num_m, nb = p.n_fast ? r % p.num_n : r / p.num_m;
       if (!(ok = mbar_wait(smem_u32(&tfull[acc]), acc_phase, abort_flag, p.flags))) break;
       tc_fence_after();
       const int row0 = mb * BM + quad * 32;
@@ -472,6 +473,7 @@ bool launch(Ctx& c, const GemmDesc& g, int splits) {
   a.K = g.K;
   a.num_m = (g.M + BM - 1) / BM;
   a.num_n = (g.N + BN - 1) / BN;
+  a.n_fast = g.M > g.N ? 1 : 0;  // reuse the larger operand across neighbouring tiles
   a.nkb = (g.K + BK - 1) / BK;
   a.splits = splits;
   a.kb_per_split = (a.nkb + splits - 1) / splits;

@@ -285,6 +285,97 @@ __global__ void k_norm_bwd(NormBwd p) {
   }
 }
 
+// Warp-per-row variant for d <= 32 * 4 * VPL: the row lives in registers (VPL
+// float4 per lane), the row reductions are warp shuffles, and each lane keeps
+// the three column partials of its columns.  Warp w of block b takes rows
+// b*8 + w, b*8 + w + 8*gridDim, ...; at the end the 8 warps' partials are
+// added in warp order through shared memory, one slot at a time.
+template <typename T, int VPL>
+__global__ void __launch_bounds__(256) k_norm_bwd_warp(NormBwd p) {
+  extern __shared__ float red[];  // [8][d]
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int d = p.d, d4 = d >> 2;
+  float4 gw[VPL];
+#pragma unroll
+  for (int k = 0; k < VPL; k++) {
+    int c = lane + 32 * k;
+    gw[k] = (!p.rms && c < d4) ? reinterpret_cast<const float4*>(p.w)[c] : make_float4(1.f, 1.f, 1.f, 1.f);
+  }
+  float4 pg[VPL], pb[VPL], pn[VPL];
+#pragma unroll
+  for (int k = 0; k < VPL; k++) pg[k] = pb[k] = pn[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (long r = (long)blockIdx.x * 8 + w; r < p.rows; r += (long)gridDim.x * 8) {
+    const float mean = p.rms ? 0.f : p.mean[r];
+    const float rstd = p.rstd[r];
+    float4 dy[VPL], xh[VPL];
+    float s1 = 0.f, s2 = 0.f;
+#pragma unroll
+    for (int k = 0; k < VPL; k++) {
+      int c = lane + 32 * k;
+      if (c < d4) {
+        dy[k] = reinterpret_cast<const float4*>(p.dy + r * d)[c];
+        float4 x = reinterpret_cast<const float4*>(p.x + r * d)[c];
+        xh[k] = make_float4((x.x - mean) * rstd, (x.y - mean) * rstd, (x.z - mean) * rstd, (x.w - mean) * rstd);
+      } else {
+        dy[k] = xh[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+      const float g0 = dy[k].x * gw[k].x, g1 = dy[k].y * gw[k].y, g2 = dy[k].z * gw[k].z, g3 = dy[k].w * gw[k].w;
+      s1 += (g0 + g1) + (g2 + g3);
+      s2 += (g0 * xh[k].x + g1 * xh[k].y) + (g2 * xh[k].z + g3 * xh[k].w);
+    }
+    s1 = warp_sum(s1);
+    s2 = warp_sum(s2);
+    const float mg = p.rms ? 0.f : s1 / d, mgx = s2 / d;
+#pragma unroll
+    for (int k = 0; k < VPL; k++) {
+      int c = lane + 32 * k;
+      if (c >= d4) continue;
+      float4* dr = reinterpret_cast<float4*>(p.dres + r * d) + c;
+      float4 o = p.accumulate ? *dr : make_float4(0.f, 0.f, 0.f, 0.f);
+      float nv[4] = {o.x + rstd * (dy[k].x * gw[k].x - mg - xh[k].x * mgx),
+                     o.y + rstd * (dy[k].y * gw[k].y - mg - xh[k].y * mgx),
+                     o.z + rstd * (dy[k].z * gw[k].z - mg - xh[k].z * mgx),
+                     o.w + rstd * (dy[k].w * gw[k].w - mg - xh[k].w * mgx)};
+      *dr = make_float4(nv[0], nv[1], nv[2], nv[3]);
+      pg[k].x += dy[k].x * xh[k].x;
+      pg[k].y += dy[k].y * xh[k].y;
+      pg[k].z += dy[k].z * xh[k].z;
+      pg[k].w += dy[k].w * xh[k].w;
+      pb[k].x += dy[k].x;
+      pb[k].y += dy[k].y;
+      pb[k].z += dy[k].z;
+      pb[k].w += dy[k].w;
+      if (p.want_dyb) {
+        float q[4];
+#pragma unroll
+        for (int e = 0; e < 4; e++) q[e] = nv[e] * drop_mul(p.drop, (uint64_t)r * d + 4 * c + e);
+        pn[k].x += q[0];
+        pn[k].y += q[1];
+        pn[k].z += q[2];
+        pn[k].w += q[3];
+        store4<T>(reinterpret_cast<T*>(p.dyb) + r * d + 4 * c, make_float4(q[0], q[1], q[2], q[3]));
+      }
+    }
+  }
+  float* out = p.part + (long)blockIdx.x * 3 * d;
+#pragma unroll
+  for (int slot = 0; slot < 3; slot++) {
+#pragma unroll
+    for (int k = 0; k < VPL; k++) {
+      int c = lane + 32 * k;
+      if (c < d4) reinterpret_cast<float4*>(red + w * d)[c] = slot == 0 ? pg[k] : (slot == 1 ? pb[k] : pn[k]);
+    }
+    __syncthreads();
+    for (int j = threadIdx.x; j < d; j += 256) {
+      float s = 0.f;
+#pragma unroll
+      for (int k = 0; k < 8; k++) s += red[k * d + j];
+      out[slot * d + j] = s;
+    }
+    __syncthreads();
+  }
+}
+
 int norm_bwd_blocks(Ctx& c, long rows) {
   long b = (long)c.num_sms * 4;
   return (int)(rows < b ? rows : b);
@@ -293,9 +384,19 @@ int norm_bwd_blocks(Ctx& c, long rows) {
 template <typename T>
 void norm_bwd(Ctx& c, const NormBwd& p) {
   int d4 = p.d / 4;
+  int vpl = (d4 + 31) / 32;
+  LaunchScope s(c, "norm_bwd");
+  size_t smem = (size_t)8 * p.d * sizeof(float);
+  if (p.use_warp_rows && vpl <= 8) {  // register-heavy: one block per SM, kept for reference
+    if (vpl <= 1) k_norm_bwd_warp<T, 1><<<p.blocks, 256, smem, c.stream>>>(p);
+    else if (vpl <= 2) k_norm_bwd_warp<T, 2><<<p.blocks, 256, smem, c.stream>>>(p);
+    else if (vpl <= 4) k_norm_bwd_warp<T, 4><<<p.blocks, 256, smem, c.stream>>>(p);
+    else if (vpl <= 6) k_norm_bwd_warp<T, 6><<<p.blocks, 256, smem, c.stream>>>(p);
+    else k_norm_bwd_warp<T, 8><<<p.blocks, 256, smem, c.stream>>>(p);
+    return;
+  }
   int threads = ((d4 + 31) / 32) * 32;
   int nw = threads / 32;
-  LaunchScope s(c, "norm_bwd");
   k_norm_bwd<T><<<p.blocks, threads, 2 * nw * 2 * sizeof(float), c.stream>>>(p);
 }
 template void norm_bwd<float>(Ctx&, const NormBwd&);
@@ -359,6 +460,30 @@ __global__ void k_colsum(const T* __restrict__ x, long rows, int N, int chunks, 
   part[(long)blockIdx.y * N + j] = s;
 }
 
+// grad[j] += sum_c part[c, j]: row group y of 8 sums chunks y, y+8, ...; the
+// group sums are added in a fixed order
+__global__ void k_colsum_reduce(const float* __restrict__ part, int chunks, int N, float* __restrict__ grad) {
+  __shared__ float sh[8][33];
+  const int x = threadIdx.x, y = threadIdx.y;
+  const int j = blockIdx.x * 32 + x;
+  float s = 0.f;
+  if (j < N)
+    for (int k = y; k < chunks; k += 8) s += part[(long)k * N + j];
+  sh[y][x] = s;
+  __syncthreads();
+  if (y == 0 && j < N) {
+    float t = 0.f;
+#pragma unroll
+    for (int k = 0; k < 8; k++) t += sh[k][x];
+    grad[j] += t;
+  }
+}
+
+void colsum_reduce(Ctx& c, const float* part, int chunks, int N, float* grad) {
+  LaunchScope s(c, "colsum");
+  k_colsum_reduce<<<(N + 31) / 32, dim3(32, 8), 0, c.stream>>>(part, chunks, N, grad);
+}
+
 template <typename T>
 void colsum_acc(Ctx& c, const T* x, long rows, int N, float* scratch, float* grad) {
   int chunks = (int)min(64L, rows);
@@ -367,7 +492,7 @@ void colsum_acc(Ctx& c, const T* x, long rows, int N, float* scratch, float* gra
     dim3 grid((N + 127) / 128, chunks);
     k_colsum<T><<<grid, 128, 0, c.stream>>>(x, rows, N, chunks, scratch);
   }
-  partial_reduce(c, scratch, chunks, 1, 0, N, grad);
+  colsum_reduce(c, scratch, chunks, N, grad);
 }
 template void colsum_acc<float>(Ctx&, const float*, long, int, float*, float*);
 template void colsum_acc<bf16>(Ctx&, const bf16*, long, int, float*, float*);
@@ -687,48 +812,7 @@ void embed_sort(Ctx& c, const int32_t* idx, long M, int32_t* sorted_tok, int32_t
 }
 
 // dwte[v] += sum over the sorted positions of token v (in position order) of
-// drop0(dres[pos]); one block per sorted slot, active only at segment starts.
-// Warp w of the 8 sums the segment's rows w, w+8, ... (float4 columns per
-// lane); the 8 warp sums are added in warp order through shared memory.
-__global__ void __launch_bounds__(256) k_embed_bwd_wte(const float* __restrict__ dres,
-                                                       const int32_t* __restrict__ stok,
-                                                       const int32_t* __restrict__ spos, int M, int d, DropKey drop,
-                                                       float* __restrict__ dwte) {
-  extern __shared__ float wsum[];  // [8][d]
-  const int i = blockIdx.x;
-  const int tok = stok[i];
-  if (i > 0 && stok[i - 1] == tok) return;  // uniform per block
-  int end = i + 1;
-  while (end < M && stok[end] == tok) end++;
-  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int d4 = d >> 2;
-  for (int c4 = lane; c4 < d4; c4 += 32) {
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int j = i + w; j < end; j += 8) {
-      long p = spos[j];
-      float4 v = reinterpret_cast<const float4*>(dres + p * d)[c4];
-      if (drop.active) {
-        uint64_t e = (uint64_t)p * d + 4 * c4;
-        v.x *= drop_mul(drop, e);
-        v.y *= drop_mul(drop, e + 1);
-        v.z *= drop_mul(drop, e + 2);
-        v.w *= drop_mul(drop, e + 3);
-      }
-      acc.x += v.x;
-      acc.y += v.y;
-      acc.z += v.z;
-      acc.w += v.w;
-    }
-    reinterpret_cast<float4*>(wsum + w * d)[c4] = acc;
-  }
-  __syncthreads();
-  for (int c = threadIdx.x; c < d; c += blockDim.x) {
-    float s = 0.f;
-#pragma unroll
-    for (int k = 0; k < 8; k++) s += wsum[k * d + c];
-    dwte[(long)tok * d + c] += s;
-  }
-}
+// drop0(dres[pos]): the segmented sums of k_embed_seg_a / k_embed_seg_b below.
 
 // dwpe[t] += sum_b drop0(dres[b, t]) (b ascending)
 __global__ void k_embed_bwd_wpe(const float* __restrict__ dres, int Bn, int Tn, int d, DropKey drop,
@@ -744,17 +828,83 @@ __global__ void k_embed_bwd_wpe(const float* __restrict__ dres, int Bn, int Tn, 
   dwpe[i] += acc;
 }
 
+// Segment sums in fixed chunks of EC sorted slots.  Kernel A: one block per
+// chunk, threads across columns, rows in sorted order; a segment that lies
+// inside the chunk is added to dwte directly, the chunk's first segment when
+// it began in an earlier chunk goes to head[chunk], its last segment when it
+// continues into the next chunk goes to tail[chunk].  Kernel B: for every
+// segment that starts in chunk c and continues, dwte[tok] += tail[c] + the
+// heads of the following chunks it covers, in chunk order.
+constexpr int EC = 32;
+
+__global__ void __launch_bounds__(256) k_embed_seg_a(const float* __restrict__ dres, const int32_t* __restrict__ stok,
+                                                     const int32_t* __restrict__ spos, int M, int d, DropKey drop,
+                                                     float* __restrict__ dwte, float* __restrict__ head,
+                                                     float* __restrict__ tail) {
+  __shared__ int s_tok[EC + 2], s_pos[EC];
+  const int c = blockIdx.x;
+  const int j0 = c * EC, j1 = min(M, j0 + EC);
+  const int n = j1 - j0;
+  if (threadIdx.x < n) {
+    s_tok[threadIdx.x + 1] = stok[j0 + threadIdx.x];
+    s_pos[threadIdx.x] = spos[j0 + threadIdx.x];
+  }
+  if (threadIdx.x == 0) {
+    s_tok[0] = j0 > 0 ? stok[j0 - 1] : -1;
+    s_tok[n + 1] = j1 < M ? stok[j1] : -1;
+  }
+  __syncthreads();
+  for (int col = threadIdx.x; col < d; col += blockDim.x) {
+    float acc = 0.f;
+    for (int k = 0; k < n; k++) {
+      const long p = s_pos[k];
+      float v = dres[p * d + col];
+      if (drop.active) v *= drop_mul(drop, (uint64_t)p * d + col);
+      acc += v;
+      const int tok = s_tok[k + 1];
+      if (k == n - 1 || s_tok[k + 2] != tok) {  // segment ends here (or at the chunk edge)
+        int seg_lo = k;
+        while (seg_lo > 0 && s_tok[seg_lo] == tok) seg_lo--;  // first slot of the segment in the chunk
+        const bool began_before = seg_lo == 0 && s_tok[0] == tok;
+        const bool continues = k == n - 1 && s_tok[n + 1] == tok;
+        if (began_before) head[(long)c * d + col] = acc;
+        else if (continues) tail[(long)c * d + col] = acc;
+        else dwte[(long)tok * d + col] += acc;
+        acc = 0.f;
+      }
+    }
+  }
+}
+
+__global__ void k_embed_seg_b(const int32_t* __restrict__ stok, int M, int d, const float* __restrict__ head,
+                              const float* __restrict__ tail, float* __restrict__ dwte) {
+  const int c = blockIdx.x;
+  const int j0 = c * EC, j1 = min(M, j0 + EC);
+  const int tok = stok[j1 - 1];
+  if (j1 >= M || stok[j1] != tok) return;  // the chunk's last segment ends inside it
+  int k = j1 - 1;
+  while (k > j0 && stok[k - 1] == tok) k--;
+  if (k == j0 && j0 > 0 && stok[j0 - 1] == tok) return;  // began earlier: its start chunk sums it
+  for (int col = threadIdx.x; col < d; col += blockDim.x) {
+    float s = tail[(long)c * d + col];
+    for (int cc = c + 1; cc * EC < M; cc++) {
+      s += head[(long)cc * d + col];
+      const int e = min(M, (cc + 1) * EC);
+      if (e >= M || stok[e] != tok) break;
+    }
+    dwte[(long)tok * d + col] += s;
+  }
+}
+
 void embed_bwd(Ctx& c, const float* dres, const int32_t* sorted_tok, const int32_t* sorted_pos, long M, int Tn,
-               int Bn, int d, DropKey drop, float* dwte, float* dwpe) {
+               int Bn, int d, DropKey drop, float* dwte, float* dwpe, float* seg_scratch) {
   {
     LaunchScope s(c, "embed_bwd_wte");
-    size_t smem = (size_t)8 * d * sizeof(float);
-    static bool attr = false;
-    if (!attr) {
-      cudaFuncSetAttribute(k_embed_bwd_wte, cudaFuncAttributeMaxDynamicSharedMemorySize, 8 * 2048 * 4);
-      attr = true;
-    }
-    k_embed_bwd_wte<<<(unsigned)M, 256, smem, c.stream>>>(dres, sorted_tok, sorted_pos, (int)M, d, drop, dwte);
+    const int chunks = (int)((M + EC - 1) / EC);
+    float* head = seg_scratch;
+    float* tail = seg_scratch + (size_t)chunks * d;
+    k_embed_seg_a<<<chunks, 256, 0, c.stream>>>(dres, sorted_tok, sorted_pos, (int)M, d, drop, dwte, head, tail);
+    k_embed_seg_b<<<chunks, 256, 0, c.stream>>>(sorted_tok, (int)M, d, head, tail, dwte);
   }
   {
     LaunchScope s(c, "embed_bwd_wpe");

@@ -133,6 +133,7 @@ struct NormBwd {
   void* dyb; DropKey drop; bool want_dyb;
   float* part; int blocks;
   long rows; int d; bool rms;
+  bool use_warp_rows = false;  // warp-per-row kernel instead of the column-per-thread one
 };
 template <typename T> void norm_bwd(Ctx& c, const NormBwd& p);
 int norm_bwd_blocks(Ctx& c, long rows);
@@ -154,8 +155,11 @@ void loss_reduce(Ctx& c, const float* row_loss, long M, float scale, float* loss
 
 // embedding backward: routing (stable sort of positions by token) + sums
 void embed_sort(Ctx& c, const int32_t* idx, long M, int32_t* sorted_tok, int32_t* sorted_pos, int32_t* n_unique);
+// seg_scratch: 2 * ceil(M / 32) * d floats (partial sums of segments that cross 32-slot chunks)
 void embed_bwd(Ctx& c, const float* dres, const int32_t* sorted_tok, const int32_t* sorted_pos, long M, int Tn,
-               int Bn, int d, DropKey drop, float* dwte, float* dwpe);
+               int Bn, int d, DropKey drop, float* dwte, float* dwpe, float* seg_scratch);
+// column partials of colsum_acc [chunks, N] -> grad (+=), 8 row groups per column
+void colsum_reduce(Ctx& c, const float* part, int chunks, int N, float* grad);
 
 // grad norm partials, clip + AdamW
 void sumsq_partials(Ctx& c, const float* g, long n, double* partials, int blocks);

@@ -139,3 +139,20 @@ def test_tc_matches_simt_bitwise_close():
     ref = A @ B.T
     for o in (o1, o2):
         assert np.abs(o.double().cpu().numpy() - ref).max() / np.abs(ref).max() < 2e-6
+
+
+def test_gelu_epilogue_accuracy_fp32():
+    # fp32 operands on the CUDA-core GEMM: the GELU and GELU' epilogues against
+    # scipy's erf to well inside the fp32-mode gradient bound
+    M, N, K = 64, 256, 64
+    rng = np.random.default_rng(9)
+    A = rng.standard_normal((M, K)).astype(np.float32)
+    B = (rng.standard_normal((N, K)) * 0.4).astype(np.float32)
+    D = A.astype(np.float64) @ B.astype(np.float64).T
+    out = torch.empty((M, N), device="cuda")
+    out2 = torch.empty((M, N), device="cuda")
+    run(SIMT_F32, M, N, K, dev_f32(A), K, 1, dev_f32(B), K, 1, 2, act=0, out=out, out2=out2, ldo=N)
+    np.testing.assert_allclose(out2.double().cpu().numpy(), gelu(D), rtol=1e-5, atol=2e-6)
+    h = (rng.standard_normal((M, N)) * 3).astype(np.float32)
+    run(SIMT_F32, M, N, K, dev_f32(A), K, 1, dev_f32(B), K, 1, 4, act=0, out=out, ldo=N, aux=dev_f32(h))
+    np.testing.assert_allclose(out.double().cpu().numpy(), D * gelu_grad(h.astype(np.float64)), rtol=1e-5, atol=2e-6)
