@@ -87,6 +87,7 @@ _PROTOS = {
     "gpt_test_gemm": (I32, [I32, I32, I32, I32, P, I64, I32, P, I64, I32, I32, I32, P, P, I32, P, P, P, P, I32, P,
                             P, P]),
     "gpt_test_attention": (I32, [I32, I32, I32, I32, I32, I32, I32, P, P, P, P, P, P, F32, U64, U64, I32, P, P]),
+    "gpt_gemm_dw_accumulate_noalloc": (I32, [I32, I32, I32, P, I64, P, I64, P, I32, P]),
 }
 
 

@@ -248,6 +248,43 @@ uint64_t gpt_launch_count(gpt_model* m);
 const char* gpt_last_error(const gpt_model* m);
 const char* gpt_status_string(gpt_status s);
 
+/* ---------------------------------------------------------------- allocation-free entry point */
+
+/* The pages have no counterpart of this entry point: it exists for callers
+ * that cannot allocate device memory -- code inside a plugin or
+ * custom-operator interface that only hands over its input and output
+ * buffers, a process whose device memory belongs to another allocator or
+ * pool, or work that must not call cudaMalloc (it synchronises the device and
+ * cannot be issued while a stream is being captured).
+ *
+ * Weight-gradient GEMM of the training step, dW[M, N] += sum_k A[k, m] *
+ * B[k, n], on the tensor cores: A is bf16 [K, M] row-major with pitch lda,
+ * B is bf16 [K, N] with pitch ldb (the layouts of a layer's output gradient
+ * and input activations, tokens outermost), dW is fp32 [M, N] with pitch N.
+ * The contraction is split into split_k ranges whose partial sums go to a
+ * 16 MiB array inside the library (split_k * M * N <= 4,194,304 floats;
+ * larger requests return GPT_ERR_WORKSPACE_TOO_SMALL) and are added to dW in
+ * a fixed order, so the result matches the same GEMM run with caller-provided
+ * scratch.  Nothing is allocated: no cudaMalloc, cudaFree or allocating
+ * library call.
+ *   - The first call on a device (with that device current) looks up the
+ *     array's device address; make that first call before any stream capture.
+ *   - Every GPU that loads the library holds the array until the process
+ *     exits.  All calls share it and it keeps the last call's contents (every
+ *     partial sum is written before it is read, so nothing needs clearing);
+ *     calls whose GPU work overlaps -- on two streams at once, or from two
+ *     threads -- race on it.
+ *   - Work is enqueued on cuda_stream (a cudaStream_t) and the call
+ *     synchronises that stream before returning.
+ * Returns GPT_ERR_INVALID_ARG for bad sizes or NULL pointers,
+ * GPT_ERR_UNSUPPORTED when the shape or alignment does not suit the tensor
+ * cores (pitches multiple of 8, M and N multiple of 8, 16-byte aligned
+ * pointers), GPT_ERR_TIMEOUT if a bounded wait in the kernel ran out,
+ * GPT_ERR_CUDA for a CUDA failure. */
+gpt_status gpt_gemm_dw_accumulate_noalloc(int32_t M, int32_t N, int32_t K, const void* d_a, int64_t lda,
+                                          const void* d_b, int64_t ldb, float* d_dw, int32_t split_k,
+                                          void* cuda_stream);
+
 #ifdef __cplusplus
 }
 #endif

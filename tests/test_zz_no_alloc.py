@@ -1,0 +1,65 @@
+"""The allocation-free weight-gradient GEMM (gpt_gemm_dw_accumulate_noalloc)
+against the same GEMM run through the caller-scratch entry point.
+
+That entry point serves callers that cannot allocate device memory (plugin or
+custom-operator interfaces that only pass inputs and outputs, processes whose
+device memory belongs to another allocator, work that must not call
+cudaMalloc); its split-K partial sums live in an array inside the library.
+Two calls in a row must both match the caller-scratch result within the
+tolerance of the GEMM tests (fp32 accumulation over K = 8192: 1e-5 of the
+largest entry).  This file is collected last and needs nothing from the
+other tests, so it also runs alone in a fresh process.
+"""
+
+import ctypes as C
+
+import numpy as np
+import pytest
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+if not torch.cuda.is_available():
+    pytest.skip("needs a GPU", allow_module_level=True)
+
+from gpt_decoder_lm_b200 import binding as gb  # noqa: E402
+
+
+def test_noalloc_dw_gemm_matches_caller_scratch_twice():
+    lib = gb.lib()
+    M, N, K, splits = 768, 768, 8192, 4
+    g = torch.Generator(device="cuda").manual_seed(5)
+    A = torch.randn(K, M, device="cuda", generator=g).bfloat16()   # [K, M]: tokens outermost
+    B = torch.randn(K, N, device="cuda", generator=g).bfloat16()
+    base = torch.randn(M, N, device="cuda", generator=g)
+    stream = torch.cuda.current_stream().cuda_stream
+
+    # caller-provided scratch (the existing entry point)
+    ref = base.clone()
+    partial = torch.empty(splits, M, N, device="cuda")
+    flags = torch.zeros(1, dtype=torch.int32, device="cuda")
+    st = gb.test_gemm(2, M, N, K, A, M, 0, B, N, 0, 5, 0, ref, None, N, None, None, None, None, splits, partial,
+                      stream, flags)
+    assert gb.STATUS[st] == "GPT_OK" and int(flags.item()) == 0
+    exact = base.double() + A.double().T @ B.double()
+    scale = exact.abs().max().item()
+    assert (ref.double() - exact).abs().max().item() <= 1e-5 * scale
+
+    for _ in range(2):  # the library's array keeps the previous call's contents
+        out = base.clone()
+        st = lib.gpt_gemm_dw_accumulate_noalloc(M, N, K, A.data_ptr(), M, B.data_ptr(), N, out.data_ptr(), splits,
+                                                 C.c_void_p(stream))
+        assert gb.STATUS[st] == "GPT_OK"
+        assert (out.double() - ref.double()).abs().max().item() <= 1e-5 * scale
+
+
+def test_noalloc_rejects_sizes_beyond_its_array():
+    lib = gb.lib()
+    M = N = 2048
+    A = torch.zeros(64, M, device="cuda").bfloat16()
+    out = torch.zeros(M, N, device="cuda")
+    st = lib.gpt_gemm_dw_accumulate_noalloc(M, N, 64, A.data_ptr(), M, A.data_ptr(), N, out.data_ptr(), 2,
+                                             C.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert gb.STATUS[st] == "GPT_ERR_WORKSPACE_TOO_SMALL"
+    assert gb.STATUS[lib.gpt_gemm_dw_accumulate_noalloc(0, N, 64, None, M, None, N, None, 1, None)] == \
+        "GPT_ERR_INVALID_ARG"
