@@ -280,10 +280,13 @@ __global__ void __launch_bounds__(192, 2) k_attn_fwd_tc(const __grid_constant__ 
 // j+1 while the softmax warps work on block j, and the softmax warps fold the
 // P V product of block j-1 into O after handing over P of block j (deferred
 // rescaling: O <- O * alpha_{j-1} + PV_{j-1}).
-// smem: Q | (K, V)[3 stages] | P[2] | barriers   (96 KB + 256 B)
-// TMEM: S[2] cols [0,64), [64,128); PV[2] cols [128,192), [192,256)
+// smem: Q | (K, V)[3 stages] | barriers   (64 KB + 256 B)
+// TMEM: S[2] cols [0,64), [64,128); PV[2] cols [128,192), [192,256).  The
+// softmax warps overwrite the first 32 columns of S[u] with bf16 P, which the
+// P V MMA reads as its TMEM A operand (tcgen05 MMAs of one thread execute in
+// issue order, so S of block j+2 lands in S[u] only after P V of block j).
 // ============================================================================
-constexpr int D_Q = 0, D_KV = TILE, D_P = 4 * TILE, D_BAR = 6 * TILE;
+constexpr int D_Q = 0, D_KV = TILE, D_BAR = 4 * TILE;
 constexpr int D_SMEM = D_BAR + 256;
 constexpr int D_STAGES = 3;
 
@@ -360,7 +363,7 @@ __global__ void __launch_bounds__(192, 2) k_attn_fwd_db(const __grid_constant__ 
         const uint32_t v = sb + D_KV + (i % D_STAGES) * TILE + HTILE;
 #pragma unroll
         for (int kk = 0; kk < 4; kk++)
-          mma_bf16_ss(tmem + 128 + 64 * u, desc_k(sb + D_P + u * TILE, TILE, kk), desc_mn64(v, kk), id_pv, kk > 0);
+          mma_bf16_ts(tmem + 128 + 64 * u, tmem + 64 * u + 8 * kk, desc_mn64(v, kk), id_pv, kk > 0);
         mma_commit(pv_full0 + 8 * u);
         mma_commit(kv_empty0 + 8 * (i % D_STAGES));
         return true;
@@ -458,10 +461,11 @@ __global__ void __launch_bounds__(192, 2) k_attn_fwd_db(const __grid_constant__ 
         pk0[i >> 1] = pack2(p0, p1);
         pk1[i >> 1] = pack2(p2, p3);
       }
-      store_chunk32(sb + D_P + u * TILE, TILE, r, 0, pk0);
-      store_chunk32(sb + D_P + u * TILE, TILE, r, 1, pk1);
+      // P (bf16 pairs) over the first 32 columns of S[u]: the A operand of P V
+      tmem_st_32x32b_x16(trow + 64 * u, pk0);
+      tmem_st_32x32b_x16(trow + 64 * u + 16, pk1);
       l = l * alpha + (ls0 + ls1);
-      fence_proxy_async_smem();
+      tmem_st_wait();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(p_full0 + 8 * u);  // one arrival per math warp
@@ -491,11 +495,10 @@ __global__ void __launch_bounds__(192, 2) k_attn_fwd_db(const __grid_constant__ 
 // blocks from the key block on.  Keys are the MMA rows:
 //   S^T = K Q^T, dP^T = V dO^T  ->  P~^T, dS^T (bf16, smem)
 //   dV += P~^T dO,  dK += dS^T Q
-// smem: K | V | (Q, dO)[2 stages] | P^T | dS^T | (lse, D)[2] | barriers (~97 KB)
+// smem: K | V | (Q, dO)[2 stages] | (lse, D)[2] | barriers (~65 KB)
 // TMEM: S^T [0,64), dP^T [64,128), dV [128,192), dK [192,256)
 // ============================================================================
-constexpr int K_K = 0, K_V = TILE, K_ST = 2 * TILE, K_P = 4 * TILE, K_DS = 5 * TILE, K_LD = 6 * TILE,
-              K_BAR = K_LD + 1024;
+constexpr int K_K = 0, K_V = TILE, K_ST = 2 * TILE, K_LD = 4 * TILE, K_BAR = K_LD + 1024;
 constexpr int K_SMEM = K_BAR + 128;
 
 __global__ void __launch_bounds__(192, 2) k_attn_bwd_kv_tc(const __grid_constant__ CUtensorMap tkv,
@@ -583,10 +586,10 @@ __global__ void __launch_bounds__(192, 2) k_attn_bwd_kv_tc(const __grid_constant
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 4; kk++)
-          mma_bf16_ss(tmem + 128, desc_k(sb + K_P, TILE, kk), desc_mn64(dO, kk), id_acc, (it > 0 || kk > 0));
+          mma_bf16_ts(tmem + 128, tmem + 8 * kk, desc_mn64(dO, kk), id_acc, (it > 0 || kk > 0));
 #pragma unroll
         for (int kk = 0; kk < 4; kk++)
-          mma_bf16_ss(tmem + 192, desc_k(sb + K_DS, TILE, kk), desc_mn64(q, kk), id_acc, (it > 0 || kk > 0));
+          mma_bf16_ts(tmem + 192, tmem + 64 + 8 * kk, desc_mn64(q, kk), id_acc, (it > 0 || kk > 0));
         mma_commit(st_empty0 + 8 * s);
       }
       mma_commit(acc_full);
@@ -638,11 +641,13 @@ __global__ void __launch_bounds__(192, 2) k_attn_bwd_kv_tc(const __grid_constant
         pd0[e >> 1] = pack2(dsv[0], dsv[1]);
         pd1[e >> 1] = pack2(dsv[2], dsv[3]);
       }
-      store_chunk32(sb + K_P, TILE, r, 0, pp0);
-      store_chunk32(sb + K_P, TILE, r, 1, pp1);
-      store_chunk32(sb + K_DS, TILE, r, 0, pd0);
-      store_chunk32(sb + K_DS, TILE, r, 1, pd1);
-      fence_proxy_async_smem();
+      // P~^T over the first 32 columns of S^T, dS^T over those of dP^T (bf16
+      // pairs): the TMEM A operands of the dV and dK MMAs
+      tmem_st_32x32b_x16(trow, pp0);
+      tmem_st_32x32b_x16(trow + 16, pp1);
+      tmem_st_32x32b_x16(trow + 64, pd0);
+      tmem_st_32x32b_x16(trow + 80, pd1);
+      tmem_st_wait();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(pds_full);
@@ -678,10 +683,10 @@ __global__ void __launch_bounds__(192, 2) k_attn_bwd_kv_tc(const __grid_constant
 // ============================================================================
 // backward, dQ: one CTA per (128-query block, b, h), walking 64-key blocks
 // up to the diagonal.  S = Q K^T, dP = dO V^T -> dS (bf16, smem); dQ += dS K
-// smem: Q | dO | (K, V)[2 stages] | dS | barriers   (~80 KB)
+// smem: Q | dO | (K, V)[2 stages] | barriers   (~64 KB)
 // TMEM: S [0,64), dP [64,128), dQ [128,192)  (256 allocated)
 // ============================================================================
-constexpr int Q_Q = 0, Q_DO = TILE, Q_ST = 2 * TILE, Q_DS = 4 * TILE, Q_BAR = 5 * TILE;
+constexpr int Q_Q = 0, Q_DO = TILE, Q_ST = 2 * TILE, Q_BAR = 4 * TILE;
 constexpr int Q_SMEM = Q_BAR + 128;
 
 __global__ void __launch_bounds__(192, 2) k_attn_bwd_q_tc(const __grid_constant__ CUtensorMap tq,
@@ -764,7 +769,7 @@ __global__ void __launch_bounds__(192, 2) k_attn_bwd_q_tc(const __grid_constant_
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 4; kk++)
-          mma_bf16_ss(tmem + 128, desc_k(sb + Q_DS, TILE, kk), desc_mn64(k, kk), id_acc, (j > 0 || kk > 0));
+          mma_bf16_ts(tmem + 128, tmem + 8 * kk, desc_mn64(k, kk), id_acc, (j > 0 || kk > 0));
         mma_commit(kv_empty0 + 8 * s);
       }
       mma_commit(acc_full);
@@ -808,9 +813,10 @@ __global__ void __launch_bounds__(192, 2) k_attn_bwd_q_tc(const __grid_constant_
         pd0[e >> 1] = pack2(dsv[0], dsv[1]);
         pd1[e >> 1] = pack2(dsv[2], dsv[3]);
       }
-      store_chunk32(sb + Q_DS, TILE, r, 0, pd0);
-      store_chunk32(sb + Q_DS, TILE, r, 1, pd1);
-      fence_proxy_async_smem();
+      // dS (bf16 pairs) over the first 32 columns of S: the TMEM A operand of dQ += dS K
+      tmem_st_32x32b_x16(trow, pd0);
+      tmem_st_32x32b_x16(trow + 16, pd1);
+      tmem_st_wait();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(ds_full);
