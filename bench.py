@@ -86,6 +86,20 @@ class Clocks:
                                       stderr=subprocess.DEVNULL)
         except Exception:
             self.p = None
+        self.offset = 0
+
+    def wait_ready(self, timeout_s: float = 10.0):
+        """Block until nvidia-smi has written its first sample: its start-up (device
+        enumeration) must not overlap the timed region."""
+        t0 = time.time()
+        while self.p is not None and time.time() - t0 < timeout_s:
+            if os.path.getsize(self.f.name) > 0 or self.p.poll() is not None:
+                break
+            time.sleep(0.05)
+
+    def mark(self):
+        """Samples written before this call (warm-up) are left out of the summary."""
+        self.offset = os.path.getsize(self.f.name)
 
     def stop(self):
         if self.p is None:
@@ -96,7 +110,11 @@ class Clocks:
         except Exception:
             self.p.kill()
         self.f.flush()
-        rows = [l.split(",") for l in open(self.f.name).read().splitlines() if l.strip()]
+        text = open(self.f.name).read()
+        if self.offset:
+            nl = text.find("\n", self.offset - 1)
+            text = text[nl + 1:] if nl >= 0 else ""
+        rows = [l.split(",") for l in text.splitlines() if l.strip()]
         os.unlink(self.f.name)
         sm = []
         smax = None
@@ -204,23 +222,29 @@ def run_ours(args, w, rank, world, local_rank):
     def lr_at(i):
         return gb.lr_cosine(w.lr, i, 100, 5000)
 
+    # clock sampler first, so that its start-up falls before the timed region
+    clocks = Clocks(local_rank) if rank == 0 else None
+    if clocks:
+        clocks.wait_ready()
     # warm-up (untimed)
     for _ in range(args.warmup):
         st += 1
         model.train_step(d_stream, data_seed, lr_at(st), st, sync=False)
     torch.cuda.synchronize()
-    clocks = Clocks(local_rank) if rank == 0 else None
-    time.sleep(0.3)
+    if clocks:
+        clocks.mark()
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
     l0 = model.launch_count()
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     ev0.record()
+    h0 = time.perf_counter()
     for _ in range(args.steps):
         st += 1
         model.train_step(d_stream, data_seed, lr_at(st), st, sync=False)
         flush.zero_()          # L2 flush between steps (256 MiB > 126 MB L2)
+    host_enqueue_ms = (time.perf_counter() - h0) * 1000.0 / args.steps
     ev1.record()
     torch.cuda.synchronize()
     if world > 1:
@@ -253,6 +277,11 @@ def run_ours(args, w, rank, world, local_rank):
         xi = torch.from_numpy(stream_host[rows].astype(np.int32)).pin_memory()
         yi = torch.from_numpy(stream_host[rows + 1].astype(np.int32)).pin_memory()
         hb.append((xi, yi))
+    # untimed warm-up of the host-buffer entry point (its first calls run eagerly
+    # and capture its CUDA graph)
+    for xi, yi in hb[:2]:
+        st += 1
+        model.train_step_host(xi, yi, lr_at(st), st)
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
@@ -307,6 +336,7 @@ def run_ours(args, w, rank, world, local_rank):
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": 2 * ga * B * T * 4,
                     "d2h_bytes_per_step": 16},
             "gpu_launches": int(launches),
+            "host_enqueue_ms_per_step": host_enqueue_ms,
             "clocks": clk,
             "final_loss": loss, "final_grad_norm": norm,
             "kernels": kern,

@@ -64,6 +64,7 @@ _PROTOS = {
     "gpt_train_step_host": (I32, [P, P, P, F32, I32, P, P]),
     "gpt_gather_batch": (I32, [P, P, U64, U64, I32, I32, P, P]),
     "gpt_set_dropout_cursor": (I32, [P, I32, I32]),
+    "gpt_set_graphs": (I32, [P, I32]),
     "gpt_num_tensors": (I32, [P, P]),
     "gpt_tensor_info": (I32, [P, I32, P, P]),
     "gpt_get_tensor": (I32, [P, I32, I32, P]),
@@ -228,6 +229,10 @@ class Model:
 
     def set_dropout_cursor(self, step: int, micro: int):
         _check(lib().gpt_set_dropout_cursor(self.h, step, micro), self.h, "set_dropout_cursor")
+
+    def set_graphs(self, on: bool):
+        """CUDA-graph replay of train_step / train_step_host (default on)."""
+        _check(lib().gpt_set_graphs(self.h, 1 if on else 0), self.h, "set_graphs")
 
     # -- introspection
     def tensors(self) -> List[Tuple[str, Tuple[int, int]]]:

@@ -129,6 +129,16 @@ struct gpt_model {
 
   Ctx ctx;
   Timing* timing = nullptr;
+  // CUDA-graph replay of the full step: [0] device token stream, [1] host batches
+  bool graphs_on = true;
+  cudaStream_t cap_stream = nullptr;
+  cudaGraphExec_t gexec[2] = {nullptr, nullptr};
+  uint64_t graph_launches[2] = {0, 0};
+  int warm[2] = {0, 0};
+  const void* g_dstream = nullptr;
+  uint64_t g_len = 0, g_seed = 0;
+  int* step_dev = nullptr;     // per-step scalars read by replayed graphs
+  float* hyper_dev = nullptr;  // {lr, 1 - b1^t, 1 - b2^t}
   bool have_forward = false;
   bool ce_grad_done = false;
   int64_t drop_counter = 0;
@@ -339,7 +349,7 @@ size_t carve(gpt_model& m, uint8_t* base) {
   m.dsum = F((size_t)M * m.H);
   m.part_blocks = (int)std::min<long>(M, 148 * 8);
   m.part = F((size_t)m.part_blocks * 3 * d);
-  m.colsum_scr = F((size_t)64 * 4 * d);
+  m.colsum_scr = F((size_t)512 * 4 * d);
   // split-K scratch: the largest dW partial set
   size_t sk = 0;
   long shapes[4][2] = {{3L * d, d}, {d, d}, {4L * d, d}, {d, 4L * d}};
@@ -667,7 +677,7 @@ gpt_status forward_any(gpt_model* m, bool fuse, float* acc, float scale, int acc
 }
 gpt_status backward_any(gpt_model* m) { return m->bf16m ? backward_t<bf16>(m) : backward_t<float>(m); }
 
-gpt_status adamw_step(gpt_model* m, float lr, int step) {
+gpt_status adamw_step(gpt_model* m, float lr, int step, bool dev_params = false) {
   Ctx& c = m->ctx;
   int blocks = sumsq_blocks(c);
   sumsq_partials(c, m->g, m->n_total, m->norm_part, blocks);
@@ -690,8 +700,14 @@ gpt_status adamw_step(gpt_model* m, float lr, int step) {
   a.clip = m->cfg.grad_clip;
   a.bc1 = (float)(1.0 - pow((double)m->cfg.beta1, (double)step));
   a.bc2 = (float)(1.0 - pow((double)m->cfg.beta2, (double)step));
+  if (dev_params) a.hyper = m->hyper_dev;
   adamw(c, a);
   return check_cuda(m, "adamw");
+}
+
+void bias_corrections(const gpt_model* m, int step, float* bc1, float* bc2) {
+  *bc1 = (float)(1.0 - pow((double)m->cfg.beta1, (double)step));
+  *bc2 = (float)(1.0 - pow((double)m->cfg.beta2, (double)step));
 }
 
 }  // namespace
@@ -766,6 +782,8 @@ gpt_status gpt_create(const gpt_config* cfg, uint64_t seed, void* d_workspace, s
   m->ws_bytes = bytes;
   m->ctx.stream = (cudaStream_t)cuda_stream;
   m->ctx.flags = reinterpret_cast<uint32_t*>(m->scal + 3);
+  m->step_dev = reinterpret_cast<int*>(m->scal + 8);
+  m->hyper_dev = m->scal + 9;
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess) m->ctx.num_sms = sms;
@@ -798,8 +816,17 @@ gpt_status gpt_create(const gpt_config* cfg, uint64_t seed, void* d_workspace, s
 
 void gpt_destroy(gpt_model* m) {
   if (!m) return;
+  for (auto& e : m->gexec)
+    if (e) cudaGraphExecDestroy(e);
+  if (m->cap_stream) cudaStreamDestroy(m->cap_stream);
   delete m->timing;
   delete m;
+}
+
+gpt_status gpt_set_graphs(gpt_model* m, int32_t on) {
+  if (!m) return GPT_ERR_INVALID_ARG;
+  m->graphs_on = on != 0;
+  return GPT_OK;
 }
 
 gpt_status gpt_set_stream(gpt_model* m, void* st) {
@@ -848,15 +875,17 @@ gpt_status gpt_clip_adamw_step(gpt_model* m, float lr, int32_t step, float* h_gr
   return s;
 }
 
-static gpt_status train_common(gpt_model* m, const void* d_stream, uint64_t len, uint64_t seed, const int32_t* h_idx,
-                               const int32_t* h_tgt, float lr, int32_t step, float* h_loss, float* h_norm) {
-  if (step < 1) return fail(m, GPT_ERR_INVALID_ARG, "step must be >= 1");
+// The kernels of one optimiser step (grad_accum micro-batches, clip + AdamW).
+// dev_params: the step index, lr and bias corrections are read from device
+// memory (the form captured into a graph and replayed every step).
+static gpt_status train_body(gpt_model* m, const void* d_stream, uint64_t len, uint64_t seed, float lr, int32_t step,
+                             bool dev_params) {
   Ctx& c = m->ctx;
   for (int mu = 0; mu < m->ga; mu++) {
     m->drop_counter = (int64_t)step * m->ga + mu;
     if (d_stream) {
       gather_batch(c, d_stream, m->cfg.token_dtype == GPT_TOK_U16, len, seed, step, mu, m->B, m->T, m->V, m->idx,
-                   m->tgt);
+                   m->tgt, dev_params ? m->step_dev : nullptr);
     } else {
       int32_t* si = m->stage_idx + (size_t)mu * m->M;
       int32_t* stg = m->stage_tgt + (size_t)mu * m->M;
@@ -868,7 +897,77 @@ static gpt_status train_common(gpt_model* m, const void* d_stream, uint64_t len,
     if (s != GPT_OK) return s;
   }
   m->have_forward = false;
-  gpt_status s = adamw_step(m, lr, step);
+  return adamw_step(m, lr, step, dev_params);
+}
+
+// Captures train_body into a CUDA graph on an internal stream (the caller's
+// stream may be the legacy default stream, which cannot be captured).
+static bool capture_step(gpt_model* m, int kind, const void* d_stream, uint64_t len, uint64_t seed, float lr,
+                         int32_t step) {
+  if (!m->cap_stream && cudaStreamCreateWithFlags(&m->cap_stream, cudaStreamNonBlocking) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  cudaStream_t user = m->ctx.stream;
+  const uint64_t l0 = m->ctx.launches;
+  m->ctx.stream = m->cap_stream;
+  cudaGraph_t g = nullptr;
+  bool ok = cudaStreamBeginCapture(m->cap_stream, cudaStreamCaptureModeThreadLocal) == cudaSuccess;
+  gpt_status s = ok ? train_body(m, d_stream, len, seed, lr, step, true) : GPT_ERR_CUDA;
+  if (ok) ok = cudaStreamEndCapture(m->cap_stream, &g) == cudaSuccess && s == GPT_OK;
+  m->ctx.stream = user;
+  if (ok) ok = cudaGraphInstantiate(&m->gexec[kind], g, 0) == cudaSuccess;
+  if (g) cudaGraphDestroy(g);
+  m->graph_launches[kind] = m->ctx.launches - l0;
+  m->ctx.launches = l0;
+  if (!ok) {
+    cudaGetLastError();
+    m->gexec[kind] = nullptr;
+  }
+  return ok;
+}
+
+static gpt_status train_common(gpt_model* m, const void* d_stream, uint64_t len, uint64_t seed, const int32_t* h_idx,
+                               const int32_t* h_tgt, float lr, int32_t step, float* h_loss, float* h_norm) {
+  if (step < 1) return fail(m, GPT_ERR_INVALID_ARG, "step must be >= 1");
+  Ctx& c = m->ctx;
+  // Replay a captured graph of the whole step when nothing in it changes from
+  // step to step: no dropout (its masks depend on the step), no per-kernel
+  // timing.  The first call of each kind runs eagerly (one-time kernel
+  // attributes), the second captures, later calls only replay.
+  const int kind = d_stream ? 0 : 1;
+  bool replay = m->graphs_on && m->cfg.dropout == 0.f && !c.timing;
+  if (replay && kind == 0 && m->gexec[0] && (m->g_dstream != d_stream || m->g_len != len || m->g_seed != seed)) {
+    cudaGraphExecDestroy(m->gexec[0]);
+    m->gexec[0] = nullptr;
+    m->warm[0] = 0;
+  }
+  if (replay && !m->gexec[kind]) {
+    if (m->warm[kind] < 1) {
+      m->warm[kind]++;
+      replay = false;
+    } else if (capture_step(m, kind, d_stream, len, seed, lr, step)) {
+      if (kind == 0) {
+        m->g_dstream = d_stream;
+        m->g_len = len;
+        m->g_seed = seed;
+      }
+    } else {
+      m->graphs_on = false;  // capture not possible here: run every step eagerly
+      replay = false;
+    }
+  }
+  gpt_status s = GPT_OK;
+  if (replay) {
+    float bc1, bc2;
+    bias_corrections(m, step, &bc1, &bc2);
+    set_step_params(c, m->step_dev, m->hyper_dev, step, lr, bc1, bc2);
+    if (cudaGraphLaunch(m->gexec[kind], c.stream) != cudaSuccess) return check_cuda(m, "graph launch");
+    c.launches += m->graph_launches[kind];
+    m->have_forward = false;
+  } else {
+    s = train_body(m, d_stream, len, seed, lr, step, false);
+  }
   if (s != GPT_OK) return s;
   if (h_loss || h_norm) {
     float sc[4];

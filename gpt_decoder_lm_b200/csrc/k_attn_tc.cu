@@ -12,10 +12,10 @@
 // Every kernel: warp 0 issues TMA loads of bf16 tiles (128-byte swizzle) from
 // the [B*T, 3, H, 64] qkv activations, warp 1 owns TMEM and issues
 // tcgen05.mma, warps 2..5 (one TMEM lane / tile row per thread) do the softmax
-// arithmetic, write bf16 probability tiles to shared memory as the A operand
-// of the next MMA, and run the epilogue.  Each kernel keeps its TMEM at 256
-// columns and its shared memory under 113 KB so that two CTAs share an SM:
-// one CTA's softmax overlaps the other's MMAs.
+// arithmetic, write the bf16 probability (or dS) tile back into TMEM, where the
+// next MMA reads it as its A operand, and run the epilogue.  Each kernel keeps
+// its TMEM at 256 columns and its shared memory under 113 KB so that two CTAs
+// share an SM: one CTA's softmax overlaps the other's MMAs.
 #include <cudaTypedefs.h>
 
 #include <mutex>
@@ -56,17 +56,6 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
-// Row r, 32-column chunk c of a K-major bf16 operand tile whose K extent is
-// split in 64-wide K-blocks of kb_bytes each (128 rows x 128 bytes, or 64).
-__device__ __forceinline__ void store_chunk32(uint32_t tile, int kb_bytes, int r, int c, const uint32_t (&pk)[16]) {
-  uint32_t rowbase = tile + (c >> 1) * kb_bytes + r * 128;
-#pragma unroll
-  for (int q = 0; q < 4; q++) {
-    int chunk = (c & 1) * 4 + q;
-    st_shared_v4(rowbase + ((chunk ^ (r & 7)) << 4), pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
-  }
-}
-
 // K-major operand: K-step kk (16 elements) of a tile with 64-wide K-blocks
 __device__ __forceinline__ uint64_t desc_k(uint32_t tile, int kb_bytes, int kk) {
   return desc_sw128(tile + (kk >> 2) * kb_bytes + (kk & 3) * 32, 16, 1024);
@@ -78,200 +67,6 @@ __device__ __forceinline__ void ld64(uint32_t taddr, uint32_t (&a)[32], uint32_t
   tmem_ld_32x32b_x32(taddr, a);
   tmem_ld_32x32b_x32(taddr + 32, b);
   tmem_ld_wait();
-}
-
-// ============================================================================
-// forward: one CTA per (128-query block, b, h), 128-key blocks
-// smem: Q | K[2] | V[2] | P (2 K-blocks) | barriers   (112 KB + 128 B)
-// TMEM: S cols [0,128), PV cols [128,192)  (256 allocated)
-// ============================================================================
-constexpr int F_Q = 0, F_K = TILE, F_V = 3 * TILE, F_P = 5 * TILE, F_BAR = 7 * TILE;
-constexpr int F_SMEM = F_BAR + 128;
-
-__global__ void __launch_bounds__(192, 2) k_attn_fwd_tc(const __grid_constant__ CUtensorMap tm, AttnTcArgs a) {
-  extern __shared__ __align__(1024) uint8_t smem[];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if (smem_u32(smem) & 1023) {  // swizzled tiles need 1024-byte alignment
-    if (threadIdx.x == 0) atomicOr(a.flags, FLAG_TIMEOUT);
-    return;
-  }
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + F_BAR);
-  uint32_t q_full = smem_u32(bars + 0), kv_full0 = smem_u32(bars + 1), kv_empty0 = smem_u32(bars + 3);
-  uint32_t s_full = smem_u32(bars + 5), p_full = smem_u32(bars + 6), pv_full = smem_u32(bars + 7);
-  uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + 8);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(tslot + 1);
-  const uint32_t sb = smem_u32(smem);
-
-  const int nqb = a.T / 128;
-  const int qb = nqb - 1 - (int)blockIdx.x;  // longest rows first
-  const int bh = blockIdx.y, b = bh / a.H, h = bh % a.H;
-  const int nkb = qb + 1;
-  const int row0 = b * a.T;
-
-  if (threadIdx.x == 0) {
-    mbar_init(q_full, 1);
-    mbar_init(kv_full0, 1);
-    mbar_init(kv_full0 + 8, 1);
-    mbar_init(kv_empty0, 1);
-    mbar_init(kv_empty0 + 8, 1);
-    mbar_init(s_full, 1);
-    mbar_init(p_full, 4);
-    mbar_init(pv_full, 1);
-    *abort_flag = 0;
-    fence_barrier_init();
-    prefetch_tmap(&tm);
-  }
-  if (warp == 1) {
-    tmem_alloc(smem_u32(tslot), 256);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tslot;
-
-  if (warp == 0) {
-    if (lane == 0) {
-      mbar_expect_tx(q_full, TILE);
-      tma_load_3d(sb + F_Q, &tm, q_full, 0, h, row0 + qb * 128);
-      for (int j = 0; j < nkb; j++) {
-        int s = j & 1;
-        if (!mbar_wait(kv_empty0 + 8 * s, ((j >> 1) & 1) ^ 1, abort_flag, a.flags)) break;
-        mbar_expect_tx(kv_full0 + 8 * s, 2 * TILE);
-        tma_load_3d(sb + F_K + s * TILE, &tm, kv_full0 + 8 * s, 0, a.H + h, row0 + j * 128);
-        tma_load_3d(sb + F_V + s * TILE, &tm, kv_full0 + 8 * s, 0, 2 * a.H + h, row0 + j * 128);
-      }
-    }
-  } else if (warp == 1) {
-    if (lane == 0) {
-      constexpr uint32_t id_s = idesc_bf16_f32(128, 128, false, false);
-      constexpr uint32_t id_pv = idesc_bf16_f32(128, 64, false, true);
-      bool ok = mbar_wait(q_full, 0, abort_flag, a.flags);
-      for (int j = 0; j < nkb && ok; j++) {
-        int s = j & 1;
-        if (!(ok = mbar_wait(kv_full0 + 8 * s, (j >> 1) & 1, abort_flag, a.flags))) break;
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < 4; kk++)
-          mma_bf16_ss(tmem, desc_k(sb + F_Q, TILE, kk), desc_k(sb + F_K + s * TILE, TILE, kk), id_s, kk > 0);
-        mma_commit(s_full);
-        if (!(ok = mbar_wait(p_full, j & 1, abort_flag, a.flags))) break;
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < 8; kk++)
-          mma_bf16_ss(tmem + 128, desc_k(sb + F_P, TILE, kk), desc_mn64(sb + F_V + s * TILE, kk), id_pv, kk > 0);
-        mma_commit(pv_full);
-        mma_commit(kv_empty0 + 8 * s);
-      }
-    }
-  } else {
-    const int quad = warp & 3;
-    const int r = quad * 32 + lane;
-    const int qi = qb * 128 + r;
-    const uint32_t trow = tmem + ((uint32_t)(quad * 32) << 16);
-    const float sl2 = a.scale_log2;
-    float m = -INFINITY, l = 0.f;
-    float o[64];
-#pragma unroll
-    for (int i = 0; i < 64; i++) o[i] = 0.f;
-    const uint64_t ebase = ((uint64_t)bh * a.T + qi) * a.T;
-    bool ok = true;
-    for (int j = 0; j < nkb; j++) {
-      if (!(ok = mbar_wait(s_full, j & 1, abort_flag, a.flags))) break;
-      tc_fence_after();
-      const bool diag = (j == qb);
-      const int key0 = j * 128;
-      // pass 1: row maximum of the raw scores (scale > 0 commutes with max)
-      float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
-#pragma unroll 1
-      for (int c = 0; c < 4; c += 2) {
-        uint32_t v0[32], v1[32];
-        ld64(trow + c * 32, v0, v1);
-        if (!diag) {
-#pragma unroll
-          for (int i = 0; i < 32; i += 2) {
-            mx0 = fmaxf(mx0, __uint_as_float(v0[i]));
-            mx1 = fmaxf(mx1, __uint_as_float(v0[i + 1]));
-            mx2 = fmaxf(mx2, __uint_as_float(v1[i]));
-            mx3 = fmaxf(mx3, __uint_as_float(v1[i + 1]));
-          }
-        } else {
-#pragma unroll
-          for (int i = 0; i < 32; i++) {
-            if (key0 + c * 32 + i <= qi) mx0 = fmaxf(mx0, __uint_as_float(v0[i]));
-            if (key0 + c * 32 + 32 + i <= qi) mx1 = fmaxf(mx1, __uint_as_float(v1[i]));
-          }
-        }
-      }
-      const float mn = fmaxf(m, fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2);
-      const float alpha = ex2(m - mn);
-      float ls0 = 0.f, ls1 = 0.f;
-      // pass 2: probabilities -> bf16 A operand of P V
-#pragma unroll 1
-      for (int c = 0; c < 4; c += 2) {
-        uint32_t v0[32], v1[32];
-        ld64(trow + c * 32, v0, v1);
-        uint32_t pk0[16], pk1[16];
-#pragma unroll
-        for (int i = 0; i < 32; i += 2) {
-          float p0 = ex2(fmaf(__uint_as_float(v0[i]), sl2, -mn));
-          float p1 = ex2(fmaf(__uint_as_float(v0[i + 1]), sl2, -mn));
-          float p2 = ex2(fmaf(__uint_as_float(v1[i]), sl2, -mn));
-          float p3 = ex2(fmaf(__uint_as_float(v1[i + 1]), sl2, -mn));
-          if (diag) {
-            int k = key0 + c * 32 + i;
-            if (k > qi) p0 = 0.f;
-            if (k + 1 > qi) p1 = 0.f;
-            if (k + 32 > qi) p2 = 0.f;
-            if (k + 33 > qi) p3 = 0.f;
-          }
-          ls0 += p0 + p1;
-          ls1 += p2 + p3;
-          if (a.drop.active) {
-            uint64_t e = ebase + key0 + c * 32 + i;
-            p0 *= drop_mul(a.drop, e);
-            p1 *= drop_mul(a.drop, e + 1);
-            p2 *= drop_mul(a.drop, e + 32);
-            p3 *= drop_mul(a.drop, e + 33);
-          }
-          pk0[i >> 1] = pack2(p0, p1);
-          pk1[i >> 1] = pack2(p2, p3);
-        }
-        store_chunk32(sb + F_P, TILE, r, c, pk0);
-        store_chunk32(sb + F_P, TILE, r, c + 1, pk1);
-      }
-      l = l * alpha + (ls0 + ls1);
-      fence_proxy_async_smem();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(p_full);  // one arrival per math warp
-      if (!(ok = mbar_wait(pv_full, j & 1, abort_flag, a.flags))) break;
-      tc_fence_after();
-      {
-        uint32_t v0[32], v1[32];
-        ld64(trow + 128, v0, v1);
-#pragma unroll
-        for (int i = 0; i < 32; i++) {
-          o[i] = fmaf(o[i], alpha, __uint_as_float(v0[i]));
-          o[32 + i] = fmaf(o[32 + i], alpha, __uint_as_float(v1[i]));
-        }
-      }
-      m = mn;
-    }
-    if (ok) {
-      const float inv = 1.0f / l;
-      uint4* dst = reinterpret_cast<uint4*>(a.o_out + ((size_t)(row0 + qi) * a.H + h) * 64);
-#pragma unroll
-      for (int q = 0; q < 8; q++)
-        dst[q] = make_uint4(pack2(o[8 * q] * inv, o[8 * q + 1] * inv), pack2(o[8 * q + 2] * inv, o[8 * q + 3] * inv),
-                            pack2(o[8 * q + 4] * inv, o[8 * q + 5] * inv), pack2(o[8 * q + 6] * inv, o[8 * q + 7] * inv));
-      a.lse[(size_t)bh * a.T + qi] = (m + log2f(l)) * LN2;
-    }
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  if (warp == 1) tmem_dealloc(tmem, 256);
 }
 
 // ============================================================================
@@ -493,7 +288,7 @@ __global__ void __launch_bounds__(192, 2) k_attn_fwd_db(const __grid_constant__ 
 // ============================================================================
 // backward, dK and dV: one CTA per (128-key block, b, h), walking 64-query
 // blocks from the key block on.  Keys are the MMA rows:
-//   S^T = K Q^T, dP^T = V dO^T  ->  P~^T, dS^T (bf16, smem)
+//   S^T = K Q^T, dP^T = V dO^T  ->  P~^T, dS^T (bf16, written into TMEM)
 //   dV += P~^T dO,  dK += dS^T Q
 // smem: K | V | (Q, dO)[2 stages] | (lse, D)[2] | barriers (~65 KB)
 // TMEM: S^T [0,64), dP^T [64,128), dV [128,192), dK [192,256)
@@ -682,7 +477,7 @@ __global__ void __launch_bounds__(192, 2) k_attn_bwd_kv_tc(const __grid_constant
 
 // ============================================================================
 // backward, dQ: one CTA per (128-query block, b, h), walking 64-key blocks
-// up to the diagonal.  S = Q K^T, dP = dO V^T -> dS (bf16, smem); dQ += dS K
+// up to the diagonal.  S = Q K^T, dP = dO V^T -> dS (bf16, written into TMEM); dQ += dS K
 // smem: Q | dO | (K, V)[2 stages] | barriers   (~64 KB)
 // TMEM: S [0,64), dP [64,128), dQ [128,192)  (256 allocated)
 // ============================================================================
@@ -844,21 +639,32 @@ __global__ void __launch_bounds__(192, 2) k_attn_bwd_q_tc(const __grid_constant_
   if (warp == 1) tmem_dealloc(tmem, 256);
 }
 
-// D[b,h,i] = sum_d dO[b,i,h,d] * O[b,i,h,d]: one warp per (row, head), 2 elements per lane
+// D[b,h,i] = sum_d dO[b,i,h,d] * O[b,i,h,d]: 8 lanes per (row, head), 8
+// elements (16 bytes) per lane, so a warp covers four heads
 __global__ void k_attn_dsum64(const bf16* __restrict__ o, const bf16* __restrict__ dout, int B, int T, int H,
                               float* __restrict__ dsum) {
-  long w = ((long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  int lane = threadIdx.x & 31;
-  if (w >= (long)B * T * H) return;
-  long row = w / H;  // b*T + t
-  int h = (int)(w % H);
-  const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(o + (row * H + h) * 64);
-  const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(dout + (row * H + h) * 64);
-  float2 x = __bfloat1622float2(a2[lane]);
-  float2 y = __bfloat1622float2(b2[lane]);
-  float s = warp_sum(x.x * y.x + x.y * y.y);
-  if (lane == 0) {
-    long b = row / T, t = row % T;
+  const long g = ((long)blockIdx.x * blockDim.x + threadIdx.x) >> 3;  // (row, head) index
+  const int sub = threadIdx.x & 7;
+  const bool valid = g < (long)B * T * H;
+  float s = 0.f;
+  if (valid) {
+    uint4 a = reinterpret_cast<const uint4*>(o + g * 64)[sub];
+    uint4 d = reinterpret_cast<const uint4*>(dout + g * 64)[sub];
+    const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&a);
+    const __nv_bfloat162* d2 = reinterpret_cast<const __nv_bfloat162*>(&d);
+#pragma unroll
+    for (int k = 0; k < 4; k++) {
+      float2 x = __bfloat1622float2(a2[k]), y = __bfloat1622float2(d2[k]);
+      s = fmaf(x.x, y.x, fmaf(x.y, y.y, s));
+    }
+  }
+  s += __shfl_xor_sync(0xffffffffu, s, 1);
+  s += __shfl_xor_sync(0xffffffffu, s, 2);
+  s += __shfl_xor_sync(0xffffffffu, s, 4);
+  if (valid && sub == 0) {
+    const long row = g / H;  // b*T + t
+    const int h = (int)(g % H);
+    const long b = row / T, t = row % T;
     dsum[(b * H + h) * T + t] = s;
   }
 }
@@ -944,9 +750,9 @@ void attn_bwd_tc(Ctx& c, const AttnDesc& d) {
   }
   tq64 = tkv64;
   {
-    long warps = (long)d.B * d.T * d.H;
+    long groups = (long)d.B * d.T * d.H;  // 8 threads each
     LaunchScope s(c, "attn_bwd_dsum");
-    k_attn_dsum64<<<(unsigned)((warps * 32 + 255) / 256), 256, 0, c.stream>>>(
+    k_attn_dsum64<<<(unsigned)((groups * 8 + 255) / 256), 256, 0, c.stream>>>(
         reinterpret_cast<const bf16*>(d.o), reinterpret_cast<const bf16*>(d.dout), d.B, d.T, d.H, d.dsum);
   }
   static bool attr = false;

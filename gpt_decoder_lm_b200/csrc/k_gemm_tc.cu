@@ -31,9 +31,11 @@ namespace {
 using namespace sm100;
 
 constexpr int BM = 128, BK = 64;
-constexpr int kThreads = 320;    // producer, MMA, 8 epilogue warps
-constexpr int EPI_WARPS = 8;
-constexpr int EPI_BUF = 4096;    // one 32x32 fp32 (or bf16) staging tile
+constexpr int EPI_WARPS = 16;                // 4 per TMEM lane quadrant
+constexpr int EPI_PARTS = EPI_WARPS / 4;     // column ranges per quadrant
+constexpr int EPI_SETS = 1;                  // staging sets per epilogue warp (2 = double-buffered)
+constexpr int kThreads = 64 + 32 * EPI_WARPS;  // producer, MMA, epilogue warps
+constexpr int EPI_BUF = 4096;                // one 32x32 fp32 (or two bf16) staging tiles
 
 struct TcArgs {
   int M, N, K;
@@ -53,7 +55,7 @@ struct TcCfg {
   static constexpr int STAGES = BN == 256 ? 3 : 5;
   static constexpr int TMEM_COLS = 2 * BN;
   static constexpr int EPI_OFF = STAGES * STAGE_BYTES;
-  static constexpr int BAR_OFF = EPI_OFF + EPI_WARPS * 2 * EPI_BUF;
+  static constexpr int BAR_OFF = EPI_OFF + EPI_WARPS * EPI_SETS * EPI_BUF;
   static constexpr int SMEM_BYTES = BAR_OFF + 512 + 1024;  // + barriers + alignment slack
 };
 
@@ -264,12 +266,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    const int ew = warp - 2;          // 0..7
+    const int ew = warp - 2;          // 0 .. EPI_WARPS-1
     const int quad = warp & 3;        // TMEM lanes quad*32 .. quad*32+31
-    const int half = ew >> 2;         // which half of the BN columns
-    // two 4 KB staging sets per warp, used by alternate chunks: a set holds one
-    // fp32 tile, or two bf16 tiles (A at +0, B at +2 KB)
-    const uint32_t stg = smem_u32(smem + C::EPI_OFF + ew * 2 * EPI_BUF);
+    const int part = ew >> 2;         // which of the EPI_PARTS column ranges
+    constexpr int CPW = BN / 32 / EPI_PARTS;  // 32-column chunks per warp and tile
+    // EPI_SETS 4 KB staging sets per warp, used by consecutive chunks in turn:
+    // a set holds one fp32 tile, or two bf16 tiles (A at +0, B at +2 KB)
+    const uint32_t stg = smem_u32(smem + C::EPI_OFF + ew * EPI_SETS * EPI_BUF);
     int set = 0;
     const uint32_t lbar = smem_u32(&ebar[ew]);
     uint32_t lphase = 0;
@@ -288,13 +291,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       const long row = row0 + lane;
       const uint32_t tbase = tmem_base + ((uint32_t)(quad * 32) << 16) + acc * BN;
 #pragma unroll 1
-      for (int c = half * (BN / 64); c < (half + 1) * (BN / 64); c++) {
+      for (int c = part * CPW; c < (part + 1) * CPW; c++) {
         const int col0 = nb * BN + c * 32;
         uint32_t raw[32];
         tmem_ld_32x32b_x32(tbase + c * 32, raw);
         const uint32_t bufA = stg + set * EPI_BUF, bufB = bufA + 2048;
-        set ^= 1;
-        if (lane == 0) bulk_wait_read1();  // the set used two chunks ago is free again
+        if (EPI_SETS == 2) {
+          set ^= 1;
+          if (lane == 0) bulk_wait_read1();  // the set used two chunks ago is free again
+        } else {
+          if (lane == 0) bulk_wait_read0();  // the previous chunk's stores have read the set
+        }
         __syncwarp();
         if (f32_in || bf16_in) {
           if (lane == 0) {

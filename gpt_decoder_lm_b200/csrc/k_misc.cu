@@ -12,10 +12,11 @@ namespace gpt {
 // target is the window shifted by one).  One thread per (b, t).
 // ============================================================================
 __global__ void k_gather(const void* __restrict__ stream, int tok_u16, uint64_t len, uint64_t seed, int step,
-                         int micro, int B, int T, int V, int32_t* __restrict__ idx, int32_t* __restrict__ tgt,
-                         uint32_t* flags) {
+                         const int* step_dev, int micro, int B, int T, int V, int32_t* __restrict__ idx,
+                         int32_t* __restrict__ tgt, uint32_t* flags) {
   long i = (long)blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= (long)B * T) return;
+  if (step_dev) step = *step_dev;  // step index held in device memory (replayed graphs)
   int b = (int)(i / T), t = (int)(i % T);
   uint64_t key = ((uint64_t)(uint32_t)step << 40) ^ ((uint64_t)(uint32_t)micro << 20) ^ (uint64_t)b;
   uint64_t ix = splitmix64(seed ^ splitmix64(key)) % (len - (uint64_t)T);
@@ -39,11 +40,24 @@ __global__ void k_gather(const void* __restrict__ stream, int tok_u16, uint64_t 
 }
 
 void gather_batch(Ctx& c, const void* stream, int tok_u16, uint64_t len, uint64_t seed, int step, int micro, int B,
-                  int T, int V, int32_t* idx, int32_t* tgt) {
+                  int T, int V, int32_t* idx, int32_t* tgt, const int* step_dev) {
   long n = (long)B * T;
   LaunchScope s(c, "gather_batch");
-  k_gather<<<(unsigned)((n + 255) / 256), 256, 0, c.stream>>>(stream, tok_u16, len, seed, step, micro, B, T, V, idx,
-                                                              tgt, c.flags);
+  k_gather<<<(unsigned)((n + 255) / 256), 256, 0, c.stream>>>(stream, tok_u16, len, seed, step, step_dev, micro, B, T,
+                                                              V, idx, tgt, c.flags);
+}
+
+// writes the per-step scalars read by replayed graphs: step, lr, 1 - b1^t, 1 - b2^t
+__global__ void k_set_step(int* step_dev, float* hyper, int step, float lr, float bc1, float bc2) {
+  *step_dev = step;
+  hyper[0] = lr;
+  hyper[1] = bc1;
+  hyper[2] = bc2;
+}
+
+void set_step_params(Ctx& c, int* step_dev, float* hyper, int step, float lr, float bc1, float bc2) {
+  LaunchScope s(c, "set_step");
+  k_set_step<<<1, 1, 0, c.stream>>>(step_dev, hyper, step, lr, bc1, bc2);
 }
 
 __global__ void k_check_tokens(const int32_t* __restrict__ idx, const int32_t* __restrict__ tgt, long n, int V,
@@ -210,7 +224,7 @@ template void norm_fwd<bf16>(Ctx&, const float*, const float*, const float*, bf1
 // ============================================================================
 template <typename T>
 __global__ void k_norm_bwd(NormBwd p) {
-  extern __shared__ float red[];  // [2 buffers][warps][2]
+  extern __shared__ float red[];  // [2 buffers][warps][4]
   int tid = threadIdx.x;
   int d4 = p.d >> 2;
   int nw = blockDim.x >> 5;
@@ -221,59 +235,69 @@ __global__ void k_norm_bwd(NormBwd p) {
   if (own && !p.rms) gw = reinterpret_cast<const float4*>(p.w)[tid];
   float pg[4] = {0, 0, 0, 0}, pb[4] = {0, 0, 0, 0}, pn[4] = {0, 0, 0, 0};
   int buf = 0;
-  for (long r = r0; r < r1; r++) {
-    float4 dy = make_float4(0, 0, 0, 0), xv = make_float4(0, 0, 0, 0);
-    float mean = p.rms ? 0.f : p.mean[r];
-    float rstd = p.rstd[r];
-    if (own) {
-      dy = reinterpret_cast<const float4*>(p.dy + r * p.d)[tid];
-      xv = reinterpret_cast<const float4*>(p.x + r * p.d)[tid];
-    }
-    float xh[4] = {(xv.x - mean) * rstd, (xv.y - mean) * rstd, (xv.z - mean) * rstd, (xv.w - mean) * rstd};
-    float dyv[4] = {dy.x, dy.y, dy.z, dy.w};
-    float wv[4] = {gw.x, gw.y, gw.z, gw.w};
-    float g[4], s1 = 0.f, s2 = 0.f;
+  const float wv[4] = {gw.x, gw.y, gw.z, gw.w};
+  // two rows per round: one barrier for both rows' reductions
+  for (long r = r0; r < r1; r += 2) {
+    float dyv[2][4], xh[2][4], g[2][4], rstd[2], s[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-    for (int k = 0; k < 4; k++) {
-      g[k] = dyv[k] * wv[k];
-      s1 += g[k];
-      s2 += g[k] * xh[k];
+    for (int u = 0; u < 2; u++) {
+      const long rr = r + u;
+      const bool live = rr < r1;
+      const float mean = (p.rms || !live) ? 0.f : p.mean[rr];
+      rstd[u] = live ? p.rstd[rr] : 0.f;
+      float4 dy = make_float4(0, 0, 0, 0), xv = make_float4(0, 0, 0, 0);
+      if (own && live) {
+        dy = reinterpret_cast<const float4*>(p.dy + rr * p.d)[tid];
+        xv = reinterpret_cast<const float4*>(p.x + rr * p.d)[tid];
+      }
+      const float dya[4] = {dy.x, dy.y, dy.z, dy.w}, xa[4] = {xv.x, xv.y, xv.z, xv.w};
+#pragma unroll
+      for (int k = 0; k < 4; k++) {
+        dyv[u][k] = dya[k];
+        xh[u][k] = (xa[k] - mean) * rstd[u];
+        g[u][k] = dya[k] * wv[k];
+        s[2 * u] += g[u][k];
+        s[2 * u + 1] += g[u][k] * xh[u][k];
+      }
     }
-    s1 = warp_sum(s1);
-    s2 = warp_sum(s2);
+#pragma unroll
+    for (int k = 0; k < 4; k++) s[k] = warp_sum(s[k]);
     if ((tid & 31) == 0) {
-      red[(buf * nw + (tid >> 5)) * 2 + 0] = s1;
-      red[(buf * nw + (tid >> 5)) * 2 + 1] = s2;
+#pragma unroll
+      for (int k = 0; k < 4; k++) red[(buf * nw + (tid >> 5)) * 4 + k] = s[k];
     }
     __syncthreads();
-    float t1 = 0.f, t2 = 0.f;
+    float t[4] = {0.f, 0.f, 0.f, 0.f};
     for (int w = 0; w < nw; w++) {
-      t1 += red[(buf * nw + w) * 2 + 0];
-      t2 += red[(buf * nw + w) * 2 + 1];
+#pragma unroll
+      for (int k = 0; k < 4; k++) t[k] += red[(buf * nw + w) * 4 + k];
     }
     buf ^= 1;
-    float mg = p.rms ? 0.f : t1 / p.d;
-    float mgx = t2 / p.d;
-    if (own) {
-      float4* dr = reinterpret_cast<float4*>(p.dres + r * p.d) + tid;
+#pragma unroll
+    for (int u = 0; u < 2; u++) {
+      const long rr = r + u;
+      if (!own || rr >= r1) continue;
+      const float mg = p.rms ? 0.f : t[2 * u] / p.d;
+      const float mgx = t[2 * u + 1] / p.d;
+      float4* dr = reinterpret_cast<float4*>(p.dres + rr * p.d) + tid;
       float4 old = p.accumulate ? *dr : make_float4(0, 0, 0, 0);
       float ov[4] = {old.x, old.y, old.z, old.w};
       float nv[4];
 #pragma unroll
       for (int k = 0; k < 4; k++) {
-        nv[k] = ov[k] + rstd * (g[k] - mg - xh[k] * mgx);
-        pg[k] += dyv[k] * xh[k];
-        pb[k] += dyv[k];
+        nv[k] = ov[k] + rstd[u] * (g[u][k] - mg - xh[u][k] * mgx);
+        pg[k] += dyv[u][k] * xh[u][k];
+        pb[k] += dyv[u][k];
       }
       *dr = make_float4(nv[0], nv[1], nv[2], nv[3]);
       if (p.want_dyb) {
         float q[4];
 #pragma unroll
         for (int k = 0; k < 4; k++) {
-          q[k] = nv[k] * drop_mul(p.drop, (uint64_t)r * p.d + 4 * tid + k);
+          q[k] = nv[k] * drop_mul(p.drop, (uint64_t)rr * p.d + 4 * tid + k);
           pn[k] += q[k];
         }
-        store4<T>(reinterpret_cast<T*>(p.dyb) + r * p.d + 4 * tid, make_float4(q[0], q[1], q[2], q[3]));
+        store4<T>(reinterpret_cast<T*>(p.dyb) + rr * p.d + 4 * tid, make_float4(q[0], q[1], q[2], q[3]));
       }
     }
   }
@@ -285,97 +309,6 @@ __global__ void k_norm_bwd(NormBwd p) {
   }
 }
 
-// Warp-per-row variant for d <= 32 * 4 * VPL: the row lives in registers (VPL
-// float4 per lane), the row reductions are warp shuffles, and each lane keeps
-// the three column partials of its columns.  Warp w of block b takes rows
-// b*8 + w, b*8 + w + 8*gridDim, ...; at the end the 8 warps' partials are
-// added in warp order through shared memory, one slot at a time.
-template <typename T, int VPL>
-__global__ void __launch_bounds__(256) k_norm_bwd_warp(NormBwd p) {
-  extern __shared__ float red[];  // [8][d]
-  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int d = p.d, d4 = d >> 2;
-  float4 gw[VPL];
-#pragma unroll
-  for (int k = 0; k < VPL; k++) {
-    int c = lane + 32 * k;
-    gw[k] = (!p.rms && c < d4) ? reinterpret_cast<const float4*>(p.w)[c] : make_float4(1.f, 1.f, 1.f, 1.f);
-  }
-  float4 pg[VPL], pb[VPL], pn[VPL];
-#pragma unroll
-  for (int k = 0; k < VPL; k++) pg[k] = pb[k] = pn[k] = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (long r = (long)blockIdx.x * 8 + w; r < p.rows; r += (long)gridDim.x * 8) {
-    const float mean = p.rms ? 0.f : p.mean[r];
-    const float rstd = p.rstd[r];
-    float4 dy[VPL], xh[VPL];
-    float s1 = 0.f, s2 = 0.f;
-#pragma unroll
-    for (int k = 0; k < VPL; k++) {
-      int c = lane + 32 * k;
-      if (c < d4) {
-        dy[k] = reinterpret_cast<const float4*>(p.dy + r * d)[c];
-        float4 x = reinterpret_cast<const float4*>(p.x + r * d)[c];
-        xh[k] = make_float4((x.x - mean) * rstd, (x.y - mean) * rstd, (x.z - mean) * rstd, (x.w - mean) * rstd);
-      } else {
-        dy[k] = xh[k] = make_float4(0.f, 0.f, 0.f, 0.f);
-      }
-      const float g0 = dy[k].x * gw[k].x, g1 = dy[k].y * gw[k].y, g2 = dy[k].z * gw[k].z, g3 = dy[k].w * gw[k].w;
-      s1 += (g0 + g1) + (g2 + g3);
-      s2 += (g0 * xh[k].x + g1 * xh[k].y) + (g2 * xh[k].z + g3 * xh[k].w);
-    }
-    s1 = warp_sum(s1);
-    s2 = warp_sum(s2);
-    const float mg = p.rms ? 0.f : s1 / d, mgx = s2 / d;
-#pragma unroll
-    for (int k = 0; k < VPL; k++) {
-      int c = lane + 32 * k;
-      if (c >= d4) continue;
-      float4* dr = reinterpret_cast<float4*>(p.dres + r * d) + c;
-      float4 o = p.accumulate ? *dr : make_float4(0.f, 0.f, 0.f, 0.f);
-      float nv[4] = {o.x + rstd * (dy[k].x * gw[k].x - mg - xh[k].x * mgx),
-                     o.y + rstd * (dy[k].y * gw[k].y - mg - xh[k].y * mgx),
-                     o.z + rstd * (dy[k].z * gw[k].z - mg - xh[k].z * mgx),
-                     o.w + rstd * (dy[k].w * gw[k].w - mg - xh[k].w * mgx)};
-      *dr = make_float4(nv[0], nv[1], nv[2], nv[3]);
-      pg[k].x += dy[k].x * xh[k].x;
-      pg[k].y += dy[k].y * xh[k].y;
-      pg[k].z += dy[k].z * xh[k].z;
-      pg[k].w += dy[k].w * xh[k].w;
-      pb[k].x += dy[k].x;
-      pb[k].y += dy[k].y;
-      pb[k].z += dy[k].z;
-      pb[k].w += dy[k].w;
-      if (p.want_dyb) {
-        float q[4];
-#pragma unroll
-        for (int e = 0; e < 4; e++) q[e] = nv[e] * drop_mul(p.drop, (uint64_t)r * d + 4 * c + e);
-        pn[k].x += q[0];
-        pn[k].y += q[1];
-        pn[k].z += q[2];
-        pn[k].w += q[3];
-        store4<T>(reinterpret_cast<T*>(p.dyb) + r * d + 4 * c, make_float4(q[0], q[1], q[2], q[3]));
-      }
-    }
-  }
-  float* out = p.part + (long)blockIdx.x * 3 * d;
-#pragma unroll
-  for (int slot = 0; slot < 3; slot++) {
-#pragma unroll
-    for (int k = 0; k < VPL; k++) {
-      int c = lane + 32 * k;
-      if (c < d4) reinterpret_cast<float4*>(red + w * d)[c] = slot == 0 ? pg[k] : (slot == 1 ? pb[k] : pn[k]);
-    }
-    __syncthreads();
-    for (int j = threadIdx.x; j < d; j += 256) {
-      float s = 0.f;
-#pragma unroll
-      for (int k = 0; k < 8; k++) s += red[k * d + j];
-      out[slot * d + j] = s;
-    }
-    __syncthreads();
-  }
-}
-
 int norm_bwd_blocks(Ctx& c, long rows) {
   long b = (long)c.num_sms * 4;
   return (int)(rows < b ? rows : b);
@@ -384,37 +317,13 @@ int norm_bwd_blocks(Ctx& c, long rows) {
 template <typename T>
 void norm_bwd(Ctx& c, const NormBwd& p) {
   int d4 = p.d / 4;
-  int vpl = (d4 + 31) / 32;
   LaunchScope s(c, "norm_bwd");
-  size_t smem = (size_t)8 * p.d * sizeof(float);
-  if (p.use_warp_rows && vpl <= 8) {  // register-heavy: one block per SM, kept for reference
-    if (vpl <= 1) k_norm_bwd_warp<T, 1><<<p.blocks, 256, smem, c.stream>>>(p);
-    else if (vpl <= 2) k_norm_bwd_warp<T, 2><<<p.blocks, 256, smem, c.stream>>>(p);
-    else if (vpl <= 4) k_norm_bwd_warp<T, 4><<<p.blocks, 256, smem, c.stream>>>(p);
-    else if (vpl <= 6) k_norm_bwd_warp<T, 6><<<p.blocks, 256, smem, c.stream>>>(p);
-    else k_norm_bwd_warp<T, 8><<<p.blocks, 256, smem, c.stream>>>(p);
-    return;
-  }
   int threads = ((d4 + 31) / 32) * 32;
   int nw = threads / 32;
-  k_norm_bwd<T><<<p.blocks, threads, 2 * nw * 2 * sizeof(float), c.stream>>>(p);
+  k_norm_bwd<T><<<p.blocks, threads, 2 * nw * 4 * sizeof(float), c.stream>>>(p);
 }
 template void norm_bwd<float>(Ctx&, const NormBwd&);
 template void norm_bwd<bf16>(Ctx&, const NormBwd&);
-
-__global__ void k_partial_reduce(const float* __restrict__ part, int blocks, int slots, int slot, int d,
-                                 float* __restrict__ grad) {
-  int j = blockIdx.x * blockDim.x + threadIdx.x;
-  if (j >= d) return;
-  float s = 0.f;
-  for (int b = 0; b < blocks; b++) s += part[((long)b * slots + slot) * d + j];
-  grad[j] += s;
-}
-
-void partial_reduce(Ctx& c, const float* part, int blocks, int slots, int slot, int d, float* grad) {
-  LaunchScope s(c, "partial_reduce");
-  k_partial_reduce<<<(d + 127) / 128, 128, 0, c.stream>>>(part, blocks, slots, slot, d, grad);
-}
 
 // grad_s[j] += sum_b part[b, s, j] for the three slots of the norm-backward
 // partials at once.  Block (32 columns x 8 row groups): row group y sums
@@ -484,13 +393,42 @@ void colsum_reduce(Ctx& c, const float* part, int chunks, int N, float* grad) {
   k_colsum_reduce<<<(N + 31) / 32, dim3(32, 8), 0, c.stream>>>(part, chunks, N, grad);
 }
 
+// bf16 rows with N % 8 == 0: each thread sums 8 adjacent columns over its
+// row chunk with 16-byte loads
+__global__ void k_colsum_bf16x8(const bf16* __restrict__ x, long rows, int N, int chunks, float* __restrict__ part) {
+  const int j8 = blockIdx.x * blockDim.x + threadIdx.x;
+  if (j8 * 8 >= N) return;
+  const long per = (rows + chunks - 1) / chunks;
+  const long r0 = blockIdx.y * per, r1 = min(rows, r0 + per);
+  float s[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  for (long r = r0; r < r1; r++) {
+    uint4 u = reinterpret_cast<const uint4*>(x + r * N)[j8];
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+    for (int k = 0; k < 4; k++) {
+      float2 f = __bfloat1622float2(h[k]);
+      s[2 * k] += f.x;
+      s[2 * k + 1] += f.y;
+    }
+  }
+  float4* dst = reinterpret_cast<float4*>(part + (long)blockIdx.y * N + j8 * 8);
+  dst[0] = make_float4(s[0], s[1], s[2], s[3]);
+  dst[1] = make_float4(s[4], s[5], s[6], s[7]);
+}
+
 template <typename T>
 void colsum_acc(Ctx& c, const T* x, long rows, int N, float* scratch, float* grad) {
-  int chunks = (int)min(64L, rows);
+  const bool vec = sizeof(T) == 2 && N % 8 == 0;
+  int chunks = (int)min(vec ? 512L : 64L, rows);  // vector path: fewer threads per row, more row chunks
   {
     LaunchScope s(c, "colsum");
-    dim3 grid((N + 127) / 128, chunks);
-    k_colsum<T><<<grid, 128, 0, c.stream>>>(x, rows, N, chunks, scratch);
+    if (vec) {
+      dim3 grid((N / 8 + 127) / 128, chunks);
+      k_colsum_bf16x8<<<grid, 128, 0, c.stream>>>(reinterpret_cast<const bf16*>(x), rows, N, chunks, scratch);
+    } else {
+      dim3 grid((N + 127) / 128, chunks);
+      k_colsum<T><<<grid, 128, 0, c.stream>>>(x, rows, N, chunks, scratch);
+    }
   }
   colsum_reduce(c, scratch, chunks, N, grad);
 }
@@ -549,85 +487,6 @@ __global__ void k_ce(T* __restrict__ logits, const int32_t* __restrict__ tgt, in
     float g = 0.f;
     if (j < V) g = (expf(to_f<T>(z[j]) - lse) - (j == t ? 1.f : 0.f)) * scale;
     z[j] = from_f<T>(g);
-  }
-}
-
-// Register-resident variant: the row is read from HBM once with 16-byte
-// loads (EPV elements per vector, up to 16 vectors per thread), max and
-// sum-exp come from registers, and the gradient is written once.
-template <typename T>
-__global__ void __launch_bounds__(512) k_ce_vec(T* __restrict__ logits, const int32_t* __restrict__ tgt, int V,
-                                                int Vp, float* __restrict__ lse_out, float* __restrict__ row_loss,
-                                                int want_grad, float scale) {
-  constexpr int EPV = 16 / sizeof(T);
-  constexpr int NV = 16;
-  __shared__ float red[16];
-  __shared__ float s_zt;
-  const long row = blockIdx.x;
-  T* z = logits + row * Vp;
-  const int nvec = Vp / EPV;
-  const int t = tgt[row];
-  if (threadIdx.x == 0) s_zt = to_f<T>(z[t]);
-  uint4 buf[NV];
-#pragma unroll
-  for (int k = 0; k < NV; k++) {
-    int vi = threadIdx.x + k * 512;
-    buf[k] = vi < nvec ? reinterpret_cast<const uint4*>(z)[vi] : make_uint4(0, 0, 0, 0);
-  }
-  auto elem = [&](const uint4& u, int e) -> float {
-    const T* p = reinterpret_cast<const T*>(&u);
-    return to_f<T>(p[e]);
-  };
-  float mx = -INFINITY;
-#pragma unroll
-  for (int k = 0; k < NV; k++) {
-    int vi = threadIdx.x + k * 512;
-#pragma unroll
-    for (int e = 0; e < EPV; e++)
-      if (vi < nvec && vi * EPV + e < V) mx = fmaxf(mx, elem(buf[k], e));
-  }
-  mx = warp_max(mx);
-  const int w = threadIdx.x >> 5;
-  if ((threadIdx.x & 31) == 0) red[w] = mx;
-  __syncthreads();
-  float M = red[0];
-#pragma unroll
-  for (int k = 1; k < 16; k++) M = fmaxf(M, red[k]);
-  __syncthreads();
-  float sum = 0.f;
-#pragma unroll
-  for (int k = 0; k < NV; k++) {
-    int vi = threadIdx.x + k * 512;
-#pragma unroll
-    for (int e = 0; e < EPV; e++)
-      if (vi < nvec && vi * EPV + e < V) sum += expf(elem(buf[k], e) - M);
-  }
-  sum = warp_sum(sum);
-  if ((threadIdx.x & 31) == 0) red[w] = sum;
-  __syncthreads();
-  float S = 0.f;
-#pragma unroll
-  for (int k = 0; k < 16; k++) S += red[k];
-  const float lse = M + logf(S);
-  if (threadIdx.x == 0) {
-    lse_out[row] = lse;
-    row_loss[row] = lse - s_zt;
-  }
-  if (!want_grad) return;
-#pragma unroll
-  for (int k = 0; k < NV; k++) {
-    int vi = threadIdx.x + k * 512;
-    if (vi >= nvec) continue;
-    uint4 outv;
-    T* o = reinterpret_cast<T*>(&outv);
-#pragma unroll
-    for (int e = 0; e < EPV; e++) {
-      int j = vi * EPV + e;
-      float g = 0.f;
-      if (j < V) g = (expf(elem(buf[k], e) - lse) - (j == t ? 1.f : 0.f)) * scale;
-      o[e] = from_f<T>(g);
-    }
-    reinterpret_cast<uint4*>(z)[vi] = outv;
   }
 }
 
@@ -969,6 +828,11 @@ __global__ void k_adamw(AdamArgs a, uint32_t* flags) {
     }
   }
   __syncthreads();
+  if (a.hyper) {  // learning rate and bias corrections of this step from device memory
+    a.lr = a.hyper[0];
+    a.bc1 = a.hyper[1];
+    a.bc2 = a.hyper[2];
+  }
   const float coef = s_coef;
   const int ok = s_ok;
   const float om1 = 1.f - a.beta1, om2 = 1.f - a.beta2;

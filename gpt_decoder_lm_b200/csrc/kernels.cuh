@@ -109,8 +109,11 @@ void attn_fwd_tc(Ctx& c, const AttnDesc& a);
 void attn_bwd_tc(Ctx& c, const AttnDesc& a);
 
 // ---------------------------------------------------------------- memory-bound kernels
+// step_dev (nullable): read the step index from device memory instead of `step`
 void gather_batch(Ctx& c, const void* stream, int tok_u16, uint64_t len, uint64_t seed, int step, int micro,
-                  int B, int T, int V, int32_t* idx, int32_t* tgt);
+                  int B, int T, int V, int32_t* idx, int32_t* tgt, const int* step_dev = nullptr);
+// one-thread kernel: *step_dev = step; hyper = {lr, bc1, bc2}
+void set_step_params(Ctx& c, int* step_dev, float* hyper, int step, float lr, float bc1, float bc2);
 void check_tokens(Ctx& c, const int32_t* idx, const int32_t* tgt, long n, int V, int32_t* idx_out,
                   int32_t* tgt_out);
 
@@ -133,12 +136,9 @@ struct NormBwd {
   void* dyb; DropKey drop; bool want_dyb;
   float* part; int blocks;
   long rows; int d; bool rms;
-  bool use_warp_rows = false;  // warp-per-row kernel instead of the column-per-thread one
 };
 template <typename T> void norm_bwd(Ctx& c, const NormBwd& p);
 int norm_bwd_blocks(Ctx& c, long rows);
-// grad[j] += sum_b part[b, slot, j] for the given slot
-void partial_reduce(Ctx& c, const float* part, int blocks, int slots, int slot, int d, float* grad);
 // the three slots of part[blocks, 3, d] into g0, g1, g2 (each nullable), one launch
 void partial_reduce3(Ctx& c, const float* part, int blocks, int d, float* g0, float* g1, float* g2);
 
@@ -169,6 +169,7 @@ struct AdamArgs {
   long n; long n_decay;
   const double* norm_partials; int norm_blocks; float* norm_out;
   float lr, beta1, beta2, eps, wd, clip, bc1, bc2;
+  const float* hyper = nullptr;  // when set: {lr, bc1, bc2} read from device memory
 };
 void adamw(Ctx& c, const AdamArgs& a);
 void to_bf16(Ctx& c, const float* src, bf16* dst, long n);

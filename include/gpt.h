@@ -181,6 +181,16 @@ gpt_status gpt_train_step(gpt_model* m, const void* d_stream, uint64_t stream_le
 gpt_status gpt_train_step_host(gpt_model* m, const int32_t* h_idx, const int32_t* h_tgt, float lr,
                                int32_t step, float* h_loss, float* h_grad_norm);
 
+/* CUDA-graph replay of gpt_train_step / gpt_train_step_host (default on).
+ * When on, and the config has no dropout and per-kernel timing is off, the
+ * first step of each kind runs eagerly, the second is captured into a graph
+ * (on a stream the library creates) and every later step replays it on the
+ * model's stream after a one-thread kernel writes the step's index, lr and
+ * bias corrections to device memory.  A new d_stream / stream_len /
+ * data_seed triggers a new capture.  The replayed step runs the same kernels
+ * with the same arguments as the eager one, so results are bit-identical. */
+gpt_status gpt_set_graphs(gpt_model* m, int32_t on);
+
 /* The batch gather of gpt_train_step on its own: writes int32
  * [batch_size, block_size] ids and targets to d_idx / d_tgt. */
 gpt_status gpt_gather_batch(gpt_model* m, const void* d_stream, uint64_t stream_len, uint64_t data_seed,

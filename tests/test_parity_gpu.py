@@ -243,3 +243,53 @@ def test_errors_reported_not_trapped():
     with pytest.raises(gb.GptError) as e:
         m.forward_loss(dev(idx), dev(tgt))
     assert e.value.name == "GPT_ERR_NONFINITE"
+
+
+def _weights(m):
+    P = m.get(gb.GPT_PARAM)
+    return np.concatenate([P[k].ravel() for k in sorted(P)])
+
+
+@pytest.mark.parametrize("host_batches", [False, True])
+def test_graph_replay_bit_identical_to_eager(host_batches):
+    # The replayed step reads its step index, lr and bias corrections from
+    # device memory; every other argument is the eager step's.  Weights, loss
+    # and norm must match bit for bit over steps with a changing lr, and a new
+    # data seed must re-capture (device-gather form).
+    w = W.CHAR
+    stream = W.token_stream(w, n=1 << 16)
+    sd = dev(stream.astype(np.int32))
+    res = []
+    for graphs in (False, True):
+        m, cfg = make(w, n_layer=2, batch_size=4, block_size=128, grad_accum=2)
+        m.set_graphs(graphs)
+        out = []
+        for step in range(1, 7):
+            lr = oracle.lr_cosine(w.lr, step - 1, 2, 6)
+            seed = w.data_seed if step < 5 else w.data_seed + 1
+            if host_batches:
+                B, T, ga = cfg.batch_size, cfg.block_size, cfg.grad_accum
+                idx, tgt = W.random_batch(w, 100 + step, B * ga, T)
+                out.append(m.train_step_host(np.ascontiguousarray(idx, np.int32),
+                                             np.ascontiguousarray(tgt, np.int32), lr, step))
+            else:
+                out.append(m.train_step(sd, seed, lr, step))
+        res.append((out, _weights(m)))
+        m.close()
+    (l0, w0), (l1, w1) = res
+    assert l0 == l1
+    assert np.array_equal(w0, w1)
+
+
+def test_graph_replay_reports_token_errors():
+    # a replayed step still checks host-supplied tokens and raises the flag
+    w = W.CHAR
+    m, cfg = make(w, n_layer=1, batch_size=2, block_size=64, grad_accum=1)
+    B, T = cfg.batch_size, cfg.block_size
+    for step in range(1, 4):
+        idx, tgt = W.random_batch(w, step, B, T)
+        m.train_step_host(np.ascontiguousarray(idx, np.int32), np.ascontiguousarray(tgt, np.int32), 1e-3, step)
+    idx[0, 0] = cfg.vocab_size + 5
+    with pytest.raises(gb.GptError) as e:
+        m.train_step_host(np.ascontiguousarray(idx, np.int32), np.ascontiguousarray(tgt, np.int32), 1e-3, 4)
+    assert e.value.name == "GPT_ERR_TOKEN_RANGE"
