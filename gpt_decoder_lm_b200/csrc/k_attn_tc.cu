@@ -11,7 +11,8 @@
 //
 // Every kernel: warp 0 issues TMA loads of bf16 tiles (128-byte swizzle) from
 // the [B*T, 3, H, 64] qkv activations, warp 1 owns TMEM and issues
-// tcgen05.mma, warps 2..5 (one TMEM lane / tile row per thread) do the softmax
+// tcgen05.mma, and the math warps (forward: warps 2..5, one TMEM lane / tile
+// row per thread; backward: warps 2..9, two per lane quadrant) do the softmax
 // arithmetic, write the bf16 probability (or dS) tile back into TMEM, where the
 // next MMA reads it as its A operand, and run the epilogue.  Each kernel keeps
 // its TMEM at 256 columns and its shared memory under 113 KB so that two CTAs
@@ -71,12 +72,14 @@ __device__ __forceinline__ void ld64(uint32_t taddr, uint32_t (&a)[32], uint32_t
 
 // ============================================================================
 // forward, pipelined: one CTA per (128-query block, b, h), 64-key blocks.
-// S and P V are double-buffered in TMEM, so the MMA warp computes S of block
-// j+1 while the softmax warps work on block j, and the softmax warps fold the
-// P V product of block j-1 into O after handing over P of block j (deferred
-// rescaling: O <- O * alpha_{j-1} + PV_{j-1}).
+// S is double-buffered in TMEM, so the MMA warp computes S of block j+1
+// while the softmax warps work on block j.  O accumulates in TMEM (the P V
+// MMAs add into it) against a per-row reference maximum m that is raised only
+// when a block's maximum exceeds it by more than 2^RESCALE_LOG2 (then the
+// softmax warps rescale that row of O and l once); otherwise probabilities are
+// taken against the stale m, which leaves O / l and m + log2 l unchanged.
 // smem: Q | (K, V)[3 stages] | barriers   (64 KB + 256 B)
-// TMEM: S[2] cols [0,64), [64,128); PV[2] cols [128,192), [192,256).  The
+// TMEM: S[2] cols [0,64), [64,128); O cols [128,192)  (256 allocated).  The
 // softmax warps overwrite the first 32 columns of S[u] with bf16 P, which the
 // P V MMA reads as its TMEM A operand (tcgen05 MMAs of one thread execute in
 // issue order, so S of block j+2 lands in S[u] only after P V of block j).
@@ -84,9 +87,11 @@ __device__ __forceinline__ void ld64(uint32_t taddr, uint32_t (&a)[32], uint32_t
 constexpr int D_Q = 0, D_KV = TILE, D_BAR = 4 * TILE;
 constexpr int D_SMEM = D_BAR + 256;
 constexpr int D_STAGES = 3;
+constexpr float RESCALE_LOG2 = 8.0f;
 
-__global__ void __launch_bounds__(192, 2) k_attn_fwd_db(const __grid_constant__ CUtensorMap tq,
-                                                        const __grid_constant__ CUtensorMap tkv64, AttnTcArgs a) {
+template <bool DROP>
+__global__ void __launch_bounds__(192, 2) k_attn_fwd_o(const __grid_constant__ CUtensorMap tq,
+                                                       const __grid_constant__ CUtensorMap tkv64, AttnTcArgs a) {
   extern __shared__ __align__(1024) uint8_t smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (smem_u32(smem) & 1023) {  // swizzled tiles need 1024-byte alignment
@@ -96,7 +101,8 @@ __global__ void __launch_bounds__(192, 2) k_attn_fwd_db(const __grid_constant__ 
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + D_BAR);
   const uint32_t q_full = smem_u32(bars + 0);
   const uint32_t kv_full0 = smem_u32(bars + 1), kv_empty0 = smem_u32(bars + 1 + D_STAGES);
-  const uint32_t s_full0 = smem_u32(bars + 1 + 2 * D_STAGES), p_full0 = s_full0 + 16, pv_full0 = s_full0 + 32;
+  // pv_done[i & 1] completes when the P V product of block i has landed in O
+  const uint32_t s_full0 = smem_u32(bars + 1 + 2 * D_STAGES), p_full0 = s_full0 + 16, pv_done0 = s_full0 + 32;
   uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + 7 + 2 * D_STAGES);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tslot + 1);
   const uint32_t sb = smem_u32(smem);
@@ -104,7 +110,7 @@ __global__ void __launch_bounds__(192, 2) k_attn_fwd_db(const __grid_constant__ 
   const int nqb = a.T / 128;
   const int qb = nqb - 1 - (int)blockIdx.x;  // longest rows first
   const int bh = blockIdx.y, b = bh / a.H, h = bh % a.H;
-  const int nkb = 2 * (qb + 1);  // 64-key blocks up to and including the diagonal
+  const int nkb = 2 * (qb + 1);  // 64-key blocks up to and including the diagonal (>= 2)
   const int row0 = b * a.T;
 
   if (threadIdx.x == 0) {
@@ -116,7 +122,7 @@ __global__ void __launch_bounds__(192, 2) k_attn_fwd_db(const __grid_constant__ 
     for (int u = 0; u < 2; u++) {
       mbar_init(s_full0 + 8 * u, 1);
       mbar_init(p_full0 + 8 * u, 4);
-      mbar_init(pv_full0 + 8 * u, 1);
+      mbar_init(pv_done0 + 8 * u, 1);
     }
     *abort_flag = 0;
     fence_barrier_init();
@@ -150,7 +156,8 @@ __global__ void __launch_bounds__(192, 2) k_attn_fwd_db(const __grid_constant__ 
       constexpr uint32_t id_n64 = idesc_bf16_f32(128, 64, false, false);
       constexpr uint32_t id_pv = idesc_bf16_f32(128, 64, false, true);
       bool ok = mbar_wait(q_full, 0, abort_flag, a.flags);
-      // PV of block i: P[i&1] (K = 64 keys) times V of block i (MN-major, N = 64)
+      // O += P V of block i: P over the first 32 columns of S[i&1] (K = 64
+      // keys), V of block i MN-major (N = 64)
       auto issue_pv = [&](int i) -> bool {
         const int u = i & 1;
         if (!mbar_wait(p_full0 + 8 * u, (i >> 1) & 1, abort_flag, a.flags)) return false;
@@ -158,8 +165,8 @@ __global__ void __launch_bounds__(192, 2) k_attn_fwd_db(const __grid_constant__ 
         const uint32_t v = sb + D_KV + (i % D_STAGES) * TILE + HTILE;
 #pragma unroll
         for (int kk = 0; kk < 4; kk++)
-          mma_bf16_ts(tmem + 128 + 64 * u, tmem + 64 * u + 8 * kk, desc_mn64(v, kk), id_pv, kk > 0);
-        mma_commit(pv_full0 + 8 * u);
+          mma_bf16_ts(tmem + 128, tmem + 64 * u + 8 * kk, desc_mn64(v, kk), id_pv, (i > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(pv_done0 + 8 * u);
         mma_commit(kv_empty0 + 8 * (i % D_STAGES));
         return true;
       };
@@ -183,26 +190,9 @@ __global__ void __launch_bounds__(192, 2) k_attn_fwd_db(const __grid_constant__ 
     const int qi = qb * 128 + r;
     const uint32_t trow = tmem + ((uint32_t)(quad * 32) << 16);
     const float sl2 = a.scale_log2;
-    float m = -INFINITY, l = 0.f, alpha_prev = 0.f;
-    float o[64];
-#pragma unroll
-    for (int i = 0; i < 64; i++) o[i] = 0.f;
+    float m = -INFINITY, l = 0.f;  // reference maximum (log2 units) and row sum against it
     const uint64_t ebase = ((uint64_t)bh * a.T + qi) * a.T;
     bool ok = true;
-    // O <- O * alpha + PV of block i
-    auto fold_pv = [&](int i, float alpha) -> bool {
-      const int u = i & 1;
-      if (!mbar_wait(pv_full0 + 8 * u, (i >> 1) & 1, abort_flag, a.flags)) return false;
-      tc_fence_after();
-      uint32_t v0[32], v1[32];
-      ld64(trow + 128 + 64 * u, v0, v1);
-#pragma unroll
-      for (int i2 = 0; i2 < 32; i2++) {
-        o[i2] = fmaf(o[i2], alpha, __uint_as_float(v0[i2]));
-        o[32 + i2] = fmaf(o[32 + i2], alpha, __uint_as_float(v1[i2]));
-      }
-      return true;
-    };
     for (int j = 0; j < nkb; j++) {
       const int u = j & 1;
       if (!(ok = mbar_wait(s_full0 + 8 * u, (j >> 1) & 1, abort_flag, a.flags))) break;
@@ -210,9 +200,9 @@ __global__ void __launch_bounds__(192, 2) k_attn_fwd_db(const __grid_constant__ 
       uint32_t v0[32], v1[32];
       ld64(trow + 64 * u, v0, v1);
       const int key0 = j * 64;
-      const bool diag = key0 + 63 > qb * 128;
+      const int lim = qi - key0;  // key key0 + i is visible iff i <= lim
       float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
-      if (!diag) {
+      if (lim >= 63) {
 #pragma unroll
         for (int i = 0; i < 32; i += 2) {
           mx0 = fmaxf(mx0, __uint_as_float(v0[i]));
@@ -223,30 +213,53 @@ __global__ void __launch_bounds__(192, 2) k_attn_fwd_db(const __grid_constant__ 
       } else {
 #pragma unroll
         for (int i = 0; i < 32; i++) {
-          if (key0 + i <= qi) mx0 = fmaxf(mx0, __uint_as_float(v0[i]));
-          if (key0 + 32 + i <= qi) mx1 = fmaxf(mx1, __uint_as_float(v1[i]));
+          if (i <= lim) mx0 = fmaxf(mx0, __uint_as_float(v0[i]));
+          if (i + 32 <= lim) mx1 = fmaxf(mx1, __uint_as_float(v1[i]));
         }
       }
-      const float mn = fmaxf(m, fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2);
-      const float alpha = ex2(m - mn);  // 0 for the first block, 1 while the row is still empty
+      const float bm = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;
+      if (j == 0) {
+        m = bm;  // key 0 is visible to every row, so m is finite from here on
+      } else {
+        const bool need = bm > m + RESCALE_LOG2;
+        if (__any_sync(0xffffffffu, need)) {
+          // O holds the P V products of blocks < j.  S of block j was issued
+          // after P V of block j-2, so P V of block j-1 is the only one that
+          // may be in flight.
+          if (!(ok = mbar_wait(pv_done0 + 8 * ((j - 1) & 1), ((j - 1) >> 1) & 1, abort_flag, a.flags))) break;
+          tc_fence_after();
+          const float sc = need ? ex2(m - bm) : 1.f;
+          uint32_t o0[32], o1[32];
+          ld64(trow + 128, o0, o1);
+          uint32_t w[16];
+#pragma unroll
+          for (int h2 = 0; h2 < 4; h2++) {
+            const uint32_t* src = h2 < 2 ? o0 + 16 * h2 : o1 + 16 * (h2 - 2);
+#pragma unroll
+            for (int i = 0; i < 16; i++) w[i] = __float_as_uint(__uint_as_float(src[i]) * sc);
+            tmem_st_32x32b_x16(trow + 128 + 16 * h2, w);
+          }
+          l *= sc;
+          if (need) m = bm;
+        }
+      }
       float ls0 = 0.f, ls1 = 0.f;
       uint32_t pk0[16], pk1[16];
 #pragma unroll
       for (int i = 0; i < 32; i += 2) {
-        float p0 = ex2(fmaf(__uint_as_float(v0[i]), sl2, -mn));
-        float p1 = ex2(fmaf(__uint_as_float(v0[i + 1]), sl2, -mn));
-        float p2 = ex2(fmaf(__uint_as_float(v1[i]), sl2, -mn));
-        float p3 = ex2(fmaf(__uint_as_float(v1[i + 1]), sl2, -mn));
-        if (diag) {
-          const int k = key0 + i;
-          if (k > qi) p0 = 0.f;
-          if (k + 1 > qi) p1 = 0.f;
-          if (k + 32 > qi) p2 = 0.f;
-          if (k + 33 > qi) p3 = 0.f;
+        float p0 = ex2(fmaf(__uint_as_float(v0[i]), sl2, -m));
+        float p1 = ex2(fmaf(__uint_as_float(v0[i + 1]), sl2, -m));
+        float p2 = ex2(fmaf(__uint_as_float(v1[i]), sl2, -m));
+        float p3 = ex2(fmaf(__uint_as_float(v1[i + 1]), sl2, -m));
+        if (lim < 63) {
+          if (i > lim) p0 = 0.f;
+          if (i + 1 > lim) p1 = 0.f;
+          if (i + 32 > lim) p2 = 0.f;
+          if (i + 33 > lim) p3 = 0.f;
         }
         ls0 += p0 + p1;
         ls1 += p2 + p3;
-        if (a.drop.active) {
+        if (DROP) {
           const uint64_t e = ebase + key0 + i;
           p0 *= drop_mul(a.drop, e);
           p1 *= drop_mul(a.drop, e + 1);
@@ -259,23 +272,29 @@ __global__ void __launch_bounds__(192, 2) k_attn_fwd_db(const __grid_constant__ 
       // P (bf16 pairs) over the first 32 columns of S[u]: the A operand of P V
       tmem_st_32x32b_x16(trow + 64 * u, pk0);
       tmem_st_32x32b_x16(trow + 64 * u + 16, pk1);
-      l = l * alpha + (ls0 + ls1);
+      l += ls0 + ls1;
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(p_full0 + 8 * u);  // one arrival per math warp
-      if (j >= 1 && !(ok = fold_pv(j - 1, alpha_prev))) break;
-      alpha_prev = alpha;
-      m = mn;
     }
-    if (ok) ok = fold_pv(nkb - 1, alpha_prev);
+    // the last two P V products may both be in flight
+    if (ok) ok = mbar_wait(pv_done0 + 8 * (nkb & 1), ((nkb - 2) >> 1) & 1, abort_flag, a.flags);
+    if (ok) ok = mbar_wait(pv_done0 + 8 * ((nkb - 1) & 1), ((nkb - 1) >> 1) & 1, abort_flag, a.flags);
     if (ok) {
+      tc_fence_after();
+      uint32_t o0[32], o1[32];
+      ld64(trow + 128, o0, o1);
       const float inv = 1.0f / l;
       uint4* dst = reinterpret_cast<uint4*>(a.o_out + ((size_t)(row0 + qi) * a.H + h) * 64);
 #pragma unroll
-      for (int q = 0; q < 8; q++)
-        dst[q] = make_uint4(pack2(o[8 * q] * inv, o[8 * q + 1] * inv), pack2(o[8 * q + 2] * inv, o[8 * q + 3] * inv),
-                            pack2(o[8 * q + 4] * inv, o[8 * q + 5] * inv), pack2(o[8 * q + 6] * inv, o[8 * q + 7] * inv));
+      for (int q = 0; q < 8; q++) {
+        const uint32_t* x = q < 4 ? o0 + 8 * q : o1 + 8 * (q - 4);
+        dst[q] = make_uint4(pack2(__uint_as_float(x[0]) * inv, __uint_as_float(x[1]) * inv),
+                            pack2(__uint_as_float(x[2]) * inv, __uint_as_float(x[3]) * inv),
+                            pack2(__uint_as_float(x[4]) * inv, __uint_as_float(x[5]) * inv),
+                            pack2(__uint_as_float(x[6]) * inv, __uint_as_float(x[7]) * inv));
+      }
       a.lse[(size_t)bh * a.T + qi] = (m + log2f(l)) * LN2;
     }
   }
@@ -285,20 +304,29 @@ __global__ void __launch_bounds__(192, 2) k_attn_fwd_db(const __grid_constant__ 
   if (warp == 1) tmem_dealloc(tmem, 256);
 }
 
+// packed bf16 pair column of element column c (0..63) of a 64-column block:
+// the half that owns c writes inside its own fp32 columns
+__device__ __forceinline__ int pcol(int c) { return (c & 32) + ((c & 31) >> 1); }
+// TMEM A-operand column of K-step kk (16 elements) under that layout
+__device__ __forceinline__ uint32_t acol(int kk) { return (uint32_t)((kk >> 1) * 32 + (kk & 1) * 8); }
+
 // ============================================================================
 // backward, dK and dV: one CTA per (128-key block, b, h), walking 64-query
 // blocks from the key block on.  Keys are the MMA rows:
 //   S^T = K Q^T, dP^T = V dO^T  ->  P~^T, dS^T (bf16, written into TMEM)
 //   dV += P~^T dO,  dK += dS^T Q
+// Eight math warps, two per TMEM lane quadrant, each take 32 of the 64 query
+// columns of a block (the backward has no row reductions).
 // smem: K | V | (Q, dO)[2 stages] | (lse, D)[2] | barriers (~65 KB)
 // TMEM: S^T [0,64), dP^T [64,128), dV [128,192), dK [192,256)
 // ============================================================================
 constexpr int K_K = 0, K_V = TILE, K_ST = 2 * TILE, K_LD = 4 * TILE, K_BAR = K_LD + 1024;
 constexpr int K_SMEM = K_BAR + 128;
 
-__global__ void __launch_bounds__(192, 2) k_attn_bwd_kv_tc(const __grid_constant__ CUtensorMap tkv,
-                                                           const __grid_constant__ CUtensorMap tq64,
-                                                           const __grid_constant__ CUtensorMap tdo64, AttnTcArgs a) {
+template <bool DROP>
+__global__ void __launch_bounds__(320, 2) k_attn_bwd_kv8(const __grid_constant__ CUtensorMap tkv,
+                                                         const __grid_constant__ CUtensorMap tq64,
+                                                         const __grid_constant__ CUtensorMap tdo64, AttnTcArgs a) {
   extern __shared__ __align__(1024) uint8_t smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (smem_u32(smem) & 1023) {
@@ -314,7 +342,7 @@ __global__ void __launch_bounds__(192, 2) k_attn_bwd_kv_tc(const __grid_constant
   const uint32_t sb = smem_u32(smem);
 
   const int nq64 = a.T / 64;
-  const int kb = (int)blockIdx.x;  // key block 0 has the most query blocks: first
+  const int kb = (int)blockIdx.x;
   const int bh = blockIdx.y, b = bh / a.H, h = bh % a.H;
   const int row0 = b * a.T;
   const int i0 = 2 * kb;
@@ -327,7 +355,7 @@ __global__ void __launch_bounds__(192, 2) k_attn_bwd_kv_tc(const __grid_constant
     mbar_init(st_empty0, 1);
     mbar_init(st_empty0 + 8, 1);
     mbar_init(sdp_full, 1);
-    mbar_init(pds_full, 4);
+    mbar_init(pds_full, 8);
     mbar_init(acc_full, 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -381,16 +409,17 @@ __global__ void __launch_bounds__(192, 2) k_attn_bwd_kv_tc(const __grid_constant
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 4; kk++)
-          mma_bf16_ts(tmem + 128, tmem + 8 * kk, desc_mn64(dO, kk), id_acc, (it > 0 || kk > 0));
+          mma_bf16_ts(tmem + 128, tmem + acol(kk), desc_mn64(dO, kk), id_acc, (it > 0 || kk > 0));
 #pragma unroll
         for (int kk = 0; kk < 4; kk++)
-          mma_bf16_ts(tmem + 192, tmem + 64 + 8 * kk, desc_mn64(q, kk), id_acc, (it > 0 || kk > 0));
+          mma_bf16_ts(tmem + 192, tmem + 64 + acol(kk), desc_mn64(q, kk), id_acc, (it > 0 || kk > 0));
         mma_commit(st_empty0 + 8 * s);
       }
       mma_commit(acc_full);
     }
   } else {
     const int quad = warp & 3;
+    const int half = (warp - 2) >> 2;
     const int r = quad * 32 + lane;
     const int kj = kb * 128 + r;
     const uint32_t trow = tmem + ((uint32_t)(quad * 32) << 16);
@@ -403,45 +432,44 @@ __global__ void __launch_bounds__(192, 2) k_attn_bwd_kv_tc(const __grid_constant
       if (!(ok = mbar_wait(st_full0 + 8 * (it & 1), (it >> 1) & 1, abort_flag, a.flags))) break;
       if (!(ok = mbar_wait(sdp_full, it & 1, abort_flag, a.flags))) break;
       tc_fence_after();
-      const bool diag = q0 < kb * 128 + 128;  // the block straddles this CTA's keys
-      uint32_t s0[32], s1[32], d0[32], d1[32];
-      tmem_ld_32x32b_x32(trow, s0);
-      tmem_ld_32x32b_x32(trow + 32, s1);
-      tmem_ld_32x32b_x32(trow + 64, d0);
-      tmem_ld_32x32b_x32(trow + 96, d1);
-      tmem_ld_wait();
-      uint32_t pp0[16], pp1[16], pd0[16], pd1[16];
+      const int lim = kj - q0;  // query column c is masked iff c < lim
 #pragma unroll
-      for (int e = 0; e < 32; e += 2) {
-        float pv[4], dsv[4];
+      for (int sub = 0; sub < 2; sub++) {
+        const int c0 = half * 32 + sub * 16;
+        uint32_t sv[16], dv[16];
+        tmem_ld_32x32b_x16(trow + c0, sv);
+        tmem_ld_32x32b_x16(trow + 64 + c0, dv);
+        tmem_ld_wait();
+        uint32_t pp[8], pd[8];
 #pragma unroll
-        for (int u = 0; u < 4; u++) {
-          const int col = (u >> 1) * 32 + e + (u & 1);
-          const uint32_t sraw = (u >> 1) ? s1[e + (u & 1)] : s0[e + (u & 1)];
-          const uint32_t draw = (u >> 1) ? d1[e + (u & 1)] : d0[e + (u & 1)];
-          float p = ex2(fmaf(__uint_as_float(sraw), sl2, -ld[col] * LOG2E));
-          if (diag && kj > q0 + col) p = 0.f;
-          float dp = __uint_as_float(draw);
-          if (a.drop.active) {
-            float mk = drop_mul(a.drop, ((uint64_t)bh * a.T + q0 + col) * a.T + kj);
-            pv[u] = p * mk;
-            dp *= mk;
-          } else {
-            pv[u] = p;
+        for (int e = 0; e < 16; e += 4) {
+          const float4 l4 = *reinterpret_cast<const float4*>(ld + c0 + e);
+          const float4 d4 = *reinterpret_cast<const float4*>(ld + 64 + c0 + e);
+          const float lv[4] = {l4.x, l4.y, l4.z, l4.w}, dd[4] = {d4.x, d4.y, d4.z, d4.w};
+          float pv[4], dsv[4];
+#pragma unroll
+          for (int u = 0; u < 4; u++) {
+            const int col = c0 + e + u;
+            float p = ex2(fmaf(__uint_as_float(sv[e + u]), sl2, -lv[u] * LOG2E));
+            if (col < lim) p = 0.f;
+            float dp = __uint_as_float(dv[e + u]);
+            if (DROP) {
+              float mk = drop_mul(a.drop, ((uint64_t)bh * a.T + q0 + col) * a.T + kj);
+              pv[u] = p * mk;
+              dp *= mk;
+            } else {
+              pv[u] = p;
+            }
+            dsv[u] = p * (dp - dd[u]);
           }
-          dsv[u] = p * (dp - ld[64 + col]);
+          pp[e >> 1] = pack2(pv[0], pv[1]);
+          pp[(e >> 1) + 1] = pack2(pv[2], pv[3]);
+          pd[e >> 1] = pack2(dsv[0], dsv[1]);
+          pd[(e >> 1) + 1] = pack2(dsv[2], dsv[3]);
         }
-        pp0[e >> 1] = pack2(pv[0], pv[1]);
-        pp1[e >> 1] = pack2(pv[2], pv[3]);
-        pd0[e >> 1] = pack2(dsv[0], dsv[1]);
-        pd1[e >> 1] = pack2(dsv[2], dsv[3]);
+        tmem_st_32x32b_x8(trow + pcol(c0), pp);
+        tmem_st_32x32b_x8(trow + 64 + pcol(c0), pd);
       }
-      // P~^T over the first 32 columns of S^T, dS^T over those of dP^T (bf16
-      // pairs): the TMEM A operands of the dV and dK MMAs
-      tmem_st_32x32b_x16(trow, pp0);
-      tmem_st_32x32b_x16(trow + 16, pp1);
-      tmem_st_32x32b_x16(trow + 64, pd0);
-      tmem_st_32x32b_x16(trow + 80, pd1);
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
@@ -450,22 +478,19 @@ __global__ void __launch_bounds__(192, 2) k_attn_bwd_kv_tc(const __grid_constant
     if (ok && mbar_wait(acc_full, 0, abort_flag, a.flags)) {
       tc_fence_after();
       bf16* rowp = a.dqkv + (size_t)(row0 + kj) * (3 * a.H * 64);
-      // dV at slot 2H+h, dK (times 1/sqrt(hd)) at slot H+h
+      // half 0: dV at slot 2H+h; half 1: dK (times 1/sqrt(hd)) at slot H+h
+      const float f = half == 0 ? 1.0f : a.scale;
+      uint4* dst = reinterpret_cast<uint4*>(rowp + (size_t)((half == 0 ? 2 : 1) * a.H + h) * 64);
 #pragma unroll
-      for (int w2 = 0; w2 < 2; w2++) {
-        const float f = w2 == 0 ? 1.0f : a.scale;
-        uint4* dst = reinterpret_cast<uint4*>(rowp + (size_t)((w2 == 0 ? 2 : 1) * a.H + h) * 64);
-        uint32_t v0[32], v1[32];
-        ld64(trow + 128 + w2 * 64, v0, v1);
-#pragma unroll
-        for (int q = 0; q < 4; q++) {
-          const float* x = reinterpret_cast<const float*>(v0) + 8 * q;
-          const float* y = reinterpret_cast<const float*>(v1) + 8 * q;
-          dst[q] = make_uint4(pack2(x[0] * f, x[1] * f), pack2(x[2] * f, x[3] * f), pack2(x[4] * f, x[5] * f),
-                              pack2(x[6] * f, x[7] * f));
-          dst[4 + q] = make_uint4(pack2(y[0] * f, y[1] * f), pack2(y[2] * f, y[3] * f), pack2(y[4] * f, y[5] * f),
-                                  pack2(y[6] * f, y[7] * f));
-        }
+      for (int c = 0; c < 4; c++) {
+        uint32_t v[16];
+        tmem_ld_32x32b_x16(trow + 128 + half * 64 + c * 16, v);
+        tmem_ld_wait();
+        const float* x = reinterpret_cast<const float*>(v);
+        dst[2 * c] = make_uint4(pack2(x[0] * f, x[1] * f), pack2(x[2] * f, x[3] * f), pack2(x[4] * f, x[5] * f),
+                                pack2(x[6] * f, x[7] * f));
+        dst[2 * c + 1] = make_uint4(pack2(x[8] * f, x[9] * f), pack2(x[10] * f, x[11] * f),
+                                    pack2(x[12] * f, x[13] * f), pack2(x[14] * f, x[15] * f));
       }
     }
   }
@@ -477,16 +502,18 @@ __global__ void __launch_bounds__(192, 2) k_attn_bwd_kv_tc(const __grid_constant
 
 // ============================================================================
 // backward, dQ: one CTA per (128-query block, b, h), walking 64-key blocks
-// up to the diagonal.  S = Q K^T, dP = dO V^T -> dS (bf16, written into TMEM); dQ += dS K
+// up to the diagonal.  S = Q K^T, dP = dO V^T -> dS (bf16, written into TMEM);
+// dQ += dS K.  Eight math warps as in the dK/dV kernel.
 // smem: Q | dO | (K, V)[2 stages] | barriers   (~64 KB)
 // TMEM: S [0,64), dP [64,128), dQ [128,192)  (256 allocated)
 // ============================================================================
 constexpr int Q_Q = 0, Q_DO = TILE, Q_ST = 2 * TILE, Q_BAR = 4 * TILE;
 constexpr int Q_SMEM = Q_BAR + 128;
 
-__global__ void __launch_bounds__(192, 2) k_attn_bwd_q_tc(const __grid_constant__ CUtensorMap tq,
-                                                          const __grid_constant__ CUtensorMap tdo,
-                                                          const __grid_constant__ CUtensorMap tkv64, AttnTcArgs a) {
+template <bool DROP>
+__global__ void __launch_bounds__(320, 2) k_attn_bwd_q8(const __grid_constant__ CUtensorMap tq,
+                                                        const __grid_constant__ CUtensorMap tdo,
+                                                        const __grid_constant__ CUtensorMap tkv64, AttnTcArgs a) {
   extern __shared__ __align__(1024) uint8_t smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (smem_u32(smem) & 1023) {
@@ -504,7 +531,7 @@ __global__ void __launch_bounds__(192, 2) k_attn_bwd_q_tc(const __grid_constant_
   const int qb = nqb - 1 - (int)blockIdx.x;
   const int bh = blockIdx.y, b = bh / a.H, h = bh % a.H;
   const int row0 = b * a.T;
-  const int nkb = 2 * (qb + 1);  // 64-key blocks up to and including the diagonal
+  const int nkb = 2 * (qb + 1);
 
   if (threadIdx.x == 0) {
     mbar_init(qd_full, 1);
@@ -513,7 +540,7 @@ __global__ void __launch_bounds__(192, 2) k_attn_bwd_q_tc(const __grid_constant_
     mbar_init(kv_empty0, 1);
     mbar_init(kv_empty0 + 8, 1);
     mbar_init(sdp_full, 1);
-    mbar_init(ds_full, 4);
+    mbar_init(ds_full, 8);
     mbar_init(acc_full, 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -564,13 +591,14 @@ __global__ void __launch_bounds__(192, 2) k_attn_bwd_q_tc(const __grid_constant_
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 4; kk++)
-          mma_bf16_ts(tmem + 128, tmem + 8 * kk, desc_mn64(k, kk), id_acc, (j > 0 || kk > 0));
+          mma_bf16_ts(tmem + 128, tmem + acol(kk), desc_mn64(k, kk), id_acc, (j > 0 || kk > 0));
         mma_commit(kv_empty0 + 8 * s);
       }
       mma_commit(acc_full);
     }
   } else {
     const int quad = warp & 3;
+    const int half = (warp - 2) >> 2;
     const int r = quad * 32 + lane;
     const int qi = qb * 128 + r;
     const uint32_t trow = tmem + ((uint32_t)(quad * 32) << 16);
@@ -583,34 +611,31 @@ __global__ void __launch_bounds__(192, 2) k_attn_bwd_q_tc(const __grid_constant_
       if (!(ok = mbar_wait(sdp_full, j & 1, abort_flag, a.flags))) break;
       tc_fence_after();
       const int key0 = j * 64;
-      const bool diag = key0 + 64 > qb * 128;
-      uint32_t s0[32], s1[32], d0[32], d1[32];
-      tmem_ld_32x32b_x32(trow, s0);
-      tmem_ld_32x32b_x32(trow + 32, s1);
-      tmem_ld_32x32b_x32(trow + 64, d0);
-      tmem_ld_32x32b_x32(trow + 96, d1);
-      tmem_ld_wait();
-      uint32_t pd0[16], pd1[16];
+      const int lim = qi - key0;  // key column c is visible iff c <= lim
 #pragma unroll
-      for (int e = 0; e < 32; e += 2) {
-        float dsv[4];
+      for (int sub = 0; sub < 2; sub++) {
+        const int c0 = half * 32 + sub * 16;
+        uint32_t sv[16], dv[16];
+        tmem_ld_32x32b_x16(trow + c0, sv);
+        tmem_ld_32x32b_x16(trow + 64 + c0, dv);
+        tmem_ld_wait();
+        uint32_t pd[8];
 #pragma unroll
-        for (int u = 0; u < 4; u++) {
-          const int col = (u >> 1) * 32 + e + (u & 1);
-          const uint32_t sraw = (u >> 1) ? s1[e + (u & 1)] : s0[e + (u & 1)];
-          const uint32_t draw = (u >> 1) ? d1[e + (u & 1)] : d0[e + (u & 1)];
-          float p = ex2(fmaf(__uint_as_float(sraw), sl2, -lse2));
-          if (diag && key0 + col > qi) p = 0.f;
-          float dp = __uint_as_float(draw);
-          if (a.drop.active) dp *= drop_mul(a.drop, ebase + key0 + col);
-          dsv[u] = p * (dp - Di);
+        for (int e = 0; e < 16; e += 2) {
+          float ds2[2];
+#pragma unroll
+          for (int u = 0; u < 2; u++) {
+            const int col = c0 + e + u;
+            float p = ex2(fmaf(__uint_as_float(sv[e + u]), sl2, -lse2));
+            if (col > lim) p = 0.f;
+            float dp = __uint_as_float(dv[e + u]);
+            if (DROP) dp *= drop_mul(a.drop, ebase + key0 + col);
+            ds2[u] = p * (dp - Di);
+          }
+          pd[e >> 1] = pack2(ds2[0], ds2[1]);
         }
-        pd0[e >> 1] = pack2(dsv[0], dsv[1]);
-        pd1[e >> 1] = pack2(dsv[2], dsv[3]);
+        tmem_st_32x32b_x8(trow + pcol(c0), pd);
       }
-      // dS (bf16 pairs) over the first 32 columns of S: the TMEM A operand of dQ += dS K
-      tmem_st_32x32b_x16(trow, pd0);
-      tmem_st_32x32b_x16(trow + 16, pd1);
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
@@ -618,18 +643,18 @@ __global__ void __launch_bounds__(192, 2) k_attn_bwd_q_tc(const __grid_constant_
     }
     if (ok && mbar_wait(acc_full, 0, abort_flag, a.flags)) {
       tc_fence_after();
-      uint4* dst = reinterpret_cast<uint4*>(a.dqkv + (size_t)(row0 + qi) * (3 * a.H * 64) + (size_t)h * 64);
-      uint32_t v0[32], v1[32];
-      ld64(trow + 128, v0, v1);
+      uint4* dst = reinterpret_cast<uint4*>(a.dqkv + (size_t)(row0 + qi) * (3 * a.H * 64) + (size_t)h * 64 + half * 32);
       const float f = a.scale;
 #pragma unroll
-      for (int q = 0; q < 4; q++) {
-        const float* x = reinterpret_cast<const float*>(v0) + 8 * q;
-        const float* y = reinterpret_cast<const float*>(v1) + 8 * q;
-        dst[q] = make_uint4(pack2(x[0] * f, x[1] * f), pack2(x[2] * f, x[3] * f), pack2(x[4] * f, x[5] * f),
-                            pack2(x[6] * f, x[7] * f));
-        dst[4 + q] = make_uint4(pack2(y[0] * f, y[1] * f), pack2(y[2] * f, y[3] * f), pack2(y[4] * f, y[5] * f),
-                                pack2(y[6] * f, y[7] * f));
+      for (int c = 0; c < 2; c++) {
+        uint32_t v[16];
+        tmem_ld_32x32b_x16(trow + 128 + half * 32 + c * 16, v);
+        tmem_ld_wait();
+        const float* x = reinterpret_cast<const float*>(v);
+        dst[2 * c] = make_uint4(pack2(x[0] * f, x[1] * f), pack2(x[2] * f, x[3] * f), pack2(x[4] * f, x[5] * f),
+                                pack2(x[6] * f, x[7] * f));
+        dst[2 * c + 1] = make_uint4(pack2(x[8] * f, x[9] * f), pack2(x[10] * f, x[11] * f),
+                                    pack2(x[12] * f, x[13] * f), pack2(x[14] * f, x[15] * f));
       }
     }
   }
@@ -732,12 +757,14 @@ void attn_fwd_tc(Ctx& c, const AttnDesc& d) {
   }
   static bool attr = false;
   if (!attr) {
-    cudaFuncSetAttribute(k_attn_fwd_db, cudaFuncAttributeMaxDynamicSharedMemorySize, D_SMEM);
+    cudaFuncSetAttribute(k_attn_fwd_o<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, D_SMEM);
+    cudaFuncSetAttribute(k_attn_fwd_o<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, D_SMEM);
     attr = true;
   }
   dim3 grid(d.T / 128, d.B * d.H);
   LaunchScope s(c, "attn_fwd_tc");
-  k_attn_fwd_db<<<grid, 192, D_SMEM, c.stream>>>(tq, tkv64, make_args(d, c.flags));
+  if (d.drop.active) k_attn_fwd_o<true><<<grid, 192, D_SMEM, c.stream>>>(tq, tkv64, make_args(d, c.flags));
+  else k_attn_fwd_o<false><<<grid, 192, D_SMEM, c.stream>>>(tq, tkv64, make_args(d, c.flags));
 }
 
 void attn_bwd_tc(Ctx& c, const AttnDesc& d) {
@@ -757,19 +784,24 @@ void attn_bwd_tc(Ctx& c, const AttnDesc& d) {
   }
   static bool attr = false;
   if (!attr) {
-    cudaFuncSetAttribute(k_attn_bwd_kv_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, K_SMEM);
-    cudaFuncSetAttribute(k_attn_bwd_q_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, Q_SMEM);
+    cudaFuncSetAttribute(k_attn_bwd_kv8<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, K_SMEM);
+    cudaFuncSetAttribute(k_attn_bwd_kv8<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, K_SMEM);
+    cudaFuncSetAttribute(k_attn_bwd_q8<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, Q_SMEM);
+    cudaFuncSetAttribute(k_attn_bwd_q8<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, Q_SMEM);
     attr = true;
   }
   AttnTcArgs a = make_args(d, c.flags);
   dim3 grid(d.T / 128, d.B * d.H);
+  const bool drop = d.drop.active;
   {
     LaunchScope s(c, "attn_bwd_kv_tc");
-    k_attn_bwd_kv_tc<<<grid, 192, K_SMEM, c.stream>>>(tkv, tq64, tdo64, a);
+    if (drop) k_attn_bwd_kv8<true><<<grid, 320, K_SMEM, c.stream>>>(tkv, tq64, tdo64, a);
+    else k_attn_bwd_kv8<false><<<grid, 320, K_SMEM, c.stream>>>(tkv, tq64, tdo64, a);
   }
   {
     LaunchScope s(c, "attn_bwd_q_tc");
-    k_attn_bwd_q_tc<<<grid, 192, Q_SMEM, c.stream>>>(tkv, tdo, tkv64, a);
+    if (drop) k_attn_bwd_q8<true><<<grid, 320, Q_SMEM, c.stream>>>(tkv, tdo, tkv64, a);
+    else k_attn_bwd_q8<false><<<grid, 320, Q_SMEM, c.stream>>>(tkv, tdo, tkv64, a);
   }
 }
 
