@@ -310,6 +310,40 @@ __device__ __forceinline__ int pcol(int c) { return (c & 32) + ((c & 31) >> 1); 
 // TMEM A-operand column of K-step kk (16 elements) under that layout
 __device__ __forceinline__ uint32_t acol(int kk) { return (uint32_t)((kk >> 1) * 32 + (kk & 1) * 8); }
 
+// two fp32 lanes in one 64-bit register: the sm_100 f32x2 FMA-pipe forms
+// (each lane rounds exactly like the scalar instruction)
+__device__ __forceinline__ uint64_t f2(float a, float b) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ float2 f2split(uint64_t r) {
+  float2 v;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(v.x), "=f"(v.y) : "l"(r));
+  return v;
+}
+__device__ __forceinline__ uint64_t f2fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2mul(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2sub(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint32_t pack2v(uint64_t v) {
+  const float2 f = f2split(v);
+  return pack2(f.x, f.y);
+}
+
+constexpr int BWD_STAGES = 3;  // Q/dO (or K/V) tiles in flight
+
 // ============================================================================
 // backward, dK and dV: one CTA per (128-key block, b, h), walking 64-query
 // blocks from the key block on.  Keys are the MMA rows:
@@ -317,10 +351,10 @@ __device__ __forceinline__ uint32_t acol(int kk) { return (uint32_t)((kk >> 1) *
 //   dV += P~^T dO,  dK += dS^T Q
 // Eight math warps, two per TMEM lane quadrant, each take 32 of the 64 query
 // columns of a block (the backward has no row reductions).
-// smem: K | V | (Q, dO)[2 stages] | (lse, D)[2] | barriers (~65 KB)
+// smem: K | V | (Q, dO)[3 stages] | (lse, D)[3] | barriers (~82 KB)
 // TMEM: S^T [0,64), dP^T [64,128), dV [128,192), dK [192,256)
 // ============================================================================
-constexpr int K_K = 0, K_V = TILE, K_ST = 2 * TILE, K_LD = 4 * TILE, K_BAR = K_LD + 1024;
+constexpr int K_K = 0, K_V = TILE, K_ST = 2 * TILE, K_LD = (2 + BWD_STAGES) * TILE, K_BAR = K_LD + 2048;
 constexpr int K_SMEM = K_BAR + 128;
 
 template <bool DROP>
@@ -334,15 +368,16 @@ __global__ void __launch_bounds__(320, 2) k_attn_bwd_kv8(const __grid_constant__
     return;
   }
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + K_BAR);
-  uint32_t kv_full = smem_u32(bars + 0), st_full0 = smem_u32(bars + 1), st_empty0 = smem_u32(bars + 3);
-  uint32_t sdp_full = smem_u32(bars + 5), pds_full = smem_u32(bars + 6), acc_full = smem_u32(bars + 7);
-  uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + 8);
+  const uint32_t kv_full = smem_u32(bars + 0), st_full0 = smem_u32(bars + 1),
+                 st_empty0 = smem_u32(bars + 1 + BWD_STAGES);
+  const uint32_t sdp_full = smem_u32(bars + 1 + 2 * BWD_STAGES), pds_full = sdp_full + 8, acc_full = sdp_full + 16;
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + 4 + 2 * BWD_STAGES);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tslot + 1);
-  const float* sld = reinterpret_cast<const float*>(smem + K_LD);  // [2][lse 64 | D 64]
+  const float* sld = reinterpret_cast<const float*>(smem + K_LD);  // [stage][lse 64 | D 64]
   const uint32_t sb = smem_u32(smem);
 
   const int nq64 = a.T / 64;
-  const int kb = (int)blockIdx.x;
+  const int kb = (int)blockIdx.x;  // key block 0 has the most query blocks: first
   const int bh = blockIdx.y, b = bh / a.H, h = bh % a.H;
   const int row0 = b * a.T;
   const int i0 = 2 * kb;
@@ -350,10 +385,10 @@ __global__ void __launch_bounds__(320, 2) k_attn_bwd_kv8(const __grid_constant__
 
   if (threadIdx.x == 0) {
     mbar_init(kv_full, 1);
-    mbar_init(st_full0, 1);
-    mbar_init(st_full0 + 8, 1);
-    mbar_init(st_empty0, 1);
-    mbar_init(st_empty0 + 8, 1);
+    for (int s = 0; s < BWD_STAGES; s++) {
+      mbar_init(st_full0 + 8 * s, 1);
+      mbar_init(st_empty0 + 8 * s, 1);
+    }
     mbar_init(sdp_full, 1);
     mbar_init(pds_full, 8);
     mbar_init(acc_full, 1);
@@ -378,9 +413,9 @@ __global__ void __launch_bounds__(320, 2) k_attn_bwd_kv8(const __grid_constant__
       tma_load_3d(sb + K_K, &tkv, kv_full, 0, a.H + h, row0 + kb * 128);
       tma_load_3d(sb + K_V, &tkv, kv_full, 0, 2 * a.H + h, row0 + kb * 128);
       for (int it = 0; it < nit; it++) {
-        int i = i0 + it, s = it & 1;
-        uint32_t fb = st_full0 + 8 * s;
-        if (!mbar_wait(st_empty0 + 8 * s, ((it >> 1) & 1) ^ 1, abort_flag, a.flags)) break;
+        const int i = i0 + it, s = it % BWD_STAGES;
+        const uint32_t fb = st_full0 + 8 * s;
+        if (!mbar_wait(st_empty0 + 8 * s, ((it / BWD_STAGES) & 1) ^ 1, abort_flag, a.flags)) break;
         mbar_expect_tx(fb, 2 * HTILE + 512);
         tma_load_3d(sb + K_ST + s * TILE, &tq64, fb, 0, h, row0 + i * 64);
         tma_load_3d(sb + K_ST + s * TILE + HTILE, &tdo64, fb, 0, h, row0 + i * 64);
@@ -394,10 +429,10 @@ __global__ void __launch_bounds__(320, 2) k_attn_bwd_kv8(const __grid_constant__
       constexpr uint32_t id_acc = idesc_bf16_f32(128, 64, false, true);
       bool ok = mbar_wait(kv_full, 0, abort_flag, a.flags);
       for (int it = 0; it < nit && ok; it++) {
-        int s = it & 1;
-        if (!(ok = mbar_wait(st_full0 + 8 * s, (it >> 1) & 1, abort_flag, a.flags))) break;
+        const int s = it % BWD_STAGES;
+        if (!(ok = mbar_wait(st_full0 + 8 * s, (it / BWD_STAGES) & 1, abort_flag, a.flags))) break;
         tc_fence_after();
-        uint32_t q = sb + K_ST + s * TILE, dO = q + HTILE;
+        const uint32_t q = sb + K_ST + s * TILE, dO = q + HTILE;
 #pragma unroll
         for (int kk = 0; kk < 4; kk++)
           mma_bf16_ss(tmem, desc_k(sb + K_K, TILE, kk), desc_k(q, HTILE, kk), id_s, kk > 0);
@@ -423,16 +458,17 @@ __global__ void __launch_bounds__(320, 2) k_attn_bwd_kv8(const __grid_constant__
     const int r = quad * 32 + lane;
     const int kj = kb * 128 + r;
     const uint32_t trow = tmem + ((uint32_t)(quad * 32) << 16);
-    const float sl2 = a.scale_log2;
+    const uint64_t sl2x2 = f2(a.scale_log2, a.scale_log2), nlog2e = f2(-LOG2E, -LOG2E);
     bool ok = true;
     for (int it = 0; it < nit; it++) {
       const int i = i0 + it;
       const int q0 = i * 64;
-      const float* ld = sld + (it & 1) * 128;  // lse[64] | D[64] of this query block
-      if (!(ok = mbar_wait(st_full0 + 8 * (it & 1), (it >> 1) & 1, abort_flag, a.flags))) break;
+      const float* ld = sld + (it % BWD_STAGES) * 128;  // lse[64] | D[64] of this query block
+      if (!(ok = mbar_wait(st_full0 + 8 * (it % BWD_STAGES), (it / BWD_STAGES) & 1, abort_flag, a.flags))) break;
       if (!(ok = mbar_wait(sdp_full, it & 1, abort_flag, a.flags))) break;
       tc_fence_after();
-      const int lim = kj - q0;  // query column c is masked iff c < lim
+      const int lim = kj - q0;                        // query column c is masked iff c < lim
+      const bool masked = q0 < kb * 128 + 128;        // only blocks that reach this CTA's keys
 #pragma unroll
       for (int sub = 0; sub < 2; sub++) {
         const int c0 = half * 32 + sub * 16;
@@ -445,27 +481,47 @@ __global__ void __launch_bounds__(320, 2) k_attn_bwd_kv8(const __grid_constant__
         for (int e = 0; e < 16; e += 4) {
           const float4 l4 = *reinterpret_cast<const float4*>(ld + c0 + e);
           const float4 d4 = *reinterpret_cast<const float4*>(ld + 64 + c0 + e);
-          const float lv[4] = {l4.x, l4.y, l4.z, l4.w}, dd[4] = {d4.x, d4.y, d4.z, d4.w};
-          float pv[4], dsv[4];
-#pragma unroll
-          for (int u = 0; u < 4; u++) {
-            const int col = c0 + e + u;
-            float p = ex2(fmaf(__uint_as_float(sv[e + u]), sl2, -lv[u] * LOG2E));
-            if (col < lim) p = 0.f;
-            float dp = __uint_as_float(dv[e + u]);
-            if (DROP) {
-              float mk = drop_mul(a.drop, ((uint64_t)bh * a.T + q0 + col) * a.T + kj);
-              pv[u] = p * mk;
-              dp *= mk;
-            } else {
-              pv[u] = p;
+          if (!DROP) {
+            // P = 2^(S sl2 - lse log2 e);  dS = P (dP - D)
+            const uint64_t x01 = f2fma(f2(__uint_as_float(sv[e]), __uint_as_float(sv[e + 1])), sl2x2,
+                                       f2mul(f2(l4.x, l4.y), nlog2e));
+            const uint64_t x23 = f2fma(f2(__uint_as_float(sv[e + 2]), __uint_as_float(sv[e + 3])), sl2x2,
+                                       f2mul(f2(l4.z, l4.w), nlog2e));
+            const float2 y01 = f2split(x01), y23 = f2split(x23);
+            float p0 = ex2(y01.x), p1 = ex2(y01.y), p2 = ex2(y23.x), p3 = ex2(y23.y);
+            if (masked) {
+              const int col = c0 + e;
+              if (col < lim) p0 = 0.f;
+              if (col + 1 < lim) p1 = 0.f;
+              if (col + 2 < lim) p2 = 0.f;
+              if (col + 3 < lim) p3 = 0.f;
             }
-            dsv[u] = p * (dp - dd[u]);
+            const uint64_t P01 = f2(p0, p1), P23 = f2(p2, p3);
+            const uint64_t ds01 = f2mul(P01, f2sub(f2(__uint_as_float(dv[e]), __uint_as_float(dv[e + 1])),
+                                                   f2(d4.x, d4.y)));
+            const uint64_t ds23 = f2mul(P23, f2sub(f2(__uint_as_float(dv[e + 2]), __uint_as_float(dv[e + 3])),
+                                                   f2(d4.z, d4.w)));
+            pp[e >> 1] = pack2(p0, p1);
+            pp[(e >> 1) + 1] = pack2(p2, p3);
+            pd[e >> 1] = pack2v(ds01);
+            pd[(e >> 1) + 1] = pack2v(ds23);
+          } else {
+            const float lv[4] = {l4.x, l4.y, l4.z, l4.w}, dd[4] = {d4.x, d4.y, d4.z, d4.w};
+            float pv[4], dsv[4];
+#pragma unroll
+            for (int u = 0; u < 4; u++) {
+              const int col = c0 + e + u;
+              float p = ex2(fmaf(__uint_as_float(sv[e + u]), a.scale_log2, lv[u] * -LOG2E));
+              if (masked && col < lim) p = 0.f;
+              const float mk = drop_mul(a.drop, ((uint64_t)bh * a.T + q0 + col) * a.T + kj);
+              pv[u] = p * mk;
+              dsv[u] = p * (__uint_as_float(dv[e + u]) * mk - dd[u]);
+            }
+            pp[e >> 1] = pack2(pv[0], pv[1]);
+            pp[(e >> 1) + 1] = pack2(pv[2], pv[3]);
+            pd[e >> 1] = pack2(dsv[0], dsv[1]);
+            pd[(e >> 1) + 1] = pack2(dsv[2], dsv[3]);
           }
-          pp[e >> 1] = pack2(pv[0], pv[1]);
-          pp[(e >> 1) + 1] = pack2(pv[2], pv[3]);
-          pd[e >> 1] = pack2(dsv[0], dsv[1]);
-          pd[(e >> 1) + 1] = pack2(dsv[2], dsv[3]);
         }
         tmem_st_32x32b_x8(trow + pcol(c0), pp);
         tmem_st_32x32b_x8(trow + 64 + pcol(c0), pd);
@@ -504,10 +560,10 @@ __global__ void __launch_bounds__(320, 2) k_attn_bwd_kv8(const __grid_constant__
 // backward, dQ: one CTA per (128-query block, b, h), walking 64-key blocks
 // up to the diagonal.  S = Q K^T, dP = dO V^T -> dS (bf16, written into TMEM);
 // dQ += dS K.  Eight math warps as in the dK/dV kernel.
-// smem: Q | dO | (K, V)[2 stages] | barriers   (~64 KB)
+// smem: Q | dO | (K, V)[3 stages] | barriers   (~80 KB)
 // TMEM: S [0,64), dP [64,128), dQ [128,192)  (256 allocated)
 // ============================================================================
-constexpr int Q_Q = 0, Q_DO = TILE, Q_ST = 2 * TILE, Q_BAR = 4 * TILE;
+constexpr int Q_Q = 0, Q_DO = TILE, Q_ST = 2 * TILE, Q_BAR = (2 + BWD_STAGES) * TILE;
 constexpr int Q_SMEM = Q_BAR + 128;
 
 template <bool DROP>
@@ -521,9 +577,10 @@ __global__ void __launch_bounds__(320, 2) k_attn_bwd_q8(const __grid_constant__ 
     return;
   }
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Q_BAR);
-  uint32_t qd_full = smem_u32(bars + 0), kv_full0 = smem_u32(bars + 1), kv_empty0 = smem_u32(bars + 3);
-  uint32_t sdp_full = smem_u32(bars + 5), ds_full = smem_u32(bars + 6), acc_full = smem_u32(bars + 7);
-  uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + 8);
+  const uint32_t qd_full = smem_u32(bars + 0), kv_full0 = smem_u32(bars + 1),
+                 kv_empty0 = smem_u32(bars + 1 + BWD_STAGES);
+  const uint32_t sdp_full = smem_u32(bars + 1 + 2 * BWD_STAGES), ds_full = sdp_full + 8, acc_full = sdp_full + 16;
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + 4 + 2 * BWD_STAGES);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tslot + 1);
   const uint32_t sb = smem_u32(smem);
 
@@ -531,14 +588,14 @@ __global__ void __launch_bounds__(320, 2) k_attn_bwd_q8(const __grid_constant__ 
   const int qb = nqb - 1 - (int)blockIdx.x;
   const int bh = blockIdx.y, b = bh / a.H, h = bh % a.H;
   const int row0 = b * a.T;
-  const int nkb = 2 * (qb + 1);
+  const int nkb = 2 * (qb + 1);  // 64-key blocks up to and including the diagonal
 
   if (threadIdx.x == 0) {
     mbar_init(qd_full, 1);
-    mbar_init(kv_full0, 1);
-    mbar_init(kv_full0 + 8, 1);
-    mbar_init(kv_empty0, 1);
-    mbar_init(kv_empty0 + 8, 1);
+    for (int s = 0; s < BWD_STAGES; s++) {
+      mbar_init(kv_full0 + 8 * s, 1);
+      mbar_init(kv_empty0 + 8 * s, 1);
+    }
     mbar_init(sdp_full, 1);
     mbar_init(ds_full, 8);
     mbar_init(acc_full, 1);
@@ -563,9 +620,9 @@ __global__ void __launch_bounds__(320, 2) k_attn_bwd_q8(const __grid_constant__ 
       tma_load_3d(sb + Q_Q, &tq, qd_full, 0, h, row0 + qb * 128);
       tma_load_3d(sb + Q_DO, &tdo, qd_full, 0, h, row0 + qb * 128);
       for (int j = 0; j < nkb; j++) {
-        int s = j & 1;
-        uint32_t fb = kv_full0 + 8 * s;
-        if (!mbar_wait(kv_empty0 + 8 * s, ((j >> 1) & 1) ^ 1, abort_flag, a.flags)) break;
+        const int s = j % BWD_STAGES;
+        const uint32_t fb = kv_full0 + 8 * s;
+        if (!mbar_wait(kv_empty0 + 8 * s, ((j / BWD_STAGES) & 1) ^ 1, abort_flag, a.flags)) break;
         mbar_expect_tx(fb, 2 * HTILE);
         tma_load_3d(sb + Q_ST + s * TILE, &tkv64, fb, 0, a.H + h, row0 + j * 64);
         tma_load_3d(sb + Q_ST + s * TILE + HTILE, &tkv64, fb, 0, 2 * a.H + h, row0 + j * 64);
@@ -577,10 +634,10 @@ __global__ void __launch_bounds__(320, 2) k_attn_bwd_q8(const __grid_constant__ 
       constexpr uint32_t id_acc = idesc_bf16_f32(128, 64, false, true);
       bool ok = mbar_wait(qd_full, 0, abort_flag, a.flags);
       for (int j = 0; j < nkb && ok; j++) {
-        int s = j & 1;
-        if (!(ok = mbar_wait(kv_full0 + 8 * s, (j >> 1) & 1, abort_flag, a.flags))) break;
+        const int s = j % BWD_STAGES;
+        if (!(ok = mbar_wait(kv_full0 + 8 * s, (j / BWD_STAGES) & 1, abort_flag, a.flags))) break;
         tc_fence_after();
-        uint32_t k = sb + Q_ST + s * TILE, v = k + HTILE;
+        const uint32_t k = sb + Q_ST + s * TILE, v = k + HTILE;
 #pragma unroll
         for (int kk = 0; kk < 4; kk++) mma_bf16_ss(tmem, desc_k(sb + Q_Q, TILE, kk), desc_k(k, HTILE, kk), id_s, kk > 0);
 #pragma unroll
@@ -602,16 +659,17 @@ __global__ void __launch_bounds__(320, 2) k_attn_bwd_q8(const __grid_constant__ 
     const int r = quad * 32 + lane;
     const int qi = qb * 128 + r;
     const uint32_t trow = tmem + ((uint32_t)(quad * 32) << 16);
-    const float sl2 = a.scale_log2;
     const float lse2 = a.lse[(size_t)bh * a.T + qi] * LOG2E;
     const float Di = a.dsum[(size_t)bh * a.T + qi];
+    const uint64_t sl2x2 = f2(a.scale_log2, a.scale_log2), nlse2 = f2(-lse2, -lse2), Dx2 = f2(Di, Di);
     const uint64_t ebase = ((uint64_t)bh * a.T + qi) * a.T;
     bool ok = true;
     for (int j = 0; j < nkb; j++) {
       if (!(ok = mbar_wait(sdp_full, j & 1, abort_flag, a.flags))) break;
       tc_fence_after();
       const int key0 = j * 64;
-      const int lim = qi - key0;  // key column c is visible iff c <= lim
+      const int lim = qi - key0;                  // key column c is visible iff c <= lim
+      const bool masked = key0 + 64 > qb * 128;   // only the blocks that reach the diagonal
 #pragma unroll
       for (int sub = 0; sub < 2; sub++) {
         const int c0 = half * 32 + sub * 16;
@@ -622,17 +680,19 @@ __global__ void __launch_bounds__(320, 2) k_attn_bwd_q8(const __grid_constant__ 
         uint32_t pd[8];
 #pragma unroll
         for (int e = 0; e < 16; e += 2) {
-          float ds2[2];
-#pragma unroll
-          for (int u = 0; u < 2; u++) {
-            const int col = c0 + e + u;
-            float p = ex2(fmaf(__uint_as_float(sv[e + u]), sl2, -lse2));
-            if (col > lim) p = 0.f;
-            float dp = __uint_as_float(dv[e + u]);
-            if (DROP) dp *= drop_mul(a.drop, ebase + key0 + col);
-            ds2[u] = p * (dp - Di);
+          const int col = c0 + e;
+          const float2 y = f2split(f2fma(f2(__uint_as_float(sv[e]), __uint_as_float(sv[e + 1])), sl2x2, nlse2));
+          float p0 = ex2(y.x), p1 = ex2(y.y);
+          if (masked) {
+            if (col > lim) p0 = 0.f;
+            if (col + 1 > lim) p1 = 0.f;
           }
-          pd[e >> 1] = pack2(ds2[0], ds2[1]);
+          float dp0 = __uint_as_float(dv[e]), dp1 = __uint_as_float(dv[e + 1]);
+          if (DROP) {
+            dp0 *= drop_mul(a.drop, ebase + key0 + col);
+            dp1 *= drop_mul(a.drop, ebase + key0 + col + 1);
+          }
+          pd[e >> 1] = pack2v(f2mul(f2(p0, p1), f2sub(f2(dp0, dp1), Dx2)));
         }
         tmem_st_32x32b_x8(trow + pcol(c0), pd);
       }

@@ -8,14 +8,15 @@
 //               (128-byte swizzle; K-major or MN-major operands, so dX and dW
 //               need no transposed copies)
 //   warp 1      TMEM allocator + MMA issuer (tcgen05.mma, M=128, N=BN, K=16)
-//   warps 2..9  epilogue: two warps per TMEM lane quadrant, each taking half
-//               of the BN columns in 32x32 chunks: tcgen05.ld -> fused
-//               element-wise work -> swizzled shared-memory staging tile ->
-//               TMA tensor store (or TMA reduce-add for gradient
-//               accumulation).  Inputs the epilogue needs (the residual
-//               stream, the saved pre-activation) arrive by TMA into the same
-//               staging tiles, so every global access of the epilogue is a
-//               coalesced bulk transfer.
+//   warps 2..17 epilogue: four warps per TMEM lane quadrant, each taking a
+//               quarter of the BN columns in 32x32 chunks (processed as two
+//               16-column halves): tcgen05.ld -> fused element-wise work ->
+//               swizzled shared-memory staging tile -> TMA tensor store (or
+//               TMA reduce-add for gradient accumulation).  Inputs the
+//               epilogue needs (the residual stream, the saved
+//               pre-activation) arrive by TMA into the same staging tiles,
+//               the first one while the tile's MMAs still run, so every
+//               global access of the epilogue is a coalesced bulk transfer.
 // TMEM holds two BN-column accumulators so the epilogue of tile i overlaps
 // the MMAs of tile i+1.  Every mbarrier wait is bounded.
 #include <cudaTypedefs.h>
@@ -33,7 +34,6 @@ using namespace sm100;
 constexpr int BM = 128, BK = 64;
 constexpr int EPI_WARPS = 16;                // 4 per TMEM lane quadrant
 constexpr int EPI_PARTS = EPI_WARPS / 4;     // column ranges per quadrant
-constexpr int EPI_SETS = 1;                  // staging sets per epilogue warp (2 = double-buffered)
 constexpr int kThreads = 64 + 32 * EPI_WARPS;  // producer, MMA, epilogue warps
 constexpr int EPI_BUF = 4096;                // one 32x32 fp32 (or two bf16) staging tiles
 
@@ -55,7 +55,7 @@ struct TcCfg {
   static constexpr int STAGES = BN == 256 ? 3 : 5;
   static constexpr int TMEM_COLS = 2 * BN;
   static constexpr int EPI_OFF = STAGES * STAGE_BYTES;
-  static constexpr int BAR_OFF = EPI_OFF + EPI_WARPS * EPI_SETS * EPI_BUF;
+  static constexpr int BAR_OFF = EPI_OFF + EPI_WARPS * EPI_BUF;
   static constexpr int SMEM_BYTES = BAR_OFF + 512 + 1024;  // + barriers + alignment slack
 };
 
@@ -72,59 +72,68 @@ __device__ __forceinline__ float2 unpack_bf16(uint32_t u) {
 // fp32 rows are 128 bytes (TMA 128-byte swizzle: 16-byte chunk q of row r at
 // q ^ (r & 7)); bf16 rows are 64 bytes (64-byte swizzle: chunk q at
 // q ^ ((r >> 1) & 3)).  Both keep a warp's 16-byte accesses conflict-free.
-__device__ __forceinline__ void stage_f32(uint32_t buf, int r, const float (&x)[32]) {
+// The epilogue works on half-rows of 16 columns (h = 0, 1) to keep its
+// register footprint small.
+__device__ __forceinline__ void stage_f32(uint32_t buf, int r, int h, const float (&x)[16]) {
 #pragma unroll
-  for (int q = 0; q < 8; q++)
-    st_shared_v4(buf + r * 128 + ((q ^ (r & 7)) << 4), __float_as_uint(x[4 * q]), __float_as_uint(x[4 * q + 1]),
-                 __float_as_uint(x[4 * q + 2]), __float_as_uint(x[4 * q + 3]));
+  for (int qq = 0; qq < 4; qq++)
+    st_shared_v4(buf + r * 128 + (((4 * h + qq) ^ (r & 7)) << 4), __float_as_uint(x[4 * qq]),
+                 __float_as_uint(x[4 * qq + 1]), __float_as_uint(x[4 * qq + 2]), __float_as_uint(x[4 * qq + 3]));
 }
-__device__ __forceinline__ void unstage_f32(uint32_t buf, int r, float (&x)[32]) {
+__device__ __forceinline__ void unstage_f32(uint32_t buf, int r, int h, float (&x)[16]) {
 #pragma unroll
-  for (int q = 0; q < 8; q++) {
-    uint4 u = ld_shared_v4(buf + r * 128 + ((q ^ (r & 7)) << 4));
-    x[4 * q] = __uint_as_float(u.x);
-    x[4 * q + 1] = __uint_as_float(u.y);
-    x[4 * q + 2] = __uint_as_float(u.z);
-    x[4 * q + 3] = __uint_as_float(u.w);
+  for (int qq = 0; qq < 4; qq++) {
+    uint4 u = ld_shared_v4(buf + r * 128 + (((4 * h + qq) ^ (r & 7)) << 4));
+    x[4 * qq] = __uint_as_float(u.x);
+    x[4 * qq + 1] = __uint_as_float(u.y);
+    x[4 * qq + 2] = __uint_as_float(u.z);
+    x[4 * qq + 3] = __uint_as_float(u.w);
   }
 }
-__device__ __forceinline__ void stage_bf16(uint32_t buf, int r, const float (&x)[32]) {
+__device__ __forceinline__ void stage_bf16(uint32_t buf, int r, int h, const float (&x)[16]) {
 #pragma unroll
-  for (int q = 0; q < 4; q++)
-    st_shared_v4(buf + r * 64 + ((q ^ ((r >> 1) & 3)) << 4), pack_bf16(x[8 * q], x[8 * q + 1]),
-                 pack_bf16(x[8 * q + 2], x[8 * q + 3]), pack_bf16(x[8 * q + 4], x[8 * q + 5]),
-                 pack_bf16(x[8 * q + 6], x[8 * q + 7]));
+  for (int qq = 0; qq < 2; qq++)
+    st_shared_v4(buf + r * 64 + (((2 * h + qq) ^ ((r >> 1) & 3)) << 4), pack_bf16(x[8 * qq], x[8 * qq + 1]),
+                 pack_bf16(x[8 * qq + 2], x[8 * qq + 3]), pack_bf16(x[8 * qq + 4], x[8 * qq + 5]),
+                 pack_bf16(x[8 * qq + 6], x[8 * qq + 7]));
 }
-__device__ __forceinline__ void unstage_bf16(uint32_t buf, int r, float (&x)[32]) {
+__device__ __forceinline__ void unstage_bf16(uint32_t buf, int r, int h, float (&x)[16]) {
 #pragma unroll
-  for (int q = 0; q < 4; q++) {
-    uint4 u = ld_shared_v4(buf + r * 64 + ((q ^ ((r >> 1) & 3)) << 4));
+  for (int qq = 0; qq < 2; qq++) {
+    uint4 u = ld_shared_v4(buf + r * 64 + (((2 * h + qq) ^ ((r >> 1) & 3)) << 4));
     uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
     for (int k = 0; k < 4; k++) {
       float2 f = unpack_bf16(w[k]);
-      x[8 * q + 2 * k] = f.x;
-      x[8 * q + 2 * k + 1] = f.y;
+      x[8 * qq + 2 * k] = f.x;
+      x[8 * qq + 2 * k + 1] = f.y;
     }
   }
 }
 
-__device__ __forceinline__ void add_bias(const TcArgs& p, int col0, float (&v)[32]) {
-  if (!p.bias) return;
-  if (col0 + 32 <= p.N) {
+// The 16 bias values of a half-row, loaded before the TMEM wait so that their
+// latency overlaps it (zeros past N).
+__device__ __forceinline__ void load_bias(const TcArgs& p, int col0, float4 (&b)[4]) {
+  if (col0 + 16 <= p.N) {
     const float4* b4 = reinterpret_cast<const float4*>(p.bias + col0);
 #pragma unroll
-    for (int i = 0; i < 8; i++) {
-      float4 b = b4[i];
-      v[4 * i] += b.x;
-      v[4 * i + 1] += b.y;
-      v[4 * i + 2] += b.z;
-      v[4 * i + 3] += b.w;
-    }
+    for (int i = 0; i < 4; i++) b[i] = b4[i];
   } else {
 #pragma unroll
-    for (int i = 0; i < 32; i++)
-      if (col0 + i < p.N) v[i] += p.bias[col0 + i];
+    for (int i = 0; i < 4; i++) {
+      const int c = col0 + 4 * i;
+      b[i] = make_float4(c < p.N ? p.bias[c] : 0.f, c + 1 < p.N ? p.bias[c + 1] : 0.f,
+                         c + 2 < p.N ? p.bias[c + 2] : 0.f, c + 3 < p.N ? p.bias[c + 3] : 0.f);
+    }
+  }
+}
+__device__ __forceinline__ void add_bias(const float4 (&b)[4], float (&v)[16]) {
+#pragma unroll
+  for (int i = 0; i < 4; i++) {
+    v[4 * i] += b[i].x;
+    v[4 * i + 1] += b[i].y;
+    v[4 * i + 2] += b[i].z;
+    v[4 * i + 3] += b[i].w;
   }
 }
 
@@ -270,14 +279,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int quad = warp & 3;        // TMEM lanes quad*32 .. quad*32+31
     const int part = ew >> 2;         // which of the EPI_PARTS column ranges
     constexpr int CPW = BN / 32 / EPI_PARTS;  // 32-column chunks per warp and tile
-    // EPI_SETS 4 KB staging sets per warp, used by consecutive chunks in turn:
-    // a set holds one fp32 tile, or two bf16 tiles (A at +0, B at +2 KB)
-    const uint32_t stg = smem_u32(smem + C::EPI_OFF + ew * EPI_SETS * EPI_BUF);
-    int set = 0;
+    // one 4 KB staging set per warp: one fp32 tile, or two bf16 tiles (A at
+    // +0, B at +2 KB)
+    const uint32_t stg = smem_u32(smem + C::EPI_OFF + ew * EPI_BUF);
     const uint32_t lbar = smem_u32(&ebar[ew]);
     uint32_t lphase = 0;
     const int kind = p.kind;
     const bool f32_in = kind == EPI_RESADD, bf16_in = kind == EPI_ACT_BWD;
+    const bool has_bias = p.bias && p.splits == 1 && kind != EPI_ACT_BWD && kind < EPI_ACC_F32;
     int acc = 0;
     uint32_t acc_phase = 0;
     bool ok = true;
@@ -285,81 +294,93 @@ __global__ void __launch_bounds__(kThreads, 1)
       int split = t / (p.num_m * p.num_n);
       int r = t % (p.num_m * p.num_n);
       int mb = p.n_fast ? r / p.num_n : r % p.num_m, nb = p.n_fast ? r % p.num_n : r / p.num_m;
-      if (!(ok = mbar_wait(smem_u32(&tfull[acc]), acc_phase, abort_flag, p.flags))) break;
-      tc_fence_after();
       const int row0 = mb * BM + quad * 32;
       const long row = row0 + lane;
-      const uint32_t tbase = tmem_base + ((uint32_t)(quad * 32) << 16) + acc * BN;
-#pragma unroll 1
-      for (int c = part * CPW; c < (part + 1) * CPW; c++) {
-        const int col0 = nb * BN + c * 32;
-        uint32_t raw[32];
-        tmem_ld_32x32b_x32(tbase + c * 32, raw);
-        const uint32_t bufA = stg + set * EPI_BUF, bufB = bufA + 2048;
-        if (EPI_SETS == 2) {
-          set ^= 1;
-          if (lane == 0) bulk_wait_read1();  // the set used two chunks ago is free again
-        } else {
-          if (lane == 0) bulk_wait_read0();  // the previous chunk's stores have read the set
+      const int c_first = part * CPW;
+      // the epilogue input of a warp's first chunk (residual stream or saved
+      // pre-activation) is fetched while the tile's MMAs still run
+      auto fetch_input = [&](int c) {
+        if (lane == 0) {
+          bulk_wait_read0();  // the previous chunk's stores have read the staging set
+          mbar_expect_tx(lbar, f32_in ? 4096 : 2048);
+          tma_load_2d(f32_in ? stg : stg + 2048, &tm_in, lbar, nb * BN + c * 32, row0);
         }
         __syncwarp();
+      };
+      if (f32_in || bf16_in) fetch_input(c_first);
+      if (!(ok = mbar_wait(smem_u32(&tfull[acc]), acc_phase, abort_flag, p.flags))) {
+        if (f32_in || bf16_in) mbar_wait(lbar, lphase, abort_flag, p.flags);  // no load left in flight
+        break;
+      }
+      tc_fence_after();
+      const uint32_t tbase = tmem_base + ((uint32_t)(quad * 32) << 16) + acc * BN;
+#pragma unroll 1
+      for (int c = c_first; c < c_first + CPW; c++) {
+        const int col0 = nb * BN + c * 32;
+        const uint32_t bufA = stg, bufB = stg + 2048;
         if (f32_in || bf16_in) {
-          if (lane == 0) {
-            mbar_expect_tx(lbar, f32_in ? 4096 : 2048);
-            tma_load_2d(f32_in ? bufA : bufB, &tm_in, lbar, col0, row0);
-          }
+          if (c > c_first) fetch_input(c);
           if (!mbar_wait(lbar, lphase, abort_flag, p.flags)) {
-            tmem_ld_wait();  // no TMEM load left in flight
             ok = false;
             break;
           }
           lphase ^= 1;
-        }
-        tmem_ld_wait();
-        float v[32];
-#pragma unroll
-        for (int i = 0; i < 32; i++) v[i] = __uint_as_float(raw[i]);
-        if (p.splits > 1) {
-          stage_f32(bufA, lane, v);
         } else {
-          switch (kind) {
-            case EPI_STORE:
-            case EPI_BIAS:
-              add_bias(p, col0, v);
-              stage_bf16(bufA, lane, v);
-              break;
-            case EPI_BIAS_ACT:
-              add_bias(p, col0, v);
-              stage_bf16(bufA, lane, v);
+          if (lane == 0) bulk_wait_read0();  // the previous chunk's stores have read the staging set
+          __syncwarp();
+        }
 #pragma unroll
-              for (int i = 0; i < 32; i++) v[i] = act_fwd(p.act, v[i]);
-              stage_bf16(bufB, lane, v);
-              break;
-            case EPI_ACT_BWD: {
-              float hv[32];
-              unstage_bf16(bufB, lane, hv);
+        for (int hh = 0; hh < 2; hh++) {
+          float4 bias[4];
+          if (has_bias) load_bias(p, col0 + 16 * hh, bias);
+          uint32_t raw[16];
+          tmem_ld_32x32b_x16(tbase + c * 32 + 16 * hh, raw);
+          tmem_ld_wait();
+          float v[16];
 #pragma unroll
-              for (int i = 0; i < 32; i++) v[i] *= act_grad(p.act, hv[i]);
-              stage_bf16(bufA, lane, v);
-              break;
-            }
-            case EPI_RESADD: {
-              float x[32];
-              unstage_f32(bufA, lane, x);
-              add_bias(p, col0, v);
-              if (p.drop.active) {
-                const uint64_t el = (uint64_t)row * p.N + col0;
+          for (int i = 0; i < 16; i++) v[i] = __uint_as_float(raw[i]);
+          if (p.splits > 1) {
+            stage_f32(bufA, lane, hh, v);
+          } else {
+            switch (kind) {
+              case EPI_STORE:
+              case EPI_BIAS:
+                if (has_bias) add_bias(bias, v);
+                stage_bf16(bufA, lane, hh, v);
+                break;
+              case EPI_BIAS_ACT:
+                if (has_bias) add_bias(bias, v);
+                stage_bf16(bufA, lane, hh, v);
 #pragma unroll
-                for (int i = 0; i < 32; i++) v[i] *= drop_mul(p.drop, el + i);
+                for (int i = 0; i < 16; i++) v[i] = act_fwd(p.act, v[i]);
+                stage_bf16(bufB, lane, hh, v);
+                break;
+              case EPI_ACT_BWD: {
+                float hv[16];
+                unstage_bf16(bufB, lane, hh, hv);
+#pragma unroll
+                for (int i = 0; i < 16; i++) v[i] *= act_grad(p.act, hv[i]);
+                stage_bf16(bufA, lane, hh, v);
+                break;
               }
+              case EPI_RESADD: {
+                float x[16];
+                unstage_f32(bufA, lane, hh, x);
+                if (has_bias) add_bias(bias, v);
+                if (p.drop.active) {
+                  const uint64_t el = (uint64_t)row * p.N + col0 + 16 * hh;
 #pragma unroll
-              for (int i = 0; i < 32; i++) v[i] += x[i];
-              stage_f32(bufA, lane, v);
-              break;
+                  for (int i = 0; i < 16; i++) v[i] *= drop_mul(p.drop, el + i);
+                }
+#pragma unroll
+                for (int i = 0; i < 16; i++) v[i] += x[i];
+                stage_f32(bufA, lane, hh, v);
+                break;
+              }
+              default:  // EPI_ACC_F32, EPI_STORE_F32
+                stage_f32(bufA, lane, hh, v);
+                break;
             }
-            default:  // EPI_ACC_F32, EPI_STORE_F32
-              stage_f32(bufA, lane, v);
-              break;
           }
         }
         fence_proxy_async_smem();

@@ -28,10 +28,10 @@ def bf(x):
     return torch.from_numpy(np.asarray(x, np.float32)).bfloat16()
 
 
-def run_case(backend, B, T, H, p, seed=0):
+def run_case(backend, B, T, H, p, seed=0, qkv_np=None):
     hd = 64
     rng = np.random.default_rng(seed)
-    qkv = bf(rng.standard_normal((B, T, 3, H, hd)))
+    qkv = bf(rng.standard_normal((B, T, 3, H, hd)) if qkv_np is None else qkv_np)
     dout = bf(rng.standard_normal((B, T, H, hd)))
     q, k, v = (qkv.float().numpy().astype(np.float64)[:, :, i].transpose(0, 2, 1, 3) for i in range(3))
     do = dout.float().numpy().astype(np.float64).transpose(0, 2, 1, 3)
@@ -86,3 +86,18 @@ def test_tensor_core_matches_cuda_core():
     o1, g1 = run_case(1, 2, 256, 2, 0.0, seed=4)
     o2, g2 = run_case(0, 2, 256, 2, 0.0, seed=4)
     assert rel_l2(o1, o2) < 1e-2 and rel_l2(g1, g2) < 2e-2
+
+
+def test_attention_rescale_path():
+    # Scores that grow by about 10 log2 units per 64-key block: the forward's
+    # running maximum is exceeded by more than its rescale threshold in every
+    # block, so O and l are rescaled in TMEM each time (the path random inputs
+    # of unit scale almost never take).
+    B, T, H, hd = 1, 512, 2, 64
+    rng = np.random.default_rng(3)
+    x = rng.standard_normal((B, T, 3, H, hd))
+    u = rng.standard_normal(hd)
+    u /= np.linalg.norm(u)
+    x[:, :, 0] += 21.0 * u
+    x[:, :, 1] += (np.arange(T) / T * 21.0)[None, :, None, None] * u
+    run_case(1, B, T, H, 0.0, qkv_np=x)
