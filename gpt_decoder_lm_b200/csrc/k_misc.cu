@@ -136,62 +136,75 @@ template <typename T, int VPL>
 __global__ void k_norm_fwd(const float* __restrict__ x, const float* __restrict__ w, const float* __restrict__ b,
                            T* __restrict__ y, float* __restrict__ mean_out, float* __restrict__ rstd_out, long rows,
                            int d, int rms, float eps) {
-  long row = (long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  int lane = threadIdx.x & 31;
-  if (row >= rows) return;
-  int d4 = d >> 2;
-  const float4* xr = reinterpret_cast<const float4*>(x + row * d);
-  float4 v[VPL];
-  float s = 0.f;
+  // two rows per warp, both loaded up front: the whole launch is resident in
+  // one wave and every warp has 2 x d x 4 bytes in flight
+  const long row0 = ((long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5)) * 2;
+  const int lane = threadIdx.x & 31;
+  if (row0 >= rows) return;
+  const int d4 = d >> 2;
+  float4 v[2][VPL];
 #pragma unroll
-  for (int k = 0; k < VPL; k++) {
-    int c = lane + 32 * k;
-    v[k] = c < d4 ? xr[c] : make_float4(0.f, 0.f, 0.f, 0.f);
-    s += rms ? (v[k].x * v[k].x + v[k].y * v[k].y + v[k].z * v[k].z + v[k].w * v[k].w)
-             : (v[k].x + v[k].y + v[k].z + v[k].w);
+  for (int u = 0; u < 2; u++) {
+    const float4* xr = reinterpret_cast<const float4*>(x + (row0 + u) * d);
+    const bool live = row0 + u < rows;
+#pragma unroll
+    for (int k = 0; k < VPL; k++) {
+      int c = lane + 32 * k;
+      v[u][k] = (live && c < d4) ? xr[c] : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
   }
-  s = warp_sum(s);
-  float mean = 0.f, rstd;
-  if (rms) {
-    rstd = 1.0f / sqrtf(s / d + eps);
-  } else {
-    mean = s / d;
-    float q = 0.f;
+#pragma unroll
+  for (int u = 0; u < 2; u++) {
+    const long row = row0 + u;
+    if (row >= rows) break;
+    float s = 0.f;
+#pragma unroll
+    for (int k = 0; k < VPL; k++)
+      s += rms ? (v[u][k].x * v[u][k].x + v[u][k].y * v[u][k].y + v[u][k].z * v[u][k].z + v[u][k].w * v[u][k].w)
+               : (v[u][k].x + v[u][k].y + v[u][k].z + v[u][k].w);
+    s = warp_sum(s);
+    float mean = 0.f, rstd;
+    if (rms) {
+      rstd = 1.0f / sqrtf(s / d + eps);
+    } else {
+      mean = s / d;
+      float q = 0.f;
+#pragma unroll
+      for (int k = 0; k < VPL; k++) {
+        int c = lane + 32 * k;
+        if (c < d4) {
+          float a = v[u][k].x - mean, bb = v[u][k].y - mean, cc = v[u][k].z - mean, dd = v[u][k].w - mean;
+          q += a * a + bb * bb + cc * cc + dd * dd;
+        }
+      }
+      q = warp_sum(q);
+      rstd = 1.0f / sqrtf(q / d + eps);
+    }
+    T* yr = y + row * d;
 #pragma unroll
     for (int k = 0; k < VPL; k++) {
       int c = lane + 32 * k;
       if (c < d4) {
-        float a = v[k].x - mean, bb = v[k].y - mean, cc = v[k].z - mean, dd = v[k].w - mean;
-        q += a * a + bb * bb + cc * cc + dd * dd;
+        float4 o;
+        o.x = (v[u][k].x - mean) * rstd;
+        o.y = (v[u][k].y - mean) * rstd;
+        o.z = (v[u][k].z - mean) * rstd;
+        o.w = (v[u][k].w - mean) * rstd;
+        if (!rms) {
+          float4 ww = reinterpret_cast<const float4*>(w)[c];
+          float4 bb = reinterpret_cast<const float4*>(b)[c];
+          o.x = o.x * ww.x + bb.x;
+          o.y = o.y * ww.y + bb.y;
+          o.z = o.z * ww.z + bb.z;
+          o.w = o.w * ww.w + bb.w;
+        }
+        store4<T>(yr + 4 * c, o);
       }
     }
-    q = warp_sum(q);
-    rstd = 1.0f / sqrtf(q / d + eps);
-  }
-  T* yr = y + row * d;
-#pragma unroll
-  for (int k = 0; k < VPL; k++) {
-    int c = lane + 32 * k;
-    if (c < d4) {
-      float4 o;
-      o.x = (v[k].x - mean) * rstd;
-      o.y = (v[k].y - mean) * rstd;
-      o.z = (v[k].z - mean) * rstd;
-      o.w = (v[k].w - mean) * rstd;
-      if (!rms) {
-        float4 ww = reinterpret_cast<const float4*>(w)[c];
-        float4 bb = reinterpret_cast<const float4*>(b)[c];
-        o.x = o.x * ww.x + bb.x;
-        o.y = o.y * ww.y + bb.y;
-        o.z = o.z * ww.z + bb.z;
-        o.w = o.w * ww.w + bb.w;
-      }
-      store4<T>(yr + 4 * c, o);
+    if (lane == 0) {
+      mean_out[row] = mean;
+      rstd_out[row] = rstd;
     }
-  }
-  if (lane == 0) {
-    mean_out[row] = mean;
-    rstd_out[row] = rstd;
   }
 }
 
@@ -200,12 +213,13 @@ void norm_fwd(Ctx& c, const float* x, const float* w, const float* b, T* y, floa
               int d, bool rms, float eps) {
   int d4 = d / 4;
   int vpl = (d4 + 31) / 32;
-  unsigned grid = (unsigned)((rows + 7) / 8);
+  unsigned grid = (unsigned)((rows + 15) / 16);  // 8 warps x 2 rows per block
   LaunchScope s(c, "norm_fwd");
 #define NF(V) k_norm_fwd<T, V><<<grid, 256, 0, c.stream>>>(x, w, b, y, mean, rstd, rows, d, rms, eps)
   if (vpl <= 1) NF(1);
   else if (vpl <= 2) NF(2);
   else if (vpl <= 4) NF(4);
+  else if (vpl <= 6) NF(6);
   else if (vpl <= 8) NF(8);
   else NF(16);
 #undef NF
@@ -239,6 +253,7 @@ __global__ void k_norm_bwd(NormBwd p) {
   // two rows per round: one barrier for both rows' reductions
   for (long r = r0; r < r1; r += 2) {
     float dyv[2][4], xh[2][4], g[2][4], rstd[2], s[4] = {0.f, 0.f, 0.f, 0.f};
+    float4 old[2];  // the residual gradient these rows add to, fetched with dy and x
 #pragma unroll
     for (int u = 0; u < 2; u++) {
       const long rr = r + u;
@@ -246,9 +261,11 @@ __global__ void k_norm_bwd(NormBwd p) {
       const float mean = (p.rms || !live) ? 0.f : p.mean[rr];
       rstd[u] = live ? p.rstd[rr] : 0.f;
       float4 dy = make_float4(0, 0, 0, 0), xv = make_float4(0, 0, 0, 0);
+      old[u] = make_float4(0, 0, 0, 0);
       if (own && live) {
         dy = reinterpret_cast<const float4*>(p.dy + rr * p.d)[tid];
         xv = reinterpret_cast<const float4*>(p.x + rr * p.d)[tid];
+        if (p.accumulate) old[u] = reinterpret_cast<const float4*>(p.dres + rr * p.d)[tid];
       }
       const float dya[4] = {dy.x, dy.y, dy.z, dy.w}, xa[4] = {xv.x, xv.y, xv.z, xv.w};
 #pragma unroll
@@ -280,8 +297,7 @@ __global__ void k_norm_bwd(NormBwd p) {
       const float mg = p.rms ? 0.f : t[2 * u] / p.d;
       const float mgx = t[2 * u + 1] / p.d;
       float4* dr = reinterpret_cast<float4*>(p.dres + rr * p.d) + tid;
-      float4 old = p.accumulate ? *dr : make_float4(0, 0, 0, 0);
-      float ov[4] = {old.x, old.y, old.z, old.w};
+      const float ov[4] = {old[u].x, old[u].y, old[u].z, old[u].w};
       float nv[4];
 #pragma unroll
       for (int k = 0; k < 4; k++) {
@@ -325,34 +341,43 @@ void norm_bwd(Ctx& c, const NormBwd& p) {
 template void norm_bwd<float>(Ctx&, const NormBwd&);
 template void norm_bwd<bf16>(Ctx&, const NormBwd&);
 
-// grad_s[j] += sum_b part[b, s, j] for the three slots of the norm-backward
-// partials at once.  Block (32 columns x 8 row groups): row group y sums
-// blocks y, y+8, ...; the 8 group sums are then added in a fixed order.
-__global__ void k_partial_reduce3(const float* __restrict__ part, int blocks, int d, float* g0, float* g1, float* g2) {
-  __shared__ float sh[8][33];
-  int x = threadIdx.x, y = threadIdx.y;
-  int j = blockIdx.x * 32 + x;
-  int slot = blockIdx.y;
-  float* dst = slot == 0 ? g0 : (slot == 1 ? g1 : g2);
+// dst_y[j] += sum_{k < rows} src[y * slot_off + k * stride + j] for j < n and
+// each destination y = blockIdx.y (null: skipped), in a fixed order: block =
+// 32 columns x 32 row groups; row group g sums rows g, g + 32, ... in
+// increasing order, then the 32 group sums are added in group order.
+struct Dst3 {
+  float* p[3];
+};
+__global__ void __launch_bounds__(1024) k_rows_reduce(const float* __restrict__ src, long stride, long slot_off,
+                                                      int rows, int n, Dst3 dsts) {
+  __shared__ float sh[32][33];
+  float* dst = dsts.p[blockIdx.y];
   if (!dst) return;  // uniform per block
+  src += (long)blockIdx.y * slot_off;
+  const int x = threadIdx.x, y = threadIdx.y;
+  const int j = blockIdx.x * 32 + x;
   float s = 0.f;
-  if (j < d)
-    for (int b = y; b < blocks; b += 8) s += part[((long)b * 3 + slot) * d + j];
+  if (j < n) {
+#pragma unroll 4
+    for (int k = y; k < rows; k += 32) s += src[(long)k * stride + j];
+  }
   sh[y][x] = s;
   __syncthreads();
-  if (y == 0 && j < d) {
+  if (y == 0 && j < n) {
     float t = 0.f;
 #pragma unroll
-    for (int k = 0; k < 8; k++) t += sh[k][x];
+    for (int k = 0; k < 32; k++) t += sh[k][x];
     dst[j] += t;
   }
 }
 
+// grad_s[j] += sum_b part[b, s, j] for the three slots of the norm-backward
+// partials (each nullable), one launch
 void partial_reduce3(Ctx& c, const float* part, int blocks, int d, float* g0, float* g1, float* g2) {
   if (!g0 && !g1 && !g2) return;
   LaunchScope s(c, "partial_reduce");
-  dim3 grid((d + 31) / 32, 3);
-  k_partial_reduce3<<<grid, dim3(32, 8), 0, c.stream>>>(part, blocks, d, g0, g1, g2);
+  Dst3 g{{g0, g1, g2}};
+  k_rows_reduce<<<dim3((d + 31) / 32, 3), dim3(32, 32), 0, c.stream>>>(part, 3L * d, d, blocks, d, g);
 }
 
 // ============================================================================
@@ -371,26 +396,10 @@ __global__ void k_colsum(const T* __restrict__ x, long rows, int N, int chunks, 
 
 // grad[j] += sum_c part[c, j]: row group y of 8 sums chunks y, y+8, ...; the
 // group sums are added in a fixed order
-__global__ void k_colsum_reduce(const float* __restrict__ part, int chunks, int N, float* __restrict__ grad) {
-  __shared__ float sh[8][33];
-  const int x = threadIdx.x, y = threadIdx.y;
-  const int j = blockIdx.x * 32 + x;
-  float s = 0.f;
-  if (j < N)
-    for (int k = y; k < chunks; k += 8) s += part[(long)k * N + j];
-  sh[y][x] = s;
-  __syncthreads();
-  if (y == 0 && j < N) {
-    float t = 0.f;
-#pragma unroll
-    for (int k = 0; k < 8; k++) t += sh[k][x];
-    grad[j] += t;
-  }
-}
-
 void colsum_reduce(Ctx& c, const float* part, int chunks, int N, float* grad) {
   LaunchScope s(c, "colsum");
-  k_colsum_reduce<<<(N + 31) / 32, dim3(32, 8), 0, c.stream>>>(part, chunks, N, grad);
+  Dst3 g{{grad, nullptr, nullptr}};
+  k_rows_reduce<<<dim3((N + 31) / 32, 1), dim3(32, 32), 0, c.stream>>>(part, N, 0, chunks, N, g);
 }
 
 // bf16 rows with N % 8 == 0: each thread sums 8 adjacent columns over its
@@ -401,8 +410,7 @@ __global__ void k_colsum_bf16x8(const bf16* __restrict__ x, long rows, int N, in
   const long per = (rows + chunks - 1) / chunks;
   const long r0 = blockIdx.y * per, r1 = min(rows, r0 + per);
   float s[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-  for (long r = r0; r < r1; r++) {
-    uint4 u = reinterpret_cast<const uint4*>(x + r * N)[j8];
+  auto add = [&](const uint4& u) {
     const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
 #pragma unroll
     for (int k = 0; k < 4; k++) {
@@ -410,7 +418,19 @@ __global__ void k_colsum_bf16x8(const bf16* __restrict__ x, long rows, int N, in
       s[2 * k] += f.x;
       s[2 * k + 1] += f.y;
     }
+  };
+  long r = r0;
+  for (; r + 4 <= r1; r += 4) {  // four rows of loads in flight, added in row order
+    const uint4 u0 = reinterpret_cast<const uint4*>(x + r * N)[j8];
+    const uint4 u1 = reinterpret_cast<const uint4*>(x + (r + 1) * N)[j8];
+    const uint4 u2 = reinterpret_cast<const uint4*>(x + (r + 2) * N)[j8];
+    const uint4 u3 = reinterpret_cast<const uint4*>(x + (r + 3) * N)[j8];
+    add(u0);
+    add(u1);
+    add(u2);
+    add(u3);
   }
+  for (; r < r1; r++) add(reinterpret_cast<const uint4*>(x + r * N)[j8]);
   float4* dst = reinterpret_cast<float4*>(part + (long)blockIdx.y * N + j8 * 8);
   dst[0] = make_float4(s[0], s[1], s[2], s[3]);
   dst[1] = make_float4(s[4], s[5], s[6], s[7]);

@@ -158,7 +158,7 @@ void embed_sort(Ctx& c, const int32_t* idx, long M, int32_t* sorted_tok, int32_t
 // seg_scratch: 2 * ceil(M / 32) * d floats (partial sums of segments that cross 32-slot chunks)
 void embed_bwd(Ctx& c, const float* dres, const int32_t* sorted_tok, const int32_t* sorted_pos, long M, int Tn,
                int Bn, int d, DropKey drop, float* dwte, float* dwpe, float* seg_scratch);
-// column partials of colsum_acc [chunks, N] -> grad (+=), 8 row groups per column
+// column partials of colsum_acc [chunks, N] -> grad (+=), fixed order
 void colsum_reduce(Ctx& c, const float* part, int chunks, int N, float* grad);
 
 // grad norm partials, clip + AdamW
