@@ -350,7 +350,14 @@ constexpr int BWD_STAGES = 3;  // Q/dO (or K/V) tiles in flight
 //   S^T = K Q^T, dP^T = V dO^T  ->  P~^T, dS^T (bf16, written into TMEM)
 //   dV += P~^T dO,  dK += dS^T Q
 // Eight math warps, two per TMEM lane quadrant, each take 32 of the 64 query
-// columns of a block (the backward has no row reductions).
+// columns of a block (the backward has no row reductions).  The math runs in
+// two phases per block (P~^T from S^T, then dS^T from dP^T) with an mbarrier
+// each way, and the MMA warp issues in the order
+//   S(i) dP(i) | P~(i) ready: dV(i) S(i+1) | dS(i) ready: dK(i) dP(i+1) | ...
+// so S^T of the next block is computed while the math warps work on dS^T, and
+// dP^T of the next block while they work on P~^T.  (P~^T lives in the S^T
+// columns and dS^T in the dP^T columns; tcgen05 MMAs of one thread execute in
+// issue order, so each is read before it is overwritten.)
 // smem: K | V | (Q, dO)[3 stages] | (lse, D)[3] | barriers (~82 KB)
 // TMEM: S^T [0,64), dP^T [64,128), dV [128,192), dK [192,256)
 // ============================================================================
@@ -370,8 +377,9 @@ __global__ void __launch_bounds__(320, 2) k_attn_bwd_kv8(const __grid_constant__
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + K_BAR);
   const uint32_t kv_full = smem_u32(bars + 0), st_full0 = smem_u32(bars + 1),
                  st_empty0 = smem_u32(bars + 1 + BWD_STAGES);
-  const uint32_t sdp_full = smem_u32(bars + 1 + 2 * BWD_STAGES), pds_full = sdp_full + 8, acc_full = sdp_full + 16;
-  uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + 4 + 2 * BWD_STAGES);
+  const uint32_t s_full = smem_u32(bars + 1 + 2 * BWD_STAGES), dp_full = s_full + 8, p_ready = s_full + 16,
+                 ds_ready = s_full + 24, acc_full = s_full + 32;
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + 6 + 2 * BWD_STAGES);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tslot + 1);
   const float* sld = reinterpret_cast<const float*>(smem + K_LD);  // [stage][lse 64 | D 64]
   const uint32_t sb = smem_u32(smem);
@@ -389,8 +397,10 @@ __global__ void __launch_bounds__(320, 2) k_attn_bwd_kv8(const __grid_constant__
       mbar_init(st_full0 + 8 * s, 1);
       mbar_init(st_empty0 + 8 * s, 1);
     }
-    mbar_init(sdp_full, 1);
-    mbar_init(pds_full, 8);
+    mbar_init(s_full, 1);
+    mbar_init(dp_full, 1);
+    mbar_init(p_ready, 8);
+    mbar_init(ds_ready, 8);
     mbar_init(acc_full, 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -427,28 +437,39 @@ __global__ void __launch_bounds__(320, 2) k_attn_bwd_kv8(const __grid_constant__
     if (lane == 0) {
       constexpr uint32_t id_s = idesc_bf16_f32(128, 64, false, false);
       constexpr uint32_t id_acc = idesc_bf16_f32(128, 64, false, true);
-      bool ok = mbar_wait(kv_full, 0, abort_flag, a.flags);
-      for (int it = 0; it < nit && ok; it++) {
-        const int s = it % BWD_STAGES;
-        if (!(ok = mbar_wait(st_full0 + 8 * s, (it / BWD_STAGES) & 1, abort_flag, a.flags))) break;
+      auto q_of = [&](int it) { return sb + K_ST + (it % BWD_STAGES) * TILE; };
+      auto issue_s = [&](int it) -> bool {  // S^T = K Q^T of block it
+        if (!mbar_wait(st_full0 + 8 * (it % BWD_STAGES), (it / BWD_STAGES) & 1, abort_flag, a.flags)) return false;
         tc_fence_after();
-        const uint32_t q = sb + K_ST + s * TILE, dO = q + HTILE;
 #pragma unroll
         for (int kk = 0; kk < 4; kk++)
-          mma_bf16_ss(tmem, desc_k(sb + K_K, TILE, kk), desc_k(q, HTILE, kk), id_s, kk > 0);
+          mma_bf16_ss(tmem, desc_k(sb + K_K, TILE, kk), desc_k(q_of(it), HTILE, kk), id_s, kk > 0);
+        mma_commit(s_full);
+        return true;
+      };
+      auto issue_dp = [&](int it) {  // dP^T = V dO^T of block it (its stage is loaded)
 #pragma unroll
         for (int kk = 0; kk < 4; kk++)
-          mma_bf16_ss(tmem + 64, desc_k(sb + K_V, TILE, kk), desc_k(dO, HTILE, kk), id_s, kk > 0);
-        mma_commit(sdp_full);
-        if (!(ok = mbar_wait(pds_full, it & 1, abort_flag, a.flags))) break;
+          mma_bf16_ss(tmem + 64, desc_k(sb + K_V, TILE, kk), desc_k(q_of(it) + HTILE, HTILE, kk), id_s, kk > 0);
+        mma_commit(dp_full);
+      };
+      bool ok = mbar_wait(kv_full, 0, abort_flag, a.flags) && issue_s(0);
+      if (ok) issue_dp(0);
+      for (int it = 0; it < nit && ok; it++) {
+        const uint32_t q = q_of(it), dO = q + HTILE;
+        if (!(ok = mbar_wait(p_ready, it & 1, abort_flag, a.flags))) break;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 4; kk++)
           mma_bf16_ts(tmem + 128, tmem + acol(kk), desc_mn64(dO, kk), id_acc, (it > 0 || kk > 0));
+        if (it + 1 < nit && !(ok = issue_s(it + 1))) break;
+        if (!(ok = mbar_wait(ds_ready, it & 1, abort_flag, a.flags))) break;
+        tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 4; kk++)
           mma_bf16_ts(tmem + 192, tmem + 64 + acol(kk), desc_mn64(q, kk), id_acc, (it > 0 || kk > 0));
-        mma_commit(st_empty0 + 8 * s);
+        mma_commit(st_empty0 + 8 * (it % BWD_STAGES));
+        if (it + 1 < nit) issue_dp(it + 1);
       }
       mma_commit(acc_full);
     }
@@ -464,72 +485,75 @@ __global__ void __launch_bounds__(320, 2) k_attn_bwd_kv8(const __grid_constant__
       const int i = i0 + it;
       const int q0 = i * 64;
       const float* ld = sld + (it % BWD_STAGES) * 128;  // lse[64] | D[64] of this query block
+      // lse / D of the stage (TMA-written: observed through the stage's own
+      // barrier), then S^T of the block
       if (!(ok = mbar_wait(st_full0 + 8 * (it % BWD_STAGES), (it / BWD_STAGES) & 1, abort_flag, a.flags))) break;
-      if (!(ok = mbar_wait(sdp_full, it & 1, abort_flag, a.flags))) break;
+      if (!(ok = mbar_wait(s_full, it & 1, abort_flag, a.flags))) break;
       tc_fence_after();
-      const int lim = kj - q0;                        // query column c is masked iff c < lim
-      const bool masked = q0 < kb * 128 + 128;        // only blocks that reach this CTA's keys
+      const int lim = kj - q0;                  // query column c is masked iff c < lim
+      const bool masked = q0 < kb * 128 + 128;  // only blocks that reach this CTA's keys
+      float pk[2][16];                          // P^T of this thread's 32 columns
+      // phase 1: P^T = 2^(S^T sl2 - lse log2 e) (masked), P~^T = drop(P^T)
 #pragma unroll
       for (int sub = 0; sub < 2; sub++) {
         const int c0 = half * 32 + sub * 16;
-        uint32_t sv[16], dv[16];
+        uint32_t sv[16];
         tmem_ld_32x32b_x16(trow + c0, sv);
-        tmem_ld_32x32b_x16(trow + 64 + c0, dv);
         tmem_ld_wait();
-        uint32_t pp[8], pd[8];
+        uint32_t pp[8];
 #pragma unroll
         for (int e = 0; e < 16; e += 4) {
           const float4 l4 = *reinterpret_cast<const float4*>(ld + c0 + e);
-          const float4 d4 = *reinterpret_cast<const float4*>(ld + 64 + c0 + e);
-          if (!DROP) {
-            // P = 2^(S sl2 - lse log2 e);  dS = P (dP - D)
-            const uint64_t x01 = f2fma(f2(__uint_as_float(sv[e]), __uint_as_float(sv[e + 1])), sl2x2,
-                                       f2mul(f2(l4.x, l4.y), nlog2e));
-            const uint64_t x23 = f2fma(f2(__uint_as_float(sv[e + 2]), __uint_as_float(sv[e + 3])), sl2x2,
-                                       f2mul(f2(l4.z, l4.w), nlog2e));
-            const float2 y01 = f2split(x01), y23 = f2split(x23);
-            float p0 = ex2(y01.x), p1 = ex2(y01.y), p2 = ex2(y23.x), p3 = ex2(y23.y);
-            if (masked) {
-              const int col = c0 + e;
-              if (col < lim) p0 = 0.f;
-              if (col + 1 < lim) p1 = 0.f;
-              if (col + 2 < lim) p2 = 0.f;
-              if (col + 3 < lim) p3 = 0.f;
-            }
-            const uint64_t P01 = f2(p0, p1), P23 = f2(p2, p3);
-            const uint64_t ds01 = f2mul(P01, f2sub(f2(__uint_as_float(dv[e]), __uint_as_float(dv[e + 1])),
-                                                   f2(d4.x, d4.y)));
-            const uint64_t ds23 = f2mul(P23, f2sub(f2(__uint_as_float(dv[e + 2]), __uint_as_float(dv[e + 3])),
-                                                   f2(d4.z, d4.w)));
-            pp[e >> 1] = pack2(p0, p1);
-            pp[(e >> 1) + 1] = pack2(p2, p3);
-            pd[e >> 1] = pack2v(ds01);
-            pd[(e >> 1) + 1] = pack2v(ds23);
-          } else {
-            const float lv[4] = {l4.x, l4.y, l4.z, l4.w}, dd[4] = {d4.x, d4.y, d4.z, d4.w};
-            float pv[4], dsv[4];
+          const float2 y01 = f2split(f2fma(f2(__uint_as_float(sv[e]), __uint_as_float(sv[e + 1])), sl2x2,
+                                           f2mul(f2(l4.x, l4.y), nlog2e)));
+          const float2 y23 = f2split(f2fma(f2(__uint_as_float(sv[e + 2]), __uint_as_float(sv[e + 3])), sl2x2,
+                                           f2mul(f2(l4.z, l4.w), nlog2e)));
+          float p4[4] = {ex2(y01.x), ex2(y01.y), ex2(y23.x), ex2(y23.y)};
 #pragma unroll
-            for (int u = 0; u < 4; u++) {
-              const int col = c0 + e + u;
-              float p = ex2(fmaf(__uint_as_float(sv[e + u]), a.scale_log2, lv[u] * -LOG2E));
-              if (masked && col < lim) p = 0.f;
-              const float mk = drop_mul(a.drop, ((uint64_t)bh * a.T + q0 + col) * a.T + kj);
-              pv[u] = p * mk;
-              dsv[u] = p * (__uint_as_float(dv[e + u]) * mk - dd[u]);
-            }
-            pp[e >> 1] = pack2(pv[0], pv[1]);
-            pp[(e >> 1) + 1] = pack2(pv[2], pv[3]);
-            pd[e >> 1] = pack2(dsv[0], dsv[1]);
-            pd[(e >> 1) + 1] = pack2(dsv[2], dsv[3]);
+          for (int u = 0; u < 4; u++) {
+            if (masked && c0 + e + u < lim) p4[u] = 0.f;
+            pk[sub][e + u] = p4[u];
           }
+          if (DROP) {
+#pragma unroll
+            for (int u = 0; u < 4; u++)
+              p4[u] *= drop_mul(a.drop, ((uint64_t)bh * a.T + q0 + c0 + e + u) * a.T + kj);
+          }
+          pp[e >> 1] = pack2(p4[0], p4[1]);
+          pp[(e >> 1) + 1] = pack2(p4[2], p4[3]);
         }
         tmem_st_32x32b_x8(trow + pcol(c0), pp);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(p_ready);
+      // phase 2: dS^T = P^T (drop(dP^T) - D)
+      if (!(ok = mbar_wait(dp_full, it & 1, abort_flag, a.flags))) break;
+      tc_fence_after();
+#pragma unroll
+      for (int sub = 0; sub < 2; sub++) {
+        const int c0 = half * 32 + sub * 16;
+        uint32_t dv[16];
+        tmem_ld_32x32b_x16(trow + 64 + c0, dv);
+        tmem_ld_wait();
+        uint32_t pd[8];
+#pragma unroll
+        for (int e = 0; e < 16; e += 2) {
+          const float2 d2 = *reinterpret_cast<const float2*>(ld + 64 + c0 + e);
+          float dp0 = __uint_as_float(dv[e]), dp1 = __uint_as_float(dv[e + 1]);
+          if (DROP) {
+            dp0 *= drop_mul(a.drop, ((uint64_t)bh * a.T + q0 + c0 + e) * a.T + kj);
+            dp1 *= drop_mul(a.drop, ((uint64_t)bh * a.T + q0 + c0 + e + 1) * a.T + kj);
+          }
+          pd[e >> 1] = pack2v(f2mul(f2(pk[sub][e], pk[sub][e + 1]), f2sub(f2(dp0, dp1), f2(d2.x, d2.y))));
+        }
         tmem_st_32x32b_x8(trow + 64 + pcol(c0), pd);
       }
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(pds_full);
+      if (lane == 0) mbar_arrive(ds_ready);
     }
     if (ok && mbar_wait(acc_full, 0, abort_flag, a.flags)) {
       tc_fence_after();
@@ -558,8 +582,11 @@ __global__ void __launch_bounds__(320, 2) k_attn_bwd_kv8(const __grid_constant__
 
 // ============================================================================
 // backward, dQ: one CTA per (128-query block, b, h), walking 64-key blocks
-// up to the diagonal.  S = Q K^T, dP = dO V^T -> dS (bf16, written into TMEM);
-// dQ += dS K.  Eight math warps as in the dK/dV kernel.
+// up to the diagonal.  S = Q K^T, dP = dO V^T -> dS (bf16, written into the
+// dP columns of TMEM); dQ += dS K.  Eight math warps as in the dK/dV kernel,
+// in two phases per block (P from S, then dS from dP); the MMA warp issues
+//   S(j) dP(j) | S read: S(j+1) | dS(j) ready: dQ(j) dP(j+1) | ...
+// so S of the next block is computed while the math warps work on dS.
 // smem: Q | dO | (K, V)[3 stages] | barriers   (~80 KB)
 // TMEM: S [0,64), dP [64,128), dQ [128,192)  (256 allocated)
 // ============================================================================
@@ -579,8 +606,9 @@ __global__ void __launch_bounds__(320, 2) k_attn_bwd_q8(const __grid_constant__ 
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Q_BAR);
   const uint32_t qd_full = smem_u32(bars + 0), kv_full0 = smem_u32(bars + 1),
                  kv_empty0 = smem_u32(bars + 1 + BWD_STAGES);
-  const uint32_t sdp_full = smem_u32(bars + 1 + 2 * BWD_STAGES), ds_full = sdp_full + 8, acc_full = sdp_full + 16;
-  uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + 4 + 2 * BWD_STAGES);
+  const uint32_t s_full = smem_u32(bars + 1 + 2 * BWD_STAGES), dp_full = s_full + 8, s_read = s_full + 16,
+                 ds_ready = s_full + 24, acc_full = s_full + 32;
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + 6 + 2 * BWD_STAGES);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tslot + 1);
   const uint32_t sb = smem_u32(smem);
 
@@ -596,8 +624,10 @@ __global__ void __launch_bounds__(320, 2) k_attn_bwd_q8(const __grid_constant__ 
       mbar_init(kv_full0 + 8 * s, 1);
       mbar_init(kv_empty0 + 8 * s, 1);
     }
-    mbar_init(sdp_full, 1);
-    mbar_init(ds_full, 8);
+    mbar_init(s_full, 1);
+    mbar_init(dp_full, 1);
+    mbar_init(s_read, 8);
+    mbar_init(ds_ready, 8);
     mbar_init(acc_full, 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -632,24 +662,34 @@ __global__ void __launch_bounds__(320, 2) k_attn_bwd_q8(const __grid_constant__ 
     if (lane == 0) {
       constexpr uint32_t id_s = idesc_bf16_f32(128, 64, false, false);
       constexpr uint32_t id_acc = idesc_bf16_f32(128, 64, false, true);
-      bool ok = mbar_wait(qd_full, 0, abort_flag, a.flags);
+      auto k_of = [&](int j) { return sb + Q_ST + (j % BWD_STAGES) * TILE; };
+      auto issue_s = [&](int j) -> bool {  // S = Q K^T of block j
+        if (!mbar_wait(kv_full0 + 8 * (j % BWD_STAGES), (j / BWD_STAGES) & 1, abort_flag, a.flags)) return false;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 4; kk++)
+          mma_bf16_ss(tmem, desc_k(sb + Q_Q, TILE, kk), desc_k(k_of(j), HTILE, kk), id_s, kk > 0);
+        mma_commit(s_full);
+        return true;
+      };
+      auto issue_dp = [&](int j) {  // dP = dO V^T of block j (its stage is loaded)
+#pragma unroll
+        for (int kk = 0; kk < 4; kk++)
+          mma_bf16_ss(tmem + 64, desc_k(sb + Q_DO, TILE, kk), desc_k(k_of(j) + HTILE, HTILE, kk), id_s, kk > 0);
+        mma_commit(dp_full);
+      };
+      bool ok = mbar_wait(qd_full, 0, abort_flag, a.flags) && issue_s(0);
+      if (ok) issue_dp(0);
       for (int j = 0; j < nkb && ok; j++) {
-        const int s = j % BWD_STAGES;
-        if (!(ok = mbar_wait(kv_full0 + 8 * s, (j / BWD_STAGES) & 1, abort_flag, a.flags))) break;
-        tc_fence_after();
-        const uint32_t k = sb + Q_ST + s * TILE, v = k + HTILE;
-#pragma unroll
-        for (int kk = 0; kk < 4; kk++) mma_bf16_ss(tmem, desc_k(sb + Q_Q, TILE, kk), desc_k(k, HTILE, kk), id_s, kk > 0);
-#pragma unroll
-        for (int kk = 0; kk < 4; kk++)
-          mma_bf16_ss(tmem + 64, desc_k(sb + Q_DO, TILE, kk), desc_k(v, HTILE, kk), id_s, kk > 0);
-        mma_commit(sdp_full);
-        if (!(ok = mbar_wait(ds_full, j & 1, abort_flag, a.flags))) break;
+        if (!(ok = mbar_wait(s_read, j & 1, abort_flag, a.flags))) break;
+        if (j + 1 < nkb && !(ok = issue_s(j + 1))) break;
+        if (!(ok = mbar_wait(ds_ready, j & 1, abort_flag, a.flags))) break;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 4; kk++)
-          mma_bf16_ts(tmem + 128, tmem + acol(kk), desc_mn64(k, kk), id_acc, (j > 0 || kk > 0));
-        mma_commit(kv_empty0 + 8 * s);
+          mma_bf16_ts(tmem + 128, tmem + 64 + acol(kk), desc_mn64(k_of(j), kk), id_acc, (j > 0 || kk > 0));
+        mma_commit(kv_empty0 + 8 * (j % BWD_STAGES));
+        if (j + 1 < nkb) issue_dp(j + 1);
       }
       mma_commit(acc_full);
     }
@@ -665,41 +705,54 @@ __global__ void __launch_bounds__(320, 2) k_attn_bwd_q8(const __grid_constant__ 
     const uint64_t ebase = ((uint64_t)bh * a.T + qi) * a.T;
     bool ok = true;
     for (int j = 0; j < nkb; j++) {
-      if (!(ok = mbar_wait(sdp_full, j & 1, abort_flag, a.flags))) break;
+      if (!(ok = mbar_wait(s_full, j & 1, abort_flag, a.flags))) break;
       tc_fence_after();
       const int key0 = j * 64;
-      const int lim = qi - key0;                  // key column c is visible iff c <= lim
-      const bool masked = key0 + 64 > qb * 128;   // only the blocks that reach the diagonal
+      const int lim = qi - key0;                 // key column c is visible iff c <= lim
+      const bool masked = key0 + 64 > qb * 128;  // only the blocks that reach the diagonal
+      // phase 1: P = 2^(S sl2 - lse log2 e) (masked) into registers
+      float pk[2][16];
 #pragma unroll
       for (int sub = 0; sub < 2; sub++) {
         const int c0 = half * 32 + sub * 16;
-        uint32_t sv[16], dv[16];
+        uint32_t sv[16];
         tmem_ld_32x32b_x16(trow + c0, sv);
+        tmem_ld_wait();
+#pragma unroll
+        for (int e = 0; e < 16; e += 2) {
+          const float2 y = f2split(f2fma(f2(__uint_as_float(sv[e]), __uint_as_float(sv[e + 1])), sl2x2, nlse2));
+          pk[sub][e] = (masked && c0 + e > lim) ? 0.f : ex2(y.x);
+          pk[sub][e + 1] = (masked && c0 + e + 1 > lim) ? 0.f : ex2(y.y);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(s_read);  // S may be overwritten by the next block
+      // phase 2: dS = P (drop(dP) - D) over the dP columns
+      if (!(ok = mbar_wait(dp_full, j & 1, abort_flag, a.flags))) break;
+      tc_fence_after();
+#pragma unroll
+      for (int sub = 0; sub < 2; sub++) {
+        const int c0 = half * 32 + sub * 16;
+        uint32_t dv[16];
         tmem_ld_32x32b_x16(trow + 64 + c0, dv);
         tmem_ld_wait();
         uint32_t pd[8];
 #pragma unroll
         for (int e = 0; e < 16; e += 2) {
-          const int col = c0 + e;
-          const float2 y = f2split(f2fma(f2(__uint_as_float(sv[e]), __uint_as_float(sv[e + 1])), sl2x2, nlse2));
-          float p0 = ex2(y.x), p1 = ex2(y.y);
-          if (masked) {
-            if (col > lim) p0 = 0.f;
-            if (col + 1 > lim) p1 = 0.f;
-          }
           float dp0 = __uint_as_float(dv[e]), dp1 = __uint_as_float(dv[e + 1]);
           if (DROP) {
-            dp0 *= drop_mul(a.drop, ebase + key0 + col);
-            dp1 *= drop_mul(a.drop, ebase + key0 + col + 1);
+            dp0 *= drop_mul(a.drop, ebase + key0 + c0 + e);
+            dp1 *= drop_mul(a.drop, ebase + key0 + c0 + e + 1);
           }
-          pd[e >> 1] = pack2v(f2mul(f2(p0, p1), f2sub(f2(dp0, dp1), Dx2)));
+          pd[e >> 1] = pack2v(f2mul(f2(pk[sub][e], pk[sub][e + 1]), f2sub(f2(dp0, dp1), Dx2)));
         }
-        tmem_st_32x32b_x8(trow + pcol(c0), pd);
+        tmem_st_32x32b_x8(trow + 64 + pcol(c0), pd);
       }
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(ds_full);
+      if (lane == 0) mbar_arrive(ds_ready);
     }
     if (ok && mbar_wait(acc_full, 0, abort_flag, a.flags)) {
       tc_fence_after();
