@@ -108,8 +108,10 @@ __global__ void __launch_bounds__(192, 2) k_attn_fwd_o(const __grid_constant__ C
   const uint32_t sb = smem_u32(smem);
 
   const int nqb = a.T / 128;
-  const int qb = nqb - 1 - (int)blockIdx.x;  // longest rows first
-  const int bh = blockIdx.y, b = bh / a.H, h = bh % a.H;
+  // blocks are dispatched x-fastest: every (b, h) of the longest query block
+  // first, so the launch ends on short blocks (longest-first scheduling)
+  const int qb = nqb - 1 - (int)blockIdx.y;
+  const int bh = blockIdx.x, b = bh / a.H, h = bh % a.H;
   const int nkb = 2 * (qb + 1);  // 64-key blocks up to and including the diagonal (>= 2)
   const int row0 = b * a.T;
 
@@ -385,8 +387,8 @@ __global__ void __launch_bounds__(320, 2) k_attn_bwd_kv8(const __grid_constant__
   const uint32_t sb = smem_u32(smem);
 
   const int nq64 = a.T / 64;
-  const int kb = (int)blockIdx.x;  // key block 0 has the most query blocks: first
-  const int bh = blockIdx.y, b = bh / a.H, h = bh % a.H;
+  const int kb = (int)blockIdx.y;  // key block 0 (most query blocks) of every (b, h) first
+  const int bh = blockIdx.x, b = bh / a.H, h = bh % a.H;
   const int row0 = b * a.T;
   const int i0 = 2 * kb;
   const int nit = nq64 - i0;
@@ -613,8 +615,8 @@ __global__ void __launch_bounds__(320, 2) k_attn_bwd_q8(const __grid_constant__ 
   const uint32_t sb = smem_u32(smem);
 
   const int nqb = a.T / 128;
-  const int qb = nqb - 1 - (int)blockIdx.x;
-  const int bh = blockIdx.y, b = bh / a.H, h = bh % a.H;
+  const int qb = nqb - 1 - (int)blockIdx.y;  // longest rows of every (b, h) first
+  const int bh = blockIdx.x, b = bh / a.H, h = bh % a.H;
   const int row0 = b * a.T;
   const int nkb = 2 * (qb + 1);  // 64-key blocks up to and including the diagonal
 
@@ -874,7 +876,7 @@ void attn_fwd_tc(Ctx& c, const AttnDesc& d) {
     cudaFuncSetAttribute(k_attn_fwd_o<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, D_SMEM);
     attr = true;
   }
-  dim3 grid(d.T / 128, d.B * d.H);
+  dim3 grid(d.B * d.H, d.T / 128);
   LaunchScope s(c, "attn_fwd_tc");
   if (d.drop.active) k_attn_fwd_o<true><<<grid, 192, D_SMEM, c.stream>>>(tq, tkv64, make_args(d, c.flags));
   else k_attn_fwd_o<false><<<grid, 192, D_SMEM, c.stream>>>(tq, tkv64, make_args(d, c.flags));
@@ -904,7 +906,7 @@ void attn_bwd_tc(Ctx& c, const AttnDesc& d) {
     attr = true;
   }
   AttnTcArgs a = make_args(d, c.flags);
-  dim3 grid(d.T / 128, d.B * d.H);
+  dim3 grid(d.B * d.H, d.T / 128);
   const bool drop = d.drop.active;
   {
     LaunchScope s(c, "attn_bwd_kv_tc");
