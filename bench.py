@@ -237,16 +237,18 @@ def run_ours(args, w, rank, world, local_rank):
         dist.barrier()
     torch.cuda.synchronize()
     l0 = model.launch_count()
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+    ev0, ev1 = evs[0], evs[-1]
     ev0.record()
     h0 = time.perf_counter()
-    for _ in range(args.steps):
+    for k in range(args.steps):
         st += 1
         model.train_step(d_stream, data_seed, lr_at(st), st, sync=False)
         flush.zero_()          # L2 flush between steps (256 MiB > 126 MB L2)
+        evs[k + 1].record()
     host_enqueue_ms = (time.perf_counter() - h0) * 1000.0 / args.steps
-    ev1.record()
     torch.cuda.synchronize()
+    per_step_ms = [evs[k].elapsed_time(evs[k + 1]) for k in range(args.steps)]
     if world > 1:
         dist.barrier()
     launches = model.launch_count() - l0
@@ -337,6 +339,8 @@ def run_ours(args, w, rank, world, local_rank):
                     "d2h_bytes_per_step": 16},
             "gpu_launches": int(launches),
             "host_enqueue_ms_per_step": host_enqueue_ms,
+            "step_ms_spread": {"min": min(per_step_ms), "median": statistics.median(per_step_ms),
+                               "max": max(per_step_ms)},
             "clocks": clk,
             "final_loss": loss, "final_grad_norm": norm,
             "kernels": kern,

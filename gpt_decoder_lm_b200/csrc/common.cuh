@@ -104,4 +104,74 @@ __device__ __forceinline__ float gelu_grad_f(float x) {
   return fmaf(x * 0.3989422804014327f, e, cdf);
 }
 
+// Two fp32 lanes in one 64-bit register: the sm_100 f32x2 FMA-pipe forms
+// (each lane rounds exactly like the scalar instruction).
+__device__ __forceinline__ uint64_t f2(float a, float b) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ float2 f2split(uint64_t r) {
+  float2 v;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(v.x), "=f"(v.y) : "l"(r));
+  return v;
+}
+__device__ __forceinline__ uint64_t f2fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2mul(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2add(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2sub(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2c(float c) { return f2(c, c); }
+
+// erf_as on a pair of arguments (same operations per lane as erf_as, the
+// polynomial and the affine steps on the f32x2 pipe).  Returns the pair of
+// erf values; e receives the pair e^{-z^2}.
+__device__ __forceinline__ uint64_t erf_as2(uint64_t z2, uint64_t& e2) {
+  const float2 z = f2split(z2);
+  const uint64_t az = f2(fabsf(z.x), fabsf(z.y));
+  const float2 den = f2split(f2fma(f2c(0.3275911f), az, f2c(1.0f)));
+  const uint64_t t = f2(__fdividef(1.0f, den.x), __fdividef(1.0f, den.y));
+  uint64_t q = f2fma(t, f2c(1.061405429f), f2c(-1.453152027f));
+  q = f2fma(t, q, f2c(1.421413741f));
+  q = f2fma(t, q, f2c(-0.284496736f));
+  q = f2fma(t, q, f2c(0.254829592f));
+  const uint64_t poly = f2mul(t, q);
+  const float2 sq = f2split(f2mul(az, az));
+  e2 = f2(__expf(-sq.x), __expf(-sq.y));
+  const float2 r = f2split(f2fma(f2mul(poly, f2c(-1.0f)), e2, f2c(1.0f)));
+  return f2(copysignf(r.x, z.x), copysignf(r.y, z.y));
+}
+// gelu_f and gelu_grad_f on a pair (a, b), in place
+__device__ __forceinline__ void gelu2(float& a, float& b) {
+  const uint64_t x = f2(a, b);
+  uint64_t e;
+  const uint64_t erf = erf_as2(f2mul(x, f2c(0.70710678118654752f)), e);
+  const float2 g = f2split(f2mul(f2mul(f2c(0.5f), x), f2add(f2c(1.0f), erf)));
+  a = g.x;
+  b = g.y;
+}
+__device__ __forceinline__ void gelu_grad2(float& a, float& b) {
+  const uint64_t x = f2(a, b);
+  uint64_t e;
+  const uint64_t cdf = f2mul(f2c(0.5f), f2add(f2c(1.0f), erf_as2(f2mul(x, f2c(0.70710678118654752f)), e)));
+  const float2 g = f2split(f2fma(f2mul(x, f2c(0.3989422804014327f)), e, cdf));
+  a = g.x;
+  b = g.y;
+}
+
 }  // namespace gpt

@@ -347,7 +347,7 @@ size_t carve(gpt_model& m, uint8_t* base) {
   m.dres = F((size_t)M * d);
   m.dln = F((size_t)M * d);
   m.dsum = F((size_t)M * m.H);
-  m.part_blocks = (int)std::min<long>(M, 148 * 8);
+  m.part_blocks = (int)std::min<long>(M, 148 * 8);  // capacity; the launch count is set at create
   m.part = F((size_t)m.part_blocks * 3 * d);
   m.colsum_scr = F((size_t)512 * 4 * d);
   // split-K scratch: the largest dW partial set
@@ -787,6 +787,7 @@ gpt_status gpt_create(const gpt_config* cfg, uint64_t seed, void* d_workspace, s
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess) m->ctx.num_sms = sms;
+  m->part_blocks = std::min(m->part_blocks, norm_bwd_blocks(m->ctx, m->M, m->d, m->bf16m));
   cudaStream_t st = m->ctx.stream;
   // zero the arenas (weights, grads, moments) and the scalars
   cudaMemsetAsync(m->scal, 0, 64 * 4, st);

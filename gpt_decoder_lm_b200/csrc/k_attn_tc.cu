@@ -312,33 +312,6 @@ __device__ __forceinline__ int pcol(int c) { return (c & 32) + ((c & 31) >> 1); 
 // TMEM A-operand column of K-step kk (16 elements) under that layout
 __device__ __forceinline__ uint32_t acol(int kk) { return (uint32_t)((kk >> 1) * 32 + (kk & 1) * 8); }
 
-// two fp32 lanes in one 64-bit register: the sm_100 f32x2 FMA-pipe forms
-// (each lane rounds exactly like the scalar instruction)
-__device__ __forceinline__ uint64_t f2(float a, float b) {
-  uint64_t r;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
-  return r;
-}
-__device__ __forceinline__ float2 f2split(uint64_t r) {
-  float2 v;
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(v.x), "=f"(v.y) : "l"(r));
-  return v;
-}
-__device__ __forceinline__ uint64_t f2fma(uint64_t a, uint64_t b, uint64_t c) {
-  uint64_t d;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-  return d;
-}
-__device__ __forceinline__ uint64_t f2mul(uint64_t a, uint64_t b) {
-  uint64_t d;
-  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-  return d;
-}
-__device__ __forceinline__ uint64_t f2sub(uint64_t a, uint64_t b) {
-  uint64_t d;
-  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-  return d;
-}
 __device__ __forceinline__ uint32_t pack2v(uint64_t v) {
   const float2 f = f2split(v);
   return pack2(f.x, f.y);

@@ -250,31 +250,44 @@ __global__ void k_norm_bwd(NormBwd p) {
   float pg[4] = {0, 0, 0, 0}, pb[4] = {0, 0, 0, 0}, pn[4] = {0, 0, 0, 0};
   int buf = 0;
   const float wv[4] = {gw.x, gw.y, gw.z, gw.w};
-  // two rows per round: one barrier for both rows' reductions
-  for (long r = r0; r < r1; r += 2) {
-    float dyv[2][4], xh[2][4], g[2][4], rstd[2], s[4] = {0.f, 0.f, 0.f, 0.f};
-    float4 old[2];  // the residual gradient these rows add to, fetched with dy and x
+  // Two rows per round (one barrier for both rows' reductions); the inputs of
+  // the next round (dy, x, the residual gradient they add to, mean, rstd) are
+  // loaded before this round's work, so loads stay in flight throughout.
+  struct Rows {
+    float4 dy[2], x[2], old[2];
+    float mean[2], rstd[2];
+  };
+  auto load = [&](long r, Rows& q) {
 #pragma unroll
     for (int u = 0; u < 2; u++) {
       const long rr = r + u;
       const bool live = rr < r1;
-      const float mean = (p.rms || !live) ? 0.f : p.mean[rr];
-      rstd[u] = live ? p.rstd[rr] : 0.f;
-      float4 dy = make_float4(0, 0, 0, 0), xv = make_float4(0, 0, 0, 0);
-      old[u] = make_float4(0, 0, 0, 0);
+      q.mean[u] = (p.rms || !live) ? 0.f : p.mean[rr];
+      q.rstd[u] = live ? p.rstd[rr] : 0.f;
+      q.dy[u] = q.x[u] = q.old[u] = make_float4(0, 0, 0, 0);
       if (own && live) {
-        dy = reinterpret_cast<const float4*>(p.dy + rr * p.d)[tid];
-        xv = reinterpret_cast<const float4*>(p.x + rr * p.d)[tid];
-        if (p.accumulate) old[u] = reinterpret_cast<const float4*>(p.dres + rr * p.d)[tid];
+        q.dy[u] = reinterpret_cast<const float4*>(p.dy + rr * p.d)[tid];
+        q.x[u] = reinterpret_cast<const float4*>(p.x + rr * p.d)[tid];
+        if (p.accumulate) q.old[u] = reinterpret_cast<const float4*>(p.dres + rr * p.d)[tid];
       }
-      const float dya[4] = {dy.x, dy.y, dy.z, dy.w}, xa[4] = {xv.x, xv.y, xv.z, xv.w};
+    }
+  };
+  Rows cur;
+  if (r0 < r1) load(r0, cur);
+  for (long r = r0; r < r1; r += 2) {
+    Rows nxt;
+    if (r + 2 < r1) load(r + 2, nxt);
+    float s[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int u = 0; u < 2; u++) {
+      const float dya[4] = {cur.dy[u].x, cur.dy[u].y, cur.dy[u].z, cur.dy[u].w};
+      const float xa[4] = {cur.x[u].x, cur.x[u].y, cur.x[u].z, cur.x[u].w};
 #pragma unroll
       for (int k = 0; k < 4; k++) {
-        dyv[u][k] = dya[k];
-        xh[u][k] = (xa[k] - mean) * rstd[u];
-        g[u][k] = dya[k] * wv[k];
-        s[2 * u] += g[u][k];
-        s[2 * u + 1] += g[u][k] * xh[u][k];
+        const float xh = (xa[k] - cur.mean[u]) * cur.rstd[u];
+        const float g = dya[k] * wv[k];
+        s[2 * u] += g;
+        s[2 * u + 1] += g * xh;
       }
     }
 #pragma unroll
@@ -296,16 +309,19 @@ __global__ void k_norm_bwd(NormBwd p) {
       if (!own || rr >= r1) continue;
       const float mg = p.rms ? 0.f : t[2 * u] / p.d;
       const float mgx = t[2 * u + 1] / p.d;
-      float4* dr = reinterpret_cast<float4*>(p.dres + rr * p.d) + tid;
-      const float ov[4] = {old[u].x, old[u].y, old[u].z, old[u].w};
+      const float dya[4] = {cur.dy[u].x, cur.dy[u].y, cur.dy[u].z, cur.dy[u].w};
+      const float xa[4] = {cur.x[u].x, cur.x[u].y, cur.x[u].z, cur.x[u].w};
+      const float ov[4] = {cur.old[u].x, cur.old[u].y, cur.old[u].z, cur.old[u].w};
       float nv[4];
 #pragma unroll
       for (int k = 0; k < 4; k++) {
-        nv[k] = ov[k] + rstd[u] * (g[u][k] - mg - xh[u][k] * mgx);
-        pg[k] += dyv[u][k] * xh[u][k];
-        pb[k] += dyv[u][k];
+        const float xh = (xa[k] - cur.mean[u]) * cur.rstd[u];
+        const float g = dya[k] * wv[k];
+        nv[k] = ov[k] + cur.rstd[u] * (g - mg - xh * mgx);
+        pg[k] += dya[k] * xh;
+        pb[k] += dya[k];
       }
-      *dr = make_float4(nv[0], nv[1], nv[2], nv[3]);
+      reinterpret_cast<float4*>(p.dres + rr * p.d)[tid] = make_float4(nv[0], nv[1], nv[2], nv[3]);
       if (p.want_dyb) {
         float q[4];
 #pragma unroll
@@ -316,6 +332,7 @@ __global__ void k_norm_bwd(NormBwd p) {
         store4<T>(reinterpret_cast<T*>(p.dyb) + rr * p.d + 4 * tid, make_float4(q[0], q[1], q[2], q[3]));
       }
     }
+    cur = nxt;
   }
   if (own) {
     float* out = p.part + (long)blockIdx.x * 3 * p.d;
@@ -325,8 +342,19 @@ __global__ void k_norm_bwd(NormBwd p) {
   }
 }
 
-int norm_bwd_blocks(Ctx& c, long rows) {
-  long b = (long)c.num_sms * 4;
+// one resident wave: the SM count times the blocks of k_norm_bwd<T> that fit
+// on an SM at this row length (each block walks a contiguous row range)
+int norm_bwd_blocks(Ctx& c, long rows, int d, bool bf16_out) {
+  const int threads = ((d / 4 + 31) / 32) * 32;
+  const size_t smem = (size_t)2 * (threads / 32) * 4 * sizeof(float);
+  int occ = 0;
+  cudaError_t e = bf16_out ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k_norm_bwd<bf16>, threads, smem)
+                           : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k_norm_bwd<float>, threads, smem);
+  if (e != cudaSuccess || occ < 1) {
+    cudaGetLastError();
+    occ = 1;
+  }
+  const long b = (long)c.num_sms * occ;
   return (int)(rows < b ? rows : b);
 }
 

@@ -138,7 +138,8 @@ struct NormBwd {
   long rows; int d; bool rms;
 };
 template <typename T> void norm_bwd(Ctx& c, const NormBwd& p);
-int norm_bwd_blocks(Ctx& c, long rows);
+// partial rows k_norm_bwd writes (one resident wave of blocks)
+int norm_bwd_blocks(Ctx& c, long rows, int d, bool bf16_out);
 // the three slots of part[blocks, 3, d] into g0, g1, g2 (each nullable), one launch
 void partial_reduce3(Ctx& c, const float* part, int blocks, int d, float* g0, float* g1, float* g2);
 
