@@ -71,6 +71,11 @@ def attn_flops_per_step(w) -> float:
     return L * w.grad_accum * per_layer_fwd * (1 + 2.5)
 
 
+# dram__bytes_read.sum + dram__bytes_write.sum of k_gemm_tc per launch, averaged over the
+# 735 launches of one training step (profiles/launch_list_gpt2_124m_train_step.md): 78.1 GB
+GEMM_DRAM_BYTES_PER_LAUNCH = 78.07e9 / 735
+
+
 class Clocks:
     """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
 
@@ -306,7 +311,8 @@ def run_ours(args, w, rank, world, local_rank):
     achieved = gemm_flops / (gemm_ms / 1000.0) / 1e12 if gemm_ms > 0 else 0.0
     roofline = {"bound": "tensor", "kernel": "gemm_tc (all dense contractions)", "achieved": achieved,
                 "peak": pk["bf16_sustained"], "unit": "TFLOP/s", "frac": achieved / pk["bf16_sustained"],
-                "traffic": None, "peak_source": pk["source"] + " sustained bf16",
+                "traffic": GEMM_DRAM_BYTES_PER_LAUNCH, "traffic_unit": "bytes per launch (ncu)",
+                "peak_source": pk["source"] + " sustained bf16",
                 "launches": gemm_n, "avg_launch_ms": gemm_ms / max(gemm_n, 1)}
     step_ms = ms_max / args.steps
     kern = {k: {"ms_per_step": v[0] / args.steps, "launches_per_step": v[1] / args.steps,
