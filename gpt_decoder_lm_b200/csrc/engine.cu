@@ -126,6 +126,17 @@ struct gpt_model {
   int32_t* argmax_out;
   size_t splitk_floats = 0;
   int part_blocks = 0;
+  // Reductions deferred to the last micro-batch of a step: the column
+  // partials of every norm backward and bias column sum, and the split-K
+  // partials of every weight-gradient GEMM, accumulate across micro-batches
+  // in per-instance buffers and are added to the gradients once per step.
+  int cur_micro = 0, n_micro = 1;
+  int part_cap = 0;                 // partial rows per norm instance
+  float* norm_parts = nullptr;      // [2L+1][part_cap][3][d]
+  float* colsum_parts = nullptr;    // [L][2][colsum chunks][4d]
+  float* split_parts = nullptr;     // per (layer, dW kind): [splits, Mo, No]
+  std::vector<size_t> split_off;    // offset of each (layer, kind) instance; kind: 0 mlp proj, 1 fc, 2 attn proj, 3 qkv
+  std::vector<int> split_n;         // its split count (1: no split buffer)
 
   Ctx ctx;
   Timing* timing = nullptr;
@@ -348,8 +359,26 @@ size_t carve(gpt_model& m, uint8_t* base) {
   m.dln = F((size_t)M * d);
   m.dsum = F((size_t)M * m.H);
   m.part_blocks = (int)std::min<long>(M, 148 * 8);  // capacity; the launch count is set at create
+  m.part_cap = m.part_blocks;
   m.part = F((size_t)m.part_blocks * 3 * d);
   m.colsum_scr = F((size_t)512 * 4 * d);
+  m.norm_parts = F((size_t)(2 * L + 1) * m.part_cap * 3 * d);
+  m.colsum_parts = F((size_t)L * 2 * colsum_chunks(M) * 4 * d);
+  {
+    // weight-gradient shapes [Mo, No] of the four per-layer GEMMs
+    const long dw[4][2] = {{d, 4L * d}, {4L * d, d}, {d, d}, {3L * d, d}};
+    m.split_off.assign((size_t)L * 4, 0);
+    m.split_n.assign((size_t)L * 4, 1);
+    size_t tot = 0;
+    for (int l = 0; l < L; l++)
+      for (int k = 0; k < 4; k++) {
+        const int sp = m.bf16m ? choose_splits(dw[k][0], dw[k][1], M) : 1;
+        m.split_off[(size_t)l * 4 + k] = tot;
+        m.split_n[(size_t)l * 4 + k] = sp;
+        if (sp > 1) tot += (size_t)sp * dw[k][0] * dw[k][1];
+      }
+    m.split_parts = F(std::max<size_t>(tot, 64));
+  }
   // split-K scratch: the largest dW partial set
   size_t sk = 0;
   long shapes[4][2] = {{3L * d, d}, {d, d}, {4L * d, d}, {d, 4L * d}};
@@ -539,8 +568,8 @@ gpt_status forward_t(gpt_model* m, bool fuse_ce_grad, float* loss_acc, float los
   return check_cuda(m, "forward");
 }
 
-void add_bias_grads_from_norm(gpt_model* m, int64_t gain, int64_t beta, int64_t next_bias) {
-  partial_reduce3(m->ctx, m->part, m->part_blocks, m->d, gain >= 0 ? m->G(gain) : nullptr,
+void add_bias_grads_from_norm(gpt_model* m, const float* part, int64_t gain, int64_t beta, int64_t next_bias) {
+  partial_reduce3(m->ctx, part, m->part_blocks, m->d, gain >= 0 ? m->G(gain) : nullptr,
                   beta >= 0 ? m->G(beta) : nullptr, next_bias >= 0 ? m->G(next_bias) : nullptr);
 }
 
@@ -560,7 +589,9 @@ gpt_status backward_t(gpt_model* m) {
   T* dh = reinterpret_cast<T*>(m->dh);
   T* dqkv = reinterpret_cast<T*>(m->dqkv);
   T* datt = reinterpret_cast<T*>(m->datt);
-  auto dW = [&](int Mo, int No, const void* A, const void* Bm, float* out, const char* name) -> bool {
+  const bool first = m->cur_micro == 0, last = m->cur_micro == m->n_micro - 1;
+  // inst: (layer, kind) of a per-layer weight gradient, -1 for the lm_head
+  auto dW = [&](int Mo, int No, const void* A, const void* Bm, float* out, const char* name, int inst) -> bool {
     // out[Mo, No] += A^T B with A [M, Mo], B [M, No] (tokens outermost)
     GemmDesc g = gd(Mo, No, (int)M, A, Mo, false, Bm, No, false);
     g.epi.kind = EPI_ACC_F32;
@@ -570,8 +601,25 @@ gpt_status backward_t(gpt_model* m) {
     if (m->bf16m) {
       g.split_k = choose_splits(Mo, No, M);
       g.partial = m->splitk;
+      if (inst >= 0 && m->split_n[inst] > 1 && gemm_tc_supported(g) &&
+          gemm_tc_splits(g, c.num_sms) == m->split_n[inst]) {
+        // split partials accumulate over the step's micro-batches in this
+        // instance's buffer; the last micro-batch adds them to the gradient
+        g.partial = m->split_parts + m->split_off[inst];
+        g.partial_accumulate = !first;
+        g.reduce_partials = last;
+      }
     }
     return gemm(m, g);
+  };
+  auto norm_part = [&](int k) { return m->norm_parts + (size_t)k * m->part_cap * 3 * d; };
+  auto colsum_part = [&](int l, int which) {
+    return m->colsum_parts + ((size_t)l * 2 + which) * colsum_chunks(M) * 4 * d;
+  };
+  // bias gradient = column sums of the operand-typed gradient x [M, N]
+  auto bias_grad = [&](const T* x, int N, int l, int which, float* grad) {
+    colsum_partial<T>(c, x, M, N, colsum_part(l, which), !first);
+    if (last) colsum_reduce(c, colsum_part(l, which), colsum_chunks(M), N, grad);
   };
   // lm_head: dx_f = dlogits W_head; dW_head += dlogits^T x_f
   GemmDesc g = gd((int)M, d, Vp, dl, Vp, true, m->Wop(m->head), d, false);
@@ -580,7 +628,8 @@ gpt_status backward_t(gpt_model* m) {
   g.epi.out = m->dln;
   g.epi.ldo = d;
   if (!gemm(m, g)) return fail(m, GPT_ERR_CUDA, "lm_head dX gemm failed");
-  if (!dW(Vp, d, dl, m->lnf, m->G(m->head), "gemm_lmhead_dw")) return fail(m, GPT_ERR_CUDA, "lm_head dW gemm failed");
+  if (!dW(Vp, d, dl, m->lnf, m->G(m->head), "gemm_lmhead_dw", -1))
+    return fail(m, GPT_ERR_CUDA, "lm_head dW gemm failed");
   // final norm
   NormBwd nb;
   nb.dy = m->dln;
@@ -593,13 +642,14 @@ gpt_status backward_t(gpt_model* m) {
   nb.dyb = dyb;
   nb.drop = dkey(m, L - 1, 3);
   nb.want_dyb = true;
-  nb.part = m->part;
+  nb.part = norm_part(2 * L);
+  nb.part_accumulate = !first;
   nb.blocks = m->part_blocks;
   nb.rows = M;
   nb.d = d;
   nb.rms = rms;
   norm_bwd<T>(c, nb);
-  add_bias_grads_from_norm(m, m->lnf_w, m->lnf_b, m->layers[L - 1].pr_b);
+  if (last) add_bias_grads_from_norm(m, nb.part, m->lnf_w, m->lnf_b, m->layers[L - 1].pr_b);
   for (int l = L - 1; l >= 0; l--) {
     const LayerP& y = m->layers[l];
     T* a1 = at<T>(m->ln1, l * Md);
@@ -609,7 +659,8 @@ gpt_status backward_t(gpt_model* m) {
     T* h = at<T>(m->fch, l * 4 * Md);
     T* gg = at<T>(m->fcg, l * 4 * Md);
     // MLP projection
-    if (!dW(d, 4 * d, dyb, gg, m->G(y.pr_w), "gemm_mlpproj_dw")) return fail(m, GPT_ERR_CUDA, "proj dW failed");
+    if (!dW(d, 4 * d, dyb, gg, m->G(y.pr_w), "gemm_mlpproj_dw", l * 4 + 0))
+      return fail(m, GPT_ERR_CUDA, "proj dW failed");
     g = gd((int)M, 4 * d, d, dyb, d, true, m->Wop(y.pr_w), 4 * d, false);
     g.epi.kind = EPI_ACT_BWD;
     g.name = "gemm_mlpproj_dx";
@@ -618,8 +669,8 @@ gpt_status backward_t(gpt_model* m) {
     g.epi.out = dh;
     g.epi.ldo = 4 * d;
     if (!gemm(m, g)) return fail(m, GPT_ERR_CUDA, "proj dX failed");
-    if (y.fc_b >= 0) colsum_acc<T>(c, dh, M, 4 * d, m->colsum_scr, m->G(y.fc_b));
-    if (!dW(4 * d, d, dh, a2, m->G(y.fc_w), "gemm_fc_dw")) return fail(m, GPT_ERR_CUDA, "fc dW failed");
+    if (y.fc_b >= 0) bias_grad(dh, 4 * d, l, 0, m->G(y.fc_b));
+    if (!dW(4 * d, d, dh, a2, m->G(y.fc_w), "gemm_fc_dw", l * 4 + 1)) return fail(m, GPT_ERR_CUDA, "fc dW failed");
     g = gd((int)M, d, 4 * d, dh, 4 * d, true, m->Wop(y.fc_w), d, false);
     g.epi.kind = EPI_STORE_F32;
     g.name = "gemm_fc_dx";
@@ -634,10 +685,12 @@ gpt_status backward_t(gpt_model* m) {
     nb.accumulate = true;
     nb.drop = dkey(m, l, 2);
     nb.want_dyb = true;
+    nb.part = norm_part(2 * l + 1);
     norm_bwd<T>(c, nb);
-    add_bias_grads_from_norm(m, y.ln2_w, y.ln2_b, y.ap_b);
+    if (last) add_bias_grads_from_norm(m, nb.part, y.ln2_w, y.ln2_b, y.ap_b);
     // attention projection
-    if (!dW(d, d, dyb, o, m->G(y.ap_w), "gemm_attnproj_dw")) return fail(m, GPT_ERR_CUDA, "attn proj dW failed");
+    if (!dW(d, d, dyb, o, m->G(y.ap_w), "gemm_attnproj_dw", l * 4 + 2))
+      return fail(m, GPT_ERR_CUDA, "attn proj dW failed");
     g = gd((int)M, d, d, dyb, d, true, m->Wop(y.ap_w), d, false);
     g.epi.kind = EPI_STORE;
     g.name = "gemm_attnproj_dx";
@@ -647,8 +700,9 @@ gpt_status backward_t(gpt_model* m) {
     AttnDesc ad{m->B, m->T, m->H, m->hd, qkv, o, m->lse + (size_t)l * M * m->H, datt, dqkv, m->dsum, dkey(m, l, 1)};
     if (sizeof(T) == 2 && attn_tc_supported(ad)) attn_bwd_tc(c, ad);
     else attn_bwd_simt<T>(c, ad);
-    if (y.qkv_b >= 0) colsum_acc<T>(c, dqkv, M, 3 * d, m->colsum_scr, m->G(y.qkv_b));
-    if (!dW(3 * d, d, dqkv, a1, m->G(y.qkv_w), "gemm_qkv_dw")) return fail(m, GPT_ERR_CUDA, "qkv dW failed");
+    if (y.qkv_b >= 0) bias_grad(dqkv, 3 * d, l, 1, m->G(y.qkv_b));
+    if (!dW(3 * d, d, dqkv, a1, m->G(y.qkv_w), "gemm_qkv_dw", l * 4 + 3))
+      return fail(m, GPT_ERR_CUDA, "qkv dW failed");
     g = gd((int)M, d, 3 * d, dqkv, 3 * d, true, m->Wop(y.qkv_w), d, false);
     g.epi.kind = EPI_STORE_F32;
     g.name = "gemm_qkv_dx";
@@ -663,8 +717,9 @@ gpt_status backward_t(gpt_model* m) {
     nb.accumulate = true;
     nb.drop = l > 0 ? dkey(m, l - 1, 3) : DropKey{};
     nb.want_dyb = l > 0;
+    nb.part = norm_part(2 * l);
     norm_bwd<T>(c, nb);
-    add_bias_grads_from_norm(m, y.ln1_w, y.ln1_b, l > 0 ? m->layers[l - 1].pr_b : -1);
+    if (last) add_bias_grads_from_norm(m, nb.part, y.ln1_w, y.ln1_b, l > 0 ? m->layers[l - 1].pr_b : -1);
   }
   embed_sort(c, m->idx, M, m->stok, m->spos, m->nuniq);
   embed_bwd(c, m->dres, m->stok, m->spos, M, m->T, m->B, d, dkey(m, L, 0), m->G(m->wte), m->G(m->wpe), m->seg);
@@ -858,6 +913,8 @@ gpt_status gpt_forward_loss(gpt_model* m, const int32_t* d_idx, const int32_t* d
 gpt_status gpt_backward(gpt_model* m) {
   if (!m) return GPT_ERR_INVALID_ARG;
   if (!m->have_forward) return fail(m, GPT_ERR_STATE, "backward called without a preceding forward_loss");
+  m->cur_micro = 0;  // a stand-alone backward completes its gradients
+  m->n_micro = 1;
   gpt_status s = backward_any(m);
   m->have_forward = false;
   return s;
@@ -884,6 +941,8 @@ static gpt_status train_body(gpt_model* m, const void* d_stream, uint64_t len, u
   Ctx& c = m->ctx;
   for (int mu = 0; mu < m->ga; mu++) {
     m->drop_counter = (int64_t)step * m->ga + mu;
+    m->cur_micro = mu;
+    m->n_micro = m->ga;
     if (d_stream) {
       gather_batch(c, d_stream, m->cfg.token_dtype == GPT_TOK_U16, len, seed, step, mu, m->B, m->T, m->V, m->idx,
                    m->tgt, dev_params ? m->step_dev : nullptr);

@@ -42,6 +42,7 @@ struct TcArgs {
   int num_m, num_n, splits, kb_per_split, nkb;
   int n_fast;  // tile order: 1 = N-fastest (concurrent CTAs share A tiles in L2), 0 = M-fastest
   int kind, act;
+  int acc_partial;  // split partials: 1 = TMA reduce-add into the partial buffer, 0 = store
   const float* bias;
   DropKey drop;
   uint32_t* flags;
@@ -400,7 +401,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
-          if (p.splits > 1) tma_store_3d(&tm_out, bufA, col0, row0, split);
+          if (p.splits > 1) {
+            if (p.acc_partial) tma_reduce_add_3d(&tm_out, bufA, col0, row0, split);
+            else tma_store_3d(&tm_out, bufA, col0, row0, split);
+          }
           else if (kind == EPI_ACC_F32) tma_reduce_add_2d(&tm_out, bufA, col0, row0);
           else tma_store_2d(&tm_out, bufA, col0, row0);
           if (kind == EPI_BIAS_ACT && p.splits == 1) tma_store_2d(&tm_out2, bufB, col0, row0);
@@ -521,6 +525,7 @@ bool launch(Ctx& c, const GemmDesc& g, int splits) {
   a.kb_per_split = (a.nkb + splits - 1) / splits;
   a.kind = e.kind;
   a.act = e.act;
+  a.acc_partial = g.partial_accumulate ? 1 : 0;
   a.bias = e.bias;
   a.drop = e.drop;
   a.flags = c.flags;
@@ -589,9 +594,9 @@ bool gemm_tc_supported(const GemmDesc& g) {
   return true;
 }
 
-bool gemm_tc_bf16(Ctx& c, const GemmDesc& g) {
+int gemm_tc_splits(const GemmDesc& g, int num_sms) {
   bool split_ok = g.epi.kind == EPI_ACC_F32 && g.partial && g.split_k > 1;
-  TcPlan plan = gemm_tc_plan(g.M, g.N, g.K, split_ok, c.num_sms);
+  TcPlan plan = gemm_tc_plan(g.M, g.N, g.K, split_ok, num_sms);
   int splits = plan.splits;
   if (splits > g.split_k) splits = g.split_k < 1 ? 1 : g.split_k;  // never beyond the caller's scratch
   if (splits > 1) {  // keep every split non-empty
@@ -599,6 +604,13 @@ bool gemm_tc_bf16(Ctx& c, const GemmDesc& g) {
     int kbps = (nkb + splits - 1) / splits;
     splits = (nkb + kbps - 1) / kbps;
   }
+  return splits;
+}
+
+bool gemm_tc_bf16(Ctx& c, const GemmDesc& g) {
+  bool split_ok = g.epi.kind == EPI_ACC_F32 && g.partial && g.split_k > 1;
+  TcPlan plan = gemm_tc_plan(g.M, g.N, g.K, split_ok, c.num_sms);
+  const int splits = gemm_tc_splits(g, c.num_sms);
   bool amn = !g.a_kmajor, bmn = !g.b_kmajor;
   bool ok;
   if (plan.bn == 256) {
@@ -611,7 +623,8 @@ bool gemm_tc_bf16(Ctx& c, const GemmDesc& g) {
     else ok = launch<128, true, true>(c, g, splits);
   }
   if (!ok) return false;
-  if (splits > 1) splitk_reduce(c, g.partial, splits, (long)g.M * g.N, reinterpret_cast<float*>(g.epi.out));
+  if (splits > 1 && g.reduce_partials)
+    splitk_reduce(c, g.partial, splits, (long)g.M * g.N, reinterpret_cast<float*>(g.epi.out));
   return true;
 }
 

@@ -335,10 +335,18 @@ __global__ void k_norm_bwd(NormBwd p) {
     cur = nxt;
   }
   if (own) {
-    float* out = p.part + (long)blockIdx.x * 3 * p.d;
-    reinterpret_cast<float4*>(out)[tid] = make_float4(pg[0], pg[1], pg[2], pg[3]);
-    reinterpret_cast<float4*>(out + p.d)[tid] = make_float4(pb[0], pb[1], pb[2], pb[3]);
-    reinterpret_cast<float4*>(out + 2 * p.d)[tid] = make_float4(pn[0], pn[1], pn[2], pn[3]);
+    float4* out = reinterpret_cast<float4*>(p.part + (long)blockIdx.x * 3 * p.d) + tid;
+    float4 s0 = make_float4(pg[0], pg[1], pg[2], pg[3]), s1 = make_float4(pb[0], pb[1], pb[2], pb[3]),
+           s2 = make_float4(pn[0], pn[1], pn[2], pn[3]);
+    if (p.part_accumulate) {  // earlier micro-batches' partials of the same rows range
+      const float4 o0 = out[0], o1 = out[d4], o2 = out[2 * d4];
+      s0 = make_float4(o0.x + s0.x, o0.y + s0.y, o0.z + s0.z, o0.w + s0.w);
+      s1 = make_float4(o1.x + s1.x, o1.y + s1.y, o1.z + s1.z, o1.w + s1.w);
+      s2 = make_float4(o2.x + s2.x, o2.y + s2.y, o2.z + s2.z, o2.w + s2.w);
+    }
+    out[0] = s0;
+    out[d4] = s1;
+    out[2 * d4] = s2;
   }
 }
 
@@ -412,14 +420,16 @@ void partial_reduce3(Ctx& c, const float* part, int blocks, int d, float* g0, fl
 // column sums (bias gradients): chunk partials then a fixed-order reduce
 // ============================================================================
 template <typename T>
-__global__ void k_colsum(const T* __restrict__ x, long rows, int N, int chunks, float* __restrict__ part) {
+__global__ void k_colsum(const T* __restrict__ x, long rows, int N, int chunks, float* __restrict__ part,
+                         int accumulate) {
   int j = blockIdx.x * blockDim.x + threadIdx.x;
   if (j >= N) return;
   long per = (rows + chunks - 1) / chunks;
   long r0 = blockIdx.y * per, r1 = min(rows, r0 + per);
   float s = 0.f;
   for (long r = r0; r < r1; r++) s += to_f<T>(x[r * N + j]);
-  part[(long)blockIdx.y * N + j] = s;
+  float* dst = part + (long)blockIdx.y * N + j;
+  *dst = accumulate ? *dst + s : s;
 }
 
 // grad[j] += sum_c part[c, j]: row group y of 8 sums chunks y, y+8, ...; the
@@ -432,7 +442,8 @@ void colsum_reduce(Ctx& c, const float* part, int chunks, int N, float* grad) {
 
 // bf16 rows with N % 8 == 0: each thread sums 8 adjacent columns over its
 // row chunk with 16-byte loads
-__global__ void k_colsum_bf16x8(const bf16* __restrict__ x, long rows, int N, int chunks, float* __restrict__ part) {
+__global__ void k_colsum_bf16x8(const bf16* __restrict__ x, long rows, int N, int chunks, float* __restrict__ part,
+                                int accumulate) {
   const int j8 = blockIdx.x * blockDim.x + threadIdx.x;
   if (j8 * 8 >= N) return;
   const long per = (rows + chunks - 1) / chunks;
@@ -460,25 +471,38 @@ __global__ void k_colsum_bf16x8(const bf16* __restrict__ x, long rows, int N, in
   }
   for (; r < r1; r++) add(reinterpret_cast<const uint4*>(x + r * N)[j8]);
   float4* dst = reinterpret_cast<float4*>(part + (long)blockIdx.y * N + j8 * 8);
+  if (accumulate) {  // earlier micro-batches' sums of the same chunk
+    const float4 o0 = dst[0], o1 = dst[1];
+    s[0] += o0.x, s[1] += o0.y, s[2] += o0.z, s[3] += o0.w;
+    s[4] += o1.x, s[5] += o1.y, s[6] += o1.z, s[7] += o1.w;
+  }
   dst[0] = make_float4(s[0], s[1], s[2], s[3]);
   dst[1] = make_float4(s[4], s[5], s[6], s[7]);
 }
 
+int colsum_chunks(long rows) { return (int)min(512L, rows); }
+
+template <typename T>
+void colsum_partial(Ctx& c, const T* x, long rows, int N, float* part, bool accumulate) {
+  const bool vec = sizeof(T) == 2 && N % 8 == 0;
+  const int chunks = colsum_chunks(rows);  // few threads per row, many row chunks
+  LaunchScope s(c, "colsum");
+  if (vec) {
+    dim3 grid((N / 8 + 127) / 128, chunks);
+    k_colsum_bf16x8<<<grid, 128, 0, c.stream>>>(reinterpret_cast<const bf16*>(x), rows, N, chunks, part,
+                                                accumulate ? 1 : 0);
+  } else {
+    dim3 grid((N + 127) / 128, chunks);
+    k_colsum<T><<<grid, 128, 0, c.stream>>>(x, rows, N, chunks, part, accumulate ? 1 : 0);
+  }
+}
+template void colsum_partial<float>(Ctx&, const float*, long, int, float*, bool);
+template void colsum_partial<bf16>(Ctx&, const bf16*, long, int, float*, bool);
+
 template <typename T>
 void colsum_acc(Ctx& c, const T* x, long rows, int N, float* scratch, float* grad) {
-  const bool vec = sizeof(T) == 2 && N % 8 == 0;
-  int chunks = (int)min(vec ? 512L : 64L, rows);  // vector path: fewer threads per row, more row chunks
-  {
-    LaunchScope s(c, "colsum");
-    if (vec) {
-      dim3 grid((N / 8 + 127) / 128, chunks);
-      k_colsum_bf16x8<<<grid, 128, 0, c.stream>>>(reinterpret_cast<const bf16*>(x), rows, N, chunks, scratch);
-    } else {
-      dim3 grid((N + 127) / 128, chunks);
-      k_colsum<T><<<grid, 128, 0, c.stream>>>(x, rows, N, chunks, scratch);
-    }
-  }
-  colsum_reduce(c, scratch, chunks, N, grad);
+  colsum_partial<T>(c, x, rows, N, scratch, false);
+  colsum_reduce(c, scratch, colsum_chunks(rows), N, grad);
 }
 template void colsum_acc<float>(Ctx&, const float*, long, int, float*, float*);
 template void colsum_acc<bf16>(Ctx&, const bf16*, long, int, float*, float*);

@@ -69,6 +69,8 @@ struct GemmDesc {
   GemmEpi epi;
   int split_k = 1;            // > 1 only with EPI_ACC_F32: most splits `partial` holds
   float* partial = nullptr;   // [split_k, M, N] fp32 scratch
+  bool partial_accumulate = false;  // split partials are added into `partial` (else stored)
+  bool reduce_partials = true;      // out += sum of the partials after the GEMM
   const char* name = nullptr; // timing label
 };
 
@@ -86,6 +88,8 @@ void gemm_simt_f32(Ctx& c, const GemmDesc& g);
 void gemm_simt_bf16(Ctx& c, const GemmDesc& g);
 bool gemm_tc_supported(const GemmDesc& g);
 bool gemm_tc_bf16(Ctx& c, const GemmDesc& g);  // false: tensor-map encode failed
+// the split-K count gemm_tc_bf16 uses for g (1: none)
+int gemm_tc_splits(const GemmDesc& g, int num_sms);
 // split-K reduction: out[m,n] += sum_s partial[s,m,n] (fixed order)
 void splitk_reduce(Ctx& c, const float* partial, int splits, long MN, float* out);
 
@@ -135,6 +139,7 @@ struct NormBwd {
   float* dres; bool accumulate;
   void* dyb; DropKey drop; bool want_dyb;
   float* part; int blocks;
+  bool part_accumulate = false;  // add into part (else store)
   long rows; int d; bool rms;
 };
 template <typename T> void norm_bwd(Ctx& c, const NormBwd& p);
@@ -145,6 +150,10 @@ void partial_reduce3(Ctx& c, const float* part, int blocks, int d, float* g0, fl
 
 // column sums of an operand-typed [rows, N] matrix into grad (+=), deterministic
 template <typename T> void colsum_acc(Ctx& c, const T* x, long rows, int N, float* scratch, float* grad);
+// the chunk partials of those sums, part[colsum_chunks(rows), N] (= or += with accumulate);
+// colsum_reduce then adds them to grad
+int colsum_chunks(long rows);
+template <typename T> void colsum_partial(Ctx& c, const T* x, long rows, int N, float* part, bool accumulate);
 
 // Cross-entropy over [M, Vp] logits (operand type).  Writes per-row lse and
 // loss terms; with want_grad, overwrites logits with (softmax - onehot)*scale
