@@ -347,7 +347,7 @@ def run_ours(args, w, rank, world, local_rank):
             "gpu_launches": int(launches),
             "host_enqueue_ms_per_step": host_enqueue_ms,
             "step_ms_spread": {"min": min(per_step_ms), "median": statistics.median(per_step_ms),
-                               "max": max(per_step_ms)},
+                               "max": max(per_step_ms), "steps": [round(x, 3) for x in per_step_ms]},
             "clocks": clk,
             "final_loss": loss, "final_grad_norm": norm,
             "kernels": kern,

@@ -156,22 +156,17 @@ __device__ __forceinline__ uint64_t erf_as2(uint64_t z2, uint64_t& e2) {
   const float2 r = f2split(f2fma(f2mul(poly, f2c(-1.0f)), e2, f2c(1.0f)));
   return f2(copysignf(r.x, z.x), copysignf(r.y, z.y));
 }
-// gelu_f and gelu_grad_f on a pair (a, b), in place
-__device__ __forceinline__ void gelu2(float& a, float& b) {
-  const uint64_t x = f2(a, b);
-  uint64_t e;
-  const uint64_t erf = erf_as2(f2mul(x, f2c(0.70710678118654752f)), e);
-  const float2 g = f2split(f2mul(f2mul(f2c(0.5f), x), f2add(f2c(1.0f), erf)));
-  a = g.x;
-  b = g.y;
-}
-__device__ __forceinline__ void gelu_grad2(float& a, float& b) {
+// gelu_f and gelu_grad_f of a pair (a, b) at once (one erf / exp): the
+// activations replace (a, b), the derivatives go to (ga, gb)
+__device__ __forceinline__ void gelu_and_grad2(float& a, float& b, float& ga, float& gb) {
   const uint64_t x = f2(a, b);
   uint64_t e;
   const uint64_t cdf = f2mul(f2c(0.5f), f2add(f2c(1.0f), erf_as2(f2mul(x, f2c(0.70710678118654752f)), e)));
-  const float2 g = f2split(f2fma(f2mul(x, f2c(0.3989422804014327f)), e, cdf));
+  const float2 g = f2split(f2mul(x, cdf));
+  const float2 d = f2split(f2fma(f2mul(x, f2c(0.3989422804014327f)), e, cdf));
   a = g.x;
   b = g.y;
+  ga = d.x;
+  gb = d.y;
 }
-
 }  // namespace gpt

@@ -504,7 +504,7 @@ gpt_status forward_t(gpt_model* m, bool fuse_ce_grad, float* loss_acc, float los
     T* qkv = at<T>(m->qkv, l * 3 * Md);
     T* o = at<T>(m->atto, l * Md);
     T* a2 = at<T>(m->ln2, l * Md);
-    T* h = at<T>(m->fch, l * 4 * Md);
+    T* h = at<T>(m->fch, l * 4 * Md);  // act'(fc pre-activation), for the backward
     T* gg = at<T>(m->fcg, l * 4 * Md);
     norm_fwd<T>(c, x, rms ? nullptr : m->P(y.ln1_w), rms ? nullptr : m->P(y.ln1_b), a1, m->ln1_mean + l * M,
                 m->ln1_rstd + l * M, M, d, rms, eps);

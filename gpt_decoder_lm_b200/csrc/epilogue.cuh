@@ -21,7 +21,7 @@ __device__ __forceinline__ void epi_apply(const GemmEpi& e, int N, long m, int n
       break;
     case EPI_BIAS_ACT: {
       float h = acc + (e.bias ? e.bias[n] : 0.f);
-      reinterpret_cast<T*>(e.out)[m * e.ldo + n] = from_f<T>(h);
+      reinterpret_cast<T*>(e.out)[m * e.ldo + n] = from_f<T>(act_grad(e.act, h));
       reinterpret_cast<T*>(e.out2)[m * e.ldo + n] = from_f<T>(act_fwd(e.act, h));
       break;
     }
@@ -32,8 +32,8 @@ __device__ __forceinline__ void epi_apply(const GemmEpi& e, int N, long m, int n
       break;
     }
     case EPI_ACT_BWD: {
-      float h = to_f<T>(reinterpret_cast<const T*>(e.aux)[m * e.ldo + n]);
-      reinterpret_cast<T*>(e.out)[m * e.ldo + n] = from_f<T>(acc * act_grad(e.act, h));
+      float dact = to_f<T>(reinterpret_cast<const T*>(e.aux)[m * e.ldo + n]);
+      reinterpret_cast<T*>(e.out)[m * e.ldo + n] = from_f<T>(acc * dact);
       break;
     }
     case EPI_ACC_F32:

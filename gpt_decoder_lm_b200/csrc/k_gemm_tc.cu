@@ -349,32 +349,28 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (has_bias) add_bias(bias, v);
                 stage_bf16(bufA, lane, hh, v);
                 break;
-              case EPI_BIAS_ACT:
+              case EPI_BIAS_ACT: {
                 if (has_bias) add_bias(bias, v);
-                stage_bf16(bufA, lane, hh, v);
+                float dv[16];  // act'(h), kept for the backward pass
                 if (p.act == ACT_GELU) {
 #pragma unroll
-                  for (int i = 0; i < 16; i += 2) gelu2(v[i], v[i + 1]);
+                  for (int i = 0; i < 16; i += 2) gelu_and_grad2(v[i], v[i + 1], dv[i], dv[i + 1]);
                 } else {
 #pragma unroll
-                  for (int i = 0; i < 16; i++) v[i] = act_fwd(p.act, v[i]);
+                  for (int i = 0; i < 16; i++) {
+                    dv[i] = act_grad(p.act, v[i]);
+                    v[i] = act_fwd(p.act, v[i]);
+                  }
                 }
+                stage_bf16(bufA, lane, hh, dv);
                 stage_bf16(bufB, lane, hh, v);
                 break;
+              }
               case EPI_ACT_BWD: {
-                float hv[16];
-                unstage_bf16(bufB, lane, hh, hv);
-                if (p.act == ACT_GELU) {
+                float dv[16];  // the saved act'(h)
+                unstage_bf16(bufB, lane, hh, dv);
 #pragma unroll
-                  for (int i = 0; i < 16; i += 2) {
-                    gelu_grad2(hv[i], hv[i + 1]);
-                    v[i] *= hv[i];
-                    v[i + 1] *= hv[i + 1];
-                  }
-                } else {
-#pragma unroll
-                  for (int i = 0; i < 16; i++) v[i] *= act_grad(p.act, hv[i]);
-                }
+                for (int i = 0; i < 16; i++) v[i] *= dv[i];
                 stage_bf16(bufA, lane, hh, v);
                 break;
               }

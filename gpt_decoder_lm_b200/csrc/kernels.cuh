@@ -36,9 +36,9 @@ struct LaunchScope {
 enum EpiKind {
   EPI_STORE = 0,      // out = acc                                   (operand type)
   EPI_BIAS = 1,       // out = acc + bias                            (operand type)
-  EPI_BIAS_ACT = 2,   // out = acc + bias (pre-activation), out2 = act(out)
+  EPI_BIAS_ACT = 2,   // h = acc + bias: out = act'(h) (kept for backward), out2 = act(h)
   EPI_RESADD = 3,     // res_out = res_in + drop(acc + bias)         (fp32)
-  EPI_ACT_BWD = 4,    // out = acc * act'(aux)                       (operand type)
+  EPI_ACT_BWD = 4,    // out = acc * aux (aux = the saved act'(h))   (operand type)
   EPI_ACC_F32 = 5,    // outf += acc                                 (fp32, grad accumulation)
   EPI_STORE_F32 = 6   // outf = acc                                  (fp32)
 };
@@ -50,7 +50,7 @@ struct GemmEpi {
   void* out = nullptr;        // operand-typed output (kinds 0,1,2,4) or fp32 (5,6)
   void* out2 = nullptr;       // activation output of EPI_BIAS_ACT (same ld as out)
   int ldo = 0;
-  const void* aux = nullptr;  // pre-activation h of EPI_ACT_BWD (operand type, ld = ldo)
+  const void* aux = nullptr;  // act'(h) of EPI_ACT_BWD (operand type, ld = ldo)
   const float* bias = nullptr;
   const float* res_in = nullptr;
   float* res_out = nullptr;

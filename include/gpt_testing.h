@@ -22,8 +22,8 @@ extern "C" {
 enum { GPT_GEMM_SIMT_F32 = 0, GPT_GEMM_SIMT_BF16 = 1, GPT_GEMM_TC_BF16 = 2 };
 
 /* D[m, n] = sum_k A[m, k] * B[n, k] followed by epilogue `epi_kind`:
- *   0 out = D; 1 out = D + bias; 2 out = D + bias, out2 = act(out);
- *   3 res_out = res_in + D + bias; 4 out = D * act'(aux);
+ *   0 out = D; 1 out = D + bias; 2 with h = D + bias: out = act'(h), out2 = act(h);
+ *   3 res_out = res_in + D + bias; 4 out = D * aux (aux: a saved act'(h));
  *   5 out += D (fp32); 6 out = D (fp32).
  * A is [M, K] row-major with pitch lda when a_kmajor, else [K, M] (pitch lda);
  * B is [N, K] when b_kmajor, else [K, N].  Operands are fp32 for
