@@ -232,10 +232,12 @@ def run_ours(args, w, rank, world, local_rank):
     clocks = Clocks(local_rank) if rank == 0 else None
     if clocks:
         clocks.wait_ready()
-    # warm-up (untimed)
+    # warm-up (untimed): the same work as a timed step, L2 flush included (its first launch
+    # also loads torch's fill kernel, which must not land in the timed region)
     for _ in range(args.warmup):
         st += 1
         model.train_step(d_stream, data_seed, lr_at(st), st, sync=False)
+        flush.zero_()
     torch.cuda.synchronize()
     if clocks:
         clocks.mark()
