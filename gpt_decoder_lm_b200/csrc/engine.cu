@@ -131,6 +131,11 @@ struct gpt_model {
   // partials of every weight-gradient GEMM, accumulate across micro-batches
   // in per-instance buffers and are added to the gradients once per step.
   int cur_micro = 0, n_micro = 1;
+  // a training step gathers every micro-batch's tokens first and sorts their
+  // embedding-gradient routing in one launch (one CTA per micro-batch)
+  int32_t *idx_all = nullptr, *tgt_all = nullptr, *stok_all = nullptr, *spos_all = nullptr, *nuniq_all = nullptr;
+  int32_t *idx0 = nullptr, *tgt0 = nullptr;  // the stand-alone forward's buffers
+  bool presorted = false;
   int part_cap = 0;                 // partial rows per norm instance
   float* norm_parts = nullptr;      // [2L+1][part_cap][3][d]
   float* colsum_parts = nullptr;    // [L][2][colsum chunks][4d]
@@ -400,6 +405,13 @@ size_t carve(gpt_model& m, uint8_t* base) {
   m.stok = I(M);
   m.spos = I(M);
   m.nuniq = I(64);
+  m.idx_all = I((size_t)m.ga * M);
+  m.tgt_all = I((size_t)m.ga * M);
+  m.stok_all = I((size_t)m.ga * M);
+  m.spos_all = I((size_t)m.ga * M);
+  m.nuniq_all = I((size_t)m.ga + 64);
+  m.idx0 = m.idx;
+  m.tgt0 = m.tgt;
   m.norm_part = (double*)(base + lay.take(148 * 4 * 8 + 64));
   m.argmax_out = I(M + 64);
   return lay.off + 1024;
@@ -721,8 +733,14 @@ gpt_status backward_t(gpt_model* m) {
     norm_bwd<T>(c, nb);
     if (last) add_bias_grads_from_norm(m, nb.part, y.ln1_w, y.ln1_b, l > 0 ? m->layers[l - 1].pr_b : -1);
   }
-  embed_sort(c, m->idx, M, m->stok, m->spos, m->nuniq);
-  embed_bwd(c, m->dres, m->stok, m->spos, M, m->T, m->B, d, dkey(m, L, 0), m->G(m->wte), m->G(m->wpe), m->seg);
+  const int32_t *stok = m->stok, *spos = m->spos;
+  if (m->presorted) {
+    stok = m->stok_all + (size_t)m->cur_micro * M;
+    spos = m->spos_all + (size_t)m->cur_micro * M;
+  } else {
+    embed_sort(c, m->idx, M, m->stok, m->spos, m->nuniq);
+  }
+  embed_bwd(c, m->dres, stok, spos, M, m->T, m->B, d, dkey(m, L, 0), m->G(m->wte), m->G(m->wpe), m->seg);
   return check_cuda(m, "backward");
 }
 
@@ -939,23 +957,32 @@ gpt_status gpt_clip_adamw_step(gpt_model* m, float lr, int32_t step, float* h_gr
 static gpt_status train_body(gpt_model* m, const void* d_stream, uint64_t len, uint64_t seed, float lr, int32_t step,
                              bool dev_params) {
   Ctx& c = m->ctx;
+  const size_t Mz = (size_t)m->M;
   for (int mu = 0; mu < m->ga; mu++) {
+    if (d_stream) {
+      gather_batch(c, d_stream, m->cfg.token_dtype == GPT_TOK_U16, len, seed, step, mu, m->B, m->T, m->V,
+                   m->idx_all + mu * Mz, m->tgt_all + mu * Mz, dev_params ? m->step_dev : nullptr);
+    } else {
+      check_tokens(c, m->stage_idx + mu * Mz, m->stage_tgt + mu * Mz, m->M, m->V, m->idx_all + mu * Mz,
+                   m->tgt_all + mu * Mz);
+    }
+  }
+  embed_sort(c, m->idx_all, m->M, m->stok_all, m->spos_all, m->nuniq_all, m->ga);
+  gpt_status s = GPT_OK;
+  m->presorted = true;
+  for (int mu = 0; mu < m->ga && s == GPT_OK; mu++) {
     m->drop_counter = (int64_t)step * m->ga + mu;
     m->cur_micro = mu;
     m->n_micro = m->ga;
-    if (d_stream) {
-      gather_batch(c, d_stream, m->cfg.token_dtype == GPT_TOK_U16, len, seed, step, mu, m->B, m->T, m->V, m->idx,
-                   m->tgt, dev_params ? m->step_dev : nullptr);
-    } else {
-      int32_t* si = m->stage_idx + (size_t)mu * m->M;
-      int32_t* stg = m->stage_tgt + (size_t)mu * m->M;
-      check_tokens(c, si, stg, m->M, m->V, m->idx, m->tgt);
-    }
-    gpt_status s = forward_any(m, true, m->scal + 1, 1.0f / (float)(m->M * m->ga), mu > 0);
-    if (s != GPT_OK) return s;
-    s = backward_any(m);
-    if (s != GPT_OK) return s;
+    m->idx = m->idx_all + mu * Mz;
+    m->tgt = m->tgt_all + mu * Mz;
+    s = forward_any(m, true, m->scal + 1, 1.0f / (float)(m->M * m->ga), mu > 0);
+    if (s == GPT_OK) s = backward_any(m);
   }
+  m->presorted = false;
+  m->idx = m->idx0;
+  m->tgt = m->tgt0;
+  if (s != GPT_OK) return s;
   m->have_forward = false;
   return adamw_step(m, lr, step, dev_params);
 }

@@ -693,6 +693,11 @@ __global__ void k_embed_sort(const int32_t* __restrict__ idx, int M, int P2, int
                              int32_t* __restrict__ spos, int32_t* __restrict__ n_unique) {
   extern __shared__ uint32_t key[];
   __shared__ int cnt[32];
+  // block b sorts the b-th batch of M tokens (batches stored back to back)
+  idx += (long)blockIdx.x * M;
+  stok += (long)blockIdx.x * M;
+  spos += (long)blockIdx.x * M;
+  n_unique += blockIdx.x;
   for (int i = threadIdx.x; i < P2; i += blockDim.x)
     key[i] = i < M ? (((uint32_t)idx[i] << 16) | (uint32_t)i) : 0xFFFFFFFFu;
   __syncthreads();
@@ -729,7 +734,8 @@ __global__ void k_embed_sort(const int32_t* __restrict__ idx, int M, int P2, int
   }
 }
 
-void embed_sort(Ctx& c, const int32_t* idx, long M, int32_t* sorted_tok, int32_t* sorted_pos, int32_t* n_unique) {
+void embed_sort(Ctx& c, const int32_t* idx, long M, int32_t* sorted_tok, int32_t* sorted_pos, int32_t* n_unique,
+                int batches) {
   int P2 = 1;
   while (P2 < M) P2 <<= 1;
   size_t smem = (size_t)P2 * 4;
@@ -739,7 +745,7 @@ void embed_sort(Ctx& c, const int32_t* idx, long M, int32_t* sorted_tok, int32_t
     attr_set = true;
   }
   LaunchScope s(c, "embed_sort");
-  k_embed_sort<<<1, 1024, smem, c.stream>>>(idx, (int)M, P2, sorted_tok, sorted_pos, n_unique);
+  k_embed_sort<<<batches, 1024, smem, c.stream>>>(idx, (int)M, P2, sorted_tok, sorted_pos, n_unique);
 }
 
 // dwte[v] += sum over the sorted positions of token v (in position order) of
@@ -786,10 +792,16 @@ __global__ void __launch_bounds__(256) k_embed_seg_a(const float* __restrict__ d
   }
   __syncthreads();
   for (int col = threadIdx.x; col < d; col += blockDim.x) {
+    // the chunk's rows of this column, all loads issued before the sums
+    float vals[EC];
+#pragma unroll
+    for (int k = 0; k < EC; k++) vals[k] = k < n ? dres[(long)s_pos[k] * d + col] : 0.f;
     float acc = 0.f;
-    for (int k = 0; k < n; k++) {
+#pragma unroll
+    for (int k = 0; k < EC; k++) {
+      if (k >= n) break;
       const long p = s_pos[k];
-      float v = dres[p * d + col];
+      float v = vals[k];
       if (drop.active) v *= drop_mul(drop, (uint64_t)p * d + col);
       acc += v;
       const int tok = s_tok[k + 1];

@@ -164,7 +164,9 @@ void ce_fwd_bwd(Ctx& c, T* logits, const int32_t* tgt, long M, int V, int Vp, fl
 void loss_reduce(Ctx& c, const float* row_loss, long M, float scale, float* loss_acc, int accumulate);
 
 // embedding backward: routing (stable sort of positions by token) + sums
-void embed_sort(Ctx& c, const int32_t* idx, long M, int32_t* sorted_tok, int32_t* sorted_pos, int32_t* n_unique);
+// `batches` independent sorts of M tokens each, stored back to back (one CTA each)
+void embed_sort(Ctx& c, const int32_t* idx, long M, int32_t* sorted_tok, int32_t* sorted_pos, int32_t* n_unique,
+                int batches = 1);
 // seg_scratch: 2 * ceil(M / 32) * d floats (partial sums of segments that cross 32-slot chunks)
 void embed_bwd(Ctx& c, const float* dres, const int32_t* sorted_tok, const int32_t* sorted_pos, long M, int Tn,
                int Bn, int d, DropKey drop, float* dwte, float* dwpe, float* seg_scratch);
