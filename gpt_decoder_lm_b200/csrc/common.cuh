@@ -62,6 +62,15 @@ template <typename T> GPT_HD T from_f(float v);
 template <> GPT_HD float from_f<float>(float v) { return v; }
 template <> GPT_HD bf16 from_f<bf16>(float v) { return __float2bfloat16_rn(v); }
 
+// Programmatic dependent launch: a kernel lets the next kernel of the stream
+// begin launching once all of its own blocks have started (the next kernel's
+// blocks then fill SMs as this kernel's last wave drains); a kernel launched
+// with the programmatic-serialization attribute waits in pdl_wait() until its
+// predecessor has completed and its writes are visible, and touches no global
+// memory before that.  Both are no-ops without such a launch.
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // flags (device word in the workspace)
 enum : uint32_t { FLAG_TOKEN = 1u, FLAG_LOSS = 2u, FLAG_NORM = 4u, FLAG_TIMEOUT = 8u };
 

@@ -38,6 +38,7 @@ __device__ __forceinline__ void load_tile(float (*dst)[HD + 1], const T* qkv, in
 
 template <typename T, int HD>
 __global__ void __launch_bounds__(256) k_attn_fwd(AttnDesc a) {
+  pdl_trigger();
   constexpr int DPT = HD / 4;
   extern __shared__ float smem_f[];
   float(*Ks)[HD + 1] = reinterpret_cast<float(*)[HD + 1]>(smem_f);
@@ -102,6 +103,7 @@ __global__ void __launch_bounds__(256) k_attn_fwd(AttnDesc a) {
 // D[b,h,i] = sum_d dO[b,i,h,d] * O[b,i,h,d]
 template <typename T, int HD>
 __global__ void k_attn_dsum(AttnDesc a) {
+  pdl_trigger();
   long i = (long)blockIdx.x * blockDim.x + threadIdx.x;
   long n = (long)a.B * a.H * a.T;
   if (i >= n) return;
@@ -128,6 +130,7 @@ __device__ __forceinline__ void load_do_tile(float (*dst)[HD + 1], const T* dout
 // dK, dV: each 4-thread group owns one key j and walks the queries i >= j.
 template <typename T, int HD>
 __global__ void __launch_bounds__(256) k_attn_bwd_kv(AttnDesc a) {
+  pdl_trigger();
   constexpr int DPT = HD / 4;
   extern __shared__ float smem_f[];
   float(*Qs)[HD + 1] = reinterpret_cast<float(*)[HD + 1]>(smem_f);
@@ -194,6 +197,7 @@ __global__ void __launch_bounds__(256) k_attn_bwd_kv(AttnDesc a) {
 // dQ: each 4-thread group owns one query i and walks the keys j <= i.
 template <typename T, int HD>
 __global__ void __launch_bounds__(256) k_attn_bwd_q(AttnDesc a) {
+  pdl_trigger();
   constexpr int DPT = HD / 4;
   extern __shared__ float smem_f[];
   float(*Ks)[HD + 1] = reinterpret_cast<float(*)[HD + 1]>(smem_f);

@@ -92,6 +92,7 @@ constexpr float RESCALE_LOG2 = 8.0f;
 template <bool DROP>
 __global__ void __launch_bounds__(192, 2) k_attn_fwd_o(const __grid_constant__ CUtensorMap tq,
                                                        const __grid_constant__ CUtensorMap tkv64, AttnTcArgs a) {
+  pdl_trigger();
   extern __shared__ __align__(1024) uint8_t smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (smem_u32(smem) & 1023) {  // swizzled tiles need 1024-byte alignment
@@ -343,6 +344,7 @@ template <bool DROP>
 __global__ void __launch_bounds__(320, 2) k_attn_bwd_kv8(const __grid_constant__ CUtensorMap tkv,
                                                          const __grid_constant__ CUtensorMap tq64,
                                                          const __grid_constant__ CUtensorMap tdo64, AttnTcArgs a) {
+  pdl_trigger();
   extern __shared__ __align__(1024) uint8_t smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (smem_u32(smem) & 1023) {
@@ -572,6 +574,7 @@ template <bool DROP>
 __global__ void __launch_bounds__(320, 2) k_attn_bwd_q8(const __grid_constant__ CUtensorMap tq,
                                                         const __grid_constant__ CUtensorMap tdo,
                                                         const __grid_constant__ CUtensorMap tkv64, AttnTcArgs a) {
+  pdl_trigger();
   extern __shared__ __align__(1024) uint8_t smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (smem_u32(smem) & 1023) {
@@ -756,6 +759,7 @@ __global__ void __launch_bounds__(320, 2) k_attn_bwd_q8(const __grid_constant__ 
 // elements (16 bytes) per lane, so a warp covers four heads
 __global__ void k_attn_dsum64(const bf16* __restrict__ o, const bf16* __restrict__ dout, int B, int T, int H,
                               float* __restrict__ dsum) {
+  pdl_trigger();
   const long g = ((long)blockIdx.x * blockDim.x + threadIdx.x) >> 3;  // (row, head) index
   const int sub = threadIdx.x & 7;
   const bool valid = g < (long)B * T * H;

@@ -8,6 +8,7 @@ namespace gpt {
 
 template <typename T>
 __global__ void __launch_bounds__(256) k_gemm_simt(GemmDesc g) {
+  pdl_trigger();
   __shared__ float As[16][64 + 4];
   __shared__ float Bs[16][64 + 4];
   const T* A = reinterpret_cast<const T*>(g.A);
@@ -84,6 +85,7 @@ void gemm_simt_bf16(Ctx& c, const GemmDesc& g) {
 }
 
 __global__ void k_splitk_reduce(const float* __restrict__ part, int splits, long MN, float* __restrict__ out) {
+  pdl_trigger();
   long i = (long)blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= MN) return;
   float s = 0.f;
@@ -94,6 +96,7 @@ __global__ void k_splitk_reduce(const float* __restrict__ part, int splits, long
 // the same sums, four adjacent elements per thread with 16-byte accesses; the
 // partial loads of up to 8 splits are issued before any add (same add order)
 __global__ void k_splitk_reduce4(const float4* __restrict__ part, int splits, long MN4, float4* __restrict__ out) {
+  pdl_trigger();
   long i = (long)blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= MN4) return;
   float4 s = make_float4(0.f, 0.f, 0.f, 0.f);

@@ -144,6 +144,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               const __grid_constant__ CUtensorMap tm_out, const __grid_constant__ CUtensorMap tm_out2,
               const __grid_constant__ CUtensorMap tm_in, TcArgs p) {
   using C = TcCfg<BN>;
+  pdl_trigger();
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);
@@ -181,6 +182,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  // the set-up above overlaps the previous kernel's tail; its outputs (our
+  // operands, epilogue inputs, the buffers we write) are ready from here on
+  pdl_wait();
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
@@ -533,7 +537,20 @@ bool launch(Ctx& c, const GemmDesc& g, int splits) {
     attr = true;
   }
   LaunchScope s(c, g.name ? g.name : "gemm_tc");
-  k_gemm_tc<BN, A_MN, B_MN><<<grid, kThreads, Cf::SMEM_BYTES, c.stream>>>(ma, mb, mo, mo2, mi, a);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = Cf::SMEM_BYTES;
+  cfg.stream = c.stream;
+  cudaLaunchAttribute pdl[1];
+  pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  pdl[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = pdl;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, k_gemm_tc<BN, A_MN, B_MN>, ma, mb, mo, mo2, mi, a) != cudaSuccess) {
+    cudaGetLastError();  // programmatic serialization refused: an ordinary launch
+    k_gemm_tc<BN, A_MN, B_MN><<<grid, kThreads, Cf::SMEM_BYTES, c.stream>>>(ma, mb, mo, mo2, mi, a);
+  }
   return true;
 }
 

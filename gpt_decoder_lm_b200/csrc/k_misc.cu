@@ -14,6 +14,7 @@ namespace gpt {
 __global__ void k_gather(const void* __restrict__ stream, int tok_u16, uint64_t len, uint64_t seed, int step,
                          const int* step_dev, int micro, int B, int T, int V, int32_t* __restrict__ idx,
                          int32_t* __restrict__ tgt, uint32_t* flags) {
+  pdl_trigger();
   long i = (long)blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= (long)B * T) return;
   if (step_dev) step = *step_dev;  // step index held in device memory (replayed graphs)
@@ -49,6 +50,7 @@ void gather_batch(Ctx& c, const void* stream, int tok_u16, uint64_t len, uint64_
 
 // writes the per-step scalars read by replayed graphs: step, lr, 1 - b1^t, 1 - b2^t
 __global__ void k_set_step(int* step_dev, float* hyper, int step, float lr, float bc1, float bc2) {
+  pdl_trigger();
   *step_dev = step;
   hyper[0] = lr;
   hyper[1] = bc1;
@@ -62,6 +64,7 @@ void set_step_params(Ctx& c, int* step_dev, float* hyper, int step, float lr, fl
 
 __global__ void k_check_tokens(const int32_t* __restrict__ idx, const int32_t* __restrict__ tgt, long n, int V,
                                int32_t* __restrict__ io, int32_t* __restrict__ to, uint32_t* flags) {
+  pdl_trigger();
   long i = (long)blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= n) return;
   int x = idx[i], y = tgt[i];
@@ -86,6 +89,7 @@ void check_tokens(Ctx& c, const int32_t* idx, const int32_t* tgt, long n, int V,
 __global__ void k_embed_fwd(const int32_t* __restrict__ idx, const float* __restrict__ wte,
                             const float* __restrict__ wpe, float* __restrict__ res, int T, int d, long n4,
                             DropKey drop) {
+  pdl_trigger();
   long i = (long)blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= n4) return;
   int d4 = d >> 2;
@@ -136,6 +140,7 @@ template <typename T, int VPL>
 __global__ void k_norm_fwd(const float* __restrict__ x, const float* __restrict__ w, const float* __restrict__ b,
                            T* __restrict__ y, float* __restrict__ mean_out, float* __restrict__ rstd_out, long rows,
                            int d, int rms, float eps) {
+  pdl_trigger();
   // two rows per warp, both loaded up front: the whole launch is resident in
   // one wave and every warp has 2 x d x 4 bytes in flight
   const long row0 = ((long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5)) * 2;
@@ -238,6 +243,7 @@ template void norm_fwd<bf16>(Ctx&, const float*, const float*, const float*, bf1
 // ============================================================================
 template <typename T>
 __global__ void k_norm_bwd(NormBwd p) {
+  pdl_trigger();
   extern __shared__ float red[];  // [2 buffers][warps][4]
   int tid = threadIdx.x;
   int d4 = p.d >> 2;
@@ -386,6 +392,7 @@ struct Dst3 {
 };
 __global__ void __launch_bounds__(1024) k_rows_reduce(const float* __restrict__ src, long stride, long slot_off,
                                                       int rows, int n, Dst3 dsts) {
+  pdl_trigger();
   __shared__ float sh[32][33];
   float* dst = dsts.p[blockIdx.y];
   if (!dst) return;  // uniform per block
@@ -422,6 +429,7 @@ void partial_reduce3(Ctx& c, const float* part, int blocks, int d, float* g0, fl
 template <typename T>
 __global__ void k_colsum(const T* __restrict__ x, long rows, int N, int chunks, float* __restrict__ part,
                          int accumulate) {
+  pdl_trigger();
   int j = blockIdx.x * blockDim.x + threadIdx.x;
   if (j >= N) return;
   long per = (rows + chunks - 1) / chunks;
@@ -444,6 +452,7 @@ void colsum_reduce(Ctx& c, const float* part, int chunks, int N, float* grad) {
 // row chunk with 16-byte loads
 __global__ void k_colsum_bf16x8(const bf16* __restrict__ x, long rows, int N, int chunks, float* __restrict__ part,
                                 int accumulate) {
+  pdl_trigger();
   const int j8 = blockIdx.x * blockDim.x + threadIdx.x;
   if (j8 * 8 >= N) return;
   const long per = (rows + chunks - 1) / chunks;
@@ -516,6 +525,7 @@ template void colsum_acc<bf16>(Ctx&, const bf16*, long, int, float*, float*);
 template <typename T>
 __global__ void k_ce(T* __restrict__ logits, const int32_t* __restrict__ tgt, int V, int Vp,
                      float* __restrict__ lse_out, float* __restrict__ row_loss, int want_grad, float scale) {
+  pdl_trigger();
   __shared__ float sm[32], ss[32];
   long row = blockIdx.x;
   T* z = logits + row * Vp;
@@ -583,6 +593,7 @@ template <typename T>
 __global__ void __launch_bounds__(256, 4) k_ce_stream(T* __restrict__ logits, const int32_t* __restrict__ tgt, int V,
                                                       int Vp, float* __restrict__ lse_out,
                                                       float* __restrict__ row_loss, int want_grad, float scale) {
+  pdl_trigger();
   constexpr int EPV = 16 / sizeof(T);
   constexpr float LOG2E = 1.4426950408889634f;
   __shared__ float sm[8], ss[8];
@@ -665,6 +676,7 @@ template void ce_fwd_bwd<bf16>(Ctx&, bf16*, const int32_t*, long, int, int, floa
 // loss_acc[0] (+)= scale * sum(row_loss); fixed-order double reduction.
 __global__ void k_loss_reduce(const float* __restrict__ rl, long M, float scale, float* acc, int accumulate,
                               uint32_t* flags) {
+  pdl_trigger();
   __shared__ double sh[32];
   double s = 0.0;
   for (long i = threadIdx.x; i < M; i += blockDim.x) s += (double)rl[i];
@@ -691,6 +703,7 @@ void loss_reduce(Ctx& c, const float* row_loss, long M, float scale, float* loss
 // ============================================================================
 __global__ void k_embed_sort(const int32_t* __restrict__ idx, int M, int P2, int32_t* __restrict__ stok,
                              int32_t* __restrict__ spos, int32_t* __restrict__ n_unique) {
+  pdl_trigger();
   extern __shared__ uint32_t key[];
   __shared__ int cnt[32];
   // block b sorts the b-th batch of M tokens (batches stored back to back)
@@ -754,6 +767,7 @@ void embed_sort(Ctx& c, const int32_t* idx, long M, int32_t* sorted_tok, int32_t
 // dwpe[t] += sum_b drop0(dres[b, t]) (b ascending)
 __global__ void k_embed_bwd_wpe(const float* __restrict__ dres, int Bn, int Tn, int d, DropKey drop,
                                 float* __restrict__ dwpe) {
+  pdl_trigger();
   long i = (long)blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= (long)Tn * d) return;
   int t = (int)(i / d), c = (int)(i % d);
@@ -778,6 +792,7 @@ __global__ void __launch_bounds__(256) k_embed_seg_a(const float* __restrict__ d
                                                      const int32_t* __restrict__ spos, int M, int d, DropKey drop,
                                                      float* __restrict__ dwte, float* __restrict__ head,
                                                      float* __restrict__ tail) {
+  pdl_trigger();
   __shared__ int s_tok[EC + 2], s_pos[EC];
   const int c = blockIdx.x;
   const int j0 = c * EC, j1 = min(M, j0 + EC);
@@ -821,6 +836,7 @@ __global__ void __launch_bounds__(256) k_embed_seg_a(const float* __restrict__ d
 
 __global__ void k_embed_seg_b(const int32_t* __restrict__ stok, int M, int d, const float* __restrict__ head,
                               const float* __restrict__ tail, float* __restrict__ dwte) {
+  pdl_trigger();
   const int c = blockIdx.x;
   const int j0 = c * EC, j1 = min(M, j0 + EC);
   const int tok = stok[j1 - 1];
@@ -862,6 +878,7 @@ void embed_bwd(Ctx& c, const float* dres, const int32_t* sorted_tok, const int32
 int sumsq_blocks(Ctx& c) { return c.num_sms * 4 < 592 ? c.num_sms * 4 : 592; }  // partial buffer holds 592
 
 __global__ void k_sumsq(const float* __restrict__ g, long n4, double* __restrict__ part) {
+  pdl_trigger();
   __shared__ double sh[32];
   double s = 0.0;
   for (long i = (long)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += (long)gridDim.x * blockDim.x) {
@@ -892,6 +909,7 @@ void sumsq_partials(Ctx& c, const float* g, long n, double* partials, int blocks
 // A non-finite norm skips the update (gradients are still zeroed).
 // ============================================================================
 __global__ void k_adamw(AdamArgs a, uint32_t* flags) {
+  pdl_trigger();
   __shared__ float s_coef;
   __shared__ int s_ok;
   if (threadIdx.x < 32) {
@@ -977,6 +995,7 @@ void adamw(Ctx& c, const AdamArgs& a) {
 }
 
 __global__ void k_to_bf16(const float* __restrict__ s, bf16* __restrict__ d, long n) {
+  pdl_trigger();
   long i = (long)blockIdx.x * blockDim.x + threadIdx.x;
   if (i < n) d[i] = __float2bfloat16_rn(s[i]);
 }
@@ -988,6 +1007,7 @@ void to_bf16(Ctx& c, const float* src, bf16* dst, long n) {
 
 // row argmax, ties to the lowest index
 __global__ void k_argmax(const void* __restrict__ x, int is_bf16, int cols, int ld, int32_t* __restrict__ out) {
+  pdl_trigger();
   __shared__ float bv[32];
   __shared__ int bi[32];
   long row = blockIdx.x;
@@ -1029,6 +1049,7 @@ void argmax_rows(Ctx& c, const void* x, int is_bf16, long rows, int cols, int ld
 }
 
 __global__ void k_dropmask(DropKey k, long n, uint8_t* out) {
+  pdl_trigger();
   long i = (long)blockIdx.x * blockDim.x + threadIdx.x;
   if (i < n) out[i] = drop_keep(k, (uint64_t)i) ? 1 : 0;
 }
