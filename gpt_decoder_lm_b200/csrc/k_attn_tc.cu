@@ -38,7 +38,7 @@ struct AttnTcArgs {
   int B, T, H;
   bf16* o_out;
   float* lse;         // [B, H, T] natural log
-  const float* dsum;  // [B, H, T]
+  float* dsum;        // [B, H, T] D = rowsum(dO * O): written by the dQ kernel, read by dK/dV
   bf16* dqkv;
   float scale_log2;   // log2(e) / sqrt(64)
   float scale;        // 1 / sqrt(64)
@@ -564,16 +564,20 @@ __global__ void __launch_bounds__(320, 2) k_attn_bwd_kv8(const __grid_constant__
 // in two phases per block (P from S, then dS from dP); the MMA warp issues
 //   S(j) dP(j) | S read: S(j+1) | dS(j) ready: dQ(j) dP(j+1) | ...
 // so S of the next block is computed while the math warps work on dS.
-// smem: Q | dO | (K, V)[3 stages] | barriers   (~80 KB)
+// The kernel also computes D_i = sum_d dO_id O_id of its rows from the dO and
+// O tiles in shared memory and stores it for the dK/dV kernel, which runs
+// after it.
+// smem: Q | dO | O | (K, V)[3 stages] | barriers   (~96 KB)
 // TMEM: S [0,64), dP [64,128), dQ [128,192)  (256 allocated)
 // ============================================================================
-constexpr int Q_Q = 0, Q_DO = TILE, Q_ST = 2 * TILE, Q_BAR = (2 + BWD_STAGES) * TILE;
+constexpr int Q_Q = 0, Q_DO = TILE, Q_OT = 2 * TILE, Q_ST = 3 * TILE, Q_BAR = (3 + BWD_STAGES) * TILE;
 constexpr int Q_SMEM = Q_BAR + 128;
 
 template <bool DROP>
 __global__ void __launch_bounds__(320, 2) k_attn_bwd_q8(const __grid_constant__ CUtensorMap tq,
                                                         const __grid_constant__ CUtensorMap tdo,
-                                                        const __grid_constant__ CUtensorMap tkv64, AttnTcArgs a) {
+                                                        const __grid_constant__ CUtensorMap tkv64,
+                                                        const __grid_constant__ CUtensorMap tout, AttnTcArgs a) {
   pdl_trigger();
   extern __shared__ __align__(1024) uint8_t smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -612,6 +616,7 @@ __global__ void __launch_bounds__(320, 2) k_attn_bwd_q8(const __grid_constant__ 
     prefetch_tmap(&tq);
     prefetch_tmap(&tdo);
     prefetch_tmap(&tkv64);
+    prefetch_tmap(&tout);
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(tslot), 256);
@@ -624,9 +629,10 @@ __global__ void __launch_bounds__(320, 2) k_attn_bwd_q8(const __grid_constant__ 
 
   if (warp == 0) {
     if (lane == 0) {
-      mbar_expect_tx(qd_full, 2 * TILE);
+      mbar_expect_tx(qd_full, 3 * TILE);
       tma_load_3d(sb + Q_Q, &tq, qd_full, 0, h, row0 + qb * 128);
       tma_load_3d(sb + Q_DO, &tdo, qd_full, 0, h, row0 + qb * 128);
+      tma_load_3d(sb + Q_OT, &tout, qd_full, 0, h, row0 + qb * 128);
       for (int j = 0; j < nkb; j++) {
         const int s = j % BWD_STAGES;
         const uint32_t fb = kv_full0 + 8 * s;
@@ -678,11 +684,28 @@ __global__ void __launch_bounds__(320, 2) k_attn_bwd_q8(const __grid_constant__ 
     const int qi = qb * 128 + r;
     const uint32_t trow = tmem + ((uint32_t)(quad * 32) << 16);
     const float lse2 = a.lse[(size_t)bh * a.T + qi] * LOG2E;
-    const float Di = a.dsum[(size_t)bh * a.T + qi];
+    // D of this row from the dO and O tiles (128-byte rows, 128-byte swizzle:
+    // 16-byte chunk q of row r at q ^ (r & 7)); both halves compute it
+    bool ok = mbar_wait(qd_full, 0, abort_flag, a.flags);
+    float Di = 0.f;
+    if (ok) {
+#pragma unroll
+      for (int q = 0; q < 8; q++) {
+        const uint32_t off = r * 128 + ((q ^ (r & 7)) << 4);
+        const uint4 x = ld_shared_v4(sb + Q_DO + off), y = ld_shared_v4(sb + Q_OT + off);
+        const uint32_t xw[4] = {x.x, x.y, x.z, x.w}, yw[4] = {y.x, y.y, y.z, y.w};
+#pragma unroll
+        for (int k = 0; k < 4; k++) {
+          const float2 xf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&xw[k]));
+          const float2 yf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&yw[k]));
+          Di = fmaf(xf.x, yf.x, fmaf(xf.y, yf.y, Di));
+        }
+      }
+      if (half == 0) a.dsum[(size_t)bh * a.T + qi] = Di;
+    }
     const uint64_t sl2x2 = f2(a.scale_log2, a.scale_log2), nlse2 = f2(-lse2, -lse2), Dx2 = f2(Di, Di);
     const uint64_t ebase = ((uint64_t)bh * a.T + qi) * a.T;
-    bool ok = true;
-    for (int j = 0; j < nkb; j++) {
+    for (int j = 0; j < nkb && ok; j++) {
       if (!(ok = mbar_wait(s_full, j & 1, abort_flag, a.flags))) break;
       tc_fence_after();
       const int key0 = j * 64;
@@ -753,37 +776,6 @@ __global__ void __launch_bounds__(320, 2) k_attn_bwd_q8(const __grid_constant__ 
   __syncthreads();
   tc_fence_after();
   if (warp == 1) tmem_dealloc(tmem, 256);
-}
-
-// D[b,h,i] = sum_d dO[b,i,h,d] * O[b,i,h,d]: 8 lanes per (row, head), 8
-// elements (16 bytes) per lane, so a warp covers four heads
-__global__ void k_attn_dsum64(const bf16* __restrict__ o, const bf16* __restrict__ dout, int B, int T, int H,
-                              float* __restrict__ dsum) {
-  pdl_trigger();
-  const long g = ((long)blockIdx.x * blockDim.x + threadIdx.x) >> 3;  // (row, head) index
-  const int sub = threadIdx.x & 7;
-  const bool valid = g < (long)B * T * H;
-  float s = 0.f;
-  if (valid) {
-    uint4 a = reinterpret_cast<const uint4*>(o + g * 64)[sub];
-    uint4 d = reinterpret_cast<const uint4*>(dout + g * 64)[sub];
-    const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&a);
-    const __nv_bfloat162* d2 = reinterpret_cast<const __nv_bfloat162*>(&d);
-#pragma unroll
-    for (int k = 0; k < 4; k++) {
-      float2 x = __bfloat1622float2(a2[k]), y = __bfloat1622float2(d2[k]);
-      s = fmaf(x.x, y.x, fmaf(x.y, y.y, s));
-    }
-  }
-  s += __shfl_xor_sync(0xffffffffu, s, 1);
-  s += __shfl_xor_sync(0xffffffffu, s, 2);
-  s += __shfl_xor_sync(0xffffffffu, s, 4);
-  if (valid && sub == 0) {
-    const long row = g / H;  // b*T + t
-    const int h = (int)(g % H);
-    const long b = row / T, t = row % T;
-    dsum[(b * H + h) * T + t] = s;
-  }
 }
 
 // ---------------------------------------------------------------- host side
@@ -860,20 +852,15 @@ void attn_fwd_tc(Ctx& c, const AttnDesc& d) {
 }
 
 void attn_bwd_tc(Ctx& c, const AttnDesc& d) {
-  CUtensorMap tkv, tkv64, tq64, tdo, tdo64;
+  CUtensorMap tkv, tkv64, tq64, tdo, tdo64, tout;
   long rows = (long)d.B * d.T;
   if (!map_rows(&tkv, d.qkv, 3 * d.H, rows, 128) || !map_rows(&tkv64, d.qkv, 3 * d.H, rows, 64) ||
-      !map_rows(&tdo, d.dout, d.H, rows, 128) || !map_rows(&tdo64, d.dout, d.H, rows, 64)) {
+      !map_rows(&tdo, d.dout, d.H, rows, 128) || !map_rows(&tdo64, d.dout, d.H, rows, 64) ||
+      !map_rows(&tout, d.o, d.H, rows, 128)) {
     attn_bwd_simt<bf16>(c, d);
     return;
   }
   tq64 = tkv64;
-  {
-    long groups = (long)d.B * d.T * d.H;  // 8 threads each
-    LaunchScope s(c, "attn_bwd_dsum");
-    k_attn_dsum64<<<(unsigned)((groups * 8 + 255) / 256), 256, 0, c.stream>>>(
-        reinterpret_cast<const bf16*>(d.o), reinterpret_cast<const bf16*>(d.dout), d.B, d.T, d.H, d.dsum);
-  }
   static bool attr = false;
   if (!attr) {
     cudaFuncSetAttribute(k_attn_bwd_kv8<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, K_SMEM);
@@ -885,15 +872,15 @@ void attn_bwd_tc(Ctx& c, const AttnDesc& d) {
   AttnTcArgs a = make_args(d, c.flags);
   dim3 grid(d.B * d.H, d.T / 128);
   const bool drop = d.drop.active;
+  {  // dQ first: it also stores D = rowsum(dO * O), which the dK/dV kernel reads
+    LaunchScope s(c, "attn_bwd_q_tc");
+    if (drop) k_attn_bwd_q8<true><<<grid, 320, Q_SMEM, c.stream>>>(tkv, tdo, tkv64, tout, a);
+    else k_attn_bwd_q8<false><<<grid, 320, Q_SMEM, c.stream>>>(tkv, tdo, tkv64, tout, a);
+  }
   {
     LaunchScope s(c, "attn_bwd_kv_tc");
     if (drop) k_attn_bwd_kv8<true><<<grid, 320, K_SMEM, c.stream>>>(tkv, tq64, tdo64, a);
     else k_attn_bwd_kv8<false><<<grid, 320, K_SMEM, c.stream>>>(tkv, tq64, tdo64, a);
-  }
-  {
-    LaunchScope s(c, "attn_bwd_q_tc");
-    if (drop) k_attn_bwd_q8<true><<<grid, 320, Q_SMEM, c.stream>>>(tkv, tdo, tkv64, a);
-    else k_attn_bwd_q8<false><<<grid, 320, Q_SMEM, c.stream>>>(tkv, tdo, tkv64, a);
   }
 }
 
