@@ -72,9 +72,9 @@ def attn_flops_per_step(w) -> float:
 
 
 # dram__bytes_read.sum + dram__bytes_write.sum of k_gemm_tc per launch, averaged over the
-# launches of one training step in profiles/launch_list_gpt2_124m_train_step.md; None while the
-# kernel has changed since that capture
-GEMM_DRAM_BYTES_PER_LAUNCH = None
+# launches of one training step in profiles/launch_list_gpt2_124m_train_step.md (81.2 GB
+# over 735 launches); None while the kernel has changed since that capture
+GEMM_DRAM_BYTES_PER_LAUNCH = 8.116e+10 / 735
 
 
 class Clocks:
