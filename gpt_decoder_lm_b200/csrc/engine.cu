@@ -118,7 +118,7 @@ struct gpt_model {
   float *row_loss, *row_lse;
   int32_t *idx, *tgt, *stage_idx, *stage_tgt;
   // backward scratch
-  float *dres, *dln, *dsum, *part, *colsum_scr, *splitk, *seg;
+  float *dres, *dln, *dsum, *splitk, *seg;
   uint8_t *dyb, *dqkv, *datt, *dh;
   int32_t *stok, *spos, *nuniq;
   double* norm_part;
@@ -365,8 +365,6 @@ size_t carve(gpt_model& m, uint8_t* base) {
   m.dsum = F((size_t)M * m.H);
   m.part_blocks = (int)std::min<long>(M, 148 * 8);  // capacity; the launch count is set at create
   m.part_cap = m.part_blocks;
-  m.part = F((size_t)m.part_blocks * 3 * d);
-  m.colsum_scr = F((size_t)512 * 4 * d);
   m.norm_parts = F((size_t)(2 * L + 1) * m.part_cap * 3 * d);
   m.colsum_parts = F((size_t)L * 2 * colsum_chunks(M) * 4 * d);
   {

@@ -508,13 +508,6 @@ void colsum_partial(Ctx& c, const T* x, long rows, int N, float* part, bool accu
 template void colsum_partial<float>(Ctx&, const float*, long, int, float*, bool);
 template void colsum_partial<bf16>(Ctx&, const bf16*, long, int, float*, bool);
 
-template <typename T>
-void colsum_acc(Ctx& c, const T* x, long rows, int N, float* scratch, float* grad) {
-  colsum_partial<T>(c, x, rows, N, scratch, false);
-  colsum_reduce(c, scratch, colsum_chunks(rows), N, grad);
-}
-template void colsum_acc<float>(Ctx&, const float*, long, int, float*, float*);
-template void colsum_acc<bf16>(Ctx&, const bf16*, long, int, float*, float*);
 
 // ============================================================================
 // cross-entropy (microGPT "核心训练循环": loss = -log softmax(z)[target],

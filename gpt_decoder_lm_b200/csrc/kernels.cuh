@@ -148,10 +148,9 @@ int norm_bwd_blocks(Ctx& c, long rows, int d, bool bf16_out);
 // the three slots of part[blocks, 3, d] into g0, g1, g2 (each nullable), one launch
 void partial_reduce3(Ctx& c, const float* part, int blocks, int d, float* g0, float* g1, float* g2);
 
-// column sums of an operand-typed [rows, N] matrix into grad (+=), deterministic
-template <typename T> void colsum_acc(Ctx& c, const T* x, long rows, int N, float* scratch, float* grad);
-// the chunk partials of those sums, part[colsum_chunks(rows), N] (= or += with accumulate);
-// colsum_reduce then adds them to grad
+// column sums of an operand-typed [rows, N] matrix, deterministic: chunk
+// partials part[colsum_chunks(rows), N] (= or += with accumulate), which
+// colsum_reduce adds to grad
 int colsum_chunks(long rows);
 template <typename T> void colsum_partial(Ctx& c, const T* x, long rows, int N, float* part, bool accumulate);
 
@@ -170,7 +169,7 @@ void embed_sort(Ctx& c, const int32_t* idx, long M, int32_t* sorted_tok, int32_t
 // seg_scratch: 2 * ceil(M / 32) * d floats (partial sums of segments that cross 32-slot chunks)
 void embed_bwd(Ctx& c, const float* dres, const int32_t* sorted_tok, const int32_t* sorted_pos, long M, int Tn,
                int Bn, int d, DropKey drop, float* dwte, float* dwpe, float* seg_scratch);
-// column partials of colsum_acc [chunks, N] -> grad (+=), fixed order
+// column partials [chunks, N] -> grad (+=), fixed order
 void colsum_reduce(Ctx& c, const float* part, int chunks, int N, float* grad);
 
 // grad norm partials, clip + AdamW
