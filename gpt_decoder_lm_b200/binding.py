@@ -65,6 +65,8 @@ _PROTOS = {
     "gpt_gather_batch": (I32, [P, P, U64, U64, I32, I32, P, P]),
     "gpt_set_dropout_cursor": (I32, [P, I32, I32]),
     "gpt_set_graphs": (I32, [P, I32]),
+    "gpt_eval_loss": (I32, [P, P, U64, U64, I32, P]),
+    "gpt_sample": (I32, [P, I32, I32, I32, I64, F32, I32, F32, P, P, P]),
     "gpt_num_tensors": (I32, [P, P]),
     "gpt_tensor_info": (I32, [P, I32, P, P]),
     "gpt_get_tensor": (I32, [P, I32, I32, P]),
@@ -230,6 +232,13 @@ class Model:
     def set_dropout_cursor(self, step: int, micro: int):
         _check(lib().gpt_set_dropout_cursor(self.h, step, micro), self.h, "set_dropout_cursor")
 
+    def eval_loss(self, stream_tokens, data_seed: int, n_batches: int) -> float:
+        """Mean loss of n_batches evaluation batches (forward only, no dropout)."""
+        out = C.c_float()
+        _check(lib().gpt_eval_loss(self.h, _ptr(stream_tokens), stream_tokens.numel(), data_seed, n_batches,
+                                   C.byref(out)), self.h, "eval_loss")
+        return float(out.value)
+
     def set_graphs(self, on: bool):
         """CUDA-graph replay of train_step / train_step_host (default on)."""
         _check(lib().gpt_set_graphs(self.h, 1 if on else 0), self.h, "set_graphs")
@@ -327,6 +336,16 @@ class Model:
 
     def launch_count(self) -> int:
         return int(lib().gpt_launch_count(self.h))
+
+
+def sample(logits, temperature: float, top_k: int, top_p: float, uniform, out, V=None, stream=None):
+    """One draw per row of a device logits tensor [rows, ld] (bf16 or fp32);
+    uniform: device fp32 [rows]; out: device int32 [rows]."""
+    import torch
+    rows, ld = logits.shape
+    st = stream if stream is not None else torch.cuda.current_stream().cuda_stream
+    _check(lib().gpt_sample(_ptr(logits), 1 if logits.dtype == torch.bfloat16 else 0, rows, V or ld, ld, temperature,
+                            top_k, top_p, _ptr(uniform), _ptr(out), st), None, "sample")
 
 
 def test_gemm(backend, M, N, K, A, lda, a_kmajor, B, ldb, b_kmajor, epi_kind, act=0, out=None, out2=None, ldo=0,

@@ -1079,6 +1079,41 @@ gpt_status gpt_train_step_host(gpt_model* m, const int32_t* h_idx, const int32_t
   return train_common(m, nullptr, 0, 0, h_idx, h_tgt, lr, step, h_loss, h_grad_norm);
 }
 
+gpt_status gpt_eval_loss(gpt_model* m, const void* d_stream, uint64_t stream_len, uint64_t data_seed,
+                         int32_t n_batches, float* h_loss) {
+  if (!m || !d_stream || !h_loss || n_batches < 1) return fail(m, GPT_ERR_INVALID_ARG, "eval_loss: bad argument");
+  if (stream_len <= (uint64_t)m->T) return fail(m, GPT_ERR_INVALID_ARG, "stream shorter than block_size + 1");
+  Ctx& c = m->ctx;
+  const float saved_drop = m->cfg.dropout;
+  m->cfg.dropout = 0.f;  // evaluation runs without dropout
+  gpt_status s = GPT_OK;
+  for (int i = 0; i < n_batches && s == GPT_OK; i++) {
+    gather_batch(c, d_stream, m->cfg.token_dtype == GPT_TOK_U16, stream_len, data_seed, i + 1, 0, m->B, m->T, m->V,
+                 m->idx, m->tgt);
+    s = forward_any(m, false, m->scal + 5, 1.0f / (float)(m->M * (long)n_batches), i > 0);
+  }
+  m->cfg.dropout = saved_drop;
+  m->have_forward = false;
+  if (s != GPT_OK) return s;
+  float v = 0.f;
+  cudaMemcpyAsync(&v, m->scal + 5, 4, cudaMemcpyDeviceToHost, c.stream);
+  s = sync_and_flags(m, "eval_loss", nullptr);
+  *h_loss = v;
+  return s;
+}
+
+gpt_status gpt_sample(const void* d_logits, int32_t logits_bf16, int32_t rows, int32_t V, int64_t ld,
+                      float temperature, int32_t top_k, float top_p, const float* d_uniform, int32_t* d_out,
+                      void* cuda_stream) {
+  if (!d_logits || !d_uniform || !d_out || rows < 1 || V < 1 || ld < V) return GPT_ERR_INVALID_ARG;
+  Ctx c;
+  c.stream = (cudaStream_t)cuda_stream;
+  // top_p <= 0: the nucleus is the most probable token(s)
+  sample_rows(c, d_logits, logits_bf16 != 0, rows, V, ld, temperature, top_k, top_p > 0.f ? top_p : 1e-30f,
+              d_uniform, d_out);
+  return cudaGetLastError() == cudaSuccess ? GPT_OK : GPT_ERR_CUDA;
+}
+
 gpt_status gpt_gather_batch(gpt_model* m, const void* d_stream, uint64_t stream_len, uint64_t data_seed, int32_t step,
                             int32_t micro, int32_t* d_idx, int32_t* d_tgt) {
   if (!m || !d_stream || !d_idx || !d_tgt) return fail(m, GPT_ERR_INVALID_ARG, "gather_batch: null argument");

@@ -1,0 +1,231 @@
+// Fused softmax-sample of rows of logits: temperature, top-k, top-p
+// (nucleus) and an inverse-CDF draw at a caller-given uniform, one CTA per
+// row, every reduction in a fixed order (deterministic).
+//
+// Pipeline of the microGPT page, section "单 GPU 高效推理：采样 + KV Cache"
+// (logits / temperature -> top-k -> softmax -> top-p -> draw) and nanoGPT's
+// sample.py (README section "采样 / 推理"):
+//   temperature <= 0       greedy: arg-max, lowest index on ties
+//   0 < top_k < V          keep logits >= the k-th largest logit (ties kept)
+//   p_i = exp((z_i - max) / temperature) over the kept tokens
+//   top_p < 1              keep p_i >= tau, tau the largest value with
+//                          sum_{p_j >= tau} p_j >= top_p * sum_j p_j
+//   draw                   the first token (index order) whose running sum
+//                          of kept p exceeds u * (kept mass)
+// The k-th largest logit is found by an MSB-first radix select over an
+// order-preserving integer image of the floats, tau by bisection over the
+// bit pattern of positive floats.
+#include "kernels.cuh"
+
+namespace gpt {
+namespace {
+
+constexpr int ST = 1024;  // threads per row
+
+// order-preserving image of a float as an unsigned integer
+__device__ __forceinline__ uint32_t fkey(float f) {
+  const uint32_t b = __float_as_uint(f);
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+
+// block sum in a fixed order: warp trees in lane order, then the warp sums
+__device__ float block_sum(float v, float* red) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  v = warp_sum(v);
+  __syncthreads();
+  if (lane == 0) red[w] = v;
+  __syncthreads();
+  float t = 0.f;
+  if (w == 0) {
+    t = lane < (int)(blockDim.x >> 5) ? red[lane] : 0.f;
+    t = warp_sum(t);
+    if (lane == 0) red[32] = t;
+  }
+  __syncthreads();
+  return red[32];
+}
+
+template <typename T>
+__global__ void __launch_bounds__(ST) k_sample(const T* __restrict__ logits, long ld, int V, float temperature,
+                                               int top_k, float top_p, const float* __restrict__ uniform,
+                                               int32_t* __restrict__ out) {
+  __shared__ float red[33];
+  __shared__ uint32_t hist[256];
+  __shared__ uint32_t sel[2];
+  __shared__ int pick;
+  const T* z = logits + (long)blockIdx.x * ld;
+  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+
+  // maximum (and its lowest index, for greedy decoding)
+  float best = -INFINITY;
+  int bi = 0x7fffffff;
+  for (int i = tid; i < V; i += ST) {
+    const float v = to_f<T>(z[i]);
+    if (v > best) {  // strided order: the first hit of a thread is its lowest index
+      best = v;
+      bi = i;
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const float ob = __shfl_xor_sync(0xffffffffu, best, o);
+    const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+    if (ob > best || (ob == best && oi < bi)) {
+      best = ob;
+      bi = oi;
+    }
+  }
+  __shared__ float wb[32];
+  __shared__ int wi[32];
+  if (lane == 0) {
+    wb[w] = best;
+    wi[w] = bi;
+  }
+  __syncthreads();
+  if (tid == 0) {
+    float b = wb[0];
+    int ix = wi[0];
+    for (int k = 1; k < ST / 32; k++)
+      if (wb[k] > b || (wb[k] == b && wi[k] < ix)) {
+        b = wb[k];
+        ix = wi[k];
+      }
+    red[0] = b;
+    pick = ix;
+  }
+  __syncthreads();
+  const float zmax = red[0];
+  if (temperature <= 0.f) {
+    if (tid == 0) out[blockIdx.x] = pick;
+    return;
+  }
+  __syncthreads();
+
+  // top-k: the integer image of the k-th largest logit
+  uint32_t thr = 0;
+  if (top_k > 0 && top_k < V) {
+    uint32_t prefix = 0, mask = 0;
+    int need = top_k;
+    for (int shift = 24; shift >= 0; shift -= 8) {
+      for (int b = tid; b < 256; b += ST) hist[b] = 0;
+      __syncthreads();
+      for (int i = tid; i < V; i += ST) {
+        const uint32_t key = fkey(to_f<T>(z[i]));
+        if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
+      }
+      __syncthreads();
+      if (tid == 0) {
+        int cum = 0, b = 255;
+        for (; b > 0; b--) {
+          if (cum + (int)hist[b] >= need) break;
+          cum += (int)hist[b];
+        }
+        sel[0] = prefix | ((uint32_t)b << shift);
+        sel[1] = (uint32_t)(need - cum);
+      }
+      __syncthreads();
+      prefix = sel[0];
+      need = (int)sel[1];
+      mask |= 255u << shift;
+      __syncthreads();
+    }
+    thr = prefix;
+  }
+  const float inv_t = 1.0f / temperature;
+  auto prob = [&](int i) -> float {  // unnormalised, 0 outside the top-k set
+    const float v = to_f<T>(z[i]);
+    return fkey(v) >= thr ? __expf((v - zmax) * inv_t) : 0.f;
+  };
+
+  // top-p: tau by bisection over the bits of a positive float
+  float tau = 0.f;
+  if (top_p < 1.f) {
+    float s = 0.f;
+    for (int i = tid; i < V; i += ST) s += prob(i);
+    const float target = top_p * block_sum(s, red);
+    uint32_t cur = 0;
+    for (int bit = 30; bit >= 0; bit--) {
+      const uint32_t cand = cur | (1u << bit);
+      const float t = __uint_as_float(cand);
+      float m = 0.f;
+      for (int i = tid; i < V; i += ST) {
+        const float p = prob(i);
+        if (p >= t) m += p;
+      }
+      if (block_sum(m, red) >= target) cur = cand;
+    }
+    tau = __uint_as_float(cur);
+  }
+
+  // draw: contiguous segments per thread, a fixed-order scan of the segment sums
+  const int seg = (V + ST - 1) / ST;
+  const int i0 = min(V, tid * seg), i1 = min(V, i0 + seg);
+  float local = 0.f;
+  int last = -1;
+  for (int i = i0; i < i1; i++) {
+    const float p = prob(i);
+    if (p >= tau && p > 0.f) {
+      local += p;
+      last = i;
+    }
+  }
+  // inclusive scan over threads: lanes in order, then warps in order
+  float incl = local;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const float n = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += n;
+  }
+  __shared__ float wsum[32];
+  if (lane == 31) wsum[w] = incl;
+  if (tid == 0) pick = 0x7fffffff;
+  __syncthreads();
+  if (tid == 0) {
+    float run = 0.f;
+    for (int k = 0; k < ST / 32; k++) {
+      const float t = wsum[k];
+      wsum[k] = run;  // exclusive prefix of warp k
+      run += t;
+    }
+    red[1] = run;  // kept mass
+  }
+  __syncthreads();
+  const float excl = wsum[w] + (incl - local);
+  const float target = uniform[blockIdx.x] * red[1];
+  if (excl + local > target && excl <= target) {  // the crossing lies in this segment
+    float run = excl;
+    for (int i = i0; i < i1; i++) {
+      const float p = prob(i);
+      if (p >= tau && p > 0.f) {
+        run += p;
+        if (run > target) {
+          atomicMin(&pick, i);
+          break;
+        }
+      }
+    }
+  }
+  __syncthreads();
+  // rounding can leave the target at or past the total: the last kept token
+  __shared__ int last_kept;
+  if (tid == 0) last_kept = -1;
+  __syncthreads();
+  if (last >= 0) atomicMax(&last_kept, last);
+  __syncthreads();
+  if (tid == 0) out[blockIdx.x] = pick != 0x7fffffff ? pick : last_kept;
+}
+
+}  // namespace
+
+void sample_rows(Ctx& c, const void* logits, bool bf16_logits, int rows, int V, long ld, float temperature, int top_k,
+                 float top_p, const float* uniform, int32_t* out) {
+  LaunchScope s(c, "sample");
+  if (bf16_logits)
+    k_sample<bf16><<<rows, ST, 0, c.stream>>>(reinterpret_cast<const bf16*>(logits), ld, V, temperature, top_k,
+                                             top_p, uniform, out);
+  else
+    k_sample<float><<<rows, ST, 0, c.stream>>>(reinterpret_cast<const float*>(logits), ld, V, temperature, top_k,
+                                              top_p, uniform, out);
+}
+
+}  // namespace gpt

@@ -186,5 +186,8 @@ void adamw(Ctx& c, const AdamArgs& a);
 void to_bf16(Ctx& c, const float* src, bf16* dst, long n);
 void argmax_rows(Ctx& c, const void* x, int is_bf16, long rows, int cols, int ld, int32_t* out);
 void dropout_mask(Ctx& c, DropKey k, long n, uint8_t* out);
+// one draw per row of logits [rows, ld] (temperature, top-k, top-p, uniform[row])
+void sample_rows(Ctx& c, const void* logits, bool bf16_logits, int rows, int V, long ld, float temperature, int top_k,
+                 float top_p, const float* uniform, int32_t* out);
 
 }  // namespace gpt

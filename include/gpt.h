@@ -200,6 +200,33 @@ gpt_status gpt_gather_batch(gpt_model* m, const void* d_stream, uint64_t stream_
  * step*grad_accum + micro. */
 gpt_status gpt_set_dropout_cursor(gpt_model* m, int32_t step, int32_t micro);
 
+/* ---------------------------------------------------------------- evaluation and sampling */
+
+/* Evaluation loss (nanoGPT README, train.py's estimate_loss: the mean loss of
+ * eval_iters batches): the mean over n_batches >= 1 batches of the batch's
+ * mean token loss, forward only, without dropout.  Batch i is the training
+ * gather's window set for step i + 1, micro-batch 0, of d_stream /
+ * data_seed (a validation stream and seed in practice).  Overwrites the
+ * activations (a following gpt_backward is GPT_ERR_STATE); synchronising.
+ * *h_loss receives the mean. */
+gpt_status gpt_eval_loss(gpt_model* m, const void* d_stream, uint64_t stream_len, uint64_t data_seed,
+                         int32_t n_batches, float* h_loss);
+
+/* One draw from each of `rows` rows of logits (microGPT page, section
+ * "单 GPU 高效推理：采样 + KV Cache"; nanoGPT sample.py): d_logits is
+ * [rows, ld] (bf16 when logits_bf16, else fp32; device), V <= ld valid
+ * columns.  temperature <= 0: greedy (arg-max, lowest index on ties).
+ * Otherwise: top_k in (0, V) keeps the logits >= the k-th largest (ties
+ * kept); p = exp((z - max) / temperature) over those; top_p < 1 keeps
+ * p >= tau for the largest tau whose kept mass reaches top_p of the total
+ * (top_p <= 0 keeps the maximum); the token is the first, in index order,
+ * whose running kept mass exceeds d_uniform[row] (in [0, 1), device fp32)
+ * times the kept mass.  d_out: int32 [rows] (device).  Asynchronous on
+ * cuda_stream; GPT_ERR_INVALID_ARG on null pointers, rows < 1 or V < 1. */
+gpt_status gpt_sample(const void* d_logits, int32_t logits_bf16, int32_t rows, int32_t V, int64_t ld,
+                      float temperature, int32_t top_k, float top_p, const float* d_uniform, int32_t* d_out,
+                      void* cuda_stream);
+
 /* ---------------------------------------------------------------- introspection (tests, resume) */
 
 gpt_status gpt_num_tensors(gpt_model* m, int32_t* n);
