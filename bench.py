@@ -207,6 +207,51 @@ def run_reference(args, w, rank):
     print(json.dumps(line), flush=True)
 
 
+def decode_bytes_per_step(w, pos: float) -> float:
+    """Algorithmic HBM bytes of one decoding step over the batch rows: every
+    bf16 weight matrix once (the four per-layer matrices and the tied head)
+    plus the bf16 keys and values of positions 0..pos of every row and layer."""
+    d, L = w.n_embd, w.n_layer
+    vp = ((w.vocab_size + 63) // 64) * 64
+    weights = 2.0 * (L * 12 * d * d + vp * d)
+    kv = 2.0 * 2 * d * (pos + 1) * w.batch_size * L
+    return weights + kv
+
+
+def measure_decode(model, w, stream_host, dev, rank):
+    """Autoregressive sampling through gpt_generate at the workload's batch:
+    a 64-token prompt and 64 new tokens (temperature 0.8, top-k 40, top-p
+    0.95).  The per-token step time is (t(64 new) - t(1 new)) / 63, which
+    removes the prompt's forward pass."""
+    import torch
+    B, T0, n_new = w.batch_size, 64, 64
+    rng = np.random.default_rng(17 + rank)
+    starts = rng.integers(0, len(stream_host) - T0, B)
+    prompt = torch.from_numpy(np.stack([stream_host[s:s + T0] for s in starts]).astype(np.int32)).to(dev)
+    U = torch.from_numpy(rng.random((n_new, B)).astype(np.float32)).to(dev)
+    out = torch.empty((B, T0 + n_new), dtype=torch.int32, device=dev)
+
+    def timed(n):
+        model.generate(prompt, n, 0.8, 40, 0.95, U, out)  # warm-up
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        model.generate(prompt, n, 0.8, 40, 0.95, U, out)
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1)
+
+    t_full, t_one = timed(n_new), timed(1)
+    step_ms = (t_full - t_one) / (n_new - 1)
+    pos = T0 + n_new / 2.0
+    achieved = decode_bytes_per_step(w, pos) / (step_ms / 1000.0) / 1e9
+    hbm = peaks()["hbm_gbs"]
+    return {"tokens_per_s": B * n_new / (t_full / 1000.0), "ms_per_token_step": step_ms, "prefill_ms": t_one,
+            "batch": B, "prompt": T0, "new_tokens": n_new, "sampling": "temperature 0.8, top-k 40, top-p 0.95",
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
+                         "per_step_bytes": decode_bytes_per_step(w, pos),
+                         "note": "one decoding step (weights once + the rows' keys / values) at mean position"}}
+
+
 def run_ours(args, w, rank, world, local_rank):
     import torch
     import torch.distributed as dist
@@ -305,6 +350,8 @@ def run_ours(args, w, rank, world, local_rank):
     e2e_ms = reduce_max(e0.elapsed_time(e1), dev)
     e2e_value = world * args.steps * tok_step / (e2e_ms / 1000.0)
 
+    decode = measure_decode(model, w, stream_host, dev, rank)
+
     pk = peaks()
     gemm_names = [k for k in kt if k.startswith("gemm")]
     gemm_ms = sum(kt[k][0] for k in gemm_names)
@@ -343,6 +390,7 @@ def run_ours(args, w, rank, world, local_rank):
                        "l2": "256 MiB buffer zeroed between timed steps; step working set ~8 GB"},
             "mfu": {"nominal_2250": mfu_nom, "measured_peak": mfu_meas, "flops_per_token": fpt},
             "roofline": roofline,
+            "decode": decode,
             "cpu_baseline": cpu,
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": 2 * ga * B * T * 4,
                     "d2h_bytes_per_step": 16},

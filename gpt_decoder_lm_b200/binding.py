@@ -67,6 +67,7 @@ _PROTOS = {
     "gpt_set_graphs": (I32, [P, I32]),
     "gpt_eval_loss": (I32, [P, P, U64, U64, I32, P]),
     "gpt_sample": (I32, [P, I32, I32, I32, I64, F32, I32, F32, P, P, P]),
+    "gpt_generate": (I32, [P, P, I32, I32, F32, I32, F32, P, P]),
     "gpt_num_tensors": (I32, [P, P]),
     "gpt_tensor_info": (I32, [P, I32, P, P]),
     "gpt_get_tensor": (I32, [P, I32, I32, P]),
@@ -238,6 +239,12 @@ class Model:
         _check(lib().gpt_eval_loss(self.h, _ptr(stream_tokens), stream_tokens.numel(), data_seed, n_batches,
                                    C.byref(out)), self.h, "eval_loss")
         return float(out.value)
+
+    def generate(self, prompt, n_new: int, temperature: float, top_k: int, top_p: float, uniform, out):
+        """prompt: device int32 [batch_size, T0]; uniform: device fp32 [n_new, batch_size];
+        out: device int32 [batch_size, T0 + n_new]."""
+        _check(lib().gpt_generate(self.h, _ptr(prompt), prompt.shape[1], n_new, temperature, top_k, top_p,
+                                  _ptr(uniform), _ptr(out)), self.h, "generate")
 
     def set_graphs(self, on: bool):
         """CUDA-graph replay of train_step / train_step_host (default on)."""

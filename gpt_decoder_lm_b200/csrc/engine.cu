@@ -136,6 +136,10 @@ struct gpt_model {
   int32_t *idx_all = nullptr, *tgt_all = nullptr, *stok_all = nullptr, *spos_all = nullptr, *nuniq_all = nullptr;
   int32_t *idx0 = nullptr, *tgt0 = nullptr;  // the stand-alone forward's buffers
   bool presorted = false;
+  // decoding scratch, [B] rows of one position each
+  int32_t* dec_tok = nullptr;
+  float *dec_res = nullptr, *dec_mean = nullptr, *dec_rstd = nullptr;
+  uint8_t *dec_a = nullptr, *dec_o = nullptr, *dec_dact = nullptr, *dec_g = nullptr, *dec_logits = nullptr;
   int part_cap = 0;                 // partial rows per norm instance
   float* norm_parts = nullptr;      // [2L+1][part_cap][3][d]
   float* colsum_parts = nullptr;    // [L][2][colsum chunks][4d]
@@ -410,6 +414,15 @@ size_t carve(gpt_model& m, uint8_t* base) {
   m.nuniq_all = I((size_t)m.ga + 64);
   m.idx0 = m.idx;
   m.tgt0 = m.tgt;
+  m.dec_tok = I((size_t)m.B + 64);
+  m.dec_res = F((size_t)m.B * d);
+  m.dec_mean = F((size_t)m.B + 64);
+  m.dec_rstd = F((size_t)m.B + 64);
+  m.dec_a = Bt((size_t)m.B * d);
+  m.dec_o = Bt((size_t)m.B * d);
+  m.dec_dact = Bt((size_t)m.B * 4 * d);
+  m.dec_g = Bt((size_t)m.B * 4 * d);
+  m.dec_logits = Bt((size_t)m.B * m.Vp);
   m.norm_part = (double*)(base + lay.take(148 * 4 * 8 + 64));
   m.argmax_out = I(M + 64);
   return lay.off + 1024;
@@ -786,6 +799,75 @@ void bias_corrections(const gpt_model* m, int step, float* bc1, float* bc2) {
 // ============================================================================
 // C ABI
 // ============================================================================
+// One decoding step for every batch row: the token dec_tok[b] at position t
+// goes through the model with the per-layer qkv activations as the key /
+// value cache (this step's K and V are written at position t), leaving the
+// logits of the next token in dec_logits [B, Vp].
+template <typename T>
+gpt_status decode_step_t(gpt_model* m, int t) {
+  Ctx& c = m->ctx;
+  const int B = m->B, d = m->d, L = m->L, Tn = m->T;
+  const bool rms = m->micro;
+  const float eps = 1e-5f;
+  const int act = m->micro ? ACT_RELU : ACT_GELU;
+  const size_t Md = (size_t)m->M * d;
+  T* a = reinterpret_cast<T*>(m->dec_a);
+  T* o = reinterpret_cast<T*>(m->dec_o);
+  embed_fwd<T>(c, m->dec_tok, m->P(m->wte), m->P(m->wpe) + (size_t)t * d, m->dec_res, B, 1, d, DropKey{});
+  for (int l = 0; l < L; l++) {
+    const LayerP& y = m->layers[l];
+    T* qkv = at<T>(m->qkv, l * 3 * Md);
+    norm_fwd<T>(c, m->dec_res, rms ? nullptr : m->P(y.ln1_w), rms ? nullptr : m->P(y.ln1_b), a, m->dec_mean,
+                m->dec_rstd, B, d, rms, eps);
+    GemmDesc g = gd(B, 3 * d, d, a, d, true, m->Wop(y.qkv_w), d, true);
+    g.epi.kind = EPI_BIAS;
+    g.name = "gemm_qkv_decode";
+    g.epi.bias = y.qkv_b >= 0 ? m->P(y.qkv_b) : nullptr;
+    g.epi.out = qkv + (size_t)t * 3 * d;  // row b at position t of the cache
+    g.epi.ldo = Tn * 3 * d;
+    if (!gemm(m, g)) return fail(m, GPT_ERR_CUDA, "decode qkv gemm failed");
+    attn_decode<T>(c, qkv, B, Tn, m->H, m->hd, t, o);
+    g = gd(B, d, d, o, d, true, m->Wop(y.ap_w), d, true);
+    g.epi.kind = EPI_RESADD;
+    g.name = "gemm_attnproj_decode";
+    g.epi.bias = y.ap_b >= 0 ? m->P(y.ap_b) : nullptr;
+    g.epi.res_in = m->dec_res;
+    g.epi.res_out = m->dec_res;
+    g.epi.ld_res = d;
+    g.epi.ldo = d;
+    if (!gemm(m, g)) return fail(m, GPT_ERR_CUDA, "decode attn proj gemm failed");
+    norm_fwd<T>(c, m->dec_res, rms ? nullptr : m->P(y.ln2_w), rms ? nullptr : m->P(y.ln2_b), a, m->dec_mean,
+                m->dec_rstd, B, d, rms, eps);
+    g = gd(B, 4 * d, d, a, d, true, m->Wop(y.fc_w), d, true);
+    g.epi.kind = EPI_BIAS_ACT;
+    g.name = "gemm_fc_decode";
+    g.epi.act = act;
+    g.epi.bias = y.fc_b >= 0 ? m->P(y.fc_b) : nullptr;
+    g.epi.out = m->dec_dact;
+    g.epi.out2 = m->dec_g;
+    g.epi.ldo = 4 * d;
+    if (!gemm(m, g)) return fail(m, GPT_ERR_CUDA, "decode fc gemm failed");
+    g = gd(B, d, 4 * d, m->dec_g, 4 * d, true, m->Wop(y.pr_w), 4 * d, true);
+    g.epi.kind = EPI_RESADD;
+    g.name = "gemm_mlpproj_decode";
+    g.epi.bias = y.pr_b >= 0 ? m->P(y.pr_b) : nullptr;
+    g.epi.res_in = m->dec_res;
+    g.epi.res_out = m->dec_res;
+    g.epi.ld_res = d;
+    g.epi.ldo = d;
+    if (!gemm(m, g)) return fail(m, GPT_ERR_CUDA, "decode mlp proj gemm failed");
+  }
+  norm_fwd<T>(c, m->dec_res, rms ? nullptr : m->P(m->lnf_w), rms ? nullptr : m->P(m->lnf_b), a, m->dec_mean,
+              m->dec_rstd, B, d, rms, eps);
+  GemmDesc g = gd(B, m->Vp, d, a, d, true, m->Wop(m->head), d, true);
+  g.epi.kind = EPI_STORE;
+  g.name = "gemm_lmhead_decode";
+  g.epi.out = m->dec_logits;
+  g.epi.ldo = m->Vp;
+  if (!gemm(m, g)) return fail(m, GPT_ERR_CUDA, "decode lm_head gemm failed");
+  return check_cuda(m, "decode step");
+}
+
 extern "C" {
 
 const char* gpt_status_string(gpt_status s) {
@@ -1077,6 +1159,49 @@ gpt_status gpt_train_step_host(gpt_model* m, const int32_t* h_idx, const int32_t
   cudaMemcpyAsync(m->stage_idx, h_idx, bytes, cudaMemcpyHostToDevice, m->ctx.stream);
   cudaMemcpyAsync(m->stage_tgt, h_tgt, bytes, cudaMemcpyHostToDevice, m->ctx.stream);
   return train_common(m, nullptr, 0, 0, h_idx, h_tgt, lr, step, h_loss, h_grad_norm);
+}
+
+gpt_status gpt_generate(gpt_model* m, const int32_t* d_prompt, int32_t T0, int32_t n_new, float temperature,
+                        int32_t top_k, float top_p, const float* d_uniform, int32_t* d_out) {
+  if (!m || !d_prompt || !d_uniform || !d_out) return fail(m, GPT_ERR_INVALID_ARG, "generate: null argument");
+  if (T0 < 1 || n_new < 1 || (long)T0 + n_new > m->T)
+    return fail(m, GPT_ERR_INVALID_ARG, "generate: need 1 <= prompt length and prompt + new tokens <= block_size");
+  Ctx& c = m->ctx;
+  const int B = m->B, Tn = m->T, Tout = T0 + n_new;
+  const size_t es = m->asz;
+  const float saved_drop = m->cfg.dropout;
+  m->cfg.dropout = 0.f;  // inference runs without dropout
+  const float tp = top_p > 0.f ? top_p : 1e-30f;
+  // prefill: the prompt (zero-padded to block_size; causal attention keeps the
+  // padding out of the prompt's positions) through the full forward, which
+  // fills the qkv caches of positions < T0 and the logits of position T0 - 1
+  cudaMemsetAsync(m->stage_idx, 0, (size_t)m->M * 4, c.stream);
+  cudaMemsetAsync(m->stage_tgt, 0, (size_t)m->M * 4, c.stream);
+  cudaMemcpy2DAsync(m->stage_idx, (size_t)Tn * 4, d_prompt, (size_t)T0 * 4, (size_t)T0 * 4, B,
+                    cudaMemcpyDeviceToDevice, c.stream);
+  cudaMemcpy2DAsync(d_out, (size_t)Tout * 4, d_prompt, (size_t)T0 * 4, (size_t)T0 * 4, B, cudaMemcpyDeviceToDevice,
+                    c.stream);
+  check_tokens(c, m->stage_idx, m->stage_tgt, m->M, m->V, m->idx, m->tgt);
+  gpt_status s = forward_any(m, false, m->scal + 6, 1.0f / (float)m->M, 0);
+  if (s == GPT_OK) {
+    sample_rows(c, m->logits + (size_t)(T0 - 1) * m->Vp * es, m->bf16m, B, m->V, (long)Tn * m->Vp, temperature,
+                top_k, tp, d_uniform, m->dec_tok);
+    cudaMemcpy2DAsync(d_out + T0, (size_t)Tout * 4, m->dec_tok, 4, 4, B, cudaMemcpyDeviceToDevice, c.stream);
+  }
+  for (int i = 1; i < n_new && s == GPT_OK; i++) {
+    const int t = T0 + i - 1;  // position of the token just drawn
+    s = m->bf16m ? decode_step_t<bf16>(m, t) : decode_step_t<float>(m, t);
+    if (s != GPT_OK) break;
+    sample_rows(c, m->dec_logits, m->bf16m, B, m->V, m->Vp, temperature, top_k, tp, d_uniform + (size_t)i * B,
+                m->dec_tok);
+    cudaMemcpy2DAsync(d_out + t + 1, (size_t)Tout * 4, m->dec_tok, 4, 4, B, cudaMemcpyDeviceToDevice, c.stream);
+  }
+  m->cfg.dropout = saved_drop;
+  m->have_forward = false;
+  if (s != GPT_OK) return s;
+  s = check_cuda(m, "generate");
+  if (s != GPT_OK) return s;
+  return sync_and_flags(m, "generate", nullptr);
 }
 
 gpt_status gpt_eval_loss(gpt_model* m, const void* d_stream, uint64_t stream_len, uint64_t data_seed,

@@ -111,6 +111,9 @@ template <typename T> void attn_bwd_simt(Ctx& c, const AttnDesc& a);
 bool attn_tc_supported(const AttnDesc& a);
 void attn_fwd_tc(Ctx& c, const AttnDesc& a);
 void attn_bwd_tc(Ctx& c, const AttnDesc& a);
+// decoding: o [B, H*hd] = attention of position t against positions 0..t of
+// the cache qkv [B, T, 3, H, hd]
+template <typename T> void attn_decode(Ctx& c, const T* qkv, int B, int Tn, int H, int hd, int t, T* o);
 
 // ---------------------------------------------------------------- memory-bound kernels
 // step_dev (nullable): read the step index from device memory instead of `step`

@@ -212,6 +212,21 @@ gpt_status gpt_set_dropout_cursor(gpt_model* m, int32_t step, int32_t micro);
 gpt_status gpt_eval_loss(gpt_model* m, const void* d_stream, uint64_t stream_len, uint64_t data_seed,
                          int32_t n_batches, float* h_loss);
 
+/* Autoregressive generation with a key / value cache (nanoGPT sample.py,
+ * README section "采样 / 推理"; microGPT page, section "单 GPU 高效推理：
+ * 采样 + KV Cache"): d_prompt int32 [batch_size, T0] (device), n_new >= 1
+ * new tokens per row, T0 + n_new <= block_size.  The prompt runs through the
+ * forward once (prefill); every further token costs one decoding step over
+ * the batch rows, whose attention reads the keys / values of the earlier
+ * positions from the forward's own qkv activations (the cache) and appends
+ * its own.  Draws as gpt_sample with d_uniform fp32 [n_new, batch_size]
+ * (device, row i for the i-th new token).  d_out int32 [batch_size,
+ * T0 + n_new] (device) receives prompt and continuation.  No dropout.
+ * Overwrites the activations (a following gpt_backward is GPT_ERR_STATE);
+ * synchronising; GPT_ERR_TOKEN_RANGE for prompt ids outside the vocabulary. */
+gpt_status gpt_generate(gpt_model* m, const int32_t* d_prompt, int32_t T0, int32_t n_new, float temperature,
+                        int32_t top_k, float top_p, const float* d_uniform, int32_t* d_out);
+
 /* One draw from each of `rows` rows of logits (microGPT page, section
  * "单 GPU 高效推理：采样 + KV Cache"; nanoGPT sample.py): d_logits is
  * [rows, ld] (bf16 when logits_bf16, else fp32; device), V <= ld valid
