@@ -221,8 +221,9 @@ def decode_bytes_per_step(w, pos: float) -> float:
 def measure_decode(model, w, stream_host, dev, rank):
     """Autoregressive sampling through gpt_generate at the workload's batch:
     a 64-token prompt and 64 new tokens (temperature 0.8, top-k 40, top-p
-    0.95).  The per-token step time is (t(64 new) - t(1 new)) / 63, which
-    removes the prompt's forward pass."""
+    0.95), replayed as a CUDA graph after two untimed calls.  The per-token
+    step time is (t(64 new) - t(1 new)) / 63, which removes the prompt's
+    forward pass."""
     import torch
     B, T0, n_new = w.batch_size, 64, 64
     rng = np.random.default_rng(17 + rank)
@@ -232,7 +233,8 @@ def measure_decode(model, w, stream_host, dev, rank):
     out = torch.empty((B, T0 + n_new), dtype=torch.int32, device=dev)
 
     def timed(n):
-        model.generate(prompt, n, 0.8, 40, 0.95, U, out)  # warm-up
+        for _ in range(2):  # warm-up: the first call runs eagerly, the second captures its CUDA graph
+            model.generate(prompt, n, 0.8, 40, 0.95, U, out)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record()
         model.generate(prompt, n, 0.8, 40, 0.95, U, out)

@@ -247,7 +247,7 @@ class Model:
                                   _ptr(uniform), _ptr(out)), self.h, "generate")
 
     def set_graphs(self, on: bool):
-        """CUDA-graph replay of train_step / train_step_host (default on)."""
+        """CUDA-graph replay of train_step / train_step_host / generate (default on)."""
         _check(lib().gpt_set_graphs(self.h, 1 if on else 0), self.h, "set_graphs")
 
     # -- introspection

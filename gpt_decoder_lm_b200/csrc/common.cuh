@@ -66,8 +66,10 @@ template <> GPT_HD bf16 from_f<bf16>(float v) { return __float2bfloat16_rn(v); }
 // begin launching once all of its own blocks have started (the next kernel's
 // blocks then fill SMs as this kernel's last wave drains); a kernel launched
 // with the programmatic-serialization attribute waits in pdl_wait() until its
-// predecessor has completed and its writes are visible, and touches no global
-// memory before that.  Both are no-ops without such a launch.
+// predecessor has completed and its writes are visible, and before that reads
+// only memory that no kernel of the stream writes while it may run (the
+// decoding GEMM prefetches weights) and writes none.  Both are no-ops without
+// such a launch.
 __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 

@@ -140,6 +140,11 @@ struct gpt_model {
   int32_t* dec_tok = nullptr;
   float *dec_res = nullptr, *dec_mean = nullptr, *dec_rstd = nullptr;
   uint8_t *dec_a = nullptr, *dec_o = nullptr, *dec_dact = nullptr, *dec_g = nullptr, *dec_logits = nullptr;
+  // CUDA-graph replay of gpt_generate for a repeated call shape
+  cudaGraphExec_t gen_exec = nullptr;
+  int gen_warm = 0;
+  uint64_t gen_launches = 0;
+  uint64_t gen_key[8] = {0, 0, 0, 0, 0, 0, 0, 0};
   int part_cap = 0;                 // partial rows per norm instance
   float* norm_parts = nullptr;      // [2L+1][part_cap][3][d]
   float* colsum_parts = nullptr;    // [L][2][colsum chunks][4d]
@@ -481,6 +486,10 @@ gpt_status sync_and_flags(gpt_model* m, const char* where, float* h_scal /* 4 fl
 bool gemm(gpt_model* m, GemmDesc& g) {
   if (!m->bf16m) {
     gemm_simt_f32(m->ctx, g);
+    return true;
+  }
+  if (gemm_skinny_supported(g)) {
+    gemm_skinny_bf16(m->ctx, g);
     return true;
   }
   if (gemm_tc_supported(g)) return gemm_tc_bf16(m->ctx, g);
@@ -972,6 +981,7 @@ void gpt_destroy(gpt_model* m) {
   if (!m) return;
   for (auto& e : m->gexec)
     if (e) cudaGraphExecDestroy(e);
+  if (m->gen_exec) cudaGraphExecDestroy(m->gen_exec);
   if (m->cap_stream) cudaStreamDestroy(m->cap_stream);
   delete m->timing;
   delete m;
@@ -1161,11 +1171,10 @@ gpt_status gpt_train_step_host(gpt_model* m, const int32_t* h_idx, const int32_t
   return train_common(m, nullptr, 0, 0, h_idx, h_tgt, lr, step, h_loss, h_grad_norm);
 }
 
-gpt_status gpt_generate(gpt_model* m, const int32_t* d_prompt, int32_t T0, int32_t n_new, float temperature,
-                        int32_t top_k, float top_p, const float* d_uniform, int32_t* d_out) {
-  if (!m || !d_prompt || !d_uniform || !d_out) return fail(m, GPT_ERR_INVALID_ARG, "generate: null argument");
-  if (T0 < 1 || n_new < 1 || (long)T0 + n_new > m->T)
-    return fail(m, GPT_ERR_INVALID_ARG, "generate: need 1 <= prompt length and prompt + new tokens <= block_size");
+// The kernels and copies of one gpt_generate call (prefill, draws, decoding
+// steps), enqueued on the model's stream.
+static gpt_status generate_body(gpt_model* m, const int32_t* d_prompt, int32_t T0, int32_t n_new, float temperature,
+                                int32_t top_k, float top_p, const float* d_uniform, int32_t* d_out) {
   Ctx& c = m->ctx;
   const int B = m->B, Tn = m->T, Tout = T0 + n_new;
   const size_t es = m->asz;
@@ -1197,9 +1206,66 @@ gpt_status gpt_generate(gpt_model* m, const int32_t* d_prompt, int32_t T0, int32
     cudaMemcpy2DAsync(d_out + t + 1, (size_t)Tout * 4, m->dec_tok, 4, 4, B, cudaMemcpyDeviceToDevice, c.stream);
   }
   m->cfg.dropout = saved_drop;
-  m->have_forward = false;
   if (s != GPT_OK) return s;
-  s = check_cuda(m, "generate");
+  return check_cuda(m, "generate");
+}
+
+gpt_status gpt_generate(gpt_model* m, const int32_t* d_prompt, int32_t T0, int32_t n_new, float temperature,
+                        int32_t top_k, float top_p, const float* d_uniform, int32_t* d_out) {
+  if (!m || !d_prompt || !d_uniform || !d_out) return fail(m, GPT_ERR_INVALID_ARG, "generate: null argument");
+  if (T0 < 1 || n_new < 1 || (long)T0 + n_new > m->T)
+    return fail(m, GPT_ERR_INVALID_ARG, "generate: need 1 <= prompt length and prompt + new tokens <= block_size");
+  Ctx& c = m->ctx;
+  // A repeated call shape (same buffers, lengths and sampling parameters)
+  // replays a CUDA graph of the whole call: the first call runs eagerly, the
+  // second is captured, later ones replay.
+  uint64_t key[8] = {(uint64_t)(uintptr_t)d_prompt, (uint64_t)(uintptr_t)d_uniform, (uint64_t)(uintptr_t)d_out,
+                     (uint64_t)T0, (uint64_t)n_new, 0, (uint64_t)(uint32_t)top_k, 0};
+  memcpy(&key[5], &temperature, 4);
+  memcpy(&key[7], &top_p, 4);
+  bool replay = m->graphs_on && !c.timing;
+  if (memcmp(key, m->gen_key, sizeof key) != 0) {  // a new call shape starts over
+    if (m->gen_exec) cudaGraphExecDestroy(m->gen_exec);
+    m->gen_exec = nullptr;
+    m->gen_warm = 0;
+    memcpy(m->gen_key, key, sizeof key);
+  }
+  gpt_status s = GPT_OK;
+  if (replay && !m->gen_exec) {
+    if (m->gen_warm < 1) {
+      m->gen_warm++;
+      replay = false;
+    } else {
+      bool ok = m->cap_stream || cudaStreamCreateWithFlags(&m->cap_stream, cudaStreamNonBlocking) == cudaSuccess;
+      cudaStream_t user = c.stream;
+      const uint64_t l0 = c.launches;
+      cudaGraph_t g = nullptr;
+      if (ok) ok = cudaStreamBeginCapture(m->cap_stream, cudaStreamCaptureModeThreadLocal) == cudaSuccess;
+      if (ok) {
+        c.stream = m->cap_stream;
+        s = generate_body(m, d_prompt, T0, n_new, temperature, top_k, top_p, d_uniform, d_out);
+        c.stream = user;
+        m->gen_launches = c.launches - l0;
+        ok = cudaStreamEndCapture(m->cap_stream, &g) == cudaSuccess && s == GPT_OK;
+      }
+      if (ok) ok = cudaGraphInstantiate(&m->gen_exec, g, 0) == cudaSuccess;
+      if (g) cudaGraphDestroy(g);
+      c.launches = l0;
+      if (!ok) {
+        cudaGetLastError();
+        m->gen_exec = nullptr;
+        replay = false;
+        s = GPT_OK;
+      }
+    }
+  }
+  if (replay && m->gen_exec) {
+    if (cudaGraphLaunch(m->gen_exec, c.stream) != cudaSuccess) return check_cuda(m, "generate graph launch");
+    c.launches += m->gen_launches;
+  } else {
+    s = generate_body(m, d_prompt, T0, n_new, temperature, top_k, top_p, d_uniform, d_out);
+  }
+  m->have_forward = false;
   if (s != GPT_OK) return s;
   return sync_and_flags(m, "generate", nullptr);
 }

@@ -13,14 +13,18 @@
 //   draw                   the first token (index order) whose running sum
 //                          of kept p exceeds u * (kept mass)
 // The k-th largest logit is found by an MSB-first radix select over an
-// order-preserving integer image of the floats, tau by bisection over the
-// bit pattern of positive floats.
+// order-preserving integer image of the floats (warp-aggregated histogram
+// updates), tau by bisection over the bit pattern of positive floats.  When
+// the kept set is small (top-k), it is first compacted in index order into
+// shared memory with its probabilities, and one warp runs the bisection and
+// the draw over that list instead of the whole row.
 #include "kernels.cuh"
 
 namespace gpt {
 namespace {
 
-constexpr int ST = 1024;  // threads per row
+constexpr int ST = 1024;   // threads per row
+constexpr int CAP = 4096;  // kept tokens handled by the compacted path
 
 // order-preserving image of a float as an unsigned integer
 __device__ __forceinline__ uint32_t fkey(float f) {
@@ -59,6 +63,7 @@ __global__ void __launch_bounds__(ST) k_sample(const T* __restrict__ logits, lon
   // maximum (and its lowest index, for greedy decoding)
   float best = -INFINITY;
   int bi = 0x7fffffff;
+#pragma unroll 4
   for (int i = tid; i < V; i += ST) {
     const float v = to_f<T>(z[i]);
     if (v > best) {  // strided order: the first hit of a thread is its lowest index
@@ -109,9 +114,23 @@ __global__ void __launch_bounds__(ST) k_sample(const T* __restrict__ logits, lon
     for (int shift = 24; shift >= 0; shift -= 8) {
       for (int b = tid; b < 256; b += ST) hist[b] = 0;
       __syncthreads();
-      for (int i = tid; i < V; i += ST) {
-        const uint32_t key = fkey(to_f<T>(z[i]));
-        if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
+      for (int i0 = 0; i0 < V; i0 += 4 * ST) {  // whole warps iterate together, 4 loads in flight
+        uint32_t key[4];
+#pragma unroll
+        for (int u = 0; u < 4; u++) {
+          const int i = i0 + u * ST + tid;
+          key[u] = i < V ? fkey(to_f<T>(z[i])) : 0u;
+        }
+#pragma unroll
+        for (int u = 0; u < 4; u++) {
+          const bool hit = i0 + u * ST + tid < V && (key[u] & mask) == prefix;
+          const uint32_t want = __ballot_sync(0xffffffffu, hit);
+          if (hit) {  // one shared-memory atomic per distinct bin of the warp
+            const uint32_t bin = (key[u] >> shift) & 255u;
+            const uint32_t peers = __match_any_sync(want, bin);
+            if (lane == __ffs(peers) - 1) atomicAdd(&hist[bin], (uint32_t)__popc(peers));
+          }
+        }
       }
       __syncthreads();
       if (tid == 0) {
@@ -136,6 +155,122 @@ __global__ void __launch_bounds__(ST) k_sample(const T* __restrict__ logits, lon
     const float v = to_f<T>(z[i]);
     return fkey(v) >= thr ? __expf((v - zmax) * inv_t) : 0.f;
   };
+
+  // compacted path: the kept tokens (logit key >= thr) of each warp's
+  // contiguous index range, counted, then written in index order with their
+  // probabilities; one warp finishes when they fit in shared memory
+  __shared__ int c_idx[CAP];
+  __shared__ float c_p[CAP];
+  __shared__ int wbase[33];
+  if (thr != 0u) {
+    const int segw = (V + 31) / 32 / 128 * 128 + 128;  // per-warp range, a multiple of 128
+    const int w0 = min(V, w * segw), w1 = min(V, w0 + segw);
+    int cnt = 0;
+    for (int i0 = w0 + lane; i0 - lane < w1; i0 += 128) {  // 4 loads in flight
+      float v[4];
+#pragma unroll
+      for (int u = 0; u < 4; u++) v[u] = i0 + 32 * u < w1 ? to_f<T>(z[i0 + 32 * u]) : 0.f;
+#pragma unroll
+      for (int u = 0; u < 4; u++) cnt += __popc(__ballot_sync(0xffffffffu, i0 + 32 * u < w1 && fkey(v[u]) >= thr));
+    }
+    if (lane == 0) wbase[w] = cnt;
+    __syncthreads();
+    if (tid == 0) {
+      int run = 0;
+      for (int k = 0; k < ST / 32; k++) {
+        const int t = wbase[k];
+        wbase[k] = run;
+        run += t;
+      }
+      wbase[32] = run;
+    }
+    __syncthreads();
+    const int n = wbase[32];
+    if (n <= CAP) {
+      int off = wbase[w];
+      for (int i0 = w0 + lane; i0 - lane < w1; i0 += 128) {
+        float v[4];
+#pragma unroll
+        for (int u = 0; u < 4; u++) v[u] = i0 + 32 * u < w1 ? to_f<T>(z[i0 + 32 * u]) : 0.f;
+#pragma unroll
+        for (int u = 0; u < 4; u++) {
+          const int i = i0 + 32 * u;
+          const bool k = i < w1 && fkey(v[u]) >= thr;
+          const uint32_t b = __ballot_sync(0xffffffffu, k);
+          if (k) {
+            const int o = off + __popc(b & ((1u << lane) - 1u));
+            c_idx[o] = i;
+            c_p[o] = __expf((v[u] - zmax) * inv_t);
+          }
+          off += __popc(b);
+        }
+      }
+      __syncthreads();
+      if (w != 0) return;
+      // top-p over the list: lane-strided sums, butterfly totals (identical in every lane)
+      float tau_c = 0.f;
+      if (top_p < 1.f) {
+        float s0 = 0.f;
+        for (int j = lane; j < n; j += 32) s0 += c_p[j];
+        const float target = top_p * warp_sum(s0);
+        uint32_t cur = 0;
+        for (int bit = 30; bit >= 0; bit--) {
+          const uint32_t cand = cur | (1u << bit);
+          const float t = __uint_as_float(cand);
+          float m = 0.f;
+          for (int j = lane; j < n; j += 32) {
+            const float p = c_p[j];
+            if (p >= t) m += p;
+          }
+          if (warp_sum(m) >= target) cur = cand;
+        }
+        tau_c = __uint_as_float(cur);
+      }
+      // draw: contiguous runs of the list per lane, a lane-order scan of their sums
+      const int cs = (n + 31) / 32;
+      const int j0 = min(n, lane * cs), j1 = min(n, j0 + cs);
+      float local = 0.f;
+      int last = -1;
+      for (int j = j0; j < j1; j++) {
+        const float p = c_p[j];
+        if (p >= tau_c && p > 0.f) {
+          local += p;
+          last = c_idx[j];
+        }
+      }
+      float incl = local;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const float x = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += x;
+      }
+      const float total = __shfl_sync(0xffffffffu, incl, 31);
+      const float excl = incl - local;
+      const float target = uniform[blockIdx.x] * total;
+      int hit = 0x7fffffff;
+      if (excl + local > target && excl <= target) {
+        float run = excl;
+        for (int j = j0; j < j1; j++) {
+          const float p = c_p[j];
+          if (p >= tau_c && p > 0.f) {
+            run += p;
+            if (run > target) {
+              hit = c_idx[j];
+              break;
+            }
+          }
+        }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        hit = min(hit, __shfl_xor_sync(0xffffffffu, hit, o));
+        last = max(last, __shfl_xor_sync(0xffffffffu, last, o));
+      }
+      if (lane == 0) out[blockIdx.x] = hit != 0x7fffffff ? hit : last;
+      return;
+    }
+    __syncthreads();
+  }
 
   // top-p: tau by bisection over the bits of a positive float
   float tau = 0.f;

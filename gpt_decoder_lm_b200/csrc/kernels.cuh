@@ -87,6 +87,9 @@ TcPlan gemm_tc_plan(long M, long N, long K, bool split_ok, int num_sms);
 void gemm_simt_f32(Ctx& c, const GemmDesc& g);
 void gemm_simt_bf16(Ctx& c, const GemmDesc& g);
 bool gemm_tc_supported(const GemmDesc& g);
+// GEMMs of at most 16 rows (decoding): bf16, both operands K-major, no split-K
+bool gemm_skinny_supported(const GemmDesc& g);
+void gemm_skinny_bf16(Ctx& c, const GemmDesc& g);
 bool gemm_tc_bf16(Ctx& c, const GemmDesc& g);  // false: tensor-map encode failed
 // the split-K count gemm_tc_bf16 uses for g (1: none)
 int gemm_tc_splits(const GemmDesc& g, int num_sms);

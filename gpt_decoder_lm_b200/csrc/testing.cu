@@ -45,6 +45,10 @@ extern "C" gpt_status gpt_test_gemm(int32_t backend, int32_t M, int32_t N, int32
       if (!gemm_tc_supported(g)) return GPT_ERR_UNSUPPORTED;
       if (!gemm_tc_bf16(c, g)) return GPT_ERR_CUDA;
       break;
+    case GPT_GEMM_SKINNY_BF16:
+      if (!gemm_skinny_supported(g)) return GPT_ERR_UNSUPPORTED;
+      gemm_skinny_bf16(c, g);
+      break;
     default: return GPT_ERR_INVALID_ARG;
   }
   if (cudaStreamSynchronize(c.stream) != cudaSuccess || cudaGetLastError() != cudaSuccess) return GPT_ERR_CUDA;

@@ -181,7 +181,8 @@ gpt_status gpt_train_step(gpt_model* m, const void* d_stream, uint64_t stream_le
 gpt_status gpt_train_step_host(gpt_model* m, const int32_t* h_idx, const int32_t* h_tgt, float lr,
                                int32_t step, float* h_loss, float* h_grad_norm);
 
-/* CUDA-graph replay of gpt_train_step / gpt_train_step_host (default on).
+/* CUDA-graph replay of gpt_train_step / gpt_train_step_host (default on;
+ * gpt_generate is replayed under the same switch).
  * When on, and the config has no dropout and per-kernel timing is off, the
  * first step of each kind runs eagerly, the second is captured into a graph
  * (on a stream the library creates) and every later step replays it on the
@@ -223,7 +224,10 @@ gpt_status gpt_eval_loss(gpt_model* m, const void* d_stream, uint64_t stream_len
  * (device, row i for the i-th new token).  d_out int32 [batch_size,
  * T0 + n_new] (device) receives prompt and continuation.  No dropout.
  * Overwrites the activations (a following gpt_backward is GPT_ERR_STATE);
- * synchronising; GPT_ERR_TOKEN_RANGE for prompt ids outside the vocabulary. */
+ * synchronising; GPT_ERR_TOKEN_RANGE for prompt ids outside the vocabulary.
+ * With graphs on (gpt_set_graphs), a call repeating the previous call's
+ * buffers, lengths and sampling parameters replays a CUDA graph of the whole
+ * call (the first such call runs eagerly, the second is captured). */
 gpt_status gpt_generate(gpt_model* m, const int32_t* d_prompt, int32_t T0, int32_t n_new, float temperature,
                         int32_t top_k, float top_p, const float* d_uniform, int32_t* d_out);
 

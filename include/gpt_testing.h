@@ -19,7 +19,7 @@ extern "C" {
 #endif
 
 /* Backends of gpt_test_gemm. */
-enum { GPT_GEMM_SIMT_F32 = 0, GPT_GEMM_SIMT_BF16 = 1, GPT_GEMM_TC_BF16 = 2 };
+enum { GPT_GEMM_SIMT_F32 = 0, GPT_GEMM_SIMT_BF16 = 1, GPT_GEMM_TC_BF16 = 2, GPT_GEMM_SKINNY_BF16 = 3 };
 
 /* D[m, n] = sum_k A[m, k] * B[n, k] followed by epilogue `epi_kind`:
  *   0 out = D; 1 out = D + bias; 2 with h = D + bias: out = act'(h), out2 = act(h);
@@ -30,8 +30,10 @@ enum { GPT_GEMM_SIMT_F32 = 0, GPT_GEMM_SIMT_BF16 = 1, GPT_GEMM_TC_BF16 = 2 };
  * GPT_GEMM_SIMT_F32 and bf16 otherwise; outputs of kinds 0-2 and 4 have the
  * operand type, kinds 3, 5 and 6 are fp32.  act: 0 GELU (erf), 1 ReLU.
  * split_k > 1 (kind 5 only, tensor-core backend) needs `partial`
- * [split_k, M, N] fp32 scratch.  GPT_ERR_UNSUPPORTED when the tensor-core
- * backend cannot take the shape. */
+ * [split_k, M, N] fp32 scratch.  GPT_GEMM_SKINNY_BF16 (the decoding-step
+ * GEMM) takes M <= 16, K a multiple of 32, both operands K-major, no split-K.
+ * GPT_ERR_UNSUPPORTED when the tensor-core or skinny backend cannot take the
+ * shape. */
 gpt_status gpt_test_gemm(int32_t backend, int32_t M, int32_t N, int32_t K, const void* A, int64_t lda,
                          int32_t a_kmajor, const void* B, int64_t ldb, int32_t b_kmajor, int32_t epi_kind,
                          int32_t act, void* out, void* out2, int32_t ldo, const void* aux, const float* bias,

@@ -19,7 +19,7 @@ if not torch.cuda.is_available():
 from gpt_decoder_lm_b200 import binding as gb  # noqa: E402
 from scipy.special import erf  # noqa: E402
 
-TC, SIMT_BF16, SIMT_F32 = 2, 1, 0
+SKINNY, TC, SIMT_BF16, SIMT_F32 = 3, 2, 1, 0
 
 
 def bf16_round(x: np.ndarray) -> np.ndarray:
@@ -77,9 +77,10 @@ def test_tc_gemm_store_f32(M, N, K, ak, bk):
     assert err < 2e-6, err
 
 
-@pytest.mark.parametrize("backend", [TC, SIMT_BF16], ids=["tc", "simt"])
-def test_epilogues(backend):
-    M, N, K = 384, 512, 256
+@pytest.mark.parametrize("backend,M", [(TC, 384), (SIMT_BF16, 384), (SKINNY, 12), (SKINNY, 5)],
+                         ids=["tc", "simt", "skinny12", "skinny5"])
+def test_epilogues(backend, M):
+    N, K = 512, 256
     rng = np.random.default_rng(7)
     A, B, Ad, Bd, lda, ldb = operands(M, N, K, 1, 1, 3)
     D = A @ B.T
@@ -116,6 +117,52 @@ def test_epilogues(backend):
     acc = dev_f32(acc0)
     run(backend, M, N, K, Ad, lda, 1, Bd, ldb, 1, 5, out=acc, ldo=N)
     np.testing.assert_allclose(acc.double().cpu().numpy(), acc0 + D, rtol=1e-5, atol=1e-4)
+
+
+SKINNY_SHAPES = [(1, 16, 32), (5, 200, 96), (8, 1000, 64), (12, 2304, 768), (12, 768, 3072), (16, 3072, 768),
+                 (12, 50304, 768), (9, 40, 4096)]
+
+
+@pytest.mark.parametrize("M,N,K", SKINNY_SHAPES, ids=[f"{m}x{n}x{k}" for m, n, k in SKINNY_SHAPES])
+def test_skinny_gemm_store_f32(M, N, K):
+    """The decoding-step GEMM (at most 16 rows): every row count of an 8-row
+    tile pair, ragged N, each K split of the warps, the GPT-2 124M shapes."""
+    A, B, Ad, Bd, lda, ldb = operands(M, N, K, 1, 1, M * 7 + N + K)
+    out = torch.full((M, N), float("nan"), device="cuda")
+    run(SKINNY, M, N, K, Ad, lda, 1, Bd, ldb, 1, 6, out=out, ldo=N)
+    ref = A @ B.T
+    got = out.double().cpu().numpy()
+    err = np.abs(got - ref).max() / np.abs(ref).max()
+    assert err < 2e-6, err
+
+
+def test_skinny_gemm_pitches():
+    """Row pitches wider than the rows (lda, ldb, ldo) and a strided output,
+    as the decoding step writes into the key / value cache."""
+    M, N, K = 12, 2304, 768
+    rng = np.random.default_rng(4)
+    A = bf16_round(rng.standard_normal((M, K)))
+    B = bf16_round(rng.standard_normal((N, K)))
+    Ad = dev_bf16(np.concatenate([A, np.zeros((M, 64))], 1))
+    Bd = dev_bf16(np.concatenate([B, np.ones((N, 32))], 1))
+    out = torch.full((M, 3 * N), float("nan"), device="cuda")
+    run(SKINNY, M, N, K, Ad, K + 64, 1, Bd, K + 32, 1, 6, out=out, ldo=3 * N)
+    got = out.double().cpu().numpy()
+    err = np.abs(got[:, :N] - A @ B.T).max() / np.abs(A @ B.T).max()
+    assert err < 2e-6, err
+    assert np.isnan(got[:, N:]).all()
+
+
+def test_skinny_gemm_unsupported():
+    A, B, Ad, Bd, lda, ldb = operands(17, 64, 64, 1, 1, 1)
+    flags = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = torch.empty((17, 64), device="cuda")
+    st = gb.test_gemm(SKINNY, 17, 64, 64, Ad, lda, 1, Bd, ldb, 1, 6, out=out, ldo=64,
+                      stream=torch.cuda.current_stream().cuda_stream, flags=flags)
+    assert gb.STATUS[st] == "GPT_ERR_UNSUPPORTED"
+    st = gb.test_gemm(SKINNY, 8, 64, 48, Ad, lda, 1, Bd, ldb, 1, 6, out=out, ldo=64,
+                      stream=torch.cuda.current_stream().cuda_stream, flags=flags)
+    assert gb.STATUS[st] == "GPT_ERR_UNSUPPORTED"  # K not a multiple of 32
 
 
 @pytest.mark.parametrize("splits", [2, 5])

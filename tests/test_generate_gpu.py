@@ -131,3 +131,43 @@ def test_generate_errors():
         m.generate(prompt, 2, 1.0, 0, 1.0, U, out)
     assert e.value.name == "GPT_ERR_TOKEN_RANGE"
     m.close()
+
+
+def test_generate_graph_replay_matches_eager():
+    """A repeated call shape replays a CUDA graph of the whole call (the first
+    call is eager, the second captured); replays read the prompt and uniforms
+    in place, so new contents give the eager result for those contents."""
+    w = W.CHAR.with_(precision="bf16", init_std=0.3)
+    over = dict(n_layer=2, batch_size=4, block_size=128)
+    m_graph, cfg, _, _ = setup(w, **over)
+    m_eager, _, _, _ = setup(w, **over)
+    m_eager.set_graphs(False)
+    B, T0, n_new = cfg.batch_size, 7, 16
+    prompt = torch.zeros((B, T0), dtype=torch.int32, device="cuda")
+    U = torch.zeros((n_new, B), device="cuda")
+    out_g = torch.full((B, T0 + n_new), -1, dtype=torch.int32, device="cuda")
+    out_e = torch.full_like(out_g, -1)
+    rng = np.random.default_rng(5)
+    for call in range(5):
+        prompt.copy_(torch.from_numpy(rng.integers(0, cfg.vocab_size, (B, T0)).astype(np.int32)))
+        U.copy_(torch.from_numpy(rng.random((n_new, B)).astype(np.float32)))
+        m_graph.generate(prompt, n_new, 1.0, 5, 0.95, U, out_g)
+        m_eager.generate(prompt, n_new, 1.0, 5, 0.95, U, out_e)
+        assert torch.equal(out_g, out_e), call
+    # the token-range check still reports from a replayed graph
+    prompt.fill_(cfg.vocab_size + 1)
+    with pytest.raises(gb.GptError) as e:
+        m_graph.generate(prompt, n_new, 1.0, 5, 0.95, U, out_g)
+    assert e.value.name == "GPT_ERR_TOKEN_RANGE"
+    # a new call shape starts over (eager, capture, replay) and stays exact
+    p3 = torch.zeros((B, 3), dtype=torch.int32, device="cuda")
+    short_g = torch.full((B, 3 + n_new), -1, dtype=torch.int32, device="cuda")
+    short_e = torch.full_like(short_g, -1)
+    for call in range(4):
+        p3.copy_(torch.from_numpy(rng.integers(0, cfg.vocab_size, (B, 3)).astype(np.int32)))
+        U.copy_(torch.from_numpy(rng.random((n_new, B)).astype(np.float32)))
+        m_graph.generate(p3, n_new, 0.7, 0, 0.9, U, short_g)
+        m_eager.generate(p3, n_new, 0.7, 0, 0.9, U, short_e)
+        assert torch.equal(short_g, short_e), call
+    m_graph.close()
+    m_eager.close()

@@ -66,7 +66,7 @@ def run_case(V, rows, dtype, temperature, top_k, top_p, seed):
 
 @pytest.mark.parametrize("temperature,top_k,top_p", [
     (0.0, 0, 1.0), (1.0, 0, 1.0), (0.7, 40, 1.0), (1.3, 0, 0.9), (0.8, 40, 0.9), (1.0, 1, 1.0), (1.0, 5, 0.5),
-    (1.0, 0, 0.0)])
+    (1.0, 0, 0.0), (1.0, 4000, 0.95), (1.0, 5000, 0.9)])
 def test_sample_vocab_bf16(temperature, top_k, top_p):
     run_case(50257, 24, torch.bfloat16, temperature, top_k, top_p, seed=int(temperature * 10) + top_k)
 
@@ -74,6 +74,30 @@ def test_sample_vocab_bf16(temperature, top_k, top_p):
 @pytest.mark.parametrize("V", [1, 7, 1000, 4097])
 def test_sample_small_vocab_fp32(V):
     run_case(V, 16, torch.float32, 0.9, min(3, V), 0.95, seed=V)
+
+
+@pytest.mark.parametrize("V", [1000, 20000])
+def test_sample_top_k_ties(V):
+    """Logits on a coarse grid: the k-th largest value is shared by many
+    tokens, all of which are kept (a few hundred in shared memory at V = 1000,
+    more than it holds at V = 20000)."""
+    rows = 16
+    rng = np.random.default_rng(V)
+    z = rng.integers(0, 4, (rows, V)).astype(np.float32)
+    u = rng.random(rows).astype(np.float32)
+    out = torch.empty(rows, dtype=torch.int32, device="cuda")
+    gb.sample(torch.from_numpy(z).cuda(), 1.0, 5, 0.8, torch.from_numpy(u).cuda(), out)
+    got = out.cpu().numpy()
+    for r in range(rows):
+        ref = S.sample_row(z[r].astype(np.float64), 1.0, 5, 0.8, float(u[r]))
+        p = S._kept_probs(z[r].astype(np.float64), 1.0, 5, 0.8)
+        assert p[got[r]] > 0, (r, got[r])
+        # equal probabilities: the draw is the token whose CDF interval holds u
+        # up to rounding of the running sum
+        c = np.cumsum(p) / p.sum()
+        lo = np.searchsorted(c, u[r] - 1e-5, side="right")
+        hi = np.searchsorted(c, u[r] + 1e-5, side="right")
+        assert min(lo, ref) <= got[r] <= max(hi, ref), (r, got[r], ref, lo, hi)
 
 
 def test_sample_frequencies_follow_the_kept_softmax():
