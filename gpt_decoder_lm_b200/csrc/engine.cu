@@ -822,19 +822,38 @@ gpt_status decode_step_t(gpt_model* m, int t) {
   const size_t Md = (size_t)m->M * d;
   T* a = reinterpret_cast<T*>(m->dec_a);
   T* o = reinterpret_cast<T*>(m->dec_o);
+  // norm of the residual rows, then a GEMM on it: one skinny GEMM that
+  // computes the norm itself where it applies, else the two kernels
+  auto norm_gemm = [&](int64_t wi, int64_t bi, GemmDesc& g) -> bool {
+    const float* nw = rms ? nullptr : m->P(wi);
+    const float* nb = rms ? nullptr : m->P(bi);
+    if (m->bf16m && gemm_skinny_supported(g)) {
+      SkinnyNorm n;
+      n.x = m->dec_res;
+      n.w = nw;
+      n.b = nb;
+      n.ldx = d;
+      n.rms = rms ? 1 : 0;
+      n.eps = eps;
+      if (skinny_norm_supported(g, n)) {
+        gemm_skinny_bf16(c, g, &n);
+        return true;
+      }
+    }
+    norm_fwd<T>(c, m->dec_res, nw, nb, a, m->dec_mean, m->dec_rstd, B, d, rms, eps);
+    return gemm(m, g);
+  };
   embed_fwd<T>(c, m->dec_tok, m->P(m->wte), m->P(m->wpe) + (size_t)t * d, m->dec_res, B, 1, d, DropKey{});
   for (int l = 0; l < L; l++) {
     const LayerP& y = m->layers[l];
     T* qkv = at<T>(m->qkv, l * 3 * Md);
-    norm_fwd<T>(c, m->dec_res, rms ? nullptr : m->P(y.ln1_w), rms ? nullptr : m->P(y.ln1_b), a, m->dec_mean,
-                m->dec_rstd, B, d, rms, eps);
     GemmDesc g = gd(B, 3 * d, d, a, d, true, m->Wop(y.qkv_w), d, true);
     g.epi.kind = EPI_BIAS;
     g.name = "gemm_qkv_decode";
     g.epi.bias = y.qkv_b >= 0 ? m->P(y.qkv_b) : nullptr;
     g.epi.out = qkv + (size_t)t * 3 * d;  // row b at position t of the cache
     g.epi.ldo = Tn * 3 * d;
-    if (!gemm(m, g)) return fail(m, GPT_ERR_CUDA, "decode qkv gemm failed");
+    if (!norm_gemm(y.ln1_w, y.ln1_b, g)) return fail(m, GPT_ERR_CUDA, "decode qkv gemm failed");
     attn_decode<T>(c, qkv, B, Tn, m->H, m->hd, t, o);
     g = gd(B, d, d, o, d, true, m->Wop(y.ap_w), d, true);
     g.epi.kind = EPI_RESADD;
@@ -845,8 +864,6 @@ gpt_status decode_step_t(gpt_model* m, int t) {
     g.epi.ld_res = d;
     g.epi.ldo = d;
     if (!gemm(m, g)) return fail(m, GPT_ERR_CUDA, "decode attn proj gemm failed");
-    norm_fwd<T>(c, m->dec_res, rms ? nullptr : m->P(y.ln2_w), rms ? nullptr : m->P(y.ln2_b), a, m->dec_mean,
-                m->dec_rstd, B, d, rms, eps);
     g = gd(B, 4 * d, d, a, d, true, m->Wop(y.fc_w), d, true);
     g.epi.kind = EPI_BIAS_ACT;
     g.name = "gemm_fc_decode";
@@ -855,7 +872,7 @@ gpt_status decode_step_t(gpt_model* m, int t) {
     g.epi.out = m->dec_dact;
     g.epi.out2 = m->dec_g;
     g.epi.ldo = 4 * d;
-    if (!gemm(m, g)) return fail(m, GPT_ERR_CUDA, "decode fc gemm failed");
+    if (!norm_gemm(y.ln2_w, y.ln2_b, g)) return fail(m, GPT_ERR_CUDA, "decode fc gemm failed");
     g = gd(B, d, 4 * d, m->dec_g, 4 * d, true, m->Wop(y.pr_w), 4 * d, true);
     g.epi.kind = EPI_RESADD;
     g.name = "gemm_mlpproj_decode";
@@ -866,14 +883,12 @@ gpt_status decode_step_t(gpt_model* m, int t) {
     g.epi.ldo = d;
     if (!gemm(m, g)) return fail(m, GPT_ERR_CUDA, "decode mlp proj gemm failed");
   }
-  norm_fwd<T>(c, m->dec_res, rms ? nullptr : m->P(m->lnf_w), rms ? nullptr : m->P(m->lnf_b), a, m->dec_mean,
-              m->dec_rstd, B, d, rms, eps);
   GemmDesc g = gd(B, m->Vp, d, a, d, true, m->Wop(m->head), d, true);
   g.epi.kind = EPI_STORE;
   g.name = "gemm_lmhead_decode";
   g.epi.out = m->dec_logits;
   g.epi.ldo = m->Vp;
-  if (!gemm(m, g)) return fail(m, GPT_ERR_CUDA, "decode lm_head gemm failed");
+  if (!norm_gemm(m->lnf_w, m->lnf_b, g)) return fail(m, GPT_ERR_CUDA, "decode lm_head gemm failed");
   return check_cuda(m, "decode step");
 }
 

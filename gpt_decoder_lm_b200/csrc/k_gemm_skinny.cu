@@ -56,7 +56,7 @@ __device__ __forceinline__ uint4 ld_stream(const uint4* p) {
 // ks = warps splitting K (a power of two up to SK_WARPS); pitch =
 // shared-memory row pitch of the staged activations in bytes.
 template <int NT>
-__global__ void __launch_bounds__(SK_WARPS * 32) k_gemm_skinny(GemmDesc g, int ks, int pitch) {
+__global__ void __launch_bounds__(SK_WARPS * 32) k_gemm_skinny(GemmDesc g, SkinnyNorm nrm, int ks, int pitch) {
   extern __shared__ __align__(16) uint8_t smem[];
   pdl_trigger();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -86,9 +86,74 @@ __global__ void __launch_bounds__(SK_WARPS * 32) k_gemm_skinny(GemmDesc g, int k
   load(kb0);
   pdl_wait();
 
-  // activations -> shared memory, rows M .. 8 NT - 1 zero; eight 16-byte
-  // loads per thread in flight before their stores
-  {
+  if (nrm.x) {
+    // A = norm(x) computed here (one warp per row, the norm kernel's formulas
+    // and summation order): LayerNorm (x - mean) rstd w + b, or RMSNorm x rstd
+    const int d4 = g.K >> 2;
+    for (int r = warp; r < 8 * NT; r += SK_WARPS) {
+      uint8_t* srow = smem + (size_t)r * pitch;
+      if (r >= g.M) {
+        for (int c8 = lane; c8 < (g.K >> 3); c8 += 32)
+          *reinterpret_cast<uint4*>(srow + 16 * c8) = make_uint4(0u, 0u, 0u, 0u);
+        continue;
+      }
+      const float4* xr = reinterpret_cast<const float4*>(nrm.x + (long)r * nrm.ldx);
+      float sum = 0.f;
+#pragma unroll 4
+      for (int c = lane; c < d4; c += 32) {
+        const float4 v = xr[c];
+        sum += nrm.rms ? (v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w) : (v.x + v.y + v.z + v.w);
+      }
+      sum = warp_sum(sum);
+      float mean = 0.f, rstd;
+      if (nrm.rms) {
+        rstd = 1.0f / sqrtf(sum / g.K + nrm.eps);
+      } else {
+        mean = sum / g.K;
+        float qs = 0.f;
+#pragma unroll 4
+        for (int c = lane; c < d4; c += 32) {
+          const float4 v = xr[c];
+          const float a = v.x - mean, b = v.y - mean, cc = v.z - mean, dd = v.w - mean;
+          qs += a * a + b * b + cc * cc + dd * dd;
+        }
+        qs = warp_sum(qs);
+        rstd = 1.0f / sqrtf(qs / g.K + nrm.eps);
+      }
+#pragma unroll 2
+      for (int c8 = lane; c8 < (g.K >> 3); c8 += 32) {
+        float y[8];
+#pragma unroll
+        for (int h = 0; h < 2; h++) {
+          const float4 v = xr[2 * c8 + h];
+          y[4 * h + 0] = (v.x - mean) * rstd;
+          y[4 * h + 1] = (v.y - mean) * rstd;
+          y[4 * h + 2] = (v.z - mean) * rstd;
+          y[4 * h + 3] = (v.w - mean) * rstd;
+          if (!nrm.rms) {
+            const float4 ww = reinterpret_cast<const float4*>(nrm.w)[2 * c8 + h];
+            const float4 bb = reinterpret_cast<const float4*>(nrm.b)[2 * c8 + h];
+            y[4 * h + 0] = y[4 * h + 0] * ww.x + bb.x;
+            y[4 * h + 1] = y[4 * h + 1] * ww.y + bb.y;
+            y[4 * h + 2] = y[4 * h + 2] * ww.z + bb.z;
+            y[4 * h + 3] = y[4 * h + 3] * ww.w + bb.w;
+          }
+        }
+        uint4 o;
+        uint32_t* ow = reinterpret_cast<uint32_t*>(&o);
+#pragma unroll
+        for (int k = 0; k < 4; k++) {
+          __nv_bfloat162 p2;
+          p2.x = __float2bfloat16_rn(y[2 * k]);
+          p2.y = __float2bfloat16_rn(y[2 * k + 1]);
+          ow[k] = *reinterpret_cast<uint32_t*>(&p2);
+        }
+        *reinterpret_cast<uint4*>(srow + 16 * c8) = o;
+      }
+    }
+  } else {
+    // activations -> shared memory, rows M .. 8 NT - 1 zero; eight 16-byte
+    // loads per thread in flight before their stores
     const bf16* A = reinterpret_cast<const bf16*>(g.A);
     const int cpr = g.K >> 3;  // 16-byte chunks per row
     const int total = 8 * NT * cpr;
@@ -175,7 +240,7 @@ size_t skinny_smem(const GemmDesc& g, int ks) {
 }
 
 template <int NT>
-void launch_skinny(Ctx& c, const GemmDesc& g) {
+void launch_skinny(Ctx& c, const GemmDesc& g, const SkinnyNorm& nrm) {
   const int ks = skinny_ks(g, c.num_sms);
   const int cw = SK_WARPS / ks, groups = (g.N + 15) / 16;
   const int pitch = skinny_pitch(g.K);
@@ -196,9 +261,9 @@ void launch_skinny(Ctx& c, const GemmDesc& g) {
   pdl[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = pdl;
   cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, k_gemm_skinny<NT>, g, ks, pitch) != cudaSuccess) {
+  if (cudaLaunchKernelEx(&cfg, k_gemm_skinny<NT>, g, nrm, ks, pitch) != cudaSuccess) {
     cudaGetLastError();  // programmatic serialization refused: an ordinary launch
-    k_gemm_skinny<NT><<<cfg.gridDim, cfg.blockDim, smem, c.stream>>>(g, ks, pitch);
+    k_gemm_skinny<NT><<<cfg.gridDim, cfg.blockDim, smem, c.stream>>>(g, nrm, ks, pitch);
   }
 }
 
@@ -212,9 +277,16 @@ bool gemm_skinny_supported(const GemmDesc& g) {
   return skinny_smem(g, SK_WARPS) <= (size_t)SK_MAX_SMEM;
 }
 
-void gemm_skinny_bf16(Ctx& c, const GemmDesc& g) {
-  if (g.M > 8) launch_skinny<2>(c, g);
-  else launch_skinny<1>(c, g);
+bool skinny_norm_supported(const GemmDesc& g, const SkinnyNorm& n) {
+  auto al = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; };
+  return n.x && al(n.x) && (n.ldx % 4) == 0 && n.ldx >= g.K && (n.rms || (n.w && n.b && al(n.w) && al(n.b)));
+}
+
+void gemm_skinny_bf16(Ctx& c, const GemmDesc& g, const SkinnyNorm* nrm) {
+  const SkinnyNorm none{};
+  const SkinnyNorm& n = nrm ? *nrm : none;
+  if (g.M > 8) launch_skinny<2>(c, g, n);
+  else launch_skinny<1>(c, g, n);
 }
 
 }  // namespace gpt

@@ -87,9 +87,20 @@ TcPlan gemm_tc_plan(long M, long N, long K, bool split_ok, int num_sms);
 void gemm_simt_f32(Ctx& c, const GemmDesc& g);
 void gemm_simt_bf16(Ctx& c, const GemmDesc& g);
 bool gemm_tc_supported(const GemmDesc& g);
-// GEMMs of at most 16 rows (decoding): bf16, both operands K-major, no split-K
+// GEMMs of at most 16 rows (decoding): bf16, both operands K-major, no split-K.
+// With a SkinnyNorm, A is not read: the kernel computes it as the norm of the
+// fp32 rows x [M, ldx] over K columns (LayerNorm with w, b; RMSNorm without).
+struct SkinnyNorm {
+  const float* x = nullptr;
+  const float* w = nullptr;
+  const float* b = nullptr;
+  long ldx = 0;
+  int rms = 0;
+  float eps = 1e-5f;
+};
 bool gemm_skinny_supported(const GemmDesc& g);
-void gemm_skinny_bf16(Ctx& c, const GemmDesc& g);
+bool skinny_norm_supported(const GemmDesc& g, const SkinnyNorm& n);
+void gemm_skinny_bf16(Ctx& c, const GemmDesc& g, const SkinnyNorm* nrm = nullptr);
 bool gemm_tc_bf16(Ctx& c, const GemmDesc& g);  // false: tensor-map encode failed
 // the split-K count gemm_tc_bf16 uses for g (1: none)
 int gemm_tc_splits(const GemmDesc& g, int num_sms);

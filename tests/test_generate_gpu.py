@@ -50,10 +50,12 @@ def oracle_logits(oc, P, prefix):
 
 
 @pytest.mark.parametrize("wname,precision,tol", [("char", "bf16", 0.05), ("char", "fp32", 1e-4),
-                                                  ("micro", "fp32", 1e-4)])
+                                                  ("micro", "fp32", 1e-4), ("micro64", "bf16", 0.05)])
 def test_greedy_generation_matches_oracle(wname, precision, tol):
     w = (W.CHAR if wname == "char" else W.MICRO).with_(precision=precision)
-    over = dict(n_layer=2, batch_size=4, block_size=128) if wname == "char" else {}
+    # micro64: the RMSNorm variant wide enough for the decoding GEMM that computes the norm itself
+    over = {"char": dict(n_layer=2, batch_size=4, block_size=128), "micro": {},
+            "micro64": dict(n_layer=2, n_embd=64, n_head=4)}[wname]
     m, cfg, P, oc = setup(w, **over)
     T0, n_new = (9, 20) if wname == "char" else (4, 12)
     seq, _ = generate(m, cfg, T0, n_new, 0.0, 0, 1.0, seed=1)
