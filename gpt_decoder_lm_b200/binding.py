@@ -35,7 +35,7 @@ class GptConfig(C.Structure):
         ("batch_size", C.c_int32), ("grad_accum", C.c_int32), ("precision", C.c_int32), ("variant", C.c_int32),
         ("token_dtype", C.c_int32), ("dropout", C.c_float), ("beta1", C.c_float),
         ("beta2", C.c_float), ("eps", C.c_float), ("weight_decay", C.c_float), ("grad_clip", C.c_float),
-        ("decay_1d", C.c_int32), ("reserved0", C.c_int32), ("dropout_seed", C.c_uint64),
+        ("decay_1d", C.c_int32), ("recompute", C.c_int32), ("dropout_seed", C.c_uint64),
         ("init_std", C.c_double),
     ]
 

@@ -100,6 +100,7 @@ struct gpt_model {
   int V, Vp, L, H, d, T, B, ga, hd;
   long M;
   bool bf16m, micro;
+  bool rc;     // activation recompute: one slot of per-layer activations
   size_t asz;  // bytes per activation element (2 bf16 / 4 fp32)
   std::vector<TensorRec> tensors;
   std::vector<LayerP> layers;
@@ -226,6 +227,7 @@ gpt_status validate(const gpt_config* c, std::string* why) {
   if (!(c->dropout >= 0.f && c->dropout < 1.f)) return bad("dropout must be in [0, 1)");
   if (!(c->beta1 >= 0.f && c->beta1 < 1.f && c->beta2 >= 0.f && c->beta2 < 1.f)) return bad("betas in [0, 1)");
   if (!(c->eps > 0.f) || !(c->init_std >= 0.0)) return bad("eps > 0 and init_std >= 0 required");
+  if (c->recompute != 0 && c->recompute != 1) return bad("recompute must be 0 or 1");
   return GPT_OK;
 }
 
@@ -328,6 +330,7 @@ void derive(gpt_model& m, const gpt_config* c) {
   m.M = (long)m.B * m.T;
   m.bf16m = c->precision == GPT_PREC_BF16;
   m.micro = c->variant == GPT_VARIANT_MICRO;
+  m.rc = c->recompute != 0;
   m.asz = m.bf16m ? 2 : 4;
   build_tensors(m);
 }
@@ -347,18 +350,19 @@ size_t carve(gpt_model& m, uint8_t* base) {
   m.am = F(P);
   m.av = F(P);
   m.wb = m.bf16m ? (bf16*)(base + lay.take(P * 2)) : nullptr;
+  const int La = m.rc ? 1 : L;  // slots of the recomputable activations
   m.res = F((size_t)(2 * L + 1) * M * d);
-  m.ln1 = Bt((size_t)L * M * d);
+  m.ln1 = Bt((size_t)La * M * d);
   m.ln1_mean = F((size_t)L * M);
   m.ln1_rstd = F((size_t)L * M);
-  m.qkv = Bt((size_t)L * M * 3 * d);
-  m.atto = Bt((size_t)L * M * d);
+  m.qkv = Bt((size_t)La * M * 3 * d);
+  m.atto = Bt((size_t)La * M * d);
   m.lse = F((size_t)L * M * m.H);
-  m.ln2 = Bt((size_t)L * M * d);
+  m.ln2 = Bt((size_t)La * M * d);
   m.ln2_mean = F((size_t)L * M);
   m.ln2_rstd = F((size_t)L * M);
-  m.fch = Bt((size_t)L * M * 4 * d);
-  m.fcg = Bt((size_t)L * M * 4 * d);
+  m.fch = Bt((size_t)La * M * 4 * d);
+  m.fcg = Bt((size_t)La * M * 4 * d);
   m.lnf = Bt((size_t)M * d);
   m.lnf_mean = F(M);
   m.lnf_rstd = F(M);
@@ -529,15 +533,16 @@ gpt_status forward_t(gpt_model* m, bool fuse_ce_grad, float* loss_acc, float los
   embed_fwd<T>(c, m->idx, m->P(m->wte), m->P(m->wpe), m->res, m->B, m->T, d, dkey(m, L, 0));
   for (int l = 0; l < L; l++) {
     const LayerP& y = m->layers[l];
+    const size_t sl = m->rc ? 0 : l;  // activation slot
     float* x = m->res + (size_t)(2 * l) * Md;
     float* xm = m->res + (size_t)(2 * l + 1) * Md;
     float* xo = m->res + (size_t)(2 * l + 2) * Md;
-    T* a1 = at<T>(m->ln1, l * Md);
-    T* qkv = at<T>(m->qkv, l * 3 * Md);
-    T* o = at<T>(m->atto, l * Md);
-    T* a2 = at<T>(m->ln2, l * Md);
-    T* h = at<T>(m->fch, l * 4 * Md);  // act'(fc pre-activation), for the backward
-    T* gg = at<T>(m->fcg, l * 4 * Md);
+    T* a1 = at<T>(m->ln1, sl * Md);
+    T* qkv = at<T>(m->qkv, sl * 3 * Md);
+    T* o = at<T>(m->atto, sl * Md);
+    T* a2 = at<T>(m->ln2, sl * Md);
+    T* h = at<T>(m->fch, sl * 4 * Md);  // act'(fc pre-activation), for the backward
+    T* gg = at<T>(m->fcg, sl * 4 * Md);
     norm_fwd<T>(c, x, rms ? nullptr : m->P(y.ln1_w), rms ? nullptr : m->P(y.ln1_b), a1, m->ln1_mean + l * M,
                 m->ln1_rstd + l * M, M, d, rms, eps);
     GemmDesc g = gd((int)M, 3 * d, d, a1, d, true, m->Wop(y.qkv_w), d, true);
@@ -603,6 +608,52 @@ gpt_status forward_t(gpt_model* m, bool fuse_ce_grad, float* loss_acc, float los
 void add_bias_grads_from_norm(gpt_model* m, const float* part, int64_t gain, int64_t beta, int64_t next_bias) {
   partial_reduce3(m->ctx, part, m->part_blocks, m->d, gain >= 0 ? m->G(gain) : nullptr,
                   beta >= 0 ? m->G(beta) : nullptr, next_bias >= 0 ? m->G(next_bias) : nullptr);
+}
+
+// Activation recompute of layer l into the single activation slot: the
+// layer's forward from its stored residual inputs, minus the two projection
+// GEMMs whose outputs are those residuals.  The same kernels on the same
+// inputs (dropout keys included) as the forward, so the activations are
+// bit-identical to the ones the forward wrote.
+template <typename T>
+gpt_status recompute_layer(gpt_model* m, int l) {
+  Ctx& c = m->ctx;
+  const long M = m->M;
+  const int d = m->d;
+  const bool rms = m->micro;
+  const float eps = 1e-5f;
+  const int act = m->micro ? ACT_RELU : ACT_GELU;
+  const size_t Md = (size_t)M * d;
+  const LayerP& y = m->layers[l];
+  T* a1 = at<T>(m->ln1, 0);
+  T* qkv = at<T>(m->qkv, 0);
+  T* o = at<T>(m->atto, 0);
+  T* a2 = at<T>(m->ln2, 0);
+  norm_fwd<T>(c, m->res + (size_t)(2 * l) * Md, rms ? nullptr : m->P(y.ln1_w), rms ? nullptr : m->P(y.ln1_b), a1,
+              m->ln1_mean + l * M, m->ln1_rstd + l * M, M, d, rms, eps);
+  GemmDesc g = gd((int)M, 3 * d, d, a1, d, true, m->Wop(y.qkv_w), d, true);
+  g.epi.kind = EPI_BIAS;
+  g.name = "gemm_qkv_recompute";
+  g.epi.bias = y.qkv_b >= 0 ? m->P(y.qkv_b) : nullptr;
+  g.epi.out = qkv;
+  g.epi.ldo = 3 * d;
+  if (!gemm(m, g)) return fail(m, GPT_ERR_CUDA, "qkv recompute gemm failed");
+  AttnDesc ad{m->B, m->T, m->H, m->hd, qkv, o, m->lse + (size_t)l * M * m->H, nullptr, nullptr, nullptr,
+              dkey(m, l, 1)};
+  if (sizeof(T) == 2 && attn_tc_supported(ad)) attn_fwd_tc(c, ad);
+  else attn_fwd_simt<T>(c, ad);
+  norm_fwd<T>(c, m->res + (size_t)(2 * l + 1) * Md, rms ? nullptr : m->P(y.ln2_w), rms ? nullptr : m->P(y.ln2_b),
+              a2, m->ln2_mean + l * M, m->ln2_rstd + l * M, M, d, rms, eps);
+  g = gd((int)M, 4 * d, d, a2, d, true, m->Wop(y.fc_w), d, true);
+  g.epi.kind = EPI_BIAS_ACT;
+  g.name = "gemm_fc_recompute";
+  g.epi.act = act;
+  g.epi.bias = y.fc_b >= 0 ? m->P(y.fc_b) : nullptr;
+  g.epi.out = at<T>(m->fch, 0);
+  g.epi.out2 = at<T>(m->fcg, 0);
+  g.epi.ldo = 4 * d;
+  if (!gemm(m, g)) return fail(m, GPT_ERR_CUDA, "fc recompute gemm failed");
+  return GPT_OK;
 }
 
 template <typename T>
@@ -684,12 +735,18 @@ gpt_status backward_t(gpt_model* m) {
   if (last) add_bias_grads_from_norm(m, nb.part, m->lnf_w, m->lnf_b, m->layers[L - 1].pr_b);
   for (int l = L - 1; l >= 0; l--) {
     const LayerP& y = m->layers[l];
-    T* a1 = at<T>(m->ln1, l * Md);
-    T* qkv = at<T>(m->qkv, l * 3 * Md);
-    T* o = at<T>(m->atto, l * Md);
-    T* a2 = at<T>(m->ln2, l * Md);
-    T* h = at<T>(m->fch, l * 4 * Md);
-    T* gg = at<T>(m->fcg, l * 4 * Md);
+    // with recompute the slot still holds the last layer's forward activations
+    if (m->rc && l != L - 1) {
+      const gpt_status rs = recompute_layer<T>(m, l);
+      if (rs != GPT_OK) return rs;
+    }
+    const size_t sl = m->rc ? 0 : l;
+    T* a1 = at<T>(m->ln1, sl * Md);
+    T* qkv = at<T>(m->qkv, sl * 3 * Md);
+    T* o = at<T>(m->atto, sl * Md);
+    T* a2 = at<T>(m->ln2, sl * Md);
+    T* h = at<T>(m->fch, sl * 4 * Md);
+    T* gg = at<T>(m->fcg, sl * 4 * Md);
     // MLP projection
     if (!dW(d, 4 * d, dyb, gg, m->G(y.pr_w), "gemm_mlpproj_dw", l * 4 + 0))
       return fail(m, GPT_ERR_CUDA, "proj dW failed");
@@ -1230,6 +1287,7 @@ gpt_status gpt_generate(gpt_model* m, const int32_t* d_prompt, int32_t T0, int32
   if (!m || !d_prompt || !d_uniform || !d_out) return fail(m, GPT_ERR_INVALID_ARG, "generate: null argument");
   if (T0 < 1 || n_new < 1 || (long)T0 + n_new > m->T)
     return fail(m, GPT_ERR_INVALID_ARG, "generate: need 1 <= prompt length and prompt + new tokens <= block_size");
+  if (m->rc) return fail(m, GPT_ERR_UNSUPPORTED, "generate: the key / value cache needs recompute = 0");
   Ctx& c = m->ctx;
   // A repeated call shape (same buffers, lengths and sampling parameters)
   // replays a CUDA graph of the whole call: the first call runs eagerly, the

@@ -105,7 +105,16 @@ typedef struct gpt_config {
                              decay_1d != 0                                           */
   float grad_clip;        /* global-norm clip threshold; <= 0 disables clipping      */
   int32_t decay_1d;
-  int32_t reserved0;
+  int32_t recompute;      /* 0: keep every layer's activations for the backward.
+                             1: activation recompute (checkpointing): per layer only
+                             the residual stream, the norm statistics and the
+                             attention LSE are kept; the backward re-runs each
+                             layer's norms, QKV GEMM, attention forward and fc GEMM
+                             from them before that layer's backward.  Results are
+                             bit-identical to 0; the workspace holds one layer of
+                             the other activations instead of L (14 M d elements
+                             of the operand type per layer saved); gpt_generate is
+                             GPT_ERR_UNSUPPORTED (its cache is those activations). */
   uint64_t dropout_seed;  /* key of the dropout counter hash                         */
   double init_std;        /* std of the Gaussian init of matrices and embeddings
                              (double: the init is computed in double precision and

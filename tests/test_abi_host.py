@@ -71,3 +71,22 @@ def test_null_arguments(lib):
     assert gb.STATUS[lib.gpt_create(C.byref(cfg), 1, None, 0, None, C.byref(out))] == "GPT_ERR_INVALID_ARG"
     assert lib.gpt_param_count(None) == 0
     assert lib.gpt_status_string(0) == b"ok"
+
+
+@pytest.mark.parametrize("w", [W.GPT2_124M, W.CHAR, W.MICRO], ids=["gpt2_124m", "char", "micro"])
+def test_recompute_workspace_saving(lib, w):
+    """Activation recompute keeps one layer of the norms' outputs, qkv, the
+    attention output and both fc outputs (14 M d operand-type elements per
+    layer) instead of L of them; everything else is laid out as before."""
+    full = gb.workspace_bytes(gb.make_config(w))
+    rc = gb.workspace_bytes(gb.make_config(w, recompute=1))
+    M, d, L = w.batch_size * w.block_size, w.n_embd, w.n_layer
+    esz = 2 if w.precision == "bf16" else 4
+    saved = (L - 1) * 14 * M * d * esz
+    assert abs((full - rc) - saved) <= 6 * 256, (full - rc, saved)  # six buffers, 256-byte granules
+
+
+def test_recompute_flag_validated(lib):
+    cfg = gb.make_config(W.CHAR, recompute=2)
+    n = C.c_size_t()
+    assert gb.STATUS[lib.gpt_workspace_bytes(C.byref(cfg), C.byref(n))] == "GPT_ERR_CONFIG"

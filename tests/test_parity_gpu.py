@@ -293,3 +293,31 @@ def test_graph_replay_reports_token_errors():
     with pytest.raises(gb.GptError) as e:
         m.train_step_host(np.ascontiguousarray(idx, np.int32), np.ascontiguousarray(tgt, np.int32), 1e-3, 4)
     assert e.value.name == "GPT_ERR_TOKEN_RANGE"
+
+
+@pytest.mark.parametrize("wname", ["char", "dropout", "micro"])
+def test_recompute_bit_identical(wname):
+    # Activation recompute re-runs each layer's norms, QKV GEMM, attention
+    # forward and fc GEMM in the backward with the forward's kernels, inputs
+    # and dropout keys: losses, norms and weights over several accumulated
+    # steps must equal the stored-activation run bit for bit.
+    w, over = {"char": (W.CHAR, dict(n_layer=3, batch_size=4, block_size=128, grad_accum=2)),
+               "dropout": (W.DROPOUT_512, dict(n_layer=3, batch_size=2, block_size=128, grad_accum=2)),
+               "micro": (W.MICRO, dict(n_layer=3))}[wname]
+    sd = dev(W.token_stream(w, n=1 << 16).astype(np.int32))
+    res = []
+    for rc in (0, 1):
+        m, cfg = make(w, recompute=rc, token_dtype=gb.GPT_TOK_I32, **over)
+        out = [m.train_step(sd, w.data_seed, 1e-3, step) for step in range(1, 4)]
+        res.append((out, _weights(m)))
+        if rc:
+            prompt = torch.zeros((cfg.batch_size, 2), dtype=torch.int32, device="cuda")
+            U = torch.zeros((2, cfg.batch_size), device="cuda")
+            o = torch.empty((cfg.batch_size, 4), dtype=torch.int32, device="cuda")
+            with pytest.raises(gb.GptError) as e:
+                m.generate(prompt, 2, 1.0, 0, 1.0, U, o)
+            assert e.value.name == "GPT_ERR_UNSUPPORTED"
+        m.close()
+    (l0, w0), (l1, w1) = res
+    assert l0 == l1
+    assert np.array_equal(w0, w1)
