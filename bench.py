@@ -254,6 +254,41 @@ def measure_decode(model, w, stream_host, dev, rank):
                          "note": "one decoding step (weights once + the rows' keys / values) at mean position"}}
 
 
+def measure_recompute(w, d_stream, data_seed, dev, warmup):
+    """The same training step with activation recompute (each layer's norms,
+    QKV GEMM, attention forward and fc GEMM re-run in the backward): device
+    time over 5 graph-replayed steps with the L2 flush between them, and the
+    workspace with and without recompute."""
+    import torch
+
+    from gpt_decoder_lm_b200 import binding as gb
+
+    cfg = gb.make_config(w, recompute=1)
+    m = gb.Model(cfg, seed=w.weight_seed, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    st = 0
+    for _ in range(max(warmup, 3)):
+        st += 1
+        m.train_step(d_stream, data_seed, 1e-4, st, sync=False)
+        flush.zero_()
+    torch.cuda.synchronize()
+    n = 5
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(n):
+        st += 1
+        m.train_step(d_stream, data_seed, 1e-4, st, sync=False)
+        flush.zero_()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / n
+    m.close()
+    del m
+    return {"ms_per_step": ms, "tokens_per_s": w.tokens_per_step / (ms / 1000.0), "steps": n,
+            "workspace_gb": gb.workspace_bytes(cfg) / 1e9,
+            "workspace_gb_stored": gb.workspace_bytes(gb.make_config(w)) / 1e9}
+
+
 def run_ours(args, w, rank, world, local_rank):
     import torch
     import torch.distributed as dist
@@ -353,6 +388,7 @@ def run_ours(args, w, rank, world, local_rank):
     e2e_value = world * args.steps * tok_step / (e2e_ms / 1000.0)
 
     decode = measure_decode(model, w, stream_host, dev, rank)
+    recompute = measure_recompute(w, d_stream, data_seed, dev, args.warmup)
 
     pk = peaks()
     gemm_names = [k for k in kt if k.startswith("gemm")]
@@ -393,6 +429,7 @@ def run_ours(args, w, rank, world, local_rank):
             "mfu": {"nominal_2250": mfu_nom, "measured_peak": mfu_meas, "flops_per_token": fpt},
             "roofline": roofline,
             "decode": decode,
+            "recompute": recompute,
             "cpu_baseline": cpu,
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": 2 * ga * B * T * 4,
                     "d2h_bytes_per_step": 16},

@@ -192,9 +192,12 @@ class Model:
         self.M = cfg.batch_size * cfg.block_size
 
     def close(self):
-        if getattr(self, "h", None):
-            lib().gpt_destroy(self.h)
+        h = getattr(self, "h", None)
+        if h:
             self.h = None
+            f = globals().get("lib")  # None while the interpreter shuts down
+            if f is not None:
+                f().gpt_destroy(h)
 
     __del__ = close
 
