@@ -56,3 +56,13 @@ def test_flop_accounting():
     assert abs(bench.flops_per_token(w) - 855_166_464) < 1
     d, L, V, M = 768, 12, 50257, 12 * 1024
     assert bench.gemm_flops_per_step(w) == 3 * 5 * 2 * M * (L * 12 * d * d + V * d)
+
+
+def test_decode_bytes_accounting():
+    # GPT-2 124M: 12 layers x 12 d^2 bf16 weights + the padded tied head, plus
+    # keys and values (2 x d bf16 per position, layer and row) up to pos
+    w = W.GPT2_124M
+    weights = 2 * (12 * 12 * 768 * 768 + 50304 * 768)
+    assert bench.decode_bytes_per_step(w, 0) == weights + 2 * 2 * 768 * 1 * 12 * 12
+    assert bench.decode_bytes_per_step(w, 95.0) == weights + 2 * 2 * 768 * 96 * 12 * 12
+    assert abs(bench.decode_bytes_per_step(w, 96.0) - 290_045_952) < 1  # the bench line's per_step_bytes
