@@ -23,6 +23,7 @@ GPT_PREC_FP32, GPT_PREC_BF16 = 0, 1
 GPT_VARIANT_GPT2, GPT_VARIANT_MICRO = 0, 1
 GPT_TOK_I32, GPT_TOK_U16 = 0, 1
 GPT_PARAM, GPT_GRAD, GPT_ADAM_M, GPT_ADAM_V = 0, 1, 2, 3
+GPT_PATH_GEMM_TC, GPT_PATH_ATTN_TC = 1, 2
 STATUS = ["GPT_OK", "GPT_ERR_INVALID_ARG", "GPT_ERR_CONFIG", "GPT_ERR_WORKSPACE_TOO_SMALL", "GPT_ERR_CUDA",
           "GPT_ERR_TOKEN_RANGE", "GPT_ERR_NONFINITE", "GPT_ERR_STATE", "GPT_ERR_UNSUPPORTED", "GPT_ERR_TIMEOUT"]
 FLAG_TOKEN, FLAG_LOSS, FLAG_NORM, FLAG_TIMEOUT = 1, 2, 4, 8
@@ -51,6 +52,7 @@ _lib = None
 P, I32, I64, U32, U64, F32, SZ = C.c_void_p, C.c_int32, C.c_int64, C.c_uint32, C.c_uint64, C.c_float, C.c_size_t
 _PROTOS = {
     "gpt_param_count": (SZ, [P]),
+    "gpt_config_kernel_paths": (I32, [P, P]),
     "gpt_workspace_bytes": (I32, [P, P]),
     "gpt_lr_cosine": (F32, [F32, I32, I32, I32]),
     "gpt_lr_linear": (F32, [F32, I32, I32]),
@@ -91,6 +93,7 @@ _PROTOS = {
     "gpt_test_gemm": (I32, [I32, I32, I32, I32, P, I64, I32, P, I64, I32, I32, I32, P, P, I32, P, P, P, P, I32, P,
                             P, P]),
     "gpt_test_attention": (I32, [I32, I32, I32, I32, I32, I32, I32, P, P, P, P, P, P, F32, U64, U64, I32, P, P]),
+    "gpt_test_wait_timeout": (I32, [U64, P, P, P]),
     "gpt_gemm_dw_accumulate_noalloc": (I32, [I32, I32, I32, P, I64, P, I64, P, I32, P]),
 }
 
@@ -154,6 +157,13 @@ def make_config(w, **over) -> GptConfig:
     for k, v in d.items():
         setattr(c, k, v)
     return c
+
+
+def kernel_paths(cfg: GptConfig) -> int:
+    """GPT_PATH_* bits: which kernels a model with this config runs."""
+    n = C.c_uint32(0)
+    _check(lib().gpt_config_kernel_paths(C.byref(cfg), C.byref(n)), None, "config_kernel_paths")
+    return int(n.value)
 
 
 def param_count(cfg: GptConfig) -> int:
@@ -370,3 +380,9 @@ def test_attention(backend, backward, dtype, B, T, H, hd, qkv, o, lse, dout=None
     return int(lib().gpt_test_attention(backend, backward, dtype, B, T, H, hd, _ptr(qkv), _ptr(o), _ptr(lse),
                                         _ptr(dout), _ptr(dqkv), _ptr(dsum), p, seed, counter, layer, stream,
                                         _ptr(flags)))
+
+
+def test_wait_timeout(limit_ns: int, flags, gave_up, stream=None) -> int:
+    """The kernels' bounded mbarrier wait with a short limit, on a barrier
+    nothing arrives at; returns the status code."""
+    return int(lib().gpt_test_wait_timeout(limit_ns, stream, _ptr(flags), _ptr(gave_up)))

@@ -24,23 +24,60 @@ GPT_HD uint64_t splitmix64(uint64_t x) {
 
 // Dropout sites (GPT-2 placement): 0 embedding output (layer = n_layer),
 // 1 attention probabilities, 2 attention projection output, 3 MLP output.
+// The key of a site is splitmix64(seed ^ splitmix64(counter<<32 ^ layer<<8 ^
+// site)) with counter = step * grad_accum + micro.  Eagerly launched kernels
+// get it computed on the host; kernels of a replayed CUDA graph get step_dev
+// (the step index the replay writes to device memory) and derive the key
+// from it with drop_live(), so one captured step serves every step.
 struct DropKey {
-  uint64_t key;      // splitmix64(seed ^ splitmix64(counter<<32 ^ layer<<8 ^ site))
+  uint64_t key;      // the site's key (valid when step_dev is null)
   uint32_t thresh;   // floor(p * 2^32); keep iff hash >> 32 >= thresh
   float scale;       // 1 / (1 - p)
   int active;
+  int micro, ga;     // counter = (*step_dev) * ga + micro
+  uint64_t seed, tag;  // tag = layer<<8 ^ site
+  const int* step_dev;
 };
+
+GPT_HD uint64_t drop_site_key(uint64_t seed, uint64_t counter, uint64_t tag) {
+  return splitmix64(seed ^ splitmix64((counter << 32) ^ tag));
+}
 
 GPT_HD DropKey make_drop_key(uint64_t seed, uint64_t counter, int layer, int site, float p) {
   DropKey k;
-  uint64_t tag = (counter << 32) ^ ((uint64_t)layer << 8) ^ (uint64_t)site;
-  k.key = splitmix64(seed ^ splitmix64(tag));
+  k.tag = ((uint64_t)layer << 8) ^ (uint64_t)site;
+  k.seed = seed;
+  k.key = drop_site_key(seed, counter, k.tag);
   double t = (double)p * 4294967296.0;
   k.thresh = (uint32_t)(t >= 4294967295.0 ? 4294967295.0 : t);
   k.scale = p > 0.f ? 1.0f / (1.0f - p) : 1.0f;
   k.active = p > 0.f;
+  k.micro = 0;
+  k.ga = 1;
+  k.step_dev = nullptr;
   return k;
 }
+
+// the key of a replayed graph's kernel: counter from the device step index
+inline DropKey make_drop_key_dev(uint64_t seed, const int* step_dev, int ga, int micro, int layer, int site,
+                                 float p) {
+  DropKey k = make_drop_key(seed, 0, layer, site, p);
+  k.step_dev = step_dev;
+  k.ga = ga;
+  k.micro = micro;
+  return k;
+}
+
+#ifdef __CUDACC__
+__device__ __forceinline__ DropKey drop_live(DropKey k) {
+  if (k.active && k.step_dev) {
+    const uint64_t counter = (uint64_t)((int64_t)(*k.step_dev) * k.ga + k.micro);
+    k.key = drop_site_key(k.seed, counter, k.tag);
+    k.step_dev = nullptr;
+  }
+  return k;
+}
+#endif
 
 GPT_HD bool drop_keep(const DropKey& k, uint64_t elem) {
   return (uint32_t)(splitmix64(k.key ^ elem) >> 32) >= k.thresh;

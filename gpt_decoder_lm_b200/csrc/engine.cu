@@ -165,6 +165,8 @@ struct gpt_model {
   uint64_t g_len = 0, g_seed = 0;
   int* step_dev = nullptr;     // per-step scalars read by replayed graphs
   float* hyper_dev = nullptr;  // {lr, 1 - b1^t, 1 - b2^t}
+  bool dev_keys = false;  // dropout keys from the device step index (a graph being captured)
+  bool attn_tc = false;   // attention on the tensor-core kernels (gpt_config_kernel_paths)
   bool have_forward = false;
   bool ce_grad_done = false;
   int64_t drop_counter = 0;
@@ -487,6 +489,10 @@ gpt_status sync_and_flags(gpt_model* m, const char* where, float* h_scal /* 4 fl
 }
 
 // ---------------------------------------------------------------- step pieces
+// fp32 mode: CUDA-core GEMM.  bf16 mode: the tensor-core GEMM, or the
+// decoding GEMM for at most 16 rows; every bf16 shape of a valid config suits
+// one of them, so false means the launch failed (a tensor map that could not
+// be encoded), never a switch to another kernel.
 bool gemm(gpt_model* m, GemmDesc& g) {
   if (!m->bf16m) {
     gemm_simt_f32(m->ctx, g);
@@ -496,9 +502,23 @@ bool gemm(gpt_model* m, GemmDesc& g) {
     gemm_skinny_bf16(m->ctx, g);
     return true;
   }
-  if (gemm_tc_supported(g)) return gemm_tc_bf16(m->ctx, g);
-  gemm_simt_bf16(m->ctx, g);
-  return true;
+  if (!gemm_tc_supported(g)) return false;
+  return gemm_tc_bf16(m->ctx, g);
+}
+
+// causal attention: the tensor-core kernels where the config's shape rule
+// allows them (bf16, head_dim 64, T a multiple of 128), else the CUDA-core
+// kernels; decided once per model, a failed launch is an error
+template <typename T>
+gpt_status attention(gpt_model* m, const AttnDesc& ad, bool backward) {
+  if (m->attn_tc) {
+    const bool ok = attn_tc_supported(ad) && (backward ? attn_bwd_tc(m->ctx, ad) : attn_fwd_tc(m->ctx, ad));
+    if (!ok) return fail(m, GPT_ERR_CUDA, "tensor-core attention could not be launched (tensor map encode failed)");
+    return GPT_OK;
+  }
+  if (backward) attn_bwd_simt<T>(m->ctx, ad);
+  else attn_fwd_simt<T>(m->ctx, ad);
+  return GPT_OK;
 }
 
 GemmDesc gd(int M, int N, int K, const void* A, long lda, bool ak, const void* B, long ldb, bool bk) {
@@ -516,6 +536,8 @@ GemmDesc gd(int M, int N, int K, const void* A, long lda, bool ak, const void* B
 }
 
 DropKey dkey(gpt_model* m, int layer, int site) {
+  if (m->dev_keys)
+    return make_drop_key_dev(m->cfg.dropout_seed, m->step_dev, m->ga, m->cur_micro, layer, site, m->cfg.dropout);
   return make_drop_key(m->cfg.dropout_seed, (uint64_t)m->drop_counter, layer, site, m->cfg.dropout);
 }
 
@@ -554,8 +576,8 @@ gpt_status forward_t(gpt_model* m, bool fuse_ce_grad, float* loss_acc, float los
     if (!gemm(m, g)) return fail(m, GPT_ERR_CUDA, "qkv gemm: tensor map encode failed");
     AttnDesc ad{m->B, m->T, m->H, m->hd, qkv, o, m->lse + (size_t)l * M * m->H, nullptr, nullptr, nullptr,
                 dkey(m, l, 1)};
-    if (sizeof(T) == 2 && attn_tc_supported(ad)) attn_fwd_tc(c, ad);
-    else attn_fwd_simt<T>(c, ad);
+    const gpt_status as = attention<T>(m, ad, false);
+    if (as != GPT_OK) return as;
     g = gd((int)M, d, d, o, d, true, m->Wop(y.ap_w), d, true);
     g.epi.kind = EPI_RESADD;
     g.name = "gemm_attnproj_fwd";
@@ -640,8 +662,8 @@ gpt_status recompute_layer(gpt_model* m, int l) {
   if (!gemm(m, g)) return fail(m, GPT_ERR_CUDA, "qkv recompute gemm failed");
   AttnDesc ad{m->B, m->T, m->H, m->hd, qkv, o, m->lse + (size_t)l * M * m->H, nullptr, nullptr, nullptr,
               dkey(m, l, 1)};
-  if (sizeof(T) == 2 && attn_tc_supported(ad)) attn_fwd_tc(c, ad);
-  else attn_fwd_simt<T>(c, ad);
+  const gpt_status as = attention<T>(m, ad, false);
+  if (as != GPT_OK) return as;
   norm_fwd<T>(c, m->res + (size_t)(2 * l + 1) * Md, rms ? nullptr : m->P(y.ln2_w), rms ? nullptr : m->P(y.ln2_b),
               a2, m->ln2_mean + l * M, m->ln2_rstd + l * M, M, d, rms, eps);
   g = gd((int)M, 4 * d, d, a2, d, true, m->Wop(y.fc_w), d, true);
@@ -787,8 +809,8 @@ gpt_status backward_t(gpt_model* m) {
     g.epi.ldo = d;
     if (!gemm(m, g)) return fail(m, GPT_ERR_CUDA, "attn proj dX failed");
     AttnDesc ad{m->B, m->T, m->H, m->hd, qkv, o, m->lse + (size_t)l * M * m->H, datt, dqkv, m->dsum, dkey(m, l, 1)};
-    if (sizeof(T) == 2 && attn_tc_supported(ad)) attn_bwd_tc(c, ad);
-    else attn_bwd_simt<T>(c, ad);
+    const gpt_status as = attention<T>(m, ad, true);
+    if (as != GPT_OK) return as;
     if (y.qkv_b >= 0) bias_grad(dqkv, 3 * d, l, 1, m->G(y.qkv_b));
     if (!dW(3 * d, d, dqkv, a1, m->G(y.qkv_w), "gemm_qkv_dw", l * 4 + 3))
       return fail(m, GPT_ERR_CUDA, "qkv dW failed");
@@ -986,6 +1008,19 @@ gpt_status gpt_workspace_bytes(const gpt_config* c, size_t* out) {
   return GPT_OK;
 }
 
+gpt_status gpt_config_kernel_paths(const gpt_config* c, uint32_t* out) {
+  if (!out) return GPT_ERR_INVALID_ARG;
+  gpt_status s = validate(c, nullptr);
+  if (s != GPT_OK) return s;
+  uint32_t p = 0;
+  if (c->precision == GPT_PREC_BF16) {
+    p |= GPT_PATH_GEMM_TC;
+    if (attn_tc_shape_ok(c->block_size, c->n_embd / c->n_head)) p |= GPT_PATH_ATTN_TC;
+  }
+  *out = p;
+  return GPT_OK;
+}
+
 float gpt_lr_cosine(float lr, int32_t it, int32_t warmup, int32_t max_iters) {
   if (it < warmup) return (float)((double)lr * it / warmup);
   double r = (double)(it - warmup) / (double)(max_iters - warmup);
@@ -1022,6 +1057,7 @@ gpt_status gpt_create(const gpt_config* cfg, uint64_t seed, void* d_workspace, s
   cudaGetDevice(&dev);
   if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess) m->ctx.num_sms = sms;
   m->part_blocks = std::min(m->part_blocks, norm_bwd_blocks(m->ctx, m->M, m->d, m->bf16m));
+  m->attn_tc = m->bf16m && attn_tc_shape_ok(m->T, m->hd);
   cudaStream_t st = m->ctx.stream;
   // zero the arenas (weights, grads, moments) and the scalars
   cudaMemsetAsync(m->scal, 0, 64 * 4, st);
@@ -1162,7 +1198,9 @@ static bool capture_step(gpt_model* m, int kind, const void* d_stream, uint64_t 
   m->ctx.stream = m->cap_stream;
   cudaGraph_t g = nullptr;
   bool ok = cudaStreamBeginCapture(m->cap_stream, cudaStreamCaptureModeThreadLocal) == cudaSuccess;
+  m->dev_keys = true;  // dropout keys follow the step index the replay writes
   gpt_status s = ok ? train_body(m, d_stream, len, seed, lr, step, true) : GPT_ERR_CUDA;
+  m->dev_keys = false;
   if (ok) ok = cudaStreamEndCapture(m->cap_stream, &g) == cudaSuccess && s == GPT_OK;
   m->ctx.stream = user;
   if (ok) ok = cudaGraphInstantiate(&m->gexec[kind], g, 0) == cudaSuccess;
@@ -1180,12 +1218,13 @@ static gpt_status train_common(gpt_model* m, const void* d_stream, uint64_t len,
                                const int32_t* h_tgt, float lr, int32_t step, float* h_loss, float* h_norm) {
   if (step < 1) return fail(m, GPT_ERR_INVALID_ARG, "step must be >= 1");
   Ctx& c = m->ctx;
-  // Replay a captured graph of the whole step when nothing in it changes from
-  // step to step: no dropout (its masks depend on the step), no per-kernel
-  // timing.  The first call of each kind runs eagerly (one-time kernel
-  // attributes), the second captures, later calls only replay.
+  // Replay a captured graph of the whole step: everything that changes from
+  // step to step (the step index, the learning rate, the bias corrections and
+  // through the step index the dropout keys) is read from device memory.  Not
+  // with per-kernel timing.  The first call of each kind runs eagerly, the
+  // second captures, later calls only replay.
   const int kind = d_stream ? 0 : 1;
-  bool replay = m->graphs_on && m->cfg.dropout == 0.f && !c.timing;
+  bool replay = m->graphs_on && !c.timing;
   if (replay && kind == 0 && m->gexec[0] && (m->g_dstream != d_stream || m->g_len != len || m->g_seed != seed)) {
     cudaGraphExecDestroy(m->gexec[0]);
     m->gexec[0] = nullptr;
@@ -1202,8 +1241,11 @@ static gpt_status train_common(gpt_model* m, const void* d_stream, uint64_t len,
         m->g_seed = seed;
       }
     } else {
-      m->graphs_on = false;  // capture not possible here: run every step eagerly
-      replay = false;
+      // reported, not hidden: the step did not run; the next call tries the
+      // capture again, and gpt_set_graphs(m, 0) runs every step eagerly
+      return fail(m, GPT_ERR_CUDA,
+                  "train_step: capturing the step into a CUDA graph failed (graphs stay on; "
+                  "gpt_set_graphs(m, 0) runs steps eagerly)");
     }
   }
   gpt_status s = GPT_OK;
@@ -1327,8 +1369,12 @@ gpt_status gpt_generate(gpt_model* m, const int32_t* d_prompt, int32_t T0, int32
       if (!ok) {
         cudaGetLastError();
         m->gen_exec = nullptr;
-        replay = false;
-        s = GPT_OK;
+        m->gen_warm = 0;
+        m->have_forward = false;
+        if (s != GPT_OK) return s;
+        return fail(m, GPT_ERR_CUDA,
+                    "generate: capturing the call into a CUDA graph failed (nothing ran; "
+                    "gpt_set_graphs(m, 0) runs calls eagerly)");
       }
     }
   }

@@ -27,7 +27,7 @@ __device__ __forceinline__ void epi_apply(const GemmEpi& e, int N, long m, int n
     }
     case EPI_RESADD: {
       float y = acc + (e.bias ? e.bias[n] : 0.f);
-      y *= drop_mul(e.drop, (uint64_t)m * N + n);
+      if (e.drop.active) y *= drop_mul(drop_live(e.drop), (uint64_t)m * N + n);
       e.res_out[m * e.ld_res + n] = e.res_in[m * e.ld_res + n] + y;
       break;
     }

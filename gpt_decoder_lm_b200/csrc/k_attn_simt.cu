@@ -39,6 +39,7 @@ __device__ __forceinline__ void load_tile(float (*dst)[HD + 1], const T* qkv, in
 template <typename T, int HD>
 __global__ void __launch_bounds__(256) k_attn_fwd(AttnDesc a) {
   pdl_trigger();
+  const DropKey dropk = drop_live(a.drop);
   constexpr int DPT = HD / 4;
   extern __shared__ float smem_f[];
   float(*Ks)[HD + 1] = reinterpret_cast<float(*)[HD + 1]>(smem_f);
@@ -86,7 +87,7 @@ __global__ void __launch_bounds__(256) k_attn_fwd(AttnDesc a) {
     for (int j = 0; j < QB; j++) {
       float p = s[j] == -INFINITY ? 0.f : expf(s[j] - mn);
       l += p;
-      float pd = p * drop_mul(a.drop, ebase + k0 + j);
+      float pd = p * drop_mul(dropk, ebase + k0 + j);
 #pragma unroll
       for (int k = 0; k < DPT; k++) o[k] = fmaf(pd, Vs[j][part * DPT + k], o[k]);
     }
@@ -131,6 +132,7 @@ __device__ __forceinline__ void load_do_tile(float (*dst)[HD + 1], const T* dout
 template <typename T, int HD>
 __global__ void __launch_bounds__(256) k_attn_bwd_kv(AttnDesc a) {
   pdl_trigger();
+  const DropKey dropk = drop_live(a.drop);
   constexpr int DPT = HD / 4;
   extern __shared__ float smem_f[];
   float(*Qs)[HD + 1] = reinterpret_cast<float(*)[HD + 1]>(smem_f);
@@ -176,7 +178,7 @@ __global__ void __launch_bounds__(256) k_attn_bwd_kv(AttnDesc a) {
       dpt = grp4_sum(dpt);
       if (!(valid && qi < a.T && kj <= qi)) continue;
       float p = expf(s * scale - Ls[i]);
-      float mk = drop_mul(a.drop, (((uint64_t)bh) * a.T + qi) * a.T + kj);
+      float mk = drop_mul(dropk, (((uint64_t)bh) * a.T + qi) * a.T + kj);
       float ds = p * (dpt * mk - Dsum[i]);
 #pragma unroll
       for (int k = 0; k < DPT; k++) {
@@ -198,6 +200,7 @@ __global__ void __launch_bounds__(256) k_attn_bwd_kv(AttnDesc a) {
 template <typename T, int HD>
 __global__ void __launch_bounds__(256) k_attn_bwd_q(AttnDesc a) {
   pdl_trigger();
+  const DropKey dropk = drop_live(a.drop);
   constexpr int DPT = HD / 4;
   extern __shared__ float smem_f[];
   float(*Ks)[HD + 1] = reinterpret_cast<float(*)[HD + 1]>(smem_f);
@@ -237,7 +240,7 @@ __global__ void __launch_bounds__(256) k_attn_bwd_q(AttnDesc a) {
       dpt = grp4_sum(dpt);
       if (!(valid && kj <= qi)) continue;
       float p = expf(s * scale - lse);
-      float mk = drop_mul(a.drop, (((uint64_t)bh) * a.T + qi) * a.T + kj);
+      float mk = drop_mul(dropk, (((uint64_t)bh) * a.T + qi) * a.T + kj);
       float ds = p * (dpt * mk - Di);
 #pragma unroll
       for (int k = 0; k < DPT; k++) dq[k] = fmaf(ds * scale, Ks[j][part * DPT + k], dq[k]);
@@ -252,11 +255,8 @@ __global__ void __launch_bounds__(256) k_attn_bwd_q(AttnDesc a) {
 template <typename T, int HD>
 void run_fwd(Ctx& c, const AttnDesc& a) {
   size_t smem = 2 * QB * (HD + 1) * sizeof(float);
-  static bool attr = false;
-  if (!attr) {
-    cudaFuncSetAttribute(k_attn_fwd<T, HD>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    attr = true;
-  }
+  // per-device function attribute: set before every launch
+  cudaFuncSetAttribute(k_attn_fwd<T, HD>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   dim3 grid((a.T + QB - 1) / QB, a.B * a.H);
   LaunchScope s(c, "attn_fwd_simt");
   k_attn_fwd<T, HD><<<grid, 256, smem, c.stream>>>(a);
@@ -272,12 +272,9 @@ void run_bwd(Ctx& c, const AttnDesc& a) {
   dim3 grid((a.T + QB - 1) / QB, a.B * a.H);
   size_t smem_kv = (2 * QB * (HD + 1) + 2 * QB) * sizeof(float);
   size_t smem_q = 2 * QB * (HD + 1) * sizeof(float);
-  static bool attr = false;
-  if (!attr) {
-    cudaFuncSetAttribute(k_attn_bwd_kv<T, HD>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_kv);
-    cudaFuncSetAttribute(k_attn_bwd_q<T, HD>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_q);
-    attr = true;
-  }
+  // per-device function attribute: set before every launch
+  cudaFuncSetAttribute(k_attn_bwd_kv<T, HD>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_kv);
+  cudaFuncSetAttribute(k_attn_bwd_q<T, HD>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_q);
   {
     LaunchScope s(c, "attn_bwd_kv_simt");
     k_attn_bwd_kv<T, HD><<<grid, 256, smem_kv, c.stream>>>(a);

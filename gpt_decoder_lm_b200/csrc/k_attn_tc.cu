@@ -93,6 +93,8 @@ template <bool DROP>
 __global__ void __launch_bounds__(192, 2) k_attn_fwd_o(const __grid_constant__ CUtensorMap tq,
                                                        const __grid_constant__ CUtensorMap tkv64, AttnTcArgs a) {
   pdl_trigger();
+  // the dropout key of this launch (derived from the device step index in a replayed graph)
+  const DropKey dk = DROP ? drop_live(a.drop) : a.drop;
   extern __shared__ __align__(1024) uint8_t smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (smem_u32(smem) & 1023) {  // swizzled tiles need 1024-byte alignment
@@ -264,10 +266,10 @@ __global__ void __launch_bounds__(192, 2) k_attn_fwd_o(const __grid_constant__ C
         ls1 += p2 + p3;
         if (DROP) {
           const uint64_t e = ebase + key0 + i;
-          p0 *= drop_mul(a.drop, e);
-          p1 *= drop_mul(a.drop, e + 1);
-          p2 *= drop_mul(a.drop, e + 32);
-          p3 *= drop_mul(a.drop, e + 33);
+          p0 *= drop_mul(dk, e);
+          p1 *= drop_mul(dk, e + 1);
+          p2 *= drop_mul(dk, e + 32);
+          p3 *= drop_mul(dk, e + 33);
         }
         pk0[i >> 1] = pack2(p0, p1);
         pk1[i >> 1] = pack2(p2, p3);
@@ -345,6 +347,8 @@ __global__ void __launch_bounds__(320, 2) k_attn_bwd_kv8(const __grid_constant__
                                                          const __grid_constant__ CUtensorMap tq64,
                                                          const __grid_constant__ CUtensorMap tdo64, AttnTcArgs a) {
   pdl_trigger();
+  // the dropout key of this launch (derived from the device step index in a replayed graph)
+  const DropKey dk = DROP ? drop_live(a.drop) : a.drop;
   extern __shared__ __align__(1024) uint8_t smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (smem_u32(smem) & 1023) {
@@ -494,7 +498,7 @@ __global__ void __launch_bounds__(320, 2) k_attn_bwd_kv8(const __grid_constant__
           if (DROP) {
 #pragma unroll
             for (int u = 0; u < 4; u++)
-              p4[u] *= drop_mul(a.drop, ((uint64_t)bh * a.T + q0 + c0 + e + u) * a.T + kj);
+              p4[u] *= drop_mul(dk, ((uint64_t)bh * a.T + q0 + c0 + e + u) * a.T + kj);
           }
           pp[e >> 1] = pack2(p4[0], p4[1]);
           pp[(e >> 1) + 1] = pack2(p4[2], p4[3]);
@@ -520,8 +524,8 @@ __global__ void __launch_bounds__(320, 2) k_attn_bwd_kv8(const __grid_constant__
           const float2 d2 = *reinterpret_cast<const float2*>(ld + 64 + c0 + e);
           float dp0 = __uint_as_float(dv[e]), dp1 = __uint_as_float(dv[e + 1]);
           if (DROP) {
-            dp0 *= drop_mul(a.drop, ((uint64_t)bh * a.T + q0 + c0 + e) * a.T + kj);
-            dp1 *= drop_mul(a.drop, ((uint64_t)bh * a.T + q0 + c0 + e + 1) * a.T + kj);
+            dp0 *= drop_mul(dk, ((uint64_t)bh * a.T + q0 + c0 + e) * a.T + kj);
+            dp1 *= drop_mul(dk, ((uint64_t)bh * a.T + q0 + c0 + e + 1) * a.T + kj);
           }
           pd[e >> 1] = pack2v(f2mul(f2(pk[sub][e], pk[sub][e + 1]), f2sub(f2(dp0, dp1), f2(d2.x, d2.y))));
         }
@@ -579,6 +583,8 @@ __global__ void __launch_bounds__(320, 2) k_attn_bwd_q8(const __grid_constant__ 
                                                         const __grid_constant__ CUtensorMap tkv64,
                                                         const __grid_constant__ CUtensorMap tout, AttnTcArgs a) {
   pdl_trigger();
+  // the dropout key of this launch (derived from the device step index in a replayed graph)
+  const DropKey dk = DROP ? drop_live(a.drop) : a.drop;
   extern __shared__ __align__(1024) uint8_t smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (smem_u32(smem) & 1023) {
@@ -743,8 +749,8 @@ __global__ void __launch_bounds__(320, 2) k_attn_bwd_q8(const __grid_constant__ 
         for (int e = 0; e < 16; e += 2) {
           float dp0 = __uint_as_float(dv[e]), dp1 = __uint_as_float(dv[e + 1]);
           if (DROP) {
-            dp0 *= drop_mul(a.drop, ebase + key0 + c0 + e);
-            dp1 *= drop_mul(a.drop, ebase + key0 + c0 + e + 1);
+            dp0 *= drop_mul(dk, ebase + key0 + c0 + e);
+            dp1 *= drop_mul(dk, ebase + key0 + c0 + e + 1);
           }
           pd[e >> 1] = pack2v(f2mul(f2(pk[sub][e], pk[sub][e + 1]), f2sub(f2(dp0, dp1), Dx2)));
         }
@@ -823,8 +829,10 @@ AttnTcArgs make_args(const AttnDesc& d, uint32_t* flags) {
 
 }  // namespace
 
+bool attn_tc_shape_ok(int T, int hd) { return hd == 64 && T > 0 && T % 128 == 0; }
+
 bool attn_tc_supported(const AttnDesc& a) {
-  if (a.hd != 64 || a.T % 128 != 0 || a.T <= 0 || !encode_fn()) return false;
+  if (!attn_tc_shape_ok(a.T, a.hd) || !encode_fn()) return false;
   if ((reinterpret_cast<uintptr_t>(a.qkv) & 15) || (reinterpret_cast<uintptr_t>(a.o) & 15)) return false;
   if (a.dout && (reinterpret_cast<uintptr_t>(a.dout) & 15)) return false;
   if (a.lse && (reinterpret_cast<uintptr_t>(a.lse) & 15)) return false;
@@ -832,46 +840,38 @@ bool attn_tc_supported(const AttnDesc& a) {
   return true;
 }
 
-void attn_fwd_tc(Ctx& c, const AttnDesc& d) {
+// The dynamic shared-memory limit is a per-device function attribute: it is
+// set before every launch (a host-side call, not captured into graphs), so a
+// model on any device of the process gets it.
+bool attn_fwd_tc(Ctx& c, const AttnDesc& d) {
   CUtensorMap tq, tkv64;
   long rows = (long)d.B * d.T;
-  if (!map_rows(&tq, d.qkv, 3 * d.H, rows, 128) || !map_rows(&tkv64, d.qkv, 3 * d.H, rows, 64)) {
-    attn_fwd_simt<bf16>(c, d);
-    return;
-  }
-  static bool attr = false;
-  if (!attr) {
-    cudaFuncSetAttribute(k_attn_fwd_o<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, D_SMEM);
-    cudaFuncSetAttribute(k_attn_fwd_o<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, D_SMEM);
-    attr = true;
-  }
+  if (!map_rows(&tq, d.qkv, 3 * d.H, rows, 128) || !map_rows(&tkv64, d.qkv, 3 * d.H, rows, 64)) return false;
+  const bool drop = d.drop.active;
+  cudaFuncSetAttribute(drop ? k_attn_fwd_o<true> : k_attn_fwd_o<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                       D_SMEM);
   dim3 grid(d.B * d.H, d.T / 128);
   LaunchScope s(c, "attn_fwd_tc");
-  if (d.drop.active) k_attn_fwd_o<true><<<grid, 192, D_SMEM, c.stream>>>(tq, tkv64, make_args(d, c.flags));
+  if (drop) k_attn_fwd_o<true><<<grid, 192, D_SMEM, c.stream>>>(tq, tkv64, make_args(d, c.flags));
   else k_attn_fwd_o<false><<<grid, 192, D_SMEM, c.stream>>>(tq, tkv64, make_args(d, c.flags));
+  return true;
 }
 
-void attn_bwd_tc(Ctx& c, const AttnDesc& d) {
+bool attn_bwd_tc(Ctx& c, const AttnDesc& d) {
   CUtensorMap tkv, tkv64, tq64, tdo, tdo64, tout;
   long rows = (long)d.B * d.T;
   if (!map_rows(&tkv, d.qkv, 3 * d.H, rows, 128) || !map_rows(&tkv64, d.qkv, 3 * d.H, rows, 64) ||
       !map_rows(&tdo, d.dout, d.H, rows, 128) || !map_rows(&tdo64, d.dout, d.H, rows, 64) ||
-      !map_rows(&tout, d.o, d.H, rows, 128)) {
-    attn_bwd_simt<bf16>(c, d);
-    return;
-  }
+      !map_rows(&tout, d.o, d.H, rows, 128))
+    return false;
   tq64 = tkv64;
-  static bool attr = false;
-  if (!attr) {
-    cudaFuncSetAttribute(k_attn_bwd_kv8<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, K_SMEM);
-    cudaFuncSetAttribute(k_attn_bwd_kv8<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, K_SMEM);
-    cudaFuncSetAttribute(k_attn_bwd_q8<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, Q_SMEM);
-    cudaFuncSetAttribute(k_attn_bwd_q8<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, Q_SMEM);
-    attr = true;
-  }
+  const bool drop = d.drop.active;
+  cudaFuncSetAttribute(drop ? k_attn_bwd_kv8<true> : k_attn_bwd_kv8<false>,
+                       cudaFuncAttributeMaxDynamicSharedMemorySize, K_SMEM);
+  cudaFuncSetAttribute(drop ? k_attn_bwd_q8<true> : k_attn_bwd_q8<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                       Q_SMEM);
   AttnTcArgs a = make_args(d, c.flags);
   dim3 grid(d.B * d.H, d.T / 128);
-  const bool drop = d.drop.active;
   {  // dQ first: it also stores D = rowsum(dO * O), which the dK/dV kernel reads
     LaunchScope s(c, "attn_bwd_q_tc");
     if (drop) k_attn_bwd_q8<true><<<grid, 320, Q_SMEM, c.stream>>>(tkv, tdo, tkv64, tout, a);
@@ -882,6 +882,7 @@ void attn_bwd_tc(Ctx& c, const AttnDesc& d) {
     if (drop) k_attn_bwd_kv8<true><<<grid, 320, K_SMEM, c.stream>>>(tkv, tq64, tdo64, a);
     else k_attn_bwd_kv8<false><<<grid, 320, K_SMEM, c.stream>>>(tkv, tq64, tdo64, a);
   }
+  return true;
 }
 
 }  // namespace gpt

@@ -245,11 +245,8 @@ void launch_skinny(Ctx& c, const GemmDesc& g, const SkinnyNorm& nrm) {
   const int cw = SK_WARPS / ks, groups = (g.N + 15) / 16;
   const int pitch = skinny_pitch(g.K);
   const size_t smem = skinny_smem(g, ks);
-  static bool attr = false;
-  if (!attr) {
-    cudaFuncSetAttribute(k_gemm_skinny<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, SK_MAX_SMEM);
-    attr = true;
-  }
+  // per-device function attribute: set before every launch
+  cudaFuncSetAttribute(k_gemm_skinny<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, SK_MAX_SMEM);
   LaunchScope s(c, g.name ? g.name : "gemm_skinny");
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((groups + cw - 1) / cw);

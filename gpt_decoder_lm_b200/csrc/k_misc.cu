@@ -101,6 +101,7 @@ __global__ void k_embed_fwd(const int32_t* __restrict__ idx, const float* __rest
   float4 p = reinterpret_cast<const float4*>(wpe + (long)t * d)[c4];
   float4 r = make_float4(a.x + p.x, a.y + p.y, a.z + p.z, a.w + p.w);
   if (drop.active) {
+    drop = drop_live(drop);
     uint64_t e = (uint64_t)m * d + c4 * 4;
     r.x *= drop_mul(drop, e);
     r.y *= drop_mul(drop, e + 1);
@@ -253,6 +254,7 @@ __global__ void k_norm_bwd(NormBwd p) {
   long r0 = blockIdx.x * per, r1 = min(p.rows, r0 + per);
   float4 gw = make_float4(1.f, 1.f, 1.f, 1.f);
   if (own && !p.rms) gw = reinterpret_cast<const float4*>(p.w)[tid];
+  const DropKey dk = drop_live(p.drop);
   float pg[4] = {0, 0, 0, 0}, pb[4] = {0, 0, 0, 0}, pn[4] = {0, 0, 0, 0};
   int buf = 0;
   const float wv[4] = {gw.x, gw.y, gw.z, gw.w};
@@ -332,7 +334,7 @@ __global__ void k_norm_bwd(NormBwd p) {
         float q[4];
 #pragma unroll
         for (int k = 0; k < 4; k++) {
-          q[k] = nv[k] * drop_mul(p.drop, (uint64_t)rr * p.d + 4 * tid + k);
+          q[k] = nv[k] * drop_mul(dk, (uint64_t)rr * p.d + 4 * tid + k);
           pn[k] += q[k];
         }
         store4<T>(reinterpret_cast<T*>(p.dyb) + rr * p.d + 4 * tid, make_float4(q[0], q[1], q[2], q[3]));
@@ -745,11 +747,8 @@ void embed_sort(Ctx& c, const int32_t* idx, long M, int32_t* sorted_tok, int32_t
   int P2 = 1;
   while (P2 < M) P2 <<= 1;
   size_t smem = (size_t)P2 * 4;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaFuncSetAttribute(k_embed_sort, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
-    attr_set = true;
-  }
+  // per-device function attribute: set before every launch
+  cudaFuncSetAttribute(k_embed_sort, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
   LaunchScope s(c, "embed_sort");
   k_embed_sort<<<batches, 1024, smem, c.stream>>>(idx, (int)M, P2, sorted_tok, sorted_pos, n_unique);
 }
@@ -764,6 +763,7 @@ __global__ void k_embed_bwd_wpe(const float* __restrict__ dres, int Bn, int Tn, 
   long i = (long)blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= (long)Tn * d) return;
   int t = (int)(i / d), c = (int)(i % d);
+  drop = drop_live(drop);
   float acc = 0.f;
   for (int b = 0; b < Bn; b++) {
     long m = (long)b * Tn + t;
@@ -787,6 +787,7 @@ __global__ void __launch_bounds__(256) k_embed_seg_a(const float* __restrict__ d
                                                      float* __restrict__ tail) {
   pdl_trigger();
   __shared__ int s_tok[EC + 2], s_pos[EC];
+  drop = drop_live(drop);
   const int c = blockIdx.x;
   const int j0 = c * EC, j1 = min(M, j0 + EC);
   const int n = j1 - j0;
@@ -837,13 +838,24 @@ __global__ void k_embed_seg_b(const int32_t* __restrict__ stok, int M, int d, co
   int k = j1 - 1;
   while (k > j0 && stok[k - 1] == tok) k--;
   if (k == j0 && j0 > 0 && stok[j0 - 1] == tok) return;  // began earlier: its start chunk sums it
+  // the last chunk cend whose head belongs to the segment: the first chunk
+  // after c at whose end the token changes (or the stream ends), found by all
+  // threads at once rather than one chunk after another
+  __shared__ int s_end;
+  const int nch = (M + EC - 1) / EC;
+  if (threadIdx.x == 0) s_end = nch;
+  __syncthreads();
+  for (int cc = c + 1 + threadIdx.x; cc < nch; cc += blockDim.x) {
+    const int e = min(M, (cc + 1) * EC);
+    if (e >= M || stok[e] != tok) atomicMin(&s_end, cc);
+  }
+  __syncthreads();
+  const int cend = s_end < nch ? s_end : c;  // (the segment continues past c, so a later chunk ends it)
   for (int col = threadIdx.x; col < d; col += blockDim.x) {
     float s = tail[(long)c * d + col];
-    for (int cc = c + 1; cc * EC < M; cc++) {
-      s += head[(long)cc * d + col];
-      const int e = min(M, (cc + 1) * EC);
-      if (e >= M || stok[e] != tok) break;
-    }
+    // the heads of chunks c+1 .. cend, added in chunk order (independent loads)
+#pragma unroll 4
+    for (int cc = c + 1; cc <= cend; cc++) s += head[(long)cc * d + col];
     dwte[(long)tok * d + col] += s;
   }
 }

@@ -87,6 +87,8 @@ TcPlan gemm_tc_plan(long M, long N, long K, bool split_ok, int num_sms);
 void gemm_simt_f32(Ctx& c, const GemmDesc& g);
 void gemm_simt_bf16(Ctx& c, const GemmDesc& g);
 bool gemm_tc_supported(const GemmDesc& g);
+// pair-CTA variant (256-row tiles over two SMs, cta_group::2); same support rules
+bool gemm_tc2_bf16(Ctx& c, const GemmDesc& g);
 // GEMMs of at most 16 rows (decoding): bf16, both operands K-major, no split-K.
 // With a SkinnyNorm, A is not read: the kernel computes it as the norm of the
 // fp32 rows x [M, ldx] over K columns (LayerNorm with w, b; RMSNorm without).
@@ -122,9 +124,12 @@ struct AttnDesc {
 };
 template <typename T> void attn_fwd_simt(Ctx& c, const AttnDesc& a);
 template <typename T> void attn_bwd_simt(Ctx& c, const AttnDesc& a);
-bool attn_tc_supported(const AttnDesc& a);
-void attn_fwd_tc(Ctx& c, const AttnDesc& a);
-void attn_bwd_tc(Ctx& c, const AttnDesc& a);
+// the tensor-core kernels' shape rule: head_dim 64 and T a multiple of 128
+bool attn_tc_shape_ok(int T, int hd);
+bool attn_tc_supported(const AttnDesc& a);  // shape rule plus 16-byte aligned pointers
+// false: a tensor map could not be encoded (nothing launched)
+bool attn_fwd_tc(Ctx& c, const AttnDesc& a);
+bool attn_bwd_tc(Ctx& c, const AttnDesc& a);
 // decoding: o [B, H*hd] = attention of position t against positions 0..t of
 // the cache qkv [B, T, 3, H, hd]
 template <typename T> void attn_decode(Ctx& c, const T* qkv, int B, int Tn, int H, int hd, int t, T* o);

@@ -4,9 +4,8 @@
 // Some callers cannot allocate device memory: code running inside a plugin or
 // custom-operator interface that only hands over its input and output buffers,
 // a process whose device memory is owned by another allocator or pool, or work
-// that must not call cudaMalloc (which synchronises the device and cannot be
-// issued while a stream is being captured).  They call
-// gpt_gemm_dw_accumulate_noalloc with inputs and outputs only.
+// that must not call cudaMalloc (which synchronises the whole device).  They
+// call gpt_gemm_dw_accumulate_noalloc with inputs and outputs only.
 //
 // The scratch array is part of this library's device image: every GPU that
 // loads the library holds its 16 MiB until the process exits.  Host code gets
@@ -80,10 +79,17 @@ extern "C" gpt_status gpt_gemm_dw_accumulate_noalloc(int32_t M, int32_t N, int32
   g.name = "gemm_dw_noalloc";
   if (!gemm_tc_supported(g)) return GPT_ERR_UNSUPPORTED;
   if (cudaMemsetAsync(flags, 0, sizeof(uint32_t), c.stream) != cudaSuccess) return GPT_ERR_CUDA;
+  // A launch error of our own kernels shows as a new last error; one the
+  // caller's earlier work left behind is not ours to report or to clear.
+  const bool clean_before = cudaPeekAtLastError() == cudaSuccess;
   if (!gemm_tc_bf16(c, g)) return GPT_ERR_CUDA;
+  if (clean_before && cudaPeekAtLastError() != cudaSuccess) {
+    cudaGetLastError();
+    return GPT_ERR_CUDA;
+  }
   uint32_t h_flags = 0;
   if (cudaMemcpyAsync(&h_flags, flags, sizeof(uint32_t), cudaMemcpyDeviceToHost, c.stream) != cudaSuccess)
     return GPT_ERR_CUDA;
-  if (cudaStreamSynchronize(c.stream) != cudaSuccess || cudaGetLastError() != cudaSuccess) return GPT_ERR_CUDA;
+  if (cudaStreamSynchronize(c.stream) != cudaSuccess) return GPT_ERR_CUDA;
   return (h_flags & FLAG_TIMEOUT) ? GPT_ERR_TIMEOUT : GPT_OK;
 }

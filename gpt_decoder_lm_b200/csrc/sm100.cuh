@@ -42,16 +42,18 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
 }
 
 // Bounded wait for the phase of parity `parity` of an mbarrier.  Gives up
-// after ~2 s (or as soon as another warp of the block gave up), sets the
-// timeout bit in the device flag word and returns false.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag, uint32_t* gflags) {
+// after limit_ns (2 s unless given; or as soon as another warp of the block
+// gave up), sets the timeout bit in the device flag word and returns false.
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag, uint32_t* gflags,
+                                          uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   uint64_t t0 = globaltimer_ns();
   for (uint32_t it = 1;; it++) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 127u) == 0) {
       if (*abort_flag) return false;
-      if (globaltimer_ns() - t0 > 2000000000ull) {
+      if (globaltimer_ns() - t0 > limit_ns) {
         *abort_flag = 1;
         atomicOr(gflags, FLAG_TIMEOUT);
         return false;

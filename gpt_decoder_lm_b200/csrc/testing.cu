@@ -1,6 +1,7 @@
 // Kernel-level entry points for the parity tests (include/gpt_testing.h).
 #include "../../include/gpt_testing.h"
 #include "kernels.cuh"
+#include "sm100.cuh"
 
 using namespace gpt;
 
@@ -45,6 +46,10 @@ extern "C" gpt_status gpt_test_gemm(int32_t backend, int32_t M, int32_t N, int32
       if (!gemm_tc_supported(g)) return GPT_ERR_UNSUPPORTED;
       if (!gemm_tc_bf16(c, g)) return GPT_ERR_CUDA;
       break;
+    case GPT_GEMM_TC2_BF16:
+      if (!gemm_tc_supported(g)) return GPT_ERR_UNSUPPORTED;
+      if (!gemm_tc2_bf16(c, g)) return GPT_ERR_CUDA;
+      break;
     case GPT_GEMM_SKINNY_BF16:
       if (!gemm_skinny_supported(g)) return GPT_ERR_UNSUPPORTED;
       gemm_skinny_bf16(c, g);
@@ -67,8 +72,7 @@ extern "C" gpt_status gpt_test_attention(int32_t backend, int32_t backward, int3
   AttnDesc a{B, T, H, hd, qkv, o, lse, dout, dqkv, dsum, make_drop_key(seed, counter, layer, 1, p)};
   if (backend == 1) {
     if (dtype != 1 || !attn_tc_supported(a)) return GPT_ERR_UNSUPPORTED;
-    if (backward) attn_bwd_tc(c, a);
-    else attn_fwd_tc(c, a);
+    if (!(backward ? attn_bwd_tc(c, a) : attn_fwd_tc(c, a))) return GPT_ERR_CUDA;
   } else if (backend == 0) {
     if (hd != 4 && hd != 8 && hd != 16 && hd != 32 && hd != 64 && hd != 128) return GPT_ERR_UNSUPPORTED;
     if (dtype == 1) {
@@ -83,4 +87,30 @@ extern "C" gpt_status gpt_test_attention(int32_t backend, int32_t backward, int3
   }
   if (cudaStreamSynchronize(c.stream) != cudaSuccess || cudaGetLastError() != cudaSuccess) return GPT_ERR_CUDA;
   return GPT_OK;
+}
+
+// One warp waits on an mbarrier that nothing ever arrives at, through the
+// same bounded wait the tensor-core kernels use, with the given limit.
+__global__ void k_test_wait_timeout(uint64_t limit_ns, uint32_t* flags, int* gave_up) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  const uint32_t b = sm100::smem_u32(&bar);
+  if (threadIdx.x == 0) {
+    sm100::mbar_init(b, 1);
+    abort_flag = 0;
+    sm100::fence_barrier_init();
+  }
+  __syncthreads();
+  const bool ok = sm100::mbar_wait(b, 0, &abort_flag, flags, limit_ns);
+  if (!ok && threadIdx.x == 0) *gave_up = 1;
+}
+
+extern "C" gpt_status gpt_test_wait_timeout(uint64_t limit_ns, void* stream, uint32_t* d_flags, int32_t* d_gave_up) {
+  if (!d_flags || !d_gave_up || limit_ns < 1000 || limit_ns > 10000000000ull) return GPT_ERR_INVALID_ARG;
+  cudaStream_t st = (cudaStream_t)stream;
+  k_test_wait_timeout<<<1, 32, 0, st>>>(limit_ns, d_flags, d_gave_up);
+  if (cudaGetLastError() != cudaSuccess || cudaStreamSynchronize(st) != cudaSuccess) return GPT_ERR_CUDA;
+  uint32_t f = 0;
+  if (cudaMemcpy(&f, d_flags, 4, cudaMemcpyDeviceToHost) != cudaSuccess) return GPT_ERR_CUDA;
+  return (f & FLAG_TIMEOUT) ? GPT_ERR_TIMEOUT : GPT_OK;
 }

@@ -92,7 +92,7 @@ typedef struct gpt_config {
                              excluded from the loss (their logits are masked).       */
   int32_t n_layer;        /* L >= 1                                                  */
   int32_t n_head;         /* H; head_dim = n_embd / n_head (run log section 2.2)     */
-  int32_t n_embd;         /* d, multiple of 8 (multiple of 64 in bf16 mode)          */
+  int32_t n_embd;         /* d, multiple of 8, at most 2048                          */
   int32_t block_size;     /* T: sequence length of every window                      */
   int32_t batch_size;     /* B: windows per micro-batch                              */
   int32_t grad_accum;     /* micro-batches per optimiser step (>= 1)                 */
@@ -133,6 +133,21 @@ size_t gpt_param_count(const gpt_config* cfg);
 
 /* Bytes of device workspace a model with this config needs (out). */
 gpt_status gpt_workspace_bytes(const gpt_config* cfg, size_t* out);
+
+/* Which kernels a model with this config runs (pure host; out receives
+ * GPT_PATH_* bits).  The choice is a fixed rule of the config, made once, and
+ * never a fallback taken at run time (a kernel that cannot be launched is
+ * GPT_ERR_CUDA):
+ *   - GPT_PATH_GEMM_TC: bf16 mode.  Every dense contraction runs on the
+ *     tcgen05 tensor-core GEMM, except products of at most 16 rows (the
+ *     decoding step of gpt_generate), which run on the decoding GEMM (warp
+ *     MMAs streaming the weights).  fp32 mode runs CUDA-core GEMMs.
+ *   - GPT_PATH_ATTN_TC: bf16 mode with head_dim 64 and block_size a multiple
+ *     of 128 (every bf16 workload of the pages' configurations).  The causal
+ *     attention runs on the tcgen05 flash kernels; other shapes, and fp32
+ *     mode, run the CUDA-core attention kernels. */
+enum { GPT_PATH_GEMM_TC = 1u << 0, GPT_PATH_ATTN_TC = 1u << 1 };
+gpt_status gpt_config_kernel_paths(const gpt_config* cfg, uint32_t* out);
 
 /* get_lr of the practical guide, section 6: lr*it/warmup while it < warmup,
  * then lr*0.5*(1+cos(pi*(it-warmup)/(max_iters-warmup))).  Pure function. */
@@ -192,13 +207,16 @@ gpt_status gpt_train_step_host(gpt_model* m, const int32_t* h_idx, const int32_t
 
 /* CUDA-graph replay of gpt_train_step / gpt_train_step_host (default on;
  * gpt_generate is replayed under the same switch).
- * When on, and the config has no dropout and per-kernel timing is off, the
- * first step of each kind runs eagerly, the second is captured into a graph
- * (on a stream the library creates) and every later step replays it on the
- * model's stream after a one-thread kernel writes the step's index, lr and
- * bias corrections to device memory.  A new d_stream / stream_len /
+ * When on, and per-kernel timing is off, the first step of each kind runs
+ * eagerly, the second is captured into a graph (on a stream the library
+ * creates) and every later step replays it on the model's stream after a
+ * one-thread kernel writes the step's index, lr and bias corrections to
+ * device memory; the replayed kernels read them there, and derive their
+ * dropout keys from that step index.  A new d_stream / stream_len /
  * data_seed triggers a new capture.  The replayed step runs the same kernels
- * with the same arguments as the eager one, so results are bit-identical. */
+ * on the same values as the eager one, so results are bit-identical.  A
+ * capture that fails returns GPT_ERR_CUDA (that step did not run; graphs stay
+ * on, and gpt_set_graphs(m, 0) runs every step eagerly). */
 gpt_status gpt_set_graphs(gpt_model* m, int32_t on);
 
 /* The batch gather of gpt_train_step on its own: writes int32
@@ -319,8 +337,8 @@ const char* gpt_status_string(gpt_status s);
  * that cannot allocate device memory -- code inside a plugin or
  * custom-operator interface that only hands over its input and output
  * buffers, a process whose device memory belongs to another allocator or
- * pool, or work that must not call cudaMalloc (it synchronises the device and
- * cannot be issued while a stream is being captured).
+ * pool, or work that must not call cudaMalloc (it synchronises the whole
+ * device).
  *
  * Weight-gradient GEMM of the training step, dW[M, N] += sum_k A[k, m] *
  * B[k, n], on the tensor cores: A is bf16 [K, M] row-major with pitch lda,
@@ -340,7 +358,8 @@ const char* gpt_status_string(gpt_status s);
  *     calls whose GPU work overlaps -- on two streams at once, or from two
  *     threads -- race on it.
  *   - Work is enqueued on cuda_stream (a cudaStream_t) and the call
- *     synchronises that stream before returning.
+ *     synchronises that stream before returning.  A CUDA error left pending
+ *     by the caller's own earlier work is neither reported nor cleared.
  * Returns GPT_ERR_INVALID_ARG for bad sizes or NULL pointers,
  * GPT_ERR_UNSUPPORTED when the shape or alignment does not suit the tensor
  * cores (pitches multiple of 8, M and N multiple of 8, 16-byte aligned

@@ -19,7 +19,13 @@ extern "C" {
 #endif
 
 /* Backends of gpt_test_gemm. */
-enum { GPT_GEMM_SIMT_F32 = 0, GPT_GEMM_SIMT_BF16 = 1, GPT_GEMM_TC_BF16 = 2, GPT_GEMM_SKINNY_BF16 = 3 };
+enum {
+  GPT_GEMM_SIMT_F32 = 0,
+  GPT_GEMM_SIMT_BF16 = 1,
+  GPT_GEMM_TC_BF16 = 2,
+  GPT_GEMM_SKINNY_BF16 = 3,
+  GPT_GEMM_TC2_BF16 = 4  /* pair-CTA tensor-core GEMM (256-row tiles over two SMs) */
+};
 
 /* D[m, n] = sum_k A[m, k] * B[n, k] followed by epilogue `epi_kind`:
  *   0 out = D; 1 out = D + bias; 2 with h = D + bias: out = act'(h), out2 = act(h);
@@ -50,6 +56,15 @@ gpt_status gpt_test_attention(int32_t backend, int32_t backward, int32_t dtype, 
                               int32_t hd, const void* qkv, void* o, float* lse, const void* dout, void* dqkv,
                               float* dsum, float p, uint64_t seed, uint64_t counter, int32_t layer, void* stream,
                               uint32_t* d_flags);
+
+/* The bounded device-side wait of the tensor-core kernels, made to run out:
+ * one warp waits on an mbarrier that nothing arrives at, with a limit of
+ * limit_ns nanoseconds (1e3 .. 1e10) instead of the kernels' 2 s.  The wait
+ * gives up, sets GPT_FLAG_TIMEOUT in *d_flags and 1 in *d_gave_up (device
+ * uint32 / int32, zeroed by the caller), and the kernel returns: the GPU
+ * context stays usable.  Synchronising.  Returns GPT_ERR_TIMEOUT when the
+ * flag was raised (the expected outcome), GPT_OK otherwise. */
+gpt_status gpt_test_wait_timeout(uint64_t limit_ns, void* stream, uint32_t* d_flags, int32_t* d_gave_up);
 
 #ifdef __cplusplus
 }

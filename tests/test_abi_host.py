@@ -90,3 +90,20 @@ def test_recompute_flag_validated(lib):
     cfg = gb.make_config(W.CHAR, recompute=2)
     n = C.c_size_t()
     assert gb.STATUS[lib.gpt_workspace_bytes(C.byref(cfg), C.byref(n))] == "GPT_ERR_CONFIG"
+
+
+@pytest.mark.parametrize("w,over,want", [
+    (W.GPT2_124M, {}, gb.GPT_PATH_GEMM_TC | gb.GPT_PATH_ATTN_TC),
+    (W.GPT2_XL, {}, gb.GPT_PATH_GEMM_TC | gb.GPT_PATH_ATTN_TC),
+    (W.DROPOUT_512, {}, gb.GPT_PATH_GEMM_TC | gb.GPT_PATH_ATTN_TC),
+    (W.CHAR, {}, gb.GPT_PATH_GEMM_TC | gb.GPT_PATH_ATTN_TC),
+    (W.CHAR, {"block_size": 96}, gb.GPT_PATH_GEMM_TC),          # T not a multiple of 128
+    (W.CHAR, {"n_head": 12}, gb.GPT_PATH_GEMM_TC),              # head_dim 32
+    (W.MICRO, {}, 0),                                           # fp32 mode
+    (W.CHAR.with_(precision="fp32"), {}, 0),
+], ids=["gpt2_124m", "gpt2_xl", "dropout_512", "char", "char_T96", "char_hd32", "micro", "char_fp32"])
+def test_kernel_paths_follow_the_shape_rule(lib, w, over, want):
+    """Which kernels a config runs is a stated rule of the config (bf16: the
+    tensor-core GEMM; tensor-core attention at head_dim 64 and T a multiple
+    of 128), never a fallback taken at run time."""
+    assert gb.kernel_paths(gb.make_config(w, **over)) == want

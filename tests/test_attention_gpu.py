@@ -71,7 +71,10 @@ def run_case(backend, B, T, H, p, seed=0, qkv_np=None):
     return o, g
 
 
-@pytest.mark.parametrize("B,T,H", [(2, 256, 3), (1, 512, 2), (1, 128, 1)])
+# the last three are the benchmarked shapes: GPT-2 124M (T 1024, 12 heads;
+# two batch rows so the longest-block-first order spans several (b, h)) and
+# GPT-2 XL (T 1024, 25 heads)
+@pytest.mark.parametrize("B,T,H", [(2, 256, 3), (1, 512, 2), (1, 128, 1), (2, 1024, 12), (1, 1024, 25)])
 @pytest.mark.parametrize("p", [0.0, 0.1], ids=["nodrop", "dropout"])
 def test_attention_tensor_core(B, T, H, p):
     run_case(1, B, T, H, p)

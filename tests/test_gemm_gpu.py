@@ -19,7 +19,7 @@ if not torch.cuda.is_available():
 from gpt_decoder_lm_b200 import binding as gb  # noqa: E402
 from scipy.special import erf  # noqa: E402
 
-SKINNY, TC, SIMT_BF16, SIMT_F32 = 3, 2, 1, 0
+TC2, SKINNY, TC, SIMT_BF16, SIMT_F32 = 4, 3, 2, 1, 0
 
 
 def bf16_round(x: np.ndarray) -> np.ndarray:
@@ -65,20 +65,21 @@ LAYOUTS = [(1, 1), (1, 0), (0, 0)]   # forward (TN), dX (B MN-major), dW (both M
 SHAPES = [(128, 128, 64), (256, 384, 192), (200, 328, 136), (1024, 2304, 256), (4096, 1024, 128), (64, 96, 520)]
 
 
+@pytest.mark.parametrize("backend", [TC, TC2], ids=["tc", "tc2"])
 @pytest.mark.parametrize("ak,bk", LAYOUTS, ids=["tn", "b_mn", "ab_mn"])
 @pytest.mark.parametrize("M,N,K", SHAPES, ids=[f"{m}x{n}x{k}" for m, n, k in SHAPES])
-def test_tc_gemm_store_f32(M, N, K, ak, bk):
+def test_tc_gemm_store_f32(M, N, K, ak, bk, backend):
     A, B, Ad, Bd, lda, ldb = operands(M, N, K, ak, bk, M + N + K)
     out = torch.full((M, N), float("nan"), device="cuda")
-    run(TC, M, N, K, Ad, lda, ak, Bd, ldb, bk, 6, out=out, ldo=N)
+    run(backend, M, N, K, Ad, lda, ak, Bd, ldb, bk, 6, out=out, ldo=N)
     ref = A @ B.T
     got = out.double().cpu().numpy()
     err = np.abs(got - ref).max() / np.abs(ref).max()
     assert err < 2e-6, err
 
 
-@pytest.mark.parametrize("backend,M", [(TC, 384), (SIMT_BF16, 384), (SKINNY, 12), (SKINNY, 5)],
-                         ids=["tc", "simt", "skinny12", "skinny5"])
+@pytest.mark.parametrize("backend,M", [(TC, 384), (TC2, 384), (SIMT_BF16, 384), (SKINNY, 12), (SKINNY, 5)],
+                         ids=["tc", "tc2", "simt", "skinny12", "skinny5"])
 def test_epilogues(backend, M):
     N, K = 512, 256
     rng = np.random.default_rng(7)
@@ -165,14 +166,15 @@ def test_skinny_gemm_unsupported():
     assert gb.STATUS[st] == "GPT_ERR_UNSUPPORTED"  # K not a multiple of 32
 
 
+@pytest.mark.parametrize("backend", [TC, TC2], ids=["tc", "tc2"])
 @pytest.mark.parametrize("splits", [2, 5])
-def test_tc_split_k_accumulate(splits):
+def test_tc_split_k_accumulate(splits, backend):
     M, N, K = 256, 384, 4096      # dW-like: both operands MN-major, long contraction
     A, B, Ad, Bd, lda, ldb = operands(M, N, K, 0, 0, 11)
     acc0 = np.random.default_rng(2).standard_normal((M, N)).astype(np.float32)
     acc = dev_f32(acc0)
     partial = torch.empty((splits, M, N), device="cuda")
-    run(TC, M, N, K, Ad, lda, 0, Bd, ldb, 0, 5, out=acc, ldo=N, split_k=splits, partial=partial)
+    run(backend, M, N, K, Ad, lda, 0, Bd, ldb, 0, 5, out=acc, ldo=N, split_k=splits, partial=partial)
     ref = acc0 + A @ B.T
     err = np.abs(acc.double().cpu().numpy() - ref).max() / np.abs(ref).max()
     # fp32 accumulation over K = 4096 products: rounding grows like sqrt(K) * 2^-24
@@ -207,3 +209,79 @@ def test_gelu_epilogue_accuracy_fp32():
     dd = gelu_grad(rng.standard_normal((M, N)) * 3).astype(np.float32)
     run(SIMT_F32, M, N, K, dev_f32(A), K, 1, dev_f32(B), K, 1, 4, act=0, out=out, ldo=N, aux=dev_f32(dd))
     np.testing.assert_allclose(out.double().cpu().numpy(), D * dd.astype(np.float64), rtol=1e-5, atol=2e-6)
+
+
+# The contractions of the benchmarked step at their own shapes: GPT-2 124M
+# (M = 12 x 1024 rows, d 768, 3d 2304, 4d 3072) and GPT-2 XL's layer (M =
+# 2 x 1024, d 1600, 3d 4800 and 4d 6400, both ragged against the 256-column
+# tile).  (M, N, K) with the layout each one runs in: forward TN, dX with W
+# MN-major, dW with both operands MN-major (K = the token count).
+FULL_SHAPES = [
+    ("qkv_fwd_124m", 12288, 2304, 768, 1, 1), ("fc_dx_124m", 12288, 768, 3072, 1, 0),
+    ("fc_dw_124m", 3072, 768, 12288, 0, 0),
+    ("qkv_fwd_xl", 2048, 4800, 1600, 1, 1), ("proj_fwd_xl", 2048, 1600, 6400, 1, 1),
+    ("qkv_dx_xl", 2048, 1600, 4800, 1, 0), ("fc_dx_xl", 2048, 1600, 6400, 1, 0),
+    ("qkv_dw_xl", 4800, 1600, 2048, 0, 0), ("fc_dw_xl", 6400, 1600, 2048, 0, 0),
+]
+
+
+@pytest.mark.parametrize("backend", [TC, TC2], ids=["tc", "tc2"])
+@pytest.mark.parametrize("name,M,N,K,ak,bk", FULL_SHAPES, ids=[s[0] for s in FULL_SHAPES])
+def test_tc_gemm_full_shapes(name, M, N, K, ak, bk, backend):
+    A, B, Ad, Bd, lda, ldb = operands(M, N, K, ak, bk, M + N + K)
+    out = torch.full((M, N), float("nan"), device="cuda")
+    run(backend, M, N, K, Ad, lda, ak, Bd, ldb, bk, 6, out=out, ldo=N)
+    ref = A @ B.T
+    got = out.double().cpu().numpy()
+    err = np.abs(got - ref).max() / np.abs(ref).max()
+    # fp32 accumulation of K bf16 products: rounding grows like sqrt(K) 2^-24
+    assert err < (2e-6 if K <= 2048 else 1e-5), err
+
+
+@pytest.mark.parametrize("splits", [1, 4])
+def test_tc_gemm_dw_split_full_shape(splits):
+    # the fc weight gradient of GPT-2 124M (3072 x 768 over 12288 tokens),
+    # split-K partials added to an existing fp32 gradient in a fixed order
+    M, N, K = 3072, 768, 12288
+    A, B, Ad, Bd, lda, ldb = operands(M, N, K, 0, 0, 21)
+    acc0 = np.random.default_rng(3).standard_normal((M, N)).astype(np.float32)
+    acc = dev_f32(acc0)
+    partial = torch.empty((splits, M, N), device="cuda")
+    run(TC, M, N, K, Ad, lda, 0, Bd, ldb, 0, 5, out=acc, ldo=N, split_k=splits, partial=partial)
+    ref = acc0 + A @ B.T
+    err = np.abs(acc.double().cpu().numpy() - ref).max() / np.abs(ref).max()
+    assert err < 1e-5, err
+
+
+@pytest.mark.parametrize("layout", ["fwd", "dw"])
+def test_tc_gemm_lm_head_sampled(layout):
+    # the lm_head at full size: logits [12288, 50304] = x [12288, 768] W^T
+    # (forward, TN) and its weight gradient [50304, 768] over 12288 tokens
+    # (both operands MN-major, as dlogits and the final norm's output are
+    # stored).  Operands are drawn on the device (seeded) and rounded to
+    # bf16 there; the float64 reference is formed on the host for 96 sampled
+    # output rows.
+    gen = torch.Generator(device="cuda").manual_seed(41)
+    Mx, V, d = 12288, 50304, 768
+    if layout == "fwd":
+        M, N, K, ak, bk = Mx, V, d, 1, 1
+        Ad = torch.randn((M, K), generator=gen, device="cuda").bfloat16()
+        Bd = torch.randn((N, K), generator=gen, device="cuda").bfloat16()
+        lda, ldb = K, K
+    else:
+        M, N, K, ak, bk = V, d, Mx, 0, 0
+        Ad = torch.randn((K, M), generator=gen, device="cuda").bfloat16()
+        Bd = torch.randn((K, N), generator=gen, device="cuda").bfloat16()
+        lda, ldb = M, N
+    out = torch.full((M, N), float("nan"), device="cuda")
+    run(TC, M, N, K, Ad, lda, ak, Bd, ldb, bk, 6, out=out, ldo=N)
+    rng = np.random.default_rng(31)
+    rows = np.sort(np.concatenate([rng.choice(M, 94, replace=False), [0, M - 1]]))
+    r = torch.from_numpy(rows).cuda()
+    a_rows = (Ad[r] if ak else Ad[:, r].t()).double().cpu().numpy()      # [96, K]
+    b_all = (Bd if bk else Bd.t()).double().cpu().numpy()                # [N, K]
+    ref = a_rows @ b_all.T
+    got = out[r].double().cpu().numpy()
+    err = np.abs(got - ref).max() / np.abs(ref).max()
+    assert err < (2e-6 if K <= 2048 else 1e-5), err
+    assert not torch.isnan(out).any().item()

@@ -50,14 +50,18 @@ def oracle_logits(oc, P, prefix):
 
 
 @pytest.mark.parametrize("wname,precision,tol", [("char", "bf16", 0.05), ("char", "fp32", 1e-4),
-                                                  ("micro", "fp32", 1e-4), ("micro64", "bf16", 0.05)])
+                                                  ("micro", "fp32", 1e-4), ("micro64", "bf16", 0.05),
+                                                  ("char12", "bf16", 0.05)])
 def test_greedy_generation_matches_oracle(wname, precision, tol):
-    w = (W.CHAR if wname == "char" else W.MICRO).with_(precision=precision)
-    # micro64: the RMSNorm variant wide enough for the decoding GEMM that computes the norm itself
+    w = (W.CHAR if wname.startswith("char") else W.MICRO).with_(precision=precision)
+    # micro64: the RMSNorm variant wide enough for the decoding GEMM that computes the norm itself;
+    # char12: 12 rows, the two-tile (9-16 row) decoding GEMM with the LayerNorm computed inside it,
+    # as GPT-2 124M decoding at batch 12 runs it
     over = {"char": dict(n_layer=2, batch_size=4, block_size=128), "micro": {},
-            "micro64": dict(n_layer=2, n_embd=64, n_head=4)}[wname]
+            "micro64": dict(n_layer=2, n_embd=64, n_head=4),
+            "char12": dict(n_layer=2, batch_size=12, block_size=128)}[wname]
     m, cfg, P, oc = setup(w, **over)
-    T0, n_new = (9, 20) if wname == "char" else (4, 12)
+    T0, n_new = (9, 20) if wname.startswith("char") else (4, 12)
     seq, _ = generate(m, cfg, T0, n_new, 0.0, 0, 1.0, seed=1)
     exact = 0
     for s in range(n_new):

@@ -138,16 +138,44 @@ def test_gpt2_fp32_small(dropout):
     check_step(w, cfg, m, 4, 1e-5, True, 1e-4, drop_counter=3)
 
 
-def test_char_bf16_reduced_batch():
+def test_char_bf16_full_config():
+    # the char-level workload at its own size: 6 layers, d 384, 6 heads,
+    # T 256, batch 64, vocab 65 (padded to 128)
     w = W.CHAR
-    m, cfg = make(w, batch_size=4)
+    m, cfg = make(w)
     check_step(w, cfg, m, 5, 2e-3, False, 2e-2)
 
 
-def test_dropout_bf16_reduced():
+def test_dropout_bf16_full_config():
+    # the 12-layer / 512-wide dropout workload at its own size: 8 heads,
+    # T 512, batch 12, vocab 50257, dropout 0.1 at every site
     w = W.DROPOUT_512
-    m, cfg = make(w, n_layer=3, batch_size=2, block_size=256)
+    m, cfg = make(w, token_dtype=gb.GPT_TOK_I32)
     check_step(w, cfg, m, 6, 2e-3, False, 2e-2, drop_counter=1)
+
+
+@pytest.mark.parametrize("wname", ["char_bf16", "dropout_bf16", "gpt2_fp32", "micro_fp32"])
+def test_recompute_matches_oracle(wname):
+    # activation recompute against the oracle (not only against the stored
+    # run): one forward + backward, bf16 and fp32, with and without dropout
+    if wname == "char_bf16":
+        w, over, tol = W.CHAR, dict(n_layer=3, batch_size=4, block_size=128), (2e-3, False, 2e-2)
+    elif wname == "dropout_bf16":
+        w, over, tol = W.DROPOUT_512, dict(n_layer=3, batch_size=2, block_size=256), (2e-3, False, 2e-2)
+    elif wname == "gpt2_fp32":
+        w = W.CHAR.with_(precision="fp32", dropout=0.1)
+        over, tol = dict(n_layer=3, n_head=4, n_embd=64, block_size=96, batch_size=3), (1e-5, True, 1e-4)
+    else:
+        w, over, tol = W.MICRO, dict(n_layer=3), (1e-5, True, 1e-4)
+    m, cfg = make(w, recompute=1, token_dtype=gb.GPT_TOK_I32, **over)
+    check_step(w, cfg, m, 12, *tol, drop_counter=2)
+
+
+def test_recompute_ten_steps_adamw_bf16():
+    w = W.CHAR
+    m, cfg = make(w, n_layer=2, batch_size=4, block_size=128, grad_accum=2, recompute=1)
+    glob, per = _ten_steps(w, cfg, m, lambda o: 2e-3, 2e-2)
+    assert glob <= 1e-3, (glob, sorted(per.items(), key=lambda kv: -kv[1])[:6])
 
 
 def _ten_steps(w, cfg, m, loss_tol, norm_tol):
@@ -250,18 +278,23 @@ def _weights(m):
     return np.concatenate([P[k].ravel() for k in sorted(P)])
 
 
-@pytest.mark.parametrize("host_batches", [False, True])
-def test_graph_replay_bit_identical_to_eager(host_batches):
+@pytest.mark.parametrize("wname,host_batches", [("char", False), ("char", True), ("dropout", False),
+                                                ("dropout", True)])
+def test_graph_replay_bit_identical_to_eager(wname, host_batches):
     # The replayed step reads its step index, lr and bias corrections from
-    # device memory; every other argument is the eager step's.  Weights, loss
-    # and norm must match bit for bit over steps with a changing lr, and a new
-    # data seed must re-capture (device-gather form).
-    w = W.CHAR
+    # device memory, and derives the dropout keys of every site from that
+    # step index; every other argument is the eager step's.  Weights, loss
+    # and norm must match bit for bit over steps with a changing lr (and
+    # changing dropout masks), and a new data seed must re-capture
+    # (device-gather form).
+    w, over = {"char": (W.CHAR, dict(n_layer=2, batch_size=4, block_size=128, grad_accum=2)),
+               "dropout": (W.DROPOUT_512, dict(n_layer=2, batch_size=2, block_size=256, grad_accum=2,
+                                               token_dtype=gb.GPT_TOK_I32))}[wname]
     stream = W.token_stream(w, n=1 << 16)
     sd = dev(stream.astype(np.int32))
     res = []
     for graphs in (False, True):
-        m, cfg = make(w, n_layer=2, batch_size=4, block_size=128, grad_accum=2)
+        m, cfg = make(w, **over)
         m.set_graphs(graphs)
         out = []
         for step in range(1, 7):
@@ -321,3 +354,71 @@ def test_recompute_bit_identical(wname):
     (l0, w0), (l1, w1) = res
     assert l0 == l1
     assert np.array_equal(w0, w1)
+
+
+def test_resume_five_plus_five_equals_ten():
+    # checkpoint / resume: 5 steps, save the state (weights, AdamW moments),
+    # restore it into a NEW model, 5 more steps: bit-identical to 10
+    # uninterrupted steps (losses, norms, weights, moments)
+    w = W.CHAR
+    over = dict(n_layer=2, batch_size=4, block_size=128, grad_accum=2)
+    sd = dev(W.token_stream(w, n=1 << 16).astype(np.int32))
+    lrs = [oracle.lr_cosine(w.lr, s - 1, w.warmup, w.max_iters) for s in range(1, 11)]
+    m, cfg = make(w, **over)
+    full = [m.train_step(sd, w.data_seed, lrs[s - 1], s) for s in range(1, 11)]
+    ref_state = m.get_state()
+    m.close()
+    m1, _ = make(w, **over)
+    first = [m1.train_step(sd, w.data_seed, lrs[s - 1], s) for s in range(1, 6)]
+    p, mm, vv = m1.get_state()
+    m1.close()
+    m2, _ = make(w.with_(weight_seed=w.weight_seed + 99), **over)   # different init: overwritten
+    m2.set_state(p, mm, vv)
+    second = [m2.train_step(sd, w.data_seed, lrs[s - 1], s) for s in range(6, 11)]
+    st = m2.get_state()
+    m2.close()
+    assert first + second == full
+    for a, b in zip(st, ref_state):
+        assert np.array_equal(a, b)
+
+
+def test_nonfinite_gradient_skips_update():
+    # an Inf planted in one gradient: the clip + AdamW call reports
+    # GPT_ERR_NONFINITE, leaves weights and moments untouched and zeroes
+    # the gradients
+    w = W.CHAR
+    m, cfg = make(w, n_layer=1, batch_size=2, block_size=128)
+    idx, tgt = W.random_batch(w, 3, cfg.batch_size, cfg.block_size)
+    m.forward_loss(dev(idx), dev(tgt))
+    m.backward()
+    m.clip_adamw_step(1e-3, 1)          # non-zero moments to protect
+    m.forward_loss(dev(idx), dev(tgt))
+    m.backward()
+    before = [m.get(k) for k in (gb.GPT_PARAM, gb.GPT_ADAM_M, gb.GPT_ADAM_V)]
+    G = m.get(gb.GPT_GRAD)
+    G["h.0.mlp.c_fc.weight"][3, 5] = np.inf
+    m.set({"h.0.mlp.c_fc.weight": G["h.0.mlp.c_fc.weight"]}, gb.GPT_GRAD)
+    with pytest.raises(gb.GptError) as e:
+        m.clip_adamw_step(1e-3, 2)
+    assert e.value.name == "GPT_ERR_NONFINITE"
+    after = [m.get(k) for k in (gb.GPT_PARAM, gb.GPT_ADAM_M, gb.GPT_ADAM_V)]
+    for a, b in zip(before, after):
+        for k in a:
+            assert np.array_equal(a[k], b[k]), k
+    assert all(np.all(v == 0) for v in m.get(gb.GPT_GRAD).values())
+    m.close()
+
+
+def test_bounded_wait_gives_up_and_returns():
+    # the bounded mbarrier wait of the tensor-core kernels, on a barrier that
+    # nothing arrives at, with a 1 ms limit: it gives up, raises the timeout
+    # flag and the kernel returns; the context stays usable afterwards
+    flags = torch.zeros(1, dtype=torch.int32, device="cuda")
+    gave_up = torch.zeros(1, dtype=torch.int32, device="cuda")
+    st = torch.cuda.current_stream().cuda_stream
+    rc = gb.test_wait_timeout(1_000_000, flags, gave_up, st)
+    assert gb.STATUS[rc] == "GPT_ERR_TIMEOUT"
+    assert int(flags.item()) & gb.FLAG_TIMEOUT
+    assert int(gave_up.item()) == 1
+    x = torch.arange(10, device="cuda").sum().item()   # the device still works
+    assert x == 45
