@@ -52,7 +52,10 @@ def peaks():
 def flops_per_token(w) -> float:
     """6 N + 12 L d T with N = parameters excluding wpe (PaLM appendix convention)."""
     d, L, T, V = w.n_embd, w.n_layer, w.block_size, w.vocab_size
-    n = V * d + L * (12 * d * d + 13 * d) + 2 * d
+    if w.variant == "micro":  # untied lm_head, no biases, parameter-free norms
+        n = 2 * V * d + 12 * L * d * d
+    else:
+        n = V * d + L * (12 * d * d + 13 * d) + 2 * d
     return 6.0 * n + 12.0 * L * d * T
 
 
@@ -289,6 +292,119 @@ def measure_recompute(w, d_stream, data_seed, dev, warmup):
             "workspace_gb_stored": gb.workspace_bytes(gb.make_config(w)) / 1e9}
 
 
+def measure_lora(w, d_stream, data_seed, dev, warmup):
+    """The LoRA fine-tuning step (rank 8 on q and v, alpha 16) at the same
+    workload: device time over 5 graph-replayed steps, L2 flushed between them."""
+    import torch
+
+    from gpt_decoder_lm_b200 import binding as gb
+
+    cfg = gb.make_config(w)
+    m = gb.Model(cfg, seed=w.weight_seed, device=dev)
+    r, blocks = 8, 2 * w.n_layer
+    A = np.random.default_rng(1).standard_normal((blocks, r, w.n_embd)).astype(np.float32) / np.sqrt(w.n_embd)
+    m.lora_attach(r, 16.0, 1 | 4, A)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    st = 0
+    for _ in range(max(warmup, 3)):
+        st += 1
+        m.train_step(d_stream, data_seed, 1e-4, st, sync=False)
+        flush.zero_()
+    torch.cuda.synchronize()
+    n = 5
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(n):
+        st += 1
+        m.train_step(d_stream, data_seed, 1e-4, st, sync=False)
+        flush.zero_()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / n
+    m.close()
+    return {"ms_per_step": ms, "tokens_per_s": w.tokens_per_step / (ms / 1000.0), "steps": n, "rank": r,
+            "targets": "q,v", "trainable_params": blocks * 2 * r * w.n_embd}
+
+
+# bounded oracle samples for the other workloads: (batch, window) per step
+ORACLE_SAMPLES = {W.MICRO.name: (8, 16), W.CHAR.name: (1, 256), W.DROPOUT_512.name: (1, 128),
+                  W.GPT2_XL.name: (1, 16)}
+
+
+def oracle_tokens_per_s(w, B: int, T: int, threads: int | None):
+    """Oracle tokens/s on one step of a B x T sample at the workload's model
+    dims (fwd + bwd + clip + AdamW), with the BLAS pool limited to `threads`
+    (None: every core)."""
+    import oracle
+    from threadpoolctl import threadpool_limits
+    cfg = oracle.Config(vocab_size=w.vocab_size, n_layer=w.n_layer, n_head=w.n_head, n_embd=w.n_embd,
+                        block_size=T, batch_size=B, grad_accum=1, variant=w.variant, init_std=w.init_std,
+                        beta1=w.beta1, beta2=w.beta2, eps=w.eps, weight_decay=w.weight_decay, grad_clip=w.grad_clip,
+                        dropout=w.dropout, dropout_seed=w.dropout_seed)
+    P = oracle.init_params(cfg, w.weight_seed)
+    stream = W.token_stream(w, n=1 << 16).astype(np.int64)
+    with threadpool_limits(limits=threads, user_api="blas"):
+        n = blas_threads()
+        t0 = time.perf_counter()
+        oracle.train_step(cfg, P, oracle.AdamState(), stream, w.data_seed, w.lr, 1)
+        dt = time.perf_counter() - t0
+    return B * T / dt, n
+
+
+def measure_configs(dev, warmup: int, with_oracle: bool):
+    """Every other workload of the pages' configurations at its own size: the
+    graph-replayed training step timed over 5 steps (L2 flushed between
+    them), tokens/s and MFU, next to the oracle's tokens/s on a bounded
+    sample at one core and at every core."""
+    import torch
+
+    from gpt_decoder_lm_b200 import binding as gb
+    out = {}
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    pk = peaks()
+    for w in (W.MICRO, W.CHAR, W.DROPOUT_512, W.GPT2_XL):
+        cfg = gb.make_config(w)
+        m = gb.Model(cfg, seed=w.weight_seed, device=dev)
+        host = W.token_stream(w)
+        d_stream = torch.from_numpy(host.view(np.int16) if host.dtype == np.uint16 else host).to(dev)
+        st = 0
+        for _ in range(max(warmup, 3)):
+            st += 1
+            m.train_step(d_stream, w.data_seed, w.lr, st, sync=False)
+            flush.zero_()
+        torch.cuda.synchronize()
+        n = 5
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(n):
+            st += 1
+            m.train_step(d_stream, w.data_seed, w.lr, st, sync=False)
+            flush.zero_()
+        e1.record()
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / n
+        loss, norm = m.train_step(d_stream, w.data_seed, w.lr, st + 1)
+        m.close()
+        del m, d_stream
+        torch.cuda.empty_cache()
+        tps = w.tokens_per_step / (ms / 1000.0)
+        fpt = flops_per_token(w)
+        rec = {"ms_per_step": ms, "tokens_per_s": tps, "tokens_per_step": w.tokens_per_step,
+               "dtype": "f32" if w.precision == "fp32" else "bf16", "flops_per_token": fpt,
+               "mfu_nominal_2250": tps * fpt / (NOMINAL_BF16_TFLOPS * 1e12),
+               "mfu_measured_peak": tps * fpt / (pk["bf16"] * 1e12), "steps": n,
+               "final_loss": loss, "final_grad_norm": norm}
+        if with_oracle:
+            B, T = ORACLE_SAMPLES[w.name]
+            one, _ = oracle_tokens_per_s(w, B, T, 1)
+            allc, nc = oracle_tokens_per_s(w, B, T, None)
+            rec["oracle"] = {"tokens_per_s_1_core": one, "tokens_per_s_all_cores": allc, "cores": nc,
+                             "sample": f"{B} x {T} tokens per step at the full model dims (fp64 numpy "
+                                       f"fwd+bwd+clip+AdamW)"}
+        out[w.name] = rec
+    return out
+
+
 def run_ours(args, w, rank, world, local_rank):
     import torch
     import torch.distributed as dist
@@ -389,6 +505,10 @@ def run_ours(args, w, rank, world, local_rank):
 
     decode = measure_decode(model, w, stream_host, dev, rank)
     recompute = measure_recompute(w, d_stream, data_seed, dev, args.warmup)
+    lora = measure_lora(w, d_stream, data_seed, dev, args.warmup)
+    configs = None
+    if not args.no_configs:
+        configs = measure_configs(dev, args.warmup, rank == 0 and world == 1 and not args.no_cpu_baseline)
 
     pk = peaks()
     gemm_names = [k for k in kt if k.startswith("gemm")]
@@ -430,6 +550,8 @@ def run_ours(args, w, rank, world, local_rank):
             "roofline": roofline,
             "decode": decode,
             "recompute": recompute,
+            "lora": lora,
+            "configs": configs,
             "cpu_baseline": cpu,
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": 2 * ga * B * T * 4,
                     "d2h_bytes_per_step": 16},
@@ -492,6 +614,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default=W.GPT2_124M.name, choices=list(W.ALL))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-configs", action="store_true", help="skip the other workloads' step timings")
     ap.add_argument("--kernels", action="store_true",
                     help="one launch of each hot kernel at the workload's shapes (for ncu), then exit")
     args = ap.parse_args()

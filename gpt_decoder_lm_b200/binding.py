@@ -70,6 +70,11 @@ _PROTOS = {
     "gpt_eval_loss": (I32, [P, P, U64, U64, I32, P]),
     "gpt_sample": (I32, [P, I32, I32, I32, I64, F32, I32, F32, P, P, P]),
     "gpt_generate": (I32, [P, P, I32, I32, F32, I32, F32, P, P]),
+    "gpt_lora_workspace_bytes": (I32, [P, I32, I32, P]),
+    "gpt_lora_attach": (I32, [P, I32, F32, I32, P, P, SZ]),
+    "gpt_lora_detach": (I32, [P]),
+    "gpt_lora_read": (I32, [P, I32, P, SZ]),
+    "gpt_lora_write": (I32, [P, P, SZ]),
     "gpt_num_tensors": (I32, [P, P]),
     "gpt_tensor_info": (I32, [P, I32, P, P]),
     "gpt_get_tensor": (I32, [P, I32, I32, P]),
@@ -94,6 +99,7 @@ _PROTOS = {
                             P, P]),
     "gpt_test_attention": (I32, [I32, I32, I32, I32, I32, I32, I32, P, P, P, P, P, P, F32, U64, U64, I32, P, P]),
     "gpt_test_wait_timeout": (I32, [U64, P, P, P]),
+    "gpt_test_exp2": (I32, [P, P, P, I64, P]),
     "gpt_gemm_dw_accumulate_noalloc": (I32, [I32, I32, I32, P, I64, P, I64, P, I32, P]),
 }
 
@@ -259,6 +265,32 @@ class Model:
         _check(lib().gpt_generate(self.h, _ptr(prompt), prompt.shape[1], n_new, temperature, top_k, top_p,
                                   _ptr(uniform), _ptr(out)), self.h, "generate")
 
+    # -- LoRA adapters on the fused QKV blocks (targets: 1 q, 2 k, 4 v)
+    def lora_attach(self, r: int, alpha: float, targets: int, A):
+        """A: host float32 [blocks, r, d] (the adapted blocks' A; B starts at 0).
+        Allocates the adapter workspace as a torch tensor owned by the model."""
+        import torch
+        n = C.c_size_t(0)
+        _check(lib().gpt_lora_workspace_bytes(C.byref(self.cfg), r, targets, C.byref(n)), self.h, "lora_workspace")
+        self.lora_ws = torch.empty(int(n.value), dtype=torch.uint8, device=self.device)
+        A = np.ascontiguousarray(A, np.float32)
+        _check(lib().gpt_lora_attach(self.h, r, alpha, targets, A.ctypes.data_as(C.c_void_p), self.lora_ws.data_ptr(),
+                                     self.lora_ws.numel()), self.h, "lora_attach")
+        self.lora_n = int(np.prod(A.shape)) * 2
+
+    def lora_detach(self):
+        _check(lib().gpt_lora_detach(self.h), self.h, "lora_detach")
+        self.lora_ws = None
+
+    def lora_read(self, which: int = 0) -> np.ndarray:
+        out = np.empty(self.lora_n, np.float32)
+        _check(lib().gpt_lora_read(self.h, which, out.ctypes.data_as(C.c_void_p), out.size), self.h, "lora_read")
+        return out
+
+    def lora_write(self, params):
+        params = np.ascontiguousarray(params, np.float32)
+        _check(lib().gpt_lora_write(self.h, params.ctypes.data_as(C.c_void_p), params.size), self.h, "lora_write")
+
     def set_graphs(self, on: bool):
         """CUDA-graph replay of train_step / train_step_host / generate (default on)."""
         _check(lib().gpt_set_graphs(self.h, 1 if on else 0), self.h, "set_graphs")
@@ -386,3 +418,8 @@ def test_wait_timeout(limit_ns: int, flags, gave_up, stream=None) -> int:
     """The kernels' bounded mbarrier wait with a short limit, on a barrier
     nothing arrives at; returns the status code."""
     return int(lib().gpt_test_wait_timeout(limit_ns, stream, _ptr(flags), _ptr(gave_up)))
+
+
+def test_exp2(x, y_poly, y_ref, stream=None) -> int:
+    """Device polynomial 2^x and CUDA's exp2f on the same arguments."""
+    return int(lib().gpt_test_exp2(_ptr(x), _ptr(y_poly), _ptr(y_ref), x.numel(), stream))

@@ -158,6 +158,14 @@ struct gpt_model {
   // CUDA-graph replay of the full step: [0] device token stream, [1] host batches
   bool graphs_on = true;
   cudaStream_t cap_stream = nullptr;
+  struct {
+    bool on = false;
+    int targets = 0;
+    float alpha = 0.f;
+    LoraBlocks lb;
+    float *m = nullptr, *v = nullptr;  // Adam moments of the adapters
+    long n = 0;                        // adapter parameters (2 r d per block)
+  } lora;
   cudaGraphExec_t gexec[2] = {nullptr, nullptr};
   uint64_t graph_launches[2] = {0, 0};
   int warm[2] = {0, 0};
@@ -696,7 +704,11 @@ gpt_status backward_t(gpt_model* m) {
   T* datt = reinterpret_cast<T*>(m->datt);
   const bool first = m->cur_micro == 0, last = m->cur_micro == m->n_micro - 1;
   // inst: (layer, kind) of a per-layer weight gradient, -1 for the lm_head
+  // with adapters attached the base weights are frozen: their gradients are
+  // not formed, except the adapted QKV blocks' (the adapters' chain rule)
+  const bool frozen = m->lora.on;
   auto dW = [&](int Mo, int No, const void* A, const void* Bm, float* out, const char* name, int inst) -> bool {
+    if (frozen) return true;
     // out[Mo, No] += A^T B with A [M, Mo], B [M, No] (tokens outermost)
     GemmDesc g = gd(Mo, No, (int)M, A, Mo, false, Bm, No, false);
     g.epi.kind = EPI_ACC_F32;
@@ -723,6 +735,7 @@ gpt_status backward_t(gpt_model* m) {
   };
   // bias gradient = column sums of the operand-typed gradient x [M, N]
   auto bias_grad = [&](const T* x, int N, int l, int which, float* grad) {
+    if (frozen) return;
     colsum_partial<T>(c, x, M, N, colsum_part(l, which), !first);
     if (last) colsum_reduce(c, colsum_part(l, which), colsum_chunks(M), N, grad);
   };
@@ -754,7 +767,7 @@ gpt_status backward_t(gpt_model* m) {
   nb.d = d;
   nb.rms = rms;
   norm_bwd<T>(c, nb);
-  if (last) add_bias_grads_from_norm(m, nb.part, m->lnf_w, m->lnf_b, m->layers[L - 1].pr_b);
+  if (last && !frozen) add_bias_grads_from_norm(m, nb.part, m->lnf_w, m->lnf_b, m->layers[L - 1].pr_b);
   for (int l = L - 1; l >= 0; l--) {
     const LayerP& y = m->layers[l];
     // with recompute the slot still holds the last layer's forward activations
@@ -798,7 +811,7 @@ gpt_status backward_t(gpt_model* m) {
     nb.want_dyb = true;
     nb.part = norm_part(2 * l + 1);
     norm_bwd<T>(c, nb);
-    if (last) add_bias_grads_from_norm(m, nb.part, y.ln2_w, y.ln2_b, y.ap_b);
+    if (last && !frozen) add_bias_grads_from_norm(m, nb.part, y.ln2_w, y.ln2_b, y.ap_b);
     // attention projection
     if (!dW(d, d, dyb, o, m->G(y.ap_w), "gemm_attnproj_dw", l * 4 + 2))
       return fail(m, GPT_ERR_CUDA, "attn proj dW failed");
@@ -814,6 +827,22 @@ gpt_status backward_t(gpt_model* m) {
     if (y.qkv_b >= 0) bias_grad(dqkv, 3 * d, l, 1, m->G(y.qkv_b));
     if (!dW(3 * d, d, dqkv, a1, m->G(y.qkv_w), "gemm_qkv_dw", l * 4 + 3))
       return fail(m, GPT_ERR_CUDA, "qkv dW failed");
+    if (frozen) {
+      // the adapted blocks only: G[t d .. t d + d) += dqkv[:, t d .. t d + d)^T a1
+      for (int t = 0; t < 3; t++) {
+        if (!(m->lora.targets & (1 << t))) continue;
+        GemmDesc gq = gd(d, d, (int)M, dqkv + (size_t)t * d, 3 * d, false, a1, d, false);
+        gq.epi.kind = EPI_ACC_F32;
+        gq.name = "gemm_qkv_dw_adapted";
+        gq.epi.out = m->G(y.qkv_w) + (size_t)t * d * d;
+        gq.epi.ldo = d;
+        if (m->bf16m) {
+          gq.split_k = choose_splits(d, d, M);
+          gq.partial = m->splitk;
+        }
+        if (!gemm(m, gq)) return fail(m, GPT_ERR_CUDA, "adapted qkv dW failed");
+      }
+    }
     g = gd((int)M, d, 3 * d, dqkv, 3 * d, true, m->Wop(y.qkv_w), d, false);
     g.epi.kind = EPI_STORE_F32;
     g.name = "gemm_qkv_dx";
@@ -830,7 +859,12 @@ gpt_status backward_t(gpt_model* m) {
     nb.want_dyb = l > 0;
     nb.part = norm_part(2 * l);
     norm_bwd<T>(c, nb);
-    if (last) add_bias_grads_from_norm(m, nb.part, y.ln1_w, y.ln1_b, l > 0 ? m->layers[l - 1].pr_b : -1);
+    if (last && !frozen)
+      add_bias_grads_from_norm(m, nb.part, y.ln1_w, y.ln1_b, l > 0 ? m->layers[l - 1].pr_b : -1);
+  }
+  if (frozen) {  // no embedding gradients; the adapters' from the merged blocks
+    if (last) lora_grads(c, m->lora.lb, m->g);
+    return check_cuda(m, "backward");
   }
   const int32_t *stok = m->stok, *spos = m->spos;
   if (m->presorted) {
@@ -849,7 +883,10 @@ gpt_status forward_any(gpt_model* m, bool fuse, float* acc, float scale, int acc
 }
 gpt_status backward_any(gpt_model* m) { return m->bf16m ? backward_t<bf16>(m) : backward_t<float>(m); }
 
+gpt_status lora_step(gpt_model* m, float lr, int step, bool dev_params);
+
 gpt_status adamw_step(gpt_model* m, float lr, int step, bool dev_params = false) {
+  if (m->lora.on) return lora_step(m, lr, step, dev_params);
   Ctx& c = m->ctx;
   int blocks = sumsq_blocks(c);
   sumsq_partials(c, m->g, m->n_total, m->norm_part, blocks);
@@ -875,6 +912,42 @@ gpt_status adamw_step(gpt_model* m, float lr, int step, bool dev_params = false)
   if (dev_params) a.hyper = m->hyper_dev;
   adamw(c, a);
   return check_cuda(m, "adamw");
+}
+
+// The optimiser step with adapters attached: the base weights are frozen.
+// The adapters' gradients (formed at the end of the step's last backward from
+// the merged QKV blocks' gradient) go through clip + AdamW (every adapter
+// tensor is 2-D, hence decayed) alone; the base gradient arena is cleared (the base
+// AdamW is what clears it otherwise); the merged operands are rebuilt.
+gpt_status lora_step(gpt_model* m, float lr, int step, bool dev_params) {
+  Ctx& c = m->ctx;
+  auto& L = m->lora;
+  const int blocks = sumsq_blocks(c);
+  sumsq_partials(c, L.lb.grads, L.n, m->norm_part, blocks);
+  AdamArgs a;
+  a.w = L.lb.params;
+  a.g = L.lb.grads;
+  a.m = L.m;
+  a.v = L.v;
+  a.wb = nullptr;
+  a.n = L.n;
+  a.n_decay = L.n;
+  a.norm_partials = m->norm_part;
+  a.norm_blocks = blocks;
+  a.norm_out = m->scal + 2;
+  a.lr = lr;
+  a.beta1 = m->cfg.beta1;
+  a.beta2 = m->cfg.beta2;
+  a.eps = m->cfg.eps;
+  a.wd = m->cfg.weight_decay;
+  a.clip = m->cfg.grad_clip;
+  a.bc1 = (float)(1.0 - pow((double)m->cfg.beta1, (double)step));
+  a.bc2 = (float)(1.0 - pow((double)m->cfg.beta2, (double)step));
+  if (dev_params) a.hyper = m->hyper_dev;
+  adamw(c, a);
+  cudaMemsetAsync(m->g, 0, (size_t)m->n_total * 4, c.stream);
+  lora_merge(c, L.lb, m->w, m->wb);
+  return check_cuda(m, "lora step");
 }
 
 void bias_corrections(const gpt_model* m, int step, float* bc1, float* bc2) {
@@ -1626,5 +1699,109 @@ gpt_status gpt_kernel_times(gpt_model* m, int32_t cap, const char** names, float
 }
 
 uint64_t gpt_launch_count(gpt_model* m) { return m ? m->ctx.launches : 0; }
+
+
+// ---------------------------------------------------------------- LoRA adapters
+static int lora_blocks(int L, int targets) { return L * __builtin_popcount((unsigned)targets & 7u); }
+
+static size_t lora_bytes(long n) { return 4 * (((size_t)n * 4 + 255) / 256 * 256) + 1024; }
+
+static void drop_train_graphs(gpt_model* m) {
+  for (int k = 0; k < 2; k++) {
+    if (m->gexec[k]) cudaGraphExecDestroy(m->gexec[k]);
+    m->gexec[k] = nullptr;
+    m->warm[k] = 0;
+  }
+}
+
+gpt_status gpt_lora_workspace_bytes(const gpt_config* cfg, int32_t r, int32_t targets, size_t* out) {
+  if (!cfg || !out) return GPT_ERR_INVALID_ARG;
+  if (validate(cfg, nullptr) != GPT_OK) return GPT_ERR_CONFIG;
+  if (r < 1 || r > 256 || targets < 1 || targets > 7) return GPT_ERR_INVALID_ARG;
+  const long n = (long)lora_blocks(cfg->n_layer, targets) * 2 * r * cfg->n_embd;
+  *out = lora_bytes(n);
+  return GPT_OK;
+}
+
+gpt_status gpt_lora_attach(gpt_model* m, int32_t r, float alpha, int32_t targets, const float* h_a, void* d_ws,
+                           size_t ws_bytes) {
+  if (!m || !h_a || !d_ws) return fail(m, GPT_ERR_INVALID_ARG, "lora_attach: null argument");
+  if (!m->bf16m) return fail(m, GPT_ERR_UNSUPPORTED, "lora_attach: adapters need the bf16 operand copies");
+  if (r < 1 || r > 256 || targets < 1 || targets > 7 || !(alpha > 0.f))
+    return fail(m, GPT_ERR_INVALID_ARG, "lora_attach: need 1 <= r <= 256, targets in 1..7, alpha > 0");
+  const int d = m->d, nblk = lora_blocks(m->L, targets);
+  if (nblk > LORA_MAX_BLOCKS) return fail(m, GPT_ERR_UNSUPPORTED, "lora_attach: too many adapted blocks");
+  if (((long)r * d) % 4) return fail(m, GPT_ERR_INVALID_ARG, "lora_attach: r * n_embd must be a multiple of 4");
+  const long n = (long)nblk * 2 * r * d;
+  if (ws_bytes < lora_bytes(n) || (reinterpret_cast<uintptr_t>(d_ws) & 255))
+    return fail(m, GPT_ERR_WORKSPACE_TOO_SMALL, "lora_attach: workspace too small or not 256-byte aligned");
+  if (m->lora.on) {
+    gpt_status s = gpt_lora_detach(m);
+    if (s != GPT_OK) return s;
+  }
+  auto& L = m->lora;
+  uint8_t* base = reinterpret_cast<uint8_t*>(d_ws);
+  const size_t part = ((size_t)n * 4 + 255) / 256 * 256;
+  L.lb.params = reinterpret_cast<float*>(base);
+  L.lb.grads = reinterpret_cast<float*>(base + part);
+  L.m = reinterpret_cast<float*>(base + 2 * part);
+  L.v = reinterpret_cast<float*>(base + 3 * part);
+  L.lb.d = d;
+  L.lb.r = r;
+  L.lb.nblk = nblk;
+  L.lb.scale = alpha / (float)r;
+  L.alpha = alpha;
+  L.targets = targets;
+  L.n = n;
+  int b = 0;
+  for (int l = 0; l < m->L; l++)
+    for (int t = 0; t < 3; t++)
+      if (targets & (1 << t)) L.lb.w_off[b++] = (long)m->layers[l].qkv_w + (long)t * d * d;
+  // A from the caller, B = 0: the adapted model starts as the base model
+  std::vector<float> host((size_t)n, 0.f);
+  for (int k = 0; k < nblk; k++)
+    memcpy(host.data() + (size_t)k * 2 * r * d, h_a + (size_t)k * r * d, (size_t)r * d * 4);
+  Ctx& c = m->ctx;
+  cudaMemcpyAsync(L.lb.params, host.data(), (size_t)n * 4, cudaMemcpyHostToDevice, c.stream);
+  cudaMemsetAsync(L.lb.grads, 0, (size_t)n * 4, c.stream);
+  cudaMemsetAsync(L.m, 0, (size_t)n * 4, c.stream);
+  cudaMemsetAsync(L.v, 0, (size_t)n * 4, c.stream);
+  lora_merge(c, L.lb, m->w, m->wb);
+  drop_train_graphs(m);
+  L.on = true;
+  return sync_and_flags(m, "lora_attach", nullptr);
+}
+
+gpt_status gpt_lora_detach(gpt_model* m) {
+  if (!m) return GPT_ERR_INVALID_ARG;
+  auto& L = m->lora;
+  if (!L.on) return GPT_OK;
+  const long dd = (long)m->d * m->d;
+  for (int k = 0; k < L.lb.nblk; k++) to_bf16(m->ctx, m->w + L.lb.w_off[k], m->wb + L.lb.w_off[k], dd);
+  L.on = false;
+  drop_train_graphs(m);
+  return sync_and_flags(m, "lora_detach", nullptr);
+}
+
+gpt_status gpt_lora_read(gpt_model* m, int32_t which, float* h_out, size_t count) {
+  if (!m || !h_out) return GPT_ERR_INVALID_ARG;
+  auto& L = m->lora;
+  if (!L.on) return fail(m, GPT_ERR_STATE, "lora_read: no adapters attached");
+  if (count != (size_t)L.n || which < 0 || which > 3) return fail(m, GPT_ERR_INVALID_ARG, "lora_read: bad which/count");
+  const float* src = which == 0 ? L.lb.params : which == 1 ? L.lb.grads : which == 2 ? L.m : L.v;
+  cudaStreamSynchronize(m->ctx.stream);
+  if (cudaMemcpy(h_out, src, count * 4, cudaMemcpyDeviceToHost) != cudaSuccess) return check_cuda(m, "lora_read");
+  return GPT_OK;
+}
+
+gpt_status gpt_lora_write(gpt_model* m, const float* h_params, size_t count) {
+  if (!m || !h_params) return GPT_ERR_INVALID_ARG;
+  auto& L = m->lora;
+  if (!L.on) return fail(m, GPT_ERR_STATE, "lora_write: no adapters attached");
+  if (count != (size_t)L.n) return fail(m, GPT_ERR_INVALID_ARG, "lora_write: count must be the adapter size");
+  cudaMemcpyAsync(L.lb.params, h_params, count * 4, cudaMemcpyHostToDevice, m->ctx.stream);
+  lora_merge(m->ctx, L.lb, m->w, m->wb);
+  return sync_and_flags(m, "lora_write", nullptr);
+}
 
 }  // extern "C"

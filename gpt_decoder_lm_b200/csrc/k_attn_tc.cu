@@ -309,6 +309,283 @@ __global__ void __launch_bounds__(192, 2) k_attn_fwd_o(const __grid_constant__ C
   if (warp == 1) tmem_dealloc(tmem, 256);
 }
 
+// ============================================================================
+// forward, ping-pong: one CTA per (pair of 128-query tiles, b, h), 128-key
+// blocks.  Two softmax warpgroups, one per query tile, alternate on the
+// tensor core: while warpgroup 0 turns S0 of key block j into P0, the MMA
+// warp runs P1 V of block j-1 and S1 of block j for warpgroup 1, and the
+// other way round, so the softmax arithmetic of one tile hides the MMAs of
+// the other.  A tile's S is single-buffered: S_t(j+1) is issued after
+// P_t(j) V (tcgen05 MMAs of one thread execute in issue order), which also
+// means O_t holds every P V product of the blocks before j, and none is in
+// flight, while warpgroup t works on block j, so it may rescale O_t in place.
+// One exponential pair in every F_POLY_EVERY is computed on the FMA pipe
+// (exp2_poly2) instead of the SFU, which otherwise bounds the softmax.
+// Tile 0 covers queries [256 p, 256 p + 128) and key blocks 0..2p; tile 1
+// (absent when T / 128 is odd and p is the last pair) queries
+// [256 p + 128, 256 p + 256) and key blocks 0..2p+1.
+// smem: Q0 | Q1 | (K, V)[3 stages] | barriers   (128 KB + 256 B)
+// TMEM: S0 [0,128), S1 [128,256), O0 [256,320), O1 [320,384)  (512 allocated)
+// ============================================================================
+constexpr int F_Q = 0, F_KV = 2 * TILE, F_BAR = 8 * TILE;
+constexpr int F_SMEM = F_BAR + 256;
+constexpr int F_STAGES = 3;
+constexpr int F_POLY_EVERY = 4;
+
+template <bool DROP>
+__global__ void __maxnreg__(200) k_attn_fwd_pp(const __grid_constant__ CUtensorMap t128, AttnTcArgs a) {
+  pdl_trigger();
+  const DropKey dk = DROP ? drop_live(a.drop) : a.drop;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (smem_u32(smem) & 1023) {  // swizzled tiles need 1024-byte alignment
+    if (threadIdx.x == 0) atomicOr(a.flags, FLAG_TIMEOUT);
+    return;
+  }
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + F_BAR);
+  const uint32_t q_full = smem_u32(bars + 0);
+  const uint32_t kv_full0 = smem_u32(bars + 1), kv_empty0 = smem_u32(bars + 1 + F_STAGES);
+  const uint32_t s_full0 = smem_u32(bars + 1 + 2 * F_STAGES), p_full0 = s_full0 + 16, pv_done0 = s_full0 + 32;
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + 7 + 2 * F_STAGES);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tslot + 1);
+  const uint32_t sb = smem_u32(smem);
+
+  const int nqb = a.T / 128, npair = (nqb + 1) / 2;
+  const int p = npair - 1 - (int)blockIdx.y;  // longest pairs first
+  const int bh = blockIdx.x, b = bh / a.H, h = bh % a.H;
+  const bool has1 = 2 * p + 1 < nqb;
+  const int jl0 = 2 * p, jl1 = 2 * p + 1;    // last key block of each tile
+  const int nk = has1 ? jl1 + 1 : jl0 + 1;   // key blocks of the CTA
+  const int row0 = b * a.T;
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int s = 0; s < F_STAGES; s++) {
+      mbar_init(kv_full0 + 8 * s, 1);
+      mbar_init(kv_empty0 + 8 * s, 1);
+    }
+    for (int t = 0; t < 2; t++) {
+      mbar_init(s_full0 + 8 * t, 1);
+      mbar_init(p_full0 + 8 * t, 4);
+      mbar_init(pv_done0 + 8 * t, 1);
+    }
+    *abort_flag = 0;
+    fence_barrier_init();
+    prefetch_tmap(&t128);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tslot), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tslot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      mbar_expect_tx(q_full, (has1 ? 2 : 1) * TILE);
+      tma_load_3d(sb + F_Q, &t128, q_full, 0, h, row0 + 2 * p * 128);
+      if (has1) tma_load_3d(sb + F_Q + TILE, &t128, q_full, 0, h, row0 + (2 * p + 1) * 128);
+      int issued = 0;
+      bool ok = true;
+      for (int j = 0; j < nk; j++) {
+        const int s = j % F_STAGES;
+        const uint32_t fb = kv_full0 + 8 * s;
+        if (!(ok = mbar_wait(kv_empty0 + 8 * s, ((j / F_STAGES) & 1) ^ 1, abort_flag, a.flags))) break;
+        mbar_expect_tx(fb, 2 * TILE);
+        tma_load_3d(sb + F_KV + s * 2 * TILE, &t128, fb, 0, a.H + h, row0 + j * 128);
+        tma_load_3d(sb + F_KV + s * 2 * TILE + TILE, &t128, fb, 0, 2 * a.H + h, row0 + j * 128);
+        issued = j + 1;
+      }
+      if (!ok) {  // the loads already issued land before the CTA can exit
+        mbar_wait(q_full, 0, abort_flag, a.flags);
+        for (int j = issued - F_STAGES < 0 ? 0 : issued - F_STAGES; j < issued; j++)
+          mbar_wait(kv_full0 + 8 * (j % F_STAGES), (j / F_STAGES) & 1, abort_flag, a.flags);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t id_s = idesc_bf16_f32(128, 128, false, false);
+      constexpr uint32_t id_pv = idesc_bf16_f32(128, 64, false, true);
+      bool ok = mbar_wait(q_full, 0, abort_flag, a.flags);
+      // S_t(j) = Q_t K_j^T (M 128 queries, N 128 keys, K 64)
+      auto issue_s = [&](int t, int j) {
+        const uint32_t kt = sb + F_KV + (j % F_STAGES) * 2 * TILE;
+#pragma unroll
+        for (int kk = 0; kk < 4; kk++)
+          mma_bf16_ss(tmem + 128 * t, desc_k(sb + F_Q + t * TILE, TILE, kk), desc_k(kt, TILE, kk), id_s, kk > 0);
+        mma_commit(s_full0 + 8 * t);
+      };
+      // O_t += P_t(i) V_i: P over the first 64 columns of S_t (K = 128 keys), V MN-major (N = 64)
+      auto issue_pv = [&](int t, int i) -> bool {
+        if (!mbar_wait(p_full0 + 8 * t, i & 1, abort_flag, a.flags)) return false;
+        tc_fence_after();
+        const uint32_t v = sb + F_KV + (i % F_STAGES) * 2 * TILE + TILE;
+#pragma unroll
+        for (int kk = 0; kk < 8; kk++)
+          mma_bf16_ts(tmem + 256 + 64 * t, tmem + 128 * t + 8 * kk, desc_mn64(v, kk), id_pv,
+                      (i > 0 || kk > 0) ? 1u : 0u);
+        return true;
+      };
+      for (int j = 0; j < nk && ok; j++) {
+        const int s = j % F_STAGES;
+        if (!(ok = mbar_wait(kv_full0 + 8 * s, (j / F_STAGES) & 1, abort_flag, a.flags))) break;
+        tc_fence_after();
+        if (j <= jl0) {
+          if (j > 0 && !(ok = issue_pv(0, j - 1))) break;
+          issue_s(0, j);
+        } else if (j == jl0 + 1) {
+          if (!(ok = issue_pv(0, j - 1))) break;
+          mma_commit(pv_done0);
+        }
+        if (has1) {
+          if (j > 0 && !(ok = issue_pv(1, j - 1))) break;
+          if (j > 0) mma_commit(kv_empty0 + 8 * ((j - 1) % F_STAGES));
+          issue_s(1, j);
+        } else if (j > 0) {
+          mma_commit(kv_empty0 + 8 * ((j - 1) % F_STAGES));
+        }
+      }
+      if (ok) {
+        const int t = has1 ? 1 : 0;
+        if (issue_pv(t, nk - 1)) mma_commit(pv_done0 + 8 * t);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ softmax warpgroups
+    const int t = (warp - 2) >> 2;  // query tile
+    const int quad = warp & 3;
+    const int r = quad * 32 + lane;
+    const int qi = (2 * p + t) * 128 + r;
+    const bool live = t == 0 || has1;
+    const int jl = t == 0 ? jl0 : jl1;
+    const uint32_t trow = tmem + ((uint32_t)(quad * 32) << 16);
+    const uint32_t s_col = 128 * t, o_col = 256 + 64 * t;
+    const float sl2 = a.scale_log2;
+    float m = -INFINITY, l = 0.f;  // reference maximum (log2 units) and row sum against it
+    const uint64_t ebase = ((uint64_t)bh * a.T + qi) * a.T;
+    bool ok = live;
+    for (int j = 0; j <= jl && ok; j++) {
+      if (!(ok = mbar_wait(s_full0 + 8 * t, j & 1, abort_flag, a.flags))) break;
+      tc_fence_after();
+      uint32_t v0[32], v1[32], v2[32], v3[32];
+      tmem_ld_32x32b_x32(trow + s_col, v0);
+      tmem_ld_32x32b_x32(trow + s_col + 32, v1);
+      tmem_ld_32x32b_x32(trow + s_col + 64, v2);
+      tmem_ld_32x32b_x32(trow + s_col + 96, v3);
+      tmem_ld_wait();
+      const bool diag = j == jl;  // key j*128 + i is visible iff i <= r
+      float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
+      if (!diag) {
+#pragma unroll
+        for (int i = 0; i < 32; i++) {
+          mx0 = fmaxf(mx0, __uint_as_float(v0[i]));
+          mx1 = fmaxf(mx1, __uint_as_float(v1[i]));
+          mx2 = fmaxf(mx2, __uint_as_float(v2[i]));
+          mx3 = fmaxf(mx3, __uint_as_float(v3[i]));
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; i++) {
+          if (i <= r) mx0 = fmaxf(mx0, __uint_as_float(v0[i]));
+          if (i + 32 <= r) mx1 = fmaxf(mx1, __uint_as_float(v1[i]));
+          if (i + 64 <= r) mx2 = fmaxf(mx2, __uint_as_float(v2[i]));
+          if (i + 96 <= r) mx3 = fmaxf(mx3, __uint_as_float(v3[i]));
+        }
+      }
+      const float bm = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;
+      if (j == 0) {
+        m = bm;  // key 0 is visible to every row, so m is finite from here on
+      } else {
+        const bool need = bm > m + RESCALE_LOG2;
+        if (__any_sync(0xffffffffu, need)) {
+          // O_t holds P V of blocks < j and nothing is in flight into it
+          const float sc = need ? ex2(m - bm) : 1.f;
+#pragma unroll
+          for (int q = 0; q < 4; q++) {  // 16 columns at a time: S stays in registers
+            uint32_t o[16];
+            tmem_ld_32x32b_x16(trow + o_col + 16 * q, o);
+            tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 16; i++) o[i] = __float_as_uint(__uint_as_float(o[i]) * sc);
+            tmem_st_32x32b_x16(trow + o_col + 16 * q, o);
+          }
+          l *= sc;
+          if (need) m = bm;
+        }
+      }
+      // probabilities of the 128 keys, packed bf16 pairs (P = the A operand of P V)
+      const uint64_t neg_m = f2c(-m), scl = f2c(sl2);
+      float lsum = 0.f;
+#pragma unroll
+      for (int half = 0; half < 2; half++) {  // 64 keys per half: its packed P goes to TMEM before the next
+        uint32_t pk[32];
+#pragma unroll
+        for (int cc = 0; cc < 2; cc++) {
+        const int c = 2 * half + cc;
+        const uint32_t* vc = c == 0 ? v0 : c == 1 ? v1 : c == 2 ? v2 : v3;
+#pragma unroll
+        for (int i = 0; i < 32; i += 2) {
+          const int k = 32 * c + i;  // key offset in the block
+          const uint64_t x2 = f2fma(f2(__uint_as_float(vc[i]), __uint_as_float(vc[i + 1])), scl, neg_m);
+          float p0, p1;
+          if (((k >> 1) % F_POLY_EVERY) == F_POLY_EVERY - 1) {
+            const float2 e = f2split(exp2_poly2(x2));
+            p0 = e.x;
+            p1 = e.y;
+          } else {
+            const float2 x = f2split(x2);
+            p0 = ex2(x.x);
+            p1 = ex2(x.y);
+          }
+          if (diag) {
+            if (k > r) p0 = 0.f;
+            if (k + 1 > r) p1 = 0.f;
+          }
+          lsum += p0 + p1;
+          if (DROP) {
+            const uint64_t e = ebase + (uint64_t)j * 128 + k;
+            p0 *= drop_mul(dk, e);
+            p1 *= drop_mul(dk, e + 1);
+          }
+          pk[(k - 64 * half) >> 1] = pack2(p0, p1);
+        }
+        }
+        tmem_st_32x32b_x32(trow + s_col + 32 * half, pk);
+      }
+      l += lsum;
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(p_full0 + 8 * t);  // one arrival per warp of the warpgroup
+    }
+    if (ok) ok = mbar_wait(pv_done0 + 8 * t, 0, abort_flag, a.flags);
+    if (ok) {
+      tc_fence_after();
+      uint32_t o0[32], o1[32];
+      ld64(trow + o_col, o0, o1);
+      const float inv = 1.0f / l;
+      uint4* dst = reinterpret_cast<uint4*>(a.o_out + ((size_t)(row0 + qi) * a.H + h) * 64);
+#pragma unroll
+      for (int q = 0; q < 8; q++) {
+        const uint32_t* x = q < 4 ? o0 + 8 * q : o1 + 8 * (q - 4);
+        dst[q] = make_uint4(pack2(__uint_as_float(x[0]) * inv, __uint_as_float(x[1]) * inv),
+                            pack2(__uint_as_float(x[2]) * inv, __uint_as_float(x[3]) * inv),
+                            pack2(__uint_as_float(x[4]) * inv, __uint_as_float(x[5]) * inv),
+                            pack2(__uint_as_float(x[6]) * inv, __uint_as_float(x[7]) * inv));
+      }
+      a.lse[(size_t)bh * a.T + qi] = (m + log2f(l)) * LN2;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, 512);
+}
+
 // packed bf16 pair column of element column c (0..63) of a 64-column block:
 // the half that owns c writes inside its own fp32 columns
 __device__ __forceinline__ int pcol(int c) { return (c & 32) + ((c & 31) >> 1); }
@@ -854,6 +1131,22 @@ bool attn_fwd_tc(Ctx& c, const AttnDesc& d) {
   LaunchScope s(c, "attn_fwd_tc");
   if (drop) k_attn_fwd_o<true><<<grid, 192, D_SMEM, c.stream>>>(tq, tkv64, make_args(d, c.flags));
   else k_attn_fwd_o<false><<<grid, 192, D_SMEM, c.stream>>>(tq, tkv64, make_args(d, c.flags));
+  return true;
+}
+
+// the ping-pong forward (two 128-query tiles per CTA, 128-key blocks)
+bool attn_fwd_tc_pp(Ctx& c, const AttnDesc& d) {
+  CUtensorMap t128;
+  long rows = (long)d.B * d.T;
+  if (!map_rows(&t128, d.qkv, 3 * d.H, rows, 128)) return false;
+  const bool drop = d.drop.active;
+  cudaFuncSetAttribute(drop ? k_attn_fwd_pp<true> : k_attn_fwd_pp<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                       F_SMEM);
+  const int npair = (d.T / 128 + 1) / 2;
+  dim3 grid(d.B * d.H, npair);
+  LaunchScope s(c, "attn_fwd_tc");
+  if (drop) k_attn_fwd_pp<true><<<grid, 320, F_SMEM, c.stream>>>(t128, make_args(d, c.flags));
+  else k_attn_fwd_pp<false><<<grid, 320, F_SMEM, c.stream>>>(t128, make_args(d, c.flags));
   return true;
 }
 

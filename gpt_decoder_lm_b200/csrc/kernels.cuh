@@ -129,6 +129,7 @@ bool attn_tc_shape_ok(int T, int hd);
 bool attn_tc_supported(const AttnDesc& a);  // shape rule plus 16-byte aligned pointers
 // false: a tensor map could not be encoded (nothing launched)
 bool attn_fwd_tc(Ctx& c, const AttnDesc& a);
+bool attn_fwd_tc_pp(Ctx& c, const AttnDesc& a);  // two query tiles per CTA, 128-key blocks
 bool attn_bwd_tc(Ctx& c, const AttnDesc& a);
 // decoding: o [B, H*hd] = attention of position t against positions 0..t of
 // the cache qkv [B, T, 3, H, hd]
@@ -205,6 +206,20 @@ struct AdamArgs {
   const float* hyper = nullptr;  // when set: {lr, bc1, bc2} read from device memory
 };
 void adamw(Ctx& c, const AdamArgs& a);
+
+// LoRA adapters on row blocks (d x d) of the fused QKV weight
+constexpr int LORA_MAX_BLOCKS = 144;
+struct LoraBlocks {
+  int d = 0, r = 0, nblk = 0;
+  float scale = 0.f;            // alpha / r
+  float* params = nullptr;      // per block: A [r, d], then B [d, r]
+  float* grads = nullptr;       // the same layout
+  long w_off[LORA_MAX_BLOCKS];  // element offset of each block's first row in the weight arena
+};
+// wb (bf16 operand copy) of every adapted block <- W0 + scale B A
+void lora_merge(Ctx& c, const LoraBlocks& lb, const float* w, bf16* wb);
+// adapter gradients from the gradient g of the merged weights (weight arena layout)
+void lora_grads(Ctx& c, const LoraBlocks& lb, const float* g);
 void to_bf16(Ctx& c, const float* src, bf16* dst, long n);
 void argmax_rows(Ctx& c, const void* x, int is_bf16, long rows, int cols, int ld, int32_t* out);
 void dropout_mask(Ctx& c, DropKey k, long n, uint8_t* out);

@@ -369,6 +369,47 @@ gpt_status gpt_gemm_dw_accumulate_noalloc(int32_t M, int32_t N, int32_t K, const
                                           const void* d_b, int64_t ldb, float* d_dw, int32_t split_k,
                                           void* cuda_stream);
 
+/* ---------------------------------------------------------------- LoRA adapters
+ * Low-rank adapters on row blocks of each layer's fused QKV weight ("使用
+ * nanoGPT 构建中型 GPT 微调管道" page, LoRA integration paragraph): the base
+ * weights stay frozen and a block computes h = W0 x + s B (A x), s = alpha / r,
+ * A [r, d], B [d, r].  targets: bit 0 q (rows 0..d-1), bit 1 k (d..2d-1),
+ * bit 2 v (2d..3d-1); the page adapts q and v (targets = 5).  Adapter layout
+ * (params, grads, Adam moments alike): per adapted block, layers ascending and
+ * q, k, v ascending within a layer, A row-major then B row-major.
+ * While attached, gpt_train_step / gpt_train_step_host / gpt_clip_adamw_step
+ * train the adapters only: the step's forward and backward run on the merged
+ * operand W0 + s B A, the adapters' gradients follow from the merged blocks'
+ * gradient G (dB = s G A^T, dA = s B^T G), clip + AdamW (the config's
+ * hyper-parameters; every adapter tensor decayed) run over the adapters, and
+ * the base weights and their Adam state are not touched.  The reported grad
+ * norm is the adapters'.  bf16 models only (GPT_ERR_UNSUPPORTED otherwise). */
+
+/* Bytes of device memory the adapters of (cfg, r, targets) need. */
+gpt_status gpt_lora_workspace_bytes(const gpt_config* cfg, int32_t r, int32_t targets, size_t* out);
+
+/* Attaches adapters of rank r (1..256) on `targets`: h_a (host) holds A of
+ * every adapted block ([blocks][r][d] fp32; random numbers are inputs), B
+ * starts at zero, so the model is unchanged until the first step.  d_ws:
+ * device memory of gpt_lora_workspace_bytes, 256-byte aligned, owned by the
+ * caller until detach.  Replaces adapters already attached.  Synchronising. */
+gpt_status gpt_lora_attach(gpt_model* m, int32_t r, float alpha, int32_t targets, const float* h_a, void* d_ws,
+                           size_t ws_bytes);
+
+/* Detaches the adapters: the QKV operands return to the base weights (the
+ * adapters are not merged into them).  Synchronising; no-op when none. */
+gpt_status gpt_lora_detach(gpt_model* m);
+
+/* Copies the adapter parameters (which 0), their gradients (1: formed by the
+ * backward of the step's last micro-batch, zero again after the optimiser
+ * step), or the Adam moments (2, 3) to host memory; count must be the adapter
+ * size.  Synchronising. */
+gpt_status gpt_lora_read(gpt_model* m, int32_t which, float* h_out, size_t count);
+
+/* Replaces the adapter parameters (host, adapter layout) and rebuilds the
+ * merged operands.  Synchronising. */
+gpt_status gpt_lora_write(gpt_model* m, const float* h_params, size_t count);
+
 #ifdef __cplusplus
 }
 #endif

@@ -74,10 +74,15 @@ def run_case(backend, B, T, H, p, seed=0, qkv_np=None):
 # the last three are the benchmarked shapes: GPT-2 124M (T 1024, 12 heads;
 # two batch rows so the longest-block-first order spans several (b, h)) and
 # GPT-2 XL (T 1024, 25 heads)
-@pytest.mark.parametrize("B,T,H", [(2, 256, 3), (1, 512, 2), (1, 128, 1), (2, 1024, 12), (1, 1024, 25)])
+@pytest.mark.parametrize("B,T,H", [(2, 256, 3), (1, 512, 2), (1, 128, 1), (1, 384, 2), (2, 1024, 12),
+                                   (1, 1024, 25)])
 @pytest.mark.parametrize("p", [0.0, 0.1], ids=["nodrop", "dropout"])
-def test_attention_tensor_core(B, T, H, p):
-    run_case(1, B, T, H, p)
+@pytest.mark.parametrize("backend", [1, 2], ids=["fwd64", "fwd_pingpong"])
+def test_attention_tensor_core(B, T, H, p, backend):
+    # backend 2: the forward with two 128-query tiles per CTA and 128-key
+    # blocks (T = 128 and 384 leave a CTA with one tile); the backward is the
+    # same kernel pair for both
+    run_case(backend, B, T, H, p)
 
 
 @pytest.mark.parametrize("p", [0.0, 0.1], ids=["nodrop", "dropout"])
@@ -104,3 +109,4 @@ def test_attention_rescale_path():
     x[:, :, 0] += 21.0 * u
     x[:, :, 1] += (np.arange(T) / T * 21.0)[None, :, None, None] * u
     run_case(1, B, T, H, 0.0, qkv_np=x)
+    run_case(2, B, T, H, 0.0, qkv_np=x)

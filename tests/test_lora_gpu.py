@@ -1,0 +1,119 @@
+"""LoRA adapters on the QKV blocks (gpt_lora_*) against the LoRA oracle
+(oracle/lora.py): the model is unchanged while B = 0 and after detaching,
+the adapter gradients match, the training steps match, and the base weights
+stay bit-frozen."""
+
+import numpy as np
+import pytest
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+if not torch.cuda.is_available():
+    pytest.skip("needs a GPU", allow_module_level=True)
+
+import oracle  # noqa: E402
+from oracle import lora as LR  # noqa: E402
+from gpt_decoder_lm_b200 import binding as gb  # noqa: E402
+from gpt_decoder_lm_b200 import workloads as W  # noqa: E402
+from tests.helpers import oracle_config, rel_l2  # noqa: E402
+
+OVER = dict(n_layer=2, batch_size=4, block_size=128, grad_accum=2)
+Q_V = 1 | 4
+
+
+def dev(a):
+    return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+
+
+def flat(oc, lc, Lp):
+    return np.concatenate([np.concatenate([Lp[na].ravel(), Lp[nb].ravel()])
+                           for _, _, na, nb in LR.lora_names(oc, lc)]).astype(np.float32)
+
+
+def unflat(oc, lc, v):
+    out, o, r, d = {}, 0, lc.r, oc.n_embd
+    for _, _, na, nb in LR.lora_names(oc, lc):
+        out[na] = v[o:o + r * d].reshape(r, d)
+        o += r * d
+        out[nb] = v[o:o + d * r].reshape(d, r)
+        o += d * r
+    return out
+
+
+def setup(r=4, alpha=16.0, b_std=0.0, seed=3):
+    w = W.CHAR
+    cfg = gb.make_config(w, **OVER)
+    m = gb.Model(cfg, seed=w.weight_seed)
+    oc = oracle_config(w).with_(**OVER)
+    P = oracle.init_params(oc, w.weight_seed)
+    lc = LR.LoraConfig(r=r, alpha=alpha, targets=("q", "v"))
+    Lp = LR.init_lora(oc, lc, seed, b_std=b_std)
+    A = np.stack([Lp[na] for _, _, na, _ in LR.lora_names(oc, lc)])
+    return w, cfg, m, oc, P, lc, Lp, A
+
+
+def _batch(w, cfg, seed):
+    idx, tgt = W.random_batch(w, seed, cfg.batch_size, cfg.block_size)
+    return idx, tgt
+
+
+def test_zero_B_and_detach_leave_the_base_model():
+    w, cfg, m, oc, P, lc, Lp, A = setup()
+    idx, tgt = _batch(w, cfg, 5)
+    base = m.forward_loss(dev(idx), dev(tgt))
+    m.lora_attach(lc.r, lc.alpha, Q_V, A)
+    assert m.forward_loss(dev(idx), dev(tgt)) == base  # B = 0: merged operand = base operand
+    m.lora_write(flat(oc, lc, LR.init_lora(oc, lc, 4, b_std=0.1)))
+    assert m.forward_loss(dev(idx), dev(tgt)) != base
+    m.lora_detach()
+    assert m.forward_loss(dev(idx), dev(tgt)) == base
+    m.close()
+
+
+def test_adapter_gradients_match_oracle():
+    w, cfg, m, oc, P, lc, Lp, A = setup(b_std=0.05)
+    m.lora_attach(lc.r, lc.alpha, Q_V, A)
+    m.lora_write(flat(oc, lc, Lp))
+    idx, tgt = _batch(w, cfg, 6)
+    loss = m.forward_loss(dev(idx), dev(tgt))
+    m.backward()
+    got = unflat(oc, lc, m.lora_read(1))
+    # a lone micro-batch carries the step's 1 / grad_accum scale, as in the base parity tests
+    oloss, GL, _ = LR.loss_and_grads(oc, P, Lp, lc, idx.astype(np.int64), tgt.astype(np.int64), None,
+                                     1.0 / cfg.grad_accum)
+    assert abs(loss - oloss) <= 2e-3, (loss, oloss)
+    bad = {k: rel_l2(got[k], GL[k]) for k in GL if rel_l2(got[k], GL[k]) > 2e-2}
+    assert not bad, bad
+    m.close()
+
+
+def test_training_steps_match_oracle_and_freeze_the_base():
+    w, cfg, m, oc, P, lc, Lp, A = setup(b_std=0.0)
+    m.lora_attach(lc.r, lc.alpha, Q_V, A)
+    base0 = m.get(gb.GPT_PARAM)
+    stream = W.token_stream(w, n=1 << 16)
+    sd = dev(stream.astype(np.int32))
+    S = LR.LoraAdamState()
+    for step in range(1, 6):
+        lr = 1e-3
+        loss, norm = m.train_step(sd, w.data_seed, lr, step)
+        oloss, onorm = LR.train_step(oc, P, Lp, lc, S, stream.astype(np.int64), w.data_seed, lr, step)
+        assert abs(loss - oloss) <= 2e-3, (step, loss, oloss)
+        assert abs(norm - onorm) <= 2e-2 * onorm, (step, norm, onorm)
+    assert rel_l2(m.lora_read(0), flat(oc, lc, Lp)) <= 1e-3
+    assert not m.lora_read(1).any()  # gradients cleared by the optimiser step
+    base1 = m.get(gb.GPT_PARAM)
+    for k in base0:
+        assert np.array_equal(base0[k], base1[k]), k
+    m.close()
+
+
+def test_fp32_models_refuse_adapters():
+    w = W.MICRO
+    cfg = gb.make_config(w)
+    m = gb.Model(cfg, seed=w.weight_seed)
+    with pytest.raises(gb.GptError) as e:
+        m.lora_attach(2, 4.0, Q_V, np.zeros((2, 2, w.n_embd), np.float32))
+    assert e.value.name == "GPT_ERR_UNSUPPORTED"
+    m.close()
