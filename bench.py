@@ -6,9 +6,11 @@ A step is one full optimiser step of the GPT-2 124M workload (vocab 50257,
 12 layers, 12 heads, d 768, block 1024, micro-batch 12, grad-accum 5 ->
 61,440 tokens): batch gather from a device-resident synthetic token stream,
 forward, cross-entropy, backward, clip and AdamW, all in libgpt.so.  For
-N > 1 (torchrun) every rank trains its own replica on its own data: the
-step does not shard, so there is no collective on the data path; the
-barrier and the max-over-ranks timing use torch.distributed.
+N > 1 (torchrun) every rank gathers its own micro-batches and the replicas'
+gradients are averaged before clip + AdamW (data-parallel training: a
+bucketed NCCL all-reduce on a second stream, overlapping the backward;
+gpt_decoder_lm_b200/ddp.py); --replicas runs independent replicas instead.
+The barrier and the max-over-ranks timing use torch.distributed.
 
 `--impl reference` times the CPU oracle (float64 numpy) on a bounded sample
 of the same workload on the host cores (rank 0 only).
@@ -426,6 +428,19 @@ def run_ours(args, w, rank, world, local_rank):
     def lr_at(i):
         return gb.lr_cosine(w.lr, i, 100, 5000)
 
+    # N > 1: data-parallel training (the gradients of the replicas averaged by a
+    # bucketed NCCL all-reduce that overlaps the backward) unless --replicas
+    use_ddp = world > 1 and not args.replicas
+    trainer = None
+    if use_ddp:
+        from gpt_decoder_lm_b200 import ddp
+        trainer = ddp.DataParallelTrainer(model)
+
+    def step_fn(i, sync=False):
+        if trainer is not None:
+            return trainer.step(d_stream, data_seed, lr_at(i), i, sync=sync)
+        return model.train_step(d_stream, data_seed, lr_at(i), i, sync=sync)
+
     # clock sampler first, so that its start-up falls before the timed region
     clocks = Clocks(local_rank) if rank == 0 else None
     if clocks:
@@ -434,7 +449,7 @@ def run_ours(args, w, rank, world, local_rank):
     # also loads torch's fill kernel, which must not land in the timed region)
     for _ in range(args.warmup):
         st += 1
-        model.train_step(d_stream, data_seed, lr_at(st), st, sync=False)
+        step_fn(st)
         flush.zero_()
     torch.cuda.synchronize()
     if clocks:
@@ -449,7 +464,7 @@ def run_ours(args, w, rank, world, local_rank):
     h0 = time.perf_counter()
     for k in range(args.steps):
         st += 1
-        model.train_step(d_stream, data_seed, lr_at(st), st, sync=False)
+        step_fn(st)
         flush.zero_()          # L2 flush between steps (256 MiB > 126 MB L2)
         evs[k + 1].record()
     host_enqueue_ms = (time.perf_counter() - h0) * 1000.0 / args.steps
@@ -461,7 +476,7 @@ def run_ours(args, w, rank, world, local_rank):
     ms = ev0.elapsed_time(ev1)
     ms_max = reduce_max(ms, dev)
     clk = clocks.stop() if clocks else None
-    loss, norm = model.train_step(d_stream, data_seed, lr_at(st + 1), st + 1)
+    loss, norm = step_fn(st + 1, sync=True)
     st += 1
     value = world * args.steps * tok_step / (ms_max / 1000.0)
 
@@ -487,9 +502,14 @@ def run_ours(args, w, rank, world, local_rank):
         hb.append((xi, yi))
     # untimed warm-up of the host-buffer entry point (its first calls run eagerly
     # and capture its CUDA graph)
+    def host_step(xi, yi, i):
+        if trainer is not None:
+            return trainer.step_host(xi, yi, lr_at(i), i)
+        return model.train_step_host(xi, yi, lr_at(i), i)
+
     for xi, yi in hb[:2]:
         st += 1
-        model.train_step_host(xi, yi, lr_at(st), st)
+        host_step(xi, yi, st)
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
@@ -497,7 +517,7 @@ def run_ours(args, w, rank, world, local_rank):
     e0.record()
     for xi, yi in hb:
         st += 1
-        model.train_step_host(xi, yi, lr_at(st), st)
+        host_step(xi, yi, st)
     e1.record()
     torch.cuda.synchronize()
     e2e_ms = reduce_max(e0.elapsed_time(e1), dev)
@@ -544,7 +564,9 @@ def run_ours(args, w, rank, world, local_rank):
             "config": {"workload": w.name, "vocab": w.vocab_size, "n_layer": w.n_layer, "n_head": w.n_head,
                        "n_embd": w.n_embd, "seq_len": w.block_size, "micro_batch": w.batch_size,
                        "grad_accum": w.grad_accum, "tokens_per_step_per_gpu": tok_step,
-                       "global_batch_tokens": tok_step * world, "parallelism": f"replicas x{world}",
+                       "global_batch_tokens": tok_step * world,
+                       "parallelism": f"dp{world} (bucketed NCCL all-reduce overlapped with the backward)"
+                       if use_ddp else f"replicas x{world}",
                        "l2": "256 MiB buffer zeroed between timed steps; step working set ~8 GB"},
             "mfu": {"nominal_2250": mfu_nom, "measured_peak": mfu_meas, "flops_per_token": fpt},
             "roofline": roofline,
@@ -615,6 +637,8 @@ def main():
     ap.add_argument("--workload", default=W.GPT2_124M.name, choices=list(W.ALL))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-configs", action="store_true", help="skip the other workloads' step timings")
+    ap.add_argument("--replicas", action="store_true",
+                    help="N > 1: independent replicas instead of data-parallel training")
     ap.add_argument("--kernels", action="store_true",
                     help="one launch of each hot kernel at the workload's shapes (for ncu), then exit")
     args = ap.parse_args()

@@ -54,6 +54,12 @@ _PROTOS = {
     "gpt_param_count": (SZ, [P]),
     "gpt_config_kernel_paths": (I32, [P, P]),
     "gpt_workspace_bytes": (I32, [P, P]),
+    "gpt_grad_buckets": (I32, [P, I32, P, P, P, P]),
+    "gpt_grad_arena": (I32, [P, P, P]),
+    "gpt_train_step_accumulate": (I32, [P, P, U64, U64, I32, P]),
+    "gpt_stream_wait_bucket": (I32, [P, I32, P]),
+    "gpt_step_loss": (I32, [P, P]),
+    "gpt_train_step_host_accumulate": (I32, [P, P, P, I32, P]),
     "gpt_lr_cosine": (F32, [F32, I32, I32, I32]),
     "gpt_lr_linear": (F32, [F32, I32, I32]),
     "gpt_create": (I32, [P, U64, P, SZ, P, P]),
@@ -165,6 +171,18 @@ def make_config(w, **over) -> GptConfig:
     return c
 
 
+def grad_buckets(cfg: GptConfig):
+    """The gradient exchange plan: [(offset, count, bucket)] in the order the
+    backward finalises the buckets."""
+    n = C.c_int32(0)
+    _check(lib().gpt_grad_buckets(C.byref(cfg), 0, None, None, None, C.byref(n)), None, "grad_buckets")
+    off = (C.c_int64 * n.value)()
+    cnt = (C.c_int64 * n.value)()
+    bkt = (C.c_int32 * n.value)()
+    _check(lib().gpt_grad_buckets(C.byref(cfg), n.value, off, cnt, bkt, C.byref(n)), None, "grad_buckets")
+    return [(int(off[i]), int(cnt[i]), int(bkt[i])) for i in range(n.value)]
+
+
 def kernel_paths(cfg: GptConfig) -> int:
     """GPT_PATH_* bits: which kernels a model with this config runs."""
     n = C.c_uint32(0)
@@ -244,6 +262,36 @@ class Model:
         _check(lib().gpt_train_step_host(self.h, _ptr(h_idx), _ptr(h_tgt), lr, step, C.byref(loss), C.byref(norm)),
                self.h, "train_step_host")
         return float(loss.value), float(norm.value)
+
+    def train_step_accumulate(self, stream_tokens, data_seed: int, step: int, sync: bool = False):
+        loss = C.c_float()
+        _check(lib().gpt_train_step_accumulate(self.h, _ptr(stream_tokens), stream_tokens.numel(), data_seed, step,
+                                               C.byref(loss) if sync else None), self.h, "train_step_accumulate")
+        return float(loss.value) if sync else None
+
+    def train_step_host_accumulate(self, h_idx, h_tgt, step: int, sync: bool = False):
+        loss = C.c_float()
+        _check(lib().gpt_train_step_host_accumulate(self.h, _ptr(h_idx), _ptr(h_tgt), step,
+                                                    C.byref(loss) if sync else None), self.h,
+               "train_step_host_accumulate")
+        return float(loss.value) if sync else None
+
+    def step_loss(self) -> float:
+        out = C.c_float()
+        _check(lib().gpt_step_loss(self.h, C.byref(out)), self.h, "step_loss")
+        return float(out.value)
+
+    def stream_wait_bucket(self, bucket: int, stream):
+        _check(lib().gpt_stream_wait_bucket(self.h, bucket, stream.cuda_stream), self.h, "stream_wait_bucket")
+
+    def grad_arena(self):
+        """The fp32 gradient arena as a torch tensor view of the workspace."""
+        import torch
+        p, n = C.c_void_p(), C.c_int64()
+        _check(lib().gpt_grad_arena(self.h, C.byref(p), C.byref(n)), self.h, "grad_arena")
+        off = p.value - self.ws.data_ptr()
+        assert off % 4 == 0 and off >= 0
+        return self.ws[off:off + 4 * n.value].view(torch.float32)
 
     def gather_batch(self, stream_tokens, data_seed: int, step: int, micro: int, idx, tgt):
         _check(lib().gpt_gather_batch(self.h, _ptr(stream_tokens), stream_tokens.numel(), data_seed, step, micro,

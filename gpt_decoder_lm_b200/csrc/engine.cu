@@ -3,6 +3,7 @@
 // weights from the seed, and enqueues the kernels of one training step on the
 // model's stream.  No device allocation happens here.
 #include <math.h>
+#include <stdlib.h>
 #include <stdarg.h>
 #include <stdio.h>
 #include <string.h>
@@ -144,6 +145,7 @@ struct gpt_model {
   // CUDA-graph replay of gpt_generate for a repeated call shape
   cudaGraphExec_t gen_exec = nullptr;
   int gen_warm = 0;
+  bool capturing = false;  // a graph of the step is being captured
   uint64_t gen_launches = 0;
   uint64_t gen_key[8] = {0, 0, 0, 0, 0, 0, 0, 0};
   int part_cap = 0;                 // partial rows per norm instance
@@ -166,11 +168,18 @@ struct gpt_model {
     float *m = nullptr, *v = nullptr;  // Adam moments of the adapters
     long n = 0;                        // adapter parameters (2 r d per block)
   } lora;
-  cudaGraphExec_t gexec[2] = {nullptr, nullptr};
-  uint64_t graph_launches[2] = {0, 0};
-  int warm[2] = {0, 0};
-  const void* g_dstream = nullptr;
-  uint64_t g_len = 0, g_seed = 0;
+  // graph kinds: [0] device token stream, [1] host batches, [2] / [3] the
+  // same without the optimiser (the data-parallel step's accumulate part)
+  cudaGraphExec_t gexec[4] = {nullptr, nullptr, nullptr, nullptr};
+  uint64_t graph_launches[4] = {0, 0, 0, 0};
+  int warm[4] = {0, 0, 0, 0};
+  const void* g_dstream[4] = {nullptr, nullptr, nullptr, nullptr};
+  uint64_t g_len[4] = {0, 0, 0, 0}, g_seed[4] = {0, 0, 0, 0};
+  // data-parallel gradient exchange: one event per bucket of the gradient
+  // arena, recorded in the last micro-batch's backward as the bucket's
+  // gradients become final (gpt_train_step_accumulate)
+  bool bucket_record = false;
+  std::vector<cudaEvent_t> bucket_ev;
   int* step_dev = nullptr;     // per-step scalars read by replayed graphs
   float* hyper_dev = nullptr;  // {lr, 1 - b1^t, 1 - b2^t}
   bool dev_keys = false;  // dropout keys from the device step index (a graph being captured)
@@ -551,6 +560,40 @@ DropKey dkey(gpt_model* m, int layer, int site) {
 
 template <typename T> T* at(uint8_t* base, size_t elems) { return reinterpret_cast<T*>(base) + elems; }
 
+// Bucket i of the data-parallel gradient exchange is final: record its event
+// on the model's stream (an external event node when a graph is captured).
+void record_bucket(gpt_model* m, int i) {
+  if (!m->bucket_record || i >= (int)m->bucket_ev.size()) return;
+  if (m->capturing) cudaEventRecordWithFlags(m->bucket_ev[i], m->ctx.stream, cudaEventRecordExternal);
+  else cudaEventRecord(m->bucket_ev[i], m->ctx.stream);
+}
+
+struct GradRange {
+  int64_t off, count;
+  int bucket;
+};
+// The gradient arena as ranges in the order the backward finalises them:
+// bucket i < L holds layer L-1-i (its four matrices, contiguous in the decayed
+// part of the arena, and its vectors, contiguous in the rest); bucket L the
+// token and position embeddings, the final norm and an untied head.
+std::vector<GradRange> grad_ranges(const gpt_model& m) {
+  std::vector<GradRange> t;  // every tensor with its bucket, then merged runs
+  for (auto& x : m.tensors) {
+    int bucket = m.L;
+    if (x.name.compare(0, 2, "h.") == 0) bucket = m.L - 1 - atoi(x.name.c_str() + 2);
+    t.push_back({x.off, ((x.alloc_rows * x.cols + 63) / 64) * 64, bucket});
+  }
+  std::sort(t.begin(), t.end(), [](const GradRange& a, const GradRange& b) {
+    return a.bucket != b.bucket ? a.bucket < b.bucket : a.off < b.off;
+  });
+  std::vector<GradRange> r;
+  for (auto& x : t) {
+    if (!r.empty() && r.back().bucket == x.bucket && r.back().off + r.back().count == x.off) r.back().count += x.count;
+    else r.push_back(x);
+  }
+  return r;
+}
+
 template <typename T>
 gpt_status forward_t(gpt_model* m, bool fuse_ce_grad, float* loss_acc, float loss_scale, int accumulate) {
   Ctx& c = m->ctx;
@@ -861,6 +904,7 @@ gpt_status backward_t(gpt_model* m) {
     norm_bwd<T>(c, nb);
     if (last && !frozen)
       add_bias_grads_from_norm(m, nb.part, y.ln1_w, y.ln1_b, l > 0 ? m->layers[l - 1].pr_b : -1);
+    if (last) record_bucket(m, L - 1 - l);  // layer l's gradients are final
   }
   if (frozen) {  // no embedding gradients; the adapters' from the merged blocks
     if (last) lora_grads(c, m->lora.lb, m->g);
@@ -874,6 +918,7 @@ gpt_status backward_t(gpt_model* m) {
     embed_sort(c, m->idx, M, m->stok, m->spos, m->nuniq);
   }
   embed_bwd(c, m->dres, stok, spos, M, m->T, m->B, d, dkey(m, L, 0), m->G(m->wte), m->G(m->wpe), m->seg);
+  if (last) record_bucket(m, L);  // the embeddings, the final norm (and an untied head)
   return check_cuda(m, "backward");
 }
 
@@ -1162,6 +1207,7 @@ void gpt_destroy(gpt_model* m) {
   if (!m) return;
   for (auto& e : m->gexec)
     if (e) cudaGraphExecDestroy(e);
+  for (auto e : m->bucket_ev) cudaEventDestroy(e);
   if (m->gen_exec) cudaGraphExecDestroy(m->gen_exec);
   if (m->cap_stream) cudaStreamDestroy(m->cap_stream);
   delete m->timing;
@@ -1222,11 +1268,12 @@ gpt_status gpt_clip_adamw_step(gpt_model* m, float lr, int32_t step, float* h_gr
   return s;
 }
 
-// The kernels of one optimiser step (grad_accum micro-batches, clip + AdamW).
+// The kernels of one optimiser step (grad_accum micro-batches, clip + AdamW;
+// without the optimiser for the data-parallel accumulate step, kind 2).
 // dev_params: the step index, lr and bias corrections are read from device
 // memory (the form captured into a graph and replayed every step).
-static gpt_status train_body(gpt_model* m, const void* d_stream, uint64_t len, uint64_t seed, float lr, int32_t step,
-                             bool dev_params) {
+static gpt_status train_body(gpt_model* m, int kind, const void* d_stream, uint64_t len, uint64_t seed, float lr,
+                             int32_t step, bool dev_params) {
   Ctx& c = m->ctx;
   const size_t Mz = (size_t)m->M;
   for (int mu = 0; mu < m->ga; mu++) {
@@ -1255,6 +1302,7 @@ static gpt_status train_body(gpt_model* m, const void* d_stream, uint64_t len, u
   m->tgt = m->tgt0;
   if (s != GPT_OK) return s;
   m->have_forward = false;
+  if (kind >= 2) return GPT_OK;  // the caller exchanges the gradients, then runs clip + AdamW
   return adamw_step(m, lr, step, dev_params);
 }
 
@@ -1272,7 +1320,9 @@ static bool capture_step(gpt_model* m, int kind, const void* d_stream, uint64_t 
   cudaGraph_t g = nullptr;
   bool ok = cudaStreamBeginCapture(m->cap_stream, cudaStreamCaptureModeThreadLocal) == cudaSuccess;
   m->dev_keys = true;  // dropout keys follow the step index the replay writes
-  gpt_status s = ok ? train_body(m, d_stream, len, seed, lr, step, true) : GPT_ERR_CUDA;
+  m->capturing = true;
+  gpt_status s = ok ? train_body(m, kind, d_stream, len, seed, lr, step, true) : GPT_ERR_CUDA;
+  m->capturing = false;
   m->dev_keys = false;
   if (ok) ok = cudaStreamEndCapture(m->cap_stream, &g) == cudaSuccess && s == GPT_OK;
   m->ctx.stream = user;
@@ -1287,32 +1337,31 @@ static bool capture_step(gpt_model* m, int kind, const void* d_stream, uint64_t 
   return ok;
 }
 
-static gpt_status train_common(gpt_model* m, const void* d_stream, uint64_t len, uint64_t seed, const int32_t* h_idx,
-                               const int32_t* h_tgt, float lr, int32_t step, float* h_loss, float* h_norm) {
+static gpt_status train_common(gpt_model* m, int kind, const void* d_stream, uint64_t len, uint64_t seed, float lr,
+                               int32_t step, float* h_loss, float* h_norm) {
   if (step < 1) return fail(m, GPT_ERR_INVALID_ARG, "step must be >= 1");
   Ctx& c = m->ctx;
+  m->bucket_record = kind >= 2;
   // Replay a captured graph of the whole step: everything that changes from
   // step to step (the step index, the learning rate, the bias corrections and
   // through the step index the dropout keys) is read from device memory.  Not
   // with per-kernel timing.  The first call of each kind runs eagerly, the
   // second captures, later calls only replay.
-  const int kind = d_stream ? 0 : 1;
   bool replay = m->graphs_on && !c.timing;
-  if (replay && kind == 0 && m->gexec[0] && (m->g_dstream != d_stream || m->g_len != len || m->g_seed != seed)) {
-    cudaGraphExecDestroy(m->gexec[0]);
-    m->gexec[0] = nullptr;
-    m->warm[0] = 0;
+  if (replay && (kind == 0 || kind == 2) && m->gexec[kind] &&
+      (m->g_dstream[kind] != d_stream || m->g_len[kind] != len || m->g_seed[kind] != seed)) {
+    cudaGraphExecDestroy(m->gexec[kind]);
+    m->gexec[kind] = nullptr;
+    m->warm[kind] = 0;
   }
   if (replay && !m->gexec[kind]) {
     if (m->warm[kind] < 1) {
       m->warm[kind]++;
       replay = false;
     } else if (capture_step(m, kind, d_stream, len, seed, lr, step)) {
-      if (kind == 0) {
-        m->g_dstream = d_stream;
-        m->g_len = len;
-        m->g_seed = seed;
-      }
+      m->g_dstream[kind] = d_stream;
+      m->g_len[kind] = len;
+      m->g_seed[kind] = seed;
     } else {
       // reported, not hidden: the step did not run; the next call tries the
       // capture again, and gpt_set_graphs(m, 0) runs every step eagerly
@@ -1330,8 +1379,9 @@ static gpt_status train_common(gpt_model* m, const void* d_stream, uint64_t len,
     c.launches += m->graph_launches[kind];
     m->have_forward = false;
   } else {
-    s = train_body(m, d_stream, len, seed, lr, step, false);
+    s = train_body(m, kind, d_stream, len, seed, lr, step, false);
   }
+  m->bucket_record = false;
   if (s != GPT_OK) return s;
   if (h_loss || h_norm) {
     float sc[4];
@@ -1346,7 +1396,83 @@ gpt_status gpt_train_step(gpt_model* m, const void* d_stream, uint64_t stream_le
                           int32_t step, float* h_loss, float* h_grad_norm) {
   if (!m || !d_stream) return fail(m, GPT_ERR_INVALID_ARG, "train_step: null argument");
   if (stream_len <= (uint64_t)m->T) return fail(m, GPT_ERR_INVALID_ARG, "stream shorter than block_size + 1");
-  return train_common(m, d_stream, stream_len, data_seed, nullptr, nullptr, lr, step, h_loss, h_grad_norm);
+  return train_common(m, 0, d_stream, stream_len, data_seed, lr, step, h_loss, h_grad_norm);
+}
+
+static gpt_status make_bucket_events(gpt_model* m) {
+  if (!m->bucket_ev.empty()) return GPT_OK;
+  for (int i = 0; i < m->L + 1; i++) {
+    cudaEvent_t e;
+    if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess)
+      return check_cuda(m, "train_step_accumulate: event creation");
+    m->bucket_ev.push_back(e);
+  }
+  return GPT_OK;
+}
+
+gpt_status gpt_train_step_accumulate(gpt_model* m, const void* d_stream, uint64_t stream_len, uint64_t data_seed,
+                                     int32_t step, float* h_loss) {
+  if (!m || !d_stream) return fail(m, GPT_ERR_INVALID_ARG, "train_step_accumulate: null argument");
+  if (stream_len <= (uint64_t)m->T) return fail(m, GPT_ERR_INVALID_ARG, "stream shorter than block_size + 1");
+  if (m->lora.on) return fail(m, GPT_ERR_UNSUPPORTED, "train_step_accumulate: not with adapters attached");
+  gpt_status s = make_bucket_events(m);
+  if (s != GPT_OK) return s;
+  return train_common(m, 2, d_stream, stream_len, data_seed, 0.f, step, h_loss, nullptr);
+}
+
+gpt_status gpt_train_step_host_accumulate(gpt_model* m, const int32_t* h_idx, const int32_t* h_tgt, int32_t step,
+                                          float* h_loss) {
+  if (!m || !h_idx || !h_tgt) return fail(m, GPT_ERR_INVALID_ARG, "train_step_host_accumulate: null argument");
+  if (m->lora.on) return fail(m, GPT_ERR_UNSUPPORTED, "train_step_host_accumulate: not with adapters attached");
+  gpt_status s = make_bucket_events(m);
+  if (s != GPT_OK) return s;
+  size_t bytes = (size_t)m->ga * m->M * 4;
+  cudaMemcpyAsync(m->stage_idx, h_idx, bytes, cudaMemcpyHostToDevice, m->ctx.stream);
+  cudaMemcpyAsync(m->stage_tgt, h_tgt, bytes, cudaMemcpyHostToDevice, m->ctx.stream);
+  return train_common(m, 3, nullptr, 0, 0, 0.f, step, h_loss, nullptr);
+}
+
+gpt_status gpt_stream_wait_bucket(gpt_model* m, int32_t bucket, void* cuda_stream) {
+  if (!m) return GPT_ERR_INVALID_ARG;
+  if (bucket < 0 || bucket >= (int)m->bucket_ev.size())
+    return fail(m, GPT_ERR_INVALID_ARG, "stream_wait_bucket: no such bucket (run gpt_train_step_accumulate first)");
+  if (cudaStreamWaitEvent((cudaStream_t)cuda_stream, m->bucket_ev[bucket], 0) != cudaSuccess)
+    return check_cuda(m, "stream_wait_bucket");
+  return GPT_OK;
+}
+
+gpt_status gpt_step_loss(gpt_model* m, float* h_loss) {
+  if (!m || !h_loss) return GPT_ERR_INVALID_ARG;
+  float sc[4];
+  gpt_status s = sync_and_flags(m, "step_loss", sc);
+  *h_loss = sc[1];
+  return s;
+}
+
+gpt_status gpt_grad_arena(gpt_model* m, float** d_grad, int64_t* n_floats) {
+  if (!m || !d_grad || !n_floats) return GPT_ERR_INVALID_ARG;
+  *d_grad = m->g;
+  *n_floats = m->n_total;
+  return GPT_OK;
+}
+
+gpt_status gpt_grad_buckets(const gpt_config* cfg, int32_t cap, int64_t* h_offset, int64_t* h_count,
+                            int32_t* h_bucket, int32_t* n_ranges) {
+  if (!n_ranges) return GPT_ERR_INVALID_ARG;
+  gpt_status s = validate(cfg, nullptr);
+  if (s != GPT_OK) return s;
+  gpt_model m;
+  derive(m, cfg);
+  const std::vector<GradRange> r = grad_ranges(m);
+  *n_ranges = (int32_t)r.size();
+  if (cap < (int32_t)r.size()) return h_offset ? GPT_ERR_INVALID_ARG : GPT_OK;
+  if (!h_offset || !h_count || !h_bucket) return GPT_ERR_INVALID_ARG;
+  for (size_t i = 0; i < r.size(); i++) {
+    h_offset[i] = r[i].off;
+    h_count[i] = r[i].count;
+    h_bucket[i] = r[i].bucket;
+  }
+  return GPT_OK;
 }
 
 gpt_status gpt_train_step_host(gpt_model* m, const int32_t* h_idx, const int32_t* h_tgt, float lr, int32_t step,
@@ -1355,7 +1481,7 @@ gpt_status gpt_train_step_host(gpt_model* m, const int32_t* h_idx, const int32_t
   size_t bytes = (size_t)m->ga * m->M * 4;
   cudaMemcpyAsync(m->stage_idx, h_idx, bytes, cudaMemcpyHostToDevice, m->ctx.stream);
   cudaMemcpyAsync(m->stage_tgt, h_tgt, bytes, cudaMemcpyHostToDevice, m->ctx.stream);
-  return train_common(m, nullptr, 0, 0, h_idx, h_tgt, lr, step, h_loss, h_grad_norm);
+  return train_common(m, 1, nullptr, 0, 0, lr, step, h_loss, h_grad_norm);
 }
 
 // The kernels and copies of one gpt_generate call (prefill, draws, decoding
@@ -1707,7 +1833,7 @@ static int lora_blocks(int L, int targets) { return L * __builtin_popcount((unsi
 static size_t lora_bytes(long n) { return 4 * (((size_t)n * 4 + 255) / 256 * 256) + 1024; }
 
 static void drop_train_graphs(gpt_model* m) {
-  for (int k = 0; k < 2; k++) {
+  for (int k = 0; k < 4; k++) {
     if (m->gexec[k]) cudaGraphExecDestroy(m->gexec[k]);
     m->gexec[k] = nullptr;
     m->warm[k] = 0;

@@ -219,6 +219,45 @@ gpt_status gpt_train_step_host(gpt_model* m, const int32_t* h_idx, const int32_t
  * on, and gpt_set_graphs(m, 0) runs every step eagerly). */
 gpt_status gpt_set_graphs(gpt_model* m, int32_t on);
 
+/* ---------------------------------------------------------------- data-parallel training
+ * The nanoGPT README's multi-GPU training ("复现 GPT-2": torchrun over 8 GPUs
+ * with DDP) averages the gradients of the replicas before the optimiser
+ * step.  The library runs the step in two calls around that exchange; the
+ * exchange itself is NCCL's all-reduce, issued by the caller (the Python
+ * layer, gpt_decoder_lm_b200/ddp.py) on a second stream so that it overlaps
+ * the rest of the backward:
+ *   gpt_train_step_accumulate   gather + grad_accum forward/backward passes,
+ *                               no optimiser; records one event per bucket of
+ *                               the gradient arena as the last micro-batch's
+ *                               backward makes the bucket final
+ *   gpt_stream_wait_bucket      makes a stream wait for a bucket's event
+ *   (caller)                    all-reduce (mean) of the bucket's ranges
+ *   gpt_clip_adamw_step         clip + AdamW on the averaged gradients
+ * gpt_grad_buckets gives the plan: the arena as ranges (element offset,
+ * count) with their bucket, buckets in the order the backward finalises
+ * them (bucket i < n_layer: layer n_layer-1-i; bucket n_layer: embeddings,
+ * final norm, an untied head).  Pure host; with cap < the number of ranges
+ * (or null arrays) only *n_ranges is written. */
+gpt_status gpt_grad_buckets(const gpt_config* cfg, int32_t cap, int64_t* h_offset, int64_t* h_count,
+                            int32_t* h_bucket, int32_t* n_ranges);
+/* Mean loss of the last training step (gpt_train_step*, including the
+ * accumulate forms).  Synchronising. */
+gpt_status gpt_step_loss(gpt_model* m, float* h_loss);
+/* Device address and length (floats) of the fp32 gradient arena. */
+gpt_status gpt_grad_arena(gpt_model* m, float** d_grad, int64_t* n_floats);
+/* The step of gpt_train_step without clip + AdamW; gradients are left in
+ * the arena (added to what it holds).  Replayed as its own CUDA graph with
+ * graphs on.  h_loss (nullable) as gpt_train_step.  GPT_ERR_UNSUPPORTED with
+ * LoRA adapters attached. */
+gpt_status gpt_train_step_accumulate(gpt_model* m, const void* d_stream, uint64_t stream_len, uint64_t data_seed,
+                                     int32_t step, float* h_loss);
+/* The same with the micro-batches from host memory (as gpt_train_step_host). */
+gpt_status gpt_train_step_host_accumulate(gpt_model* m, const int32_t* h_idx, const int32_t* h_tgt, int32_t step,
+                                          float* h_loss);
+/* cudaStreamWaitEvent(cuda_stream, event of `bucket`) for the last
+ * gpt_train_step_accumulate / gpt_train_step_host_accumulate. */
+gpt_status gpt_stream_wait_bucket(gpt_model* m, int32_t bucket, void* cuda_stream);
+
 /* The batch gather of gpt_train_step on its own: writes int32
  * [batch_size, block_size] ids and targets to d_idx / d_tgt. */
 gpt_status gpt_gather_batch(gpt_model* m, const void* d_stream, uint64_t stream_len, uint64_t data_seed,
