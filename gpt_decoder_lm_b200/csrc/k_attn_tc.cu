@@ -598,6 +598,9 @@ __device__ __forceinline__ uint32_t pack2v(uint64_t v) {
 }
 
 constexpr int BWD_STAGES = 3;  // Q/dO (or K/V) tiles in flight
+// one probability pair in every BWD_POLY_EVERY is computed on the FMA pipe
+// (exp2_poly2) instead of the SFU
+constexpr int BWD_POLY_EVERY = 2;
 
 // ============================================================================
 // backward, dK and dV: one CTA per (128-key block, b, h), walking 64-query
@@ -766,7 +769,23 @@ __global__ void __launch_bounds__(320, 2) k_attn_bwd_kv8(const __grid_constant__
                                            f2mul(f2(l4.x, l4.y), nlog2e)));
           const float2 y23 = f2split(f2fma(f2(__uint_as_float(sv[e + 2]), __uint_as_float(sv[e + 3])), sl2x2,
                                            f2mul(f2(l4.z, l4.w), nlog2e)));
-          float p4[4] = {ex2(y01.x), ex2(y01.y), ex2(y23.x), ex2(y23.y)};
+          float p4[4];
+          if (((e >> 1) % BWD_POLY_EVERY) == BWD_POLY_EVERY - 1) {
+            const float2 q01 = f2split(exp2_poly2(f2(y01.x, y01.y)));
+            p4[0] = q01.x;
+            p4[1] = q01.y;
+          } else {
+            p4[0] = ex2(y01.x);
+            p4[1] = ex2(y01.y);
+          }
+          if ((((e >> 1) + 1) % BWD_POLY_EVERY) == BWD_POLY_EVERY - 1) {
+            const float2 q23 = f2split(exp2_poly2(f2(y23.x, y23.y)));
+            p4[2] = q23.x;
+            p4[3] = q23.y;
+          } else {
+            p4[2] = ex2(y23.x);
+            p4[3] = ex2(y23.y);
+          }
 #pragma unroll
           for (int u = 0; u < 4; u++) {
             if (masked && c0 + e + u < lim) p4[u] = 0.f;
@@ -1004,9 +1023,19 @@ __global__ void __launch_bounds__(320, 2) k_attn_bwd_q8(const __grid_constant__ 
         tmem_ld_wait();
 #pragma unroll
         for (int e = 0; e < 16; e += 2) {
-          const float2 y = f2split(f2fma(f2(__uint_as_float(sv[e]), __uint_as_float(sv[e + 1])), sl2x2, nlse2));
-          pk[sub][e] = (masked && c0 + e > lim) ? 0.f : ex2(y.x);
-          pk[sub][e + 1] = (masked && c0 + e + 1 > lim) ? 0.f : ex2(y.y);
+          const uint64_t y2 = f2fma(f2(__uint_as_float(sv[e]), __uint_as_float(sv[e + 1])), sl2x2, nlse2);
+          float e0, e1;
+          if (((e >> 1) % BWD_POLY_EVERY) == BWD_POLY_EVERY - 1) {
+            const float2 q = f2split(exp2_poly2(y2));
+            e0 = q.x;
+            e1 = q.y;
+          } else {
+            const float2 y = f2split(y2);
+            e0 = ex2(y.x);
+            e1 = ex2(y.y);
+          }
+          pk[sub][e] = (masked && c0 + e > lim) ? 0.f : e0;
+          pk[sub][e + 1] = (masked && c0 + e + 1 > lim) ? 0.f : e1;
         }
       }
       tc_fence_before();

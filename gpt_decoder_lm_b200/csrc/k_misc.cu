@@ -137,37 +137,37 @@ template <> __device__ __forceinline__ void store4<bf16>(bf16* p, float4 v) {
   *reinterpret_cast<uint2*>(p) = u;
 }
 
+// One warp per row at a time, rows strided over a single resident wave of
+// warps; the next row's loads are issued before the current row's
+// reductions, so every warp keeps a row of loads in flight while it computes.
 template <typename T, int VPL>
-__global__ void k_norm_fwd(const float* __restrict__ x, const float* __restrict__ w, const float* __restrict__ b,
-                           T* __restrict__ y, float* __restrict__ mean_out, float* __restrict__ rstd_out, long rows,
-                           int d, int rms, float eps) {
+__global__ void __launch_bounds__(256) k_norm_fwd(const float* __restrict__ x, const float* __restrict__ w,
+                                                  const float* __restrict__ b, T* __restrict__ y,
+                                                  float* __restrict__ mean_out, float* __restrict__ rstd_out,
+                                                  long rows, int d, int rms, float eps) {
   pdl_trigger();
-  // two rows per warp, both loaded up front: the whole launch is resident in
-  // one wave and every warp has 2 x d x 4 bytes in flight
-  const long row0 = ((long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5)) * 2;
   const int lane = threadIdx.x & 31;
-  if (row0 >= rows) return;
+  const long nwarps = (long)gridDim.x * (blockDim.x >> 5);
+  long row = (long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int d4 = d >> 2;
-  float4 v[2][VPL];
-#pragma unroll
-  for (int u = 0; u < 2; u++) {
-    const float4* xr = reinterpret_cast<const float4*>(x + (row0 + u) * d);
-    const bool live = row0 + u < rows;
+  float4 cur[VPL], nxt[VPL];
+  auto load = [&](long r, float4 (&v)[VPL]) {
+    const float4* xr = reinterpret_cast<const float4*>(x + r * d);
 #pragma unroll
     for (int k = 0; k < VPL; k++) {
-      int c = lane + 32 * k;
-      v[u][k] = (live && c < d4) ? xr[c] : make_float4(0.f, 0.f, 0.f, 0.f);
+      const int c = lane + 32 * k;
+      v[k] = (r < rows && c < d4) ? xr[c] : make_float4(0.f, 0.f, 0.f, 0.f);
     }
-  }
-#pragma unroll
-  for (int u = 0; u < 2; u++) {
-    const long row = row0 + u;
-    if (row >= rows) break;
+  };
+  if (row >= rows) return;
+  load(row, cur);
+  for (; row < rows; row += nwarps) {
+    load(row + nwarps, nxt);  // in flight while this row is reduced and written
     float s = 0.f;
 #pragma unroll
     for (int k = 0; k < VPL; k++)
-      s += rms ? (v[u][k].x * v[u][k].x + v[u][k].y * v[u][k].y + v[u][k].z * v[u][k].z + v[u][k].w * v[u][k].w)
-               : (v[u][k].x + v[u][k].y + v[u][k].z + v[u][k].w);
+      s += rms ? (cur[k].x * cur[k].x + cur[k].y * cur[k].y + cur[k].z * cur[k].z + cur[k].w * cur[k].w)
+               : (cur[k].x + cur[k].y + cur[k].z + cur[k].w);
     s = warp_sum(s);
     float mean = 0.f, rstd;
     if (rms) {
@@ -177,9 +177,8 @@ __global__ void k_norm_fwd(const float* __restrict__ x, const float* __restrict_
       float q = 0.f;
 #pragma unroll
       for (int k = 0; k < VPL; k++) {
-        int c = lane + 32 * k;
-        if (c < d4) {
-          float a = v[u][k].x - mean, bb = v[u][k].y - mean, cc = v[u][k].z - mean, dd = v[u][k].w - mean;
+        if (lane + 32 * k < d4) {
+          const float a = cur[k].x - mean, bb = cur[k].y - mean, cc = cur[k].z - mean, dd = cur[k].w - mean;
           q += a * a + bb * bb + cc * cc + dd * dd;
         }
       }
@@ -189,16 +188,16 @@ __global__ void k_norm_fwd(const float* __restrict__ x, const float* __restrict_
     T* yr = y + row * d;
 #pragma unroll
     for (int k = 0; k < VPL; k++) {
-      int c = lane + 32 * k;
+      const int c = lane + 32 * k;
       if (c < d4) {
         float4 o;
-        o.x = (v[u][k].x - mean) * rstd;
-        o.y = (v[u][k].y - mean) * rstd;
-        o.z = (v[u][k].z - mean) * rstd;
-        o.w = (v[u][k].w - mean) * rstd;
+        o.x = (cur[k].x - mean) * rstd;
+        o.y = (cur[k].y - mean) * rstd;
+        o.z = (cur[k].z - mean) * rstd;
+        o.w = (cur[k].w - mean) * rstd;
         if (!rms) {
-          float4 ww = reinterpret_cast<const float4*>(w)[c];
-          float4 bb = reinterpret_cast<const float4*>(b)[c];
+          const float4 ww = reinterpret_cast<const float4*>(w)[c];
+          const float4 bb = reinterpret_cast<const float4*>(b)[c];
           o.x = o.x * ww.x + bb.x;
           o.y = o.y * ww.y + bb.y;
           o.z = o.z * ww.z + bb.z;
@@ -211,7 +210,25 @@ __global__ void k_norm_fwd(const float* __restrict__ x, const float* __restrict_
       mean_out[row] = mean;
       rstd_out[row] = rstd;
     }
+#pragma unroll
+    for (int k = 0; k < VPL; k++) cur[k] = nxt[k];
   }
+}
+
+// a single resident wave: the SM count times the blocks of this instantiation
+// that fit on an SM, at most one warp per row
+template <typename T, int VPL>
+void launch_norm_fwd(Ctx& c, const float* x, const float* w, const float* b, T* y, float* mean, float* rstd,
+                     long rows, int d, bool rms, float eps) {
+  int occ = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k_norm_fwd<T, VPL>, 256, 0) != cudaSuccess || occ < 1) {
+    cudaGetLastError();
+    occ = 1;
+  }
+  long grid = (long)c.num_sms * occ;
+  const long need = (rows + 7) / 8;
+  if (grid > need) grid = need;
+  k_norm_fwd<T, VPL><<<(unsigned)grid, 256, 0, c.stream>>>(x, w, b, y, mean, rstd, rows, d, rms, eps);
 }
 
 template <typename T>
@@ -219,9 +236,8 @@ void norm_fwd(Ctx& c, const float* x, const float* w, const float* b, T* y, floa
               int d, bool rms, float eps) {
   int d4 = d / 4;
   int vpl = (d4 + 31) / 32;
-  unsigned grid = (unsigned)((rows + 15) / 16);  // 8 warps x 2 rows per block
   LaunchScope s(c, "norm_fwd");
-#define NF(V) k_norm_fwd<T, V><<<grid, 256, 0, c.stream>>>(x, w, b, y, mean, rstd, rows, d, rms, eps)
+#define NF(V) launch_norm_fwd<T, V>(c, x, w, b, y, mean, rstd, rows, d, rms, eps)
   if (vpl <= 1) NF(1);
   else if (vpl <= 2) NF(2);
   else if (vpl <= 4) NF(4);
