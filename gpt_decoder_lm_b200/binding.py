@@ -102,7 +102,7 @@ _PROTOS = {
     "gpt_last_error": (C.c_char_p, [P]),
     "gpt_status_string": (C.c_char_p, [I32]),
     "gpt_test_gemm": (I32, [I32, I32, I32, I32, P, I64, I32, P, I64, I32, I32, I32, P, P, I32, P, P, P, P, I32, P,
-                            P, P]),
+                            P, P, P]),
     "gpt_test_attention": (I32, [I32, I32, I32, I32, I32, I32, I32, P, P, P, P, P, P, F32, U64, U64, I32, P, P]),
     "gpt_test_wait_timeout": (I32, [U64, P, P, P]),
     "gpt_test_exp2": (I32, [P, P, P, I64, P]),
@@ -449,10 +449,11 @@ def sample(logits, temperature: float, top_k: int, top_p: float, uniform, out, V
 
 
 def test_gemm(backend, M, N, K, A, lda, a_kmajor, B, ldb, b_kmajor, epi_kind, act=0, out=None, out2=None, ldo=0,
-              aux=None, bias=None, res_in=None, res_out=None, split_k=1, partial=None, stream=None, flags=None):
+              aux=None, bias=None, res_in=None, res_out=None, split_k=1, partial=None, stream=None, flags=None,
+              colsum=None):
     return int(lib().gpt_test_gemm(backend, M, N, K, _ptr(A), lda, a_kmajor, _ptr(B), ldb, b_kmajor, epi_kind, act,
                                    _ptr(out), _ptr(out2), ldo, _ptr(aux), _ptr(bias), _ptr(res_in), _ptr(res_out),
-                                   split_k, _ptr(partial), stream, _ptr(flags)))
+                                   split_k, _ptr(partial), _ptr(colsum), stream, _ptr(flags)))
 
 
 def test_attention(backend, backward, dtype, B, T, H, hd, qkv, o, lse, dout=None, dqkv=None, dsum=None, p=0.0,

@@ -150,7 +150,8 @@ struct gpt_model {
   uint64_t gen_key[8] = {0, 0, 0, 0, 0, 0, 0, 0};
   int part_cap = 0;                 // partial rows per norm instance
   float* norm_parts = nullptr;      // [2L+1][part_cap][3][d]
-  float* colsum_parts = nullptr;    // [L][2][colsum chunks][4d]
+  float* colsum_parts = nullptr;    // [L][2][colsum_rows][4d]
+  long colsum_rows = 0;             // partial rows per instance: row chunks, or 32-row groups
   float* split_parts = nullptr;     // per (layer, dW kind): [splits, Mo, No]
   std::vector<size_t> split_off;    // offset of each (layer, kind) instance; kind: 0 mlp proj, 1 fc, 2 attn proj, 3 qkv
   std::vector<int> split_n;         // its split count (1: no split buffer)
@@ -398,7 +399,8 @@ size_t carve(gpt_model& m, uint8_t* base) {
   m.part_blocks = (int)std::min<long>(M, 148 * 8);  // capacity; the launch count is set at create
   m.part_cap = m.part_blocks;
   m.norm_parts = F((size_t)(2 * L + 1) * m.part_cap * 3 * d);
-  m.colsum_parts = F((size_t)L * 2 * colsum_chunks(M) * 4 * d);
+  m.colsum_rows = std::max<long>(colsum_chunks(M), (M + 31) / 32);
+  m.colsum_parts = F((size_t)L * 2 * m.colsum_rows * 4 * d);
   {
     // weight-gradient shapes [Mo, No] of the four per-layer GEMMs
     const long dw[4][2] = {{d, 4L * d}, {4L * d, d}, {d, d}, {3L * d, d}};
@@ -774,7 +776,7 @@ gpt_status backward_t(gpt_model* m) {
   };
   auto norm_part = [&](int k) { return m->norm_parts + (size_t)k * m->part_cap * 3 * d; };
   auto colsum_part = [&](int l, int which) {
-    return m->colsum_parts + ((size_t)l * 2 + which) * colsum_chunks(M) * 4 * d;
+    return m->colsum_parts + ((size_t)l * 2 + which) * m->colsum_rows * 4 * d;
   };
   // bias gradient = column sums of the operand-typed gradient x [M, N]
   auto bias_grad = [&](const T* x, int N, int l, int which, float* grad) {
@@ -835,8 +837,19 @@ gpt_status backward_t(gpt_model* m) {
     g.epi.aux = h;
     g.epi.out = dh;
     g.epi.ldo = 4 * d;
+    // bf16: the fc bias gradient's column sums of dh come from this GEMM's
+    // epilogue (one partial row per 32-row group), not from a second pass
+    const bool fused_colsum = m->bf16m && y.fc_b >= 0 && !frozen;
+    if (fused_colsum) {
+      g.epi.colsum = colsum_part(l, 0);
+      g.epi.colsum_acc = !first;
+    }
     if (!gemm(m, g)) return fail(m, GPT_ERR_CUDA, "proj dX failed");
-    if (y.fc_b >= 0) bias_grad(dh, 4 * d, l, 0, m->G(y.fc_b));
+    if (fused_colsum) {
+      if (last) colsum_reduce(c, colsum_part(l, 0), (int)((M + 31) / 32), 4 * d, m->G(y.fc_b));
+    } else if (y.fc_b >= 0) {
+      bias_grad(dh, 4 * d, l, 0, m->G(y.fc_b));
+    }
     if (!dW(4 * d, d, dh, a2, m->G(y.fc_w), "gemm_fc_dw", l * 4 + 1)) return fail(m, GPT_ERR_CUDA, "fc dW failed");
     g = gd((int)M, d, 4 * d, dh, 4 * d, true, m->Wop(y.fc_w), d, false);
     g.epi.kind = EPI_STORE_F32;

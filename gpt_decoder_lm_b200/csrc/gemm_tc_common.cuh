@@ -31,7 +31,29 @@ struct TcArgs {
   const float* bias;
   DropKey drop;
   uint32_t* flags;
+  float* colsum;    // EPI_ACT_BWD: column sums per 32-row group (null: none)
+  int colsum_acc;
 };
+
+// Column sums of a warp's staged 32 x 32 bf16 chunk (64-byte rows, 64-byte
+// swizzle: 16-byte chunk q of row r at q ^ ((r >> 1) & 3)): lane c adds
+// column c over the 32 rows in order and writes (or adds) the group's partial.
+__device__ __forceinline__ void chunk_colsum(const TcArgs& p, uint32_t buf, int lane, int row0, int col0) {
+  if (row0 >= p.M) return;
+  float s = 0.f;
+#pragma unroll 8
+  for (int r = 0; r < 32; r++) {
+    const uint32_t addr = buf + r * 64 + ((((lane >> 3) ^ ((r >> 1) & 3))) << 4) + (lane & 7) * 2;
+    unsigned short u;
+    asm volatile("ld.shared.u16 %0, [%1];" : "=h"(u) : "r"(addr));
+    s += __bfloat162float(__ushort_as_bfloat16(u));
+  }
+  const int col = col0 + lane;
+  if (col < p.N) {
+    float* dst = p.colsum + (size_t)(row0 >> 5) * p.N + col;
+    *dst = p.colsum_acc ? *dst + s : s;
+  }
+}
 
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
   __nv_bfloat162 v = __floats2bfloat162_rn(a, b);

@@ -300,6 +300,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         fence_proxy_async_smem();
         __syncwarp();
+        if (kind == EPI_ACT_BWD && p.colsum && p.splits == 1) chunk_colsum(p, bufA, lane, row0, col0);
         if (lane == 0) {
           if (p.splits > 1) {
             if (p.acc_partial) tma_reduce_add_3d(&tm_out, bufA, col0, row0, split);
@@ -385,6 +386,8 @@ bool launch(Ctx& c, const GemmDesc& g, int splits) {
   a.bias = e.bias;
   a.drop = e.drop;
   a.flags = c.flags;
+  a.colsum = (e.kind == EPI_ACT_BWD && splits == 1) ? e.colsum : nullptr;
+  a.colsum_acc = e.colsum_acc ? 1 : 0;
   int tiles = a.num_m * a.num_n * splits;
   int grid = tiles < c.num_sms ? tiles : c.num_sms;
   // per-device function attribute: set before every launch

@@ -56,6 +56,11 @@ struct GemmEpi {
   float* res_out = nullptr;
   int ld_res = 0;
   DropKey drop{};             // EPI_RESADD; element index = m * N + n
+  // EPI_ACT_BWD on the tensor cores: column sums of the stored (operand-typed)
+  // output, one fp32 row per 32-row group: colsum[m / 32][n] (= or += with
+  // colsum_acc).  Null: none.
+  float* colsum = nullptr;
+  bool colsum_acc = false;
 };
 
 struct GemmDesc {

@@ -9,7 +9,7 @@ extern "C" gpt_status gpt_test_gemm(int32_t backend, int32_t M, int32_t N, int32
                                     int32_t a_kmajor, const void* B, int64_t ldb, int32_t b_kmajor, int32_t epi_kind,
                                     int32_t act, void* out, void* out2, int32_t ldo, const void* aux,
                                     const float* bias, const float* res_in, float* res_out, int32_t split_k,
-                                    float* partial, void* stream, uint32_t* d_flags) {
+                                    float* partial, float* colsum, void* stream, uint32_t* d_flags) {
   if (M <= 0 || N <= 0 || K <= 0 || !A || !B || epi_kind < 0 || epi_kind > 6) return GPT_ERR_INVALID_ARG;
   Ctx c;
   c.stream = (cudaStream_t)stream;
@@ -39,6 +39,7 @@ extern "C" gpt_status gpt_test_gemm(int32_t backend, int32_t M, int32_t N, int32
   g.epi.ld_res = ldo;
   g.split_k = split_k;
   g.partial = partial;
+  g.epi.colsum = colsum;
   switch (backend) {
     case GPT_GEMM_SIMT_F32: gemm_simt_f32(c, g); break;
     case GPT_GEMM_SIMT_BF16: gemm_simt_bf16(c, g); break;

@@ -39,12 +39,14 @@ enum {
  * [split_k, M, N] fp32 scratch.  GPT_GEMM_SKINNY_BF16 (the decoding-step
  * GEMM) takes M <= 16, K a multiple of 32, both operands K-major, no split-K.
  * GPT_ERR_UNSUPPORTED when the tensor-core or skinny backend cannot take the
- * shape. */
+ * shape.  colsum (nullable; kind 4 on the tensor-core backends): fp32
+ * [ceil(M / 32), N] receives the column sums of the stored output over each
+ * 32-row group. */
 gpt_status gpt_test_gemm(int32_t backend, int32_t M, int32_t N, int32_t K, const void* A, int64_t lda,
                          int32_t a_kmajor, const void* B, int64_t ldb, int32_t b_kmajor, int32_t epi_kind,
                          int32_t act, void* out, void* out2, int32_t ldo, const void* aux, const float* bias,
-                         const float* res_in, float* res_out, int32_t split_k, float* partial, void* stream,
-                         uint32_t* d_flags);
+                         const float* res_in, float* res_out, int32_t split_k, float* partial, float* colsum,
+                         void* stream, uint32_t* d_flags);
 
 /* Causal attention of one layer.  qkv [B, T, 3, H, hd], o [B, T, H, hd],
  * lse fp32 [B, H, T]; backward also takes dout [B, T, H, hd] and writes

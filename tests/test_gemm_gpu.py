@@ -285,3 +285,26 @@ def test_tc_gemm_lm_head_sampled(layout):
     err = np.abs(got - ref).max() / np.abs(ref).max()
     assert err < (2e-6 if K <= 2048 else 1e-5), err
     assert not torch.isnan(out).any().item()
+
+
+@pytest.mark.parametrize("backend", [TC, TC2], ids=["tc", "tc2"])
+@pytest.mark.parametrize("M", [384, 200, 12288])
+def test_act_bwd_epilogue_column_sums(backend, M):
+    # the activation-backward GEMM (dh = (dy W) * act'(h)) also writes the
+    # column sums of the stored bf16 dh over each 32-row group (the fc bias
+    # gradient's partials): against the sums of the stored values
+    N, K = 3072, 768
+    rng = np.random.default_rng(13)
+    A, B, Ad, Bd, lda, ldb = operands(M, N, K, 1, 0, 17)
+    aux = dev_bf16(gelu_grad(rng.standard_normal((M, N))))
+    out = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    groups = (M + 31) // 32
+    cs = torch.full((groups, N), float("nan"), device="cuda")
+    run(backend, M, N, K, Ad, lda, 1, Bd, ldb, 0, 4, act=0, out=out, ldo=N, aux=aux, colsum=cs)
+    dh = out.double().cpu().numpy()
+    pad = np.zeros((groups * 32, N))
+    pad[:M] = dh
+    want = pad.reshape(groups, 32, N).sum(axis=1)
+    got = cs.double().cpu().numpy()
+    assert np.isfinite(got).all()
+    assert np.abs(got - want).max() <= 1e-5 * max(1.0, np.abs(want).max())
