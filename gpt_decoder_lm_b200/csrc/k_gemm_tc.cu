@@ -412,27 +412,36 @@ bool launch(Ctx& c, const GemmDesc& g, int splits) {
 
 }  // namespace
 
-// Tile width and split-K count from a simple cost model: MMA cycles per work
-// unit (k-blocks x cycles per k-block, 128-wide tiles paying for their lower
-// operand reuse), whole waves over the SMs, and the traffic of split-K
-// partials (written and read back once).
-TcPlan gemm_tc_plan(long M, long N, long K, bool split_ok, int num_sms) {
-  TcPlan best{256, 1};
+// Kernel, tile width and split-K count from a simple cost model: MMA cycles
+// per work unit (k-blocks x cycles per k-block; 128-wide tiles pay for their
+// lower operand reuse, pair tiles gain from each SM loading half of B), whole
+// waves over the SMs (pairs of SMs for the pair kernel), and the traffic of
+// split-K partials (written and read back once).
+constexpr double KB_CYCLES_256 = 512.0, KB_CYCLES_128 = 330.0, KB_CYCLES_PAIR = 530.0;
+TcPlan gemm_tc_plan(long M, long N, long K, bool split_ok, int num_sms, int mode) {
+  TcPlan best{256, 1, 0};
   double best_t = 1e30;
   long nkb = (K + BK - 1) / BK;
-  for (int bn : {256, 128}) {
-    if (bn == 256 && N <= 128) continue;
-    long tiles = ((M + BM - 1) / BM) * ((N + bn - 1) / bn);
-    for (int s = 1; s <= 16; s++) {
-      if (s > 1 && (!split_ok || s > nkb / 8)) break;
-      long units = tiles * s;
-      long waves = (units + num_sms - 1) / num_sms;
-      double per_unit = (double)((nkb + s - 1) / s) * (bn == 256 ? 512.0 : 330.0) + bn * 12.0;
-      double t = waves * per_unit;
-      if (s > 1) t += 2.0 * s * M * N * 4 / (num_sms * 48.0);
-      if (t < best_t * 0.98) {
-        best_t = t;
-        best = TcPlan{bn, s};
+  for (int pair = 0; pair < 2; pair++) {
+    if ((mode == TC_SINGLE && pair) || (mode == TC_PAIR && !pair)) continue;
+    if (mode == TC_ANY && pair && M < 256) continue;
+    const int slots = pair ? num_sms / 2 : num_sms;
+    for (int bn : {256, 128}) {
+      if (pair && bn != 256) continue;
+      if (!pair && bn == 256 && N <= 128) continue;
+      long tiles = ((M + (pair ? 2 * BM : BM) - 1) / (pair ? 2 * BM : BM)) * ((N + bn - 1) / bn);
+      for (int s = 1; s <= 16; s++) {
+        if (s > 1 && (!split_ok || s > nkb / 8)) break;
+        long units = tiles * s;
+        long waves = (units + slots - 1) / slots;
+        const double kbc = pair ? KB_CYCLES_PAIR : (bn == 256 ? KB_CYCLES_256 : KB_CYCLES_128);
+        double per_unit = (double)((nkb + s - 1) / s) * kbc + bn * 12.0;
+        double t = waves * per_unit;
+        if (s > 1) t += 2.0 * s * M * N * 4 / (num_sms * 48.0);
+        if (t < best_t * 0.98) {
+          best_t = t;
+          best = TcPlan{bn, s, pair};
+        }
       }
     }
   }
@@ -463,9 +472,9 @@ bool gemm_tc_supported(const GemmDesc& g) {
   return true;
 }
 
-int gemm_tc_splits(const GemmDesc& g, int num_sms) {
+int gemm_tc_splits(const GemmDesc& g, int num_sms, int mode) {
   bool split_ok = g.epi.kind == EPI_ACC_F32 && g.partial && g.split_k > 1;
-  TcPlan plan = gemm_tc_plan(g.M, g.N, g.K, split_ok, num_sms);
+  TcPlan plan = gemm_tc_plan(g.M, g.N, g.K, split_ok, num_sms, mode);
   int splits = plan.splits;
   if (splits > g.split_k) splits = g.split_k < 1 ? 1 : g.split_k;  // never beyond the caller's scratch
   if (splits > 1) {  // keep every split non-empty
@@ -476,13 +485,15 @@ int gemm_tc_splits(const GemmDesc& g, int num_sms) {
   return splits;
 }
 
-bool gemm_tc_bf16(Ctx& c, const GemmDesc& g) {
+bool gemm_tc_bf16(Ctx& c, const GemmDesc& g, int mode) {
   bool split_ok = g.epi.kind == EPI_ACC_F32 && g.partial && g.split_k > 1;
-  TcPlan plan = gemm_tc_plan(g.M, g.N, g.K, split_ok, c.num_sms);
-  const int splits = gemm_tc_splits(g, c.num_sms);
+  TcPlan plan = gemm_tc_plan(g.M, g.N, g.K, split_ok, c.num_sms, mode);
+  const int splits = gemm_tc_splits(g, c.num_sms, mode);
   bool amn = !g.a_kmajor, bmn = !g.b_kmajor;
   bool ok;
-  if (plan.bn == 256) {
+  if (plan.pair) {
+    ok = gemm_tc2_launch(c, g, splits);
+  } else if (plan.bn == 256) {
     if (!amn && !bmn) ok = launch<256, false, false>(c, g, splits);
     else if (!amn && bmn) ok = launch<256, false, true>(c, g, splits);
     else ok = launch<256, true, true>(c, g, splits);

@@ -464,17 +464,12 @@ bool launch2(Ctx& c, const GemmDesc& g, int splits) {
 
 }  // namespace
 
-bool gemm_tc2_bf16(Ctx& c, const GemmDesc& g) {
-  const int splits = gemm_tc_splits(g, c.num_sms);
+// launch only: the caller (gemm_tc_bf16) reduces split partials
+bool gemm_tc2_launch(Ctx& c, const GemmDesc& g, int splits) {
   const bool amn = !g.a_kmajor, bmn = !g.b_kmajor;
-  bool ok;
-  if (!amn && !bmn) ok = launch2<256, false, false>(c, g, splits);
-  else if (!amn && bmn) ok = launch2<256, false, true>(c, g, splits);
-  else ok = launch2<256, true, true>(c, g, splits);
-  if (!ok) return false;
-  if (splits > 1 && g.reduce_partials)
-    splitk_reduce(c, g.partial, splits, (long)g.M * g.N, reinterpret_cast<float*>(g.epi.out));
-  return true;
+  if (!amn && !bmn) return launch2<256, false, false>(c, g, splits);
+  if (!amn && bmn) return launch2<256, false, true>(c, g, splits);
+  return launch2<256, true, true>(c, g, splits);
 }
 
 }  // namespace gpt

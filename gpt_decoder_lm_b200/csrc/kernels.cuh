@@ -79,21 +79,27 @@ struct GemmDesc {
   const char* name = nullptr; // timing label
 };
 
-// Tile width (256 or 128 columns) and split-K count the tensor-core GEMM uses
-// for an M x N x K problem on `num_sms` SMs (split_ok: fp32-accumulating dW).
+// Kernel, tile width and split-K count the tensor-core GEMM uses for an
+// M x N x K problem on `num_sms` SMs (split_ok: fp32-accumulating dW): the
+// single-CTA kernel (128 x bn tiles, bn 256 or 128) or the pair-CTA kernel
+// (256 x 256 tiles over two SMs).  mode: TC_ANY (the cost model picks),
+// TC_SINGLE or TC_PAIR (forced; kernel tests).
+enum { TC_ANY = 0, TC_SINGLE = 1, TC_PAIR = 2 };
 struct TcPlan {
   int bn;
   int splits;
+  int pair;
 };
-TcPlan gemm_tc_plan(long M, long N, long K, bool split_ok, int num_sms);
+TcPlan gemm_tc_plan(long M, long N, long K, bool split_ok, int num_sms, int mode = TC_ANY);
 
 // fp32 operands on CUDA cores (fp32 mode); bf16 operands on CUDA cores
 // (reference path used by tests); bf16 operands on tcgen05 tensor cores.
 void gemm_simt_f32(Ctx& c, const GemmDesc& g);
 void gemm_simt_bf16(Ctx& c, const GemmDesc& g);
 bool gemm_tc_supported(const GemmDesc& g);
-// pair-CTA variant (256-row tiles over two SMs, cta_group::2); same support rules
-bool gemm_tc2_bf16(Ctx& c, const GemmDesc& g);
+// the pair-CTA kernel (256-row tiles over two SMs, cta_group::2) with a
+// given split count; gemm_tc_bf16 calls it when the plan says so
+bool gemm_tc2_launch(Ctx& c, const GemmDesc& g, int splits);
 // GEMMs of at most 16 rows (decoding): bf16, both operands K-major, no split-K.
 // With a SkinnyNorm, A is not read: the kernel computes it as the norm of the
 // fp32 rows x [M, ldx] over K columns (LayerNorm with w, b; RMSNorm without).
@@ -108,9 +114,9 @@ struct SkinnyNorm {
 bool gemm_skinny_supported(const GemmDesc& g);
 bool skinny_norm_supported(const GemmDesc& g, const SkinnyNorm& n);
 void gemm_skinny_bf16(Ctx& c, const GemmDesc& g, const SkinnyNorm* nrm = nullptr);
-bool gemm_tc_bf16(Ctx& c, const GemmDesc& g);  // false: tensor-map encode failed
+bool gemm_tc_bf16(Ctx& c, const GemmDesc& g, int mode = TC_ANY);  // false: tensor-map encode failed
 // the split-K count gemm_tc_bf16 uses for g (1: none)
-int gemm_tc_splits(const GemmDesc& g, int num_sms);
+int gemm_tc_splits(const GemmDesc& g, int num_sms, int mode = TC_ANY);
 // split-K reduction: out[m,n] += sum_s partial[s,m,n] (fixed order)
 void splitk_reduce(Ctx& c, const float* partial, int splits, long MN, float* out);
 

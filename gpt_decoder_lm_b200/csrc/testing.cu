@@ -11,6 +11,7 @@ extern "C" gpt_status gpt_test_gemm(int32_t backend, int32_t M, int32_t N, int32
                                     const float* bias, const float* res_in, float* res_out, int32_t split_k,
                                     float* partial, float* colsum, void* stream, uint32_t* d_flags) {
   if (M <= 0 || N <= 0 || K <= 0 || !A || !B || epi_kind < 0 || epi_kind > 6) return GPT_ERR_INVALID_ARG;
+  if (colsum && epi_kind != EPI_ACT_BWD) return GPT_ERR_INVALID_ARG;
   Ctx c;
   c.stream = (cudaStream_t)stream;
   c.flags = d_flags;
@@ -44,12 +45,11 @@ extern "C" gpt_status gpt_test_gemm(int32_t backend, int32_t M, int32_t N, int32
     case GPT_GEMM_SIMT_F32: gemm_simt_f32(c, g); break;
     case GPT_GEMM_SIMT_BF16: gemm_simt_bf16(c, g); break;
     case GPT_GEMM_TC_BF16:
-      if (!gemm_tc_supported(g)) return GPT_ERR_UNSUPPORTED;
-      if (!gemm_tc_bf16(c, g)) return GPT_ERR_CUDA;
-      break;
     case GPT_GEMM_TC2_BF16:
+    case GPT_GEMM_TC_PLANNED:
       if (!gemm_tc_supported(g)) return GPT_ERR_UNSUPPORTED;
-      if (!gemm_tc2_bf16(c, g)) return GPT_ERR_CUDA;
+      if (!gemm_tc_bf16(c, g, backend == GPT_GEMM_TC_BF16 ? TC_SINGLE : backend == GPT_GEMM_TC2_BF16 ? TC_PAIR : TC_ANY))
+        return GPT_ERR_CUDA;
       break;
     case GPT_GEMM_SKINNY_BF16:
       if (!gemm_skinny_supported(g)) return GPT_ERR_UNSUPPORTED;

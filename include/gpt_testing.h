@@ -18,13 +18,15 @@
 extern "C" {
 #endif
 
-/* Backends of gpt_test_gemm. */
+/* Backends of gpt_test_gemm (GPT_GEMM_TC_BF16 forces the single-CTA
+ * tensor-core kernel). */
 enum {
   GPT_GEMM_SIMT_F32 = 0,
   GPT_GEMM_SIMT_BF16 = 1,
   GPT_GEMM_TC_BF16 = 2,
   GPT_GEMM_SKINNY_BF16 = 3,
-  GPT_GEMM_TC2_BF16 = 4  /* pair-CTA tensor-core GEMM (256-row tiles over two SMs) */
+  GPT_GEMM_TC2_BF16 = 4,  /* pair-CTA tensor-core GEMM (256-row tiles over two SMs) */
+  GPT_GEMM_TC_PLANNED = 5 /* the tensor-core kernel and split the training step's cost model picks */
 };
 
 /* D[m, n] = sum_k A[m, k] * B[n, k] followed by epilogue `epi_kind`:
