@@ -591,13 +591,16 @@ def run_ours(args, w, rank, world, local_rank):
 
 def run_kernels(w):
     """One launch of each hot kernel at the workload's micro-batch shapes through
-    the kernel-level test entry points (the small case for ncu captures)."""
+    the kernel-level test entry points (the small case for ncu captures): the
+    GEMMs with the kernel and split the step's cost model picks, both
+    tensor-core attention forwards and the attention backward."""
     import torch
 
     from gpt_decoder_lm_b200 import binding as gb
     st = torch.cuda.current_stream().cuda_stream
     flags = torch.zeros(1, dtype=torch.int32, device="cuda")
     M, d, Vp = w.batch_size * w.block_size, w.n_embd, ((w.vocab_size + 63) // 64) * 64
+    PLANNED = 5
 
     def bf(*s):
         return torch.randn(*s, device="cuda").bfloat16()
@@ -605,23 +608,24 @@ def run_kernels(w):
     x, wqkv, wfc = bf(M, d), bf(3 * d, d), bf(4 * d, d)
     qkv_out = torch.empty(M, 3 * d, dtype=torch.bfloat16, device="cuda")
     h, g = (torch.empty(M, 4 * d, dtype=torch.bfloat16, device="cuda") for _ in range(2))
-    assert gb.test_gemm(2, M, 3 * d, d, x, d, 1, wqkv, d, 1, 1, 0, qkv_out, None, 3 * d, None, None, None, None,
+    assert gb.test_gemm(PLANNED, M, 3 * d, d, x, d, 1, wqkv, d, 1, 1, 0, qkv_out, None, 3 * d, None, None, None, None,
                         1, None, st, flags) == 0
-    assert gb.test_gemm(2, M, 4 * d, d, x, d, 1, wfc, d, 1, 2, 0, h, g, 4 * d, None, torch.zeros(4 * d, device="cuda"),
-                        None, None, 1, None, st, flags) == 0
+    assert gb.test_gemm(PLANNED, M, 4 * d, d, x, d, 1, wfc, d, 1, 2, 0, h, g, 4 * d, None,
+                        torch.zeros(4 * d, device="cuda"), None, None, 1, None, st, flags) == 0
     wte = bf(Vp, d)
     logits = torch.empty(M, Vp, dtype=torch.bfloat16, device="cuda")
-    assert gb.test_gemm(2, M, Vp, d, x, d, 1, wte, d, 1, 0, 0, logits, None, Vp, None, None, None, None, 1, None, st,
-                        flags) == 0
+    assert gb.test_gemm(PLANNED, M, Vp, d, x, d, 1, wte, d, 1, 0, 0, logits, None, Vp, None, None, None, None, 1, None,
+                        st, flags) == 0
     dwte = torch.zeros(Vp, d, device="cuda")
-    assert gb.test_gemm(2, Vp, d, M, logits, Vp, 0, x, d, 0, 5, 0, dwte, None, d, None, None, None, None, 1, None, st,
-                        flags) == 0
+    assert gb.test_gemm(PLANNED, Vp, d, M, logits, Vp, 0, x, d, 0, 5, 0, dwte, None, d, None, None, None, None, 1, None,
+                        st, flags) == 0
     B, T, H = w.batch_size, w.block_size, w.n_head
     q = bf(B, T, 3, H, 64)
     o = torch.empty(B, T, H, 64, dtype=torch.bfloat16, device="cuda")
     lse = torch.empty(B, H, T, device="cuda")
     do, dq, ds = bf(B, T, H, 64), torch.empty_like(q), torch.empty_like(lse)
     assert gb.test_attention(1, 0, 1, B, T, H, 64, q, o, lse, stream=st, flags=flags) == 0
+    assert gb.test_attention(2, 0, 1, B, T, H, 64, q, o, lse, stream=st, flags=flags) == 0
     assert gb.test_attention(1, 1, 1, B, T, H, 64, q, o, lse, do, dq, ds, stream=st, flags=flags) == 0
     torch.cuda.synchronize()
     assert int(flags.item()) == 0

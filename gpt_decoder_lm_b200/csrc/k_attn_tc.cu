@@ -333,7 +333,7 @@ constexpr int F_STAGES = 3;
 constexpr int F_POLY_EVERY = 4;
 
 template <bool DROP>
-__global__ void __maxnreg__(200) k_attn_fwd_pp(const __grid_constant__ CUtensorMap t128, AttnTcArgs a) {
+__global__ void __launch_bounds__(320, 1) k_attn_fwd_pp(const __grid_constant__ CUtensorMap t128, AttnTcArgs a) {
   pdl_trigger();
   const DropKey dk = DROP ? drop_live(a.drop) : a.drop;
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -471,32 +471,31 @@ __global__ void __maxnreg__(200) k_attn_fwd_pp(const __grid_constant__ CUtensorM
     for (int j = 0; j <= jl && ok; j++) {
       if (!(ok = mbar_wait(s_full0 + 8 * t, j & 1, abort_flag, a.flags))) break;
       tc_fence_after();
-      uint32_t v0[32], v1[32], v2[32], v3[32];
-      tmem_ld_32x32b_x32(trow + s_col, v0);
-      tmem_ld_32x32b_x32(trow + s_col + 32, v1);
-      tmem_ld_32x32b_x32(trow + s_col + 64, v2);
-      tmem_ld_32x32b_x32(trow + s_col + 96, v3);
-      tmem_ld_wait();
       const bool diag = j == jl;  // key j*128 + i is visible iff i <= r
-      float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
-      if (!diag) {
+      // row maximum, 64 columns at a time (the register budget of ten warps
+      // is 168 per thread); the second half stays in registers for the exps
+      uint32_t va[32], vb[32];
+      float mx0 = -INFINITY, mx1 = -INFINITY;
 #pragma unroll
-        for (int i = 0; i < 32; i++) {
-          mx0 = fmaxf(mx0, __uint_as_float(v0[i]));
-          mx1 = fmaxf(mx1, __uint_as_float(v1[i]));
-          mx2 = fmaxf(mx2, __uint_as_float(v2[i]));
-          mx3 = fmaxf(mx3, __uint_as_float(v3[i]));
-        }
-      } else {
+      for (int hh = 0; hh < 2; hh++) {
+        tmem_ld_32x32b_x32(trow + s_col + 64 * hh, va);
+        tmem_ld_32x32b_x32(trow + s_col + 64 * hh + 32, vb);
+        tmem_ld_wait();
+        if (!diag) {
 #pragma unroll
-        for (int i = 0; i < 32; i++) {
-          if (i <= r) mx0 = fmaxf(mx0, __uint_as_float(v0[i]));
-          if (i + 32 <= r) mx1 = fmaxf(mx1, __uint_as_float(v1[i]));
-          if (i + 64 <= r) mx2 = fmaxf(mx2, __uint_as_float(v2[i]));
-          if (i + 96 <= r) mx3 = fmaxf(mx3, __uint_as_float(v3[i]));
+          for (int i = 0; i < 32; i++) {
+            mx0 = fmaxf(mx0, __uint_as_float(va[i]));
+            mx1 = fmaxf(mx1, __uint_as_float(vb[i]));
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; i++) {
+            if (64 * hh + i <= r) mx0 = fmaxf(mx0, __uint_as_float(va[i]));
+            if (64 * hh + i + 32 <= r) mx1 = fmaxf(mx1, __uint_as_float(vb[i]));
+          }
         }
       }
-      const float bm = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;
+      const float bm = fmaxf(mx0, mx1) * sl2;
       if (j == 0) {
         m = bm;  // key 0 is visible to every row, so m is finite from here on
       } else {
@@ -517,44 +516,49 @@ __global__ void __maxnreg__(200) k_attn_fwd_pp(const __grid_constant__ CUtensorM
           if (need) m = bm;
         }
       }
-      // probabilities of the 128 keys, packed bf16 pairs (P = the A operand of P V)
+      // probabilities of the 128 keys, packed bf16 pairs (P = the A operand of
+      // P V), the half of keys 64..127 (still in registers) first
       const uint64_t neg_m = f2c(-m), scl = f2c(sl2);
       float lsum = 0.f;
 #pragma unroll
-      for (int half = 0; half < 2; half++) {  // 64 keys per half: its packed P goes to TMEM before the next
+      for (int hi = 1; hi >= 0; hi--) {
+        if (hi == 0) {
+          tmem_ld_32x32b_x32(trow + s_col, va);
+          tmem_ld_32x32b_x32(trow + s_col + 32, vb);
+          tmem_ld_wait();
+        }
         uint32_t pk[32];
 #pragma unroll
         for (int cc = 0; cc < 2; cc++) {
-        const int c = 2 * half + cc;
-        const uint32_t* vc = c == 0 ? v0 : c == 1 ? v1 : c == 2 ? v2 : v3;
+          const uint32_t* vc = cc == 0 ? va : vb;
 #pragma unroll
-        for (int i = 0; i < 32; i += 2) {
-          const int k = 32 * c + i;  // key offset in the block
-          const uint64_t x2 = f2fma(f2(__uint_as_float(vc[i]), __uint_as_float(vc[i + 1])), scl, neg_m);
-          float p0, p1;
-          if (((k >> 1) % F_POLY_EVERY) == F_POLY_EVERY - 1) {
-            const float2 e = f2split(exp2_poly2(x2));
-            p0 = e.x;
-            p1 = e.y;
-          } else {
-            const float2 x = f2split(x2);
-            p0 = ex2(x.x);
-            p1 = ex2(x.y);
+          for (int i = 0; i < 32; i += 2) {
+            const int k = 64 * hi + 32 * cc + i;  // key offset in the block
+            const uint64_t x2 = f2fma(f2(__uint_as_float(vc[i]), __uint_as_float(vc[i + 1])), scl, neg_m);
+            float p0, p1;
+            if (((k >> 1) % F_POLY_EVERY) == F_POLY_EVERY - 1) {
+              const float2 e = f2split(exp2_poly2(x2));
+              p0 = e.x;
+              p1 = e.y;
+            } else {
+              const float2 x = f2split(x2);
+              p0 = ex2(x.x);
+              p1 = ex2(x.y);
+            }
+            if (diag) {
+              if (k > r) p0 = 0.f;
+              if (k + 1 > r) p1 = 0.f;
+            }
+            lsum += p0 + p1;
+            if (DROP) {
+              const uint64_t e = ebase + (uint64_t)j * 128 + k;
+              p0 *= drop_mul(dk, e);
+              p1 *= drop_mul(dk, e + 1);
+            }
+            pk[(32 * cc + i) >> 1] = pack2(p0, p1);
           }
-          if (diag) {
-            if (k > r) p0 = 0.f;
-            if (k + 1 > r) p1 = 0.f;
-          }
-          lsum += p0 + p1;
-          if (DROP) {
-            const uint64_t e = ebase + (uint64_t)j * 128 + k;
-            p0 *= drop_mul(dk, e);
-            p1 *= drop_mul(dk, e + 1);
-          }
-          pk[(k - 64 * half) >> 1] = pack2(p0, p1);
         }
-        }
-        tmem_st_32x32b_x32(trow + s_col + 32 * half, pk);
+        tmem_st_32x32b_x32(trow + s_col + 32 * hi, pk);
       }
       l += lsum;
       tmem_st_wait();

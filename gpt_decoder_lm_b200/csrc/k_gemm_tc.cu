@@ -417,7 +417,7 @@ bool launch(Ctx& c, const GemmDesc& g, int splits) {
 // lower operand reuse, pair tiles gain from each SM loading half of B), whole
 // waves over the SMs (pairs of SMs for the pair kernel), and the traffic of
 // split-K partials (written and read back once).
-constexpr double KB_CYCLES_256 = 512.0, KB_CYCLES_128 = 330.0, KB_CYCLES_PAIR = 530.0;
+constexpr double KB_CYCLES_256 = 512.0, KB_CYCLES_128 = 330.0, KB_CYCLES_PAIR = 470.0;
 TcPlan gemm_tc_plan(long M, long N, long K, bool split_ok, int num_sms, int mode) {
   TcPlan best{256, 1, 0};
   double best_t = 1e30;

@@ -32,7 +32,9 @@ def _caller_scratch(A, B, base, M, N, K, splits, stream):
     out = base.clone()
     partial = torch.empty(splits, M, N, device="cuda")
     flags = torch.zeros(1, dtype=torch.int32, device="cuda")
-    st = gb.test_gemm(2, M, N, K, A, M, 0, B, N, 0, 5, 0, out, None, N, None, None, None, None, splits, partial,
+    # backend 5: the kernel and split count the library's cost model picks,
+    # which the allocation-free entry point runs too
+    st = gb.test_gemm(5, M, N, K, A, M, 0, B, N, 0, 5, 0, out, None, N, None, None, None, None, splits, partial,
                       stream, flags)
     assert gb.STATUS[st] == "GPT_OK" and int(flags.item()) == 0
     return out
