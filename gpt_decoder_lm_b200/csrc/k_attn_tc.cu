@@ -1094,6 +1094,484 @@ __global__ void __launch_bounds__(320, 2) k_attn_bwd_q8(const __grid_constant__ 
   if (warp == 1) tmem_dealloc(tmem, 256);
 }
 
+// ============================================================================
+// backward, wide: the dK/dV and dQ kernels with 128-wide inner blocks (N = 128
+// MMAs: half the MMA issues per FLOP of the 64-wide kernels), one CTA per SM
+// (TMEM: S 128 | dP 128 | accumulators).  Eight math warps, two per TMEM lane
+// quadrant, each taking 64 of the 128 columns; the same two math phases per
+// block and the same MMA issue order as the 64-wide kernels; the packed bf16
+// P~ / dS of a warp's 64 columns go into the first 32 of them (already read).
+// ============================================================================
+// TMEM A-operand column of K-step kk (16 elements) of a 128-wide block whose
+// halves pack into their own first 32 columns
+__device__ __forceinline__ uint32_t acolw(int kk) { return (uint32_t)((kk >> 2) * 64 + (kk & 3) * 8); }
+
+constexpr int KW_K = 0, KW_V = TILE, KW_ST = 2 * TILE, KW_LD = (2 + 2 * BWD_STAGES) * TILE;
+constexpr int KW_BAR = KW_LD + 1024 * BWD_STAGES;
+constexpr int KW_SMEM = KW_BAR + 128;
+
+template <bool DROP>
+__global__ void __launch_bounds__(320, 1) k_attn_bwd_kvw(const __grid_constant__ CUtensorMap tkv,
+                                                         const __grid_constant__ CUtensorMap tdo, AttnTcArgs a) {
+  pdl_trigger();
+  const DropKey dk = DROP ? drop_live(a.drop) : a.drop;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (smem_u32(smem) & 1023) {
+    if (threadIdx.x == 0) atomicOr(a.flags, FLAG_TIMEOUT);
+    return;
+  }
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + KW_BAR);
+  const uint32_t kv_full = smem_u32(bars + 0), st_full0 = smem_u32(bars + 1),
+                 st_empty0 = smem_u32(bars + 1 + BWD_STAGES);
+  const uint32_t s_full = smem_u32(bars + 1 + 2 * BWD_STAGES), dp_full = s_full + 8, p_ready = s_full + 16,
+                 ds_ready = s_full + 24, acc_full = s_full + 32;
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + 6 + 2 * BWD_STAGES);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tslot + 1);
+  const float* sld = reinterpret_cast<const float*>(smem + KW_LD);  // [stage][lse 128 | D 128]
+  const uint32_t sb = smem_u32(smem);
+
+  const int nqb = a.T / 128;
+  const int kb = (int)blockIdx.y;  // key block 0 (most query blocks) of every (b, h) first
+  const int bh = blockIdx.x, b = bh / a.H, h = bh % a.H;
+  const int row0 = b * a.T;
+  const int nit = nqb - kb;  // query blocks kb .. nqb-1
+
+  if (threadIdx.x == 0) {
+    mbar_init(kv_full, 1);
+    for (int s = 0; s < BWD_STAGES; s++) {
+      mbar_init(st_full0 + 8 * s, 1);
+      mbar_init(st_empty0 + 8 * s, 1);
+    }
+    mbar_init(s_full, 1);
+    mbar_init(dp_full, 1);
+    mbar_init(p_ready, 8);
+    mbar_init(ds_ready, 8);
+    mbar_init(acc_full, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+    prefetch_tmap(&tkv);
+    prefetch_tmap(&tdo);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tslot), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tslot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      mbar_expect_tx(kv_full, 2 * TILE);
+      tma_load_3d(sb + KW_K, &tkv, kv_full, 0, a.H + h, row0 + kb * 128);
+      tma_load_3d(sb + KW_V, &tkv, kv_full, 0, 2 * a.H + h, row0 + kb * 128);
+      int issued = 0;
+      bool ok = true;
+      for (int it = 0; it < nit; it++) {
+        const int i = kb + it, s = it % BWD_STAGES;
+        const uint32_t fb = st_full0 + 8 * s;
+        if (!(ok = mbar_wait(st_empty0 + 8 * s, ((it / BWD_STAGES) & 1) ^ 1, abort_flag, a.flags))) break;
+        mbar_expect_tx(fb, 2 * TILE + 1024);
+        tma_load_3d(sb + KW_ST + s * 2 * TILE, &tkv, fb, 0, h, row0 + i * 128);
+        tma_load_3d(sb + KW_ST + s * 2 * TILE + TILE, &tdo, fb, 0, h, row0 + i * 128);
+        bulk_load(sb + KW_LD + s * 1024, a.lse + (size_t)bh * a.T + i * 128, 512, fb);
+        bulk_load(sb + KW_LD + s * 1024 + 512, a.dsum + (size_t)bh * a.T + i * 128, 512, fb);
+        issued = it + 1;
+      }
+      if (!ok) {  // the loads already issued land before the CTA can exit
+        mbar_wait(kv_full, 0, abort_flag, a.flags);
+        for (int it = issued - BWD_STAGES < 0 ? 0 : issued - BWD_STAGES; it < issued; it++)
+          mbar_wait(st_full0 + 8 * (it % BWD_STAGES), (it / BWD_STAGES) & 1, abort_flag, a.flags);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t id_s = idesc_bf16_f32(128, 128, false, false);
+      constexpr uint32_t id_acc = idesc_bf16_f32(128, 64, false, true);
+      auto q_of = [&](int it) { return sb + KW_ST + (it % BWD_STAGES) * 2 * TILE; };
+      auto issue_s = [&](int it) -> bool {  // S^T = K Q^T of block it
+        if (!mbar_wait(st_full0 + 8 * (it % BWD_STAGES), (it / BWD_STAGES) & 1, abort_flag, a.flags)) return false;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 4; kk++)
+          mma_bf16_ss(tmem, desc_k(sb + KW_K, TILE, kk), desc_k(q_of(it), TILE, kk), id_s, kk > 0);
+        mma_commit(s_full);
+        return true;
+      };
+      auto issue_dp = [&](int it) {  // dP^T = V dO^T of block it (its stage is loaded)
+#pragma unroll
+        for (int kk = 0; kk < 4; kk++)
+          mma_bf16_ss(tmem + 128, desc_k(sb + KW_V, TILE, kk), desc_k(q_of(it) + TILE, TILE, kk), id_s, kk > 0);
+        mma_commit(dp_full);
+      };
+      bool ok = mbar_wait(kv_full, 0, abort_flag, a.flags) && issue_s(0);
+      if (ok) issue_dp(0);
+      for (int it = 0; it < nit && ok; it++) {
+        const uint32_t q = q_of(it), dO = q + TILE;
+        if (!(ok = mbar_wait(p_ready, it & 1, abort_flag, a.flags))) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 8; kk++)  // dV += P~^T dO (K = the block's 128 queries)
+          mma_bf16_ts(tmem + 256, tmem + acolw(kk), desc_mn64(dO, kk), id_acc, (it > 0 || kk > 0));
+        if (it + 1 < nit && !(ok = issue_s(it + 1))) break;
+        if (!(ok = mbar_wait(ds_ready, it & 1, abort_flag, a.flags))) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 8; kk++)  // dK += dS^T Q
+          mma_bf16_ts(tmem + 320, tmem + 128 + acolw(kk), desc_mn64(q, kk), id_acc, (it > 0 || kk > 0));
+        mma_commit(st_empty0 + 8 * (it % BWD_STAGES));
+        if (it + 1 < nit) issue_dp(it + 1);
+      }
+      mma_commit(acc_full);
+    }
+  } else {
+    const int quad = warp & 3;
+    const int half = (warp - 2) >> 2;
+    const int r = quad * 32 + lane;
+    const int kj = kb * 128 + r;
+    const uint32_t trow = tmem + ((uint32_t)(quad * 32) << 16);
+    const uint64_t sl2x2 = f2(a.scale_log2, a.scale_log2), nlog2e = f2(-LOG2E, -LOG2E);
+    bool ok = true;
+    for (int it = 0; it < nit; it++) {
+      const int i = kb + it;
+      const int q0 = i * 128;
+      const float* ld = sld + (it % BWD_STAGES) * 256;  // lse[128] | D[128] of this query block
+      if (!(ok = mbar_wait(st_full0 + 8 * (it % BWD_STAGES), (it / BWD_STAGES) & 1, abort_flag, a.flags))) break;
+      if (!(ok = mbar_wait(s_full, it & 1, abort_flag, a.flags))) break;
+      tc_fence_after();
+      const bool masked = it == 0;  // the diagonal block: query column c is masked iff c < r
+      float pk[4][16];              // P^T of this thread's 64 columns
+      // phase 1: P^T = 2^(S^T sl2 - lse log2 e) (masked), P~^T = drop(P^T)
+#pragma unroll
+      for (int sub = 0; sub < 4; sub++) {
+        const int c0 = half * 64 + sub * 16;
+        uint32_t sv[16];
+        tmem_ld_32x32b_x16(trow + c0, sv);
+        tmem_ld_wait();
+        uint32_t pp[8];
+#pragma unroll
+        for (int e = 0; e < 16; e += 4) {
+          const float4 l4 = *reinterpret_cast<const float4*>(ld + c0 + e);
+          const uint64_t y01 = f2fma(f2(__uint_as_float(sv[e]), __uint_as_float(sv[e + 1])), sl2x2,
+                                     f2mul(f2(l4.x, l4.y), nlog2e));
+          const uint64_t y23 = f2fma(f2(__uint_as_float(sv[e + 2]), __uint_as_float(sv[e + 3])), sl2x2,
+                                     f2mul(f2(l4.z, l4.w), nlog2e));
+          float p4[4];
+          if (((e >> 1) % BWD_POLY_EVERY) == BWD_POLY_EVERY - 1) {
+            const float2 q01 = f2split(exp2_poly2(y01));
+            p4[0] = q01.x;
+            p4[1] = q01.y;
+          } else {
+            const float2 x01 = f2split(y01);
+            p4[0] = ex2(x01.x);
+            p4[1] = ex2(x01.y);
+          }
+          if ((((e >> 1) + 1) % BWD_POLY_EVERY) == BWD_POLY_EVERY - 1) {
+            const float2 q23 = f2split(exp2_poly2(y23));
+            p4[2] = q23.x;
+            p4[3] = q23.y;
+          } else {
+            const float2 x23 = f2split(y23);
+            p4[2] = ex2(x23.x);
+            p4[3] = ex2(x23.y);
+          }
+#pragma unroll
+          for (int u = 0; u < 4; u++) {
+            if (masked && c0 + e + u < r) p4[u] = 0.f;
+            pk[sub][e + u] = p4[u];
+          }
+          if (DROP) {
+#pragma unroll
+            for (int u = 0; u < 4; u++)
+              p4[u] *= drop_mul(dk, ((uint64_t)bh * a.T + q0 + c0 + e + u) * a.T + kj);
+          }
+          pp[e >> 1] = pack2(p4[0], p4[1]);
+          pp[(e >> 1) + 1] = pack2(p4[2], p4[3]);
+        }
+        tmem_st_32x32b_x8(trow + half * 64 + sub * 8, pp);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(p_ready);
+      // phase 2: dS^T = P^T (drop(dP^T) - D)
+      if (!(ok = mbar_wait(dp_full, it & 1, abort_flag, a.flags))) break;
+      tc_fence_after();
+#pragma unroll
+      for (int sub = 0; sub < 4; sub++) {
+        const int c0 = half * 64 + sub * 16;
+        uint32_t dv[16];
+        tmem_ld_32x32b_x16(trow + 128 + c0, dv);
+        tmem_ld_wait();
+        uint32_t pd[8];
+#pragma unroll
+        for (int e = 0; e < 16; e += 2) {
+          const float2 d2 = *reinterpret_cast<const float2*>(ld + 128 + c0 + e);
+          float dp0 = __uint_as_float(dv[e]), dp1 = __uint_as_float(dv[e + 1]);
+          if (DROP) {
+            dp0 *= drop_mul(dk, ((uint64_t)bh * a.T + q0 + c0 + e) * a.T + kj);
+            dp1 *= drop_mul(dk, ((uint64_t)bh * a.T + q0 + c0 + e + 1) * a.T + kj);
+          }
+          pd[e >> 1] = pack2v(f2mul(f2(pk[sub][e], pk[sub][e + 1]), f2sub(f2(dp0, dp1), f2(d2.x, d2.y))));
+        }
+        tmem_st_32x32b_x8(trow + 128 + half * 64 + sub * 8, pd);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(ds_ready);
+    }
+    if (ok && mbar_wait(acc_full, 0, abort_flag, a.flags)) {
+      tc_fence_after();
+      bf16* rowp = a.dqkv + (size_t)(row0 + kj) * (3 * a.H * 64);
+      // half 0: dV at slot 2H+h; half 1: dK (times 1/sqrt(hd)) at slot H+h
+      const float f = half == 0 ? 1.0f : a.scale;
+      uint4* dst = reinterpret_cast<uint4*>(rowp + (size_t)((half == 0 ? 2 : 1) * a.H + h) * 64);
+#pragma unroll
+      for (int c = 0; c < 4; c++) {
+        uint32_t v[16];
+        tmem_ld_32x32b_x16(trow + 256 + half * 64 + c * 16, v);
+        tmem_ld_wait();
+        const float* x = reinterpret_cast<const float*>(v);
+        dst[2 * c] = make_uint4(pack2(x[0] * f, x[1] * f), pack2(x[2] * f, x[3] * f), pack2(x[4] * f, x[5] * f),
+                                pack2(x[6] * f, x[7] * f));
+        dst[2 * c + 1] = make_uint4(pack2(x[8] * f, x[9] * f), pack2(x[10] * f, x[11] * f),
+                                    pack2(x[12] * f, x[13] * f), pack2(x[14] * f, x[15] * f));
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, 512);
+}
+
+constexpr int QW_Q = 0, QW_DO = TILE, QW_OT = 2 * TILE, QW_ST = 3 * TILE, QW_BAR = (3 + 2 * BWD_STAGES) * TILE;
+constexpr int QW_SMEM = QW_BAR + 128;
+
+template <bool DROP>
+__global__ void __launch_bounds__(320, 1) k_attn_bwd_qw(const __grid_constant__ CUtensorMap tkv,
+                                                        const __grid_constant__ CUtensorMap tdo,
+                                                        const __grid_constant__ CUtensorMap tout, AttnTcArgs a) {
+  pdl_trigger();
+  const DropKey dk = DROP ? drop_live(a.drop) : a.drop;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (smem_u32(smem) & 1023) {
+    if (threadIdx.x == 0) atomicOr(a.flags, FLAG_TIMEOUT);
+    return;
+  }
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + QW_BAR);
+  const uint32_t qd_full = smem_u32(bars + 0), kv_full0 = smem_u32(bars + 1),
+                 kv_empty0 = smem_u32(bars + 1 + BWD_STAGES);
+  const uint32_t s_full = smem_u32(bars + 1 + 2 * BWD_STAGES), dp_full = s_full + 8, s_read = s_full + 16,
+                 ds_ready = s_full + 24, acc_full = s_full + 32;
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + 6 + 2 * BWD_STAGES);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tslot + 1);
+  const uint32_t sb = smem_u32(smem);
+
+  const int nqb = a.T / 128;
+  const int qb = nqb - 1 - (int)blockIdx.y;  // longest rows of every (b, h) first
+  const int bh = blockIdx.x, b = bh / a.H, h = bh % a.H;
+  const int row0 = b * a.T;
+  const int nkb = qb + 1;  // 128-key blocks up to and including the diagonal
+
+  if (threadIdx.x == 0) {
+    mbar_init(qd_full, 1);
+    for (int s = 0; s < BWD_STAGES; s++) {
+      mbar_init(kv_full0 + 8 * s, 1);
+      mbar_init(kv_empty0 + 8 * s, 1);
+    }
+    mbar_init(s_full, 1);
+    mbar_init(dp_full, 1);
+    mbar_init(s_read, 8);
+    mbar_init(ds_ready, 8);
+    mbar_init(acc_full, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+    prefetch_tmap(&tkv);
+    prefetch_tmap(&tdo);
+    prefetch_tmap(&tout);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tslot), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tslot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      mbar_expect_tx(qd_full, 3 * TILE);
+      tma_load_3d(sb + QW_Q, &tkv, qd_full, 0, h, row0 + qb * 128);
+      tma_load_3d(sb + QW_DO, &tdo, qd_full, 0, h, row0 + qb * 128);
+      tma_load_3d(sb + QW_OT, &tout, qd_full, 0, h, row0 + qb * 128);
+      int issued = 0;
+      bool ok = true;
+      for (int j = 0; j < nkb; j++) {
+        const int s = j % BWD_STAGES;
+        const uint32_t fb = kv_full0 + 8 * s;
+        if (!(ok = mbar_wait(kv_empty0 + 8 * s, ((j / BWD_STAGES) & 1) ^ 1, abort_flag, a.flags))) break;
+        mbar_expect_tx(fb, 2 * TILE);
+        tma_load_3d(sb + QW_ST + s * 2 * TILE, &tkv, fb, 0, a.H + h, row0 + j * 128);
+        tma_load_3d(sb + QW_ST + s * 2 * TILE + TILE, &tkv, fb, 0, 2 * a.H + h, row0 + j * 128);
+        issued = j + 1;
+      }
+      if (!ok) {  // the loads already issued land before the CTA can exit
+        mbar_wait(qd_full, 0, abort_flag, a.flags);
+        for (int j = issued - BWD_STAGES < 0 ? 0 : issued - BWD_STAGES; j < issued; j++)
+          mbar_wait(kv_full0 + 8 * (j % BWD_STAGES), (j / BWD_STAGES) & 1, abort_flag, a.flags);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t id_s = idesc_bf16_f32(128, 128, false, false);
+      constexpr uint32_t id_acc = idesc_bf16_f32(128, 64, false, true);
+      auto k_of = [&](int j) { return sb + QW_ST + (j % BWD_STAGES) * 2 * TILE; };
+      auto issue_s = [&](int j) -> bool {  // S = Q K^T of block j
+        if (!mbar_wait(kv_full0 + 8 * (j % BWD_STAGES), (j / BWD_STAGES) & 1, abort_flag, a.flags)) return false;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 4; kk++)
+          mma_bf16_ss(tmem, desc_k(sb + QW_Q, TILE, kk), desc_k(k_of(j), TILE, kk), id_s, kk > 0);
+        mma_commit(s_full);
+        return true;
+      };
+      auto issue_dp = [&](int j) {  // dP = dO V^T of block j (its stage is loaded)
+#pragma unroll
+        for (int kk = 0; kk < 4; kk++)
+          mma_bf16_ss(tmem + 128, desc_k(sb + QW_DO, TILE, kk), desc_k(k_of(j) + TILE, TILE, kk), id_s, kk > 0);
+        mma_commit(dp_full);
+      };
+      bool ok = mbar_wait(qd_full, 0, abort_flag, a.flags) && issue_s(0);
+      if (ok) issue_dp(0);
+      for (int j = 0; j < nkb && ok; j++) {
+        if (!(ok = mbar_wait(s_read, j & 1, abort_flag, a.flags))) break;
+        if (j + 1 < nkb && !(ok = issue_s(j + 1))) break;
+        if (!(ok = mbar_wait(ds_ready, j & 1, abort_flag, a.flags))) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 8; kk++)  // dQ += dS K (K = the block's 128 keys)
+          mma_bf16_ts(tmem + 256, tmem + 128 + acolw(kk), desc_mn64(k_of(j), kk), id_acc, (j > 0 || kk > 0));
+        mma_commit(kv_empty0 + 8 * (j % BWD_STAGES));
+        if (j + 1 < nkb) issue_dp(j + 1);
+      }
+      mma_commit(acc_full);
+    }
+  } else {
+    const int quad = warp & 3;
+    const int half = (warp - 2) >> 2;
+    const int r = quad * 32 + lane;
+    const int qi = qb * 128 + r;
+    const uint32_t trow = tmem + ((uint32_t)(quad * 32) << 16);
+    const float lse2 = a.lse[(size_t)bh * a.T + qi] * LOG2E;
+    // D of this row from the dO and O tiles (128-byte rows, 128-byte swizzle:
+    // 16-byte chunk q of row r at q ^ (r & 7)); both halves compute it
+    bool ok = mbar_wait(qd_full, 0, abort_flag, a.flags);
+    float Di = 0.f;
+    if (ok) {
+#pragma unroll
+      for (int q = 0; q < 8; q++) {
+        const uint32_t off = r * 128 + ((q ^ (r & 7)) << 4);
+        const uint4 x = ld_shared_v4(sb + QW_DO + off), y = ld_shared_v4(sb + QW_OT + off);
+        const uint32_t xw[4] = {x.x, x.y, x.z, x.w}, yw[4] = {y.x, y.y, y.z, y.w};
+#pragma unroll
+        for (int k = 0; k < 4; k++) {
+          const float2 xf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&xw[k]));
+          const float2 yf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&yw[k]));
+          Di = fmaf(xf.x, yf.x, fmaf(xf.y, yf.y, Di));
+        }
+      }
+      if (half == 0) a.dsum[(size_t)bh * a.T + qi] = Di;
+    }
+    const uint64_t sl2x2 = f2(a.scale_log2, a.scale_log2), nlse2 = f2(-lse2, -lse2), Dx2 = f2(Di, Di);
+    const uint64_t ebase = ((uint64_t)bh * a.T + qi) * a.T;
+    for (int j = 0; j < nkb && ok; j++) {
+      if (!(ok = mbar_wait(s_full, j & 1, abort_flag, a.flags))) break;
+      tc_fence_after();
+      const int key0 = j * 128;
+      const bool masked = j == qb;  // the diagonal block: key column c is visible iff c <= r
+      // phase 1: P = 2^(S sl2 - lse log2 e) (masked) into registers
+      float pk[4][16];
+#pragma unroll
+      for (int sub = 0; sub < 4; sub++) {
+        const int c0 = half * 64 + sub * 16;
+        uint32_t sv[16];
+        tmem_ld_32x32b_x16(trow + c0, sv);
+        tmem_ld_wait();
+#pragma unroll
+        for (int e = 0; e < 16; e += 2) {
+          const uint64_t y2 = f2fma(f2(__uint_as_float(sv[e]), __uint_as_float(sv[e + 1])), sl2x2, nlse2);
+          float e0, e1;
+          if (((e >> 1) % BWD_POLY_EVERY) == BWD_POLY_EVERY - 1) {
+            const float2 q = f2split(exp2_poly2(y2));
+            e0 = q.x;
+            e1 = q.y;
+          } else {
+            const float2 y = f2split(y2);
+            e0 = ex2(y.x);
+            e1 = ex2(y.y);
+          }
+          pk[sub][e] = (masked && c0 + e > r) ? 0.f : e0;
+          pk[sub][e + 1] = (masked && c0 + e + 1 > r) ? 0.f : e1;
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(s_read);  // S may be overwritten by the next block
+      // phase 2: dS = P (drop(dP) - D) over the dP columns
+      if (!(ok = mbar_wait(dp_full, j & 1, abort_flag, a.flags))) break;
+      tc_fence_after();
+#pragma unroll
+      for (int sub = 0; sub < 4; sub++) {
+        const int c0 = half * 64 + sub * 16;
+        uint32_t dv[16];
+        tmem_ld_32x32b_x16(trow + 128 + c0, dv);
+        tmem_ld_wait();
+        uint32_t pd[8];
+#pragma unroll
+        for (int e = 0; e < 16; e += 2) {
+          float dp0 = __uint_as_float(dv[e]), dp1 = __uint_as_float(dv[e + 1]);
+          if (DROP) {
+            dp0 *= drop_mul(dk, ebase + key0 + c0 + e);
+            dp1 *= drop_mul(dk, ebase + key0 + c0 + e + 1);
+          }
+          pd[e >> 1] = pack2v(f2mul(f2(pk[sub][e], pk[sub][e + 1]), f2sub(f2(dp0, dp1), Dx2)));
+        }
+        tmem_st_32x32b_x8(trow + 128 + half * 64 + sub * 8, pd);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(ds_ready);
+    }
+    if (ok && mbar_wait(acc_full, 0, abort_flag, a.flags)) {
+      tc_fence_after();
+      uint4* dst = reinterpret_cast<uint4*>(a.dqkv + (size_t)(row0 + qi) * (3 * a.H * 64) + (size_t)h * 64 + half * 32);
+      const float f = a.scale;
+#pragma unroll
+      for (int c = 0; c < 2; c++) {
+        uint32_t v[16];
+        tmem_ld_32x32b_x16(trow + 256 + half * 32 + c * 16, v);
+        tmem_ld_wait();
+        const float* x = reinterpret_cast<const float*>(v);
+        dst[2 * c] = make_uint4(pack2(x[0] * f, x[1] * f), pack2(x[2] * f, x[3] * f), pack2(x[4] * f, x[5] * f),
+                                pack2(x[6] * f, x[7] * f));
+        dst[2 * c + 1] = make_uint4(pack2(x[8] * f, x[9] * f), pack2(x[10] * f, x[11] * f),
+                                    pack2(x[12] * f, x[13] * f), pack2(x[14] * f, x[15] * f));
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, 512);
+}
+
 // ---------------------------------------------------------------- host side
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
@@ -1180,6 +1658,33 @@ bool attn_fwd_tc_pp(Ctx& c, const AttnDesc& d) {
   LaunchScope s(c, "attn_fwd_tc");
   if (drop) k_attn_fwd_pp<true><<<grid, 320, F_SMEM, c.stream>>>(t128, make_args(d, c.flags));
   else k_attn_fwd_pp<false><<<grid, 320, F_SMEM, c.stream>>>(t128, make_args(d, c.flags));
+  return true;
+}
+
+// the wide backward (128-wide inner blocks, one CTA per SM): dQ (with D) first
+bool attn_bwd_tc_wide(Ctx& c, const AttnDesc& d) {
+  CUtensorMap tkv, tdo, tout;
+  long rows = (long)d.B * d.T;
+  if (!map_rows(&tkv, d.qkv, 3 * d.H, rows, 128) || !map_rows(&tdo, d.dout, d.H, rows, 128) ||
+      !map_rows(&tout, d.o, d.H, rows, 128))
+    return false;
+  const bool drop = d.drop.active;
+  cudaFuncSetAttribute(drop ? k_attn_bwd_kvw<true> : k_attn_bwd_kvw<false>,
+                       cudaFuncAttributeMaxDynamicSharedMemorySize, KW_SMEM);
+  cudaFuncSetAttribute(drop ? k_attn_bwd_qw<true> : k_attn_bwd_qw<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                       QW_SMEM);
+  AttnTcArgs a = make_args(d, c.flags);
+  dim3 grid(d.B * d.H, d.T / 128);
+  {
+    LaunchScope s(c, "attn_bwd_q_tc");
+    if (drop) k_attn_bwd_qw<true><<<grid, 320, QW_SMEM, c.stream>>>(tkv, tdo, tout, a);
+    else k_attn_bwd_qw<false><<<grid, 320, QW_SMEM, c.stream>>>(tkv, tdo, tout, a);
+  }
+  {
+    LaunchScope s(c, "attn_bwd_kv_tc");
+    if (drop) k_attn_bwd_kvw<true><<<grid, 320, KW_SMEM, c.stream>>>(tkv, tdo, a);
+    else k_attn_bwd_kvw<false><<<grid, 320, KW_SMEM, c.stream>>>(tkv, tdo, a);
+  }
   return true;
 }
 

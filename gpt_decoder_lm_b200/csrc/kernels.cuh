@@ -142,6 +142,7 @@ bool attn_tc_supported(const AttnDesc& a);  // shape rule plus 16-byte aligned p
 bool attn_fwd_tc(Ctx& c, const AttnDesc& a);
 bool attn_fwd_tc_pp(Ctx& c, const AttnDesc& a);  // two query tiles per CTA, 128-key blocks
 bool attn_bwd_tc(Ctx& c, const AttnDesc& a);
+bool attn_bwd_tc_wide(Ctx& c, const AttnDesc& a);  // 128-wide inner blocks, one CTA per SM
 // decoding: o [B, H*hd] = attention of position t against positions 0..t of
 // the cache qkv [B, T, 3, H, hd]
 template <typename T> void attn_decode(Ctx& c, const T* qkv, int B, int Tn, int H, int hd, int t, T* o);

@@ -71,9 +71,10 @@ extern "C" gpt_status gpt_test_attention(int32_t backend, int32_t backward, int3
   c.stream = (cudaStream_t)stream;
   c.flags = d_flags;
   AttnDesc a{B, T, H, hd, qkv, o, lse, dout, dqkv, dsum, make_drop_key(seed, counter, layer, 1, p)};
-  if (backend == 1 || backend == 2) {
+  if (backend >= 1 && backend <= 3) {
     if (dtype != 1 || !attn_tc_supported(a)) return GPT_ERR_UNSUPPORTED;
-    const bool ok = backward ? attn_bwd_tc(c, a) : backend == 2 ? attn_fwd_tc_pp(c, a) : attn_fwd_tc(c, a);
+    const bool ok = backward ? (backend == 3 ? attn_bwd_tc_wide(c, a) : attn_bwd_tc(c, a))
+                             : (backend == 1 ? attn_fwd_tc(c, a) : attn_fwd_tc_pp(c, a));
     if (!ok) return GPT_ERR_CUDA;
   } else if (backend == 0) {
     if (hd != 4 && hd != 8 && hd != 16 && hd != 32 && hd != 64 && hd != 128) return GPT_ERR_UNSUPPORTED;

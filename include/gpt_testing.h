@@ -54,8 +54,9 @@ gpt_status gpt_test_gemm(int32_t backend, int32_t M, int32_t N, int32_t K, const
  * lse fp32 [B, H, T]; backward also takes dout [B, T, H, hd] and writes
  * dqkv [B, T, 3, H, hd] using dsum fp32 [B, H, T] as scratch.  dtype: 0 fp32,
  * 1 bf16.  backend: 0 CUDA cores, 1 tensor cores, 2 tensor cores with the
- * two-tile (ping-pong) forward kernel (GPT_ERR_UNSUPPORTED when the shape is
- * not supported).  Dropout on the probabilities with
+ * two-tile (ping-pong) forward kernel, 3 the ping-pong forward and the
+ * backward kernels with 128-wide inner blocks (GPT_ERR_UNSUPPORTED when the
+ * shape is not supported).  Dropout on the probabilities with
  * (p, seed, counter, layer) as in the model (site 1); p = 0 disables it. */
 gpt_status gpt_test_attention(int32_t backend, int32_t backward, int32_t dtype, int32_t B, int32_t T, int32_t H,
                               int32_t hd, const void* qkv, void* o, float* lse, const void* dout, void* dqkv,

@@ -77,11 +77,11 @@ def run_case(backend, B, T, H, p, seed=0, qkv_np=None):
 @pytest.mark.parametrize("B,T,H", [(2, 256, 3), (1, 512, 2), (1, 128, 1), (1, 384, 2), (2, 1024, 12),
                                    (1, 1024, 25)])
 @pytest.mark.parametrize("p", [0.0, 0.1], ids=["nodrop", "dropout"])
-@pytest.mark.parametrize("backend", [1, 2], ids=["fwd64", "fwd_pingpong"])
+@pytest.mark.parametrize("backend", [1, 2, 3], ids=["fwd64", "fwd_pingpong", "wide"])
 def test_attention_tensor_core(B, T, H, p, backend):
     # backend 2: the forward with two 128-query tiles per CTA and 128-key
-    # blocks (T = 128 and 384 leave a CTA with one tile); the backward is the
-    # same kernel pair for both
+    # blocks (T = 128 and 384 leave a CTA with one tile); backend 3: that
+    # forward and the backward kernels with 128-wide inner blocks
     run_case(backend, B, T, H, p)
 
 
@@ -108,5 +108,5 @@ def test_attention_rescale_path():
     u /= np.linalg.norm(u)
     x[:, :, 0] += 21.0 * u
     x[:, :, 1] += (np.arange(T) / T * 21.0)[None, :, None, None] * u
-    run_case(1, B, T, H, 0.0, qkv_np=x)
-    run_case(2, B, T, H, 0.0, qkv_np=x)
+    for backend in (1, 2, 3):
+        run_case(backend, B, T, H, 0.0, qkv_np=x)
