@@ -103,7 +103,7 @@ _PROTOS = {
     "gpt_status_string": (C.c_char_p, [I32]),
     "gpt_test_gemm": (I32, [I32, I32, I32, I32, P, I64, I32, P, I64, I32, I32, I32, P, P, I32, P, P, P, P, I32, P,
                             P, P, P]),
-    "gpt_test_attention": (I32, [I32, I32, I32, I32, I32, I32, I32, P, P, P, P, P, P, F32, U64, U64, I32, P, P]),
+    "gpt_test_attention": (I32, [I32, I32, I32, I32, I32, I32, I32, P, P, P, P, P, P, P, F32, U64, U64, I32, P, P]),
     "gpt_test_wait_timeout": (I32, [U64, P, P, P]),
     "gpt_test_exp2": (I32, [P, P, P, I64, P]),
     "gpt_gemm_dw_accumulate_noalloc": (I32, [I32, I32, I32, P, I64, P, I64, P, I32, P]),
@@ -457,10 +457,10 @@ def test_gemm(backend, M, N, K, A, lda, a_kmajor, B, ldb, b_kmajor, epi_kind, ac
 
 
 def test_attention(backend, backward, dtype, B, T, H, hd, qkv, o, lse, dout=None, dqkv=None, dsum=None, p=0.0,
-                   seed=0, counter=0, layer=0, stream=None, flags=None):
+                   seed=0, counter=0, layer=0, stream=None, flags=None, colsum=None):
     return int(lib().gpt_test_attention(backend, backward, dtype, B, T, H, hd, _ptr(qkv), _ptr(o), _ptr(lse),
-                                        _ptr(dout), _ptr(dqkv), _ptr(dsum), p, seed, counter, layer, stream,
-                                        _ptr(flags)))
+                                        _ptr(dout), _ptr(dqkv), _ptr(dsum), _ptr(colsum), p, seed, counter, layer,
+                                        stream, _ptr(flags)))
 
 
 def test_wait_timeout(limit_ns: int, flags, gave_up, stream=None) -> int:

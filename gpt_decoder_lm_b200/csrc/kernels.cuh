@@ -132,6 +132,10 @@ struct AttnDesc {
   void* dqkv;         // bwd: [B, T, 3, H, hd]
   float* dsum;        // bwd scratch: rowsum(dO * O) [B, H, T]
   DropKey drop;       // site 1; elem = ((b*H + h)*T + i)*T + j
+  // wide backward kernels: column sums of the stored dqkv per 128-row block,
+  // colsum[m / 128][3 H hd] (= or += with colsum_acc); null: none
+  float* colsum = nullptr;
+  int colsum_acc = 0;
 };
 template <typename T> void attn_fwd_simt(Ctx& c, const AttnDesc& a);
 template <typename T> void attn_bwd_simt(Ctx& c, const AttnDesc& a);

@@ -63,14 +63,17 @@ extern "C" gpt_status gpt_test_gemm(int32_t backend, int32_t M, int32_t N, int32
 
 extern "C" gpt_status gpt_test_attention(int32_t backend, int32_t backward, int32_t dtype, int32_t B, int32_t T,
                                          int32_t H, int32_t hd, const void* qkv, void* o, float* lse,
-                                         const void* dout, void* dqkv, float* dsum, float p, uint64_t seed,
-                                         uint64_t counter, int32_t layer, void* stream, uint32_t* d_flags) {
+                                         const void* dout, void* dqkv, float* dsum, float* colsum, float p,
+                                         uint64_t seed, uint64_t counter, int32_t layer, void* stream,
+                                         uint32_t* d_flags) {
   if (B <= 0 || T <= 0 || H <= 0 || !qkv || !o || !lse) return GPT_ERR_INVALID_ARG;
   if (backward && (!dout || !dqkv || !dsum)) return GPT_ERR_INVALID_ARG;
   Ctx c;
   c.stream = (cudaStream_t)stream;
   c.flags = d_flags;
   AttnDesc a{B, T, H, hd, qkv, o, lse, dout, dqkv, dsum, make_drop_key(seed, counter, layer, 1, p)};
+  if (colsum && !(backward && backend == 3)) return GPT_ERR_INVALID_ARG;
+  a.colsum = colsum;
   if (backend >= 1 && backend <= 3) {
     if (dtype != 1 || !attn_tc_supported(a)) return GPT_ERR_UNSUPPORTED;
     const bool ok = backward ? (backend == 3 ? attn_bwd_tc_wide(c, a) : attn_bwd_tc(c, a))

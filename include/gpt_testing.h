@@ -56,12 +56,14 @@ gpt_status gpt_test_gemm(int32_t backend, int32_t M, int32_t N, int32_t K, const
  * 1 bf16.  backend: 0 CUDA cores, 1 tensor cores, 2 tensor cores with the
  * two-tile (ping-pong) forward kernel, 3 the ping-pong forward and the
  * backward kernels with 128-wide inner blocks (GPT_ERR_UNSUPPORTED when the
- * shape is not supported).  Dropout on the probabilities with
+ * shape is not supported).  colsum (nullable; backward of backend 3 only):
+ * fp32 [B T / 128, 3 H hd] receives the column sums of the stored dqkv over
+ * each 128-row block.  Dropout on the probabilities with
  * (p, seed, counter, layer) as in the model (site 1); p = 0 disables it. */
 gpt_status gpt_test_attention(int32_t backend, int32_t backward, int32_t dtype, int32_t B, int32_t T, int32_t H,
                               int32_t hd, const void* qkv, void* o, float* lse, const void* dout, void* dqkv,
-                              float* dsum, float p, uint64_t seed, uint64_t counter, int32_t layer, void* stream,
-                              uint32_t* d_flags);
+                              float* dsum, float* colsum, float p, uint64_t seed, uint64_t counter, int32_t layer,
+                              void* stream, uint32_t* d_flags);
 
 /* The bounded device-side wait of the tensor-core kernels, made to run out:
  * one warp waits on an mbarrier that nothing arrives at, with a limit of

@@ -56,9 +56,17 @@ def run_case(backend, B, T, H, p, seed=0, qkv_np=None):
     rc = gb.test_attention(backend, 0, 1, B, T, H, hd, d_qkv, d_o, d_lse, p=p, seed=SEED, counter=COUNTER,
                            layer=LAYER, stream=st, flags=flags)
     assert gb.STATUS[rc] == "GPT_OK", gb.STATUS[rc]
+    # the wide backward also writes the column sums of the stored dqkv per
+    # 128-row block (the qkv bias gradient's partials)
+    cs = torch.full((B * T // 128, 3 * H * hd), float("nan"), device="cuda") if backend == 3 else None
     rc = gb.test_attention(backend, 1, 1, B, T, H, hd, d_qkv, d_o, d_lse, d_do, d_dqkv, d_dsum, p=p, seed=SEED,
-                           counter=COUNTER, layer=LAYER, stream=st, flags=flags)
+                           counter=COUNTER, layer=LAYER, stream=st, flags=flags, colsum=cs)
     assert gb.STATUS[rc] == "GPT_OK", gb.STATUS[rc]
+    if cs is not None:
+        stored = d_dqkv.double().cpu().numpy().reshape(B * T // 128, 128, 3 * H * hd).sum(axis=1)
+        got = cs.double().cpu().numpy()
+        assert np.isfinite(got).all()
+        assert np.abs(got - stored).max() <= 1e-5 * max(1.0, np.abs(stored).max())
     assert int(flags.item()) == 0
     o = d_o.float().cpu().numpy().astype(np.float64).transpose(0, 2, 1, 3)
     assert rel_l2(o, o_ref) < 2e-2
