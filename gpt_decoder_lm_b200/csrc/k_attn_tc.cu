@@ -475,11 +475,12 @@ __global__ void __launch_bounds__(320, 1) k_attn_fwd_pp(const __grid_constant__ 
       tc_fence_after();
       const bool diag = j == jl;  // key j*128 + i is visible iff i <= r
       // row maximum, 64 columns at a time (the register budget of ten warps
-      // is 168 per thread); the second half stays in registers for the exps
+      // is 168 per thread), keys 64..127 first, so that keys 0..63 stay in
+      // registers for the exps
       uint32_t va[32], vb[32];
       float mx0 = -INFINITY, mx1 = -INFINITY;
 #pragma unroll
-      for (int hh = 0; hh < 2; hh++) {
+      for (int hh = 1; hh >= 0; hh--) {
         tmem_ld_32x32b_x32(trow + s_col + 64 * hh, va);
         tmem_ld_32x32b_x32(trow + s_col + 64 * hh + 32, vb);
         tmem_ld_wait();
@@ -519,14 +520,16 @@ __global__ void __launch_bounds__(320, 1) k_attn_fwd_pp(const __grid_constant__ 
         }
       }
       // probabilities of the 128 keys, packed bf16 pairs (P = the A operand of
-      // P V), the half of keys 64..127 (still in registers) first
+      // P V): keys 0..63 (in registers) go to columns 0..31, whose S they
+      // replace; then keys 64..127, re-read from their untouched columns, go
+      // to columns 32..63 (the S of keys 32..63, consumed by then)
       const uint64_t neg_m = f2c(-m), scl = f2c(sl2);
       float lsum = 0.f;
 #pragma unroll
-      for (int hi = 1; hi >= 0; hi--) {
-        if (hi == 0) {
-          tmem_ld_32x32b_x32(trow + s_col, va);
-          tmem_ld_32x32b_x32(trow + s_col + 32, vb);
+      for (int hi = 0; hi < 2; hi++) {
+        if (hi == 1) {
+          tmem_ld_32x32b_x32(trow + s_col + 64, va);
+          tmem_ld_32x32b_x32(trow + s_col + 96, vb);
           tmem_ld_wait();
         }
         uint32_t pk[32];
@@ -605,8 +608,9 @@ __device__ __forceinline__ uint32_t pack2v(uint64_t v) {
 
 constexpr int BWD_STAGES = 3;  // Q/dO (or K/V) tiles in flight
 // one probability pair in every BWD_POLY_EVERY is computed on the FMA pipe
-// (exp2_poly2) instead of the SFU
-constexpr int BWD_POLY_EVERY = 2;
+// (exp2_poly2) instead of the SFU; 0: none.  The backward kernels are issue-
+// rather than SFU-bound (half on the FMA pipe measured 10% slower), so none.
+constexpr int BWD_POLY_EVERY = 0;
 
 // ============================================================================
 // backward, dK and dV: one CTA per (128-key block, b, h), walking 64-query
@@ -776,7 +780,7 @@ __global__ void __launch_bounds__(320, 2) k_attn_bwd_kv8(const __grid_constant__
           const float2 y23 = f2split(f2fma(f2(__uint_as_float(sv[e + 2]), __uint_as_float(sv[e + 3])), sl2x2,
                                            f2mul(f2(l4.z, l4.w), nlog2e)));
           float p4[4];
-          if (((e >> 1) % BWD_POLY_EVERY) == BWD_POLY_EVERY - 1) {
+          if (BWD_POLY_EVERY > 0 && ((e >> 1) % (BWD_POLY_EVERY > 0 ? BWD_POLY_EVERY : 1)) == BWD_POLY_EVERY - 1) {
             const float2 q01 = f2split(exp2_poly2(f2(y01.x, y01.y)));
             p4[0] = q01.x;
             p4[1] = q01.y;
@@ -784,7 +788,7 @@ __global__ void __launch_bounds__(320, 2) k_attn_bwd_kv8(const __grid_constant__
             p4[0] = ex2(y01.x);
             p4[1] = ex2(y01.y);
           }
-          if ((((e >> 1) + 1) % BWD_POLY_EVERY) == BWD_POLY_EVERY - 1) {
+          if (BWD_POLY_EVERY > 0 && (((e >> 1) + 1) % (BWD_POLY_EVERY > 0 ? BWD_POLY_EVERY : 1)) == BWD_POLY_EVERY - 1) {
             const float2 q23 = f2split(exp2_poly2(f2(y23.x, y23.y)));
             p4[2] = q23.x;
             p4[3] = q23.y;
@@ -1031,7 +1035,7 @@ __global__ void __launch_bounds__(320, 2) k_attn_bwd_q8(const __grid_constant__ 
         for (int e = 0; e < 16; e += 2) {
           const uint64_t y2 = f2fma(f2(__uint_as_float(sv[e]), __uint_as_float(sv[e + 1])), sl2x2, nlse2);
           float e0, e1;
-          if (((e >> 1) % BWD_POLY_EVERY) == BWD_POLY_EVERY - 1) {
+          if (BWD_POLY_EVERY > 0 && ((e >> 1) % (BWD_POLY_EVERY > 0 ? BWD_POLY_EVERY : 1)) == BWD_POLY_EVERY - 1) {
             const float2 q = f2split(exp2_poly2(y2));
             e0 = q.x;
             e1 = q.y;
@@ -1297,7 +1301,7 @@ __global__ void __launch_bounds__(320, 1) k_attn_bwd_kvw(const __grid_constant__
           const uint64_t y23 = f2fma(f2(__uint_as_float(sv[e + 2]), __uint_as_float(sv[e + 3])), sl2x2,
                                      f2mul(f2(l4.z, l4.w), nlog2e));
           float p4[4];
-          if (((e >> 1) % BWD_POLY_EVERY) == BWD_POLY_EVERY - 1) {
+          if (BWD_POLY_EVERY > 0 && ((e >> 1) % (BWD_POLY_EVERY > 0 ? BWD_POLY_EVERY : 1)) == BWD_POLY_EVERY - 1) {
             const float2 q01 = f2split(exp2_poly2(y01));
             p4[0] = q01.x;
             p4[1] = q01.y;
@@ -1306,7 +1310,7 @@ __global__ void __launch_bounds__(320, 1) k_attn_bwd_kvw(const __grid_constant__
             p4[0] = ex2(x01.x);
             p4[1] = ex2(x01.y);
           }
-          if ((((e >> 1) + 1) % BWD_POLY_EVERY) == BWD_POLY_EVERY - 1) {
+          if (BWD_POLY_EVERY > 0 && (((e >> 1) + 1) % (BWD_POLY_EVERY > 0 ? BWD_POLY_EVERY : 1)) == BWD_POLY_EVERY - 1) {
             const float2 q23 = f2split(exp2_poly2(y23));
             p4[2] = q23.x;
             p4[3] = q23.y;
@@ -1567,7 +1571,7 @@ __global__ void __launch_bounds__(320, 1) k_attn_bwd_qw(const __grid_constant__ 
         for (int e = 0; e < 16; e += 2) {
           const uint64_t y2 = f2fma(f2(__uint_as_float(sv[e]), __uint_as_float(sv[e + 1])), sl2x2, nlse2);
           float e0, e1;
-          if (((e >> 1) % BWD_POLY_EVERY) == BWD_POLY_EVERY - 1) {
+          if (BWD_POLY_EVERY > 0 && ((e >> 1) % (BWD_POLY_EVERY > 0 ? BWD_POLY_EVERY : 1)) == BWD_POLY_EVERY - 1) {
             const float2 q = f2split(exp2_poly2(y2));
             e0 = q.x;
             e1 = q.y;
