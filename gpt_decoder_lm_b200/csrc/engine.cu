@@ -878,9 +878,20 @@ gpt_status backward_t(gpt_model* m) {
     g.epi.ldo = d;
     if (!gemm(m, g)) return fail(m, GPT_ERR_CUDA, "attn proj dX failed");
     AttnDesc ad{m->B, m->T, m->H, m->hd, qkv, o, m->lse + (size_t)l * M * m->H, datt, dqkv, m->dsum, dkey(m, l, 1)};
+    // tensor-core attention: the qkv bias gradient's column sums of dqkv come
+    // from the backward kernels' epilogues (one partial row per 128-row block)
+    const bool fused_qkv_colsum = m->attn_tc && y.qkv_b >= 0 && !frozen;
+    if (fused_qkv_colsum) {
+      ad.colsum = colsum_part(l, 1);
+      ad.colsum_acc = first ? 0 : 1;
+    }
     const gpt_status as = attention<T>(m, ad, true);
     if (as != GPT_OK) return as;
-    if (y.qkv_b >= 0) bias_grad(dqkv, 3 * d, l, 1, m->G(y.qkv_b));
+    if (fused_qkv_colsum) {
+      if (last) colsum_reduce(c, colsum_part(l, 1), (int)(M / 128), 3 * d, m->G(y.qkv_b));
+    } else if (y.qkv_b >= 0) {
+      bias_grad(dqkv, 3 * d, l, 1, m->G(y.qkv_b));
+    }
     if (!dW(3 * d, d, dqkv, a1, m->G(y.qkv_w), "gemm_qkv_dw", l * 4 + 3))
       return fail(m, GPT_ERR_CUDA, "qkv dW failed");
     if (frozen) {

@@ -606,6 +606,41 @@ __device__ __forceinline__ uint32_t pack2v(uint64_t v) {
   return pack2(f.x, f.y);
 }
 
+// Column sums of a warp's 32 rows (one per lane) x 32 columns (v[c] in lane
+// order): a butterfly in which each step hands half of a lane's columns to its
+// partner, so lane c ends with the sum of column c (31 shuffles, fixed order).
+__device__ __forceinline__ float warp_colsum32(float (&v)[32], int lane) {
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) {
+    const bool upper = (lane & o) != 0;
+#pragma unroll
+    for (int i = 0; i < o; i++) {
+      const float send = upper ? v[i] : v[i + o];
+      const float keep = upper ? v[i + o] : v[i];
+      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+    }
+  }
+  return v[0];
+}
+
+// The 128-row block's column sums of 32 columns held by the four lane-quadrant
+// warps of one half (sum_q: this warp's column sums, lane c for column c):
+// combined in quadrant order through shared memory by the quadrant-0 warp,
+// which writes (or adds to) colsum[blk][col0 + c].  All eight math warps
+// must call it (named barrier 1).
+__device__ __forceinline__ void block_colsum(float* s_red, int half, int quad, int lane, float sum_q, float* colsum,
+                                             size_t blk, long ld, long col0, int acc) {
+  s_red[(half * 4 + quad) * 32 + lane] = sum_q;
+  asm volatile("bar.sync 1, 256;" ::: "memory");
+  if (quad == 0) {
+    const float t = ((s_red[(half * 4 + 0) * 32 + lane] + s_red[(half * 4 + 1) * 32 + lane]) +
+                     s_red[(half * 4 + 2) * 32 + lane]) + s_red[(half * 4 + 3) * 32 + lane];
+    float* dst = colsum + blk * ld + col0 + lane;
+    *dst = acc ? *dst + t : t;
+  }
+  asm volatile("bar.sync 1, 256;" ::: "memory");
+}
+
 constexpr int BWD_STAGES = 3;  // Q/dO (or K/V) tiles in flight
 // one probability pair in every BWD_POLY_EVERY is computed on the FMA pipe
 // (exp2_poly2) instead of the SFU; 0: none.  The backward kernels are issue-
@@ -630,7 +665,8 @@ constexpr int BWD_POLY_EVERY = 0;
 // TMEM: S^T [0,64), dP^T [64,128), dV [128,192), dK [192,256)
 // ============================================================================
 constexpr int K_K = 0, K_V = TILE, K_ST = 2 * TILE, K_LD = (2 + BWD_STAGES) * TILE, K_BAR = K_LD + 2048;
-constexpr int K_SMEM = K_BAR + 128;
+constexpr int K_RED = K_BAR + 128;  // [2 halves][4 quadrants][32] column partials
+constexpr int K_SMEM = K_RED + 1024;
 
 template <bool DROP>
 __global__ void __launch_bounds__(320, 2) k_attn_bwd_kv8(const __grid_constant__ CUtensorMap tkv,
@@ -842,23 +878,44 @@ __global__ void __launch_bounds__(320, 2) k_attn_bwd_kv8(const __grid_constant__
       __syncwarp();
       if (lane == 0) mbar_arrive(ds_ready);
     }
-    if (ok && mbar_wait(acc_full, 0, abort_flag, a.flags)) {
+    const bool done = ok && mbar_wait(acc_full, 0, abort_flag, a.flags);
+    if (done) {
       tc_fence_after();
       bf16* rowp = a.dqkv + (size_t)(row0 + kj) * (3 * a.H * 64);
       // half 0: dV at slot 2H+h; half 1: dK (times 1/sqrt(hd)) at slot H+h
       const float f = half == 0 ? 1.0f : a.scale;
-      uint4* dst = reinterpret_cast<uint4*>(rowp + (size_t)((half == 0 ? 2 : 1) * a.H + h) * 64);
+      const int slot = (half == 0 ? 2 : 1) * a.H + h;
+      uint4* dst = reinterpret_cast<uint4*>(rowp + (size_t)slot * 64);
 #pragma unroll
-      for (int c = 0; c < 4; c++) {
-        uint32_t v[16];
-        tmem_ld_32x32b_x16(trow + 128 + half * 64 + c * 16, v);
-        tmem_ld_wait();
-        const float* x = reinterpret_cast<const float*>(v);
-        dst[2 * c] = make_uint4(pack2(x[0] * f, x[1] * f), pack2(x[2] * f, x[3] * f), pack2(x[4] * f, x[5] * f),
-                                pack2(x[6] * f, x[7] * f));
-        dst[2 * c + 1] = make_uint4(pack2(x[8] * f, x[9] * f), pack2(x[10] * f, x[11] * f),
-                                    pack2(x[12] * f, x[13] * f), pack2(x[14] * f, x[15] * f));
+      for (int c2 = 0; c2 < 2; c2++) {  // 32 columns at a time: stored, then their block column sums
+        float cs[32];
+#pragma unroll
+        for (int c1 = 0; c1 < 2; c1++) {
+          const int c = 2 * c2 + c1;
+          uint32_t v[16];
+          tmem_ld_32x32b_x16(trow + 128 + half * 64 + c * 16, v);
+          tmem_ld_wait();
+          const float* x = reinterpret_cast<const float*>(v);
+          uint32_t w[8];
+#pragma unroll
+          for (int k = 0; k < 8; k++) {
+            w[k] = pack2(x[2 * k] * f, x[2 * k + 1] * f);
+            const float2 bk = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[k]));
+            cs[16 * c1 + 2 * k] = bk.x;  // the stored (bf16) values
+            cs[16 * c1 + 2 * k + 1] = bk.y;
+          }
+          dst[2 * c] = make_uint4(w[0], w[1], w[2], w[3]);
+          dst[2 * c + 1] = make_uint4(w[4], w[5], w[6], w[7]);
+        }
+        if (a.colsum) {
+          const float sq = warp_colsum32(cs, lane);
+          block_colsum(reinterpret_cast<float*>(smem + K_RED), half, quad, lane, sq, a.colsum,
+                       (size_t)(row0 + kb * 128) / 128, 3L * a.H * 64, (long)slot * 64 + 32 * c2, a.colsum_acc);
+        }
       }
+    } else if (a.colsum) {
+      // every math warp takes part in the column-sum barriers, even on a failed wait
+      for (int c2 = 0; c2 < 4; c2++) asm volatile("bar.sync 1, 256;" ::: "memory");
     }
   }
   tc_fence_before();
@@ -881,7 +938,8 @@ __global__ void __launch_bounds__(320, 2) k_attn_bwd_kv8(const __grid_constant__
 // TMEM: S [0,64), dP [64,128), dQ [128,192)  (256 allocated)
 // ============================================================================
 constexpr int Q_Q = 0, Q_DO = TILE, Q_OT = 2 * TILE, Q_ST = 3 * TILE, Q_BAR = (3 + BWD_STAGES) * TILE;
-constexpr int Q_SMEM = Q_BAR + 128;
+constexpr int Q_RED = Q_BAR + 128;
+constexpr int Q_SMEM = Q_RED + 1024;
 
 template <bool DROP>
 __global__ void __launch_bounds__(320, 2) k_attn_bwd_q8(const __grid_constant__ CUtensorMap tq,
@@ -1077,21 +1135,37 @@ __global__ void __launch_bounds__(320, 2) k_attn_bwd_q8(const __grid_constant__ 
       __syncwarp();
       if (lane == 0) mbar_arrive(ds_ready);
     }
-    if (ok && mbar_wait(acc_full, 0, abort_flag, a.flags)) {
+    const bool done = ok && mbar_wait(acc_full, 0, abort_flag, a.flags);
+    if (done) {
       tc_fence_after();
       uint4* dst = reinterpret_cast<uint4*>(a.dqkv + (size_t)(row0 + qi) * (3 * a.H * 64) + (size_t)h * 64 + half * 32);
       const float f = a.scale;
+      float cs[32];
 #pragma unroll
       for (int c = 0; c < 2; c++) {
         uint32_t v[16];
         tmem_ld_32x32b_x16(trow + 128 + half * 32 + c * 16, v);
         tmem_ld_wait();
         const float* x = reinterpret_cast<const float*>(v);
-        dst[2 * c] = make_uint4(pack2(x[0] * f, x[1] * f), pack2(x[2] * f, x[3] * f), pack2(x[4] * f, x[5] * f),
-                                pack2(x[6] * f, x[7] * f));
-        dst[2 * c + 1] = make_uint4(pack2(x[8] * f, x[9] * f), pack2(x[10] * f, x[11] * f),
-                                    pack2(x[12] * f, x[13] * f), pack2(x[14] * f, x[15] * f));
+        uint32_t w[8];
+#pragma unroll
+        for (int k = 0; k < 8; k++) {
+          w[k] = pack2(x[2 * k] * f, x[2 * k + 1] * f);
+          const float2 bk = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[k]));
+          cs[16 * c + 2 * k] = bk.x;  // the stored (bf16) values
+          cs[16 * c + 2 * k + 1] = bk.y;
+        }
+        dst[2 * c] = make_uint4(w[0], w[1], w[2], w[3]);
+        dst[2 * c + 1] = make_uint4(w[4], w[5], w[6], w[7]);
       }
+      if (a.colsum) {
+        const float sq = warp_colsum32(cs, lane);
+        block_colsum(reinterpret_cast<float*>(smem + Q_RED), half, quad, lane, sq, a.colsum,
+                     (size_t)(row0 + qb * 128) / 128, 3L * a.H * 64, (long)h * 64 + 32 * half, a.colsum_acc);
+      }
+    } else if (a.colsum) {
+      // every math warp takes part in the column-sum barriers, even on a failed wait
+      for (int c2 = 0; c2 < 2; c2++) asm volatile("bar.sync 1, 256;" ::: "memory");
     }
   }
   tc_fence_before();
@@ -1111,41 +1185,6 @@ __global__ void __launch_bounds__(320, 2) k_attn_bwd_q8(const __grid_constant__ 
 // TMEM A-operand column of K-step kk (16 elements) of a 128-wide block whose
 // halves pack into their own first 32 columns
 __device__ __forceinline__ uint32_t acolw(int kk) { return (uint32_t)((kk >> 2) * 64 + (kk & 3) * 8); }
-
-// Column sums of a warp's 32 rows (one per lane) x 32 columns (v[c] in lane
-// order): a butterfly in which each step hands half of a lane's columns to its
-// partner, so lane c ends with the sum of column c (31 shuffles, fixed order).
-__device__ __forceinline__ float warp_colsum32(float (&v)[32], int lane) {
-#pragma unroll
-  for (int o = 16; o >= 1; o >>= 1) {
-    const bool upper = (lane & o) != 0;
-#pragma unroll
-    for (int i = 0; i < o; i++) {
-      const float send = upper ? v[i] : v[i + o];
-      const float keep = upper ? v[i + o] : v[i];
-      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
-    }
-  }
-  return v[0];
-}
-
-// The 128-row block's column sums of 32 columns held by the four lane-quadrant
-// warps of one half (sum_q: this warp's column sums, lane c for column c):
-// combined in quadrant order through shared memory by the quadrant-0 warp,
-// which writes (or adds to) colsum[blk][col0 + c].  All eight math warps
-// must call it (named barrier 1).
-__device__ __forceinline__ void block_colsum(float* s_red, int half, int quad, int lane, float sum_q, float* colsum,
-                                             size_t blk, long ld, long col0, int acc) {
-  s_red[(half * 4 + quad) * 32 + lane] = sum_q;
-  asm volatile("bar.sync 1, 256;" ::: "memory");
-  if (quad == 0) {
-    const float t = ((s_red[(half * 4 + 0) * 32 + lane] + s_red[(half * 4 + 1) * 32 + lane]) +
-                     s_red[(half * 4 + 2) * 32 + lane]) + s_red[(half * 4 + 3) * 32 + lane];
-    float* dst = colsum + blk * ld + col0 + lane;
-    *dst = acc ? *dst + t : t;
-  }
-  asm volatile("bar.sync 1, 256;" ::: "memory");
-}
 
 constexpr int KW_K = 0, KW_V = TILE, KW_ST = 2 * TILE, KW_LD = (2 + 2 * BWD_STAGES) * TILE;
 constexpr int KW_BAR = KW_LD + 1024 * BWD_STAGES;

@@ -72,7 +72,7 @@ extern "C" gpt_status gpt_test_attention(int32_t backend, int32_t backward, int3
   c.stream = (cudaStream_t)stream;
   c.flags = d_flags;
   AttnDesc a{B, T, H, hd, qkv, o, lse, dout, dqkv, dsum, make_drop_key(seed, counter, layer, 1, p)};
-  if (colsum && !(backward && backend == 3)) return GPT_ERR_INVALID_ARG;
+  if (colsum && !(backward && (backend == 1 || backend == 3))) return GPT_ERR_INVALID_ARG;
   a.colsum = colsum;
   if (backend >= 1 && backend <= 3) {
     if (dtype != 1 || !attn_tc_supported(a)) return GPT_ERR_UNSUPPORTED;

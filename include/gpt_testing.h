@@ -56,7 +56,7 @@ gpt_status gpt_test_gemm(int32_t backend, int32_t M, int32_t N, int32_t K, const
  * 1 bf16.  backend: 0 CUDA cores, 1 tensor cores, 2 tensor cores with the
  * two-tile (ping-pong) forward kernel, 3 the ping-pong forward and the
  * backward kernels with 128-wide inner blocks (GPT_ERR_UNSUPPORTED when the
- * shape is not supported).  colsum (nullable; backward of backend 3 only):
+ * shape is not supported).  colsum (nullable; backward of backends 1, 3):
  * fp32 [B T / 128, 3 H hd] receives the column sums of the stored dqkv over
  * each 128-row block.  Dropout on the probabilities with
  * (p, seed, counter, layer) as in the model (site 1); p = 0 disables it. */

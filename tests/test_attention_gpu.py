@@ -56,9 +56,9 @@ def run_case(backend, B, T, H, p, seed=0, qkv_np=None):
     rc = gb.test_attention(backend, 0, 1, B, T, H, hd, d_qkv, d_o, d_lse, p=p, seed=SEED, counter=COUNTER,
                            layer=LAYER, stream=st, flags=flags)
     assert gb.STATUS[rc] == "GPT_OK", gb.STATUS[rc]
-    # the wide backward also writes the column sums of the stored dqkv per
-    # 128-row block (the qkv bias gradient's partials)
-    cs = torch.full((B * T // 128, 3 * H * hd), float("nan"), device="cuda") if backend == 3 else None
+    # the tensor-core backward also writes the column sums of the stored dqkv
+    # per 128-row block (the qkv bias gradient's partials)
+    cs = torch.full((B * T // 128, 3 * H * hd), float("nan"), device="cuda") if backend in (1, 3) else None
     rc = gb.test_attention(backend, 1, 1, B, T, H, hd, d_qkv, d_o, d_lse, d_do, d_dqkv, d_dsum, p=p, seed=SEED,
                            counter=COUNTER, layer=LAYER, stream=st, flags=flags, colsum=cs)
     assert gb.STATUS[rc] == "GPT_OK", gb.STATUS[rc]
