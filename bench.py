@@ -593,8 +593,8 @@ def run_ours(args, w, rank, world, local_rank):
 def run_kernels(w):
     """One launch of each hot kernel at the workload's micro-batch shapes through
     the kernel-level test entry points (the small case for ncu captures): the
-    GEMMs with the kernel and split the step's cost model picks, both
-    tensor-core attention forwards and the attention backward."""
+    GEMMs with the kernel and split the step's cost model picks, the
+    tensor-core attention forward and backward."""
     import torch
 
     from gpt_decoder_lm_b200 import binding as gb
@@ -626,7 +626,6 @@ def run_kernels(w):
     lse = torch.empty(B, H, T, device="cuda")
     do, dq, ds = bf(B, T, H, 64), torch.empty_like(q), torch.empty_like(lse)
     assert gb.test_attention(1, 0, 1, B, T, H, 64, q, o, lse, stream=st, flags=flags) == 0
-    assert gb.test_attention(2, 0, 1, B, T, H, 64, q, o, lse, stream=st, flags=flags) == 0
     assert gb.test_attention(1, 1, 1, B, T, H, 64, q, o, lse, do, dq, ds, stream=st, flags=flags) == 0
     torch.cuda.synchronize()
     assert int(flags.item()) == 0

@@ -105,7 +105,6 @@ _PROTOS = {
                             P, P, P]),
     "gpt_test_attention": (I32, [I32, I32, I32, I32, I32, I32, I32, P, P, P, P, P, P, P, F32, U64, U64, I32, P, P]),
     "gpt_test_wait_timeout": (I32, [U64, P, P, P]),
-    "gpt_test_exp2": (I32, [P, P, P, I64, P]),
     "gpt_gemm_dw_accumulate_noalloc": (I32, [I32, I32, I32, P, I64, P, I64, P, I32, P]),
 }
 
@@ -467,8 +466,3 @@ def test_wait_timeout(limit_ns: int, flags, gave_up, stream=None) -> int:
     """The kernels' bounded mbarrier wait with a short limit, on a barrier
     nothing arrives at; returns the status code."""
     return int(lib().gpt_test_wait_timeout(limit_ns, stream, _ptr(flags), _ptr(gave_up)))
-
-
-def test_exp2(x, y_poly, y_ref, stream=None) -> int:
-    """Device polynomial 2^x and CUDA's exp2f on the same arguments."""
-    return int(lib().gpt_test_exp2(_ptr(x), _ptr(y_poly), _ptr(y_ref), x.numel(), stream))

@@ -186,32 +186,6 @@ __device__ __forceinline__ uint64_t f2sub(uint64_t a, uint64_t b) {
 }
 __device__ __forceinline__ uint64_t f2c(float c) { return f2(c, c); }
 
-// 2^x for a pair of arguments on the FMA pipe (f32x2), without the SFU:
-// Cody-Waite reduction x = n + f, n = round(x) (adding 1.5 * 2^23 leaves n in
-// the low mantissa bits), f in [-1/2, 1/2]; 2^f by the degree-4 Chebyshev
-// interpolant of 2^f on [-1/2, 1/2] (coefficients derived in exp2_poly.py,
-// relative error < 3.6e-6); 2^n added to the exponent field.  Arguments are
-// clamped to >= -125 (the exponent field stays >= 1; the result there is
-// ~2^-125 instead of the true value below it, which is just as negligible
-// next to a softmax maximum of 1).  For x <= 64.
-__device__ __forceinline__ uint64_t exp2_poly2(uint64_t x2) {
-  float2 x = f2split(x2);
-  x.x = fmaxf(x.x, -125.0f);
-  x.y = fmaxf(x.y, -125.0f);
-  const uint64_t magic = f2c(12582912.0f);
-  const uint64_t t = f2add(f2(x.x, x.y), magic);
-  const uint64_t f = f2sub(f2(x.x, x.y), f2sub(t, magic));
-  uint64_t p = f2fma(f2c(0.00966636836528778f), f, f2c(0.055921975523233414f));
-  p = f2fma(p, f, f2c(0.2402234971523285f));
-  p = f2fma(p, f, f2c(0.6931210160255432f));
-  p = f2fma(p, f, f2c(1.0f));
-  // n << 23 is the low 32-bit word of each lane of t shifted: the bits of
-  // 1.5 * 2^23 vanish under the shift
-  const uint32_t tl = (uint32_t)t, th = (uint32_t)(t >> 32);
-  const uint32_t pl = (uint32_t)p + (tl << 23), ph = (uint32_t)(p >> 32) + (th << 23);
-  return ((uint64_t)ph << 32) | pl;
-}
-
 // erf_as on a pair of arguments (same operations per lane as erf_as, the
 // polynomial and the affine steps on the f32x2 pipe).  Returns the pair of
 // erf values; e receives the pair e^{-z^2}.

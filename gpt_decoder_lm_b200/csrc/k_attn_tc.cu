@@ -44,7 +44,7 @@ struct AttnTcArgs {
   float scale;        // 1 / sqrt(64)
   DropKey drop;
   uint32_t* flags;
-  float* colsum;      // wide backward: column sums of dqkv per 128-row block (null: none)
+  float* colsum;      // backward: column sums of dqkv per 128-row block (null: none)
   int colsum_acc;
 };
 
@@ -311,290 +311,6 @@ __global__ void __launch_bounds__(192, 2) k_attn_fwd_o(const __grid_constant__ C
   if (warp == 1) tmem_dealloc(tmem, 256);
 }
 
-// ============================================================================
-// forward, ping-pong: one CTA per (pair of 128-query tiles, b, h), 128-key
-// blocks.  Two softmax warpgroups, one per query tile, alternate on the
-// tensor core: while warpgroup 0 turns S0 of key block j into P0, the MMA
-// warp runs P1 V of block j-1 and S1 of block j for warpgroup 1, and the
-// other way round, so the softmax arithmetic of one tile hides the MMAs of
-// the other.  A tile's S is single-buffered: S_t(j+1) is issued after
-// P_t(j) V (tcgen05 MMAs of one thread execute in issue order), which also
-// means O_t holds every P V product of the blocks before j, and none is in
-// flight, while warpgroup t works on block j, so it may rescale O_t in place.
-// One exponential pair in every F_POLY_EVERY is computed on the FMA pipe
-// (exp2_poly2) instead of the SFU, which otherwise bounds the softmax.
-// Tile 0 covers queries [256 p, 256 p + 128) and key blocks 0..2p; tile 1
-// (absent when T / 128 is odd and p is the last pair) queries
-// [256 p + 128, 256 p + 256) and key blocks 0..2p+1.
-// smem: Q0 | Q1 | (K, V)[3 stages] | barriers   (128 KB + 256 B)
-// TMEM: S0 [0,128), S1 [128,256), O0 [256,320), O1 [320,384)  (512 allocated)
-// ============================================================================
-constexpr int F_Q = 0, F_KV = 2 * TILE, F_BAR = 8 * TILE;
-constexpr int F_SMEM = F_BAR + 256;
-constexpr int F_STAGES = 3;
-constexpr int F_POLY_EVERY = 4;
-
-template <bool DROP>
-__global__ void __launch_bounds__(320, 1) k_attn_fwd_pp(const __grid_constant__ CUtensorMap t128, AttnTcArgs a) {
-  pdl_trigger();
-  const DropKey dk = DROP ? drop_live(a.drop) : a.drop;
-  extern __shared__ __align__(1024) uint8_t smem[];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if (smem_u32(smem) & 1023) {  // swizzled tiles need 1024-byte alignment
-    if (threadIdx.x == 0) atomicOr(a.flags, FLAG_TIMEOUT);
-    return;
-  }
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + F_BAR);
-  const uint32_t q_full = smem_u32(bars + 0);
-  const uint32_t kv_full0 = smem_u32(bars + 1), kv_empty0 = smem_u32(bars + 1 + F_STAGES);
-  const uint32_t s_full0 = smem_u32(bars + 1 + 2 * F_STAGES), p_full0 = s_full0 + 16, pv_done0 = s_full0 + 32;
-  uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + 7 + 2 * F_STAGES);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(tslot + 1);
-  const uint32_t sb = smem_u32(smem);
-
-  const int nqb = a.T / 128, npair = (nqb + 1) / 2;
-  const int p = npair - 1 - (int)blockIdx.y;  // longest pairs first
-  const int bh = blockIdx.x, b = bh / a.H, h = bh % a.H;
-  const bool has1 = 2 * p + 1 < nqb;
-  const int jl0 = 2 * p, jl1 = 2 * p + 1;    // last key block of each tile
-  const int nk = has1 ? jl1 + 1 : jl0 + 1;   // key blocks of the CTA
-  const int row0 = b * a.T;
-
-  if (threadIdx.x == 0) {
-    mbar_init(q_full, 1);
-    for (int s = 0; s < F_STAGES; s++) {
-      mbar_init(kv_full0 + 8 * s, 1);
-      mbar_init(kv_empty0 + 8 * s, 1);
-    }
-    for (int t = 0; t < 2; t++) {
-      mbar_init(s_full0 + 8 * t, 1);
-      mbar_init(p_full0 + 8 * t, 4);
-      mbar_init(pv_done0 + 8 * t, 1);
-    }
-    *abort_flag = 0;
-    fence_barrier_init();
-    prefetch_tmap(&t128);
-  }
-  if (warp == 1) {
-    tmem_alloc(smem_u32(tslot), 512);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tslot;
-
-  if (warp == 0) {
-    // ------------------------------------------------------------ TMA producer
-    if (lane == 0) {
-      mbar_expect_tx(q_full, (has1 ? 2 : 1) * TILE);
-      tma_load_3d(sb + F_Q, &t128, q_full, 0, h, row0 + 2 * p * 128);
-      if (has1) tma_load_3d(sb + F_Q + TILE, &t128, q_full, 0, h, row0 + (2 * p + 1) * 128);
-      int issued = 0;
-      bool ok = true;
-      for (int j = 0; j < nk; j++) {
-        const int s = j % F_STAGES;
-        const uint32_t fb = kv_full0 + 8 * s;
-        if (!(ok = mbar_wait(kv_empty0 + 8 * s, ((j / F_STAGES) & 1) ^ 1, abort_flag, a.flags))) break;
-        mbar_expect_tx(fb, 2 * TILE);
-        tma_load_3d(sb + F_KV + s * 2 * TILE, &t128, fb, 0, a.H + h, row0 + j * 128);
-        tma_load_3d(sb + F_KV + s * 2 * TILE + TILE, &t128, fb, 0, 2 * a.H + h, row0 + j * 128);
-        issued = j + 1;
-      }
-      if (!ok) {  // the loads already issued land before the CTA can exit
-        mbar_wait(q_full, 0, abort_flag, a.flags);
-        for (int j = issued - F_STAGES < 0 ? 0 : issued - F_STAGES; j < issued; j++)
-          mbar_wait(kv_full0 + 8 * (j % F_STAGES), (j / F_STAGES) & 1, abort_flag, a.flags);
-      }
-    }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t id_s = idesc_bf16_f32(128, 128, false, false);
-      constexpr uint32_t id_pv = idesc_bf16_f32(128, 64, false, true);
-      bool ok = mbar_wait(q_full, 0, abort_flag, a.flags);
-      // S_t(j) = Q_t K_j^T (M 128 queries, N 128 keys, K 64)
-      auto issue_s = [&](int t, int j) {
-        const uint32_t kt = sb + F_KV + (j % F_STAGES) * 2 * TILE;
-#pragma unroll
-        for (int kk = 0; kk < 4; kk++)
-          mma_bf16_ss(tmem + 128 * t, desc_k(sb + F_Q + t * TILE, TILE, kk), desc_k(kt, TILE, kk), id_s, kk > 0);
-        mma_commit(s_full0 + 8 * t);
-      };
-      // O_t += P_t(i) V_i: P over the first 64 columns of S_t (K = 128 keys), V MN-major (N = 64)
-      auto issue_pv = [&](int t, int i) -> bool {
-        if (!mbar_wait(p_full0 + 8 * t, i & 1, abort_flag, a.flags)) return false;
-        tc_fence_after();
-        const uint32_t v = sb + F_KV + (i % F_STAGES) * 2 * TILE + TILE;
-#pragma unroll
-        for (int kk = 0; kk < 8; kk++)
-          mma_bf16_ts(tmem + 256 + 64 * t, tmem + 128 * t + 8 * kk, desc_mn64(v, kk), id_pv,
-                      (i > 0 || kk > 0) ? 1u : 0u);
-        return true;
-      };
-      for (int j = 0; j < nk && ok; j++) {
-        const int s = j % F_STAGES;
-        if (!(ok = mbar_wait(kv_full0 + 8 * s, (j / F_STAGES) & 1, abort_flag, a.flags))) break;
-        tc_fence_after();
-        if (j <= jl0) {
-          if (j > 0 && !(ok = issue_pv(0, j - 1))) break;
-          issue_s(0, j);
-        } else if (j == jl0 + 1) {
-          if (!(ok = issue_pv(0, j - 1))) break;
-          mma_commit(pv_done0);
-        }
-        if (has1) {
-          if (j > 0 && !(ok = issue_pv(1, j - 1))) break;
-          if (j > 0) mma_commit(kv_empty0 + 8 * ((j - 1) % F_STAGES));
-          issue_s(1, j);
-        } else if (j > 0) {
-          mma_commit(kv_empty0 + 8 * ((j - 1) % F_STAGES));
-        }
-      }
-      if (ok) {
-        const int t = has1 ? 1 : 0;
-        if (issue_pv(t, nk - 1)) mma_commit(pv_done0 + 8 * t);
-      }
-    }
-  } else {
-    // ------------------------------------------------------------ softmax warpgroups
-    const int t = (warp - 2) >> 2;  // query tile
-    const int quad = warp & 3;
-    const int r = quad * 32 + lane;
-    const int qi = (2 * p + t) * 128 + r;
-    const bool live = t == 0 || has1;
-    const int jl = t == 0 ? jl0 : jl1;
-    const uint32_t trow = tmem + ((uint32_t)(quad * 32) << 16);
-    const uint32_t s_col = 128 * t, o_col = 256 + 64 * t;
-    const float sl2 = a.scale_log2;
-    float m = -INFINITY, l = 0.f;  // reference maximum (log2 units) and row sum against it
-    const uint64_t ebase = ((uint64_t)bh * a.T + qi) * a.T;
-    bool ok = live;
-    for (int j = 0; j <= jl && ok; j++) {
-      if (!(ok = mbar_wait(s_full0 + 8 * t, j & 1, abort_flag, a.flags))) break;
-      tc_fence_after();
-      const bool diag = j == jl;  // key j*128 + i is visible iff i <= r
-      // row maximum, 64 columns at a time (the register budget of ten warps
-      // is 168 per thread), keys 64..127 first, so that keys 0..63 stay in
-      // registers for the exps
-      uint32_t va[32], vb[32];
-      float mx0 = -INFINITY, mx1 = -INFINITY;
-#pragma unroll
-      for (int hh = 1; hh >= 0; hh--) {
-        tmem_ld_32x32b_x32(trow + s_col + 64 * hh, va);
-        tmem_ld_32x32b_x32(trow + s_col + 64 * hh + 32, vb);
-        tmem_ld_wait();
-        if (!diag) {
-#pragma unroll
-          for (int i = 0; i < 32; i++) {
-            mx0 = fmaxf(mx0, __uint_as_float(va[i]));
-            mx1 = fmaxf(mx1, __uint_as_float(vb[i]));
-          }
-        } else {
-#pragma unroll
-          for (int i = 0; i < 32; i++) {
-            if (64 * hh + i <= r) mx0 = fmaxf(mx0, __uint_as_float(va[i]));
-            if (64 * hh + i + 32 <= r) mx1 = fmaxf(mx1, __uint_as_float(vb[i]));
-          }
-        }
-      }
-      const float bm = fmaxf(mx0, mx1) * sl2;
-      if (j == 0) {
-        m = bm;  // key 0 is visible to every row, so m is finite from here on
-      } else {
-        const bool need = bm > m + RESCALE_LOG2;
-        if (__any_sync(0xffffffffu, need)) {
-          // O_t holds P V of blocks < j and nothing is in flight into it
-          const float sc = need ? ex2(m - bm) : 1.f;
-#pragma unroll
-          for (int q = 0; q < 4; q++) {  // 16 columns at a time: S stays in registers
-            uint32_t o[16];
-            tmem_ld_32x32b_x16(trow + o_col + 16 * q, o);
-            tmem_ld_wait();
-#pragma unroll
-            for (int i = 0; i < 16; i++) o[i] = __float_as_uint(__uint_as_float(o[i]) * sc);
-            tmem_st_32x32b_x16(trow + o_col + 16 * q, o);
-          }
-          l *= sc;
-          if (need) m = bm;
-        }
-      }
-      // probabilities of the 128 keys, packed bf16 pairs (P = the A operand of
-      // P V): keys 0..63 (in registers) go to columns 0..31, whose S they
-      // replace; then keys 64..127, re-read from their untouched columns, go
-      // to columns 32..63 (the S of keys 32..63, consumed by then)
-      const uint64_t neg_m = f2c(-m), scl = f2c(sl2);
-      float lsum = 0.f;
-#pragma unroll
-      for (int hi = 0; hi < 2; hi++) {
-        if (hi == 1) {
-          tmem_ld_32x32b_x32(trow + s_col + 64, va);
-          tmem_ld_32x32b_x32(trow + s_col + 96, vb);
-          tmem_ld_wait();
-        }
-        uint32_t pk[32];
-#pragma unroll
-        for (int cc = 0; cc < 2; cc++) {
-          const uint32_t* vc = cc == 0 ? va : vb;
-#pragma unroll
-          for (int i = 0; i < 32; i += 2) {
-            const int k = 64 * hi + 32 * cc + i;  // key offset in the block
-            const uint64_t x2 = f2fma(f2(__uint_as_float(vc[i]), __uint_as_float(vc[i + 1])), scl, neg_m);
-            float p0, p1;
-            if (((k >> 1) % F_POLY_EVERY) == F_POLY_EVERY - 1) {
-              const float2 e = f2split(exp2_poly2(x2));
-              p0 = e.x;
-              p1 = e.y;
-            } else {
-              const float2 x = f2split(x2);
-              p0 = ex2(x.x);
-              p1 = ex2(x.y);
-            }
-            if (diag) {
-              if (k > r) p0 = 0.f;
-              if (k + 1 > r) p1 = 0.f;
-            }
-            lsum += p0 + p1;
-            if (DROP) {
-              const uint64_t e = ebase + (uint64_t)j * 128 + k;
-              p0 *= drop_mul(dk, e);
-              p1 *= drop_mul(dk, e + 1);
-            }
-            pk[(32 * cc + i) >> 1] = pack2(p0, p1);
-          }
-        }
-        tmem_st_32x32b_x32(trow + s_col + 32 * hi, pk);
-      }
-      l += lsum;
-      tmem_st_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(p_full0 + 8 * t);  // one arrival per warp of the warpgroup
-    }
-    if (ok) ok = mbar_wait(pv_done0 + 8 * t, 0, abort_flag, a.flags);
-    if (ok) {
-      tc_fence_after();
-      uint32_t o0[32], o1[32];
-      ld64(trow + o_col, o0, o1);
-      const float inv = 1.0f / l;
-      uint4* dst = reinterpret_cast<uint4*>(a.o_out + ((size_t)(row0 + qi) * a.H + h) * 64);
-#pragma unroll
-      for (int q = 0; q < 8; q++) {
-        const uint32_t* x = q < 4 ? o0 + 8 * q : o1 + 8 * (q - 4);
-        dst[q] = make_uint4(pack2(__uint_as_float(x[0]) * inv, __uint_as_float(x[1]) * inv),
-                            pack2(__uint_as_float(x[2]) * inv, __uint_as_float(x[3]) * inv),
-                            pack2(__uint_as_float(x[4]) * inv, __uint_as_float(x[5]) * inv),
-                            pack2(__uint_as_float(x[6]) * inv, __uint_as_float(x[7]) * inv));
-      }
-      a.lse[(size_t)bh * a.T + qi] = (m + log2f(l)) * LN2;
-    }
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  if (warp == 1) tmem_dealloc(tmem, 512);
-}
-
 // packed bf16 pair column of element column c (0..63) of a 64-column block:
 // the half that owns c writes inside its own fp32 columns
 __device__ __forceinline__ int pcol(int c) { return (c & 32) + ((c & 31) >> 1); }
@@ -642,10 +358,6 @@ __device__ __forceinline__ void block_colsum(float* s_red, int half, int quad, i
 }
 
 constexpr int BWD_STAGES = 3;  // Q/dO (or K/V) tiles in flight
-// one probability pair in every BWD_POLY_EVERY is computed on the FMA pipe
-// (exp2_poly2) instead of the SFU; 0: none.  The backward kernels are issue-
-// rather than SFU-bound (half on the FMA pipe measured 10% slower), so none.
-constexpr int BWD_POLY_EVERY = 0;
 
 // ============================================================================
 // backward, dK and dV: one CTA per (128-key block, b, h), walking 64-query
@@ -815,23 +527,7 @@ __global__ void __launch_bounds__(320, 2) k_attn_bwd_kv8(const __grid_constant__
                                            f2mul(f2(l4.x, l4.y), nlog2e)));
           const float2 y23 = f2split(f2fma(f2(__uint_as_float(sv[e + 2]), __uint_as_float(sv[e + 3])), sl2x2,
                                            f2mul(f2(l4.z, l4.w), nlog2e)));
-          float p4[4];
-          if (BWD_POLY_EVERY > 0 && ((e >> 1) % (BWD_POLY_EVERY > 0 ? BWD_POLY_EVERY : 1)) == BWD_POLY_EVERY - 1) {
-            const float2 q01 = f2split(exp2_poly2(f2(y01.x, y01.y)));
-            p4[0] = q01.x;
-            p4[1] = q01.y;
-          } else {
-            p4[0] = ex2(y01.x);
-            p4[1] = ex2(y01.y);
-          }
-          if (BWD_POLY_EVERY > 0 && (((e >> 1) + 1) % (BWD_POLY_EVERY > 0 ? BWD_POLY_EVERY : 1)) == BWD_POLY_EVERY - 1) {
-            const float2 q23 = f2split(exp2_poly2(f2(y23.x, y23.y)));
-            p4[2] = q23.x;
-            p4[3] = q23.y;
-          } else {
-            p4[2] = ex2(y23.x);
-            p4[3] = ex2(y23.y);
-          }
+          float p4[4] = {ex2(y01.x), ex2(y01.y), ex2(y23.x), ex2(y23.y)};
 #pragma unroll
           for (int u = 0; u < 4; u++) {
             if (masked && c0 + e + u < lim) p4[u] = 0.f;
@@ -1091,19 +787,9 @@ __global__ void __launch_bounds__(320, 2) k_attn_bwd_q8(const __grid_constant__ 
         tmem_ld_wait();
 #pragma unroll
         for (int e = 0; e < 16; e += 2) {
-          const uint64_t y2 = f2fma(f2(__uint_as_float(sv[e]), __uint_as_float(sv[e + 1])), sl2x2, nlse2);
-          float e0, e1;
-          if (BWD_POLY_EVERY > 0 && ((e >> 1) % (BWD_POLY_EVERY > 0 ? BWD_POLY_EVERY : 1)) == BWD_POLY_EVERY - 1) {
-            const float2 q = f2split(exp2_poly2(y2));
-            e0 = q.x;
-            e1 = q.y;
-          } else {
-            const float2 y = f2split(y2);
-            e0 = ex2(y.x);
-            e1 = ex2(y.y);
-          }
-          pk[sub][e] = (masked && c0 + e > lim) ? 0.f : e0;
-          pk[sub][e + 1] = (masked && c0 + e + 1 > lim) ? 0.f : e1;
+          const float2 y = f2split(f2fma(f2(__uint_as_float(sv[e]), __uint_as_float(sv[e + 1])), sl2x2, nlse2));
+          pk[sub][e] = (masked && c0 + e > lim) ? 0.f : ex2(y.x);
+          pk[sub][e + 1] = (masked && c0 + e + 1 > lim) ? 0.f : ex2(y.y);
         }
       }
       tc_fence_before();
@@ -1172,523 +858,6 @@ __global__ void __launch_bounds__(320, 2) k_attn_bwd_q8(const __grid_constant__ 
   __syncthreads();
   tc_fence_after();
   if (warp == 1) tmem_dealloc(tmem, 256);
-}
-
-// ============================================================================
-// backward, wide: the dK/dV and dQ kernels with 128-wide inner blocks (N = 128
-// MMAs: half the MMA issues per FLOP of the 64-wide kernels), one CTA per SM
-// (TMEM: S 128 | dP 128 | accumulators).  Eight math warps, two per TMEM lane
-// quadrant, each taking 64 of the 128 columns; the same two math phases per
-// block and the same MMA issue order as the 64-wide kernels; the packed bf16
-// P~ / dS of a warp's 64 columns go into the first 32 of them (already read).
-// ============================================================================
-// TMEM A-operand column of K-step kk (16 elements) of a 128-wide block whose
-// halves pack into their own first 32 columns
-__device__ __forceinline__ uint32_t acolw(int kk) { return (uint32_t)((kk >> 2) * 64 + (kk & 3) * 8); }
-
-constexpr int KW_K = 0, KW_V = TILE, KW_ST = 2 * TILE, KW_LD = (2 + 2 * BWD_STAGES) * TILE;
-constexpr int KW_BAR = KW_LD + 1024 * BWD_STAGES;
-constexpr int KW_RED = KW_BAR + 128;   // [2 halves][4 quadrants][32] column partials
-constexpr int KW_SMEM = KW_RED + 1024;
-
-template <bool DROP>
-__global__ void __launch_bounds__(320, 1) k_attn_bwd_kvw(const __grid_constant__ CUtensorMap tkv,
-                                                         const __grid_constant__ CUtensorMap tdo, AttnTcArgs a) {
-  pdl_trigger();
-  const DropKey dk = DROP ? drop_live(a.drop) : a.drop;
-  extern __shared__ __align__(1024) uint8_t smem[];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if (smem_u32(smem) & 1023) {
-    if (threadIdx.x == 0) atomicOr(a.flags, FLAG_TIMEOUT);
-    return;
-  }
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + KW_BAR);
-  const uint32_t kv_full = smem_u32(bars + 0), st_full0 = smem_u32(bars + 1),
-                 st_empty0 = smem_u32(bars + 1 + BWD_STAGES);
-  const uint32_t s_full = smem_u32(bars + 1 + 2 * BWD_STAGES), dp_full = s_full + 8, p_ready = s_full + 16,
-                 ds_ready = s_full + 24, acc_full = s_full + 32;
-  uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + 6 + 2 * BWD_STAGES);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(tslot + 1);
-  const float* sld = reinterpret_cast<const float*>(smem + KW_LD);  // [stage][lse 128 | D 128]
-  const uint32_t sb = smem_u32(smem);
-
-  const int nqb = a.T / 128;
-  const int kb = (int)blockIdx.y;  // key block 0 (most query blocks) of every (b, h) first
-  const int bh = blockIdx.x, b = bh / a.H, h = bh % a.H;
-  const int row0 = b * a.T;
-  const int nit = nqb - kb;  // query blocks kb .. nqb-1
-
-  if (threadIdx.x == 0) {
-    mbar_init(kv_full, 1);
-    for (int s = 0; s < BWD_STAGES; s++) {
-      mbar_init(st_full0 + 8 * s, 1);
-      mbar_init(st_empty0 + 8 * s, 1);
-    }
-    mbar_init(s_full, 1);
-    mbar_init(dp_full, 1);
-    mbar_init(p_ready, 8);
-    mbar_init(ds_ready, 8);
-    mbar_init(acc_full, 1);
-    *abort_flag = 0;
-    fence_barrier_init();
-    prefetch_tmap(&tkv);
-    prefetch_tmap(&tdo);
-  }
-  if (warp == 1) {
-    tmem_alloc(smem_u32(tslot), 512);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tslot;
-
-  if (warp == 0) {
-    if (lane == 0) {
-      mbar_expect_tx(kv_full, 2 * TILE);
-      tma_load_3d(sb + KW_K, &tkv, kv_full, 0, a.H + h, row0 + kb * 128);
-      tma_load_3d(sb + KW_V, &tkv, kv_full, 0, 2 * a.H + h, row0 + kb * 128);
-      int issued = 0;
-      bool ok = true;
-      for (int it = 0; it < nit; it++) {
-        const int i = kb + it, s = it % BWD_STAGES;
-        const uint32_t fb = st_full0 + 8 * s;
-        if (!(ok = mbar_wait(st_empty0 + 8 * s, ((it / BWD_STAGES) & 1) ^ 1, abort_flag, a.flags))) break;
-        mbar_expect_tx(fb, 2 * TILE + 1024);
-        tma_load_3d(sb + KW_ST + s * 2 * TILE, &tkv, fb, 0, h, row0 + i * 128);
-        tma_load_3d(sb + KW_ST + s * 2 * TILE + TILE, &tdo, fb, 0, h, row0 + i * 128);
-        bulk_load(sb + KW_LD + s * 1024, a.lse + (size_t)bh * a.T + i * 128, 512, fb);
-        bulk_load(sb + KW_LD + s * 1024 + 512, a.dsum + (size_t)bh * a.T + i * 128, 512, fb);
-        issued = it + 1;
-      }
-      if (!ok) {  // the loads already issued land before the CTA can exit
-        mbar_wait(kv_full, 0, abort_flag, a.flags);
-        for (int it = issued - BWD_STAGES < 0 ? 0 : issued - BWD_STAGES; it < issued; it++)
-          mbar_wait(st_full0 + 8 * (it % BWD_STAGES), (it / BWD_STAGES) & 1, abort_flag, a.flags);
-      }
-    }
-  } else if (warp == 1) {
-    if (lane == 0) {
-      constexpr uint32_t id_s = idesc_bf16_f32(128, 128, false, false);
-      constexpr uint32_t id_acc = idesc_bf16_f32(128, 64, false, true);
-      auto q_of = [&](int it) { return sb + KW_ST + (it % BWD_STAGES) * 2 * TILE; };
-      auto issue_s = [&](int it) -> bool {  // S^T = K Q^T of block it
-        if (!mbar_wait(st_full0 + 8 * (it % BWD_STAGES), (it / BWD_STAGES) & 1, abort_flag, a.flags)) return false;
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < 4; kk++)
-          mma_bf16_ss(tmem, desc_k(sb + KW_K, TILE, kk), desc_k(q_of(it), TILE, kk), id_s, kk > 0);
-        mma_commit(s_full);
-        return true;
-      };
-      auto issue_dp = [&](int it) {  // dP^T = V dO^T of block it (its stage is loaded)
-#pragma unroll
-        for (int kk = 0; kk < 4; kk++)
-          mma_bf16_ss(tmem + 128, desc_k(sb + KW_V, TILE, kk), desc_k(q_of(it) + TILE, TILE, kk), id_s, kk > 0);
-        mma_commit(dp_full);
-      };
-      bool ok = mbar_wait(kv_full, 0, abort_flag, a.flags) && issue_s(0);
-      if (ok) issue_dp(0);
-      for (int it = 0; it < nit && ok; it++) {
-        const uint32_t q = q_of(it), dO = q + TILE;
-        if (!(ok = mbar_wait(p_ready, it & 1, abort_flag, a.flags))) break;
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < 8; kk++)  // dV += P~^T dO (K = the block's 128 queries)
-          mma_bf16_ts(tmem + 256, tmem + acolw(kk), desc_mn64(dO, kk), id_acc, (it > 0 || kk > 0));
-        if (it + 1 < nit && !(ok = issue_s(it + 1))) break;
-        if (!(ok = mbar_wait(ds_ready, it & 1, abort_flag, a.flags))) break;
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < 8; kk++)  // dK += dS^T Q
-          mma_bf16_ts(tmem + 320, tmem + 128 + acolw(kk), desc_mn64(q, kk), id_acc, (it > 0 || kk > 0));
-        mma_commit(st_empty0 + 8 * (it % BWD_STAGES));
-        if (it + 1 < nit) issue_dp(it + 1);
-      }
-      mma_commit(acc_full);
-    }
-  } else {
-    const int quad = warp & 3;
-    const int half = (warp - 2) >> 2;
-    const int r = quad * 32 + lane;
-    const int kj = kb * 128 + r;
-    const uint32_t trow = tmem + ((uint32_t)(quad * 32) << 16);
-    const uint64_t sl2x2 = f2(a.scale_log2, a.scale_log2), nlog2e = f2(-LOG2E, -LOG2E);
-    bool ok = true;
-    for (int it = 0; it < nit; it++) {
-      const int i = kb + it;
-      const int q0 = i * 128;
-      const float* ld = sld + (it % BWD_STAGES) * 256;  // lse[128] | D[128] of this query block
-      if (!(ok = mbar_wait(st_full0 + 8 * (it % BWD_STAGES), (it / BWD_STAGES) & 1, abort_flag, a.flags))) break;
-      if (!(ok = mbar_wait(s_full, it & 1, abort_flag, a.flags))) break;
-      tc_fence_after();
-      const bool masked = it == 0;  // the diagonal block: query column c is masked iff c < r
-      float pk[4][16];              // P^T of this thread's 64 columns
-      // phase 1: P^T = 2^(S^T sl2 - lse log2 e) (masked), P~^T = drop(P^T)
-#pragma unroll
-      for (int sub = 0; sub < 4; sub++) {
-        const int c0 = half * 64 + sub * 16;
-        uint32_t sv[16];
-        tmem_ld_32x32b_x16(trow + c0, sv);
-        tmem_ld_wait();
-        uint32_t pp[8];
-#pragma unroll
-        for (int e = 0; e < 16; e += 4) {
-          const float4 l4 = *reinterpret_cast<const float4*>(ld + c0 + e);
-          const uint64_t y01 = f2fma(f2(__uint_as_float(sv[e]), __uint_as_float(sv[e + 1])), sl2x2,
-                                     f2mul(f2(l4.x, l4.y), nlog2e));
-          const uint64_t y23 = f2fma(f2(__uint_as_float(sv[e + 2]), __uint_as_float(sv[e + 3])), sl2x2,
-                                     f2mul(f2(l4.z, l4.w), nlog2e));
-          float p4[4];
-          if (BWD_POLY_EVERY > 0 && ((e >> 1) % (BWD_POLY_EVERY > 0 ? BWD_POLY_EVERY : 1)) == BWD_POLY_EVERY - 1) {
-            const float2 q01 = f2split(exp2_poly2(y01));
-            p4[0] = q01.x;
-            p4[1] = q01.y;
-          } else {
-            const float2 x01 = f2split(y01);
-            p4[0] = ex2(x01.x);
-            p4[1] = ex2(x01.y);
-          }
-          if (BWD_POLY_EVERY > 0 && (((e >> 1) + 1) % (BWD_POLY_EVERY > 0 ? BWD_POLY_EVERY : 1)) == BWD_POLY_EVERY - 1) {
-            const float2 q23 = f2split(exp2_poly2(y23));
-            p4[2] = q23.x;
-            p4[3] = q23.y;
-          } else {
-            const float2 x23 = f2split(y23);
-            p4[2] = ex2(x23.x);
-            p4[3] = ex2(x23.y);
-          }
-#pragma unroll
-          for (int u = 0; u < 4; u++) {
-            if (masked && c0 + e + u < r) p4[u] = 0.f;
-            pk[sub][e + u] = p4[u];
-          }
-          if (DROP) {
-#pragma unroll
-            for (int u = 0; u < 4; u++)
-              p4[u] *= drop_mul(dk, ((uint64_t)bh * a.T + q0 + c0 + e + u) * a.T + kj);
-          }
-          pp[e >> 1] = pack2(p4[0], p4[1]);
-          pp[(e >> 1) + 1] = pack2(p4[2], p4[3]);
-        }
-        tmem_st_32x32b_x8(trow + half * 64 + sub * 8, pp);
-      }
-      tmem_st_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(p_ready);
-      // phase 2: dS^T = P^T (drop(dP^T) - D)
-      if (!(ok = mbar_wait(dp_full, it & 1, abort_flag, a.flags))) break;
-      tc_fence_after();
-#pragma unroll
-      for (int sub = 0; sub < 4; sub++) {
-        const int c0 = half * 64 + sub * 16;
-        uint32_t dv[16];
-        tmem_ld_32x32b_x16(trow + 128 + c0, dv);
-        tmem_ld_wait();
-        uint32_t pd[8];
-#pragma unroll
-        for (int e = 0; e < 16; e += 2) {
-          const float2 d2 = *reinterpret_cast<const float2*>(ld + 128 + c0 + e);
-          float dp0 = __uint_as_float(dv[e]), dp1 = __uint_as_float(dv[e + 1]);
-          if (DROP) {
-            dp0 *= drop_mul(dk, ((uint64_t)bh * a.T + q0 + c0 + e) * a.T + kj);
-            dp1 *= drop_mul(dk, ((uint64_t)bh * a.T + q0 + c0 + e + 1) * a.T + kj);
-          }
-          pd[e >> 1] = pack2v(f2mul(f2(pk[sub][e], pk[sub][e + 1]), f2sub(f2(dp0, dp1), f2(d2.x, d2.y))));
-        }
-        tmem_st_32x32b_x8(trow + 128 + half * 64 + sub * 8, pd);
-      }
-      tmem_st_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(ds_ready);
-    }
-    const bool done = ok && mbar_wait(acc_full, 0, abort_flag, a.flags);
-    if (done) {
-      tc_fence_after();
-      bf16* rowp = a.dqkv + (size_t)(row0 + kj) * (3 * a.H * 64);
-      // half 0: dV at slot 2H+h; half 1: dK (times 1/sqrt(hd)) at slot H+h
-      const float f = half == 0 ? 1.0f : a.scale;
-      const int slot = (half == 0 ? 2 : 1) * a.H + h;
-      uint4* dst = reinterpret_cast<uint4*>(rowp + (size_t)slot * 64);
-#pragma unroll
-      for (int c2 = 0; c2 < 2; c2++) {  // 32 columns at a time: stored, then their block column sums
-        float cs[32];
-#pragma unroll
-        for (int c1 = 0; c1 < 2; c1++) {
-          const int c = 2 * c2 + c1;
-          uint32_t v[16];
-          tmem_ld_32x32b_x16(trow + 256 + half * 64 + c * 16, v);
-          tmem_ld_wait();
-          const float* x = reinterpret_cast<const float*>(v);
-          uint32_t w[8];
-#pragma unroll
-          for (int k = 0; k < 8; k++) {
-            w[k] = pack2(x[2 * k] * f, x[2 * k + 1] * f);
-            const float2 bk = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[k]));
-            cs[16 * c1 + 2 * k] = bk.x;  // the stored (bf16) values
-            cs[16 * c1 + 2 * k + 1] = bk.y;
-          }
-          dst[2 * c] = make_uint4(w[0], w[1], w[2], w[3]);
-          dst[2 * c + 1] = make_uint4(w[4], w[5], w[6], w[7]);
-        }
-        if (a.colsum) {
-          const float sq = warp_colsum32(cs, lane);
-          block_colsum(reinterpret_cast<float*>(smem + KW_RED), half, quad, lane, sq, a.colsum,
-                       (size_t)(row0 + kb * 128) / 128, 3L * a.H * 64, (long)slot * 64 + 32 * c2, a.colsum_acc);
-        }
-      }
-    } else if (a.colsum) {
-      // every math warp takes part in the column-sum barriers, even on a failed wait
-      for (int c2 = 0; c2 < 4; c2++) asm volatile("bar.sync 1, 256;" ::: "memory");
-    }
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  if (warp == 1) tmem_dealloc(tmem, 512);
-}
-
-constexpr int QW_Q = 0, QW_DO = TILE, QW_OT = 2 * TILE, QW_ST = 3 * TILE, QW_BAR = (3 + 2 * BWD_STAGES) * TILE;
-constexpr int QW_RED = QW_BAR + 128;
-constexpr int QW_SMEM = QW_RED + 1024;
-
-template <bool DROP>
-__global__ void __launch_bounds__(320, 1) k_attn_bwd_qw(const __grid_constant__ CUtensorMap tkv,
-                                                        const __grid_constant__ CUtensorMap tdo,
-                                                        const __grid_constant__ CUtensorMap tout, AttnTcArgs a) {
-  pdl_trigger();
-  const DropKey dk = DROP ? drop_live(a.drop) : a.drop;
-  extern __shared__ __align__(1024) uint8_t smem[];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if (smem_u32(smem) & 1023) {
-    if (threadIdx.x == 0) atomicOr(a.flags, FLAG_TIMEOUT);
-    return;
-  }
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + QW_BAR);
-  const uint32_t qd_full = smem_u32(bars + 0), kv_full0 = smem_u32(bars + 1),
-                 kv_empty0 = smem_u32(bars + 1 + BWD_STAGES);
-  const uint32_t s_full = smem_u32(bars + 1 + 2 * BWD_STAGES), dp_full = s_full + 8, s_read = s_full + 16,
-                 ds_ready = s_full + 24, acc_full = s_full + 32;
-  uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + 6 + 2 * BWD_STAGES);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(tslot + 1);
-  const uint32_t sb = smem_u32(smem);
-
-  const int nqb = a.T / 128;
-  const int qb = nqb - 1 - (int)blockIdx.y;  // longest rows of every (b, h) first
-  const int bh = blockIdx.x, b = bh / a.H, h = bh % a.H;
-  const int row0 = b * a.T;
-  const int nkb = qb + 1;  // 128-key blocks up to and including the diagonal
-
-  if (threadIdx.x == 0) {
-    mbar_init(qd_full, 1);
-    for (int s = 0; s < BWD_STAGES; s++) {
-      mbar_init(kv_full0 + 8 * s, 1);
-      mbar_init(kv_empty0 + 8 * s, 1);
-    }
-    mbar_init(s_full, 1);
-    mbar_init(dp_full, 1);
-    mbar_init(s_read, 8);
-    mbar_init(ds_ready, 8);
-    mbar_init(acc_full, 1);
-    *abort_flag = 0;
-    fence_barrier_init();
-    prefetch_tmap(&tkv);
-    prefetch_tmap(&tdo);
-    prefetch_tmap(&tout);
-  }
-  if (warp == 1) {
-    tmem_alloc(smem_u32(tslot), 512);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tslot;
-
-  if (warp == 0) {
-    if (lane == 0) {
-      mbar_expect_tx(qd_full, 3 * TILE);
-      tma_load_3d(sb + QW_Q, &tkv, qd_full, 0, h, row0 + qb * 128);
-      tma_load_3d(sb + QW_DO, &tdo, qd_full, 0, h, row0 + qb * 128);
-      tma_load_3d(sb + QW_OT, &tout, qd_full, 0, h, row0 + qb * 128);
-      int issued = 0;
-      bool ok = true;
-      for (int j = 0; j < nkb; j++) {
-        const int s = j % BWD_STAGES;
-        const uint32_t fb = kv_full0 + 8 * s;
-        if (!(ok = mbar_wait(kv_empty0 + 8 * s, ((j / BWD_STAGES) & 1) ^ 1, abort_flag, a.flags))) break;
-        mbar_expect_tx(fb, 2 * TILE);
-        tma_load_3d(sb + QW_ST + s * 2 * TILE, &tkv, fb, 0, a.H + h, row0 + j * 128);
-        tma_load_3d(sb + QW_ST + s * 2 * TILE + TILE, &tkv, fb, 0, 2 * a.H + h, row0 + j * 128);
-        issued = j + 1;
-      }
-      if (!ok) {  // the loads already issued land before the CTA can exit
-        mbar_wait(qd_full, 0, abort_flag, a.flags);
-        for (int j = issued - BWD_STAGES < 0 ? 0 : issued - BWD_STAGES; j < issued; j++)
-          mbar_wait(kv_full0 + 8 * (j % BWD_STAGES), (j / BWD_STAGES) & 1, abort_flag, a.flags);
-      }
-    }
-  } else if (warp == 1) {
-    if (lane == 0) {
-      constexpr uint32_t id_s = idesc_bf16_f32(128, 128, false, false);
-      constexpr uint32_t id_acc = idesc_bf16_f32(128, 64, false, true);
-      auto k_of = [&](int j) { return sb + QW_ST + (j % BWD_STAGES) * 2 * TILE; };
-      auto issue_s = [&](int j) -> bool {  // S = Q K^T of block j
-        if (!mbar_wait(kv_full0 + 8 * (j % BWD_STAGES), (j / BWD_STAGES) & 1, abort_flag, a.flags)) return false;
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < 4; kk++)
-          mma_bf16_ss(tmem, desc_k(sb + QW_Q, TILE, kk), desc_k(k_of(j), TILE, kk), id_s, kk > 0);
-        mma_commit(s_full);
-        return true;
-      };
-      auto issue_dp = [&](int j) {  // dP = dO V^T of block j (its stage is loaded)
-#pragma unroll
-        for (int kk = 0; kk < 4; kk++)
-          mma_bf16_ss(tmem + 128, desc_k(sb + QW_DO, TILE, kk), desc_k(k_of(j) + TILE, TILE, kk), id_s, kk > 0);
-        mma_commit(dp_full);
-      };
-      bool ok = mbar_wait(qd_full, 0, abort_flag, a.flags) && issue_s(0);
-      if (ok) issue_dp(0);
-      for (int j = 0; j < nkb && ok; j++) {
-        if (!(ok = mbar_wait(s_read, j & 1, abort_flag, a.flags))) break;
-        if (j + 1 < nkb && !(ok = issue_s(j + 1))) break;
-        if (!(ok = mbar_wait(ds_ready, j & 1, abort_flag, a.flags))) break;
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < 8; kk++)  // dQ += dS K (K = the block's 128 keys)
-          mma_bf16_ts(tmem + 256, tmem + 128 + acolw(kk), desc_mn64(k_of(j), kk), id_acc, (j > 0 || kk > 0));
-        mma_commit(kv_empty0 + 8 * (j % BWD_STAGES));
-        if (j + 1 < nkb) issue_dp(j + 1);
-      }
-      mma_commit(acc_full);
-    }
-  } else {
-    const int quad = warp & 3;
-    const int half = (warp - 2) >> 2;
-    const int r = quad * 32 + lane;
-    const int qi = qb * 128 + r;
-    const uint32_t trow = tmem + ((uint32_t)(quad * 32) << 16);
-    const float lse2 = a.lse[(size_t)bh * a.T + qi] * LOG2E;
-    // D of this row from the dO and O tiles (128-byte rows, 128-byte swizzle:
-    // 16-byte chunk q of row r at q ^ (r & 7)); both halves compute it
-    bool ok = mbar_wait(qd_full, 0, abort_flag, a.flags);
-    float Di = 0.f;
-    if (ok) {
-#pragma unroll
-      for (int q = 0; q < 8; q++) {
-        const uint32_t off = r * 128 + ((q ^ (r & 7)) << 4);
-        const uint4 x = ld_shared_v4(sb + QW_DO + off), y = ld_shared_v4(sb + QW_OT + off);
-        const uint32_t xw[4] = {x.x, x.y, x.z, x.w}, yw[4] = {y.x, y.y, y.z, y.w};
-#pragma unroll
-        for (int k = 0; k < 4; k++) {
-          const float2 xf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&xw[k]));
-          const float2 yf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&yw[k]));
-          Di = fmaf(xf.x, yf.x, fmaf(xf.y, yf.y, Di));
-        }
-      }
-      if (half == 0) a.dsum[(size_t)bh * a.T + qi] = Di;
-    }
-    const uint64_t sl2x2 = f2(a.scale_log2, a.scale_log2), nlse2 = f2(-lse2, -lse2), Dx2 = f2(Di, Di);
-    const uint64_t ebase = ((uint64_t)bh * a.T + qi) * a.T;
-    for (int j = 0; j < nkb && ok; j++) {
-      if (!(ok = mbar_wait(s_full, j & 1, abort_flag, a.flags))) break;
-      tc_fence_after();
-      const int key0 = j * 128;
-      const bool masked = j == qb;  // the diagonal block: key column c is visible iff c <= r
-      // phase 1: P = 2^(S sl2 - lse log2 e) (masked) into registers
-      float pk[4][16];
-#pragma unroll
-      for (int sub = 0; sub < 4; sub++) {
-        const int c0 = half * 64 + sub * 16;
-        uint32_t sv[16];
-        tmem_ld_32x32b_x16(trow + c0, sv);
-        tmem_ld_wait();
-#pragma unroll
-        for (int e = 0; e < 16; e += 2) {
-          const uint64_t y2 = f2fma(f2(__uint_as_float(sv[e]), __uint_as_float(sv[e + 1])), sl2x2, nlse2);
-          float e0, e1;
-          if (BWD_POLY_EVERY > 0 && ((e >> 1) % (BWD_POLY_EVERY > 0 ? BWD_POLY_EVERY : 1)) == BWD_POLY_EVERY - 1) {
-            const float2 q = f2split(exp2_poly2(y2));
-            e0 = q.x;
-            e1 = q.y;
-          } else {
-            const float2 y = f2split(y2);
-            e0 = ex2(y.x);
-            e1 = ex2(y.y);
-          }
-          pk[sub][e] = (masked && c0 + e > r) ? 0.f : e0;
-          pk[sub][e + 1] = (masked && c0 + e + 1 > r) ? 0.f : e1;
-        }
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(s_read);  // S may be overwritten by the next block
-      // phase 2: dS = P (drop(dP) - D) over the dP columns
-      if (!(ok = mbar_wait(dp_full, j & 1, abort_flag, a.flags))) break;
-      tc_fence_after();
-#pragma unroll
-      for (int sub = 0; sub < 4; sub++) {
-        const int c0 = half * 64 + sub * 16;
-        uint32_t dv[16];
-        tmem_ld_32x32b_x16(trow + 128 + c0, dv);
-        tmem_ld_wait();
-        uint32_t pd[8];
-#pragma unroll
-        for (int e = 0; e < 16; e += 2) {
-          float dp0 = __uint_as_float(dv[e]), dp1 = __uint_as_float(dv[e + 1]);
-          if (DROP) {
-            dp0 *= drop_mul(dk, ebase + key0 + c0 + e);
-            dp1 *= drop_mul(dk, ebase + key0 + c0 + e + 1);
-          }
-          pd[e >> 1] = pack2v(f2mul(f2(pk[sub][e], pk[sub][e + 1]), f2sub(f2(dp0, dp1), Dx2)));
-        }
-        tmem_st_32x32b_x8(trow + 128 + half * 64 + sub * 8, pd);
-      }
-      tmem_st_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(ds_ready);
-    }
-    const bool done = ok && mbar_wait(acc_full, 0, abort_flag, a.flags);
-    if (done) {
-      tc_fence_after();
-      uint4* dst = reinterpret_cast<uint4*>(a.dqkv + (size_t)(row0 + qi) * (3 * a.H * 64) + (size_t)h * 64 + half * 32);
-      const float f = a.scale;
-      float cs[32];
-#pragma unroll
-      for (int c = 0; c < 2; c++) {
-        uint32_t v[16];
-        tmem_ld_32x32b_x16(trow + 256 + half * 32 + c * 16, v);
-        tmem_ld_wait();
-        const float* x = reinterpret_cast<const float*>(v);
-        uint32_t w[8];
-#pragma unroll
-        for (int k = 0; k < 8; k++) {
-          w[k] = pack2(x[2 * k] * f, x[2 * k + 1] * f);
-          const float2 bk = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[k]));
-          cs[16 * c + 2 * k] = bk.x;  // the stored (bf16) values
-          cs[16 * c + 2 * k + 1] = bk.y;
-        }
-        dst[2 * c] = make_uint4(w[0], w[1], w[2], w[3]);
-        dst[2 * c + 1] = make_uint4(w[4], w[5], w[6], w[7]);
-      }
-      if (a.colsum) {
-        const float sq = warp_colsum32(cs, lane);
-        block_colsum(reinterpret_cast<float*>(smem + QW_RED), half, quad, lane, sq, a.colsum,
-                     (size_t)(row0 + qb * 128) / 128, 3L * a.H * 64, (long)h * 64 + 32 * half, a.colsum_acc);
-      }
-    } else if (a.colsum) {
-      // every math warp takes part in the column-sum barriers, even on a failed wait
-      for (int c2 = 0; c2 < 2; c2++) asm volatile("bar.sync 1, 256;" ::: "memory");
-    }
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  if (warp == 1) tmem_dealloc(tmem, 512);
 }
 
 // ---------------------------------------------------------------- host side
@@ -1763,49 +932,6 @@ bool attn_fwd_tc(Ctx& c, const AttnDesc& d) {
   LaunchScope s(c, "attn_fwd_tc");
   if (drop) k_attn_fwd_o<true><<<grid, 192, D_SMEM, c.stream>>>(tq, tkv64, make_args(d, c.flags));
   else k_attn_fwd_o<false><<<grid, 192, D_SMEM, c.stream>>>(tq, tkv64, make_args(d, c.flags));
-  return true;
-}
-
-// the ping-pong forward (two 128-query tiles per CTA, 128-key blocks)
-bool attn_fwd_tc_pp(Ctx& c, const AttnDesc& d) {
-  CUtensorMap t128;
-  long rows = (long)d.B * d.T;
-  if (!map_rows(&t128, d.qkv, 3 * d.H, rows, 128)) return false;
-  const bool drop = d.drop.active;
-  cudaFuncSetAttribute(drop ? k_attn_fwd_pp<true> : k_attn_fwd_pp<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                       F_SMEM);
-  const int npair = (d.T / 128 + 1) / 2;
-  dim3 grid(d.B * d.H, npair);
-  LaunchScope s(c, "attn_fwd_tc");
-  if (drop) k_attn_fwd_pp<true><<<grid, 320, F_SMEM, c.stream>>>(t128, make_args(d, c.flags));
-  else k_attn_fwd_pp<false><<<grid, 320, F_SMEM, c.stream>>>(t128, make_args(d, c.flags));
-  return true;
-}
-
-// the wide backward (128-wide inner blocks, one CTA per SM): dQ (with D) first
-bool attn_bwd_tc_wide(Ctx& c, const AttnDesc& d) {
-  CUtensorMap tkv, tdo, tout;
-  long rows = (long)d.B * d.T;
-  if (!map_rows(&tkv, d.qkv, 3 * d.H, rows, 128) || !map_rows(&tdo, d.dout, d.H, rows, 128) ||
-      !map_rows(&tout, d.o, d.H, rows, 128))
-    return false;
-  const bool drop = d.drop.active;
-  cudaFuncSetAttribute(drop ? k_attn_bwd_kvw<true> : k_attn_bwd_kvw<false>,
-                       cudaFuncAttributeMaxDynamicSharedMemorySize, KW_SMEM);
-  cudaFuncSetAttribute(drop ? k_attn_bwd_qw<true> : k_attn_bwd_qw<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                       QW_SMEM);
-  AttnTcArgs a = make_args(d, c.flags);
-  dim3 grid(d.B * d.H, d.T / 128);
-  {
-    LaunchScope s(c, "attn_bwd_q_tc");
-    if (drop) k_attn_bwd_qw<true><<<grid, 320, QW_SMEM, c.stream>>>(tkv, tdo, tout, a);
-    else k_attn_bwd_qw<false><<<grid, 320, QW_SMEM, c.stream>>>(tkv, tdo, tout, a);
-  }
-  {
-    LaunchScope s(c, "attn_bwd_kv_tc");
-    if (drop) k_attn_bwd_kvw<true><<<grid, 320, KW_SMEM, c.stream>>>(tkv, tdo, a);
-    else k_attn_bwd_kvw<false><<<grid, 320, KW_SMEM, c.stream>>>(tkv, tdo, a);
-  }
   return true;
 }
 

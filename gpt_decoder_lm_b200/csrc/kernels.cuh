@@ -132,8 +132,8 @@ struct AttnDesc {
   void* dqkv;         // bwd: [B, T, 3, H, hd]
   float* dsum;        // bwd scratch: rowsum(dO * O) [B, H, T]
   DropKey drop;       // site 1; elem = ((b*H + h)*T + i)*T + j
-  // wide backward kernels: column sums of the stored dqkv per 128-row block,
-  // colsum[m / 128][3 H hd] (= or += with colsum_acc); null: none
+  // bwd (tensor-core kernels): column sums of the stored dqkv per 128-row
+  // block, colsum[m / 128][3 H hd] (= or += with colsum_acc); null: none
   float* colsum = nullptr;
   int colsum_acc = 0;
 };
@@ -144,9 +144,7 @@ bool attn_tc_shape_ok(int T, int hd);
 bool attn_tc_supported(const AttnDesc& a);  // shape rule plus 16-byte aligned pointers
 // false: a tensor map could not be encoded (nothing launched)
 bool attn_fwd_tc(Ctx& c, const AttnDesc& a);
-bool attn_fwd_tc_pp(Ctx& c, const AttnDesc& a);  // two query tiles per CTA, 128-key blocks
 bool attn_bwd_tc(Ctx& c, const AttnDesc& a);
-bool attn_bwd_tc_wide(Ctx& c, const AttnDesc& a);  // 128-wide inner blocks, one CTA per SM
 // decoding: o [B, H*hd] = attention of position t against positions 0..t of
 // the cache qkv [B, T, 3, H, hd]
 template <typename T> void attn_decode(Ctx& c, const T* qkv, int B, int Tn, int H, int hd, int t, T* o);

@@ -72,13 +72,11 @@ extern "C" gpt_status gpt_test_attention(int32_t backend, int32_t backward, int3
   c.stream = (cudaStream_t)stream;
   c.flags = d_flags;
   AttnDesc a{B, T, H, hd, qkv, o, lse, dout, dqkv, dsum, make_drop_key(seed, counter, layer, 1, p)};
-  if (colsum && !(backward && (backend == 1 || backend == 3))) return GPT_ERR_INVALID_ARG;
+  if (colsum && !(backward && backend == 1)) return GPT_ERR_INVALID_ARG;
   a.colsum = colsum;
-  if (backend >= 1 && backend <= 3) {
+  if (backend == 1) {
     if (dtype != 1 || !attn_tc_supported(a)) return GPT_ERR_UNSUPPORTED;
-    const bool ok = backward ? (backend == 3 ? attn_bwd_tc_wide(c, a) : attn_bwd_tc(c, a))
-                             : (backend == 1 ? attn_fwd_tc(c, a) : attn_fwd_tc_pp(c, a));
-    if (!ok) return GPT_ERR_CUDA;
+    if (!(backward ? attn_bwd_tc(c, a) : attn_fwd_tc(c, a))) return GPT_ERR_CUDA;
   } else if (backend == 0) {
     if (hd != 4 && hd != 8 && hd != 16 && hd != 32 && hd != 64 && hd != 128) return GPT_ERR_UNSUPPORTED;
     if (dtype == 1) {
@@ -121,26 +119,3 @@ extern "C" gpt_status gpt_test_wait_timeout(uint64_t limit_ns, void* stream, uin
   return (f & FLAG_TIMEOUT) ? GPT_ERR_TIMEOUT : GPT_OK;
 }
 
-// the attention kernels' FMA-pipe 2^x next to CUDA's exp2f, element by element
-__global__ void k_test_exp2(const float* __restrict__ x, float* __restrict__ y_poly, float* __restrict__ y_ref,
-                            long n) {
-  const long i = 2 * ((long)blockIdx.x * blockDim.x + threadIdx.x);
-  if (i >= n) return;
-  const float a = x[i], b = i + 1 < n ? x[i + 1] : 0.f;
-  const float2 p = f2split(exp2_poly2(f2(a, b)));
-  y_poly[i] = p.x;
-  y_ref[i] = exp2f(a);
-  if (i + 1 < n) {
-    y_poly[i + 1] = p.y;
-    y_ref[i + 1] = exp2f(b);
-  }
-}
-
-extern "C" gpt_status gpt_test_exp2(const float* d_x, float* d_y_poly, float* d_y_ref, int64_t n, void* stream) {
-  if (!d_x || !d_y_poly || !d_y_ref || n < 1) return GPT_ERR_INVALID_ARG;
-  cudaStream_t st = (cudaStream_t)stream;
-  const long pairs = (n + 1) / 2;
-  k_test_exp2<<<(unsigned)((pairs + 255) / 256), 256, 0, st>>>(d_x, d_y_poly, d_y_ref, n);
-  if (cudaGetLastError() != cudaSuccess || cudaStreamSynchronize(st) != cudaSuccess) return GPT_ERR_CUDA;
-  return GPT_OK;
-}

@@ -53,10 +53,8 @@ gpt_status gpt_test_gemm(int32_t backend, int32_t M, int32_t N, int32_t K, const
 /* Causal attention of one layer.  qkv [B, T, 3, H, hd], o [B, T, H, hd],
  * lse fp32 [B, H, T]; backward also takes dout [B, T, H, hd] and writes
  * dqkv [B, T, 3, H, hd] using dsum fp32 [B, H, T] as scratch.  dtype: 0 fp32,
- * 1 bf16.  backend: 0 CUDA cores, 1 tensor cores, 2 tensor cores with the
- * two-tile (ping-pong) forward kernel, 3 the ping-pong forward and the
- * backward kernels with 128-wide inner blocks (GPT_ERR_UNSUPPORTED when the
- * shape is not supported).  colsum (nullable; backward of backends 1, 3):
+ * 1 bf16.  backend: 0 CUDA cores, 1 tensor cores (GPT_ERR_UNSUPPORTED when
+ * the shape is not supported).  colsum (nullable; backward of backend 1):
  * fp32 [B T / 128, 3 H hd] receives the column sums of the stored dqkv over
  * each 128-row block.  Dropout on the probabilities with
  * (p, seed, counter, layer) as in the model (site 1); p = 0 disables it. */
@@ -73,12 +71,6 @@ gpt_status gpt_test_attention(int32_t backend, int32_t backward, int32_t dtype, 
  * context stays usable.  Synchronising.  Returns GPT_ERR_TIMEOUT when the
  * flag was raised (the expected outcome), GPT_OK otherwise. */
 gpt_status gpt_test_wait_timeout(uint64_t limit_ns, void* stream, uint32_t* d_flags, int32_t* d_gave_up);
-
-/* The polynomial 2^x the attention kernels evaluate on the FMA pipe for part
- * of the softmax exponentials, next to CUDA's exp2f: for n device fp32
- * arguments d_x, d_y_poly receives the polynomial's values and d_y_ref
- * exp2f's.  Synchronising. */
-gpt_status gpt_test_exp2(const float* d_x, float* d_y_poly, float* d_y_ref, int64_t n, void* stream);
 
 #ifdef __cplusplus
 }
