@@ -632,6 +632,30 @@ def run_kernels(w):
     print(json.dumps({"kernels": "ok", "workload": w.name}))
 
 
+def run_layer_case(w, layers: int):
+    """Two optimiser steps of the workload's dimensions cut to `layers` layers and
+    one micro-batch (the small case for per-kernel DRAM captures: every GEMM,
+    attention and norm launch of a layer has the full model's shapes). The
+    second step is the one to capture: 12 GEMM launches per layer (4 forward,
+    4 dX, 4 dW) and 3 for the lm_head, in the engine's own order."""
+    import dataclasses
+
+    import torch
+
+    from gpt_decoder_lm_b200 import binding as gb
+    wl = dataclasses.replace(w, n_layer=layers, grad_accum=1)
+    model = gb.Model(gb.make_config(wl), seed=wl.weight_seed, device=torch.device("cuda", 0))
+    d_stream = torch.from_numpy(W.token_stream(wl).view(np.int16)).cuda()
+    model.set_graphs(False)
+    out = []
+    for st in (1, 2):
+        l0 = model.launch_count()
+        loss, norm = model.train_step(d_stream, wl.data_seed, wl.lr, st, sync=True)
+        out.append({"step": st, "loss": loss, "launches": model.launch_count() - l0})
+    torch.cuda.synchronize()
+    print(json.dumps({"layer_case": wl.name, "n_layer": layers, "grad_accum": 1, "steps": out}))
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -645,10 +669,16 @@ def main():
                     help="N > 1: independent replicas instead of data-parallel training")
     ap.add_argument("--kernels", action="store_true",
                     help="one launch of each hot kernel at the workload's shapes (for ncu), then exit")
+    ap.add_argument("--layer-case", type=int, default=0, metavar="L",
+                    help="two eager optimiser steps at the workload's dimensions with L layers and one "
+                         "micro-batch (for per-kernel ncu captures), then exit")
     args = ap.parse_args()
     w = W.ALL[args.workload]
     if args.kernels:
         run_kernels(w)
+        return
+    if args.layer_case > 0:
+        run_layer_case(w, args.layer_case)
         return
     rank = int(os.environ.get("RANK", 0))
     world = int(os.environ.get("WORLD_SIZE", 1))
