@@ -76,10 +76,11 @@ def attn_flops_per_step(w) -> float:
     return L * w.grad_accum * per_layer_fwd * (1 + 2.5)
 
 
-# dram__bytes_read.sum + dram__bytes_write.sum of the tensor-core GEMMs per launch, averaged
-# over the launches of one training step in profiles/launch_list_gpt2_124m_train_step.md;
-# None while the kernels have changed since that capture
-GEMM_DRAM_BYTES_PER_LAUNCH = None
+# dram__bytes_read.sum + dram__bytes_write.sum of the tensor-core GEMMs per launch (ncu, one
+# pass, on `bench.py --layer-case 2`: every GEMM shape of a layer and the lm_head at full size),
+# weighted to the 12-layer step: (12 x one layer's 12 GEMMs + the lm_head's 3) / 147 launches.
+# None once the kernels change after that capture.
+GEMM_DRAM_BYTES_PER_LAUNCH = 107462595
 
 
 class Clocks:
