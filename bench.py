@@ -9,7 +9,9 @@ forward, cross-entropy, backward, clip and AdamW, all in libgpt.so.  For
 N > 1 (torchrun) every rank gathers its own micro-batches and the replicas'
 gradients are averaged before clip + AdamW (data-parallel training: a
 bucketed NCCL all-reduce on a second stream, overlapping the backward;
-gpt_decoder_lm_b200/ddp.py); --replicas runs independent replicas instead.
+gpt_decoder_lm_b200/ddp.py); --zero1 shards the optimiser step instead
+(reduce to the shard owner, clip + AdamW on the own shard, all-gather of the
+weights); --replicas runs independent replicas.
 The barrier and the max-over-ranks timing use torch.distributed.
 
 `--impl reference` times the CPU oracle (float64 numpy) on a bounded sample
@@ -435,7 +437,7 @@ def run_ours(args, w, rank, world, local_rank):
     trainer = None
     if use_ddp:
         from gpt_decoder_lm_b200 import ddp
-        trainer = ddp.DataParallelTrainer(model)
+        trainer = ddp.ZeroTrainer(model) if args.zero1 else ddp.DataParallelTrainer(model)
 
     def step_fn(i, sync=False):
         if trainer is not None:
@@ -567,7 +569,9 @@ def run_ours(args, w, rank, world, local_rank):
                        "n_embd": w.n_embd, "seq_len": w.block_size, "micro_batch": w.batch_size,
                        "grad_accum": w.grad_accum, "tokens_per_step_per_gpu": tok_step,
                        "global_batch_tokens": tok_step * world,
-                       "parallelism": f"dp{world} (bucketed NCCL all-reduce overlapped with the backward)"
+                       "parallelism": (f"dp{world} zero1 (bucketed NCCL reduce to the shard owners overlapped "
+                                       "with the backward, sharded clip + AdamW, weight all-gather)" if args.zero1 else
+                                       f"dp{world} (bucketed NCCL all-reduce overlapped with the backward)")
                        if use_ddp else f"replicas x{world}",
                        "l2": "256 MiB buffer zeroed between timed steps; step working set ~8 GB"},
             "mfu": {"nominal_2250": mfu_nom, "measured_peak": mfu_meas, "flops_per_token": fpt},
@@ -666,6 +670,8 @@ def main():
     ap.add_argument("--workload", default=W.GPT2_124M.name, choices=list(W.ALL))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-configs", action="store_true", help="skip the other workloads' step timings")
+    ap.add_argument("--zero1", action="store_true",
+                    help="N > 1: data-parallel training with the optimiser step sharded (ZeRO stage 1)")
     ap.add_argument("--replicas", action="store_true",
                     help="N > 1: independent replicas instead of data-parallel training")
     ap.add_argument("--kernels", action="store_true",

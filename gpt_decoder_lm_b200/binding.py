@@ -56,6 +56,10 @@ _PROTOS = {
     "gpt_workspace_bytes": (I32, [P, P]),
     "gpt_grad_buckets": (I32, [P, I32, P, P, P, P]),
     "gpt_grad_arena": (I32, [P, P, P]),
+    "gpt_zero1_shard": (I32, [P, I32, I32, P, P, P]),
+    "gpt_state_arenas": (I32, [P, P, P, P, P, P, P, P]),
+    "gpt_grad_sumsq_shard": (I32, [P, I64, I64, P]),
+    "gpt_clip_adamw_shard": (I32, [P, F32, I32, I64, I64, F32, P, I32, P]),
     "gpt_train_step_accumulate": (I32, [P, P, U64, U64, I32, P]),
     "gpt_stream_wait_bucket": (I32, [P, I32, P]),
     "gpt_step_loss": (I32, [P, P]),
@@ -182,6 +186,17 @@ def grad_buckets(cfg: GptConfig):
     return [(int(off[i]), int(cnt[i]), int(bkt[i])) for i in range(n.value)]
 
 
+NORM_PARTIALS = 592  # GPT_NORM_PARTIALS
+
+
+def zero1_shard(cfg: GptConfig, world: int, rank: int):
+    """(offset, count, stride) of optimiser shard `rank` of `world`."""
+    off, cnt, stride = C.c_int64(), C.c_int64(), C.c_int64()
+    _check(lib().gpt_zero1_shard(C.byref(cfg), world, rank, C.byref(off), C.byref(cnt), C.byref(stride)), None,
+           "zero1_shard")
+    return int(off.value), int(cnt.value), int(stride.value)
+
+
 def kernel_paths(cfg: GptConfig) -> int:
     """GPT_PATH_* bits: which kernels a model with this config runs."""
     n = C.c_uint32(0)
@@ -291,6 +306,43 @@ class Model:
         off = p.value - self.ws.data_ptr()
         assert off % 4 == 0 and off >= 0
         return self.ws[off:off + 4 * n.value].view(torch.float32)
+
+    def state_arenas(self):
+        """{"param", "grad", "adam_m", "adam_v": fp32, "param_bf16": bf16 or None}
+        as torch views of the workspace, each of the allocated length (the
+        used length is ["n"])."""
+        import torch
+        ptr = [C.c_void_p() for _ in range(5)]
+        n, n_alloc = C.c_int64(), C.c_int64()
+        _check(lib().gpt_state_arenas(self.h, *[C.byref(x) for x in ptr], C.byref(n), C.byref(n_alloc)), self.h,
+               "state_arenas")
+        base = self.ws.data_ptr()
+
+        def view(p, dtype, esize):
+            if not p.value:
+                return None
+            off = p.value - base
+            assert off >= 0 and off % esize == 0
+            return self.ws[off:off + esize * n_alloc.value].view(dtype)
+        out = {k: view(p, torch.float32, 4) for k, p in zip(("param", "grad", "adam_m", "adam_v"), ptr)}
+        out["param_bf16"] = view(ptr[4], torch.bfloat16, 2)
+        out["n"] = int(n.value)
+        return out
+
+    def grad_sumsq_shard(self, offset: int, count: int, partials):
+        """NORM_PARTIALS fp64 partial sums of squares of gradient elements
+        [offset, offset + count) into the device tensor `partials`."""
+        assert partials.numel() >= NORM_PARTIALS and partials.dtype.itemsize == 8
+        _check(lib().gpt_grad_sumsq_shard(self.h, offset, count, _ptr(partials)), self.h, "grad_sumsq_shard")
+
+    def clip_adamw_shard(self, lr: float, step: int, offset: int, count: int, grad_scale: float, partials,
+                         sync: bool = True) -> Optional[float]:
+        """Clip + AdamW on one shard; the global norm from the gathered partials."""
+        out = C.c_float()
+        _check(lib().gpt_clip_adamw_shard(self.h, lr, step, offset, count, grad_scale, _ptr(partials),
+                                          partials.numel(), C.byref(out) if sync else None), self.h,
+               "clip_adamw_shard")
+        return float(out.value) if sync else None
 
     def gather_batch(self, stream_tokens, data_seed: int, step: int, micro: int, idx, tgt):
         _check(lib().gpt_gather_batch(self.h, _ptr(stream_tokens), stream_tokens.numel(), data_seed, step, micro,

@@ -90,6 +90,12 @@ struct Layout {
   }
 };
 
+// Elements allocated past the last tensor of every arena: an all-gather of
+// `world` equal shards of ceil(n / world / 64) * 64 elements (world <= 64)
+// overruns the arena by less than 64 * 64.
+constexpr int64_t kArenaSlack = 64 * 64;
+constexpr int kZeroMaxWorld = 64;
+
 // split-K count of a weight-gradient GEMM (sizes the partial-sum scratch; the
 // plan of a 148-SM B200)
 int choose_splits(long M, long N, long K) { return gemm_tc_plan(M, N, K, true, 148).splits; }
@@ -363,7 +369,9 @@ size_t carve(gpt_model& m, uint8_t* base) {
   auto I = [&](size_t n) { return (int32_t*)(base + lay.take(n * 4)); };
   long M = m.M;
   int d = m.d, L = m.L;
-  size_t P = (size_t)m.n_total;
+  // the arenas carry kArenaSlack elements past the last tensor: room for an
+  // in-place all-gather of equal optimiser shards (gpt_zero1_shard)
+  size_t P = (size_t)(m.n_total + kArenaSlack);
   m.scal = F(64);
   m.w = F(P);
   m.g = F(P);
@@ -1203,10 +1211,12 @@ gpt_status gpt_create(const gpt_config* cfg, uint64_t seed, void* d_workspace, s
   cudaStream_t st = m->ctx.stream;
   // zero the arenas (weights, grads, moments) and the scalars
   cudaMemsetAsync(m->scal, 0, 64 * 4, st);
-  cudaMemsetAsync(m->w, 0, (size_t)m->n_total * 4, st);
-  cudaMemsetAsync(m->g, 0, (size_t)m->n_total * 4, st);
-  cudaMemsetAsync(m->am, 0, (size_t)m->n_total * 4, st);
-  cudaMemsetAsync(m->av, 0, (size_t)m->n_total * 4, st);
+  const size_t arena_bytes = (size_t)(m->n_total + kArenaSlack) * 4;
+  cudaMemsetAsync(m->w, 0, arena_bytes, st);
+  cudaMemsetAsync(m->g, 0, arena_bytes, st);
+  cudaMemsetAsync(m->am, 0, arena_bytes, st);
+  cudaMemsetAsync(m->av, 0, arena_bytes, st);
+  if (m->wb) cudaMemsetAsync(m->wb, 0, arena_bytes / 2, st);
   // weights from the seed, uploaded one tensor at a time
   std::vector<float> host;
   for (size_t i = 0; i < m->tensors.size(); i++) {
@@ -1478,6 +1488,98 @@ gpt_status gpt_grad_arena(gpt_model* m, float** d_grad, int64_t* n_floats) {
   *d_grad = m->g;
   *n_floats = m->n_total;
   return GPT_OK;
+}
+
+gpt_status gpt_zero1_shard(const gpt_config* cfg, int32_t world, int32_t rank, int64_t* offset, int64_t* count,
+                           int64_t* stride) {
+  if (!offset || !count || !stride || world < 1 || world > kZeroMaxWorld || rank < 0 || rank >= world)
+    return GPT_ERR_INVALID_ARG;
+  gpt_status s = validate(cfg, nullptr);
+  if (s != GPT_OK) return s;
+  gpt_model m;
+  derive(m, cfg);
+  const int64_t n = m.n_total;
+  const int64_t S = ((n + world - 1) / world + 63) / 64 * 64;
+  *stride = S;
+  *offset = std::min<int64_t>((int64_t)rank * S, n);
+  *count = std::max<int64_t>(0, std::min<int64_t>(S, n - *offset));
+  return GPT_OK;
+}
+
+gpt_status gpt_state_arenas(gpt_model* m, float** d_param, float** d_grad, float** d_adam_m, float** d_adam_v,
+                            void** d_param_bf16, int64_t* n_floats, int64_t* n_alloc) {
+  if (!m || !d_param || !d_grad || !d_adam_m || !d_adam_v || !d_param_bf16 || !n_floats || !n_alloc)
+    return GPT_ERR_INVALID_ARG;
+  *d_param = m->w;
+  *d_grad = m->g;
+  *d_adam_m = m->am;
+  *d_adam_v = m->av;
+  *d_param_bf16 = m->wb;
+  *n_floats = m->n_total;
+  *n_alloc = m->n_total + kArenaSlack;
+  return GPT_OK;
+}
+
+// shard bounds as gpt_zero1_shard gives them: float4-aligned, inside the arena
+static gpt_status check_shard(gpt_model* m, int64_t offset, int64_t count, const char* what) {
+  if (m->lora.on) return fail(m, GPT_ERR_STATE, "%s: LoRA adapters are attached", what);
+  if (offset < 0 || count < 0 || offset % 4 || count % 4 || offset + count > m->n_total)
+    return fail(m, GPT_ERR_INVALID_ARG, "%s: shard outside the arena or not a multiple of 4", what);
+  return GPT_OK;
+}
+
+gpt_status gpt_grad_sumsq_shard(gpt_model* m, int64_t offset, int64_t count, double* d_partials) {
+  if (!m || !d_partials) return GPT_ERR_INVALID_ARG;
+  gpt_status s = check_shard(m, offset, count, "grad_sumsq_shard");
+  if (s != GPT_OK) return s;
+  Ctx& c = m->ctx;
+  const int blocks = sumsq_blocks(c);
+  cudaMemsetAsync(d_partials, 0, GPT_NORM_PARTIALS * sizeof(double), c.stream);
+  if (count > 0) sumsq_partials(c, m->g + offset, count, d_partials, blocks);
+  return check_cuda(m, "grad_sumsq_shard");
+}
+
+gpt_status gpt_clip_adamw_shard(gpt_model* m, float lr, int32_t step, int64_t offset, int64_t count,
+                                float grad_scale, const double* d_partials, int32_t n_partials, float* h_grad_norm) {
+  if (!m || !d_partials || n_partials < 1) return GPT_ERR_INVALID_ARG;
+  if (step < 1) return fail(m, GPT_ERR_INVALID_ARG, "step must be >= 1");
+  if (!(grad_scale > 0.f) || !isfinite(grad_scale)) return fail(m, GPT_ERR_INVALID_ARG, "grad_scale must be > 0");
+  gpt_status s = check_shard(m, offset, count, "clip_adamw_shard");
+  if (s != GPT_OK) return s;
+  Ctx& c = m->ctx;
+  AdamArgs a;
+  a.w = m->w + offset;
+  a.g = m->g + offset;
+  a.m = m->am + offset;
+  a.v = m->av + offset;
+  a.wb = m->wb ? m->wb + offset : nullptr;
+  a.n = count;
+  a.n_decay = std::max<int64_t>(0, std::min<int64_t>(count, m->n_decay - offset));
+  a.norm_partials = d_partials;
+  a.norm_blocks = n_partials;
+  a.norm_out = m->scal + 2;
+  a.lr = lr;
+  a.beta1 = m->cfg.beta1;
+  a.beta2 = m->cfg.beta2;
+  a.eps = m->cfg.eps;
+  a.wd = m->cfg.weight_decay;
+  a.clip = m->cfg.grad_clip;
+  a.gscale = grad_scale;
+  bias_corrections(m, step, &a.bc1, &a.bc2);
+  // k_adamw clears the shard's gradients; the rest of the arena (this
+  // replica's own sums of the other shards) is cleared here
+  if (offset > 0) cudaMemsetAsync(m->g, 0, (size_t)offset * 4, c.stream);
+  if (offset + count < m->n_total)
+    cudaMemsetAsync(m->g + offset + count, 0, (size_t)(m->n_total - offset - count) * 4, c.stream);
+  adamw(c, a);
+  s = check_cuda(m, "clip_adamw_shard");
+  if (s != GPT_OK) return s;
+  if (h_grad_norm) {
+    float sc[4];
+    s = sync_and_flags(m, "clip_adamw_shard", sc);
+    *h_grad_norm = sc[2];
+  }
+  return s;
 }
 
 gpt_status gpt_grad_buckets(const gpt_config* cfg, int32_t cap, int64_t* h_offset, int64_t* h_count,

@@ -922,7 +922,10 @@ void sumsq_partials(Ctx& c, const float* g, long n, double* partials, int blocks
 }
 
 // ============================================================================
-// clip + AdamW (one pass over the fp32 arenas; decayed tensors first).
+// clip + AdamW (one pass over the fp32 arenas; decayed tensors first).  The
+// gradient is gscale times the arena's values (1 for a whole-model step; 1 /
+// world for a shard of summed replica gradients), its norm gscale times the
+// square root of the sum of the partials.
 //   c = min(1, clip / (norm + 1e-6)); g <- c g
 //   w <- w (1 - lr wd)                      (decayed tensors only)
 //   m <- b1 m + (1 - b1) g;  v <- b2 v + (1 - b2) g^2
@@ -938,7 +941,7 @@ __global__ void k_adamw(AdamArgs a, uint32_t* flags) {
     for (int k = threadIdx.x; k < a.norm_blocks; k += 32) t += a.norm_partials[k];
     t = warp_sum_d(t);
     if (threadIdx.x == 0) {
-      double norm = sqrt(t);
+      double norm = sqrt(t) * (double)a.gscale;
       int ok = isfinite(norm) ? 1 : 0;
       float coef = 1.f;
       if (a.clip > 0.f && ok) coef = (float)fmin(1.0, (double)a.clip / (norm + 1e-6));
@@ -956,7 +959,7 @@ __global__ void k_adamw(AdamArgs a, uint32_t* flags) {
     a.bc1 = a.hyper[1];
     a.bc2 = a.hyper[2];
   }
-  const float coef = s_coef;
+  const float coef = s_coef * a.gscale;
   const int ok = s_ok;
   const float om1 = 1.f - a.beta1, om2 = 1.f - a.beta2;
   const float decay = 1.f - a.lr * a.wd;

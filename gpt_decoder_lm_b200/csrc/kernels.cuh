@@ -218,6 +218,7 @@ struct AdamArgs {
   const double* norm_partials; int norm_blocks; float* norm_out;
   float lr, beta1, beta2, eps, wd, clip, bc1, bc2;
   const float* hyper = nullptr;  // when set: {lr, bc1, bc2} read from device memory
+  float gscale = 1.f;            // the gradient is gscale times the arena's values
 };
 void adamw(Ctx& c, const AdamArgs& a);
 

@@ -258,6 +258,59 @@ gpt_status gpt_train_step_host_accumulate(gpt_model* m, const int32_t* h_idx, co
  * gpt_train_step_accumulate / gpt_train_step_host_accumulate. */
 gpt_status gpt_stream_wait_bucket(gpt_model* m, int32_t bucket, void* cuda_stream);
 
+/* ---------------------------------------------------------------- sharded optimiser (ZeRO stage 1)
+ * The fine-tuning pipelines page's distributed-training paragraph points to
+ * DeepSpeed ZeRO for models past DDP's reach; ZeRO's first stage shards the
+ * optimiser step.  Each of `world` ranks owns one contiguous shard of the
+ * arenas; the step becomes
+ *   gpt_train_step_accumulate   as for DDP (bucket events included)
+ *   (caller)                    per bucket, a sum-reduce of each part of the
+ *                               bucket to the rank whose shard holds it
+ *   gpt_grad_sumsq_shard        partial sums of squares of the own shard
+ *   (caller)                    all-gather of every rank's partials
+ *   gpt_clip_adamw_shard        clip by the global norm + AdamW on the own
+ *                               shard only; the rest of the gradient arena
+ *                               is cleared
+ *   (caller)                    all-gather of the fp32 weights and their
+ *                               bf16 copies (in place, shard by shard)
+ * Every rank sums the same gathered partials in the same order, so the
+ * norm and the clip factor are identical on every rank. */
+
+/* Number of doubles gpt_grad_sumsq_shard writes. */
+#define GPT_NORM_PARTIALS 592
+
+/* Shard `rank` of `world` (1 <= world <= 64): elements [*offset, *offset +
+ * *count) of the arenas, *stride = the shard length every rank but the last
+ * has (a multiple of 64; world * *stride never exceeds the arenas'
+ * allocated length, so an all-gather of `world` equal shards fits in
+ * place).  *count is 0 for a rank past the end.  Pure host. */
+gpt_status gpt_zero1_shard(const gpt_config* cfg, int32_t world, int32_t rank, int64_t* offset, int64_t* count,
+                           int64_t* stride);
+/* Device addresses of the model's flat arenas (all with the same element
+ * offsets): fp32 weights, gradients, AdamW first and second moments, and the
+ * bf16 operand copy of the weights (null in fp32 mode).  *n_floats elements
+ * are in use; each arena is allocated for *n_alloc >= n_floats + 4096
+ * elements (the slack is never read by the step). */
+gpt_status gpt_state_arenas(gpt_model* m, float** d_param, float** d_grad, float** d_adam_m, float** d_adam_v,
+                            void** d_param_bf16, int64_t* n_floats, int64_t* n_alloc);
+/* GPT_NORM_PARTIALS partial sums of squares (fp64, device) of gradient
+ * elements [offset, offset + count) into d_partials; their sum is the
+ * shard's squared norm.  offset and count multiples of 4 (the shard bounds
+ * of gpt_zero1_shard are).  Asynchronous.  GPT_ERR_STATE with LoRA
+ * adapters attached. */
+gpt_status gpt_grad_sumsq_shard(gpt_model* m, int64_t offset, int64_t count, double* d_partials);
+/* Clip + AdamW (as gpt_clip_adamw_step) on elements [offset, offset + count)
+ * only, with the gradient taken as grad_scale times the arena's values (1 /
+ * world for the mean of summed gradients) and its global norm as grad_scale
+ * times the square root of the sum of the n_partials doubles at d_partials
+ * (device; every rank's gpt_grad_sumsq_shard output, gathered in rank
+ * order).  Clears the whole gradient arena.  h_grad_norm (nullable): the
+ * global norm, read after a synchronise (GPT_ERR_NONFINITE as
+ * gpt_clip_adamw_step).  With offset 0, count = the arena, grad_scale 1 and
+ * the one rank's partials this is gpt_clip_adamw_step bit for bit. */
+gpt_status gpt_clip_adamw_shard(gpt_model* m, float lr, int32_t step, int64_t offset, int64_t count,
+                                float grad_scale, const double* d_partials, int32_t n_partials, float* h_grad_norm);
+
 /* The batch gather of gpt_train_step on its own: writes int32
  * [batch_size, block_size] ids and targets to d_idx / d_tgt. */
 gpt_status gpt_gather_batch(gpt_model* m, const void* d_stream, uint64_t stream_len, uint64_t data_seed,

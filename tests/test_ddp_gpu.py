@@ -4,7 +4,15 @@ NCCL group: the exchange is then the identity, so the step must equal
 gpt_train_step bit for bit (losses, norms, weights), eager and replayed.
 This checks the split of the step, the bucket events and the stream
 ordering on the GPU; the mean over several ranks is checked on CPU with two
-gloo ranks (tests/test_ddp_host.py)."""
+gloo ranks (tests/test_ddp_host.py).
+
+The sharded optimiser (ZeroTrainer, ZeRO-1) is checked the same way on one
+rank, and with two ranks emulated on one GPU: two models take the two ranks'
+batches, the reduce-to-owner and the all-gathers are done with tensor copies
+between their arenas, each model runs gpt_grad_sumsq_shard /
+gpt_clip_adamw_shard on its own shard, and the result must equal, bit for
+bit, a third model that takes the mean gradient and the whole-arena
+gpt_clip_adamw_step (the data-parallel step)."""
 
 import os
 import socket
@@ -82,3 +90,80 @@ def test_one_rank_data_parallel_host_batches(group):
         m.close()
     assert res[0][0] == res[1][0]
     assert np.array_equal(res[0][1], res[1][1])
+
+
+@pytest.mark.parametrize("wname", ["char", "dropout"])
+def test_one_rank_zero1_step_equals_train_step(group, wname):
+    w, over = {"char": (W.CHAR, dict(n_layer=2, batch_size=4, block_size=128, grad_accum=2)),
+               "dropout": (W.DROPOUT_512, dict(n_layer=2, batch_size=2, block_size=256, grad_accum=2,
+                                               token_dtype=gb.GPT_TOK_I32))}[wname]
+    sd = torch.from_numpy(W.token_stream(w, n=1 << 16).astype(np.int32)).cuda()
+    res = []
+    for use_zero in (False, True):
+        m = gb.Model(gb.make_config(w, **over), seed=w.weight_seed)
+        tr = ddp.ZeroTrainer(m) if use_zero else None
+        out = []
+        for step in range(1, 6):
+            lr = gb.lr_cosine(w.lr, step - 1, 2, 6)
+            out.append(tr.step(sd, w.data_seed, lr, step) if use_zero else m.train_step(sd, w.data_seed, lr, step))
+        res.append((out, _weights(m)))
+        assert m.flags() == 0
+        m.close()
+    (l0, w0), (l1, w1) = res
+    assert l0 == l1
+    assert np.array_equal(w0, w1)
+
+
+def test_two_ranks_zero1_emulated_equal_the_data_parallel_step():
+    w = W.CHAR
+    over = dict(n_layer=2, batch_size=4, block_size=128, grad_accum=2)
+    cfg = gb.make_config(w, **over)
+    world = 2
+    A, B, C = (gb.Model(cfg, seed=w.weight_seed) for _ in range(3))
+    ar = [A.state_arenas(), B.state_arenas()]
+    ref = C.state_arenas()
+    n = ref["n"]
+    shards = [gb.zero1_shard(cfg, world, r) for r in range(world)]
+    stride = shards[0][2]
+    parts = [p for _, ps in ddp.shard_parts(ddp.bucket_plan(cfg), stride, world) for p in ps]
+    partials = [torch.zeros(gb.NORM_PARTIALS, dtype=torch.float64, device="cuda") for _ in range(world)]
+    for step in range(1, 4):
+        lr = 1e-3 * step
+        batches = [W.random_batch(w, 100 * step + r, 8, 128) for r in range(world)]
+        for mdl, (idx, tgt) in zip((A, B), batches):
+            mdl.train_step_host_accumulate(idx, tgt, step)
+        C.train_step_host_accumulate(*batches[0], step)
+        torch.cuda.synchronize()
+        gA, gB = ar[0]["grad"], ar[1]["grad"]
+        ref["grad"][:n].copy_((gA[:n] + gB[:n]) * 0.5)           # the data-parallel mean
+        for r, off, cnt in parts:                                  # the sum reduced to each part's owner
+            ar[r]["grad"][off:off + cnt] += ar[1 - r]["grad"][off:off + cnt]
+        for r, mdl in enumerate((A, B)):
+            mdl.grad_sumsq_shard(shards[r][0], shards[r][1], partials[r])
+        gathered = torch.cat(partials)
+        norms = [mdl.clip_adamw_shard(lr, step, shards[r][0], shards[r][1], 1.0 / world, gathered)
+                 for r, mdl in enumerate((A, B))]
+        for name in ("param", "param_bf16"):                       # the all-gathers
+            for r in range(world):
+                off, cnt, _ = shards[r]
+                ar[1 - r][name][off:off + cnt].copy_(ar[r][name][off:off + cnt])
+        norm_ref = C.clip_adamw_step(lr, step)
+        torch.cuda.synchronize()
+        # every rank sums the same gathered partials: one norm; the data-parallel
+        # step sums another partition of the same squares (fp64), which rounds to
+        # the same fp32 norm unless a last-bit tie falls differently
+        assert norms[0] == norms[1]
+        assert abs(norms[0] - norm_ref) <= 1e-6 * norm_ref
+        same = (lambda a, b: torch.equal(a, b)) if norms[0] == norm_ref else \
+            (lambda a, b: torch.allclose(a.float(), b.float(), rtol=1e-5 if a.dtype == torch.float32 else 8e-3,
+                                         atol=1e-7))
+        for r in range(world):
+            assert not ar[r]["grad"][:n].any()                     # the whole arena cleared
+            for name in ("param", "param_bf16"):
+                assert same(ar[r][name][:n], ref[name][:n]), (step, r, name)
+            off, cnt, _ = shards[r]
+            for name in ("adam_m", "adam_v"):                      # each owner's moments
+                assert same(ar[r][name][off:off + cnt], ref[name][off:off + cnt]), (step, r, name)
+    for mdl in (A, B, C):
+        assert mdl.flags() == 0
+        mdl.close()
