@@ -795,14 +795,19 @@ __global__ void k_embed_bwd_wpe(const float* __restrict__ dres, int Bn, int Tn, 
 // continues into the next chunk goes to tail[chunk].  Kernel B: for every
 // segment that starts in chunk c and continues, dwte[tok] += tail[c] + the
 // heads of the following chunks it covers, in chunk order.
+// Every load a thread needs is issued before the additions that use it: the
+// chunk's rows, then the dwte rows of all its inner segments (distinct tokens,
+// so the read-modify-writes are independent), then the sums and the stores.
 constexpr int EC = 32;
+enum : int8_t { SEG_NONE = 0, SEG_INNER = 1, SEG_HEAD = 2, SEG_TAIL = 3 };
 
-__global__ void __launch_bounds__(256) k_embed_seg_a(const float* __restrict__ dres, const int32_t* __restrict__ stok,
+__global__ void __launch_bounds__(256, 2) k_embed_seg_a(const float* __restrict__ dres, const int32_t* __restrict__ stok,
                                                      const int32_t* __restrict__ spos, int M, int d, DropKey drop,
                                                      float* __restrict__ dwte, float* __restrict__ head,
                                                      float* __restrict__ tail) {
   pdl_trigger();
   __shared__ int s_tok[EC + 2], s_pos[EC];
+  __shared__ int8_t s_kind[EC];  // what ends at slot k: nothing, an inner segment, the head, the tail
   drop = drop_live(drop);
   const int c = blockIdx.x;
   const int j0 = c * EC, j1 = min(M, j0 + EC);
@@ -816,34 +821,52 @@ __global__ void __launch_bounds__(256) k_embed_seg_a(const float* __restrict__ d
     s_tok[n + 1] = j1 < M ? stok[j1] : -1;
   }
   __syncthreads();
+  if (threadIdx.x < EC) {
+    const int k = threadIdx.x;
+    int8_t kind = SEG_NONE;
+    if (k < n) {
+      const int tok = s_tok[k + 1];
+      if (k == n - 1 || s_tok[k + 2] != tok) {  // a segment ends at slot k (or at the chunk edge)
+        // sorted slots: the segment reaches slot 0 iff slot 0 holds its token
+        const bool began_before = s_tok[1] == tok && s_tok[0] == tok;
+        const bool continues = k == n - 1 && s_tok[n + 1] == tok;
+        kind = began_before ? SEG_HEAD : continues ? SEG_TAIL : SEG_INNER;
+      }
+    }
+    s_kind[k] = kind;
+  }
+  __syncthreads();
   for (int col = threadIdx.x; col < d; col += blockDim.x) {
-    // the chunk's rows of this column, all loads issued before the sums
     float vals[EC];
 #pragma unroll
     for (int k = 0; k < EC; k++) vals[k] = k < n ? dres[(long)s_pos[k] * d + col] : 0.f;
+    // segment sums in slot order, left in vals[k] at the slot where each ends
     float acc = 0.f;
 #pragma unroll
     for (int k = 0; k < EC; k++) {
-      if (k >= n) break;
-      const long p = s_pos[k];
       float v = vals[k];
-      if (drop.active) v *= drop_mul(drop, (uint64_t)p * d + col);
+      if (drop.active && k < n) v *= drop_mul(drop, (uint64_t)s_pos[k] * d + col);
       acc += v;
-      const int tok = s_tok[k + 1];
-      if (k == n - 1 || s_tok[k + 2] != tok) {  // segment ends here (or at the chunk edge)
-        int seg_lo = k;
-        while (seg_lo > 0 && s_tok[seg_lo] == tok) seg_lo--;  // first slot of the segment in the chunk
-        const bool began_before = seg_lo == 0 && s_tok[0] == tok;
-        const bool continues = k == n - 1 && s_tok[n + 1] == tok;
-        if (began_before) head[(long)c * d + col] = acc;
-        else if (continues) tail[(long)c * d + col] = acc;
-        else dwte[(long)tok * d + col] += acc;
+      if (s_kind[k] != SEG_NONE) {
+        vals[k] = acc;
         acc = 0.f;
       }
+    }
+    float old[EC];
+#pragma unroll
+    for (int k = 0; k < EC; k++) old[k] = s_kind[k] == SEG_INNER ? dwte[(long)s_tok[k + 1] * d + col] : 0.f;
+#pragma unroll
+    for (int k = 0; k < EC; k++) {
+      const int kind = s_kind[k];
+      if (kind == SEG_INNER) dwte[(long)s_tok[k + 1] * d + col] = old[k] + vals[k];
+      else if (kind == SEG_HEAD) head[(long)c * d + col] = vals[k];
+      else if (kind == SEG_TAIL) tail[(long)c * d + col] = vals[k];
     }
   }
 }
 
+// threads across groups of four columns (d a multiple of 4); the heads are
+// loaded eight chunks at a time and added in chunk order
 __global__ void k_embed_seg_b(const int32_t* __restrict__ stok, int M, int d, const float* __restrict__ head,
                               const float* __restrict__ tail, float* __restrict__ dwte) {
   pdl_trigger();
@@ -851,9 +874,8 @@ __global__ void k_embed_seg_b(const int32_t* __restrict__ stok, int M, int d, co
   const int j0 = c * EC, j1 = min(M, j0 + EC);
   const int tok = stok[j1 - 1];
   if (j1 >= M || stok[j1] != tok) return;  // the chunk's last segment ends inside it
-  int k = j1 - 1;
-  while (k > j0 && stok[k - 1] == tok) k--;
-  if (k == j0 && j0 > 0 && stok[j0 - 1] == tok) return;  // began earlier: its start chunk sums it
+  // began earlier (its start chunk sums it): slot j0 holds the token and so does slot j0 - 1
+  if (j0 > 0 && stok[j0] == tok && stok[j0 - 1] == tok) return;
   // the last chunk cend whose head belongs to the segment: the first chunk
   // after c at whose end the token changes (or the stream ends), found by all
   // threads at once rather than one chunk after another
@@ -867,12 +889,37 @@ __global__ void k_embed_seg_b(const int32_t* __restrict__ stok, int M, int d, co
   }
   __syncthreads();
   const int cend = s_end < nch ? s_end : c;  // (the segment continues past c, so a later chunk ends it)
-  for (int col = threadIdx.x; col < d; col += blockDim.x) {
-    float s = tail[(long)c * d + col];
-    // the heads of chunks c+1 .. cend, added in chunk order (independent loads)
-#pragma unroll 4
-    for (int cc = c + 1; cc <= cend; cc++) s += head[(long)cc * d + col];
-    dwte[(long)tok * d + col] += s;
+  const int d4 = d >> 2;
+  const float4* __restrict__ h4 = reinterpret_cast<const float4*>(head);
+  for (int q = threadIdx.x; q < d4; q += blockDim.x) {
+    float4 s = reinterpret_cast<const float4*>(tail)[(long)c * d4 + q];
+    int cc = c + 1;
+    for (; cc + 8 <= cend + 1; cc += 8) {
+      float4 h[8];
+#pragma unroll
+      for (int u = 0; u < 8; u++) h[u] = h4[(long)(cc + u) * d4 + q];
+#pragma unroll
+      for (int u = 0; u < 8; u++) {
+        s.x += h[u].x;
+        s.y += h[u].y;
+        s.z += h[u].z;
+        s.w += h[u].w;
+      }
+    }
+    for (; cc <= cend; cc++) {
+      const float4 h = h4[(long)cc * d4 + q];
+      s.x += h.x;
+      s.y += h.y;
+      s.z += h.z;
+      s.w += h.w;
+    }
+    float4* dst = reinterpret_cast<float4*>(dwte + (long)tok * d) + q;
+    float4 o = *dst;
+    o.x += s.x;
+    o.y += s.y;
+    o.z += s.z;
+    o.w += s.w;
+    *dst = o;
   }
 }
 
