@@ -2,6 +2,7 @@
 // LayerNorm/RMSNorm, cross-entropy, column sums, embedding backward,
 // gradient norm and the fused clip + AdamW update.
 #include "kernels.cuh"
+#include "sm100.cuh"
 
 #include <math.h>
 
@@ -671,12 +672,147 @@ __global__ void __launch_bounds__(256, 4) k_ce_stream(T* __restrict__ logits, co
   }
 }
 
+// Rows staged in shared memory: one block per SM walks its rows with the
+// next row's bulk copy (TMA, cp.async.bulk) in flight while it works on the
+// current one, so each logit is read from HBM once: pass 1 (the row's
+// log-sum-exp) and pass 2 (softmax - onehot, written in place) both read the
+// staged copy.  The per-thread order of pass 1 is k_ce_stream's (256
+// threads, 16-byte vectors strided by the block), so the two give the same
+// bits.  Every wait is bounded; a block that gives up raises FLAG_TIMEOUT,
+// waits for its own copies in flight (again bounded) and returns.
+constexpr int CE_THREADS = 256;
+constexpr uint32_t CE_CHUNK = 32768;  // bytes per bulk copy
+
+template <typename T>
+__global__ void __launch_bounds__(CE_THREADS, 1) k_ce_smem(T* __restrict__ logits, const int32_t* __restrict__ tgt,
+                                                          long M, int V, int Vp, float* __restrict__ lse_out,
+                                                          float* __restrict__ row_loss, int want_grad, float scale,
+                                                          uint32_t* flags) {
+  pdl_trigger();
+  constexpr int EPV = 16 / sizeof(T);
+  constexpr float LOG2E = 1.4426950408889634f;
+  extern __shared__ __align__(128) uint8_t smem[];
+  __shared__ float sm[8], ss[8];
+  __shared__ __align__(8) uint64_t full[2];
+  __shared__ int abort_flag;
+  const uint32_t RB = (uint32_t)Vp * sizeof(T);  // row bytes (a multiple of 16)
+  const uint32_t RBA = (RB + 127) & ~127u;       // buffer stride
+  const int nvec = Vp / EPV;
+  int issued[2] = {0, 0}, waited[2] = {0, 0};    // copies per buffer (kept by thread 0)
+  auto issue = [&](long row, int b) {            // thread 0: the bulk copies of one row into buffer b
+    issued[b]++;
+    const uint32_t bar = sm100::smem_u32(&full[b]);
+    const uint32_t dst = sm100::smem_u32(smem + b * RBA);
+    const uint8_t* src = reinterpret_cast<const uint8_t*>(logits + row * Vp);
+    sm100::fence_proxy_async_smem();  // the buffer's earlier generic reads come first
+    sm100::mbar_expect_tx(bar, RB);
+    for (uint32_t o = 0; o < RB; o += CE_CHUNK) sm100::bulk_load(dst + o, src + o, min(CE_CHUNK, RB - o), bar);
+  };
+  if (threadIdx.x == 0) {
+    sm100::mbar_init(sm100::smem_u32(&full[0]), 1);
+    sm100::mbar_init(sm100::smem_u32(&full[1]), 1);
+    abort_flag = 0;
+    sm100::fence_barrier_init();
+    if (blockIdx.x < M) issue(blockIdx.x, 0);
+  }
+  __syncthreads();
+  int it = 0;
+  for (long row = blockIdx.x; row < M; row += gridDim.x, it++) {
+    const int b = it & 1;
+    if (threadIdx.x == 0 && row + gridDim.x < M) issue(row + gridDim.x, b ^ 1);
+    const bool ok = sm100::mbar_wait(sm100::smem_u32(&full[b]), (it >> 1) & 1, &abort_flag, flags);
+    if (__syncthreads_or(!ok)) break;  // every thread takes the same branch
+    waited[b]++;
+    const T* z = reinterpret_cast<const T*>(smem + b * RBA);
+    const int t = tgt[row];
+    float m = -INFINITY, s = 0.f;
+    for (int vi = threadIdx.x; vi < nvec; vi += CE_THREADS) {
+      uint4 u = reinterpret_cast<const uint4*>(z)[vi];
+      const T* e = reinterpret_cast<const T*>(&u);
+      float x[EPV];
+      float mv = -INFINITY;
+#pragma unroll
+      for (int k = 0; k < EPV; k++) {
+        x[k] = (vi * EPV + k < V) ? to_f<T>(e[k]) * LOG2E : -INFINITY;
+        mv = fmaxf(mv, x[k]);
+      }
+      if (mv > m) {
+        s = (m == -INFINITY) ? 0.f : s * sfu_ex2(m - mv);
+        m = mv;
+      }
+#pragma unroll
+      for (int k = 0; k < EPV; k++) s += sfu_ex2(x[k] - m);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      float m2 = __shfl_xor_sync(0xffffffffu, m, o);
+      float s2 = __shfl_xor_sync(0xffffffffu, s, o);
+      lse_merge(m, s, m2, s2);
+    }
+    const int w = threadIdx.x >> 5;
+    if ((threadIdx.x & 31) == 0) {
+      sm[w] = m;
+      ss[w] = s;
+    }
+    __syncthreads();
+    float Mx = sm[0], S = ss[0];
+#pragma unroll
+    for (int k = 1; k < 8; k++) lse_merge(Mx, S, sm[k], ss[k]);
+    const float lse2 = Mx + log2f(S);  // log2-domain log-sum-exp
+    const float lse = lse2 * 0.6931471805599453f;
+    if (threadIdx.x == 0) {
+      lse_out[row] = lse;
+      row_loss[row] = lse - to_f<T>(z[t]);
+    }
+    if (want_grad) {
+      uint4* dst = reinterpret_cast<uint4*>(logits + row * Vp);
+      for (int vi = threadIdx.x; vi < nvec; vi += CE_THREADS) {
+        uint4 u = reinterpret_cast<const uint4*>(z)[vi];
+        const T* e = reinterpret_cast<const T*>(&u);
+        uint4 outv;
+        T* o = reinterpret_cast<T*>(&outv);
+#pragma unroll
+        for (int k = 0; k < EPV; k++) {
+          const int j = vi * EPV + k;
+          float g = 0.f;
+          if (j < V) g = (sfu_ex2(fmaf(to_f<T>(e[k]), LOG2E, -lse2)) - (j == t ? 1.f : 0.f)) * scale;
+          o[k] = from_f<T>(g);
+        }
+        dst[vi] = outv;
+      }
+    }
+    __syncthreads();  // the buffer and sm / ss are free again
+  }
+  if (threadIdx.x == 0) {
+    // after a failed wait: no copy of this block may still be writing its
+    // shared memory when it exits (bounded waits, which ignore the abort flag)
+    volatile int no_abort = 0;
+    for (int k = 0; k < 2; k++)
+      for (; waited[k] < issued[k]; waited[k]++)
+        if (!sm100::mbar_wait(sm100::smem_u32(&full[k]), waited[k] & 1, &no_abort, flags, 100000000ull)) break;
+  }
+}
+
+// shared memory of k_ce_smem for rows of `row_bytes` (0: the row does not fit)
+size_t ce_smem_bytes(size_t row_bytes) {
+  if (row_bytes % 16) return 0;
+  const size_t b = 2 * ((row_bytes + 127) & ~size_t(127));
+  return b <= 220 * 1024 ? b : 0;
+}
+
 template <typename T>
 void ce_fwd_bwd(Ctx& c, T* logits, const int32_t* tgt, long M, int V, int Vp, float* lse, float* row_loss,
                 bool want_grad, float scale) {
   LaunchScope s(c, want_grad ? "ce_fwd_bwd" : "ce_fwd");
   constexpr int EPV = 16 / sizeof(T);
-  if (Vp % EPV == 0)
+  const size_t sh = ce_smem_bytes((size_t)Vp * sizeof(T));
+  if (Vp % EPV == 0 && sh > 0) {
+    // per-device function attribute: set before every launch
+    cudaFuncSetAttribute(k_ce_smem<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sh);
+    const unsigned grid = (unsigned)std::min<long>(M, c.num_sms);
+    k_ce_smem<T><<<grid, CE_THREADS, sh, c.stream>>>(logits, tgt, M, V, Vp, lse, row_loss, want_grad ? 1 : 0, scale,
+                                                     c.flags);
+  } else if (Vp % EPV == 0)
     k_ce_stream<T><<<(unsigned)M, 256, 0, c.stream>>>(logits, tgt, V, Vp, lse, row_loss, want_grad ? 1 : 0, scale);
   else
     k_ce<T><<<(unsigned)M, 512, 0, c.stream>>>(logits, tgt, V, Vp, lse, row_loss, want_grad ? 1 : 0, scale);
