@@ -676,11 +676,13 @@ __global__ void __launch_bounds__(256, 4) k_ce_stream(T* __restrict__ logits, co
 // next row's bulk copy (TMA, cp.async.bulk) in flight while it works on the
 // current one, so each logit is read from HBM once: pass 1 (the row's
 // log-sum-exp) and pass 2 (softmax - onehot, written in place) both read the
-// staged copy.  The per-thread order of pass 1 is k_ce_stream's (256
-// threads, 16-byte vectors strided by the block), so the two give the same
-// bits.  Every wait is bounded; a block that gives up raises FLAG_TIMEOUT,
-// waits for its own copies in flight (again bounded) and returns.
-constexpr int CE_THREADS = 256;
+// staged copy.  The arithmetic is k_ce_stream's (16-byte vectors strided
+// over the block's threads, an online (max, sum) per thread, then warp and
+// block merges in a fixed order) on 512 threads: two exponentials per logit
+// keep the SFU busy, and 16 warps per SM hide its latency.  Every wait is
+// bounded; a block that gives up raises FLAG_TIMEOUT, waits for its own
+// copies in flight (again bounded) and returns.
+constexpr int CE_THREADS = 512;
 constexpr uint32_t CE_CHUNK = 32768;  // bytes per bulk copy
 
 template <typename T>
@@ -692,7 +694,7 @@ __global__ void __launch_bounds__(CE_THREADS, 1) k_ce_smem(T* __restrict__ logit
   constexpr int EPV = 16 / sizeof(T);
   constexpr float LOG2E = 1.4426950408889634f;
   extern __shared__ __align__(128) uint8_t smem[];
-  __shared__ float sm[8], ss[8];
+  __shared__ float sm[CE_THREADS / 32], ss[CE_THREADS / 32];
   __shared__ __align__(8) uint64_t full[2];
   __shared__ int abort_flag;
   const uint32_t RB = (uint32_t)Vp * sizeof(T);  // row bytes (a multiple of 16)
@@ -757,7 +759,7 @@ __global__ void __launch_bounds__(CE_THREADS, 1) k_ce_smem(T* __restrict__ logit
     __syncthreads();
     float Mx = sm[0], S = ss[0];
 #pragma unroll
-    for (int k = 1; k < 8; k++) lse_merge(Mx, S, sm[k], ss[k]);
+    for (int k = 1; k < CE_THREADS / 32; k++) lse_merge(Mx, S, sm[k], ss[k]);
     const float lse2 = Mx + log2f(S);  // log2-domain log-sum-exp
     const float lse = lse2 * 0.6931471805599453f;
     if (threadIdx.x == 0) {
