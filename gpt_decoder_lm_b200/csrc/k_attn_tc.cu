@@ -322,263 +322,6 @@ __device__ __forceinline__ uint32_t pack2v(uint64_t v) {
   return pack2(f.x, f.y);
 }
 
-// ============================================================================
-// forward with eight softmax warps: as k_attn_fwd_o, but two warps per TMEM
-// lane quadrant, each taking 32 of a 64-key block's columns (half 0: keys
-// 0..31, half 1: keys 32..63).  The two warps of a quadrant exchange their
-// half-row maxima through shared memory (named barrier 1 + quadrant, 64
-// threads) and so take the same reference maximum and rescale decisions;
-// each keeps the row sum of its own columns, summed at the end.  P of a half
-// is written as bf16 pairs inside that half's own S columns (the other half's
-// S is never overwritten before it is read), so the P V product reads its A
-// operand at acol().  A wait that fails is carried to the next exchange, where
-// both warps of the quadrant leave the loop together.
-// smem: Q | (K, V)[3 stages] | barriers | exchange   (64 KB + 1.3 KB)
-// ============================================================================
-constexpr int D8_X = D_BAR + 256;      // float xm[2 slots][4 quads][2 halves][32]
-constexpr int D8_XL = D8_X + 2048;     // float xl[4][2][32]
-constexpr int D8_XK = D8_XL + 1024;    // int xk[2 slots][4][2]
-constexpr int D8_SMEM = D8_XK + 128;      // int xk[2][4][2] | the final exchange's [4][2]
-
-__device__ __forceinline__ void pair_sync(int quad) {  // barrier ids as constants: five in use
-  switch (quad) {
-    case 0: asm volatile("bar.sync 1, 64;" ::: "memory"); break;
-    case 1: asm volatile("bar.sync 2, 64;" ::: "memory"); break;
-    case 2: asm volatile("bar.sync 3, 64;" ::: "memory"); break;
-    default: asm volatile("bar.sync 4, 64;" ::: "memory"); break;
-  }
-}
-
-template <bool DROP>
-__global__ void __launch_bounds__(320, 2) k_attn_fwd_o8(const __grid_constant__ CUtensorMap tq,
-                                                        const __grid_constant__ CUtensorMap tkv64, AttnTcArgs a) {
-  pdl_trigger();
-  const DropKey dk = DROP ? drop_live(a.drop) : a.drop;
-  extern __shared__ __align__(1024) uint8_t smem[];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if (smem_u32(smem) & 1023) {
-    if (threadIdx.x == 0) atomicOr(a.flags, FLAG_TIMEOUT);
-    return;
-  }
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + D_BAR);
-  const uint32_t q_full = smem_u32(bars + 0);
-  const uint32_t kv_full0 = smem_u32(bars + 1), kv_empty0 = smem_u32(bars + 1 + D_STAGES);
-  const uint32_t s_full0 = smem_u32(bars + 1 + 2 * D_STAGES), p_full0 = s_full0 + 16, pv_done0 = s_full0 + 32;
-  uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + 7 + 2 * D_STAGES);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(tslot + 1);
-  float* xm = reinterpret_cast<float*>(smem + D8_X);
-  float* xl = reinterpret_cast<float*>(smem + D8_XL);
-  volatile int* xk = reinterpret_cast<volatile int*>(smem + D8_XK);
-  const uint32_t sb = smem_u32(smem);
-
-  const int nqb = a.T / 128;
-  const int qb = nqb - 1 - (int)blockIdx.y;
-  const int bh = blockIdx.x, b = bh / a.H, h = bh % a.H;
-  const int nkb = 2 * (qb + 1);
-  const int row0 = b * a.T;
-
-  if (threadIdx.x == 0) {
-    mbar_init(q_full, 1);
-    for (int s = 0; s < D_STAGES; s++) {
-      mbar_init(kv_full0 + 8 * s, 1);
-      mbar_init(kv_empty0 + 8 * s, 1);
-    }
-    for (int u = 0; u < 2; u++) {
-      mbar_init(s_full0 + 8 * u, 1);
-      mbar_init(p_full0 + 8 * u, 8);
-      mbar_init(pv_done0 + 8 * u, 1);
-    }
-    *abort_flag = 0;
-    fence_barrier_init();
-    prefetch_tmap(&tq);
-    prefetch_tmap(&tkv64);
-  }
-  if (warp == 1) {
-    tmem_alloc(smem_u32(tslot), 256);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tslot;
-
-  if (warp == 0) {
-    if (lane == 0) {
-      mbar_expect_tx(q_full, TILE);
-      tma_load_3d(sb + D_Q, &tq, q_full, 0, h, row0 + qb * 128);
-      for (int j = 0; j < nkb; j++) {
-        const int s = j % D_STAGES;
-        const uint32_t fb = kv_full0 + 8 * s;
-        if (!mbar_wait(kv_empty0 + 8 * s, ((j / D_STAGES) & 1) ^ 1, abort_flag, a.flags)) break;
-        mbar_expect_tx(fb, 2 * HTILE);
-        tma_load_3d(sb + D_KV + s * TILE, &tkv64, fb, 0, a.H + h, row0 + j * 64);
-        tma_load_3d(sb + D_KV + s * TILE + HTILE, &tkv64, fb, 0, 2 * a.H + h, row0 + j * 64);
-      }
-    }
-  } else if (warp == 1) {
-    if (lane == 0) {
-      constexpr uint32_t id_n64 = idesc_bf16_f32(128, 64, false, false);
-      constexpr uint32_t id_pv = idesc_bf16_f32(128, 64, false, true);
-      bool ok = mbar_wait(q_full, 0, abort_flag, a.flags);
-      auto issue_pv = [&](int i) -> bool {
-        const int u = i & 1;
-        if (!mbar_wait(p_full0 + 8 * u, (i >> 1) & 1, abort_flag, a.flags)) return false;
-        tc_fence_after();
-        const uint32_t v = sb + D_KV + (i % D_STAGES) * TILE + HTILE;
-#pragma unroll
-        for (int kk = 0; kk < 4; kk++)
-          mma_bf16_ts(tmem + 128, tmem + 64 * u + acol(kk), desc_mn64(v, kk), id_pv, (i > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(pv_done0 + 8 * u);
-        mma_commit(kv_empty0 + 8 * (i % D_STAGES));
-        return true;
-      };
-      for (int j = 0; j < nkb && ok; j++) {
-        const int s = j % D_STAGES;
-        if (!(ok = mbar_wait(kv_full0 + 8 * s, (j / D_STAGES) & 1, abort_flag, a.flags))) break;
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < 4; kk++)
-          mma_bf16_ss(tmem + 64 * (j & 1), desc_k(sb + D_Q, TILE, kk), desc_k(sb + D_KV + s * TILE, HTILE, kk), id_n64,
-                      kk > 0);
-        mma_commit(s_full0 + 8 * (j & 1));
-        if (j >= 1 && !(ok = issue_pv(j - 1))) break;
-      }
-      if (ok) issue_pv(nkb - 1);
-    }
-  } else {
-    const int quad = warp & 3;
-    const int half = (warp - 2) >> 2;  // warps 2..5: keys 0..31 of a block, 6..9: keys 32..63
-    const int r = quad * 32 + lane;
-    const int qi = qb * 128 + r;
-    const uint32_t trow = tmem + ((uint32_t)(quad * 32) << 16);
-    const float sl2 = a.scale_log2;
-    const int c0 = 32 * half;
-    float m = -INFINITY, l = 0.f;  // reference maximum (log2 units, the row's) and this half's row sum
-    const uint64_t ebase = ((uint64_t)bh * a.T + qi) * a.T;
-    bool ok = true;
-    for (int j = 0; j < nkb; j++) {
-      const int u = j & 1;
-      ok = ok && mbar_wait(s_full0 + 8 * u, (j >> 1) & 1, abort_flag, a.flags);
-      ok = __all_sync(0xffffffffu, ok);
-      const int key0 = j * 64;
-      const int lim = qi - key0 - c0;  // column i of this half is visible iff i <= lim
-      uint32_t v[32];
-      float hm = -INFINITY;
-      if (ok) {
-        tc_fence_after();
-        tmem_ld_32x32b_x32(trow + 64 * u + c0, v);
-        tmem_ld_wait();
-        if (lim >= 31) {
-          float mx0 = -INFINITY, mx1 = -INFINITY;
-#pragma unroll
-          for (int i = 0; i < 32; i += 2) {
-            mx0 = fmaxf(mx0, __uint_as_float(v[i]));
-            mx1 = fmaxf(mx1, __uint_as_float(v[i + 1]));
-          }
-          hm = fmaxf(mx0, mx1);
-        } else {
-#pragma unroll
-          for (int i = 0; i < 32; i++)
-            if (i <= lim) hm = fmaxf(hm, __uint_as_float(v[i]));
-        }
-      }
-      // the two halves' maxima (and wait outcomes) through shared memory
-      const int xs = (j & 1) * 8 + quad * 2;
-      xm[(xs + half) * 32 + lane] = hm;
-      if (lane == 0) xk[xs + half] = ok ? 1 : 0;
-      pair_sync(quad);
-      const float om = xm[(xs + (half ^ 1)) * 32 + lane];
-      if (!(ok && xk[xs + (half ^ 1)] != 0)) {
-        ok = false;  // both warps of the quadrant leave here
-        break;
-      }
-      const float bm = (half == 0 ? fmaxf(hm, om) : fmaxf(om, hm)) * sl2;
-      if (j == 0) {
-        m = bm;  // key 0 is visible to every row, so m is finite from here on
-      } else {
-        const bool need = bm > m + RESCALE_LOG2;
-        if (__any_sync(0xffffffffu, need)) {
-          // P V of block j-1 is the only product that may still be in flight
-          bool okr = mbar_wait(pv_done0 + 8 * ((j - 1) & 1), ((j - 1) >> 1) & 1, abort_flag, a.flags);
-          okr = __all_sync(0xffffffffu, okr);
-          if (okr) {
-            tc_fence_after();
-            const float sc = need ? ex2(m - bm) : 1.f;
-            uint32_t o[32];
-            tmem_ld_32x32b_x32(trow + 128 + c0, o);
-            tmem_ld_wait();
-            uint32_t w[16];
-#pragma unroll
-            for (int h2 = 0; h2 < 2; h2++) {
-#pragma unroll
-              for (int i = 0; i < 16; i++) w[i] = __float_as_uint(__uint_as_float(o[16 * h2 + i]) * sc);
-              tmem_st_32x32b_x16(trow + 128 + c0 + 16 * h2, w);
-            }
-            l *= sc;
-            if (need) m = bm;
-          } else {
-            ok = false;  // carried to the next exchange
-          }
-        }
-      }
-      float ls = 0.f;
-      uint32_t pk[16];
-#pragma unroll
-      for (int i = 0; i < 32; i += 2) {
-        float p0 = ex2(fmaf(__uint_as_float(v[i]), sl2, -m));
-        float p1 = ex2(fmaf(__uint_as_float(v[i + 1]), sl2, -m));
-        if (lim < 31) {
-          if (i > lim) p0 = 0.f;
-          if (i + 1 > lim) p1 = 0.f;
-        }
-        ls += p0 + p1;
-        if (DROP) {
-          const uint64_t e = ebase + key0 + c0 + i;
-          p0 *= drop_mul(dk, e);
-          p1 *= drop_mul(dk, e + 1);
-        }
-        pk[i >> 1] = pack2(p0, p1);
-      }
-      // P (bf16 pairs) inside this half's own S columns: the A operand of P V
-      if (ok) tmem_st_32x32b_x16(trow + 64 * u + c0, pk);
-      l += ls;
-      tmem_st_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(p_full0 + 8 * u);  // one arrival per softmax warp
-    }
-    // the last two P V products may both be in flight
-    if (ok) ok = mbar_wait(pv_done0 + 8 * (nkb & 1), ((nkb - 2) >> 1) & 1, abort_flag, a.flags);
-    if (ok) ok = mbar_wait(pv_done0 + 8 * ((nkb - 1) & 1), ((nkb - 1) >> 1) & 1, abort_flag, a.flags);
-    ok = __all_sync(0xffffffffu, ok);
-    xl[(quad * 2 + half) * 32 + lane] = l;
-    if (lane == 0) xk[16 + quad * 2 + half] = ok ? 1 : 0;
-    pair_sync(quad);
-    const float lt = xl[(quad * 2) * 32 + lane] + xl[(quad * 2 + 1) * 32 + lane];
-    if (ok && xk[16 + quad * 2 + (half ^ 1)] != 0) {
-      tc_fence_after();
-      uint32_t o[32];
-      tmem_ld_32x32b_x32(trow + 128 + c0, o);
-      tmem_ld_wait();
-      const float inv = 1.0f / lt;
-      uint4* dst = reinterpret_cast<uint4*>(a.o_out + ((size_t)(row0 + qi) * a.H + h) * 64 + c0);
-#pragma unroll
-      for (int q = 0; q < 4; q++) {
-        const uint32_t* x = o + 8 * q;
-        dst[q] = make_uint4(pack2(__uint_as_float(x[0]) * inv, __uint_as_float(x[1]) * inv),
-                            pack2(__uint_as_float(x[2]) * inv, __uint_as_float(x[3]) * inv),
-                            pack2(__uint_as_float(x[4]) * inv, __uint_as_float(x[5]) * inv),
-                            pack2(__uint_as_float(x[6]) * inv, __uint_as_float(x[7]) * inv));
-      }
-      if (half == 0) a.lse[(size_t)bh * a.T + qi] = (m + log2f(lt)) * LN2;
-    }
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  if (warp == 1) tmem_dealloc(tmem, 256);
-}
-
 // Column sums of a warp's 32 rows (one per lane) x 32 columns (v[c] in lane
 // order): a butterfly in which each step hands half of a lane's columns to its
 // partner, so lane c ends with the sum of column c (31 shuffles, fixed order).
@@ -1189,20 +932,6 @@ bool attn_fwd_tc(Ctx& c, const AttnDesc& d) {
   LaunchScope s(c, "attn_fwd_tc");
   if (drop) k_attn_fwd_o<true><<<grid, 192, D_SMEM, c.stream>>>(tq, tkv64, make_args(d, c.flags));
   else k_attn_fwd_o<false><<<grid, 192, D_SMEM, c.stream>>>(tq, tkv64, make_args(d, c.flags));
-  return true;
-}
-
-bool attn_fwd_tc8(Ctx& c, const AttnDesc& d) {
-  CUtensorMap tq, tkv64;
-  long rows = (long)d.B * d.T;
-  if (!map_rows(&tq, d.qkv, 3 * d.H, rows, 128) || !map_rows(&tkv64, d.qkv, 3 * d.H, rows, 64)) return false;
-  const bool drop = d.drop.active;
-  cudaFuncSetAttribute(drop ? k_attn_fwd_o8<true> : k_attn_fwd_o8<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                       D8_SMEM);
-  dim3 grid(d.B * d.H, d.T / 128);
-  LaunchScope s(c, "attn_fwd_tc");
-  if (drop) k_attn_fwd_o8<true><<<grid, 320, D8_SMEM, c.stream>>>(tq, tkv64, make_args(d, c.flags));
-  else k_attn_fwd_o8<false><<<grid, 320, D8_SMEM, c.stream>>>(tq, tkv64, make_args(d, c.flags));
   return true;
 }
 

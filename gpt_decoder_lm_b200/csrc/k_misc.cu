@@ -678,11 +678,45 @@ __global__ void __launch_bounds__(256, 4) k_ce_stream(T* __restrict__ logits, co
 // log-sum-exp) and pass 2 (softmax - onehot, written in place) both read the
 // staged copy.  The arithmetic is k_ce_stream's (16-byte vectors strided
 // over the block's threads, an online (max, sum) per thread, then warp and
-// block merges in a fixed order) on 512 threads: two exponentials per logit
-// keep the SFU busy, and 16 warps per SM hide its latency.  Every wait is
+// block merges in a fixed order) on 512 threads, with fewer instructions per
+// logit: bf16 widened by bit shifts, the vocabulary mask and the one-hot
+// term only where they can apply, exponents and scaling as paired (f32x2)
+// operations, two running sums per thread.  Every wait is
 // bounded; a block that gives up raises FLAG_TIMEOUT, waits for its own
 // copies in flight (again bounded) and returns.
 constexpr int CE_THREADS = 512;
+
+// a 16-byte vector of logits as floats (bf16 widened exactly by bit shifts),
+// and back (round to nearest)
+template <typename T>
+__device__ __forceinline__ void ce_unpack(const uint4& u, float (&x)[16 / sizeof(T)]) {
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+  if constexpr (sizeof(T) == 2) {
+#pragma unroll
+    for (int k = 0; k < 4; k++) {
+      x[2 * k] = __uint_as_float(w[k] << 16);
+      x[2 * k + 1] = __uint_as_float(w[k] & 0xffff0000u);
+    }
+  } else {
+#pragma unroll
+    for (int k = 0; k < 4; k++) x[k] = __uint_as_float(w[k]);
+  }
+}
+template <typename T>
+__device__ __forceinline__ uint4 ce_pack(const float (&g)[16 / sizeof(T)]) {
+  uint32_t w[4];
+  if constexpr (sizeof(T) == 2) {
+#pragma unroll
+    for (int k = 0; k < 4; k++) {
+      const __nv_bfloat162 v = __floats2bfloat162_rn(g[2 * k], g[2 * k + 1]);
+      w[k] = *reinterpret_cast<const uint32_t*>(&v);
+    }
+  } else {
+#pragma unroll
+    for (int k = 0; k < 4; k++) w[k] = __float_as_uint(g[k]);
+  }
+  return make_uint4(w[0], w[1], w[2], w[3]);
+}
 constexpr uint32_t CE_CHUNK = 32768;  // bytes per bulk copy
 
 template <typename T>
@@ -726,25 +760,43 @@ __global__ void __launch_bounds__(CE_THREADS, 1) k_ce_smem(T* __restrict__ logit
     if (__syncthreads_or(!ok)) break;  // every thread takes the same branch
     waited[b]++;
     const T* z = reinterpret_cast<const T*>(smem + b * RBA);
+    const uint4* z4 = reinterpret_cast<const uint4*>(z);
     const int t = tgt[row];
-    float m = -INFINITY, s = 0.f;
+    const int vfull = V / EPV;  // vectors below it lie inside the vocabulary
+    const uint64_t l2 = f2(LOG2E, LOG2E);
+    // pass 1: online (max, sum) of 2^(z log2 e), masks only in the last vectors,
+    // the exponents as paired FMAs, two running sums
+    float m = -INFINITY, s0 = 0.f, s1 = 0.f;
     for (int vi = threadIdx.x; vi < nvec; vi += CE_THREADS) {
-      uint4 u = reinterpret_cast<const uint4*>(z)[vi];
-      const T* e = reinterpret_cast<const T*>(&u);
+      if (vi * EPV >= V) continue;
       float x[EPV];
-      float mv = -INFINITY;
+      ce_unpack<T>(z4[vi], x);
+      if (vi >= vfull) {
 #pragma unroll
-      for (int k = 0; k < EPV; k++) {
-        x[k] = (vi * EPV + k < V) ? to_f<T>(e[k]) * LOG2E : -INFINITY;
-        mv = fmaxf(mv, x[k]);
+        for (int k = 0; k < EPV; k++)
+          if (vi * EPV + k >= V) x[k] = -INFINITY;
       }
+      float mv = x[0];
+#pragma unroll
+      for (int k = 1; k < EPV; k++) mv = fmaxf(mv, x[k]);
+      mv *= LOG2E;
       if (mv > m) {
-        s = (m == -INFINITY) ? 0.f : s * sfu_ex2(m - mv);
+        if (m != -INFINITY) {
+          const float r = sfu_ex2(m - mv);
+          s0 *= r;
+          s1 *= r;
+        }
         m = mv;
       }
+      const uint64_t nm = f2(-m, -m);
 #pragma unroll
-      for (int k = 0; k < EPV; k++) s += sfu_ex2(x[k] - m);
+      for (int k = 0; k < EPV; k += 2) {
+        const float2 y = f2split(f2fma(f2(x[k], x[k + 1]), l2, nm));
+        s0 += sfu_ex2(y.x);
+        s1 += sfu_ex2(y.y);
+      }
     }
+    float s = s0 + s1;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
       float m2 = __shfl_xor_sync(0xffffffffu, m, o);
@@ -767,20 +819,36 @@ __global__ void __launch_bounds__(CE_THREADS, 1) k_ce_smem(T* __restrict__ logit
       row_loss[row] = lse - to_f<T>(z[t]);
     }
     if (want_grad) {
+      // pass 2: (2^(z log2 e - lse2) - [j == t]) * scale, zero past the vocabulary
       uint4* dst = reinterpret_cast<uint4*>(logits + row * Vp);
+      const uint64_t nl = f2(-lse2, -lse2), sc2 = f2(scale, scale);
+      const int tv = t / EPV;
       for (int vi = threadIdx.x; vi < nvec; vi += CE_THREADS) {
-        uint4 u = reinterpret_cast<const uint4*>(z)[vi];
-        const T* e = reinterpret_cast<const T*>(&u);
-        uint4 outv;
-        T* o = reinterpret_cast<T*>(&outv);
+        float x[EPV], g[EPV];
+        ce_unpack<T>(z4[vi], x);
 #pragma unroll
-        for (int k = 0; k < EPV; k++) {
-          const int j = vi * EPV + k;
-          float g = 0.f;
-          if (j < V) g = (sfu_ex2(fmaf(to_f<T>(e[k]), LOG2E, -lse2)) - (j == t ? 1.f : 0.f)) * scale;
-          o[k] = from_f<T>(g);
+        for (int k = 0; k < EPV; k += 2) {
+          const float2 y = f2split(f2fma(f2(x[k], x[k + 1]), l2, nl));
+          g[k] = sfu_ex2(y.x);
+          g[k + 1] = sfu_ex2(y.y);
         }
-        dst[vi] = outv;
+        if (vi == tv) {
+#pragma unroll
+          for (int k = 0; k < EPV; k++)
+            if (vi * EPV + k == t) g[k] -= 1.f;
+        }
+#pragma unroll
+        for (int k = 0; k < EPV; k += 2) {
+          const float2 q = f2split(f2mul(f2(g[k], g[k + 1]), sc2));
+          g[k] = q.x;
+          g[k + 1] = q.y;
+        }
+        if (vi >= vfull) {
+#pragma unroll
+          for (int k = 0; k < EPV; k++)
+            if (vi * EPV + k >= V) g[k] = 0.f;
+        }
+        dst[vi] = ce_pack<T>(g);
       }
     }
     __syncthreads();  // the buffer and sm / ss are free again

@@ -144,7 +144,6 @@ bool attn_tc_shape_ok(int T, int hd);
 bool attn_tc_supported(const AttnDesc& a);  // shape rule plus 16-byte aligned pointers
 // false: a tensor map could not be encoded (nothing launched)
 bool attn_fwd_tc(Ctx& c, const AttnDesc& a);
-bool attn_fwd_tc8(Ctx& c, const AttnDesc& a);  // eight softmax warps per CTA
 bool attn_bwd_tc(Ctx& c, const AttnDesc& a);
 // decoding: o [B, H*hd] = attention of position t against positions 0..t of
 // the cache qkv [B, T, 3, H, hd]

@@ -72,11 +72,11 @@ extern "C" gpt_status gpt_test_attention(int32_t backend, int32_t backward, int3
   c.stream = (cudaStream_t)stream;
   c.flags = d_flags;
   AttnDesc a{B, T, H, hd, qkv, o, lse, dout, dqkv, dsum, make_drop_key(seed, counter, layer, 1, p)};
-  if (colsum && !(backward && (backend == 1 || backend == 2))) return GPT_ERR_INVALID_ARG;
+  if (colsum && !(backward && backend == 1)) return GPT_ERR_INVALID_ARG;
   a.colsum = colsum;
-  if (backend == 1 || backend == 2) {
+  if (backend == 1) {
     if (dtype != 1 || !attn_tc_supported(a)) return GPT_ERR_UNSUPPORTED;
-    if (!(backward ? attn_bwd_tc(c, a) : backend == 2 ? attn_fwd_tc8(c, a) : attn_fwd_tc(c, a))) return GPT_ERR_CUDA;
+    if (!(backward ? attn_bwd_tc(c, a) : attn_fwd_tc(c, a))) return GPT_ERR_CUDA;
   } else if (backend == 0) {
     if (hd != 4 && hd != 8 && hd != 16 && hd != 32 && hd != 64 && hd != 128) return GPT_ERR_UNSUPPORTED;
     if (dtype == 1) {

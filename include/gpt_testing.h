@@ -53,9 +53,8 @@ gpt_status gpt_test_gemm(int32_t backend, int32_t M, int32_t N, int32_t K, const
 /* Causal attention of one layer.  qkv [B, T, 3, H, hd], o [B, T, H, hd],
  * lse fp32 [B, H, T]; backward also takes dout [B, T, H, hd] and writes
  * dqkv [B, T, 3, H, hd] using dsum fp32 [B, H, T] as scratch.  dtype: 0 fp32,
- * 1 bf16.  backend: 0 CUDA cores, 1 tensor cores, 2 tensor cores with the
- * forward kernel of eight softmax warps per CTA (GPT_ERR_UNSUPPORTED when
- * the shape is not supported).  colsum (nullable; backward of backends 1, 2):
+ * 1 bf16.  backend: 0 CUDA cores, 1 tensor cores (GPT_ERR_UNSUPPORTED when
+ * the shape is not supported).  colsum (nullable; backward of backend 1):
  * fp32 [B T / 128, 3 H hd] receives the column sums of the stored dqkv over
  * each 128-row block.  Dropout on the probabilities with
  * (p, seed, counter, layer) as in the model (site 1); p = 0 disables it. */
