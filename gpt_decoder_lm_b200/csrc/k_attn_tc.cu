@@ -95,11 +95,10 @@ template <bool DROP>
 __global__ void __launch_bounds__(192, 2) k_attn_fwd_o(const __grid_constant__ CUtensorMap tq,
                                                        const __grid_constant__ CUtensorMap tkv64, AttnTcArgs a) {
   pdl_trigger();
-  // the dropout key of this launch (derived from the device step index in a replayed graph)
-  const DropKey dk = DROP ? drop_live(a.drop) : a.drop;
   extern __shared__ __align__(1024) uint8_t smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (smem_u32(smem) & 1023) {  // swizzled tiles need 1024-byte alignment
+    pdl_wait();
     if (threadIdx.x == 0) atomicOr(a.flags, FLAG_TIMEOUT);
     return;
   }
@@ -144,6 +143,10 @@ __global__ void __launch_bounds__(192, 2) k_attn_fwd_o(const __grid_constant__ C
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tslot;
+  // predecessor kernels complete from here on (programmatic dependent launch);
+  // the dropout key of this launch (derived from the device step index in a replayed graph)
+  pdl_wait();
+  const DropKey dk = DROP ? drop_live(a.drop) : a.drop;
 
   if (warp == 0) {
     if (lane == 0) {
@@ -385,11 +388,10 @@ __global__ void __launch_bounds__(320, 2) k_attn_bwd_kv8(const __grid_constant__
                                                          const __grid_constant__ CUtensorMap tq64,
                                                          const __grid_constant__ CUtensorMap tdo64, AttnTcArgs a) {
   pdl_trigger();
-  // the dropout key of this launch (derived from the device step index in a replayed graph)
-  const DropKey dk = DROP ? drop_live(a.drop) : a.drop;
   extern __shared__ __align__(1024) uint8_t smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (smem_u32(smem) & 1023) {
+    pdl_wait();
     if (threadIdx.x == 0) atomicOr(a.flags, FLAG_TIMEOUT);
     return;
   }
@@ -435,6 +437,10 @@ __global__ void __launch_bounds__(320, 2) k_attn_bwd_kv8(const __grid_constant__
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tslot;
+  // predecessor kernels complete from here on (programmatic dependent launch);
+  // the dropout key of this launch (derived from the device step index in a replayed graph)
+  pdl_wait();
+  const DropKey dk = DROP ? drop_live(a.drop) : a.drop;
 
   if (warp == 0) {
     if (lane == 0) {
@@ -643,11 +649,10 @@ __global__ void __launch_bounds__(320, 2) k_attn_bwd_q8(const __grid_constant__ 
                                                         const __grid_constant__ CUtensorMap tkv64,
                                                         const __grid_constant__ CUtensorMap tout, AttnTcArgs a) {
   pdl_trigger();
-  // the dropout key of this launch (derived from the device step index in a replayed graph)
-  const DropKey dk = DROP ? drop_live(a.drop) : a.drop;
   extern __shared__ __align__(1024) uint8_t smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (smem_u32(smem) & 1023) {
+    pdl_wait();
     if (threadIdx.x == 0) atomicOr(a.flags, FLAG_TIMEOUT);
     return;
   }
@@ -692,6 +697,10 @@ __global__ void __launch_bounds__(320, 2) k_attn_bwd_q8(const __grid_constant__ 
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tslot;
+  // predecessor kernels complete from here on (programmatic dependent launch);
+  // the dropout key of this launch (derived from the device step index in a replayed graph)
+  pdl_wait();
+  const DropKey dk = DROP ? drop_live(a.drop) : a.drop;
 
   if (warp == 0) {
     if (lane == 0) {
@@ -930,8 +939,8 @@ bool attn_fwd_tc(Ctx& c, const AttnDesc& d) {
                        D_SMEM);
   dim3 grid(d.B * d.H, d.T / 128);
   LaunchScope s(c, "attn_fwd_tc");
-  if (drop) k_attn_fwd_o<true><<<grid, 192, D_SMEM, c.stream>>>(tq, tkv64, make_args(d, c.flags));
-  else k_attn_fwd_o<false><<<grid, 192, D_SMEM, c.stream>>>(tq, tkv64, make_args(d, c.flags));
+  if (drop) launch_pdl(k_attn_fwd_o<true>, grid, 192, D_SMEM, c.stream, tq, tkv64, make_args(d, c.flags));
+  else launch_pdl(k_attn_fwd_o<false>, grid, 192, D_SMEM, c.stream, tq, tkv64, make_args(d, c.flags));
   return true;
 }
 
@@ -952,13 +961,13 @@ bool attn_bwd_tc(Ctx& c, const AttnDesc& d) {
   dim3 grid(d.B * d.H, d.T / 128);
   {  // dQ first: it also stores D = rowsum(dO * O), which the dK/dV kernel reads
     LaunchScope s(c, "attn_bwd_q_tc");
-    if (drop) k_attn_bwd_q8<true><<<grid, 320, Q_SMEM, c.stream>>>(tkv, tdo, tkv64, tout, a);
-    else k_attn_bwd_q8<false><<<grid, 320, Q_SMEM, c.stream>>>(tkv, tdo, tkv64, tout, a);
+    if (drop) launch_pdl(k_attn_bwd_q8<true>, grid, 320, Q_SMEM, c.stream, tkv, tdo, tkv64, tout, a);
+    else launch_pdl(k_attn_bwd_q8<false>, grid, 320, Q_SMEM, c.stream, tkv, tdo, tkv64, tout, a);
   }
   {
     LaunchScope s(c, "attn_bwd_kv_tc");
-    if (drop) k_attn_bwd_kv8<true><<<grid, 320, K_SMEM, c.stream>>>(tkv, tq64, tdo64, a);
-    else k_attn_bwd_kv8<false><<<grid, 320, K_SMEM, c.stream>>>(tkv, tq64, tdo64, a);
+    if (drop) launch_pdl(k_attn_bwd_kv8<true>, grid, 320, K_SMEM, c.stream, tkv, tq64, tdo64, a);
+    else launch_pdl(k_attn_bwd_kv8<false>, grid, 320, K_SMEM, c.stream, tkv, tq64, tdo64, a);
   }
   return true;
 }

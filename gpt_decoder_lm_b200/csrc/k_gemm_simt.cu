@@ -97,6 +97,7 @@ __global__ void k_splitk_reduce(const float* __restrict__ part, int splits, long
 // partial loads of up to 8 splits are issued before any add (same add order)
 __global__ void k_splitk_reduce4(const float4* __restrict__ part, int splits, long MN4, float4* __restrict__ out) {
   pdl_trigger();
+  pdl_wait();
   long i = (long)blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= MN4) return;
   float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -126,8 +127,8 @@ void splitk_reduce(Ctx& c, const float* partial, int splits, long MN, float* out
   LaunchScope s(c, "splitk_reduce");
   if (MN % 4 == 0 && !(reinterpret_cast<uintptr_t>(partial) & 15) && !(reinterpret_cast<uintptr_t>(out) & 15)) {
     const long MN4 = MN / 4;
-    k_splitk_reduce4<<<(unsigned)((MN4 + 255) / 256), 256, 0, c.stream>>>(
-        reinterpret_cast<const float4*>(partial), splits, MN4, reinterpret_cast<float4*>(out));
+    launch_pdl(k_splitk_reduce4, (unsigned)((MN4 + 255) / 256), 256, 0, c.stream,
+               reinterpret_cast<const float4*>(partial), splits, MN4, reinterpret_cast<float4*>(out));
   } else {
     k_splitk_reduce<<<(unsigned)((MN + 255) / 256), 256, 0, c.stream>>>(partial, splits, MN, out);
   }

@@ -15,6 +15,7 @@ __global__ void k_gather(const void* __restrict__ stream, int tok_u16, uint64_t 
                          const int* step_dev, int micro, int B, int T, int V, int32_t* __restrict__ idx,
                          int32_t* __restrict__ tgt, uint32_t* flags) {
   pdl_trigger();
+  pdl_wait();
   long i = (long)blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= (long)B * T) return;
   if (step_dev) step = *step_dev;  // step index held in device memory (replayed graphs)
@@ -44,13 +45,14 @@ void gather_batch(Ctx& c, const void* stream, int tok_u16, uint64_t len, uint64_
                   int T, int V, int32_t* idx, int32_t* tgt, const int* step_dev) {
   long n = (long)B * T;
   LaunchScope s(c, "gather_batch");
-  k_gather<<<(unsigned)((n + 255) / 256), 256, 0, c.stream>>>(stream, tok_u16, len, seed, step, step_dev, micro, B, T,
+  launch_pdl(k_gather, (unsigned)((n + 255) / 256), 256, 0, c.stream, stream, tok_u16, len, seed, step, step_dev, micro, B, T,
                                                               V, idx, tgt, c.flags);
 }
 
 // writes the per-step scalars read by replayed graphs: step, lr, 1 - b1^t, 1 - b2^t
 __global__ void k_set_step(int* step_dev, float* hyper, int step, float lr, float bc1, float bc2) {
   pdl_trigger();
+  pdl_wait();
   *step_dev = step;
   hyper[0] = lr;
   hyper[1] = bc1;
@@ -59,12 +61,13 @@ __global__ void k_set_step(int* step_dev, float* hyper, int step, float lr, floa
 
 void set_step_params(Ctx& c, int* step_dev, float* hyper, int step, float lr, float bc1, float bc2) {
   LaunchScope s(c, "set_step");
-  k_set_step<<<1, 1, 0, c.stream>>>(step_dev, hyper, step, lr, bc1, bc2);
+  launch_pdl(k_set_step, 1, 1, 0, c.stream, step_dev, hyper, step, lr, bc1, bc2);
 }
 
 __global__ void k_check_tokens(const int32_t* __restrict__ idx, const int32_t* __restrict__ tgt, long n, int V,
                                int32_t* __restrict__ io, int32_t* __restrict__ to, uint32_t* flags) {
   pdl_trigger();
+  pdl_wait();
   long i = (long)blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= n) return;
   int x = idx[i], y = tgt[i];
@@ -79,7 +82,7 @@ __global__ void k_check_tokens(const int32_t* __restrict__ idx, const int32_t* _
 
 void check_tokens(Ctx& c, const int32_t* idx, const int32_t* tgt, long n, int V, int32_t* io, int32_t* to) {
   LaunchScope s(c, "check_tokens");
-  k_check_tokens<<<(unsigned)((n + 255) / 256), 256, 0, c.stream>>>(idx, tgt, n, V, io, to, c.flags);
+  launch_pdl(k_check_tokens, (unsigned)((n + 255) / 256), 256, 0, c.stream, idx, tgt, n, V, io, to, c.flags);
 }
 
 // ============================================================================
@@ -90,6 +93,7 @@ __global__ void k_embed_fwd(const int32_t* __restrict__ idx, const float* __rest
                             const float* __restrict__ wpe, float* __restrict__ res, int T, int d, long n4,
                             DropKey drop) {
   pdl_trigger();
+  pdl_wait();
   long i = (long)blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= n4) return;
   int d4 = d >> 2;
@@ -116,7 +120,7 @@ void embed_fwd(Ctx& c, const int32_t* idx, const float* wte, const float* wpe, f
                DropKey drop) {
   long n4 = (long)B * Tn * d / 4;
   LaunchScope s(c, "embed_fwd");
-  k_embed_fwd<<<(unsigned)((n4 + 255) / 256), 256, 0, c.stream>>>(idx, wte, wpe, res, Tn, d, n4, drop);
+  launch_pdl(k_embed_fwd, (unsigned)((n4 + 255) / 256), 256, 0, c.stream, idx, wte, wpe, res, Tn, d, n4, drop);
 }
 template void embed_fwd<float>(Ctx&, const int32_t*, const float*, const float*, float*, int, int, int, DropKey);
 template void embed_fwd<bf16>(Ctx&, const int32_t*, const float*, const float*, float*, int, int, int, DropKey);
@@ -146,6 +150,7 @@ __global__ void __launch_bounds__(256) k_norm_fwd(const float* __restrict__ x, c
                                                   float* __restrict__ mean_out, float* __restrict__ rstd_out,
                                                   long rows, int d, int rms, float eps) {
   pdl_trigger();
+  pdl_wait();
   const int lane = threadIdx.x & 31;
   const long nwarps = (long)gridDim.x * (blockDim.x >> 5);
   long row = (long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
@@ -228,7 +233,7 @@ void launch_norm_fwd(Ctx& c, const float* x, const float* w, const float* b, T* 
   long grid = (long)c.num_sms * occ;
   const long need = (rows + 7) / 8;
   if (grid > need) grid = need;
-  k_norm_fwd<T, VPL><<<(unsigned)grid, 256, 0, c.stream>>>(x, w, b, y, mean, rstd, rows, d, rms, eps);
+  launch_pdl(k_norm_fwd<T, VPL>, (unsigned)grid, 256, 0, c.stream, x, w, b, y, mean, rstd, rows, d, rms, eps);
 }
 
 template <typename T>
@@ -261,6 +266,7 @@ template void norm_fwd<bf16>(Ctx&, const float*, const float*, const float*, bf1
 template <typename T>
 __global__ void k_norm_bwd(NormBwd p) {
   pdl_trigger();
+  pdl_wait();
   extern __shared__ float red[];  // [2 buffers][warps][4]
   int tid = threadIdx.x;
   int d4 = p.d >> 2;
@@ -396,7 +402,7 @@ void norm_bwd(Ctx& c, const NormBwd& p) {
   LaunchScope s(c, "norm_bwd");
   int threads = ((d4 + 31) / 32) * 32;
   int nw = threads / 32;
-  k_norm_bwd<T><<<p.blocks, threads, 2 * nw * 4 * sizeof(float), c.stream>>>(p);
+  launch_pdl(k_norm_bwd<T>, p.blocks, threads, 2 * nw * 4 * sizeof(float), c.stream, p);
 }
 template void norm_bwd<float>(Ctx&, const NormBwd&);
 template void norm_bwd<bf16>(Ctx&, const NormBwd&);
@@ -411,6 +417,7 @@ struct Dst3 {
 __global__ void __launch_bounds__(1024) k_rows_reduce(const float* __restrict__ src, long stride, long slot_off,
                                                       int rows, int n, Dst3 dsts) {
   pdl_trigger();
+  pdl_wait();
   __shared__ float sh[32][33];
   float* dst = dsts.p[blockIdx.y];
   if (!dst) return;  // uniform per block
@@ -438,7 +445,7 @@ void partial_reduce3(Ctx& c, const float* part, int blocks, int d, float* g0, fl
   if (!g0 && !g1 && !g2) return;
   LaunchScope s(c, "partial_reduce");
   Dst3 g{{g0, g1, g2}};
-  k_rows_reduce<<<dim3((d + 31) / 32, 3), dim3(32, 32), 0, c.stream>>>(part, 3L * d, d, blocks, d, g);
+  launch_pdl(k_rows_reduce, dim3((d + 31) / 32, 3), dim3(32, 32), 0, c.stream, part, 3L * d, d, blocks, d, g);
 }
 
 // ============================================================================
@@ -448,6 +455,7 @@ template <typename T>
 __global__ void k_colsum(const T* __restrict__ x, long rows, int N, int chunks, float* __restrict__ part,
                          int accumulate) {
   pdl_trigger();
+  pdl_wait();
   int j = blockIdx.x * blockDim.x + threadIdx.x;
   if (j >= N) return;
   long per = (rows + chunks - 1) / chunks;
@@ -463,7 +471,7 @@ __global__ void k_colsum(const T* __restrict__ x, long rows, int N, int chunks, 
 void colsum_reduce(Ctx& c, const float* part, int chunks, int N, float* grad) {
   LaunchScope s(c, "colsum");
   Dst3 g{{grad, nullptr, nullptr}};
-  k_rows_reduce<<<dim3((N + 31) / 32, 1), dim3(32, 32), 0, c.stream>>>(part, N, 0, chunks, N, g);
+  launch_pdl(k_rows_reduce, dim3((N + 31) / 32, 1), dim3(32, 32), 0, c.stream, part, N, 0, chunks, N, g);
 }
 
 // bf16 rows with N % 8 == 0: each thread sums 8 adjacent columns over its
@@ -471,6 +479,7 @@ void colsum_reduce(Ctx& c, const float* part, int chunks, int N, float* grad) {
 __global__ void k_colsum_bf16x8(const bf16* __restrict__ x, long rows, int N, int chunks, float* __restrict__ part,
                                 int accumulate) {
   pdl_trigger();
+  pdl_wait();
   const int j8 = blockIdx.x * blockDim.x + threadIdx.x;
   if (j8 * 8 >= N) return;
   const long per = (rows + chunks - 1) / chunks;
@@ -516,11 +525,11 @@ void colsum_partial(Ctx& c, const T* x, long rows, int N, float* part, bool accu
   LaunchScope s(c, "colsum");
   if (vec) {
     dim3 grid((N / 8 + 127) / 128, chunks);
-    k_colsum_bf16x8<<<grid, 128, 0, c.stream>>>(reinterpret_cast<const bf16*>(x), rows, N, chunks, part,
+    launch_pdl(k_colsum_bf16x8, grid, 128, 0, c.stream, reinterpret_cast<const bf16*>(x), rows, N, chunks, part,
                                                 accumulate ? 1 : 0);
   } else {
     dim3 grid((N + 127) / 128, chunks);
-    k_colsum<T><<<grid, 128, 0, c.stream>>>(x, rows, N, chunks, part, accumulate ? 1 : 0);
+    launch_pdl(k_colsum<T>, grid, 128, 0, c.stream, x, rows, N, chunks, part, accumulate ? 1 : 0);
   }
 }
 template void colsum_partial<float>(Ctx&, const float*, long, int, float*, bool);
@@ -537,6 +546,7 @@ template <typename T>
 __global__ void k_ce(T* __restrict__ logits, const int32_t* __restrict__ tgt, int V, int Vp,
                      float* __restrict__ lse_out, float* __restrict__ row_loss, int want_grad, float scale) {
   pdl_trigger();
+  pdl_wait();
   __shared__ float sm[32], ss[32];
   long row = blockIdx.x;
   T* z = logits + row * Vp;
@@ -605,6 +615,7 @@ __global__ void __launch_bounds__(256, 4) k_ce_stream(T* __restrict__ logits, co
                                                       int Vp, float* __restrict__ lse_out,
                                                       float* __restrict__ row_loss, int want_grad, float scale) {
   pdl_trigger();
+  pdl_wait();
   constexpr int EPV = 16 / sizeof(T);
   constexpr float LOG2E = 1.4426950408889634f;
   __shared__ float sm[8], ss[8];
@@ -677,9 +688,9 @@ void ce_fwd_bwd(Ctx& c, T* logits, const int32_t* tgt, long M, int V, int Vp, fl
   LaunchScope s(c, want_grad ? "ce_fwd_bwd" : "ce_fwd");
   constexpr int EPV = 16 / sizeof(T);
   if (Vp % EPV == 0)
-    k_ce_stream<T><<<(unsigned)M, 256, 0, c.stream>>>(logits, tgt, V, Vp, lse, row_loss, want_grad ? 1 : 0, scale);
+    launch_pdl(k_ce_stream<T>, (unsigned)M, 256, 0, c.stream, logits, tgt, V, Vp, lse, row_loss, want_grad ? 1 : 0, scale);
   else
-    k_ce<T><<<(unsigned)M, 512, 0, c.stream>>>(logits, tgt, V, Vp, lse, row_loss, want_grad ? 1 : 0, scale);
+    launch_pdl(k_ce<T>, (unsigned)M, 512, 0, c.stream, logits, tgt, V, Vp, lse, row_loss, want_grad ? 1 : 0, scale);
 }
 template void ce_fwd_bwd<float>(Ctx&, float*, const int32_t*, long, int, int, float*, float*, bool, float);
 template void ce_fwd_bwd<bf16>(Ctx&, bf16*, const int32_t*, long, int, int, float*, float*, bool, float);
@@ -688,6 +699,7 @@ template void ce_fwd_bwd<bf16>(Ctx&, bf16*, const int32_t*, long, int, int, floa
 __global__ void k_loss_reduce(const float* __restrict__ rl, long M, float scale, float* acc, int accumulate,
                               uint32_t* flags) {
   pdl_trigger();
+  pdl_wait();
   __shared__ double sh[32];
   double s = 0.0;
   for (long i = threadIdx.x; i < M; i += blockDim.x) s += (double)rl[i];
@@ -705,7 +717,7 @@ __global__ void k_loss_reduce(const float* __restrict__ rl, long M, float scale,
 
 void loss_reduce(Ctx& c, const float* row_loss, long M, float scale, float* loss_acc, int accumulate) {
   LaunchScope s(c, "loss_reduce");
-  k_loss_reduce<<<1, 1024, 0, c.stream>>>(row_loss, M, scale, loss_acc, accumulate, c.flags);
+  launch_pdl(k_loss_reduce, 1, 1024, 0, c.stream, row_loss, M, scale, loss_acc, accumulate, c.flags);
 }
 
 // ============================================================================
@@ -715,6 +727,7 @@ void loss_reduce(Ctx& c, const float* row_loss, long M, float scale, float* loss
 __global__ void k_embed_sort(const int32_t* __restrict__ idx, int M, int P2, int32_t* __restrict__ stok,
                              int32_t* __restrict__ spos, int32_t* __restrict__ n_unique) {
   pdl_trigger();
+  pdl_wait();
   extern __shared__ uint32_t key[];
   __shared__ int cnt[32];
   // block b sorts the b-th batch of M tokens (batches stored back to back)
@@ -766,7 +779,7 @@ void embed_sort(Ctx& c, const int32_t* idx, long M, int32_t* sorted_tok, int32_t
   // per-device function attribute: set before every launch
   cudaFuncSetAttribute(k_embed_sort, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
   LaunchScope s(c, "embed_sort");
-  k_embed_sort<<<batches, 1024, smem, c.stream>>>(idx, (int)M, P2, sorted_tok, sorted_pos, n_unique);
+  launch_pdl(k_embed_sort, batches, 1024, smem, c.stream, idx, (int)M, P2, sorted_tok, sorted_pos, n_unique);
 }
 
 // dwte[v] += sum over the sorted positions of token v (in position order) of
@@ -776,6 +789,7 @@ void embed_sort(Ctx& c, const int32_t* idx, long M, int32_t* sorted_tok, int32_t
 __global__ void k_embed_bwd_wpe(const float* __restrict__ dres, int Bn, int Tn, int d, DropKey drop,
                                 float* __restrict__ dwpe) {
   pdl_trigger();
+  pdl_wait();
   long i = (long)blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= (long)Tn * d) return;
   int t = (int)(i / d), c = (int)(i % d);
@@ -806,6 +820,7 @@ __global__ void __launch_bounds__(256, 2) k_embed_seg_a(const float* __restrict_
                                                      float* __restrict__ dwte, float* __restrict__ head,
                                                      float* __restrict__ tail) {
   pdl_trigger();
+  pdl_wait();
   __shared__ int s_tok[EC + 2], s_pos[EC];
   __shared__ int8_t s_kind[EC];  // what ends at slot k: nothing, an inner segment, the head, the tail
   drop = drop_live(drop);
@@ -870,6 +885,7 @@ __global__ void __launch_bounds__(256, 2) k_embed_seg_a(const float* __restrict_
 __global__ void k_embed_seg_b(const int32_t* __restrict__ stok, int M, int d, const float* __restrict__ head,
                               const float* __restrict__ tail, float* __restrict__ dwte) {
   pdl_trigger();
+  pdl_wait();
   const int c = blockIdx.x;
   const int j0 = c * EC, j1 = min(M, j0 + EC);
   const int tok = stok[j1 - 1];
@@ -930,13 +946,13 @@ void embed_bwd(Ctx& c, const float* dres, const int32_t* sorted_tok, const int32
     const int chunks = (int)((M + EC - 1) / EC);
     float* head = seg_scratch;
     float* tail = seg_scratch + (size_t)chunks * d;
-    k_embed_seg_a<<<chunks, 256, 0, c.stream>>>(dres, sorted_tok, sorted_pos, (int)M, d, drop, dwte, head, tail);
-    k_embed_seg_b<<<chunks, 256, 0, c.stream>>>(sorted_tok, (int)M, d, head, tail, dwte);
+    launch_pdl(k_embed_seg_a, chunks, 256, 0, c.stream, dres, sorted_tok, sorted_pos, (int)M, d, drop, dwte, head, tail);
+    launch_pdl(k_embed_seg_b, chunks, 256, 0, c.stream, sorted_tok, (int)M, d, head, tail, dwte);
   }
   {
     LaunchScope s(c, "embed_bwd_wpe");
     long n = (long)Tn * d;
-    k_embed_bwd_wpe<<<(unsigned)((n + 255) / 256), 256, 0, c.stream>>>(dres, Bn, Tn, d, drop, dwpe);
+    launch_pdl(k_embed_bwd_wpe, (unsigned)((n + 255) / 256), 256, 0, c.stream, dres, Bn, Tn, d, drop, dwpe);
   }
 }
 
@@ -947,6 +963,7 @@ int sumsq_blocks(Ctx& c) { return c.num_sms * 4 < 592 ? c.num_sms * 4 : 592; }  
 
 __global__ void k_sumsq(const float* __restrict__ g, long n4, double* __restrict__ part) {
   pdl_trigger();
+  pdl_wait();
   __shared__ double sh[32];
   double s = 0.0;
   for (long i = (long)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += (long)gridDim.x * blockDim.x) {
@@ -965,7 +982,7 @@ __global__ void k_sumsq(const float* __restrict__ g, long n4, double* __restrict
 
 void sumsq_partials(Ctx& c, const float* g, long n, double* partials, int blocks) {
   LaunchScope s(c, "grad_norm");
-  k_sumsq<<<blocks, 512, 0, c.stream>>>(g, n / 4, partials);
+  launch_pdl(k_sumsq, blocks, 512, 0, c.stream, g, n / 4, partials);
 }
 
 // ============================================================================
@@ -981,6 +998,7 @@ void sumsq_partials(Ctx& c, const float* g, long n, double* partials, int blocks
 // ============================================================================
 __global__ void k_adamw(AdamArgs a, uint32_t* flags) {
   pdl_trigger();
+  pdl_wait();
   __shared__ float s_coef;
   __shared__ int s_ok;
   if (threadIdx.x < 32) {
@@ -1062,23 +1080,25 @@ __global__ void k_adamw(AdamArgs a, uint32_t* flags) {
 
 void adamw(Ctx& c, const AdamArgs& a) {
   LaunchScope s(c, "adamw");
-  k_adamw<<<c.num_sms * 8, 256, 0, c.stream>>>(a, c.flags);
+  launch_pdl(k_adamw, c.num_sms * 8, 256, 0, c.stream, a, c.flags);
 }
 
 __global__ void k_to_bf16(const float* __restrict__ s, bf16* __restrict__ d, long n) {
   pdl_trigger();
+  pdl_wait();
   long i = (long)blockIdx.x * blockDim.x + threadIdx.x;
   if (i < n) d[i] = __float2bfloat16_rn(s[i]);
 }
 
 void to_bf16(Ctx& c, const float* src, bf16* dst, long n) {
   LaunchScope s(c, "to_bf16");
-  k_to_bf16<<<(unsigned)((n + 255) / 256), 256, 0, c.stream>>>(src, dst, n);
+  launch_pdl(k_to_bf16, (unsigned)((n + 255) / 256), 256, 0, c.stream, src, dst, n);
 }
 
 // row argmax, ties to the lowest index
 __global__ void k_argmax(const void* __restrict__ x, int is_bf16, int cols, int ld, int32_t* __restrict__ out) {
   pdl_trigger();
+  pdl_wait();
   __shared__ float bv[32];
   __shared__ int bi[32];
   long row = blockIdx.x;
@@ -1116,18 +1136,19 @@ __global__ void k_argmax(const void* __restrict__ x, int is_bf16, int cols, int 
 
 void argmax_rows(Ctx& c, const void* x, int is_bf16, long rows, int cols, int ld, int32_t* out) {
   LaunchScope s(c, "argmax");
-  k_argmax<<<(unsigned)rows, 256, 0, c.stream>>>(x, is_bf16, cols, ld, out);
+  launch_pdl(k_argmax, (unsigned)rows, 256, 0, c.stream, x, is_bf16, cols, ld, out);
 }
 
 __global__ void k_dropmask(DropKey k, long n, uint8_t* out) {
   pdl_trigger();
+  pdl_wait();
   long i = (long)blockIdx.x * blockDim.x + threadIdx.x;
   if (i < n) out[i] = drop_keep(k, (uint64_t)i) ? 1 : 0;
 }
 
 void dropout_mask(Ctx& c, DropKey k, long n, uint8_t* out) {
   LaunchScope s(c, "dropout_mask");
-  k_dropmask<<<(unsigned)((n + 255) / 256), 256, 0, c.stream>>>(k, n, out);
+  launch_pdl(k_dropmask, (unsigned)((n + 255) / 256), 256, 0, c.stream, k, n, out);
 }
 
 }  // namespace gpt

@@ -19,6 +19,27 @@ struct Ctx {
 void timing_begin(Ctx& c, const char* name);
 void timing_end(Ctx& c, const char* name);
 
+// Launches kernel k as a programmatic dependent of the stream's previous
+// kernel (cudaLaunchAttributeProgrammaticStreamSerialization): its blocks may
+// be scheduled while that kernel's last wave drains, and wait in pdl_wait()
+// for its completion.  Every kernel launched this way calls pdl_wait() in
+// every block before any global-memory access that a kernel before it may
+// write or read.
+template <typename... KP, typename... A>
+inline cudaError_t launch_pdl(void (*k)(KP...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, A... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, k, args...);
+}
+
 struct LaunchScope {
   Ctx& c;
   const char* name;
