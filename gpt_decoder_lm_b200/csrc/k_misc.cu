@@ -45,7 +45,7 @@ void gather_batch(Ctx& c, const void* stream, int tok_u16, uint64_t len, uint64_
                   int T, int V, int32_t* idx, int32_t* tgt, const int* step_dev) {
   long n = (long)B * T;
   LaunchScope s(c, "gather_batch");
-  launch_pdl(k_gather, (unsigned)((n + 255) / 256), 256, 0, c.stream, stream, tok_u16, len, seed, step, step_dev, micro, B, T,
+  k_gather<<<(unsigned)((n + 255) / 256), 256, 0, c.stream>>>(stream, tok_u16, len, seed, step, step_dev, micro, B, T,
                                                               V, idx, tgt, c.flags);
 }
 
@@ -61,7 +61,7 @@ __global__ void k_set_step(int* step_dev, float* hyper, int step, float lr, floa
 
 void set_step_params(Ctx& c, int* step_dev, float* hyper, int step, float lr, float bc1, float bc2) {
   LaunchScope s(c, "set_step");
-  launch_pdl(k_set_step, 1, 1, 0, c.stream, step_dev, hyper, step, lr, bc1, bc2);
+  k_set_step<<<1, 1, 0, c.stream>>>(step_dev, hyper, step, lr, bc1, bc2);
 }
 
 __global__ void k_check_tokens(const int32_t* __restrict__ idx, const int32_t* __restrict__ tgt, long n, int V,
@@ -82,7 +82,7 @@ __global__ void k_check_tokens(const int32_t* __restrict__ idx, const int32_t* _
 
 void check_tokens(Ctx& c, const int32_t* idx, const int32_t* tgt, long n, int V, int32_t* io, int32_t* to) {
   LaunchScope s(c, "check_tokens");
-  launch_pdl(k_check_tokens, (unsigned)((n + 255) / 256), 256, 0, c.stream, idx, tgt, n, V, io, to, c.flags);
+  k_check_tokens<<<(unsigned)((n + 255) / 256), 256, 0, c.stream>>>(idx, tgt, n, V, io, to, c.flags);
 }
 
 // ============================================================================
@@ -120,7 +120,7 @@ void embed_fwd(Ctx& c, const int32_t* idx, const float* wte, const float* wpe, f
                DropKey drop) {
   long n4 = (long)B * Tn * d / 4;
   LaunchScope s(c, "embed_fwd");
-  launch_pdl(k_embed_fwd, (unsigned)((n4 + 255) / 256), 256, 0, c.stream, idx, wte, wpe, res, Tn, d, n4, drop);
+  k_embed_fwd<<<(unsigned)((n4 + 255) / 256), 256, 0, c.stream>>>(idx, wte, wpe, res, Tn, d, n4, drop);
 }
 template void embed_fwd<float>(Ctx&, const int32_t*, const float*, const float*, float*, int, int, int, DropKey);
 template void embed_fwd<bf16>(Ctx&, const int32_t*, const float*, const float*, float*, int, int, int, DropKey);
@@ -233,7 +233,7 @@ void launch_norm_fwd(Ctx& c, const float* x, const float* w, const float* b, T* 
   long grid = (long)c.num_sms * occ;
   const long need = (rows + 7) / 8;
   if (grid > need) grid = need;
-  launch_pdl(k_norm_fwd<T, VPL>, (unsigned)grid, 256, 0, c.stream, x, w, b, y, mean, rstd, rows, d, rms, eps);
+  k_norm_fwd<T, VPL><<<(unsigned)grid, 256, 0, c.stream>>>(x, w, b, y, mean, rstd, rows, d, rms, eps);
 }
 
 template <typename T>
@@ -402,7 +402,7 @@ void norm_bwd(Ctx& c, const NormBwd& p) {
   LaunchScope s(c, "norm_bwd");
   int threads = ((d4 + 31) / 32) * 32;
   int nw = threads / 32;
-  launch_pdl(k_norm_bwd<T>, p.blocks, threads, 2 * nw * 4 * sizeof(float), c.stream, p);
+  k_norm_bwd<T><<<p.blocks, threads, 2 * nw * 4 * sizeof(float), c.stream>>>(p);
 }
 template void norm_bwd<float>(Ctx&, const NormBwd&);
 template void norm_bwd<bf16>(Ctx&, const NormBwd&);
@@ -445,7 +445,7 @@ void partial_reduce3(Ctx& c, const float* part, int blocks, int d, float* g0, fl
   if (!g0 && !g1 && !g2) return;
   LaunchScope s(c, "partial_reduce");
   Dst3 g{{g0, g1, g2}};
-  launch_pdl(k_rows_reduce, dim3((d + 31) / 32, 3), dim3(32, 32), 0, c.stream, part, 3L * d, d, blocks, d, g);
+  k_rows_reduce<<<dim3((d + 31) / 32, 3), dim3(32, 32), 0, c.stream>>>(part, 3L * d, d, blocks, d, g);
 }
 
 // ============================================================================
@@ -471,7 +471,7 @@ __global__ void k_colsum(const T* __restrict__ x, long rows, int N, int chunks, 
 void colsum_reduce(Ctx& c, const float* part, int chunks, int N, float* grad) {
   LaunchScope s(c, "colsum");
   Dst3 g{{grad, nullptr, nullptr}};
-  launch_pdl(k_rows_reduce, dim3((N + 31) / 32, 1), dim3(32, 32), 0, c.stream, part, N, 0, chunks, N, g);
+  k_rows_reduce<<<dim3((N + 31) / 32, 1), dim3(32, 32), 0, c.stream>>>(part, N, 0, chunks, N, g);
 }
 
 // bf16 rows with N % 8 == 0: each thread sums 8 adjacent columns over its
@@ -525,11 +525,11 @@ void colsum_partial(Ctx& c, const T* x, long rows, int N, float* part, bool accu
   LaunchScope s(c, "colsum");
   if (vec) {
     dim3 grid((N / 8 + 127) / 128, chunks);
-    launch_pdl(k_colsum_bf16x8, grid, 128, 0, c.stream, reinterpret_cast<const bf16*>(x), rows, N, chunks, part,
+    k_colsum_bf16x8<<<grid, 128, 0, c.stream>>>(reinterpret_cast<const bf16*>(x), rows, N, chunks, part,
                                                 accumulate ? 1 : 0);
   } else {
     dim3 grid((N + 127) / 128, chunks);
-    launch_pdl(k_colsum<T>, grid, 128, 0, c.stream, x, rows, N, chunks, part, accumulate ? 1 : 0);
+    k_colsum<T><<<grid, 128, 0, c.stream>>>(x, rows, N, chunks, part, accumulate ? 1 : 0);
   }
 }
 template void colsum_partial<float>(Ctx&, const float*, long, int, float*, bool);
@@ -688,9 +688,9 @@ void ce_fwd_bwd(Ctx& c, T* logits, const int32_t* tgt, long M, int V, int Vp, fl
   LaunchScope s(c, want_grad ? "ce_fwd_bwd" : "ce_fwd");
   constexpr int EPV = 16 / sizeof(T);
   if (Vp % EPV == 0)
-    launch_pdl(k_ce_stream<T>, (unsigned)M, 256, 0, c.stream, logits, tgt, V, Vp, lse, row_loss, want_grad ? 1 : 0, scale);
+    k_ce_stream<T><<<(unsigned)M, 256, 0, c.stream>>>(logits, tgt, V, Vp, lse, row_loss, want_grad ? 1 : 0, scale);
   else
-    launch_pdl(k_ce<T>, (unsigned)M, 512, 0, c.stream, logits, tgt, V, Vp, lse, row_loss, want_grad ? 1 : 0, scale);
+    k_ce<T><<<(unsigned)M, 512, 0, c.stream>>>(logits, tgt, V, Vp, lse, row_loss, want_grad ? 1 : 0, scale);
 }
 template void ce_fwd_bwd<float>(Ctx&, float*, const int32_t*, long, int, int, float*, float*, bool, float);
 template void ce_fwd_bwd<bf16>(Ctx&, bf16*, const int32_t*, long, int, int, float*, float*, bool, float);
@@ -717,7 +717,7 @@ __global__ void k_loss_reduce(const float* __restrict__ rl, long M, float scale,
 
 void loss_reduce(Ctx& c, const float* row_loss, long M, float scale, float* loss_acc, int accumulate) {
   LaunchScope s(c, "loss_reduce");
-  launch_pdl(k_loss_reduce, 1, 1024, 0, c.stream, row_loss, M, scale, loss_acc, accumulate, c.flags);
+  k_loss_reduce<<<1, 1024, 0, c.stream>>>(row_loss, M, scale, loss_acc, accumulate, c.flags);
 }
 
 // ============================================================================
@@ -779,7 +779,7 @@ void embed_sort(Ctx& c, const int32_t* idx, long M, int32_t* sorted_tok, int32_t
   // per-device function attribute: set before every launch
   cudaFuncSetAttribute(k_embed_sort, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
   LaunchScope s(c, "embed_sort");
-  launch_pdl(k_embed_sort, batches, 1024, smem, c.stream, idx, (int)M, P2, sorted_tok, sorted_pos, n_unique);
+  k_embed_sort<<<batches, 1024, smem, c.stream>>>(idx, (int)M, P2, sorted_tok, sorted_pos, n_unique);
 }
 
 // dwte[v] += sum over the sorted positions of token v (in position order) of
@@ -946,13 +946,13 @@ void embed_bwd(Ctx& c, const float* dres, const int32_t* sorted_tok, const int32
     const int chunks = (int)((M + EC - 1) / EC);
     float* head = seg_scratch;
     float* tail = seg_scratch + (size_t)chunks * d;
-    launch_pdl(k_embed_seg_a, chunks, 256, 0, c.stream, dres, sorted_tok, sorted_pos, (int)M, d, drop, dwte, head, tail);
-    launch_pdl(k_embed_seg_b, chunks, 256, 0, c.stream, sorted_tok, (int)M, d, head, tail, dwte);
+    k_embed_seg_a<<<chunks, 256, 0, c.stream>>>(dres, sorted_tok, sorted_pos, (int)M, d, drop, dwte, head, tail);
+    k_embed_seg_b<<<chunks, 256, 0, c.stream>>>(sorted_tok, (int)M, d, head, tail, dwte);
   }
   {
     LaunchScope s(c, "embed_bwd_wpe");
     long n = (long)Tn * d;
-    launch_pdl(k_embed_bwd_wpe, (unsigned)((n + 255) / 256), 256, 0, c.stream, dres, Bn, Tn, d, drop, dwpe);
+    k_embed_bwd_wpe<<<(unsigned)((n + 255) / 256), 256, 0, c.stream>>>(dres, Bn, Tn, d, drop, dwpe);
   }
 }
 
@@ -982,7 +982,7 @@ __global__ void k_sumsq(const float* __restrict__ g, long n4, double* __restrict
 
 void sumsq_partials(Ctx& c, const float* g, long n, double* partials, int blocks) {
   LaunchScope s(c, "grad_norm");
-  launch_pdl(k_sumsq, blocks, 512, 0, c.stream, g, n / 4, partials);
+  k_sumsq<<<blocks, 512, 0, c.stream>>>(g, n / 4, partials);
 }
 
 // ============================================================================
@@ -1080,7 +1080,7 @@ __global__ void k_adamw(AdamArgs a, uint32_t* flags) {
 
 void adamw(Ctx& c, const AdamArgs& a) {
   LaunchScope s(c, "adamw");
-  launch_pdl(k_adamw, c.num_sms * 8, 256, 0, c.stream, a, c.flags);
+  k_adamw<<<c.num_sms * 8, 256, 0, c.stream>>>(a, c.flags);
 }
 
 __global__ void k_to_bf16(const float* __restrict__ s, bf16* __restrict__ d, long n) {
@@ -1092,7 +1092,7 @@ __global__ void k_to_bf16(const float* __restrict__ s, bf16* __restrict__ d, lon
 
 void to_bf16(Ctx& c, const float* src, bf16* dst, long n) {
   LaunchScope s(c, "to_bf16");
-  launch_pdl(k_to_bf16, (unsigned)((n + 255) / 256), 256, 0, c.stream, src, dst, n);
+  k_to_bf16<<<(unsigned)((n + 255) / 256), 256, 0, c.stream>>>(src, dst, n);
 }
 
 // row argmax, ties to the lowest index
@@ -1136,7 +1136,7 @@ __global__ void k_argmax(const void* __restrict__ x, int is_bf16, int cols, int 
 
 void argmax_rows(Ctx& c, const void* x, int is_bf16, long rows, int cols, int ld, int32_t* out) {
   LaunchScope s(c, "argmax");
-  launch_pdl(k_argmax, (unsigned)rows, 256, 0, c.stream, x, is_bf16, cols, ld, out);
+  k_argmax<<<(unsigned)rows, 256, 0, c.stream>>>(x, is_bf16, cols, ld, out);
 }
 
 __global__ void k_dropmask(DropKey k, long n, uint8_t* out) {
@@ -1148,7 +1148,7 @@ __global__ void k_dropmask(DropKey k, long n, uint8_t* out) {
 
 void dropout_mask(Ctx& c, DropKey k, long n, uint8_t* out) {
   LaunchScope s(c, "dropout_mask");
-  launch_pdl(k_dropmask, (unsigned)((n + 255) / 256), 256, 0, c.stream, k, n, out);
+  k_dropmask<<<(unsigned)((n + 255) / 256), 256, 0, c.stream>>>(k, n, out);
 }
 
 }  // namespace gpt
