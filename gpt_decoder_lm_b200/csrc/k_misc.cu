@@ -130,16 +130,11 @@ template void embed_fwd<bf16>(Ctx&, const int32_t*, const float*, const float*, 
 // lane).  LayerNorm: biased variance, y = (x - mean) * rstd * w + b.
 // RMSNorm (micro variant): y = x * rstd with rstd = 1/sqrt(mean(x^2) + eps).
 // ============================================================================
-// four consecutive operand-typed elements: the raw vector (one 16- or 8-byte
-// load) and its widening to floats, kept apart so that a load can be issued
-// long before its value is used
-template <typename T> struct Raw4 { using type = float4; };
-template <> struct Raw4<bf16> { using type = uint2; };
-template <typename T> __device__ __forceinline__ typename Raw4<T>::type load_raw4(const T* p) {
-  return *reinterpret_cast<const typename Raw4<T>::type*>(p);
-}
-__device__ __forceinline__ float4 widen4(float4 v) { return v; }
-__device__ __forceinline__ float4 widen4(uint2 u) {
+// four consecutive operand-typed elements as floats (bf16: one 8-byte load)
+template <typename T> __device__ __forceinline__ float4 load4(const T* p);
+template <> __device__ __forceinline__ float4 load4<float>(const float* p) { return *reinterpret_cast<const float4*>(p); }
+template <> __device__ __forceinline__ float4 load4<bf16>(const bf16* p) {
+  const uint2 u = *reinterpret_cast<const uint2*>(p);
   return make_float4(__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xffff0000u), __uint_as_float(u.y << 16),
                      __uint_as_float(u.y & 0xffff0000u));
 }
@@ -297,8 +292,7 @@ __global__ void k_norm_bwd(NormBwd p) {
   // the next round (dy, x, the residual gradient they add to, mean, rstd) are
   // loaded before this round's work, so loads stay in flight throughout.
   struct Rows {
-    typename Raw4<T>::type dy[2];
-    float4 x[2], old[2];
+    float4 dy[2], x[2], old[2];
     float mean[2], rstd[2];
   };
   auto load = [&](long r, Rows& q) {
@@ -308,10 +302,9 @@ __global__ void k_norm_bwd(NormBwd p) {
       const bool live = rr < r1;
       q.mean[u] = (p.rms || !live) ? 0.f : p.mean[rr];
       q.rstd[u] = live ? p.rstd[rr] : 0.f;
-      q.dy[u] = {};
-      q.x[u] = q.old[u] = make_float4(0, 0, 0, 0);
+      q.dy[u] = q.x[u] = q.old[u] = make_float4(0, 0, 0, 0);
       if (own && live) {
-        q.dy[u] = load_raw4<T>(reinterpret_cast<const T*>(p.dy) + rr * p.d + 4 * tid);
+        q.dy[u] = load4<T>(reinterpret_cast<const T*>(p.dy) + rr * p.d + 4 * tid);
         q.x[u] = reinterpret_cast<const float4*>(p.x + rr * p.d)[tid];
         if (p.accumulate) q.old[u] = reinterpret_cast<const float4*>(p.dres + rr * p.d)[tid];
       }
@@ -325,8 +318,7 @@ __global__ void k_norm_bwd(NormBwd p) {
     float s[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int u = 0; u < 2; u++) {
-      const float4 dy4 = widen4(cur.dy[u]);
-      const float dya[4] = {dy4.x, dy4.y, dy4.z, dy4.w};
+      const float dya[4] = {cur.dy[u].x, cur.dy[u].y, cur.dy[u].z, cur.dy[u].w};
       const float xa[4] = {cur.x[u].x, cur.x[u].y, cur.x[u].z, cur.x[u].w};
 #pragma unroll
       for (int k = 0; k < 4; k++) {
@@ -355,8 +347,7 @@ __global__ void k_norm_bwd(NormBwd p) {
       if (!own || rr >= r1) continue;
       const float mg = p.rms ? 0.f : t[2 * u] / p.d;
       const float mgx = t[2 * u + 1] / p.d;
-      const float4 dy4 = widen4(cur.dy[u]);
-      const float dya[4] = {dy4.x, dy4.y, dy4.z, dy4.w};
+      const float dya[4] = {cur.dy[u].x, cur.dy[u].y, cur.dy[u].z, cur.dy[u].w};
       const float xa[4] = {cur.x[u].x, cur.x[u].y, cur.x[u].z, cur.x[u].w};
       const float ov[4] = {cur.old[u].x, cur.old[u].y, cur.old[u].z, cur.old[u].w};
       float nv[4];
