@@ -126,8 +126,7 @@ struct gpt_model {
   float *row_loss, *row_lse;
   int32_t *idx, *tgt, *stage_idx, *stage_tgt;
   // backward scratch
-  float *dres, *dsum, *splitk, *seg;
-  void* dln;  // the normalised rows' gradient (operand type: the dX GEMMs' output)
+  float *dres, *dln, *dsum, *splitk, *seg;
   uint8_t *dyb, *dqkv, *datt, *dh;
   int32_t *stok, *spos, *nuniq;
   double* norm_part;
@@ -403,7 +402,7 @@ size_t carve(gpt_model& m, uint8_t* base) {
   m.stage_idx = I((size_t)m.ga * M);
   m.stage_tgt = I((size_t)m.ga * M);
   m.dres = F((size_t)M * d);
-  m.dln = Bt((size_t)M * d);
+  m.dln = F((size_t)M * d);
   m.dsum = F((size_t)M * m.H);
   m.part_blocks = (int)std::min<long>(M, 148 * 8);  // capacity; the launch count is set at create
   m.part_cap = m.part_blocks;
@@ -795,7 +794,7 @@ gpt_status backward_t(gpt_model* m) {
   };
   // lm_head: dx_f = dlogits W_head; dW_head += dlogits^T x_f
   GemmDesc g = gd((int)M, d, Vp, dl, Vp, true, m->Wop(m->head), d, false);
-  g.epi.kind = EPI_STORE;
+  g.epi.kind = EPI_STORE_F32;
   g.name = "gemm_lmhead_dx";
   g.epi.out = m->dln;
   g.epi.ldo = d;
@@ -861,7 +860,7 @@ gpt_status backward_t(gpt_model* m) {
     }
     if (!dW(4 * d, d, dh, a2, m->G(y.fc_w), "gemm_fc_dw", l * 4 + 1)) return fail(m, GPT_ERR_CUDA, "fc dW failed");
     g = gd((int)M, d, 4 * d, dh, 4 * d, true, m->Wop(y.fc_w), d, false);
-    g.epi.kind = EPI_STORE;
+    g.epi.kind = EPI_STORE_F32;
     g.name = "gemm_fc_dx";
     g.epi.out = m->dln;
     g.epi.ldo = d;
@@ -920,7 +919,7 @@ gpt_status backward_t(gpt_model* m) {
       }
     }
     g = gd((int)M, d, 3 * d, dqkv, 3 * d, true, m->Wop(y.qkv_w), d, false);
-    g.epi.kind = EPI_STORE;
+    g.epi.kind = EPI_STORE_F32;
     g.name = "gemm_qkv_dx";
     g.epi.out = m->dln;
     g.epi.ldo = d;

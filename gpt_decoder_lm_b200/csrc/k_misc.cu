@@ -130,14 +130,6 @@ template void embed_fwd<bf16>(Ctx&, const int32_t*, const float*, const float*, 
 // lane).  LayerNorm: biased variance, y = (x - mean) * rstd * w + b.
 // RMSNorm (micro variant): y = x * rstd with rstd = 1/sqrt(mean(x^2) + eps).
 // ============================================================================
-// four consecutive operand-typed elements as floats (bf16: one 8-byte load)
-template <typename T> __device__ __forceinline__ float4 load4(const T* p);
-template <> __device__ __forceinline__ float4 load4<float>(const float* p) { return *reinterpret_cast<const float4*>(p); }
-template <> __device__ __forceinline__ float4 load4<bf16>(const bf16* p) {
-  const uint2 u = *reinterpret_cast<const uint2*>(p);
-  return make_float4(__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xffff0000u), __uint_as_float(u.y << 16),
-                     __uint_as_float(u.y & 0xffff0000u));
-}
 template <typename T> __device__ __forceinline__ void store4(T* p, float4 v);
 template <> __device__ __forceinline__ void store4<float>(float* p, float4 v) { *reinterpret_cast<float4*>(p) = v; }
 template <> __device__ __forceinline__ void store4<bf16>(bf16* p, float4 v) {
@@ -304,7 +296,7 @@ __global__ void k_norm_bwd(NormBwd p) {
       q.rstd[u] = live ? p.rstd[rr] : 0.f;
       q.dy[u] = q.x[u] = q.old[u] = make_float4(0, 0, 0, 0);
       if (own && live) {
-        q.dy[u] = load4<T>(reinterpret_cast<const T*>(p.dy) + rr * p.d + 4 * tid);
+        q.dy[u] = reinterpret_cast<const float4*>(p.dy + rr * p.d)[tid];
         q.x[u] = reinterpret_cast<const float4*>(p.x + rr * p.d)[tid];
         if (p.accumulate) q.old[u] = reinterpret_cast<const float4*>(p.dres + rr * p.d)[tid];
       }

@@ -193,8 +193,7 @@ void norm_fwd(Ctx& c, const float* x, const float* w, const float* b, T* y, floa
 // with dgain = sum dy*xhat and dbias = sum dy, go to per-block partials
 // part[blocks, 3, d] (order: dgain, dbeta, dbias_next).
 struct NormBwd {
-  const void* dy;  // operand type (the dX GEMM's output)
-  const float* x; const float* mean; const float* rstd; const float* w;
+  const float* dy; const float* x; const float* mean; const float* rstd; const float* w;
   float* dres; bool accumulate;
   void* dyb; DropKey drop; bool want_dyb;
   float* part; int blocks;
