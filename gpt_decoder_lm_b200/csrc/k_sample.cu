@@ -106,12 +106,63 @@ __global__ void __launch_bounds__(ST) k_sample(const T* __restrict__ logits, lon
   }
   __syncthreads();
 
-  // top-k: the integer image of the k-th largest logit
+  // top-k: the integer image of the k-th largest logit, by an MSB-first
+  // radix select.  The first byte is taken from the four byte values at and
+  // just below the maximum's, counted in registers (no histogram atomics);
+  // only when those hold fewer than k logits does the full first-byte
+  // histogram run.  bf16 logits widen to floats whose low 16 bits (of the
+  // integer image) are the same for every logit of one sign, so two byte
+  // passes decide them and the low half follows from the sign.
   uint32_t thr = 0;
   if (top_k > 0 && top_k < V) {
+    constexpr int kLow = sizeof(T) == 2 ? 16 : 0;  // the last byte pass starts at this bit
     uint32_t prefix = 0, mask = 0;
     int need = top_k;
-    for (int shift = 24; shift >= 0; shift -= 8) {
+    int shift = 24;
+    {
+      const int mb = (int)(fkey(zmax) >> 24);
+      int cnt[4] = {0, 0, 0, 0};
+#pragma unroll 4
+      for (int i = tid; i < V; i += ST) {
+        const int d = mb - (int)(fkey(to_f<T>(z[i])) >> 24);
+#pragma unroll
+        for (int j = 0; j < 4; j++) cnt[j] += d == j ? 1 : 0;
+      }
+#pragma unroll
+      for (int j = 0; j < 4; j++) {
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) cnt[j] += __shfl_xor_sync(0xffffffffu, cnt[j], o);
+      }
+      __shared__ int wcnt[ST / 32][4];
+      if (lane == 0) {
+#pragma unroll
+        for (int j = 0; j < 4; j++) wcnt[w][j] = cnt[j];
+      }
+      __syncthreads();
+      if (tid == 0) {
+        int cum = 0, found = -1;
+        for (int j = 0; j < 4 && mb - j >= 0; j++) {
+          int c = 0;
+          for (int k = 0; k < ST / 32; k++) c += wcnt[k][j];
+          if (cum + c >= need) {
+            found = j;
+            break;
+          }
+          cum += c;
+        }
+        sel[0] = found >= 0 ? (uint32_t)(mb - found) << 24 : 0xFFFFFFFFu;
+        sel[1] = (uint32_t)(need - cum);
+      }
+      __syncthreads();
+      if (sel[0] != 0xFFFFFFFFu) {  // the first byte is decided
+        prefix = sel[0];
+        need = (int)sel[1];
+        mask = 255u << 24;
+        shift = 16;
+      }
+      __syncthreads();
+    }
+    for (; shift >= kLow; shift -= 8) {
       for (int b = tid; b < 256; b += ST) hist[b] = 0;
       __syncthreads();
       for (int i0 = 0; i0 < V; i0 += 4 * ST) {  // whole warps iterate together, 4 loads in flight
@@ -148,6 +199,8 @@ __global__ void __launch_bounds__(ST) k_sample(const T* __restrict__ logits, lon
       mask |= 255u << shift;
       __syncthreads();
     }
+    // bf16: the low 16 bits of the image are 0 for positive logits, all ones for negative ones
+    if (kLow == 16) prefix |= (prefix & 0x80000000u) ? 0u : 0xFFFFu;
     thr = prefix;
   }
   const float inv_t = 1.0f / temperature;
