@@ -226,11 +226,14 @@ constexpr int SK_MAX_SMEM = 200 * 1024;
 int skinny_pitch(int K) { return ((2 * K + 127) / 128) * 128 + 64; }
 
 // K split: the fewest warps that leave each at most SK_U k blocks (one round
-// of loads), up to the CTA's warps
-int skinny_ks(const GemmDesc& g, int /*num_sms*/) {
-  const int nkb = g.K / 32;
+// of loads), then more while the grid has fewer CTAs than the GPU has SMs and
+// every warp keeps at least two k blocks (the weight stream spread over more
+// SMs), up to the CTA's warps
+int skinny_ks(const GemmDesc& g, int num_sms) {
+  const int nkb = g.K / 32, groups = (g.N + 15) / 16;
   int ks = 1;
   while (ks < SK_WARPS && (nkb + ks - 1) / ks > SK_U) ks *= 2;
+  while (ks < SK_WARPS && (groups + SK_WARPS / ks - 1) / (SK_WARPS / ks) < num_sms && nkb / (2 * ks) >= 2) ks *= 2;
   return ks;
 }
 
