@@ -419,7 +419,9 @@ def run_ours(args, w, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     gb.lib()
-    cfg = gb.make_config(w)
+    # --zero1: each rank's workspace holds the AdamW moments of its own shard only
+    sharded = args.zero1 and world > 1 and not args.replicas
+    cfg = gb.make_config(w, zero_world=world, zero_rank=rank) if sharded else gb.make_config(w)
     model = gb.Model(cfg, seed=w.weight_seed, device=dev)
     stream_host = W.token_stream(w)
     d_stream = torch.from_numpy(stream_host.view(np.int16)).to(dev)

@@ -18,7 +18,7 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libgpt.so")
 HEADERS = [os.path.join(os.path.dirname(_PKG), "include", h) for h in ("gpt.h", "gpt_testing.h")]
 
-GPT_ABI_VERSION = 1
+GPT_ABI_VERSION = 2
 GPT_PREC_FP32, GPT_PREC_BF16 = 0, 1
 GPT_VARIANT_GPT2, GPT_VARIANT_MICRO = 0, 1
 GPT_TOK_I32, GPT_TOK_U16 = 0, 1
@@ -37,7 +37,7 @@ class GptConfig(C.Structure):
         ("token_dtype", C.c_int32), ("dropout", C.c_float), ("beta1", C.c_float),
         ("beta2", C.c_float), ("eps", C.c_float), ("weight_decay", C.c_float), ("grad_clip", C.c_float),
         ("decay_1d", C.c_int32), ("recompute", C.c_int32), ("dropout_seed", C.c_uint64),
-        ("init_std", C.c_double),
+        ("init_std", C.c_double), ("zero_world", C.c_int32), ("zero_rank", C.c_int32),
     ]
 
 
@@ -57,7 +57,7 @@ _PROTOS = {
     "gpt_grad_buckets": (I32, [P, I32, P, P, P, P]),
     "gpt_grad_arena": (I32, [P, P, P]),
     "gpt_zero1_shard": (I32, [P, I32, I32, P, P, P]),
-    "gpt_state_arenas": (I32, [P, P, P, P, P, P, P, P]),
+    "gpt_state_arenas": (I32, [P, P, P, P, P, P, P, P, P]),
     "gpt_grad_sumsq_shard": (I32, [P, I64, I64, P]),
     "gpt_clip_adamw_shard": (I32, [P, F32, I32, I64, I64, F32, P, I32, P]),
     "gpt_train_step_accumulate": (I32, [P, P, U64, U64, I32, P]),
@@ -313,20 +313,22 @@ class Model:
         used length is ["n"])."""
         import torch
         ptr = [C.c_void_p() for _ in range(5)]
-        n, n_alloc = C.c_int64(), C.c_int64()
-        _check(lib().gpt_state_arenas(self.h, *[C.byref(x) for x in ptr], C.byref(n), C.byref(n_alloc)), self.h,
-               "state_arenas")
+        n, n_alloc, n_mom = C.c_int64(), C.c_int64(), C.c_int64()
+        _check(lib().gpt_state_arenas(self.h, *[C.byref(x) for x in ptr], C.byref(n), C.byref(n_alloc),
+                                      C.byref(n_mom)), self.h, "state_arenas")
         base = self.ws.data_ptr()
 
-        def view(p, dtype, esize):
+        def view(p, dtype, esize, length):
             if not p.value:
                 return None
             off = p.value - base
             assert off >= 0 and off % esize == 0
-            return self.ws[off:off + esize * n_alloc.value].view(dtype)
-        out = {k: view(p, torch.float32, 4) for k, p in zip(("param", "grad", "adam_m", "adam_v"), ptr)}
-        out["param_bf16"] = view(ptr[4], torch.bfloat16, 2)
+            return self.ws[off:off + esize * length].view(dtype)
+        out = {k: view(p, torch.float32, 4, n_alloc.value) for k, p in zip(("param", "grad"), ptr[:2])}
+        out.update({k: view(p, torch.float32, 4, n_mom.value) for k, p in zip(("adam_m", "adam_v"), ptr[2:4])})
+        out["param_bf16"] = view(ptr[4], torch.bfloat16, 2, n_alloc.value)
         out["n"] = int(n.value)
+        out["moments_sharded"] = self.cfg.zero_world > 1
         return out
 
     def grad_sumsq_shard(self, offset: int, count: int, partials):

@@ -96,6 +96,15 @@ struct Layout {
 constexpr int64_t kArenaSlack = 64 * 64;
 constexpr int kZeroMaxWorld = 64;
 
+// shard `rank` of `world` over an arena of n elements: equal strides that are
+// multiples of 64, the last one ragged (or empty)
+void zero_shard_of(int64_t n, int world, int rank, int64_t* off, int64_t* cnt, int64_t* stride) {
+  const int64_t S = ((n + world - 1) / world + 63) / 64 * 64;
+  *stride = S;
+  *off = std::min<int64_t>((int64_t)rank * S, n);
+  *cnt = std::max<int64_t>(0, std::min<int64_t>(S, n - *off));
+}
+
 // split-K count of a weight-gradient GEMM (sizes the partial-sum scratch; the
 // plan of a 148-SM B200)
 int choose_splits(long M, long N, long K) { return gemm_tc_plan(M, N, K, true, 148).splits; }
@@ -113,6 +122,9 @@ struct gpt_model {
   std::vector<LayerP> layers;
   int64_t wte, wpe, lnf_w = -1, lnf_b = -1, head;  // offsets
   int64_t n_total = 0, n_decay = 0;
+  // ZeRO-1 (zero_world > 1): the moments hold this rank's shard only
+  bool zero_sharded = false;
+  int64_t zero_off = 0, zero_cnt = 0, zero_stride = 0;
 
   uint8_t* ws = nullptr;
   size_t ws_bytes = 0;
@@ -254,6 +266,8 @@ gpt_status validate(const gpt_config* c, std::string* why) {
   if (!(c->beta1 >= 0.f && c->beta1 < 1.f && c->beta2 >= 0.f && c->beta2 < 1.f)) return bad("betas in [0, 1)");
   if (!(c->eps > 0.f) || !(c->init_std >= 0.0)) return bad("eps > 0 and init_std >= 0 required");
   if (c->recompute != 0 && c->recompute != 1) return bad("recompute must be 0 or 1");
+  if (c->zero_world < 0 || c->zero_world > kZeroMaxWorld) return bad("zero_world must be in [0, 64]");
+  if (c->zero_rank < 0 || c->zero_rank >= std::max(1, c->zero_world)) return bad("zero_rank must be in [0, zero_world)");
   return GPT_OK;
 }
 
@@ -359,6 +373,8 @@ void derive(gpt_model& m, const gpt_config* c) {
   m.rc = c->recompute != 0;
   m.asz = m.bf16m ? 2 : 4;
   build_tensors(m);
+  m.zero_sharded = c->zero_world > 1;
+  if (m.zero_sharded) zero_shard_of(m.n_total, c->zero_world, c->zero_rank, &m.zero_off, &m.zero_cnt, &m.zero_stride);
 }
 
 // Carves the workspace (base may be null to size it).  Returns total bytes.
@@ -375,8 +391,9 @@ size_t carve(gpt_model& m, uint8_t* base) {
   m.scal = F(64);
   m.w = F(P);
   m.g = F(P);
-  m.am = F(P);
-  m.av = F(P);
+  const size_t Pm = m.zero_sharded ? (size_t)m.zero_stride : P;  // moments: the own shard under ZeRO-1
+  m.am = F(Pm);
+  m.av = F(Pm);
   m.wb = m.bf16m ? (bf16*)(base + lay.take(P * 2)) : nullptr;
   const int La = m.rc ? 1 : L;  // slots of the recomputable activations
   m.res = F((size_t)(2 * L + 1) * M * d);
@@ -1214,8 +1231,9 @@ gpt_status gpt_create(const gpt_config* cfg, uint64_t seed, void* d_workspace, s
   const size_t arena_bytes = (size_t)(m->n_total + kArenaSlack) * 4;
   cudaMemsetAsync(m->w, 0, arena_bytes, st);
   cudaMemsetAsync(m->g, 0, arena_bytes, st);
-  cudaMemsetAsync(m->am, 0, arena_bytes, st);
-  cudaMemsetAsync(m->av, 0, arena_bytes, st);
+  const size_t moment_bytes = m->zero_sharded ? (size_t)m->zero_stride * 4 : arena_bytes;
+  cudaMemsetAsync(m->am, 0, moment_bytes, st);
+  cudaMemsetAsync(m->av, 0, moment_bytes, st);
   if (m->wb) cudaMemsetAsync(m->wb, 0, arena_bytes / 2, st);
   // weights from the seed, uploaded one tensor at a time
   std::vector<float> host;
@@ -1291,6 +1309,8 @@ gpt_status gpt_backward(gpt_model* m) {
 
 gpt_status gpt_clip_adamw_step(gpt_model* m, float lr, int32_t step, float* h_grad_norm) {
   if (!m) return GPT_ERR_INVALID_ARG;
+  if (m->zero_sharded && !m->lora.on)
+    return fail(m, GPT_ERR_UNSUPPORTED, "clip_adamw_step: the moments are sharded; use gpt_clip_adamw_shard");
   if (step < 1) return fail(m, GPT_ERR_INVALID_ARG, "step must be >= 1");
   gpt_status s = adamw_step(m, lr, step);
   if (s != GPT_OK) return s;
@@ -1374,6 +1394,8 @@ static bool capture_step(gpt_model* m, int kind, const void* d_stream, uint64_t 
 static gpt_status train_common(gpt_model* m, int kind, const void* d_stream, uint64_t len, uint64_t seed, float lr,
                                int32_t step, float* h_loss, float* h_norm) {
   if (step < 1) return fail(m, GPT_ERR_INVALID_ARG, "step must be >= 1");
+  if (kind < 2 && m->zero_sharded && !m->lora.on)
+    return fail(m, GPT_ERR_UNSUPPORTED, "train_step: the moments are sharded; use the accumulate form");
   Ctx& c = m->ctx;
   m->bucket_record = kind >= 2;
   // Replay a captured graph of the whole step: everything that changes from
@@ -1498,18 +1520,16 @@ gpt_status gpt_zero1_shard(const gpt_config* cfg, int32_t world, int32_t rank, i
   if (s != GPT_OK) return s;
   gpt_model m;
   derive(m, cfg);
-  const int64_t n = m.n_total;
-  const int64_t S = ((n + world - 1) / world + 63) / 64 * 64;
-  *stride = S;
-  *offset = std::min<int64_t>((int64_t)rank * S, n);
-  *count = std::max<int64_t>(0, std::min<int64_t>(S, n - *offset));
+  zero_shard_of(m.n_total, world, rank, offset, count, stride);
   return GPT_OK;
 }
 
 gpt_status gpt_state_arenas(gpt_model* m, float** d_param, float** d_grad, float** d_adam_m, float** d_adam_v,
-                            void** d_param_bf16, int64_t* n_floats, int64_t* n_alloc) {
-  if (!m || !d_param || !d_grad || !d_adam_m || !d_adam_v || !d_param_bf16 || !n_floats || !n_alloc)
+                            void** d_param_bf16, int64_t* n_floats, int64_t* n_alloc, int64_t* n_moment_alloc) {
+  if (!m || !d_param || !d_grad || !d_adam_m || !d_adam_v || !d_param_bf16 || !n_floats || !n_alloc ||
+      !n_moment_alloc)
     return GPT_ERR_INVALID_ARG;
+  *n_moment_alloc = m->zero_sharded ? m->zero_stride : m->n_total + kArenaSlack;
   *d_param = m->w;
   *d_grad = m->g;
   *d_adam_m = m->am;
@@ -1546,12 +1566,15 @@ gpt_status gpt_clip_adamw_shard(gpt_model* m, float lr, int32_t step, int64_t of
   if (!(grad_scale > 0.f) || !isfinite(grad_scale)) return fail(m, GPT_ERR_INVALID_ARG, "grad_scale must be > 0");
   gpt_status s = check_shard(m, offset, count, "clip_adamw_shard");
   if (s != GPT_OK) return s;
+  if (m->zero_sharded && (offset != m->zero_off || count != m->zero_cnt))
+    return fail(m, GPT_ERR_INVALID_ARG, "clip_adamw_shard: the model holds the moments of shard [%lld, +%lld) only",
+                (long long)m->zero_off, (long long)m->zero_cnt);
   Ctx& c = m->ctx;
   AdamArgs a;
   a.w = m->w + offset;
   a.g = m->g + offset;
-  a.m = m->am + offset;
-  a.v = m->av + offset;
+  a.m = m->zero_sharded ? m->am : m->am + offset;  // sharded: the compact moments of the own shard
+  a.v = m->zero_sharded ? m->av : m->av + offset;
   a.wb = m->wb ? m->wb + offset : nullptr;
   a.n = count;
   a.n_decay = std::max<int64_t>(0, std::min<int64_t>(count, m->n_decay - offset));
@@ -1786,6 +1809,8 @@ static float* kind_arena(gpt_model* m, int kind) {
 
 gpt_status gpt_get_tensor(gpt_model* m, int32_t i, int32_t kind, float* h_out) {
   if (!m || !h_out || i < 0 || i >= (int32_t)m->tensors.size()) return GPT_ERR_INVALID_ARG;
+  if (m->zero_sharded && (kind == GPT_ADAM_M || kind == GPT_ADAM_V))
+    return fail(m, GPT_ERR_UNSUPPORTED, "the moments are sharded (zero_world > 1)");
   float* a = kind_arena(m, kind);
   if (!a) return GPT_ERR_INVALID_ARG;
   const TensorRec& t = m->tensors[i];
@@ -1795,6 +1820,8 @@ gpt_status gpt_get_tensor(gpt_model* m, int32_t i, int32_t kind, float* h_out) {
 
 gpt_status gpt_set_tensor(gpt_model* m, int32_t i, int32_t kind, const float* h_in) {
   if (!m || !h_in || i < 0 || i >= (int32_t)m->tensors.size()) return GPT_ERR_INVALID_ARG;
+  if (m->zero_sharded && (kind == GPT_ADAM_M || kind == GPT_ADAM_V))
+    return fail(m, GPT_ERR_UNSUPPORTED, "the moments are sharded (zero_world > 1)");
   float* a = kind_arena(m, kind);
   if (!a) return GPT_ERR_INVALID_ARG;
   const TensorRec& t = m->tensors[i];
@@ -1871,6 +1898,7 @@ size_t gpt_state_floats(gpt_model* m) {
 
 gpt_status gpt_get_state(gpt_model* m, float* hp, float* hm, float* hv) {
   if (!m || !hp || !hm || !hv) return GPT_ERR_INVALID_ARG;
+  if (m->zero_sharded) return fail(m, GPT_ERR_UNSUPPORTED, "get_state: the moments are sharded (zero_world > 1)");
   size_t o = 0;
   for (auto& t : m->tensors) {
     size_t n = (size_t)t.rows * t.cols;
@@ -1884,6 +1912,7 @@ gpt_status gpt_get_state(gpt_model* m, float* hp, float* hm, float* hv) {
 
 gpt_status gpt_set_state(gpt_model* m, const float* hp, const float* hm, const float* hv) {
   if (!m || !hp || !hm || !hv) return GPT_ERR_INVALID_ARG;
+  if (m->zero_sharded) return fail(m, GPT_ERR_UNSUPPORTED, "set_state: the moments are sharded (zero_world > 1)");
   size_t o = 0;
   for (auto& t : m->tensors) {
     size_t n = (size_t)t.rows * t.cols;

@@ -143,6 +143,8 @@ class ZeroTrainer:
         self.world = dist.get_world_size(group) if dist.is_initialized() else 1
         self.rank = dist.get_rank(group) if dist.is_initialized() else 0
         self.offset, self.count, self.stride = gb.zero1_shard(model.cfg, self.world, self.rank)
+        if model.cfg.zero_world > 1 and (model.cfg.zero_world, model.cfg.zero_rank) != (self.world, self.rank):
+            raise ValueError("the model's zero_world / zero_rank differ from the process group's")
         self.arenas = model.state_arenas()
         self.parts = shard_parts(bucket_plan(model.cfg), self.stride, self.world)
         self.side = torch.cuda.Stream(device=model.device)
@@ -175,8 +177,12 @@ class ZeroTrainer:
 
     def gather_optimizer_state(self):
         """All-gather the AdamW moments so that every replica holds all of
-        them (before gpt_get_state on a sharded run)."""
+        them (before gpt_get_state on a sharded run).  Not with a model whose
+        config shards the moments themselves (zero_world > 1): it holds its
+        own shard only, which is what it checkpoints."""
         import torch
+        if self.arenas["moments_sharded"]:
+            raise RuntimeError("the model holds its own shard of the moments only (zero_world > 1)")
         with torch.cuda.stream(self.model.stream):
             for name in ("adam_m", "adam_v"):
                 all_gather_shards(self.arenas[name], self.stride, self.world, self.rank, self.group)

@@ -51,7 +51,7 @@
 extern "C" {
 #endif
 
-#define GPT_ABI_VERSION 1u
+#define GPT_ABI_VERSION 2u
 
 typedef enum {
   GPT_OK = 0,
@@ -119,6 +119,16 @@ typedef struct gpt_config {
   double init_std;        /* std of the Gaussian init of matrices and embeddings
                              (double: the init is computed in double precision and
                              rounded to fp32 once)                                   */
+  int32_t zero_world;     /* ZeRO stage 1 (sharded optimiser state).  0 or 1: the
+                             model holds every AdamW moment.  W in 2..64: the model
+                             is rank zero_rank of W data-parallel replicas and its
+                             workspace holds the moments of its own shard only
+                             (gpt_zero1_shard); the optimiser step is then
+                             gpt_clip_adamw_shard on that shard, and the calls that
+                             need every moment (gpt_train_step*, without the
+                             accumulate forms, gpt_clip_adamw_step, gpt_get_state,
+                             gpt_set_state) return GPT_ERR_UNSUPPORTED.            */
+  int32_t zero_rank;      /* 0 <= zero_rank < zero_world (0 when zero_world <= 1)    */
 } gpt_config;
 
 typedef struct gpt_model gpt_model;
@@ -286,13 +296,16 @@ gpt_status gpt_stream_wait_bucket(gpt_model* m, int32_t bucket, void* cuda_strea
  * place).  *count is 0 for a rank past the end.  Pure host. */
 gpt_status gpt_zero1_shard(const gpt_config* cfg, int32_t world, int32_t rank, int64_t* offset, int64_t* count,
                            int64_t* stride);
-/* Device addresses of the model's flat arenas (all with the same element
- * offsets): fp32 weights, gradients, AdamW first and second moments, and the
- * bf16 operand copy of the weights (null in fp32 mode).  *n_floats elements
- * are in use; each arena is allocated for *n_alloc >= n_floats + 4096
- * elements (the slack is never read by the step). */
+/* Device addresses of the model's flat arenas: fp32 weights, gradients, the
+ * AdamW first and second moments, and the bf16 operand copy of the weights
+ * (null in fp32 mode).  *n_floats elements are in use; the weight, gradient
+ * and bf16 arenas are allocated for *n_alloc >= n_floats + 4096 elements (the
+ * slack is never read by the step).  The moments use the same offsets and
+ * length, except with zero_world > 1, where they hold the own shard only:
+ * element offset + i of the arenas at index i, *n_moment_alloc = the shard
+ * stride. */
 gpt_status gpt_state_arenas(gpt_model* m, float** d_param, float** d_grad, float** d_adam_m, float** d_adam_v,
-                            void** d_param_bf16, int64_t* n_floats, int64_t* n_alloc);
+                            void** d_param_bf16, int64_t* n_floats, int64_t* n_alloc, int64_t* n_moment_alloc);
 /* GPT_NORM_PARTIALS partial sums of squares (fp64, device) of gradient
  * elements [offset, offset + count) into d_partials; their sum is the
  * shard's squared norm.  offset and count multiples of 4 (the shard bounds
@@ -307,7 +320,9 @@ gpt_status gpt_grad_sumsq_shard(gpt_model* m, int64_t offset, int64_t count, dou
  * order).  Clears the whole gradient arena.  h_grad_norm (nullable): the
  * global norm, read after a synchronise (GPT_ERR_NONFINITE as
  * gpt_clip_adamw_step).  With offset 0, count = the arena, grad_scale 1 and
- * the one rank's partials this is gpt_clip_adamw_step bit for bit. */
+ * the one rank's partials this is gpt_clip_adamw_step bit for bit.  With
+ * zero_world > 1 in the config, offset and count must be the config's own
+ * shard (the only moments the model holds), else GPT_ERR_INVALID_ARG. */
 gpt_status gpt_clip_adamw_shard(gpt_model* m, float lr, int32_t step, int64_t offset, int64_t count,
                                 float grad_scale, const double* d_partials, int32_t n_partials, float* h_grad_norm);
 
@@ -377,7 +392,8 @@ gpt_status gpt_num_tensors(gpt_model* m, int32_t* n);
 gpt_status gpt_tensor_info(gpt_model* m, int32_t i, const char** name, int64_t shape[2]);
 /* Copies tensor i of the given kind (GPT_PARAM .. GPT_ADAM_V) as fp32
  * to / from host memory (shape as gpt_tensor_info).  Setting GPT_PARAM also
- * refreshes the bf16 copy.  Synchronising. */
+ * refreshes the bf16 copy.  Synchronising.  The moment kinds are
+ * GPT_ERR_UNSUPPORTED with zero_world > 1 (the model holds one shard). */
 gpt_status gpt_get_tensor(gpt_model* m, int32_t i, int32_t kind, float* h_out);
 gpt_status gpt_set_tensor(gpt_model* m, int32_t i, int32_t kind, const float* h_in);
 /* Logits of the last forward as fp32 [B*T, vocab_size] (pad columns

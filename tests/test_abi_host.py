@@ -54,6 +54,8 @@ def test_lr_schedules_match_oracle(lib):
     ("dropout", 1.0, "GPT_ERR_CONFIG"),
     ("precision", 7, "GPT_ERR_CONFIG"),
     ("batch_size", 1000, "GPT_ERR_CONFIG"),    # B*T above the routing limit
+    ("zero_world", 65, "GPT_ERR_CONFIG"),      # at most 64 optimiser shards
+    ("zero_rank", 1, "GPT_ERR_CONFIG"),        # a rank needs zero_world > rank
 ])
 def test_invalid_configs_rejected_on_host(lib, field, value, status):
     cfg = gb.make_config(W.CHAR)
@@ -107,3 +109,16 @@ def test_kernel_paths_follow_the_shape_rule(lib, w, over, want):
     tensor-core GEMM; tensor-core attention at head_dim 64 and T a multiple
     of 128), never a fallback taken at run time."""
     assert gb.kernel_paths(gb.make_config(w, **over)) == want
+
+
+def test_sharded_moments_shrink_the_workspace(lib):
+    """zero_world > 1: the workspace holds the AdamW moments of the rank's
+    shard only (the other arenas are unchanged)."""
+    full = gb.make_config(W.GPT2_124M)
+    n = sum(c for _, c, _ in gb.grad_buckets(full))
+    for world in (2, 8):
+        for rank in (0, world - 1):
+            cfg = gb.make_config(W.GPT2_124M, zero_world=world, zero_rank=rank)
+            off, cnt, stride = gb.zero1_shard(cfg, world, rank)
+            saved = gb.workspace_bytes(full) - gb.workspace_bytes(cfg)
+            assert abs(saved - 8 * (n + 4096 - stride)) <= 1024

@@ -119,7 +119,10 @@ def test_two_ranks_zero1_emulated_equal_the_data_parallel_step():
     over = dict(n_layer=2, batch_size=4, block_size=128, grad_accum=2)
     cfg = gb.make_config(w, **over)
     world = 2
-    A, B, C = (gb.Model(cfg, seed=w.weight_seed) for _ in range(3))
+    # the two ranks hold the moments of their own shard only (zero_world 2)
+    A, B = (gb.Model(gb.make_config(w, zero_world=world, zero_rank=r, **over), seed=w.weight_seed)
+            for r in range(world))
+    C = gb.Model(cfg, seed=w.weight_seed)
     ar = [A.state_arenas(), B.state_arenas()]
     ref = C.state_arenas()
     n = ref["n"]
@@ -162,8 +165,38 @@ def test_two_ranks_zero1_emulated_equal_the_data_parallel_step():
             for name in ("param", "param_bf16"):
                 assert same(ar[r][name][:n], ref[name][:n]), (step, r, name)
             off, cnt, _ = shards[r]
-            for name in ("adam_m", "adam_v"):                      # each owner's moments
-                assert same(ar[r][name][off:off + cnt], ref[name][off:off + cnt]), (step, r, name)
+            for name in ("adam_m", "adam_v"):                      # each owner's moments (compact)
+                assert same(ar[r][name][:cnt], ref[name][off:off + cnt]), (step, r, name)
     for mdl in (A, B, C):
         assert mdl.flags() == 0
         mdl.close()
+
+
+def test_sharded_moments_model_limits():
+    """A model whose config shards the moments (zero_world 2) holds its own
+    shard of them only: the whole-arena optimiser calls and the moment
+    accessors refuse, the shard call accepts its own shard alone, and the
+    workspace is smaller by the other shard's moments."""
+    w = W.CHAR
+    over = dict(n_layer=2, batch_size=4, block_size=128, grad_accum=2)
+    full = gb.make_config(w, **over)
+    cfg = gb.make_config(w, zero_world=2, zero_rank=1, **over)
+    off, cnt, stride = gb.zero1_shard(cfg, 2, 1)
+    n = gb.Model(full, seed=1).state_arenas()["n"]
+    assert gb.workspace_bytes(full) - gb.workspace_bytes(cfg) >= 8 * (n + 4096 - stride) - 512
+    m = gb.Model(cfg, seed=w.weight_seed)
+    sd = torch.from_numpy(W.token_stream(w, n=1 << 16).astype(np.int32)).cuda()
+    for call in (lambda: m.train_step(sd, w.data_seed, 1e-3, 1), lambda: m.clip_adamw_step(1e-3, 1),
+                 lambda: m.get(gb.GPT_ADAM_M)):
+        with pytest.raises(gb.GptError) as e:
+            call()
+        assert e.value.name == "GPT_ERR_UNSUPPORTED"
+    m.train_step_accumulate(sd, w.data_seed, 1, sync=True)
+    parts = torch.zeros(gb.NORM_PARTIALS, dtype=torch.float64, device="cuda")
+    m.grad_sumsq_shard(off, cnt, parts)
+    with pytest.raises(gb.GptError) as e:
+        m.clip_adamw_shard(1e-3, 1, 0, cnt, 0.5, parts)
+    assert e.value.name == "GPT_ERR_INVALID_ARG"
+    assert m.clip_adamw_shard(1e-3, 1, off, cnt, 0.5, parts) > 0
+    assert m.flags() == 0
+    m.close()
