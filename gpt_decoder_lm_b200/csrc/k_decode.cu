@@ -18,7 +18,6 @@ template <typename T>
 __global__ void __launch_bounds__(DT) k_attn_decode(const T* __restrict__ qkv, int Tn, int H, int hd, int t,
                                                     float scale, T* __restrict__ o) {
   pdl_trigger();
-  pdl_wait();  // the step's keys / values and query come from the QKV GEMM before it
   extern __shared__ float sc[];  // [t + 1] scores, then probabilities
   __shared__ float red[DT / 32];
   __shared__ float part[DT];
@@ -84,7 +83,6 @@ template <typename T>
 __global__ void __launch_bounds__(DT) k_attn_decode_v(const T* __restrict__ qkv, int Tn, int H, int hd, int t,
                                                       float scale, T* __restrict__ o) {
   pdl_trigger();
-  pdl_wait();  // the step's keys / values and query come from the QKV GEMM before it
   constexpr int VEC = 16 / sizeof(T);
   extern __shared__ float sc[];  // [t + 1] scores, then probabilities
   __shared__ float red[DT / 32];
@@ -182,9 +180,9 @@ void attn_decode(Ctx& c, const T* qkv, int B, int Tn, int H, int hd, int t, T* o
   const size_t smem = (size_t)(t + 1) * sizeof(float);
   const float scale = 1.0f / sqrtf((float)hd);
   if (vec_ok)
-    launch_pdl(k_attn_decode_v<T>, B * H, DT, smem, c.stream, qkv, Tn, H, hd, t, scale, o);
+    k_attn_decode_v<T><<<B * H, DT, smem, c.stream>>>(qkv, Tn, H, hd, t, scale, o);
   else
-    launch_pdl(k_attn_decode<T>, B * H, DT, smem, c.stream, qkv, Tn, H, hd, t, scale, o);
+    k_attn_decode<T><<<B * H, DT, smem, c.stream>>>(qkv, Tn, H, hd, t, scale, o);
 }
 template void attn_decode<float>(Ctx&, const float*, int, int, int, int, int, float*);
 template void attn_decode<bf16>(Ctx&, const bf16*, int, int, int, int, int, bf16*);

@@ -53,8 +53,6 @@ template <typename T>
 __global__ void __launch_bounds__(ST) k_sample(const T* __restrict__ logits, long ld, int V, float temperature,
                                                int top_k, float top_p, const float* __restrict__ uniform,
                                                int32_t* __restrict__ out) {
-  pdl_trigger();
-  pdl_wait();  // the logits come from the head GEMM before it
   __shared__ float red[33];
   __shared__ uint32_t hist[256];
   __shared__ uint32_t sel[2];
@@ -411,11 +409,11 @@ void sample_rows(Ctx& c, const void* logits, bool bf16_logits, int rows, int V, 
                  float top_p, const float* uniform, int32_t* out) {
   LaunchScope s(c, "sample");
   if (bf16_logits)
-    launch_pdl(k_sample<bf16>, rows, ST, 0, c.stream, reinterpret_cast<const bf16*>(logits), ld, V, temperature,
-               top_k, top_p, uniform, out);
+    k_sample<bf16><<<rows, ST, 0, c.stream>>>(reinterpret_cast<const bf16*>(logits), ld, V, temperature, top_k,
+                                             top_p, uniform, out);
   else
-    launch_pdl(k_sample<float>, rows, ST, 0, c.stream, reinterpret_cast<const float*>(logits), ld, V, temperature,
-               top_k, top_p, uniform, out);
+    k_sample<float><<<rows, ST, 0, c.stream>>>(reinterpret_cast<const float*>(logits), ld, V, temperature, top_k,
+                                              top_p, uniform, out);
 }
 
 }  // namespace gpt
