@@ -437,7 +437,7 @@ TcPlan gemm_tc_plan(long M, long N, long K, bool split_ok, int num_sms, int mode
         const double kbc = pair ? KB_CYCLES_PAIR : (bn == 256 ? KB_CYCLES_256 : KB_CYCLES_128);
         double per_unit = (double)((nkb + s - 1) / s) * kbc + bn * 12.0;
         double t = waves * per_unit;
-        if (s > 1) t += 2.0 * s * M * N * 4 / (num_sms * 48.0);
+        if (s > 1) t += 2.0 * s * M * N * 4 / (num_sms * 96.0);
         if (t < best_t * 0.98) {
           best_t = t;
           best = TcPlan{bn, s, pair};
