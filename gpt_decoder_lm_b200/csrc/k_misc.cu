@@ -220,8 +220,9 @@ __global__ void __launch_bounds__(256) k_norm_fwd(const float* __restrict__ x, c
   }
 }
 
-// a single resident wave: the SM count times the blocks of this instantiation
-// that fit on an SM, at most one warp per row
+// at most a single resident wave (the SM count times the blocks of this
+// instantiation that fit on an SM), trimmed so that every warp walks the same
+// number of rows: with R rounds of rows per warp, ceil(rows / R) warps
 template <typename T, int VPL>
 void launch_norm_fwd(Ctx& c, const float* x, const float* w, const float* b, T* y, float* mean, float* rstd,
                      long rows, int d, bool rms, float eps) {
@@ -230,9 +231,10 @@ void launch_norm_fwd(Ctx& c, const float* x, const float* w, const float* b, T* 
     cudaGetLastError();
     occ = 1;
   }
-  long grid = (long)c.num_sms * occ;
-  const long need = (rows + 7) / 8;
-  if (grid > need) grid = need;
+  const long resident = (long)c.num_sms * occ * 8;  // warps
+  const long rounds = (rows + resident - 1) / resident;
+  const long warps = (rows + rounds - 1) / rounds;
+  const long grid = (warps + 7) / 8;
   k_norm_fwd<T, VPL><<<(unsigned)grid, 256, 0, c.stream>>>(x, w, b, y, mean, rstd, rows, d, rms, eps);
 }
 
