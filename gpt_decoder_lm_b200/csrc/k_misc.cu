@@ -817,21 +817,29 @@ __global__ void k_embed_bwd_wpe(const float* __restrict__ dres, int Bn, int Tn, 
 constexpr int EC = 32;
 enum : int8_t { SEG_NONE = 0, SEG_INNER = 1, SEG_HEAD = 2, SEG_TAIL = 3 };
 
-__global__ void __launch_bounds__(256, 2) k_embed_seg_a(const float* __restrict__ dres, const int32_t* __restrict__ stok,
-                                                     const int32_t* __restrict__ spos, int M, int d, DropKey drop,
-                                                     float* __restrict__ dwte, float* __restrict__ head,
-                                                     float* __restrict__ tail) {
+// Grid: chunks x column groups of SEG_T columns, one column per thread, so a
+// block does one pass over its chunk; the per-slot row offsets, destination
+// rows and segment ends are prepared once per block in shared memory.
+constexpr int SEG_T = 256;
+
+template <bool DROP>
+__global__ void __launch_bounds__(SEG_T, 2) k_embed_seg_a(const float* __restrict__ dres,
+                                                          const int32_t* __restrict__ stok,
+                                                          const int32_t* __restrict__ spos, int M, int d, DropKey drop,
+                                                          float* __restrict__ dwte, float* __restrict__ head,
+                                                          float* __restrict__ tail) {
   pdl_trigger();
   pdl_wait();
-  __shared__ int s_tok[EC + 2], s_pos[EC];
-  __shared__ int8_t s_kind[EC];  // what ends at slot k: nothing, an inner segment, the head, the tail
-  drop = drop_live(drop);
+  __shared__ int s_tok[EC + 2];
+  __shared__ long long s_src[EC], s_dst[EC];  // element offsets of the slot's dres row and dwte row
+  __shared__ int8_t s_kind[EC];                // what ends at slot k: nothing, an inner segment, the head, the tail
+  if (DROP) drop = drop_live(drop);
   const int c = blockIdx.x;
   const int j0 = c * EC, j1 = min(M, j0 + EC);
   const int n = j1 - j0;
   if (threadIdx.x < n) {
     s_tok[threadIdx.x + 1] = stok[j0 + threadIdx.x];
-    s_pos[threadIdx.x] = spos[j0 + threadIdx.x];
+    s_src[threadIdx.x] = (long long)spos[j0 + threadIdx.x] * d;
   }
   if (threadIdx.x == 0) {
     s_tok[0] = j0 > 0 ? stok[j0 - 1] : -1;
@@ -849,36 +857,37 @@ __global__ void __launch_bounds__(256, 2) k_embed_seg_a(const float* __restrict_
         const bool continues = k == n - 1 && s_tok[n + 1] == tok;
         kind = began_before ? SEG_HEAD : continues ? SEG_TAIL : SEG_INNER;
       }
+      s_dst[k] = (long long)tok * d;
     }
     s_kind[k] = kind;
   }
   __syncthreads();
-  for (int col = threadIdx.x; col < d; col += blockDim.x) {
-    float vals[EC];
+  const int col = blockIdx.y * SEG_T + threadIdx.x;
+  if (col >= d) return;
+  float vals[EC];
 #pragma unroll
-    for (int k = 0; k < EC; k++) vals[k] = k < n ? dres[(long)s_pos[k] * d + col] : 0.f;
-    // segment sums in slot order, left in vals[k] at the slot where each ends
-    float acc = 0.f;
+  for (int k = 0; k < EC; k++) vals[k] = k < n ? dres[s_src[k] + col] : 0.f;
+  // segment sums in slot order, left in vals[k] at the slot where each ends
+  float acc = 0.f;
 #pragma unroll
-    for (int k = 0; k < EC; k++) {
-      float v = vals[k];
-      if (drop.active && k < n) v *= drop_mul(drop, (uint64_t)s_pos[k] * d + col);
-      acc += v;
-      if (s_kind[k] != SEG_NONE) {
-        vals[k] = acc;
-        acc = 0.f;
-      }
+  for (int k = 0; k < EC; k++) {
+    float v = vals[k];
+    if (DROP && k < n) v *= drop_mul(drop, (uint64_t)(s_src[k] + col));
+    acc += v;
+    if (s_kind[k] != SEG_NONE) {
+      vals[k] = acc;
+      acc = 0.f;
     }
-    float old[EC];
+  }
+  float old[EC];
 #pragma unroll
-    for (int k = 0; k < EC; k++) old[k] = s_kind[k] == SEG_INNER ? dwte[(long)s_tok[k + 1] * d + col] : 0.f;
+  for (int k = 0; k < EC; k++) old[k] = s_kind[k] == SEG_INNER ? dwte[s_dst[k] + col] : 0.f;
 #pragma unroll
-    for (int k = 0; k < EC; k++) {
-      const int kind = s_kind[k];
-      if (kind == SEG_INNER) dwte[(long)s_tok[k + 1] * d + col] = old[k] + vals[k];
-      else if (kind == SEG_HEAD) head[(long)c * d + col] = vals[k];
-      else if (kind == SEG_TAIL) tail[(long)c * d + col] = vals[k];
-    }
+  for (int k = 0; k < EC; k++) {
+    const int kind = s_kind[k];
+    if (kind == SEG_INNER) dwte[s_dst[k] + col] = old[k] + vals[k];
+    else if (kind == SEG_HEAD) head[(long)c * d + col] = vals[k];
+    else if (kind == SEG_TAIL) tail[(long)c * d + col] = vals[k];
   }
 }
 
@@ -948,7 +957,11 @@ void embed_bwd(Ctx& c, const float* dres, const int32_t* sorted_tok, const int32
     const int chunks = (int)((M + EC - 1) / EC);
     float* head = seg_scratch;
     float* tail = seg_scratch + (size_t)chunks * d;
-    k_embed_seg_a<<<chunks, 256, 0, c.stream>>>(dres, sorted_tok, sorted_pos, (int)M, d, drop, dwte, head, tail);
+    const dim3 ga(chunks, (d + SEG_T - 1) / SEG_T);
+    if (drop.active)
+      k_embed_seg_a<true><<<ga, SEG_T, 0, c.stream>>>(dres, sorted_tok, sorted_pos, (int)M, d, drop, dwte, head, tail);
+    else
+      k_embed_seg_a<false><<<ga, SEG_T, 0, c.stream>>>(dres, sorted_tok, sorted_pos, (int)M, d, drop, dwte, head, tail);
     k_embed_seg_b<<<chunks, 256, 0, c.stream>>>(sorted_tok, (int)M, d, head, tail, dwte);
   }
   {
