@@ -723,65 +723,127 @@ void loss_reduce(Ctx& c, const float* row_loss, long M, float scale, float* loss
 }
 
 // ============================================================================
-// embedding backward.  Routing: key = token << 16 | position is unique, so a
-// plain bitonic sort of the keys equals a stable sort of positions by token.
+// embedding backward.  Routing: the keys token << 16 | position sorted by
+// token, stably (positions ascending within a token): an LSD radix sort, four
+// passes of 4 bits of the token, one CTA of 1024 threads per batch.  A pass
+// walks the keys in their current order in rounds of 1024 (one per thread); a
+// warp ranks each lane among the lanes with the same digit by four ballots,
+// the per-(round, warp) digit counts are scanned in that order for every
+// digit, and each key moves to its digit's base + the keys of that digit
+// before it.  The keys alternate between two shared-memory arrays, or, when
+// 2 M keys do not fit, between one and the stok array.
 // ============================================================================
-__global__ void k_embed_sort(const int32_t* __restrict__ idx, int M, int P2, int32_t* __restrict__ stok,
-                             int32_t* __restrict__ spos, int32_t* __restrict__ n_unique) {
+constexpr int RS_T = 1024, RS_W = RS_T / 32, RS_MAXR = 32;  // rounds of 1024 keys: M <= 32768
+
+__global__ void __launch_bounds__(RS_T) k_embed_sort(const int32_t* __restrict__ idx, int M, int smem2,
+                                                     int32_t* __restrict__ stok, int32_t* __restrict__ spos,
+                                                     int32_t* __restrict__ n_unique) {
   pdl_trigger();
   pdl_wait();
-  extern __shared__ uint32_t key[];
-  __shared__ int cnt[32];
+  extern __shared__ uint32_t key[];                 // [M] (and the second array [M] when smem2)
+  __shared__ uint16_t cnt[RS_MAXR * RS_W][16];     // digit counts per (round, warp), then their prefixes
+  __shared__ uint32_t base[16];
+  __shared__ int ucnt[RS_W];
   // block b sorts the b-th batch of M tokens (batches stored back to back)
   idx += (long)blockIdx.x * M;
   stok += (long)blockIdx.x * M;
   spos += (long)blockIdx.x * M;
   n_unique += blockIdx.x;
-  for (int i = threadIdx.x; i < P2; i += blockDim.x)
-    key[i] = i < M ? (((uint32_t)idx[i] << 16) | (uint32_t)i) : 0xFFFFFFFFu;
-  __syncthreads();
-  for (int k = 2; k <= P2; k <<= 1) {
-    for (int j = k >> 1; j > 0; j >>= 1) {
-      for (int i = threadIdx.x; i < P2; i += blockDim.x) {
-        int l = i ^ j;
-        if (l > i) {
-          uint32_t a = key[i], b = key[l];
-          bool up = (i & k) == 0;
-          if ((a > b) == up) {
-            key[i] = b;
-            key[l] = a;
-          }
-        }
+  uint32_t* gkey = smem2 ? key + M : reinterpret_cast<uint32_t*>(stok);
+  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+  const int R = (M + RS_T - 1) / RS_T;
+  const uint32_t lt = (1u << lane) - 1u;
+  for (int i = tid; i < M; i += RS_T) key[i] = ((uint32_t)idx[i] << 16) | (uint32_t)i;
+  // lanes of this warp whose digit equals this lane's (valid lanes only)
+  auto peers = [&](bool valid, uint32_t d) {
+    uint32_t m = __ballot_sync(0xffffffffu, valid);
+#pragma unroll
+    for (int b = 0; b < 4; b++) {
+      const uint32_t bb = __ballot_sync(0xffffffffu, valid && ((d >> b) & 1u));
+      m &= ((d >> b) & 1u) ? bb : ~bb;
+    }
+    return m;
+  };
+  for (int pass = 0; pass < 4; pass++) {
+    const int sh = 16 + 4 * pass;
+    const uint32_t* src = (pass & 1) ? gkey : key;
+    uint32_t* dst = (pass & 1) ? key : gkey;
+    __syncthreads();  // the previous pass's keys are in place and its counts read
+    for (int i = tid; i < R * RS_W * 16; i += RS_T) (&cnt[0][0])[i] = 0;
+    __syncthreads();
+    for (int r = 0; r < R; r++) {
+      const int e = r * RS_T + tid;
+      const bool valid = e < M;
+      const uint32_t d = valid ? (src[e] >> sh) & 15u : 0u;
+      const uint32_t m = peers(valid, d);
+      if (valid && (m & lt) == 0) cnt[r * RS_W + w][d] = (uint16_t)__popc(m);
+    }
+    __syncthreads();
+    if (w < 16) {  // warp w: exclusive prefix of digit w's counts over the slots in order
+      const int slots = R * RS_W, per = (slots + 31) / 32;
+      const int s0 = min(slots, lane * per), s1 = min(slots, s0 + per);
+      uint32_t loc = 0;
+      for (int q = s0; q < s1; q++) loc += cnt[q][w];
+      uint32_t inc = loc;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t x = __shfl_up_sync(0xffffffffu, inc, o);
+        if (lane >= o) inc += x;
       }
-      __syncthreads();
+      uint32_t run = inc - loc;
+      for (int q = s0; q < s1; q++) {
+        const uint32_t c = cnt[q][w];
+        cnt[q][w] = (uint16_t)run;
+        run += c;
+      }
+      if (lane == 31) base[w] = inc;  // the digit's total, for now
+    }
+    __syncthreads();
+    if (tid == 0) {
+      uint32_t run = 0;
+      for (int d = 0; d < 16; d++) {
+        const uint32_t t = base[d];
+        base[d] = run;
+        run += t;
+      }
+    }
+    __syncthreads();
+    for (int r = 0; r < R; r++) {
+      const int e = r * RS_T + tid;
+      const bool valid = e < M;
+      const uint32_t k = valid ? src[e] : 0u;
+      const uint32_t d = (k >> sh) & 15u;
+      const uint32_t m = peers(valid, d);
+      if (valid) dst[base[d] + cnt[r * RS_W + w][d] + __popc(m & lt)] = k;
     }
   }
+  __syncthreads();  // the sorted keys are in shared memory
   int u = 0;
-  for (int i = threadIdx.x; i < M; i += blockDim.x) {
-    uint32_t kk = key[i];
+  for (int i = tid; i < M; i += RS_T) {
+    const uint32_t kk = key[i];
     stok[i] = (int32_t)(kk >> 16);
     spos[i] = (int32_t)(kk & 0xFFFFu);
     if (i == 0 || (key[i - 1] >> 16) != (kk >> 16)) u++;
   }
   for (int o = 16; o > 0; o >>= 1) u += __shfl_xor_sync(0xffffffffu, u, o);
-  if ((threadIdx.x & 31) == 0) cnt[threadIdx.x >> 5] = u;
+  if (lane == 0) ucnt[w] = u;
   __syncthreads();
-  if (threadIdx.x == 0) {
+  if (tid == 0) {
     int t = 0;
-    for (int k = 0; k < (int)(blockDim.x >> 5); k++) t += cnt[k];
+    for (int k = 0; k < RS_W; k++) t += ucnt[k];
     *n_unique = t;
   }
 }
 
 void embed_sort(Ctx& c, const int32_t* idx, long M, int32_t* sorted_tok, int32_t* sorted_pos, int32_t* n_unique,
                 int batches) {
-  int P2 = 1;
-  while (P2 < M) P2 <<= 1;
-  size_t smem = (size_t)P2 * 4;
+  constexpr size_t kMaxDyn = 190 * 1024;  // with the kernel's 33 KB of static shared memory
+  const int smem2 = (size_t)M * 8 <= kMaxDyn ? 1 : 0;
+  const size_t smem = (size_t)M * 4 * (smem2 ? 2 : 1);
   // per-device function attribute: set before every launch
-  cudaFuncSetAttribute(k_embed_sort, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+  cudaFuncSetAttribute(k_embed_sort, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kMaxDyn);
   LaunchScope s(c, "embed_sort");
-  k_embed_sort<<<batches, 1024, smem, c.stream>>>(idx, (int)M, P2, sorted_tok, sorted_pos, n_unique);
+  k_embed_sort<<<batches, RS_T, smem, c.stream>>>(idx, (int)M, smem2, sorted_tok, sorted_pos, n_unique);
 }
 
 // dwte[v] += sum over the sorted positions of token v (in position order) of

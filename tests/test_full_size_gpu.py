@@ -169,3 +169,24 @@ def test_embedding_routing_full_micro_batch():
     assert np.array_equal(pos, order)
     assert n == np.unique(flat).size
     m.close()
+
+
+@pytest.mark.parametrize("B,T", [(3, 1000), (24, 1024), (32, 1024)], ids=["ragged", "global24k", "max32k"])
+def test_embedding_routing_sizes(B, T):
+    # the radix routing sort at a ragged size (a partial last round of 1024
+    # keys) and past the shared-memory ping-pong (2 M keys above 190 KB: the
+    # second key array is the output array), up to the largest micro-batch a
+    # config allows (32,768 tokens); a one-layer model of the GPT-2 vocabulary
+    w = W.GPT2_124M.with_(token_dtype="int32")
+    cfg = gb.make_config(w, n_layer=1, n_head=1, n_embd=64, batch_size=B, block_size=T, grad_accum=1)
+    m = gb.Model(cfg, seed=w.weight_seed)
+    idx, tgt = W.random_batch(w, 91 + B, B, T)
+    m.forward_loss(torch.from_numpy(idx).cuda(), torch.from_numpy(tgt).cuda())
+    m.backward()
+    n, tok, pos = m.embed_routing()
+    flat = idx.reshape(-1)
+    order = np.lexsort((np.arange(flat.size), flat))
+    assert np.array_equal(tok, flat[order])
+    assert np.array_equal(pos, order)
+    assert n == np.unique(flat).size
+    m.close()
