@@ -2,6 +2,7 @@
 // LayerNorm/RMSNorm, cross-entropy, column sums, embedding backward,
 // gradient norm and the fused clip + AdamW update.
 #include "kernels.cuh"
+#include "sm100.cuh"
 
 #include <math.h>
 
@@ -684,12 +685,217 @@ __global__ void __launch_bounds__(256, 4) k_ce_stream(T* __restrict__ logits, co
   }
 }
 
+// Rows staged in shared memory: two blocks per SM, each with one row buffer,
+// walk their rows; a row arrives by bulk copies (TMA, cp.async.bulk) and both
+// passes read the staged copy, so each logit is read from HBM once: pass 1
+// (the row's log-sum-exp) and pass 2 (softmax - onehot, written in place).
+// While one block waits for its next row, the other computes.  The arithmetic
+// is k_ce_stream's (16-byte vectors strided over the block's threads, an
+// online (max, sum) per thread, then warp and block merges in a fixed order)
+// with fewer instructions per logit: bf16 widened by bit shifts, the
+// vocabulary mask and the one-hot term only where they can apply, exponents
+// and scaling as paired (f32x2) operations, two running sums per thread.
+// Every wait is bounded; a block that gives up raises FLAG_TIMEOUT, waits for
+// its own copies in flight (again bounded) and returns.
+constexpr int CE_THREADS = 512;
+
+// a 16-byte vector of logits as floats (bf16 widened exactly by bit shifts),
+// and back (round to nearest)
+template <typename T>
+__device__ __forceinline__ void ce_unpack(const uint4& u, float (&x)[16 / sizeof(T)]) {
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+  if constexpr (sizeof(T) == 2) {
+#pragma unroll
+    for (int k = 0; k < 4; k++) {
+      x[2 * k] = __uint_as_float(w[k] << 16);
+      x[2 * k + 1] = __uint_as_float(w[k] & 0xffff0000u);
+    }
+  } else {
+#pragma unroll
+    for (int k = 0; k < 4; k++) x[k] = __uint_as_float(w[k]);
+  }
+}
+template <typename T>
+__device__ __forceinline__ uint4 ce_pack(const float (&g)[16 / sizeof(T)]) {
+  uint32_t w[4];
+  if constexpr (sizeof(T) == 2) {
+#pragma unroll
+    for (int k = 0; k < 4; k++) {
+      const __nv_bfloat162 v = __floats2bfloat162_rn(g[2 * k], g[2 * k + 1]);
+      w[k] = *reinterpret_cast<const uint32_t*>(&v);
+    }
+  } else {
+#pragma unroll
+    for (int k = 0; k < 4; k++) w[k] = __float_as_uint(g[k]);
+  }
+  return make_uint4(w[0], w[1], w[2], w[3]);
+}
+constexpr uint32_t CE_CHUNK = 32768;  // bytes per bulk copy
+
+template <typename T>
+__global__ void __launch_bounds__(CE_THREADS, 2) k_ce_smem(T* __restrict__ logits, const int32_t* __restrict__ tgt,
+                                                          long M, int V, int Vp, float* __restrict__ lse_out,
+                                                          float* __restrict__ row_loss, int want_grad, float scale,
+                                                          uint32_t* flags) {
+  pdl_trigger();
+  constexpr int EPV = 16 / sizeof(T);
+  constexpr float LOG2E = 1.4426950408889634f;
+  extern __shared__ __align__(128) uint8_t smem[];
+  __shared__ float sm[CE_THREADS / 32], ss[CE_THREADS / 32];
+  __shared__ __align__(8) uint64_t full[2];
+  __shared__ int abort_flag;
+  const uint32_t RB = (uint32_t)Vp * sizeof(T);  // row bytes (a multiple of 16)
+  const uint32_t RBA = (RB + 127) & ~127u;       // buffer stride
+  const int nvec = Vp / EPV;
+  int issued[2] = {0, 0}, waited[2] = {0, 0};    // copies per buffer (kept by thread 0)
+  auto issue = [&](long row, int b) {            // thread 0: the bulk copies of one row into buffer b
+    issued[b]++;
+    const uint32_t bar = sm100::smem_u32(&full[b]);
+    const uint32_t dst = sm100::smem_u32(smem + b * RBA);
+    const uint8_t* src = reinterpret_cast<const uint8_t*>(logits + row * Vp);
+    sm100::fence_proxy_async_smem();  // the buffer's earlier generic reads come first
+    sm100::mbar_expect_tx(bar, RB);
+    for (uint32_t o = 0; o < RB; o += CE_CHUNK) sm100::bulk_load(dst + o, src + o, min(CE_CHUNK, RB - o), bar);
+  };
+  if (threadIdx.x == 0) {
+    sm100::mbar_init(sm100::smem_u32(&full[0]), 1);
+    sm100::mbar_init(sm100::smem_u32(&full[1]), 1);
+    abort_flag = 0;
+    sm100::fence_barrier_init();
+    if (blockIdx.x < M) issue(blockIdx.x, 0);
+  }
+  __syncthreads();
+  int it = 0;
+  for (long row = blockIdx.x; row < M; row += gridDim.x, it++) {
+    const int b = 0;  // one row buffer: the other block on the SM covers this one's load
+    const bool ok = sm100::mbar_wait(sm100::smem_u32(&full[b]), it & 1, &abort_flag, flags);
+    if (__syncthreads_or(!ok)) break;  // every thread takes the same branch
+    waited[b]++;
+    const T* z = reinterpret_cast<const T*>(smem + b * RBA);
+    const uint4* z4 = reinterpret_cast<const uint4*>(z);
+    const int t = tgt[row];
+    const int vfull = V / EPV;  // vectors below it lie inside the vocabulary
+    const uint64_t l2 = f2(LOG2E, LOG2E);
+    // pass 1: online (max, sum) of 2^(z log2 e), masks only in the last vectors,
+    // the exponents as paired FMAs, two running sums
+    float m = -INFINITY, s0 = 0.f, s1 = 0.f;
+    for (int vi = threadIdx.x; vi < nvec; vi += CE_THREADS) {
+      if (vi * EPV >= V) continue;
+      float x[EPV];
+      ce_unpack<T>(z4[vi], x);
+      if (vi >= vfull) {
+#pragma unroll
+        for (int k = 0; k < EPV; k++)
+          if (vi * EPV + k >= V) x[k] = -INFINITY;
+      }
+      float mv = x[0];
+#pragma unroll
+      for (int k = 1; k < EPV; k++) mv = fmaxf(mv, x[k]);
+      mv *= LOG2E;
+      if (mv > m) {
+        if (m != -INFINITY) {
+          const float r = sfu_ex2(m - mv);
+          s0 *= r;
+          s1 *= r;
+        }
+        m = mv;
+      }
+      const uint64_t nm = f2(-m, -m);
+#pragma unroll
+      for (int k = 0; k < EPV; k += 2) {
+        const float2 y = f2split(f2fma(f2(x[k], x[k + 1]), l2, nm));
+        s0 += sfu_ex2(y.x);
+        s1 += sfu_ex2(y.y);
+      }
+    }
+    float s = s0 + s1;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      float m2 = __shfl_xor_sync(0xffffffffu, m, o);
+      float s2 = __shfl_xor_sync(0xffffffffu, s, o);
+      lse_merge(m, s, m2, s2);
+    }
+    const int w = threadIdx.x >> 5;
+    if ((threadIdx.x & 31) == 0) {
+      sm[w] = m;
+      ss[w] = s;
+    }
+    __syncthreads();
+    float Mx = sm[0], S = ss[0];
+#pragma unroll
+    for (int k = 1; k < CE_THREADS / 32; k++) lse_merge(Mx, S, sm[k], ss[k]);
+    const float lse2 = Mx + log2f(S);  // log2-domain log-sum-exp
+    const float lse = lse2 * 0.6931471805599453f;
+    if (threadIdx.x == 0) {
+      lse_out[row] = lse;
+      row_loss[row] = lse - to_f<T>(z[t]);
+    }
+    if (want_grad) {
+      // pass 2: (2^(z log2 e - lse2) - [j == t]) * scale, zero past the vocabulary
+      uint4* dst = reinterpret_cast<uint4*>(logits + row * Vp);
+      const uint64_t nl = f2(-lse2, -lse2), sc2 = f2(scale, scale);
+      const int tv = t / EPV;
+      for (int vi = threadIdx.x; vi < nvec; vi += CE_THREADS) {
+        float x[EPV], g[EPV];
+        ce_unpack<T>(z4[vi], x);
+#pragma unroll
+        for (int k = 0; k < EPV; k += 2) {
+          const float2 y = f2split(f2fma(f2(x[k], x[k + 1]), l2, nl));
+          g[k] = sfu_ex2(y.x);
+          g[k + 1] = sfu_ex2(y.y);
+        }
+        if (vi == tv) {
+#pragma unroll
+          for (int k = 0; k < EPV; k++)
+            if (vi * EPV + k == t) g[k] -= 1.f;
+        }
+#pragma unroll
+        for (int k = 0; k < EPV; k += 2) {
+          const float2 q = f2split(f2mul(f2(g[k], g[k + 1]), sc2));
+          g[k] = q.x;
+          g[k + 1] = q.y;
+        }
+        if (vi >= vfull) {
+#pragma unroll
+          for (int k = 0; k < EPV; k++)
+            if (vi * EPV + k >= V) g[k] = 0.f;
+        }
+        dst[vi] = ce_pack<T>(g);
+      }
+    }
+    __syncthreads();  // the buffer and sm / ss are free again
+    if (threadIdx.x == 0 && row + gridDim.x < M) issue(row + gridDim.x, 0);
+  }
+  if (threadIdx.x == 0) {
+    // after a failed wait: no copy of this block may still be writing its
+    // shared memory when it exits (bounded waits, which ignore the abort flag)
+    volatile int no_abort = 0;
+    for (int k = 0; k < 2; k++)
+      for (; waited[k] < issued[k]; waited[k]++)
+        if (!sm100::mbar_wait(sm100::smem_u32(&full[k]), waited[k] & 1, &no_abort, flags, 100000000ull)) break;
+  }
+}
+
+// shared memory of k_ce_smem for rows of `row_bytes` (0: the row does not fit)
+size_t ce_smem_bytes(size_t row_bytes) {
+  if (row_bytes % 16) return 0;
+  const size_t b = (row_bytes + 127) & ~size_t(127);
+  return b <= 110 * 1024 ? b : 0;
+}
+
 template <typename T>
 void ce_fwd_bwd(Ctx& c, T* logits, const int32_t* tgt, long M, int V, int Vp, float* lse, float* row_loss,
                 bool want_grad, float scale) {
   LaunchScope s(c, want_grad ? "ce_fwd_bwd" : "ce_fwd");
   constexpr int EPV = 16 / sizeof(T);
-  if (Vp % EPV == 0)
+  const size_t sh = ce_smem_bytes((size_t)Vp * sizeof(T));
+  if (Vp % EPV == 0 && sh > 0) {
+    // per-device function attribute: set before every launch
+    cudaFuncSetAttribute(k_ce_smem<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sh);
+    const unsigned grid = (unsigned)std::min<long>(M, 2L * c.num_sms);
+    k_ce_smem<T><<<grid, CE_THREADS, sh, c.stream>>>(logits, tgt, M, V, Vp, lse, row_loss, want_grad ? 1 : 0, scale,
+                                                     c.flags);
+  } else if (Vp % EPV == 0)
     k_ce_stream<T><<<(unsigned)M, 256, 0, c.stream>>>(logits, tgt, V, Vp, lse, row_loss, want_grad ? 1 : 0, scale);
   else
     k_ce<T><<<(unsigned)M, 512, 0, c.stream>>>(logits, tgt, V, Vp, lse, row_loss, want_grad ? 1 : 0, scale);
