@@ -82,7 +82,7 @@ def attn_flops_per_step(w) -> float:
 # pass, on `bench.py --layer-case 2`: every GEMM shape of a layer and the lm_head at full size),
 # weighted to the 12-layer step: (12 x one layer's 12 GEMMs + the lm_head's 3) / 147 launches.
 # None once the kernels change after that capture.
-GEMM_DRAM_BYTES_PER_LAUNCH = 107803514
+GEMM_DRAM_BYTES_PER_LAUNCH = 107559868
 
 
 class Clocks:
