@@ -200,3 +200,29 @@ def test_sharded_moments_model_limits():
     assert m.clip_adamw_shard(1e-3, 1, off, cnt, 0.5, parts) > 0
     assert m.flags() == 0
     m.close()
+
+
+def test_zero1_empty_shard_rank():
+    """A rank past the end of a small arena (64 shards of the micro model's
+    4k-element arena) owns nothing: its shard calls run on an empty range,
+    clear its gradients and leave its weights as they were."""
+    w = W.MICRO
+    world, rank = 64, 63
+    cfg = gb.make_config(w, zero_world=world, zero_rank=rank)
+    off, cnt, stride = gb.zero1_shard(cfg, world, rank)
+    assert cnt == 0
+    m = gb.Model(cfg, seed=w.weight_seed)
+    ar = m.state_arenas()
+    n = ar["n"]
+    w0 = ar["param"][:n].clone()
+    idx, tgt = W.random_batch(w, 5, w.batch_size * w.grad_accum, w.block_size)
+    m.train_step_host_accumulate(idx, tgt, 1)
+    parts = torch.full((gb.NORM_PARTIALS,), 7.0, dtype=torch.float64, device="cuda")
+    m.grad_sumsq_shard(off, cnt, parts)
+    assert not parts.any()                       # an empty shard: zero partial sums
+    gathered = torch.zeros(world * gb.NORM_PARTIALS, dtype=torch.float64, device="cuda")
+    assert m.clip_adamw_shard(1e-3, 1, off, cnt, 1.0 / world, gathered) == 0.0
+    assert not ar["grad"][:n].any()
+    assert torch.equal(ar["param"][:n], w0)
+    assert m.flags() == 0
+    m.close()
