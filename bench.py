@@ -367,8 +367,7 @@ def measure_configs(dev, warmup: int, with_oracle: bool):
     out = {}
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     pk = peaks()
-    for w in (W.MICRO, W.CHAR, W.DROPOUT_512, W.GPT2_XL):
-        cfg = gb.make_config(w)
+    def timed(w, cfg):
         m = gb.Model(cfg, seed=w.weight_seed, device=dev)
         host = W.token_stream(w)
         d_stream = torch.from_numpy(host.view(np.int16) if host.dtype == np.uint16 else host).to(dev)
@@ -392,6 +391,11 @@ def measure_configs(dev, warmup: int, with_oracle: bool):
         m.close()
         del m, d_stream
         torch.cuda.empty_cache()
+        return ms, loss, norm, n
+
+    for w in (W.MICRO, W.CHAR, W.DROPOUT_512, W.GPT2_XL):
+        cfg = gb.make_config(w)
+        ms, loss, norm, n = timed(w, cfg)
         tps = w.tokens_per_step / (ms / 1000.0)
         fpt = flops_per_token(w)
         rec = {"ms_per_step": ms, "tokens_per_s": tps, "tokens_per_step": w.tokens_per_step,
@@ -399,6 +403,12 @@ def measure_configs(dev, warmup: int, with_oracle: bool):
                "mfu_nominal_2250": tps * fpt / (NOMINAL_BF16_TFLOPS * 1e12),
                "mfu_measured_peak": tps * fpt / (pk["bf16"] * 1e12), "steps": n,
                "final_loss": loss, "final_grad_norm": norm}
+        if w is W.GPT2_XL:  # the configuration activation recompute exists for
+            rcfg = gb.make_config(w, recompute=1)
+            rms, _, _, _ = timed(w, rcfg)
+            rec["recompute"] = {"ms_per_step": rms, "tokens_per_s": w.tokens_per_step / (rms / 1000.0),
+                                "workspace_gb": gb.workspace_bytes(rcfg) / 1e9,
+                                "workspace_gb_stored": gb.workspace_bytes(cfg) / 1e9}
         if with_oracle:
             B, T = ORACLE_SAMPLES[w.name]
             one, _ = oracle_tokens_per_s(w, B, T, 1)
