@@ -459,7 +459,7 @@ const char* gpt_status_string(gpt_status s);
  * scratch.  Nothing is allocated: no cudaMalloc, cudaFree or allocating
  * library call.
  *   - The first call on a device (with that device current) looks up the
- *     array's device address; make that first call before any stream capture.
+ *     array's device address.
  *   - Every GPU that loads the library holds the array until the process
  *     exits.  All calls share it and it keeps the last call's contents (every
  *     partial sum is written before it is read, so nothing needs clearing);
