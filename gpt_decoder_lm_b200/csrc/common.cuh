@@ -186,30 +186,41 @@ __device__ __forceinline__ uint64_t f2sub(uint64_t a, uint64_t b) {
 }
 __device__ __forceinline__ uint64_t f2c(float c) { return f2(c, c); }
 
-// erf_as on a pair of arguments (same operations per lane as erf_as, the
-// polynomial and the affine steps on the f32x2 pipe).  Returns the pair of
-// erf values; e receives the pair e^{-z^2}.
-__device__ __forceinline__ uint64_t erf_as2(uint64_t z2, uint64_t& e2) {
-  const float2 z = f2split(z2);
-  const uint64_t az = f2(fabsf(z.x), fabsf(z.y));
-  const float2 den = f2split(f2fma(f2c(0.3275911f), az, f2c(1.0f)));
-  const uint64_t t = f2(__fdividef(1.0f, den.x), __fdividef(1.0f, den.y));
-  uint64_t q = f2fma(t, f2c(1.061405429f), f2c(-1.453152027f));
-  q = f2fma(t, q, f2c(1.421413741f));
-  q = f2fma(t, q, f2c(-0.284496736f));
-  q = f2fma(t, q, f2c(0.254829592f));
-  const uint64_t poly = f2mul(t, q);
-  const float2 sq = f2split(f2mul(az, az));
-  e2 = f2(__expf(-sq.x), __expf(-sq.y));
-  const float2 r = f2split(f2fma(f2mul(poly, f2c(-1.0f)), e2, f2c(1.0f)));
-  return f2(copysignf(r.x, z.x), copysignf(r.y, z.y));
+// The SFU's approximate reciprocal and base-2 exponential (PTX rcp.approx and
+// ex2.approx, denormals flushed).
+__device__ __forceinline__ float sfu_rcp(float x) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
 }
-// gelu_f and gelu_grad_f of a pair (a, b) at once (one erf / exp): the
-// activations replace (a, b), the derivatives go to (ga, gb)
+__device__ __forceinline__ float sfu_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+// gelu_f and gelu_grad_f of a pair (a, b) at once: the activations replace
+// (a, b), the derivatives go to (ga, gb).  The same erf (Abramowitz & Stegun
+// 7.1.26 at z = |x| / sqrt 2) with its constants folded so that most steps are
+// f32x2 operations on the pair:
+//   t = 1 / (1 + (p / sqrt 2) |x|),   e = e^{-x^2/2} = 2^{-(log2 e / 2) x^2},
+//   q = -(a1 t + a2 t^2 + ... + a5 t^5) / 2, so that q e = (erf(|z|) - 1) / 2,
+//   Phi(x) = 1/2 + sign(x) (1/2 + q e),
+//   GELU(x) = x Phi(x),   GELU'(x) = Phi(x) + x e / sqrt(2 pi).
 __device__ __forceinline__ void gelu_and_grad2(float& a, float& b, float& ga, float& gb) {
+  constexpr float kP = 0.3275911f * 0.70710678118654752f;  // p / sqrt 2
+  constexpr float kE = -0.72134752044448170f;              // -(log2 e) / 2
   const uint64_t x = f2(a, b);
-  uint64_t e;
-  const uint64_t cdf = f2mul(f2c(0.5f), f2add(f2c(1.0f), erf_as2(f2mul(x, f2c(0.70710678118654752f)), e)));
+  const float2 den = f2split(f2fma(f2(fabsf(a), fabsf(b)), f2c(kP), f2c(1.0f)));
+  const uint64_t t = f2(sfu_rcp(den.x), sfu_rcp(den.y));
+  uint64_t q = f2fma(t, f2c(-0.5f * 1.061405429f), f2c(0.5f * 1.453152027f));
+  q = f2fma(t, q, f2c(-0.5f * 1.421413741f));
+  q = f2fma(t, q, f2c(0.5f * 0.284496736f));
+  q = f2fma(t, q, f2c(-0.5f * 0.254829592f));
+  q = f2mul(t, q);
+  const float2 y = f2split(f2mul(f2mul(x, f2c(kE)), x));
+  const uint64_t e = f2(sfu_exp2(y.x), sfu_exp2(y.y));
+  const float2 u = f2split(f2fma(q, e, f2c(0.5f)));  // erf(|x| / sqrt 2) / 2
+  const uint64_t cdf = f2add(f2(copysignf(u.x, a), copysignf(u.y, b)), f2c(0.5f));
   const float2 g = f2split(f2mul(x, cdf));
   const float2 d = f2split(f2fma(f2mul(x, f2c(0.3989422804014327f)), e, cdf));
   a = g.x;

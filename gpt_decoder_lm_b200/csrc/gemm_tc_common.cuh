@@ -107,6 +107,19 @@ __device__ __forceinline__ void unstage_bf16(uint32_t buf, int r, int h, float (
   }
 }
 
+// Row r of a bf16 staging tile as 16 packed pairs: word k holds columns 2k
+// and 2k + 1.
+__device__ __forceinline__ void load_row_bf16(uint32_t buf, int r, uint32_t (&w)[16]) {
+#pragma unroll
+  for (int q = 0; q < 4; q++) {
+    const uint4 u = ld_shared_v4(buf + r * 64 + ((q ^ ((r >> 1) & 3)) << 4));
+    w[4 * q] = u.x;
+    w[4 * q + 1] = u.y;
+    w[4 * q + 2] = u.z;
+    w[4 * q + 3] = u.w;
+  }
+}
+
 // The 16 bias values of a half-row, loaded before the TMEM wait so that their
 // latency overlaps it (zeros past N).
 __device__ __forceinline__ void load_bias(const TcArgs& p, int col0, float4 (&b)[4]) {

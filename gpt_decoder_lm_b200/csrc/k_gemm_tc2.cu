@@ -232,7 +232,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lbar = smem_u32(&ebar[ew]);
     uint32_t lphase = 0;
     const int kind = p.kind;
-    const bool f32_in = kind == EPI_RESADD, bf16_in = kind == EPI_ACT_BWD;
+    // (the split-K planner splits only EPI_ACC_F32 products)
+    const bool f32_in = kind == EPI_RESADD && p.splits == 1, bf16_in = kind == EPI_ACT_BWD && p.splits == 1;
     const bool has_bias = p.bias && p.splits == 1 && kind != EPI_ACT_BWD && kind < EPI_ACC_F32;
     int acc = 0;
     uint32_t acc_phase = 0;
@@ -245,10 +246,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       const long row = row0 + lane;
       const int c_first = part * CPW;
       // the epilogue input of a warp's first chunk (residual stream or saved
-      // pre-activation) is fetched while the tile's MMAs still run
+      // act'(h)) is fetched while the tile's MMAs still run
       auto fetch_input = [&](int c) {
         if (lane == 0) {
-          bulk_wait_read0();  // the previous chunk's stores have read the staging set
+          // the fp32 input shares its buffer with the output: the previous
+          // chunk's stores must have read it (the bf16 input has its own half)
+          if (f32_in) bulk_wait_read0();
           mbar_expect_tx(lbar, f32_in ? 4096 : 2048);
           tma_load_2d(f32_in ? stg : stg + 2048, &tm_in, lbar, nb * BN + c * 32, row0);
         }
@@ -266,78 +269,110 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int col0 = nb * BN + c * 32;
         const uint32_t bufA = stg, bufB = stg + 2048;
         if (f32_in || bf16_in) {
-          if (c > c_first) fetch_input(c);
+          if (f32_in && c > c_first) fetch_input(c);
           if (!mbar_wait(lbar, lphase, abort_flag, p.flags)) {
             ok = false;
             break;
           }
           lphase ^= 1;
-        } else {
-          if (lane == 0) bulk_wait_read0();  // the previous chunk's stores have read the staging set
-          __syncwarp();
         }
+        if (bf16_in) {
+          // EPI_ACT_BWD: the chunk's act'(h) into registers, so that the next
+          // chunk's can be fetched into the buffer while this one is computed
+          // and stored
+          uint32_t aux[16];
+          load_row_bf16(bufB, lane, aux);
+          if (c + 1 < c_first + CPW) {
+            fence_proxy_async_smem();
+            __syncwarp();
+            fetch_input(c + 1);
+          }
 #pragma unroll
-        for (int hh = 0; hh < 2; hh++) {
-          float4 bias[4];
-          if (has_bias) load_bias(p, col0 + 16 * hh, bias);
-          uint32_t raw[16];
-          tmem_ld_32x32b_x16(tbase + c * 32 + 16 * hh, raw);
-          tmem_ld_wait();
-          float v[16];
+          for (int q = 0; q < 4; q++) {  // 8 columns at a time: aux holds 16 registers
+            uint32_t raw[8];
+            tmem_ld_32x32b_x8(tbase + c * 32 + 8 * q, raw);
+            tmem_ld_wait();
+            uint32_t w[4];
 #pragma unroll
-          for (int i = 0; i < 16; i++) v[i] = __uint_as_float(raw[i]);
-          if (p.splits > 1) {
-            stage_f32(bufA, lane, hh, v);
-          } else {
-            switch (kind) {
-              case EPI_STORE:
-              case EPI_BIAS:
-                if (has_bias) add_bias(bias, v);
-                stage_bf16(bufA, lane, hh, v);
-                break;
-              case EPI_BIAS_ACT: {
-                if (has_bias) add_bias(bias, v);
-                float dv[16];  // act'(h), kept for the backward pass
-                if (p.act == ACT_GELU) {
+            for (int k = 0; k < 4; k++) {
+              const float2 d = unpack_bf16(aux[4 * q + k]);
+              w[k] = pack_bf16(__uint_as_float(raw[2 * k]) * d.x, __uint_as_float(raw[2 * k + 1]) * d.y);
+            }
+            if (q == 0) {  // the previous chunk's stores have read the output half
+              if (lane == 0) bulk_wait_read0();
+              __syncwarp();
+            }
+            st_shared_v4(bufA + lane * 64 + ((q ^ ((lane >> 1) & 3)) << 4), w[0], w[1], w[2], w[3]);
+          }
+        } else {
 #pragma unroll
-                  for (int i = 0; i < 16; i += 2) gelu_and_grad2(v[i], v[i + 1], dv[i], dv[i + 1]);
-                } else {
+          for (int hh = 0; hh < 2; hh++) {
+            float4 bias[4];
+            if (has_bias) load_bias(p, col0 + 16 * hh, bias);
+            uint32_t raw[16];
+            tmem_ld_32x32b_x16(tbase + c * 32 + 16 * hh, raw);
+            tmem_ld_wait();
+            float v[16];
 #pragma unroll
-                  for (int i = 0; i < 16; i++) {
-                    dv[i] = act_grad(p.act, v[i]);
-                    v[i] = act_fwd(p.act, v[i]);
+            for (int i = 0; i < 16; i++) v[i] = __uint_as_float(raw[i]);
+            // before the first write of a chunk's outputs: the previous
+            // chunk's stores have read the staging set (the fp32-input kind
+            // waited before its fetch)
+            auto staging_free = [&]() {
+              if (hh == 0 && !f32_in) {
+                if (lane == 0) bulk_wait_read0();
+                __syncwarp();
+              }
+            };
+            if (p.splits > 1) {
+              staging_free();
+              stage_f32(bufA, lane, hh, v);
+            } else {
+              switch (kind) {
+                case EPI_STORE:
+                case EPI_BIAS:
+                  if (has_bias) add_bias(bias, v);
+                  staging_free();
+                  stage_bf16(bufA, lane, hh, v);
+                  break;
+                case EPI_BIAS_ACT: {
+                  if (has_bias) add_bias(bias, v);
+                  float dv[16];  // act'(h), kept for the backward pass
+                  if (p.act == ACT_GELU) {
+#pragma unroll
+                    for (int i = 0; i < 16; i += 2) gelu_and_grad2(v[i], v[i + 1], dv[i], dv[i + 1]);
+                  } else {
+#pragma unroll
+                    for (int i = 0; i < 16; i++) {
+                      dv[i] = act_grad(p.act, v[i]);
+                      v[i] = act_fwd(p.act, v[i]);
+                    }
                   }
+                  staging_free();
+                  stage_bf16(bufA, lane, hh, dv);
+                  stage_bf16(bufB, lane, hh, v);
+                  break;
                 }
-                stage_bf16(bufA, lane, hh, dv);
-                stage_bf16(bufB, lane, hh, v);
-                break;
-              }
-              case EPI_ACT_BWD: {
-                float dv[16];  // the saved act'(h)
-                unstage_bf16(bufB, lane, hh, dv);
+                case EPI_RESADD: {
+                  float x[16];
+                  unstage_f32(bufA, lane, hh, x);
+                  if (has_bias) add_bias(bias, v);
+                  if (p.drop.active) {
+                    const uint64_t el = (uint64_t)row * p.N + col0 + 16 * hh;
+                    const DropKey dk = drop_live(p.drop);
 #pragma unroll
-                for (int i = 0; i < 16; i++) v[i] *= dv[i];
-                stage_bf16(bufA, lane, hh, v);
-                break;
-              }
-              case EPI_RESADD: {
-                float x[16];
-                unstage_f32(bufA, lane, hh, x);
-                if (has_bias) add_bias(bias, v);
-                if (p.drop.active) {
-                  const uint64_t el = (uint64_t)row * p.N + col0 + 16 * hh;
-                  const DropKey dk = drop_live(p.drop);
+                    for (int i = 0; i < 16; i++) v[i] *= drop_mul(dk, el + i);
+                  }
 #pragma unroll
-                  for (int i = 0; i < 16; i++) v[i] *= drop_mul(dk, el + i);
+                  for (int i = 0; i < 16; i++) v[i] += x[i];
+                  stage_f32(bufA, lane, hh, v);
+                  break;
                 }
-#pragma unroll
-                for (int i = 0; i < 16; i++) v[i] += x[i];
-                stage_f32(bufA, lane, hh, v);
-                break;
+                default:  // EPI_ACC_F32, EPI_STORE_F32
+                  staging_free();
+                  stage_f32(bufA, lane, hh, v);
+                  break;
               }
-              default:  // EPI_ACC_F32, EPI_STORE_F32
-                stage_f32(bufA, lane, hh, v);
-                break;
             }
           }
         }

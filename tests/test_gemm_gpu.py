@@ -219,6 +219,37 @@ def test_gelu_epilogue_accuracy_fp32():
     np.testing.assert_allclose(out.double().cpu().numpy(), D * dd.astype(np.float64), rtol=1e-5, atol=2e-6)
 
 
+def bf16_ulp(y):
+    """Spacing of bf16 numbers at |y| (7 stored fraction bits against fp32's 23)."""
+    return np.spacing(np.abs(np.asarray(y, np.float32))).astype(np.float64) * 2.0 ** 16
+
+
+@pytest.mark.parametrize("backend", [TC, TC2], ids=["tc", "tc2"])
+def test_gelu_epilogue_bf16_half_ulp(backend):
+    # Pre-activations known exactly: B selects one column of A per output column
+    # (one 1 per row), so the fp32 accumulator holds A's bf16 values unchanged.
+    # The two bf16 outputs are then GELU and GELU' of known values rounded once:
+    # within half a bf16 ulp of the float64 values, plus 1e-6 (1 + |x|) for the
+    # erf approximation (|error| <= 1.5e-7, Abramowitz & Stegun 7.1.26) and the
+    # fp32 arithmetic.  A wrong constant or sign moves values by far more and
+    # flips roundings near the half-ulp points.
+    M, N, K = 512, 256, 64
+    rng = np.random.default_rng(21)
+    A = rng.uniform(-8.0, 8.0, (M, K))
+    A[0, :12] = [0.0, 1.0, -1.0, 0.5, -0.5, 3.0, -3.0, 20.0, -20.0, 100.0, -100.0, 1e-3]
+    A = bf16_round(A)
+    B = np.zeros((N, K))
+    B[np.arange(N), np.arange(N) % K] = 1.0
+    x = A @ B.T
+    out = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    out2 = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    run(backend, M, N, K, dev_bf16(A), K, 1, dev_bf16(B), K, 1, 2, act=0, out=out, out2=out2, ldo=N)
+    for got, ref in ((out2.double().cpu().numpy(), gelu(x)), (out.double().cpu().numpy(), gelu_grad(x))):
+        bound = 0.5 * bf16_ulp(np.maximum(np.abs(ref), np.abs(got))) + 1e-6 * (1.0 + np.abs(x))
+        excess = np.abs(got - ref) - bound
+        assert excess.max() <= 0.0, (x.flat[excess.argmax()], got.flat[excess.argmax()], ref.flat[excess.argmax()])
+
+
 # The contractions of the benchmarked step at their own shapes: GPT-2 124M
 # (M = 12 x 1024 rows, d 768, 3d 2304, 4d 3072) and GPT-2 XL's layer (M =
 # 2 x 1024, d 1600, 3d 4800 and 4d 6400, both ragged against the 256-column
