@@ -81,8 +81,11 @@ def attn_flops_per_step(w) -> float:
 # dram__bytes_read.sum + dram__bytes_write.sum of the tensor-core GEMMs per launch (ncu, one
 # pass, on `bench.py --layer-case 2`: every GEMM shape of a layer and the lm_head at full size),
 # weighted to the 12-layer step: (12 x one layer's 12 GEMMs + the lm_head's 3) / 147 launches.
-# None once the kernels change after that capture.
-GEMM_DRAM_BYTES_PER_LAUNCH = 107559868
+# None once the kernels change after that capture: the GEMM epilogue changed after the last one,
+# which gave 107,559,868 bytes per launch.
+GEMM_DRAM_BYTES_PER_LAUNCH = None
+GEMM_DRAM_BYTES_NOTE = ("null: the GEMM epilogue changed after the last per-launch DRAM capture "
+                        "(107,559,868 bytes per launch on the layer case before the change)")
 
 
 class Clocks:
@@ -556,6 +559,7 @@ def run_ours(args, w, rank, world, local_rank):
                 "achieved": achieved,
                 "peak": pk["bf16_sustained"], "unit": "TFLOP/s", "frac": achieved / pk["bf16_sustained"],
                 "traffic": GEMM_DRAM_BYTES_PER_LAUNCH, "traffic_unit": "bytes per launch (ncu)",
+                "traffic_note": GEMM_DRAM_BYTES_NOTE,
                 "peak_source": pk["source"] + " sustained bf16",
                 "launches": gemm_n, "avg_launch_ms": gemm_ms / max(gemm_n, 1)}
     step_ms = ms_max / args.steps
