@@ -596,15 +596,10 @@ __global__ void k_ce(T* __restrict__ logits, const int32_t* __restrict__ tgt, in
   }
 }
 
-__device__ __forceinline__ float sfu_ex2(float x) {  // 2^x on the SFU (rel. error ~2^-22)
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
 __device__ __forceinline__ void lse_merge(float& m, float& s, float m2, float s2) {
   float M = fmaxf(m, m2);
   if (M == -INFINITY) return;
-  s = (m == -INFINITY ? 0.f : s * sfu_ex2(m - M)) + (m2 == -INFINITY ? 0.f : s2 * sfu_ex2(m2 - M));
+  s = (m == -INFINITY ? 0.f : s * sfu_exp2(m - M)) + (m2 == -INFINITY ? 0.f : s2 * sfu_exp2(m2 - M));
   m = M;
 }
 
@@ -640,11 +635,11 @@ __global__ void __launch_bounds__(256, 4) k_ce_stream(T* __restrict__ logits, co
       mv = fmaxf(mv, x[k]);
     }
     if (mv > m) {
-      s = (m == -INFINITY) ? 0.f : s * sfu_ex2(m - mv);
+      s = (m == -INFINITY) ? 0.f : s * sfu_exp2(m - mv);
       m = mv;
     }
 #pragma unroll
-    for (int k = 0; k < EPV; k++) s += sfu_ex2(x[k] - m);
+    for (int k = 0; k < EPV; k++) s += sfu_exp2(x[k] - m);
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
@@ -678,7 +673,7 @@ __global__ void __launch_bounds__(256, 4) k_ce_stream(T* __restrict__ logits, co
     for (int k = 0; k < EPV; k++) {
       const int j = vi * EPV + k;
       float g = 0.f;
-      if (j < V) g = (sfu_ex2(fmaf(to_f<T>(e[k]), LOG2E, -lse2)) - (j == t ? 1.f : 0.f)) * scale;
+      if (j < V) g = (sfu_exp2(fmaf(to_f<T>(e[k]), LOG2E, -lse2)) - (j == t ? 1.f : 0.f)) * scale;
       o[k] = from_f<T>(g);
     }
     reinterpret_cast<uint4*>(z)[vi] = outv;
@@ -794,7 +789,7 @@ __global__ void __launch_bounds__(CE_THREADS, 2) k_ce_smem(T* __restrict__ logit
       mv *= LOG2E;
       if (mv > m) {
         if (m != -INFINITY) {
-          const float r = sfu_ex2(m - mv);
+          const float r = sfu_exp2(m - mv);
           s0 *= r;
           s1 *= r;
         }
@@ -804,8 +799,8 @@ __global__ void __launch_bounds__(CE_THREADS, 2) k_ce_smem(T* __restrict__ logit
 #pragma unroll
       for (int k = 0; k < EPV; k += 2) {
         const float2 y = f2split(f2fma(f2(x[k], x[k + 1]), l2, nm));
-        s0 += sfu_ex2(y.x);
-        s1 += sfu_ex2(y.y);
+        s0 += sfu_exp2(y.x);
+        s1 += sfu_exp2(y.y);
       }
     }
     float s = s0 + s1;
@@ -841,8 +836,8 @@ __global__ void __launch_bounds__(CE_THREADS, 2) k_ce_smem(T* __restrict__ logit
 #pragma unroll
         for (int k = 0; k < EPV; k += 2) {
           const float2 y = f2split(f2fma(f2(x[k], x[k + 1]), l2, nl));
-          g[k] = sfu_ex2(y.x);
-          g[k + 1] = sfu_ex2(y.y);
+          g[k] = sfu_exp2(y.x);
+          g[k + 1] = sfu_exp2(y.y);
         }
         if (vi == tv) {
 #pragma unroll
