@@ -62,7 +62,7 @@ typedef enum {
   GPT_ERR_TOKEN_RANGE = 5,       /* a token id was outside [0, vocab_size)            */
   GPT_ERR_NONFINITE = 6,         /* loss or gradient norm was NaN/Inf                 */
   GPT_ERR_STATE = 7,             /* call out of sequence (backward before forward)    */
-  GPT_ERR_UNSUPPORTED = 8,       /* valid request this build does not implement       */
+  GPT_ERR_UNSUPPORTED = 8,       /* valid request the library does not implement      */
   GPT_ERR_TIMEOUT = 9            /* a bounded device-side wait ran out                */
 } gpt_status;
 
